@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the chunkwise (TFLA) mLSTM forward + backward on B200.
+
+One step = one mlstm_fwd plus one mlstm_bwd over one batch (every kernel of
+the path) at B8 H32 T4096 d128, chunk 128, mLSTMexp, bf16 I/O.  Prints one
+JSON line (rank 0).  Multi-GPU runs (torchrun) are independent replicas: each
+rank processes its own batch, no collective touches the data path; the step
+time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (heads are independent), on the host cores.
+"""
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mLSTM chunkwise fwd/bwd TFLOP/s & tokens/s (B8 H32 d128 T4k-16k), % bf16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "exp_b8h32_t4096_d128_c128"
+# CUDA-core fp32 FMA peak: 148 SMs x 128 lanes x 2 flops x 1.965 GHz max SM clock
+FP32_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+KERNEL_SOURCES = {
+    "gate_prep": "gates.cu", "bwd_token_prep": "gates.cu", "gate_grad": "gates.cu",
+    "state_fwd_simt": "simt_fwd.cu", "output_fwd_simt": "simt_fwd.cu",
+    "state_bwd_simt": "simt_bwd.cu", "dq_simt": "simt_bwd.cu", "dk_simt": "simt_bwd.cu",
+    "dv_simt": "simt_bwd.cu",
+}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic FLOP and byte counts (per (b, h) head)
+# ---------------------------------------------------------------------------
+
+def flops_fwd(T, dqk, dhv, L):
+    """States 2 T dqk dhv + inter term 2 T dqk dhv + causal intra T L (dqk + dhv)."""
+    return 4 * T * dqk * dhv + T * L * (dqk + dhv)
+
+
+def flops_bwd(T, dqk, dhv, L):
+    """Four T dqk dhv contractions x2 + causal intra dS K, dS^T Q, S, dP, A^T dH."""
+    return 8 * T * dqk * dhv + T * L * (3 * dqk + 2 * dhv)
+
+
+def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
+    """(flops, bytes) per head for every kernel of the path, algorithmic counts."""
+    NC = -(-T // L)
+    sb = io_bytes  # states are stored in the I/O dtype
+    g = 3 if exp_variant else 2  # per-token gate floats (b, log i [, m])
+    st = NC * dqk * dhv * sb
+    stn = NC * dqk * 4 if exp_variant else 0
+    tdd = 2 * T * dqk * dhv
+    tok_f = T * 4
+    return {
+        "gate_prep": (0, T * 2 * io_bytes + g * tok_f),
+        "state_fwd_simt": (tdd, T * (dqk + dhv) * io_bytes + g * tok_f + st + stn),
+        "output_fwd_simt": (tdd + T * L * (dqk + dhv),
+                            T * (2 * dqk + 2 * dhv) * io_bytes + g * tok_f + st + stn
+                            + (tok_f if exp_variant else 0)),
+        "bwd_token_prep": (0, (T * 2 * dhv * io_bytes + 2 * tok_f + 4 * tok_f) if exp_variant
+                           else 3 * tok_f),
+        "state_bwd_simt": (tdd, T * (dqk + dhv) * io_bytes + 4 * tok_f + st + stn),
+        "dq_simt": (tdd + T * L * (dhv + dqk),
+                    T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st + stn),
+        "dk_simt": (tdd + T * L * dqk, T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st + stn),
+        "dv_simt": (tdd + T * L * (dqk + dhv), T * (2 * dqk + 2 * dhv) * io_bytes + 4 * tok_f + st),
+        "gate_grad": (0, T * 4 * io_bytes + 2 * tok_f),
+    }
+
+
+def kernel_bound(name):
+    """Which roofline bounds a kernel of this implementation."""
+    if name.endswith("_simt"):
+        return "alu"
+    if name.endswith("_tc"):
+        return "tensor"
+    return "hbm"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def source_sha(kernel):
+    src = KERNEL_SOURCES.get(kernel)
+    if src is None:
+        return None
+    path = os.path.join(ROOT, "mlstm_chunkwise_attention_b200", "csrc", src)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel)
+    if not e or e.get("workload") != workload or e.get("source_sha") != source_sha(kernel):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = open(os.path.join("/tmp", f"mlstm_clocks_{os.getpid()}.csv"), "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_index)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[1]), "max": float(parts[2]), "active": parts[4],
+                                 "hw": parts[5], "hwt": parts[6], "swt": parts[7], "pcap": parts[8]})
+                except ValueError:
+                    continue
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+def oracle_sample(spec, heads, budget_s=20.0):
+    """Time the fp64 oracle (chunkwise forward + parallel-form backward) on whole heads."""
+    import numpy as np
+    import oracle
+    from mlstm_chunkwise_attention_b200.synthetic import make_inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        cores = 1
+    T, dqk, dhv, L, var = spec["T"], spec["d_qk"], spec["d_hv"], spec["chunk"], spec["variant"]
+    done, elapsed = [], 0.0
+    for (b, hh) in heads:
+        x = make_inputs(1, 1, T, dqk, dhv, seed=spec["seed"] * 1000 + b * 64 + hh,
+                        igate_mean=spec["igate_mean"], fgate_mean=spec["fgate_mean"], with_dh=True)
+        x = {k: v[0, 0].double().numpy() for k, v in x.items()}
+        t0 = time.perf_counter()
+        li, lf = oracle.gate_logs(x["igate"], x["fgate"], var)
+        oracle.chunkwise_forward(x["q"], x["k"], x["v"], li, lf, var, L)
+        g = oracle.parallel_backward(x["q"], x["k"], x["v"], li, lf, var, x["dh"])
+        oracle.preact_grads(g["dlog_i"], g["dlog_f"], x["igate"], x["fgate"], var)
+        elapsed += time.perf_counter() - t0
+        done.append((b, hh))
+        if elapsed >= budget_s:
+            break
+    flops = len(done) * (flops_fwd(T, dqk, dhv, L) + flops_bwd(T, dqk, dhv, L))
+    return {"value": flops / elapsed / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "seconds": elapsed, "heads": len(done),
+            "sample": f"{len(done)} of {spec['B'] * spec['NH']} heads of the workload "
+                      f"(T={T}, d={dqk}/{dhv}, chunk {L}): fp64 chunkwise forward + parallel-form "
+                      f"backward in numpy; throughput scaled by the algorithmic FLOPs of the heads run"}
+
+
+def run_reference(args, spec):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from mlstm_chunkwise_attention_b200.synthetic import sample_heads
+    heads = sample_heads(spec["B"], spec["NH"], args.warmup + args.steps, 4242)
+    times = []
+    info = None
+    for i, hd in enumerate(heads):
+        info = oracle_sample(spec, [hd], budget_s=0.0)
+        if i >= args.warmup:
+            times.append(info["seconds"])
+    T, dqk, dhv, L = spec["T"], spec["d_qk"], spec["d_hv"], spec["chunk"]
+    per_head = flops_fwd(T, dqk, dhv, L) + flops_bwd(T, dqk, dhv, L)
+    total_s = sum(times)
+    value = per_head * len(times) / total_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(spec, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                         "sample": "each step: one head of the workload, fp64 chunkwise forward + "
+                                   "parallel-form backward (numpy)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(spec, n):
+    return {"workload": WORKLOAD, "cell": "mLSTMexp" if spec["variant"] == 1 else "mLSTMsig",
+            "B": spec["B"], "NH": spec["NH"], "T": spec["T"], "d_qk": spec["d_qk"],
+            "d_hv": spec["d_hv"], "chunk": spec["chunk"], "pass": "fwd+bwd",
+            "global_batch": spec["B"] * n, "seq_len": spec["T"],
+            "parallelism": f"replicas{n}" if n > 1 else "single",
+            "l2": "no flush: q, k, v, dh are 268 MB each, larger than the 126 MB L2"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from mlstm_chunkwise_attention_b200.synthetic import WORKLOADS
+    spec = dict(WORKLOADS[WORKLOAD])
+
+    if args.impl == "reference":
+        return run_reference(args, spec)
+
+    import torch
+    import torch.distributed as dist
+    from mlstm_chunkwise_attention_b200 import binding
+    from mlstm_chunkwise_attention_b200.synthetic import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    B, NH, T, dqk, dhv, L, var = (spec[k] for k in ("B", "NH", "T", "d_qk", "d_hv", "chunk", "variant"))
+    dtype = torch.bfloat16
+    cpu = make_inputs(B, NH, T, dqk, dhv, seed=spec["seed"] + 1000 * rank,
+                      igate_mean=spec["igate_mean"], fgate_mean=spec["fgate_mean"], dtype=dtype,
+                      with_dh=True)
+    x = {k: v.to(dev) for k, v in cpu.items()}
+    sizes = binding.problem_sizes(x["q"], x["v"], L, var)
+    saved = torch.empty(binding.mlstm_saved_size(*sizes), dtype=torch.uint8, device=dev)
+    wsb = binding.mlstm_bwd_workspace_size(*sizes)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    h = torch.empty_like(x["v"])
+    grads = {"dq": torch.empty_like(x["q"]), "dk": torch.empty_like(x["k"]),
+             "dv": torch.empty_like(x["v"]), "dig": torch.empty_like(x["igate"]),
+             "dfg": torch.empty_like(x["fgate"])}
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    nf = binding.mlstm_fwd_launch_count(*sizes)
+    nb = binding.mlstm_bwd_launch_count(*sizes)
+    names = ([binding.mlstm_launch_name(0, i, *sizes) for i in range(nf)]
+             + [binding.mlstm_launch_name(1, i, *sizes) for i in range(nb)])
+
+    def step(src, fwd_ev=None, bwd_ev=None):
+        if fwd_ev is not None:
+            binding.mlstm_set_timing_events(fwd_ev, 2 * nf)
+        st = binding.mlstm_fwd(src["q"].data_ptr(), src["k"].data_ptr(), src["v"].data_ptr(),
+                               src["igate"].data_ptr(), src["fgate"].data_ptr(), h.data_ptr(),
+                               saved.data_ptr(), None, 0, *sizes, sh)
+        if st != 0:
+            raise binding.MLSTMError(st, "mlstm_fwd")
+        if bwd_ev is not None:
+            binding.mlstm_set_timing_events(bwd_ev, 2 * nb)
+        st = binding.mlstm_bwd(src["q"].data_ptr(), src["k"].data_ptr(), src["v"].data_ptr(),
+                               src["igate"].data_ptr(), src["fgate"].data_ptr(), h.data_ptr(),
+                               src["dh"].data_ptr(), saved.data_ptr(), grads["dq"].data_ptr(),
+                               grads["dk"].data_ptr(), grads["dv"].data_ptr(),
+                               grads["dig"].data_ptr(), grads["dfg"].data_ptr(), ws.data_ptr(),
+                               wsb, *sizes, sh)
+        binding.mlstm_set_timing_events(None, 0)
+        if st != 0:
+            raise binding.MLSTMError(st, "mlstm_bwd")
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-timed region: inputs resident in HBM
+    for _ in range(args.warmup):
+        step(x)
+    ev_keep = []
+    fwd_evs, bwd_evs = [], []
+    for _ in range(args.steps):
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nf)]
+        be = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nb)]
+        for e in fe + be:  # creates the underlying CUDA event, outside the timed region
+            e.record(stream)
+        ev_keep.append((fe, be))
+    torch.cuda.synchronize(dev)
+    for fe, be in ev_keep:
+        fwd_evs.append((ctypes.c_void_p * (2 * nf))(*[e.cuda_event for e in fe]))
+        bwd_evs.append((ctypes.c_void_p * (2 * nb))(*[e.cuda_event for e in be]))
+        assert all(p_ for p_ in fwd_evs[-1]) and all(p_ for p_ in bwd_evs[-1])
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        step(x, fwd_evs[i], bwd_evs[i])
+    end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms)
+    per_kernel = {n: 0.0 for n in names}
+    for fe, be in ev_keep:
+        for i in range(nf):
+            per_kernel[names[i]] += fe[2 * i].elapsed_time(fe[2 * i + 1])
+        for i in range(nb):
+            per_kernel[names[nf + i]] += be[2 * i].elapsed_time(be[2 * i + 1])
+    per_kernel = {n: v / args.steps for n, v in per_kernel.items()}  # ms per launch
+
+    heads = B * NH
+    step_flops = heads * (flops_fwd(T, dqk, dhv, L) + flops_bwd(T, dqk, dhv, L))
+    tflops = step_flops * args.steps * world / (ms_max * 1e-3) / 1e12
+    tokens_s = B * T * args.steps * world / (ms_max * 1e-3)
+    peaks = load_peaks()
+
+    # ---- roofline of the dominant kernel
+    costs = kernel_costs(T, dqk, dhv, L, var == 1, 2)
+    dom = max(per_kernel, key=per_kernel.get)
+    fl, by = costs[dom]
+    dur_s = per_kernel[dom] * 1e-3
+    bound = kernel_bound(dom)
+    if bound == "hbm" or (bound != "alu" and by / peaks["hbm_gbs"] > fl / (peaks["bf16_tflops"] * 1e3)):
+        bound = "hbm"
+        achieved, peak, unit = heads * by / dur_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        peak_src = peaks["source"]
+    elif bound == "tensor":
+        achieved, peak, unit = heads * fl / dur_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        peak_src = peaks["source"] + " (sustained)"
+    else:
+        achieved, peak, unit = heads * fl / dur_s / 1e12, FP32_CORE_TFLOPS, "TFLOP/s"
+        peak_src = "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz"
+    traffic = committed_traffic(dom, WORKLOAD)
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                "algorithmic_per_launch": heads * (by if bound == "hbm" else fl),
+                "ms_per_launch": per_kernel[dom]}
+
+    # ---- end to end through the C ABI with pinned host buffers
+    host_in = {k: v.pin_memory() for k, v in cpu.items()}
+    host_out = {"h": torch.empty(h.shape, dtype=dtype).pin_memory(),
+                **{k: torch.empty(v.shape, dtype=dtype).pin_memory() for k, v in grads.items()}}
+    xd = {k: torch.empty_like(v) for k, v in x.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+
+    def e2e_step():
+        for k_ in xd:
+            xd[k_].copy_(host_in[k_], non_blocking=True)
+        step(xd)
+        host_out["h"].copy_(h, non_blocking=True)
+        for k_, v in grads.items():
+            host_out[k_].copy_(v, non_blocking=True)
+
+    del x
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_tflops = step_flops * args.steps * world / (e2e_ms * 1e-3) / 1e12
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from mlstm_chunkwise_attention_b200.synthetic import sample_heads
+        cpu_base = oracle_sample(spec, sample_heads(B, NH, 8, 99), budget_s=15.0)
+        cpu_base.pop("seconds", None)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": tflops, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(spec, world),
+        "tokens_per_s": tokens_s, "pct_bf16_peak": 100.0 * tflops / (world * peaks["bf16_tflops"]),
+        "kernel_ms": per_kernel,
+        "roofline": roofline,
+        "cpu_baseline": cpu_base,
+        "e2e": {"value": e2e_tflops, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": args.steps * (nf + nb),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

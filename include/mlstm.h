@@ -1,0 +1,164 @@
+/*
+ * mlstm.h -- C ABI of the chunkwise-parallel (TFLA) mLSTM forward and backward
+ * kernels for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  "Tiled Flash Linear Attention: More Efficient Linear RNN
+ * and xLSTM Kernels" (TFLA summary page, sections Problem and Approach; arXiv
+ * abstract page, Abstract) describes the mLSTM, a gated linear RNN with a
+ * matrix memory, in two variants: mLSTMexp (exponential input gate, normaliser
+ * state n_t and max state m_t) and mLSTMsig (sigmoid input gate, no normaliser
+ * and no max state).  Both use a sigmoid forget gate and scale q by
+ * 1/sqrt(d_qk).  Per (batch, head), with C_0 = 0, n_0 = 0:
+ *
+ *   C_t = f_t C_{t-1} + i_t k_t v_t^T        n_t = f_t n_{t-1} + i_t k_t
+ *   mLSTMsig: h_t = C_t^T q'_t
+ *   mLSTMexp: h_t = C_t^T q'_t / max(|n_t . q'_t|, 1)        q'_t = q_t / sqrt(d_qk)
+ *
+ * with f_t = sigmoid(fgate_pre_t), and i_t = exp(igate_pre_t) (EXP) or
+ * sigmoid(igate_pre_t) (SIG).  The pages print no formula; this is the plainest
+ * reading of what they state.  The library evaluates it chunkwise, as the pages
+ * describe: the sequence is split into chunks of `chunk` tokens, the state
+ * entering each chunk is materialised in memory, and the outputs of all chunks
+ * are computed in parallel with the intra-chunk matmuls tiled along the
+ * sequence (the second level of TFLA), so the chunk size is not bounded by
+ * shared memory.
+ *
+ * Layout.  Row-major, contiguous, head-major:
+ *   q, k, dq, dk : [B, NH, T, d_qk]      v, h, dh, dv : [B, NH, T, d_hv]
+ *   igate_pre, fgate_pre, digate_pre, dfgate_pre : [B, NH, T]
+ * Every tensor uses the one I/O dtype (MLSTM_BF16 or MLSTM_FP32); arithmetic
+ * is fp32 (bf16 tensor-core operands with fp32 accumulation on the bf16 path).
+ * All pointers are device pointers, 16-byte aligned.
+ *
+ * Supported sizes.  B, NH >= 0; T >= 0 (T need not be a multiple of `chunk`:
+ * the last chunk is then shorter); chunk a power of two in [64, 4096];
+ * d_qk in {64, 128, 256}; d_hv in {64, 128, 256, 512}; B*NH*T < 2^31.
+ * Other values return MLSTM_ERR_UNSUPPORTED.  B*NH*T == 0 is a no-op.
+ *
+ * Ownership.  The caller allocates every buffer.  The library never
+ * allocates or frees device memory, never synchronises the stream and keeps
+ * no per-call state; all work is enqueued on `stream` (a cudaStream_t passed
+ * as void*, NULL = legacy default stream) and the call returns at once.
+ *
+ * Errors.  Argument errors are detected on the host before any launch and
+ * return MLSTM_ERR_INVALID / MLSTM_ERR_UNSUPPORTED / MLSTM_ERR_WORKSPACE with
+ * nothing enqueued.  A failed launch returns MLSTM_ERR_CUDA; an earlier sticky
+ * CUDA error in the context is reported the same way and is not cleared.
+ */
+#ifndef MLSTM_H
+#define MLSTM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MLSTM_SIG = 0, MLSTM_EXP = 1 } mlstm_variant_t;
+typedef enum { MLSTM_BF16 = 0, MLSTM_FP32 = 1 } mlstm_dtype_t;
+
+typedef enum {
+  MLSTM_OK = 0,
+  MLSTM_ERR_INVALID = 1,      /* null pointer, negative size, bad enum       */
+  MLSTM_ERR_UNSUPPORTED = 2,  /* valid but outside the supported sizes       */
+  MLSTM_ERR_WORKSPACE = 3,    /* workspace / saved buffer too small          */
+  MLSTM_ERR_CUDA = 4,         /* a CUDA launch or the context failed         */
+  MLSTM_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up          */
+} mlstm_status_t;
+
+/* Regions of the `saved` buffer that mlstm_fwd fills and mlstm_bwd reads.
+ * Offsets are in bytes from the start of the buffer, 256-byte aligned.
+ * NC = ceil(T / chunk); BH = B * NH.  Regions absent for a variant have
+ * size 0.
+ *   gate_b   float [BH, T]    in-chunk inclusive cumulative sum of log f
+ *   gate_li  float [BH, T]    log input gate (i~ for EXP, logsigmoid(i~) for SIG)
+ *   gate_m   float [BH, T]    EXP: max state m_t of the recurrence
+ *   norm     float [BH, T]    EXP: stabilised normaliser  n~_t . q'_t
+ *   state_c  [BH, NC, d_qk, d_hv]  state entering each chunk (EXP: scaled
+ *            by exp(-m) of the chunk's previous row); bf16 on the bf16 path,
+ *            float on the fp32 path
+ *   state_n  float [BH, NC, d_qk]  EXP: normaliser state entering each chunk */
+typedef struct {
+  size_t gate_b, gate_li, gate_m, norm, state_c, state_n;
+  size_t gate_b_bytes, gate_li_bytes, gate_m_bytes, norm_bytes, state_c_bytes, state_n_bytes;
+  size_t total;
+} mlstm_saved_layout_t;
+
+/* Fill *layout for the given problem.  Returns MLSTM_OK or an argument error. */
+int mlstm_saved_layout(int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                       int variant, int dtype, mlstm_saved_layout_t* layout);
+
+/* Bytes of the `saved` buffer (0 on an argument error). */
+size_t mlstm_saved_size(int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                        int variant, int dtype);
+
+/* Bytes of workspace mlstm_fwd needs when `saved` is NULL (the saved regions
+ * then live in the workspace); with a non-NULL `saved` it needs none. */
+size_t mlstm_fwd_workspace_size(int B, int NH, int T, int d_qk, int d_hv,
+                                int chunk, int variant, int dtype);
+
+/* Bytes of workspace mlstm_bwd needs (0 on an argument error). */
+size_t mlstm_bwd_workspace_size(int B, int NH, int T, int d_qk, int d_hv,
+                                int chunk, int variant, int dtype);
+
+/* Forward pass.  Reads q, k, v, igate_pre, fgate_pre; writes h and, when
+ * `saved` is non-NULL, the saved regions for mlstm_bwd (mlstm_saved_size
+ * bytes).  `workspace` may be NULL when `saved` is non-NULL.  The steps are
+ * those of the chunkwise form: gate preprocessing, the inter-chunk state
+ * recurrence, then the tiled intra-chunk outputs fused with the inter-chunk
+ * term q' C_prev and the normaliser (TFLA summary page, Approach; arXiv
+ * abstract page, Abstract). */
+int mlstm_fwd(const void* q, const void* k, const void* v,
+              const void* igate_pre, const void* fgate_pre,
+              void* h, void* saved,
+              void* workspace, size_t workspace_bytes,
+              int B, int NH, int T, int d_qk, int d_hv, int chunk,
+              int variant, int dtype, void* stream);
+
+/* Backward pass of sum(dh * h).  Reads q, k, v, the gate preactivations, the
+ * forward output h, the upstream gradient dh and `saved` as filled by
+ * mlstm_fwd on the same inputs (required, not NULL).  Writes dq, dk, dv and
+ * the preactivation gradients digate_pre, dfgate_pre.  The timed training
+ * kernels of the TFLA summary page (Key results) are this forward plus this
+ * backward. */
+int mlstm_bwd(const void* q, const void* k, const void* v,
+              const void* igate_pre, const void* fgate_pre,
+              const void* h, const void* dh, const void* saved,
+              void* dq, void* dk, void* dv, void* digate_pre, void* dfgate_pre,
+              void* workspace, size_t workspace_bytes,
+              int B, int NH, int T, int d_qk, int d_hv, int chunk,
+              int variant, int dtype, void* stream);
+
+/* Static text for a status code. */
+const char* mlstm_status_string(int status);
+
+/* Text of the CUDA error behind the calling thread's last MLSTM_ERR_CUDA
+ * ("" if none).  Valid until the thread's next call into the library. */
+const char* mlstm_last_error(void);
+
+/* Number of kernels mlstm_fwd / mlstm_bwd enqueue for this problem (0 on an
+ * argument error or an empty problem). */
+int mlstm_fwd_launch_count(int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                           int variant, int dtype);
+int mlstm_bwd_launch_count(int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                           int variant, int dtype);
+
+/* Static name of the index-th kernel that mlstm_fwd (pass 0) or mlstm_bwd
+ * (pass 1) enqueues for this problem ("" when out of range). */
+const char* mlstm_launch_name(int pass, int index, int B, int NH, int T, int d_qk,
+                              int d_hv, int chunk, int variant, int dtype);
+
+/* Per-kernel timing hook for the calling thread.  While set (count > 0),
+ * every mlstm_fwd / mlstm_bwd call records events[2i] (a cudaEvent_t passed
+ * as void*) on its stream just before its i-th kernel and events[2i+1] just
+ * after it, for i < count/2; kernels beyond that are not bracketed.  The
+ * array is borrowed, not copied: it must stay valid until the hook is
+ * cleared with (NULL, 0).  Returns MLSTM_ERR_INVALID for count < 0 or a NULL
+ * array with count > 0. */
+int mlstm_set_timing_events(void* const* events, int count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLSTM_H */

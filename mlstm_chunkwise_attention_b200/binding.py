@@ -1,0 +1,249 @@
+"""Thin Python binding of libmlstm.so (ctypes).
+
+The functions named like the C ABI (``mlstm_fwd``, ``mlstm_bwd``, the size
+queries) marshal plain integers (device pointers, sizes, a stream handle) and
+return the C status.  ``forward`` / ``backward`` are conveniences for torch
+tensors: they allocate outputs and buffers through PyTorch (plumbing only) and
+call the same entry points.  Every step of the computation runs in the CUDA
+library; if it is not built this module raises instead of computing anything.
+"""
+
+import ctypes
+import os
+
+SIG = 0
+EXP = 1
+BF16 = 0
+FP32 = 1
+
+STATUS_OK = 0
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmlstm.so")
+_lib = None
+
+
+class MLSTMError(RuntimeError):
+    def __init__(self, status, where):
+        lib = load()
+        msg = lib.mlstm_status_string(status).decode()
+        detail = lib.mlstm_last_error().decode()
+        super().__init__(f"{where}: {msg} ({status}){': ' + detail if detail else ''}")
+        self.status = status
+
+
+class SavedLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n",
+        "gate_b_bytes", "gate_li_bytes", "gate_m_bytes", "norm_bytes", "state_c_bytes",
+        "state_n_bytes", "total")]
+
+
+_SIZES = [ctypes.c_int] * 8  # B, NH, T, d_qk, d_hv, chunk, variant, dtype
+_P = ctypes.c_void_p
+
+EXPORTS = {
+    "mlstm_saved_layout": (ctypes.c_int, _SIZES + [ctypes.POINTER(SavedLayout)]),
+    "mlstm_saved_size": (ctypes.c_size_t, _SIZES),
+    "mlstm_fwd_workspace_size": (ctypes.c_size_t, _SIZES),
+    "mlstm_bwd_workspace_size": (ctypes.c_size_t, _SIZES),
+    "mlstm_fwd_launch_count": (ctypes.c_int, _SIZES),
+    "mlstm_bwd_launch_count": (ctypes.c_int, _SIZES),
+    "mlstm_fwd": (ctypes.c_int, [_P] * 7 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
+    "mlstm_bwd": (ctypes.c_int, [_P] * 13 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
+    "mlstm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mlstm_last_error": (ctypes.c_char_p, []),
+    "mlstm_launch_name": (ctypes.c_char_p, [ctypes.c_int, ctypes.c_int] + _SIZES),
+    "mlstm_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
+}
+
+
+def load(path=None):
+    """Load the CUDA library once; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library not built: {path} is missing "
+                          "(run __graft_entry__.build() or python -m mlstm_chunkwise_attention_b200._build)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in EXPORTS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+# --------------------------------------------------------------------------
+# C ABI, same names
+# --------------------------------------------------------------------------
+
+def mlstm_saved_layout(B, NH, T, d_qk, d_hv, chunk, variant, dtype):
+    lay = SavedLayout()
+    st = load().mlstm_saved_layout(B, NH, T, d_qk, d_hv, chunk, variant, dtype, ctypes.byref(lay))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_saved_layout")
+    return {n: getattr(lay, n) for n, _ in SavedLayout._fields_}
+
+
+def mlstm_saved_size(*sizes):
+    return load().mlstm_saved_size(*sizes)
+
+
+def mlstm_fwd_workspace_size(*sizes):
+    return load().mlstm_fwd_workspace_size(*sizes)
+
+
+def mlstm_bwd_workspace_size(*sizes):
+    return load().mlstm_bwd_workspace_size(*sizes)
+
+
+def mlstm_fwd_launch_count(*sizes):
+    return load().mlstm_fwd_launch_count(*sizes)
+
+
+def mlstm_bwd_launch_count(*sizes):
+    return load().mlstm_bwd_launch_count(*sizes)
+
+
+def mlstm_fwd(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_bytes,
+              B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream):
+    return load().mlstm_fwd(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_bytes,
+                            B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream)
+
+
+def mlstm_bwd(q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv, digate_pre, dfgate_pre,
+              workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream):
+    return load().mlstm_bwd(q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv, digate_pre,
+                            dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
+                            variant, dtype, stream)
+
+
+def mlstm_status_string(status):
+    return load().mlstm_status_string(status).decode()
+
+
+def mlstm_last_error():
+    return load().mlstm_last_error().decode()
+
+
+def mlstm_launch_name(pass_, index, *sizes):
+    return load().mlstm_launch_name(pass_, index, *sizes).decode()
+
+
+def mlstm_set_timing_events(events, count):
+    """events: a ctypes array of void* (cudaEvent_t handles), or None."""
+    return load().mlstm_set_timing_events(events, count)
+
+
+# --------------------------------------------------------------------------
+# torch conveniences (allocation through PyTorch, compute in the library)
+# --------------------------------------------------------------------------
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+def _check(tensors, dtype):
+    for name, t in tensors.items():
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def problem_sizes(q, v, chunk, variant):
+    B, NH, T, d_qk = q.shape
+    d_hv = v.shape[-1]
+    return (B, NH, T, d_qk, d_hv, int(chunk), int(variant), _dtype_code(q))
+
+
+def forward(q, k, v, igate_pre, fgate_pre, chunk, variant, *, keep_saved=True, h=None,
+            saved=None, stream=None):
+    """h = mLSTM(q, k, v, gates) on the current (or given) stream.
+
+    Returns (h, saved); ``saved`` (a uint8 tensor) is what ``backward`` needs,
+    or None when keep_saved is False (then a transient workspace is used).
+    """
+    import torch
+    _check({"q": q, "k": k, "v": v, "igate_pre": igate_pre, "fgate_pre": fgate_pre}, q.dtype)
+    sizes = problem_sizes(q, v, chunk, variant)
+    if h is None:
+        h = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ws = None
+    if keep_saved:
+        if saved is None:
+            saved = torch.empty(max(mlstm_saved_size(*sizes), 1), dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_bytes = None, 0
+    else:
+        nbytes = mlstm_fwd_workspace_size(*sizes)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_bytes = ws.data_ptr(), nbytes
+    st = mlstm_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
+                   fgate_pre.data_ptr(), h.data_ptr(), saved.data_ptr() if keep_saved else None,
+                   ws_ptr, ws_bytes, *sizes, _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_fwd")
+    return h, (saved if keep_saved else None)
+
+
+def backward(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, *, workspace=None,
+             stream=None):
+    """Gradients of sum(dh * h): dict of dq, dk, dv, digate_pre, dfgate_pre."""
+    import torch
+    _check({"q": q, "k": k, "v": v, "igate_pre": igate_pre, "fgate_pre": fgate_pre, "h": h,
+            "dh": dh}, q.dtype)
+    sizes = problem_sizes(q, v, chunk, variant)
+    out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "digate_pre": torch.empty_like(igate_pre), "dfgate_pre": torch.empty_like(fgate_pre)}
+    nbytes = mlstm_bwd_workspace_size(*sizes)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    st = mlstm_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
+                   fgate_pre.data_ptr(), h.data_ptr(), dh.data_ptr(), saved.data_ptr(),
+                   out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr(),
+                   out["digate_pre"].data_ptr(), out["dfgate_pre"].data_ptr(),
+                   workspace.data_ptr(), workspace.numel(), *sizes, _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_bwd")
+    return out
+
+
+def saved_views(saved, q, v, chunk, variant):
+    """Typed views of the saved regions (for tests and diagnostics)."""
+    import torch
+    B, NH, T, d_qk, d_hv, chunk, variant, dtype = problem_sizes(q, v, chunk, variant)
+    lay = mlstm_saved_layout(B, NH, T, d_qk, d_hv, chunk, variant, dtype)
+    NC = (T + chunk - 1) // chunk
+    BH = B * NH
+
+    def view(name, shape, dt):
+        nbytes = lay[name + "_bytes"]
+        if nbytes == 0:
+            return None
+        return saved[lay[name]: lay[name] + nbytes].view(dt).view(*shape)
+
+    sdt = torch.bfloat16 if dtype == BF16 else torch.float32
+    return {
+        "b": view("gate_b", (BH, T), torch.float32),
+        "log_i": view("gate_li", (BH, T), torch.float32),
+        "m": view("gate_m", (BH, T), torch.float32),
+        "abar": view("norm", (BH, T), torch.float32),
+        "C": view("state_c", (BH, NC, d_qk, d_hv), sdt),
+        "n": view("state_n", (BH, NC, d_qk), torch.float32),
+    }

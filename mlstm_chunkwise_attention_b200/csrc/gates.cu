@@ -1,0 +1,235 @@
+// Gate kernels of the chunkwise mLSTM: forward gate preprocessing (K-a), the
+// per-token backward preparation (K-d0) and the gate gradients (K-d3).
+//
+// "Tiled Flash Linear Attention: More Efficient Linear RNN and xLSTM Kernels"
+// (TFLA summary page, Approach): mLSTMexp has an exponential input gate and a
+// max state; mLSTMsig a sigmoid input gate and no max state; both a sigmoid
+// forget gate.  These kernels are bandwidth-bound warp scans over [B*NH, T].
+#include "common.cuh"
+#include "internal.h"
+
+namespace mlstm {
+
+// ---------------------------------------------------------------------------
+// K-a: per chunk, b_t = inclusive cumsum of log f_t inside the chunk and
+// log i_t; for EXP the max state m_t = b_t + max(m_{c-1}, max_{s<=t in c}(log i_s - b_s)),
+// where m_c (the max state at the chunk's last row) obeys the max-plus
+// recurrence m_c = max(g_c + m_{c-1}, g_c + max_{s in c}(log i_s - b_s)).
+// One CTA per (b, h); each warp owns whole chunks, each lane a contiguous
+// run of rows.  The chunk recurrence is an inclusive warp scan of the affine
+// max-plus maps x -> max(x + g_c, u_c).
+// ---------------------------------------------------------------------------
+template <typename TIO, bool EXPV>
+__global__ void __launch_bounds__(256) gate_prep_kernel(
+    const TIO* __restrict__ ig, const TIO* __restrict__ fg, float* __restrict__ b_out,
+    float* __restrict__ li_out, float* __restrict__ m_out, int T, int L, int NC) {
+  extern __shared__ float smem[];
+  float* sg = smem;       // g_c  (chunk decay)
+  float* su = smem + NC;  // u_c, then m_c
+  const size_t base = (size_t)blockIdx.x * T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const unsigned full = 0xffffffffu;
+
+  for (int c = warp; c < NC; c += nwarps) {
+    const int c0 = c * L;
+    const int len = min(L, T - c0);
+    const int per = (len + 31) / 32;
+    const int r0 = min(lane * per, len), r1 = min(r0 + per, len);
+    float seg = 0.f;
+    for (int r = r0; r < r1; ++r) seg += log_sigmoid(to_f32(fg[base + c0 + r]));
+    const float incl = warp_incl_sum(seg);
+    float run = incl - seg;
+    float umax = -INFINITY;
+    for (int r = r0; r < r1; ++r) {
+      const size_t idx = base + c0 + r;
+      run += log_sigmoid(to_f32(fg[idx]));
+      const float x = to_f32(ig[idx]);
+      const float li = EXPV ? x : log_sigmoid(x);
+      b_out[idx] = run;
+      li_out[idx] = li;
+      if (EXPV) {
+        umax = fmaxf(umax, li - run);
+        m_out[idx] = umax;
+      }
+    }
+    if (EXPV) {
+      const float pm = warp_incl_max(umax);
+      float excl = __shfl_up_sync(full, pm, 1);
+      if (lane == 0) excl = -INFINITY;
+      for (int r = r0; r < r1; ++r) {
+        const size_t idx = base + c0 + r;
+        m_out[idx] = fmaxf(m_out[idx], excl);
+      }
+      const float g = __shfl_sync(full, incl, 31);
+      const float tot = __shfl_sync(full, pm, 31);
+      if (lane == 0) {
+        sg[c] = g;
+        su[c] = g + tot;
+      }
+    }
+  }
+  if (!EXPV) return;
+  __syncthreads();
+  if (warp == 0) {
+    float carry = -INFINITY;
+    for (int cb = 0; cb < NC; cb += 32) {
+      const int c = cb + lane;
+      float g = c < NC ? sg[c] : 0.f;
+      float u = c < NC ? su[c] : -INFINITY;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float g2 = __shfl_up_sync(full, g, o);
+        const float u2 = __shfl_up_sync(full, u, o);
+        if (lane >= o) {
+          u = fmaxf(u2 + g, u);
+          g = g2 + g;
+        }
+      }
+      const float mc = fmaxf(carry + g, u);
+      if (c < NC) su[c] = mc;
+      carry = __shfl_sync(full, mc, 31);
+    }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int c = t / L;
+    const float mprev = c > 0 ? su[c - 1] : -INFINITY;
+    const size_t idx = base + t;
+    m_out[idx] = b_out[idx] + fmaxf(mprev, m_out[idx]);
+  }
+}
+
+cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  const size_t smem = p.exp_variant() ? 2 * sizeof(float) * (size_t)p.NC : 0;
+  dim3 grid(p.BH), block(256);
+  if (p.bf16()) {
+    if (p.exp_variant())
+      gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+    else
+      gate_prep_kernel<bf16, false><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+  } else {
+    if (p.exp_variant())
+      gate_prep_kernel<float, true><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+    else
+      gate_prep_kernel<float, false><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K-d0: per token, 1/den_t and the gradient of the stabilised normaliser,
+// da_t = -(dh_t . h_t) sign(a~_t) / den_t when |a~_t| > exp(-m_t), else 0
+// (den_t = max(|a~_t|, exp(-m_t)), h_t = num_t / den_t).  Also zeroes the
+// per-token dot-product accumulators.  One warp per token.
+// ---------------------------------------------------------------------------
+template <typename TIO, bool EXPV>
+__global__ void __launch_bounds__(256) bwd_token_prep_kernel(
+    const TIO* __restrict__ h, const TIO* __restrict__ dh, const float* __restrict__ abar,
+    const float* __restrict__ m, float* __restrict__ inv_den, float* __restrict__ da,
+    float* __restrict__ pq, float* __restrict__ pk, long long ntok, int dhv) {
+  const long long tok = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tok >= ntok) return;
+  if (lane == 0) {
+    pq[tok] = 0.f;
+    pk[tok] = 0.f;
+  }
+  if (!EXPV) {
+    if (lane == 0) inv_den[tok] = 1.f;
+    return;
+  }
+  float dot = 0.f;
+  const TIO* hr = h + tok * dhv;
+  const TIO* dr = dh + tok * dhv;
+  for (int j = lane; j < dhv; j += 32) dot += to_f32(hr[j]) * to_f32(dr[j]);
+  dot = warp_sum(dot);
+  if (lane == 0) {
+    const float a = abar[tok];
+    const float floor_ = expf(-m[tok]);
+    const float den = fmaxf(fabsf(a), floor_);
+    inv_den[tok] = 1.f / den;
+    da[tok] = fabsf(a) > floor_ ? -dot * copysignf(1.f, a) / den : 0.f;
+  }
+}
+
+cudaError_t launch_bwd_token_prep(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  const long long ntok = (long long)p.BH * p.T;
+  dim3 block(256), grid((unsigned)((ntok + 7) / 8));
+  if (p.bf16()) {
+    if (p.exp_variant())
+      bwd_token_prep_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.h, (const bf16*)a.dh, a.abar, a.m, a.inv_den, a.da, a.pq, a.pk, ntok, p.dhv);
+    else
+      bwd_token_prep_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.h, (const bf16*)a.dh, a.abar, a.m, a.inv_den, a.da, a.pq, a.pk, ntok, p.dhv);
+  } else {
+    if (p.exp_variant())
+      bwd_token_prep_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.h, (const float*)a.dh, a.abar, a.m, a.inv_den, a.da, a.pq, a.pk, ntok, p.dhv);
+    else
+      bwd_token_prep_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.h, (const float*)a.dh, a.abar, a.m, a.inv_den, a.da, a.pq, a.pk, ntok, p.dhv);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K-d3: gate gradients from the per-token dot products of the total
+// gradients.  With G_ts = dA_ts A_ts, d log i_s = sum_t G_ts = k_s . dk_s, and
+// d log f_r = sum_{t>=r} sum_{s<r} G_ts = sum_{t>=r} (q_t . dq_t - k_t . dk_t),
+// a reverse cumulative sum over the whole sequence.  Then the chain rule to
+// the preactivations: d/dx logsigmoid(x) = sigmoid(-x); the exponential input
+// gate has log i = i~.  One CTA (32 warps) per (b, h); each warp owns one
+// contiguous segment of T.
+// ---------------------------------------------------------------------------
+template <typename TIO, bool EXPV>
+__global__ void __launch_bounds__(1024) gate_grad_kernel(
+    const TIO* __restrict__ ig, const TIO* __restrict__ fg, const float* __restrict__ pq,
+    const float* __restrict__ pk, TIO* __restrict__ dig, TIO* __restrict__ dfg, int T) {
+  __shared__ float s_tot[32];
+  const size_t base = (size_t)blockIdx.x * T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = (T + 31) / 32;
+  const int sb = min(warp * seg, T), se = min(sb + seg, T);
+  float part = 0.f;
+  for (int t = sb + lane; t < se; t += 32) part += pq[base + t] - pk[base + t];
+  part = warp_sum(part);
+  if (lane == 0) s_tot[warp] = part;
+  __syncthreads();
+  if (warp == 0) {
+    const float x = s_tot[lane];
+    const float incl = warp_incl_suffix_sum(x);
+    s_tot[lane] = incl - x;  // sum of the later segments
+  }
+  __syncthreads();
+  float carry = s_tot[warp];
+  for (int e = se; e > sb; e -= 32) {
+    const int t = e - 32 + lane;
+    const bool valid = t >= sb;
+    const float pkt = valid ? pk[base + t] : 0.f;
+    const float x = valid ? pq[base + t] - pkt : 0.f;
+    const float sfx = warp_incl_suffix_sum(x);
+    const float dlf = carry + sfx;
+    carry += __shfl_sync(0xffffffffu, sfx, 0);
+    if (valid) {
+      const float f = to_f32(fg[base + t]);
+      dfg[base + t] = from_f32<TIO>(dlf * dlog_sigmoid(f));
+      const float dli = pkt;
+      dig[base + t] = from_f32<TIO>(EXPV ? dli : dli * dlog_sigmoid(to_f32(ig[base + t])));
+    }
+  }
+}
+
+cudaError_t launch_gate_grad(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  dim3 grid(p.BH), block(1024);
+  if (p.bf16()) {
+    if (p.exp_variant())
+      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T);
+    else
+      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T);
+  } else {
+    if (p.exp_variant())
+      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T);
+    else
+      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mlstm

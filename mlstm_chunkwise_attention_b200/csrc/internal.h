@@ -1,0 +1,55 @@
+// Internal interfaces between the C ABI (mlstm_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mlstm {
+
+struct Problem {
+  int B, NH, T, dqk, dhv, L, variant, dtype;
+  int BH, NC;
+  float scale;  // 1 / sqrt(d_qk)
+  bool exp_variant() const { return variant == 1; }
+  bool bf16() const { return dtype == 0; }
+};
+
+// Device pointers of one forward call.
+struct FwdArgs {
+  const void *q, *k, *v, *ig, *fg;
+  void* h;
+  float *b, *li, *m, *abar;  // per token [BH, T]
+  void* C;                   // [BH, NC, dqk, dhv] state entering each chunk
+  float* n;                  // [BH, NC, dqk]
+};
+
+// Device pointers of one backward call.
+struct BwdArgs {
+  const void *q, *k, *v, *ig, *fg, *h, *dh;
+  const float *b, *li, *m, *abar;
+  const void* C;
+  const float* n;
+  void *dq, *dk, *dv, *dig, *dfg;
+  float* inv_den;  // [BH, T] 1 / den_t
+  float* da;       // [BH, T] gradient of the stabilised normaliser (EXP)
+  float* pq;       // [BH, T] q_t . dq_t
+  float* pk;       // [BH, T] k_t . dk_t
+  void* dC;        // [BH, NC, dqk, dhv] gradient of the state leaving each chunk
+  float* dn;       // [BH, NC, dqk]
+};
+
+// gate kernels (gates.cu)
+cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_token_prep(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_gate_grad(const Problem& p, const BwdArgs& a, cudaStream_t s);
+
+// CUDA-core (fp32 FMA) kernels (simt_fwd.cu, simt_bwd.cu)
+cudaError_t launch_state_fwd_simt(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_output_fwd_simt(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dq_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dk_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dv_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
+
+}  // namespace mlstm

@@ -1,0 +1,310 @@
+// C ABI of the chunkwise mLSTM library: argument checks, buffer layouts and
+// the launch sequence of the forward and backward passes.  Declared in
+// include/mlstm.h, which states the operation, layouts, ownership and errors.
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "internal.h"
+#include "mlstm.h"
+
+namespace {
+
+using mlstm::Problem;
+
+constexpr int kMaxChunks = 6144;  // gate_prep keeps 2 floats per chunk in shared memory
+
+thread_local char g_last_error[256] = "";
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int check_sizes(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype) {
+  if (B < 0 || NH < 0 || T < 0 || d_qk <= 0 || d_hv <= 0 || chunk <= 0) return MLSTM_ERR_INVALID;
+  if (variant != MLSTM_SIG && variant != MLSTM_EXP) return MLSTM_ERR_INVALID;
+  if (dtype != MLSTM_BF16 && dtype != MLSTM_FP32) return MLSTM_ERR_INVALID;
+  if (!(d_qk == 64 || d_qk == 128 || d_qk == 256)) return MLSTM_ERR_UNSUPPORTED;
+  if (!(d_hv == 64 || d_hv == 128 || d_hv == 256 || d_hv == 512)) return MLSTM_ERR_UNSUPPORTED;
+  if (!is_pow2(chunk) || chunk < 64 || chunk > 4096) return MLSTM_ERR_UNSUPPORTED;
+  const long long tokens = (long long)B * NH * T;
+  if (tokens >= (1LL << 31)) return MLSTM_ERR_UNSUPPORTED;
+  if ((T + chunk - 1) / chunk > kMaxChunks) return MLSTM_ERR_UNSUPPORTED;
+  return MLSTM_OK;
+}
+
+Problem make_problem(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype) {
+  Problem p;
+  p.B = B; p.NH = NH; p.T = T; p.dqk = d_qk; p.dhv = d_hv; p.L = chunk;
+  p.variant = variant; p.dtype = dtype;
+  p.BH = B * NH;
+  p.NC = (T + chunk - 1) / chunk;
+  p.scale = 1.0f / sqrtf((float)d_qk);
+  return p;
+}
+
+void saved_layout(const Problem& p, mlstm_saved_layout_t* L) {
+  memset(L, 0, sizeof(*L));
+  const size_t tok = (size_t)p.BH * p.T;
+  const size_t state_elem = p.bf16() ? 2 : 4;
+  L->gate_b_bytes = tok * 4;
+  L->gate_li_bytes = tok * 4;
+  L->gate_m_bytes = p.exp_variant() ? tok * 4 : 0;
+  L->norm_bytes = p.exp_variant() ? tok * 4 : 0;
+  L->state_c_bytes = (size_t)p.BH * p.NC * p.dqk * p.dhv * state_elem;
+  L->state_n_bytes = p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0;
+  size_t off = 0;
+  L->gate_b = off;  off = align256(off + L->gate_b_bytes);
+  L->gate_li = off; off = align256(off + L->gate_li_bytes);
+  L->gate_m = off;  off = align256(off + L->gate_m_bytes);
+  L->norm = off;    off = align256(off + L->norm_bytes);
+  L->state_c = off; off = align256(off + L->state_c_bytes);
+  L->state_n = off; off = align256(off + L->state_n_bytes);
+  L->total = off;
+}
+
+struct BwdLayout {
+  size_t inv_den, da, pq, pk, dC, dn, total;
+};
+
+BwdLayout bwd_layout(const Problem& p) {
+  BwdLayout L;
+  const size_t tok = (size_t)p.BH * p.T;
+  const size_t state_elem = p.bf16() ? 2 : 4;
+  size_t off = 0;
+  L.inv_den = off; off = align256(off + tok * 4);
+  L.da = off;      off = align256(off + tok * 4);
+  L.pq = off;      off = align256(off + tok * 4);
+  L.pk = off;      off = align256(off + tok * 4);
+  L.dC = off;      off = align256(off + (size_t)p.BH * p.NC * p.dqk * p.dhv * state_elem);
+  L.dn = off;      off = align256(off + (p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0));
+  L.total = off;
+  return L;
+}
+
+bool misaligned(const void* ptr) { return ((uintptr_t)ptr & 15) != 0; }
+
+int cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return MLSTM_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+  return MLSTM_ERR_CUDA;
+}
+
+// Optional per-kernel timing events (mlstm_set_timing_events).
+thread_local void* const* g_events = nullptr;
+thread_local int g_nevents = 0;
+
+typedef cudaError_t (*FwdLauncher)(const Problem&, const mlstm::FwdArgs&, cudaStream_t);
+typedef cudaError_t (*BwdLauncher)(const Problem&, const mlstm::BwdArgs&, cudaStream_t);
+struct FwdStep { const char* name; FwdLauncher fn; };
+struct BwdStep { const char* name; BwdLauncher fn; };
+constexpr int kMaxSteps = 8;
+
+// The kernels each pass enqueues, in order.
+int fwd_plan(const Problem& p, FwdStep* st) {
+  (void)p;
+  int n = 0;
+  st[n++] = {"gate_prep", mlstm::launch_gate_prep};
+  st[n++] = {"state_fwd_simt", mlstm::launch_state_fwd_simt};
+  st[n++] = {"output_fwd_simt", mlstm::launch_output_fwd_simt};
+  return n;
+}
+
+int bwd_plan(const Problem& p, BwdStep* st) {
+  (void)p;
+  int n = 0;
+  st[n++] = {"bwd_token_prep", mlstm::launch_bwd_token_prep};
+  st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
+  st[n++] = {"dq_simt", mlstm::launch_dq_simt};
+  st[n++] = {"dk_simt", mlstm::launch_dk_simt};
+  st[n++] = {"dv_simt", mlstm::launch_dv_simt};
+  st[n++] = {"gate_grad", mlstm::launch_gate_grad};
+  return n;
+}
+
+template <typename Step, typename Args>
+int run_plan(const Step* steps, int n, const Problem& p, const Args& a, cudaStream_t s) {
+  for (int i = 0; i < n; ++i) {
+    if (g_events && 2 * i + 1 < g_nevents) {
+      int st = cuda_status(cudaEventRecord((cudaEvent_t)g_events[2 * i], s), "event record");
+      if (st != MLSTM_OK) return st;
+    }
+    int st = cuda_status(steps[i].fn(p, a, s), steps[i].name);
+    if (st != MLSTM_OK) return st;
+    if (g_events && 2 * i + 1 < g_nevents) {
+      st = cuda_status(cudaEventRecord((cudaEvent_t)g_events[2 * i + 1], s), "event record");
+      if (st != MLSTM_OK) return st;
+    }
+  }
+  return MLSTM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mlstm_saved_layout(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant,
+                       int dtype, mlstm_saved_layout_t* layout) {
+  if (!layout) return MLSTM_ERR_INVALID;
+  const int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  if (st != MLSTM_OK) return st;
+  saved_layout(make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype), layout);
+  return MLSTM_OK;
+}
+
+size_t mlstm_saved_size(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant,
+                        int dtype) {
+  mlstm_saved_layout_t L;
+  if (mlstm_saved_layout(B, NH, T, d_qk, d_hv, chunk, variant, dtype, &L) != MLSTM_OK) return 0;
+  return L.total;
+}
+
+size_t mlstm_fwd_workspace_size(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant,
+                                int dtype) {
+  return mlstm_saved_size(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+}
+
+size_t mlstm_bwd_workspace_size(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant,
+                                int dtype) {
+  if (check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype) != MLSTM_OK) return 0;
+  return bwd_layout(make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype)).total;
+}
+
+int mlstm_fwd_launch_count(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant,
+                           int dtype) {
+  if (check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype) != MLSTM_OK) return 0;
+  if ((long long)B * NH * T == 0) return 0;
+  FwdStep steps[kMaxSteps];
+  return fwd_plan(make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype), steps);
+}
+
+int mlstm_bwd_launch_count(int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant,
+                           int dtype) {
+  if (check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype) != MLSTM_OK) return 0;
+  if ((long long)B * NH * T == 0) return 0;
+  BwdStep steps[kMaxSteps];
+  return bwd_plan(make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype), steps);
+}
+
+const char* mlstm_launch_name(int pass, int index, int B, int NH, int T, int d_qk, int d_hv,
+                              int chunk, int variant, int dtype) {
+  if (check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype) != MLSTM_OK || index < 0) return "";
+  const Problem p = make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  if (pass == 0) {
+    FwdStep steps[kMaxSteps];
+    const int n = fwd_plan(p, steps);
+    return index < n ? steps[index].name : "";
+  }
+  if (pass == 1) {
+    BwdStep steps[kMaxSteps];
+    const int n = bwd_plan(p, steps);
+    return index < n ? steps[index].name : "";
+  }
+  return "";
+}
+
+int mlstm_set_timing_events(void* const* events, int count) {
+  if (count < 0 || (count > 0 && !events)) return MLSTM_ERR_INVALID;
+  g_events = count > 0 ? events : nullptr;
+  g_nevents = count;
+  return MLSTM_OK;
+}
+
+int mlstm_fwd(const void* q, const void* k, const void* v, const void* igate_pre,
+              const void* fgate_pre, void* h, void* saved, void* workspace,
+              size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
+              int variant, int dtype, void* stream) {
+  int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH * T == 0) return MLSTM_OK;
+  if (!q || !k || !v || !igate_pre || !fgate_pre || !h) return MLSTM_ERR_INVALID;
+  if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(h) ||
+      misaligned(igate_pre) || misaligned(fgate_pre) || misaligned(saved) ||
+      misaligned(workspace))
+    return MLSTM_ERR_INVALID;
+  const Problem p = make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  mlstm_saved_layout_t L;
+  saved_layout(p, &L);
+  char* base = (char*)saved;
+  if (!base) {
+    if (!workspace || workspace_bytes < L.total) return MLSTM_ERR_WORKSPACE;
+    base = (char*)workspace;
+  }
+  mlstm::FwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.ig = igate_pre; a.fg = fgate_pre; a.h = h;
+  a.b = (float*)(base + L.gate_b);
+  a.li = (float*)(base + L.gate_li);
+  a.m = p.exp_variant() ? (float*)(base + L.gate_m) : nullptr;
+  a.abar = p.exp_variant() ? (float*)(base + L.norm) : nullptr;
+  a.C = base + L.state_c;
+  a.n = p.exp_variant() ? (float*)(base + L.state_n) : nullptr;
+  cudaStream_t s = (cudaStream_t)stream;
+
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_fwd");
+  if (st != MLSTM_OK) return st;
+  FwdStep steps[kMaxSteps];
+  const int n = fwd_plan(p, steps);
+  return run_plan(steps, n, p, a, s);
+}
+
+int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre,
+              const void* fgate_pre, const void* h, const void* dh, const void* saved, void* dq,
+              void* dk, void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
+              size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
+              int variant, int dtype, void* stream) {
+  int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH * T == 0) return MLSTM_OK;
+  if (!q || !k || !v || !igate_pre || !fgate_pre || !h || !dh || !saved || !dq || !dk || !dv ||
+      !digate_pre || !dfgate_pre)
+    return MLSTM_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv,
+                        digate_pre, dfgate_pre, workspace};
+  for (const void* ptr : ptrs)
+    if (misaligned(ptr)) return MLSTM_ERR_INVALID;
+  const Problem p = make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  const BwdLayout W = bwd_layout(p);
+  if (!workspace || workspace_bytes < W.total) return MLSTM_ERR_WORKSPACE;
+  mlstm_saved_layout_t L;
+  saved_layout(p, &L);
+  const char* sv = (const char*)saved;
+  char* ws = (char*)workspace;
+  mlstm::BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.ig = igate_pre; a.fg = fgate_pre; a.h = h; a.dh = dh;
+  a.b = (const float*)(sv + L.gate_b);
+  a.li = (const float*)(sv + L.gate_li);
+  a.m = p.exp_variant() ? (const float*)(sv + L.gate_m) : nullptr;
+  a.abar = p.exp_variant() ? (const float*)(sv + L.norm) : nullptr;
+  a.C = sv + L.state_c;
+  a.n = p.exp_variant() ? (const float*)(sv + L.state_n) : nullptr;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dig = digate_pre; a.dfg = dfgate_pre;
+  a.inv_den = (float*)(ws + W.inv_den);
+  a.da = (float*)(ws + W.da);
+  a.pq = (float*)(ws + W.pq);
+  a.pk = (float*)(ws + W.pk);
+  a.dC = ws + W.dC;
+  a.dn = p.exp_variant() ? (float*)(ws + W.dn) : nullptr;
+  cudaStream_t s = (cudaStream_t)stream;
+
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_bwd");
+  if (st != MLSTM_OK) return st;
+  BwdStep steps[kMaxSteps];
+  const int n = bwd_plan(p, steps);
+  return run_plan(steps, n, p, a, s);
+}
+
+const char* mlstm_status_string(int status) {
+  switch (status) {
+    case MLSTM_OK: return "ok";
+    case MLSTM_ERR_INVALID: return "invalid argument";
+    case MLSTM_ERR_UNSUPPORTED: return "unsupported size";
+    case MLSTM_ERR_WORKSPACE: return "workspace or saved buffer too small";
+    case MLSTM_ERR_CUDA: return "CUDA error";
+    case MLSTM_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* mlstm_last_error(void) { return g_last_error; }
+
+}  // extern "C"

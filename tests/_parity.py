@@ -1,0 +1,59 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI,
+run the fp64 oracle on the same (I/O-dtype-rounded) inputs, compare."""
+
+import numpy as np
+import torch
+
+import oracle
+from mlstm_chunkwise_attention_b200 import binding
+from mlstm_chunkwise_attention_b200.synthetic import make_inputs
+
+# max|err| / max|ref| bounds for bf16 and fp32 I/O
+TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-4}
+
+
+def relerr(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "non-finite values in the CUDA result"
+    return float(np.max(np.abs(got - ref)) / max(float(np.max(np.abs(ref))), 1e-30))
+
+
+def np64(t):
+    return t.detach().double().cpu().numpy()
+
+
+def inputs(B, NH, T, d_qk, d_hv, seed, dtype, ig_mean=0.0, fg_mean=3.0, with_dh=True, **kw):
+    return make_inputs(B, NH, T, d_qk, d_hv, seed=seed, igate_mean=ig_mean, fgate_mean=fg_mean,
+                       dtype=dtype, with_dh=with_dh, **kw)
+
+
+def gpu_fwd(cpu, chunk, variant):
+    dev = {k: v.cuda() for k, v in cpu.items()}
+    h, saved = binding.forward(dev["q"], dev["k"], dev["v"], dev["igate"], dev["fgate"], chunk, variant)
+    torch.cuda.synchronize()
+    return dev, h, saved
+
+
+def gpu_bwd(dev, h, saved, chunk, variant):
+    g = binding.backward(dev["q"], dev["k"], dev["v"], dev["igate"], dev["fgate"], h, dev["dh"],
+                         saved, chunk, variant)
+    torch.cuda.synchronize()
+    return g
+
+
+def head64(cpu, b, hh):
+    return {k: np64(v[b, hh]) for k, v in cpu.items()}
+
+
+def oracle_fwd_head(x, chunk, variant):
+    li, lf = oracle.gate_logs(x["igate"], x["fgate"], variant)
+    return oracle.chunkwise_forward(x["q"], x["k"], x["v"], li, lf, variant, chunk)
+
+
+def oracle_bwd_head(x, variant):
+    li, lf = oracle.gate_logs(x["igate"], x["fgate"], variant)
+    g = oracle.parallel_backward(x["q"], x["k"], x["v"], li, lf, variant, x["dh"])
+    di, df = oracle.preact_grads(g["dlog_i"], g["dlog_f"], x["igate"], x["fgate"], variant)
+    return {"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "digate_pre": di, "dfgate_pre": df}

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI: the library loads, exports every function that
+include/*.h declares, and rejects bad arguments before touching the GPU."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from mlstm_chunkwise_attention_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for header in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(header).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(?:int|size_t|const\s+char\s*\*|void)\s*\**\s*(mlstm_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from mlstm_chunkwise_attention_b200 import _build
+        _build.build()
+    return B.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("mlstm_fwd", "mlstm_bwd", "mlstm_saved_size", "mlstm_fwd_workspace_size",
+                     "mlstm_bwd_workspace_size", "mlstm_status_string", "mlstm_saved_layout"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(B.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} declared in include/ but not exported"
+
+
+def test_binding_covers_every_declared_symbol():
+    assert declared_functions() <= set(B.EXPORTS)
+
+
+SIZES = dict(B=2, NH=3, T=300, d_qk=128, d_hv=128, chunk=128, variant=B.EXP, dtype=B.BF16)
+
+
+def sizes(**kw):
+    d = dict(SIZES)
+    d.update(kw)
+    return (d["B"], d["NH"], d["T"], d["d_qk"], d["d_hv"], d["chunk"], d["variant"], d["dtype"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(T=-5), 1), (dict(variant=2), 1), (dict(dtype=7), 1),
+    (dict(d_qk=0), 1), (dict(chunk=0), 1),
+    (dict(d_qk=96), 2), (dict(d_hv=32), 2), (dict(d_qk=512), 2), (dict(chunk=100), 2),
+    (dict(chunk=32), 2), (dict(chunk=8192), 2), (dict(B=1 << 16, NH=1 << 10, T=4096), 2),
+])
+def test_size_validation(lib, kw, status):
+    lay = B.SavedLayout()
+    assert lib.mlstm_saved_layout(*sizes(**kw), ctypes.byref(lay)) == status
+    assert lib.mlstm_saved_size(*sizes(**kw)) == 0
+    assert lib.mlstm_bwd_workspace_size(*sizes(**kw)) == 0
+    assert lib.mlstm_fwd(None, None, None, None, None, None, None, None, 0, *sizes(**kw), None) == status
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(lib):
+    fake = 1 << 20  # never dereferenced: validation fails before any launch
+    good = [fake] * 6
+    assert lib.mlstm_fwd(None, *good[1:], None, None, 0, *sizes(), None) == 1
+    assert lib.mlstm_fwd(fake + 4, *good[1:], fake, None, 0, *sizes(), None) == 1
+    # no saved buffer and no workspace
+    assert lib.mlstm_fwd(*good, None, None, 0, *sizes(), None) == 3
+    need = lib.mlstm_fwd_workspace_size(*sizes())
+    assert lib.mlstm_fwd(*good, None, fake, need - 1, *sizes(), None) == 3
+    bw = lib.mlstm_bwd_workspace_size(*sizes())
+    args13 = [fake] * 13
+    assert lib.mlstm_bwd(*args13, fake, bw - 1, *sizes(), None) == 3
+    assert lib.mlstm_bwd(*args13[:7], None, *args13[8:], fake, bw, *sizes(), None) == 1
+
+
+def test_empty_problem_is_a_noop(lib):
+    for kw in (dict(B=0), dict(NH=0), dict(T=0)):
+        assert lib.mlstm_fwd(None, None, None, None, None, None, None, None, 0, *sizes(**kw), None) == 0
+        assert lib.mlstm_bwd(*([None] * 13), None, 0, *sizes(**kw), None) == 0
+        assert lib.mlstm_fwd_launch_count(*sizes(**kw)) == 0
+
+
+def test_saved_layout_regions(lib):
+    for variant in (B.SIG, B.EXP):
+        for dtype in (B.BF16, B.FP32):
+            Bn, NH, T, dqk, dhv, L = 2, 3, 300, 128, 256, 128
+            lay = B.mlstm_saved_layout(Bn, NH, T, dqk, dhv, L, variant, dtype)
+            NC = (T + L - 1) // L
+            tok = Bn * NH * T
+            assert lay["gate_b_bytes"] == 4 * tok and lay["gate_li_bytes"] == 4 * tok
+            assert lay["gate_m_bytes"] == (4 * tok if variant == B.EXP else 0)
+            assert lay["norm_bytes"] == (4 * tok if variant == B.EXP else 0)
+            assert lay["state_c_bytes"] == Bn * NH * NC * dqk * dhv * (2 if dtype == B.BF16 else 4)
+            assert lay["state_n_bytes"] == (Bn * NH * NC * dqk * 4 if variant == B.EXP else 0)
+            regions = sorted((lay[n], lay[n + "_bytes"]) for n in
+                             ("gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n"))
+            end = 0
+            for off, nb in regions:
+                assert off % 256 == 0 and off >= end
+                end = off + nb
+            assert lay["total"] >= end
+            assert B.mlstm_saved_size(Bn, NH, T, dqk, dhv, L, variant, dtype) == lay["total"]
+            assert lib.mlstm_fwd_launch_count(Bn, NH, T, dqk, dhv, L, variant, dtype) > 0
+            assert lib.mlstm_bwd_launch_count(Bn, NH, T, dqk, dhv, L, variant, dtype) > 0
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert B.mlstm_status_string(code)
+    assert B.mlstm_status_string(99) == "unknown status"

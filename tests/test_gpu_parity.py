@@ -1,0 +1,220 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerance: max|err| / max|ref| <= 1e-2 for bf16 I/O and <= 1e-4 for fp32 I/O,
+per output tensor, on the same seeded inputs (the oracle reads the
+dtype-rounded values).  Small cases compare every element of every head;
+full-size workloads compare whole sampled heads (heads are independent) or
+sampled rows, plus properties that hold at any size.
+"""
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mlstm_chunkwise_attention_b200 import binding
+from mlstm_chunkwise_attention_b200.synthetic import WORKLOADS, sample_heads, sample_rows
+from _parity import (TOL, gpu_bwd, gpu_fwd, head64, inputs, np64, oracle_bwd_head,
+                     oracle_fwd_head, relerr)
+
+pytestmark = pytest.mark.gpu
+
+SIG, EXP = binding.SIG, binding.EXP
+F32, BF = torch.float32, torch.bfloat16
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _require_gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    binding.load()  # fails loudly if the library is not built
+
+
+# name, B, NH, T, d_qk, d_hv, chunk, variant, dtype, ig_mean, fg_mean
+SMALL = [
+    ("sig_fp32_b1h2_t256_d64", 1, 2, 256, 64, 64, 64, SIG, F32, 0.0, 3.0),
+    ("exp_fp32_ragged_t200", 1, 2, 200, 64, 128, 64, EXP, F32, -2.0, 3.0),
+    ("exp_bf16_multitile_ragged", 2, 2, 700, 128, 128, 256, EXP, BF, -2.0, 3.0),
+    ("sig_bf16_multitile_ragged", 2, 2, 700, 128, 128, 256, SIG, BF, 0.0, 3.0),
+    ("exp_bf16_dqk256_dhv512", 1, 2, 300, 256, 512, 128, EXP, BF, 0.0, 3.0),
+    ("sig_bf16_dqk256_dhv512", 1, 1, 300, 256, 512, 128, SIG, BF, -10.0, 4.0),
+    ("sig_bf16_igate_bias_m10", 1, 2, 512, 64, 64, 64, SIG, BF, -10.0, 4.0),
+    ("exp_bf16_igate_bias_m10", 1, 2, 512, 64, 64, 64, EXP, BF, -10.0, 3.0),
+    ("exp_bf16_one_partial_chunk", 1, 1, 37, 64, 64, 64, EXP, BF, 0.0, 3.0),
+    ("exp_fp32_t1", 1, 1, 1, 64, 64, 64, EXP, F32, 0.0, 3.0),
+    ("sig_bf16_chunk4096_ragged", 1, 1, 4500, 64, 64, 4096, SIG, BF, 0.0, 3.0),
+    ("exp_bf16_chunk1024", 1, 1, 2048, 128, 128, 1024, EXP, BF, 0.0, 3.0),
+    ("exp_fp32_dqk256", 1, 1, 384, 256, 64, 128, EXP, F32, 1.0, 2.0),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_forward_backward_all_heads(case):
+    name, Bn, NH, T, dqk, dhv, L, var, dt, igm, fgm = case
+    cpu = inputs(Bn, NH, T, dqk, dhv, seed=zlib.crc32(name.encode()) % 10000, dtype=dt, ig_mean=igm, fg_mean=fgm)
+    dev, h, saved = gpu_fwd(cpu, L, var)
+    g = gpu_bwd(dev, h, saved, L, var)
+    tol = TOL[dt]
+    for b in range(Bn):
+        for hh in range(NH):
+            x = head64(cpu, b, hh)
+            ref = oracle_fwd_head(x, L, var)
+            assert relerr(np64(h[b, hh]), ref["h"]) <= tol, f"h ({b},{hh})"
+            ref_g = oracle_bwd_head(x, var)
+            for key, val in ref_g.items():
+                err = relerr(np64(g[key][b, hh]), val)
+                assert err <= tol, f"{key} ({b},{hh}): {err:.3e}"
+
+
+@pytest.mark.parametrize("var", [SIG, EXP])
+def test_saved_gate_prep_and_states_match_oracle(var):
+    """K-a (cumsums, max states) and K-b (states entering each chunk)."""
+    Bn, NH, T, dqk, dhv, L = 1, 2, 320, 64, 128, 64
+    cpu = inputs(Bn, NH, T, dqk, dhv, seed=77, dtype=F32, ig_mean=-1.0, fg_mean=2.0, with_dh=False)
+    dev, h, saved = gpu_fwd(cpu, L, var)
+    sv = binding.saved_views(saved, dev["q"], dev["v"], L, var)
+    for hh in range(NH):
+        x = head64(cpu, 0, hh)
+        ref = oracle_fwd_head(x, L, var)
+        assert relerr(np64(sv["b"][hh]), ref["b"]) < 1e-5
+        assert relerr(np64(sv["log_i"][hh]), ref["log_i"]) < 1e-5
+        assert relerr(np64(sv["C"][hh]), ref["C_enter"]) < 1e-5
+        if var == EXP:
+            np.testing.assert_allclose(np64(sv["m"][hh]), ref["m_row"], rtol=1e-5, atol=1e-4)
+            assert relerr(np64(sv["abar"][hh]), ref["abar"]) < 1e-5
+            assert relerr(np64(sv["n"][hh]), ref["n_enter"]) < 1e-5
+
+
+def _preact(v, T):
+    return torch.full((1, 1, T), float(v), dtype=F32)
+
+
+def test_open_gates_sig_is_causal_linear_attention():
+    T, d = 200, 64
+    cpu = inputs(1, 1, T, d, d, seed=5, dtype=F32, with_dh=False)
+    cpu["igate"] = _preact(200.0, T)
+    cpu["fgate"] = _preact(200.0, T)
+    _, h, _ = gpu_fwd(cpu, 64, SIG)
+    q, k, v = (np64(cpu[n][0, 0]) for n in ("q", "k", "v"))
+    want = np.tril(q @ k.T / np.sqrt(d)) @ v
+    assert relerr(np64(h[0, 0]), want) <= 1e-4
+
+
+@pytest.mark.parametrize("var", [SIG, EXP])
+def test_closed_forget_gate_is_one_step_readout(var):
+    T, d = 130, 64
+    cpu = inputs(1, 1, T, d, d, seed=6, dtype=F32, with_dh=False)
+    cpu["fgate"] = _preact(-200.0, T)
+    _, h, _ = gpu_fwd(cpu, 64, var)
+    q, k, v, ig = (np64(cpu[n][0, 0]) for n in ("q", "k", "v", "igate"))
+    s = np.einsum("td,td->t", q, k) / np.sqrt(d)
+    if var == SIG:
+        want = (s / (1.0 + np.exp(-ig)))[:, None] * v
+    else:
+        want = (s / np.maximum(np.abs(s), np.exp(-ig)))[:, None] * v
+    assert relerr(np64(h[0, 0]), want) <= 1e-4
+
+
+def test_constant_decay_is_retention():
+    T, d, gamma = 256, 64, 0.95
+    cpu = inputs(1, 1, T, d, d, seed=7, dtype=F32, with_dh=False)
+    cpu["igate"] = _preact(200.0, T)
+    cpu["fgate"] = _preact(np.log(gamma / (1 - gamma)), T)
+    _, h, _ = gpu_fwd(cpu, 64, SIG)
+    q, k, v = (np64(cpu[n][0, 0]) for n in ("q", "k", "v"))
+    gam = 1.0 / (1.0 + np.exp(-float(cpu["fgate"][0, 0, 0])))
+    idx = np.arange(T)
+    lag = idx[:, None] - idx[None, :]
+    want = ((q @ k.T / np.sqrt(d)) * np.where(lag >= 0, gam ** np.clip(lag, 0, None), 0.0)) @ v
+    assert relerr(np64(h[0, 0]), want) <= 1e-4
+
+
+def test_chunk_size_invariance_on_gpu():
+    """The same inputs through chunk 64, 128, 256 and 512 give the same h."""
+    cpu = inputs(1, 2, 1024, 64, 64, seed=8, dtype=F32, with_dh=False)
+    outs = [np64(gpu_fwd(cpu, L, EXP)[1]) for L in (64, 128, 256, 512)]
+    for o in outs[1:]:
+        assert relerr(o, outs[0]) <= 1e-5
+
+
+def test_repeat_calls_are_deterministic_forward():
+    cpu = inputs(1, 2, 300, 64, 64, seed=9, dtype=BF, with_dh=False)
+    a = np64(gpu_fwd(cpu, 64, EXP)[1])
+    b = np64(gpu_fwd(cpu, 64, EXP)[1])
+    assert np.array_equal(a, b)
+
+
+def test_host_errors_on_device_buffers():
+    cpu = inputs(1, 1, 128, 64, 64, seed=10, dtype=BF, with_dh=False)
+    dev = {k: v.cuda() for k, v in cpu.items()}
+    sizes = binding.problem_sizes(dev["q"], dev["v"], 64, EXP)
+    h = torch.empty_like(dev["v"])
+    need = binding.mlstm_fwd_workspace_size(*sizes)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ptr = [dev[n].data_ptr() for n in ("q", "k", "v", "igate", "fgate")]
+    st = binding.mlstm_fwd(*ptr, h.data_ptr(), None, ws.data_ptr(), need - 1, *sizes, None)
+    assert st == 3
+    st = binding.mlstm_fwd(ptr[0] + 2, *ptr[1:], h.data_ptr(), None, ws.data_ptr(), need, *sizes, None)
+    assert st == 1
+    st = binding.mlstm_fwd(*ptr, h.data_ptr(), None, ws.data_ptr(), need, *sizes, None)
+    assert st == 0
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the benchmark times
+# ---------------------------------------------------------------------------
+
+def _full(name, variant=None, heads_fwd=2, heads_bwd=1, rows=24, whole_bwd=True):
+    spec = dict(WORKLOADS[name])
+    if variant is not None:
+        spec["variant"] = variant
+    dt = BF if spec["dtype"] == "bf16" else F32
+    cpu = inputs(spec["B"], spec["NH"], spec["T"], spec["d_qk"], spec["d_hv"], seed=spec["seed"],
+                 dtype=dt, ig_mean=spec["igate_mean"], fg_mean=spec["fgate_mean"])
+    L, var = spec["chunk"], spec["variant"]
+    dev, h, saved = gpu_fwd(cpu, L, var)
+    g = gpu_bwd(dev, h, saved, L, var)
+    tol = TOL[dt]
+    for (b, hh) in sample_heads(spec["B"], spec["NH"], heads_fwd, spec["seed"]):
+        x = head64(cpu, b, hh)
+        ref = oracle_fwd_head(x, L, var)
+        assert relerr(np64(h[b, hh]), ref["h"]) <= tol, f"h ({b},{hh})"
+    for (b, hh) in sample_heads(spec["B"], spec["NH"], heads_bwd, spec["seed"] + 1):
+        x = head64(cpu, b, hh)
+        if whole_bwd:
+            ref_g = oracle_bwd_head(x, var)
+            for key, val in ref_g.items():
+                err = relerr(np64(g[key][b, hh]), val)
+                assert err <= tol, f"{key} ({b},{hh}): {err:.3e}"
+        else:
+            fwd = oracle_fwd_head(x, L, var)
+            li, lf = oracle.gate_logs(x["igate"], x["fgate"], var)
+            a = fwd["abar"] * np.exp(fwd["m_row"]) if var == EXP else np.zeros(spec["T"])
+            den = np.maximum(np.abs(a), 1.0) if var == EXP else np.ones(spec["T"])
+            rr = sample_rows(spec["T"], rows, spec["seed"], L)
+            gr = oracle.parallel_backward_rows(x["q"], x["k"], x["v"], li, lf, var, x["dh"],
+                                               fwd["h"], a, den, rr)
+            di, _ = oracle.preact_grads(gr["dlog_i"], np.zeros(len(rr)), x["igate"][rr],
+                                        x["fgate"][rr], var)
+            for key, val in (("dq", gr["dq"]), ("dk", gr["dk"]), ("dv", gr["dv"]), ("digate_pre", di)):
+                full = np64(g[key][b, hh])
+                scale = np.max(np.abs(full))
+                err = np.max(np.abs(full[rr] - val)) / max(scale, 1e-30)
+                assert err <= tol, f"{key} rows ({b},{hh}): {err:.3e}"
+            # d log f_r = sum_{t>=r} (q_t.dq_t - k_t.dk_t), a property at any size
+            q, k = x["q"], x["k"]
+            dF = np.einsum("td,td->t", q, np64(g["dq"][b, hh])) - np.einsum("td,td->t", k, np64(g["dk"][b, hh]))
+            dlf = np.cumsum(dF[::-1])[::-1]
+            want = dlf * oracle.sigmoid(-x["fgate"])
+            assert relerr(np64(g["dfgate_pre"][b, hh]), want) <= tol
+
+
+def test_full_headline_exp_b8h32_t4096_fwd_bwd():
+    _full("exp_b8h32_t4096_d128_c128", heads_fwd=3, heads_bwd=1, whole_bwd=True)
+
+
+@pytest.mark.parametrize("var", [SIG, EXP])
+def test_full_training_b4h16_t8192_d256(var):
+    _full("train_b4h16_t8192_d256_c256", variant=var, heads_fwd=1, heads_bwd=1, whole_bwd=False)
