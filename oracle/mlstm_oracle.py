@@ -227,33 +227,35 @@ def chunkwise_forward(q, k, v, log_i, log_f, variant, L):
     a3. outputs: h_t = [alpha_t q'_t C_{k-1} + sum_{s<=t} D_ts (q'_t.k_s) v_s] / den_t
         with alpha_t = exp(b_t + m_{k-1} - m_t), D_ts = exp(b_t - b_s + log i_s - m_t),
         den_t = max(|alpha_t q'_t.n_{k-1} + sum_s D_ts q'_t.k_s|, exp(-m_t)) (EXP), 1 (SIG).
+
+    When L does not divide T the last chunk holds the remaining T mod L rows.
     """
     q, k, v, log_i, log_f = _as64(q, k, v, log_i, log_f)
     T, d_qk = q.shape
     d_hv = v.shape[1]
-    if L < 1 or T % L != 0:
-        raise ValueError("chunk size must divide T")
-    NC = T // L
+    if L < 1:
+        raise ValueError("chunk size must be positive")
+    NC = -(-T // L)
+    bounds = [(c * L, min((c + 1) * L, T)) for c in range(NC)]
     qs = q / np.sqrt(d_qk)
     exp_variant = variant == EXP
 
     # a1: gate preprocessing
     b = np.empty(T)
-    for c in range(NC):
-        sl = slice(c * L, (c + 1) * L)
-        b[sl] = np.cumsum(log_f[sl])
-    g = b[L - 1 :: L].copy()
+    for (lo, hi) in bounds:
+        b[lo:hi] = np.cumsum(log_f[lo:hi])
+    g = np.array([b[hi - 1] for (_, hi) in bounds])
     m_row = np.zeros(T)
     m_state = np.zeros(NC)
     m_enter = np.zeros(NC)
     if exp_variant:
         m_prev = -np.inf
-        for c in range(NC):
-            sl = slice(c * L, (c + 1) * L)
+        for c, (lo, hi) in enumerate(bounds):
+            sl = slice(lo, hi)
             u = np.maximum.accumulate(log_i[sl] - b[sl])
             m_row[sl] = b[sl] + np.maximum(m_prev, u)
             m_enter[c] = m_prev
-            m_state[c] = m_row[(c + 1) * L - 1]
+            m_state[c] = m_row[hi - 1]
             m_prev = m_state[c]
 
     # a2: inter-chunk states (state entering chunk c)
@@ -261,10 +263,10 @@ def chunkwise_forward(q, k, v, log_i, log_f, variant, L):
     n_enter = np.zeros((NC, d_qk))
     C = np.zeros((d_qk, d_hv))
     n = np.zeros(d_qk)
-    for c in range(NC):
+    for c, (lo, hi) in enumerate(bounds):
         C_enter[c] = C
         n_enter[c] = n
-        sl = slice(c * L, (c + 1) * L)
+        sl = slice(lo, hi)
         if exp_variant:
             beta = np.exp(g[c] + m_enter[c] - m_state[c])
             w = np.exp(g[c] - b[sl] + log_i[sl] - m_state[c])
@@ -278,9 +280,9 @@ def chunkwise_forward(q, k, v, log_i, log_f, variant, L):
     h = np.empty((T, d_hv))
     abar = np.zeros(T)
     den = np.ones(T)
-    tril = np.tril(np.ones((L, L), dtype=bool))
-    for c in range(NC):
-        sl = slice(c * L, (c + 1) * L)
+    for c, (lo, hi) in enumerate(bounds):
+        sl = slice(lo, hi)
+        tril = np.tril(np.ones((hi - lo, hi - lo), dtype=bool))
         bt = b[sl]
         mt = m_row[sl]
         alpha = np.exp(bt + m_enter[c] - mt) if exp_variant else np.exp(bt)

@@ -172,7 +172,7 @@ def check_huge_input_gates(M):
     assert rel(M.chunkwise_forward(q, k, v, li, lf, EXP, 4)["h"], s["h"]) < 1e-12
 
 
-def check_chunk_invariance(M, variant, T=48, L=16):
+def check_chunk_invariance(M, variant, T=50, L=16):
     q, k, v, ig, fg = rnd(100 + T + L, T, 8, 5, -1.0, 2.0)
     li, lf = M.gate_logs(ig, fg, variant)
     r = M.recurrent_forward(q, k, v, li, lf, variant)["h"]
@@ -337,7 +337,8 @@ def test_stabilised_survives_huge_input_gates():
 
 
 @pytest.mark.parametrize("variant", [SIG, EXP])
-@pytest.mark.parametrize("T,L", [(8, 1), (8, 2), (8, 4), (8, 8), (48, 16), (64, 64), (60, 12)])
+@pytest.mark.parametrize("T,L", [(8, 1), (8, 2), (8, 4), (8, 8), (48, 16), (64, 64), (60, 12),
+                                 (50, 16), (7, 4), (5, 8), (33, 32)])
 def test_chunkwise_invariant_to_chunk_size(variant, T, L):
     check_chunk_invariance(oracle, variant, T, L)
 
@@ -391,7 +392,10 @@ MUTATIONS = [
     ("forget chain rule sign", "dfgate = np.asarray(dlog_f) * sigmoid(-np.asarray(fgate_pre", "dfgate = np.asarray(dlog_f) * sigmoid(np.asarray(fgate_pre"),
     ("bptt forget grad uses C_t", "df[t] = np.sum(dC * Cs[t]) + dn @ ns[t]", "df[t] = np.sum(dC * Cs[t + 1]) + dn @ ns[t]"),
     ("column dA misses da", "dA_col = dnum[r:] @ v[r] + da[r:]", "dA_col = dnum[r:] @ v[r]"),
-    ("chunk mask misses diagonal", "tril = np.tril(np.ones((L, L), dtype=bool))", "tril = np.tril(np.ones((L, L), dtype=bool), -1)"),
+    ("chunk mask misses diagonal", "tril = np.tril(np.ones((hi - lo, hi - lo), dtype=bool))",
+     "tril = np.tril(np.ones((hi - lo, hi - lo), dtype=bool), -1)"),
+    ("chunk decay taken at the wrong row", "g = np.array([b[hi - 1] for (_, hi) in bounds])",
+     "g = np.array([b[lo] for (lo, _) in bounds])"),
 ]
 
 
