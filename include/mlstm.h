@@ -75,8 +75,10 @@ typedef enum {
  *   gate_m   float [BH, T]    EXP: max state m_t of the recurrence
  *   norm     float [BH, T]    EXP: stabilised normaliser  n~_t . q'_t
  *   state_c  [BH, NC, d_qk, d_hv]  state entering each chunk (EXP: scaled
- *            by exp(-m) of the chunk's previous row); bf16 on the bf16 path,
- *            float on the fp32 path
+ *            by exp(-m) of the chunk's previous row).  fp32 path: one float
+ *            plane.  bf16 path: two bf16 planes back to back, hi = bf16(C)
+ *            then lo = bf16(C - hi), so hi + lo keeps about 16 mantissa bits
+ *            for the backward pass
  *   state_n  float [BH, NC, d_qk]  EXP: normaliser state entering each chunk */
 typedef struct {
   size_t gate_b, gate_li, gate_m, norm, state_c, state_n;
@@ -128,6 +130,12 @@ int mlstm_bwd(const void* q, const void* k, const void* v,
               void* workspace, size_t workspace_bytes,
               int B, int NH, int T, int d_qk, int d_hv, int chunk,
               int variant, int dtype, void* stream);
+
+/* Synchronise `stream` and report what the kernels enqueued so far found:
+ * MLSTM_ERR_TIMEOUT if one of them gave up a bounded wait (its outputs are
+ * then invalid; the flag is cleared by this call), MLSTM_ERR_CUDA on a CUDA
+ * error, else MLSTM_OK.  This is the one call that blocks. */
+int mlstm_device_status(void* stream);
 
 /* Static text for a status code. */
 const char* mlstm_status_string(int status);

@@ -55,6 +55,7 @@ EXPORTS = {
     "mlstm_last_error": (ctypes.c_char_p, []),
     "mlstm_launch_name": (ctypes.c_char_p, [ctypes.c_int, ctypes.c_int] + _SIZES),
     "mlstm_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
+    "mlstm_device_status": (ctypes.c_int, [_P]),
 }
 
 
@@ -123,6 +124,17 @@ def mlstm_bwd(q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv, digate_pr
 
 def mlstm_status_string(status):
     return load().mlstm_status_string(status).decode()
+
+
+def mlstm_device_status(stream=None):
+    return load().mlstm_device_status(stream)
+
+
+def check_device(stream=None):
+    """Raise if a kernel enqueued so far reported a timeout or a CUDA error."""
+    st = mlstm_device_status(stream)
+    if st != STATUS_OK:
+        raise MLSTMError(st, "device status")
 
 
 def mlstm_last_error():
@@ -238,12 +250,16 @@ def saved_views(saved, q, v, chunk, variant):
             return None
         return saved[lay[name]: lay[name] + nbytes].view(dt).view(*shape)
 
-    sdt = torch.bfloat16 if dtype == BF16 else torch.float32
+    if dtype == BF16:  # two bf16 planes: hi then lo
+        planes = view("state_c", (2, BH, NC, d_qk, d_hv), torch.bfloat16)
+        C = planes[0].float() + planes[1].float()
+    else:
+        C = view("state_c", (BH, NC, d_qk, d_hv), torch.float32)
     return {
         "b": view("gate_b", (BH, T), torch.float32),
         "log_i": view("gate_li", (BH, T), torch.float32),
         "m": view("gate_m", (BH, T), torch.float32),
         "abar": view("norm", (BH, T), torch.float32),
-        "C": view("state_c", (BH, NC, d_qk, d_hv), sdt),
+        "C": C,
         "n": view("state_n", (BH, NC, d_qk), torch.float32),
     }

@@ -17,6 +17,30 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
 
+// Chunk states on the bf16 path are kept as two bf16 planes, hi = bf16(C) and
+// lo = bf16(C - hi), so hi + lo carries about 16 mantissa bits: the tensor-core
+// forward reads hi alone, the backward reads both.  The fp32 path keeps one
+// fp32 plane.  `plane` is the element count of one plane.
+template <typename TS> struct StatePlanes;
+template <> struct StatePlanes<float> {
+  static __device__ __forceinline__ void store(float* base, size_t, size_t i, float x, bool) {
+    base[i] = x;
+  }
+  static __device__ __forceinline__ float load(const float* base, size_t, size_t i, bool = true) {
+    return base[i];
+  }
+};
+template <> struct StatePlanes<bf16> {
+  static __device__ __forceinline__ void store(bf16* base, size_t plane, size_t i, float x, bool lo) {
+    const bf16 hi = __float2bfloat16_rn(x);
+    base[i] = hi;
+    if (lo) base[plane + i] = __float2bfloat16_rn(x - __bfloat162float(hi));
+  }
+  static __device__ __forceinline__ float load(const bf16* base, size_t plane, size_t i, bool lo = true) {
+    return __bfloat162float(base[i]) + (lo ? __bfloat162float(base[plane + i]) : 0.f);
+  }
+};
+
 // log sigmoid(x) = min(x, 0) - log(1 + exp(-|x|)); no overflow for any x.
 __device__ __forceinline__ float log_sigmoid(float x) {
   return fminf(x, 0.f) - log1pf(expf(-fabsf(x)));

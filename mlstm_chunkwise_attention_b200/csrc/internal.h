@@ -20,8 +20,9 @@ struct FwdArgs {
   const void *q, *k, *v, *ig, *fg;
   void* h;
   float *b, *li, *m, *abar;  // per token [BH, T]
-  void* C;                   // [BH, NC, dqk, dhv] state entering each chunk
+  void* C;                   // [BH, NC, dqk, dhv] state entering each chunk (planes, see StatePlanes)
   float* n;                  // [BH, NC, dqk]
+  bool keep_lo;              // write the low plane of bf16 states (needed by the backward)
 };
 
 // Device pointers of one backward call.
@@ -35,7 +36,7 @@ struct BwdArgs {
   float* da;       // [BH, T] gradient of the stabilised normaliser (EXP)
   float* pq;       // [BH, T] q_t . dq_t
   float* pk;       // [BH, T] k_t . dk_t
-  void* dC;        // [BH, NC, dqk, dhv] gradient of the state leaving each chunk
+  float* dC;       // [BH, NC, dqk, dhv] gradient of the state leaving each chunk (fp32)
   float* dn;       // [BH, NC, dqk]
 };
 
@@ -51,5 +52,12 @@ cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream
 cudaError_t launch_dq_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dk_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dv_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
+
+// tensor-core kernels (tc_*.cu) and their host helpers (tmap.cu)
+bool make_tmap_3d_bf16(void* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                       uint32_t box_inner, uint32_t box_mid);
+bool output_fwd_tc_supported(const Problem& p);
+cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t fetch_tc_fwd_error(unsigned int* flag);
 
 }  // namespace mlstm

@@ -51,7 +51,8 @@ void saved_layout(const Problem& p, mlstm_saved_layout_t* L) {
   L->gate_li_bytes = tok * 4;
   L->gate_m_bytes = p.exp_variant() ? tok * 4 : 0;
   L->norm_bytes = p.exp_variant() ? tok * 4 : 0;
-  L->state_c_bytes = (size_t)p.BH * p.NC * p.dqk * p.dhv * state_elem;
+  // bf16 path: hi and lo bf16 planes; fp32 path: one fp32 plane
+  L->state_c_bytes = (size_t)p.BH * p.NC * p.dqk * p.dhv * (p.bf16() ? 2 * state_elem : state_elem);
   L->state_n_bytes = p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0;
   size_t off = 0;
   L->gate_b = off;  off = align256(off + L->gate_b_bytes);
@@ -70,13 +71,12 @@ struct BwdLayout {
 BwdLayout bwd_layout(const Problem& p) {
   BwdLayout L;
   const size_t tok = (size_t)p.BH * p.T;
-  const size_t state_elem = p.bf16() ? 2 : 4;
   size_t off = 0;
   L.inv_den = off; off = align256(off + tok * 4);
   L.da = off;      off = align256(off + tok * 4);
   L.pq = off;      off = align256(off + tok * 4);
   L.pk = off;      off = align256(off + tok * 4);
-  L.dC = off;      off = align256(off + (size_t)p.BH * p.NC * p.dqk * p.dhv * state_elem);
+  L.dC = off;      off = align256(off + (size_t)p.BH * p.NC * p.dqk * p.dhv * 4);
   L.dn = off;      off = align256(off + (p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0));
   L.total = off;
   return L;
@@ -102,11 +102,13 @@ constexpr int kMaxSteps = 8;
 
 // The kernels each pass enqueues, in order.
 int fwd_plan(const Problem& p, FwdStep* st) {
-  (void)p;
   int n = 0;
   st[n++] = {"gate_prep", mlstm::launch_gate_prep};
   st[n++] = {"state_fwd_simt", mlstm::launch_state_fwd_simt};
-  st[n++] = {"output_fwd_simt", mlstm::launch_output_fwd_simt};
+  if (mlstm::output_fwd_tc_supported(p))
+    st[n++] = {"output_fwd_tc", mlstm::launch_output_fwd_tc};
+  else
+    st[n++] = {"output_fwd_simt", mlstm::launch_output_fwd_simt};
   return n;
 }
 
@@ -238,6 +240,7 @@ int mlstm_fwd(const void* q, const void* k, const void* v, const void* igate_pre
   a.abar = p.exp_variant() ? (float*)(base + L.norm) : nullptr;
   a.C = base + L.state_c;
   a.n = p.exp_variant() ? (float*)(base + L.state_n) : nullptr;
+  a.keep_lo = saved != nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_fwd");
@@ -282,7 +285,7 @@ int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre
   a.da = (float*)(ws + W.da);
   a.pq = (float*)(ws + W.pq);
   a.pk = (float*)(ws + W.pk);
-  a.dC = ws + W.dC;
+  a.dC = (float*)(ws + W.dC);
   a.dn = p.exp_variant() ? (float*)(ws + W.dn) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
@@ -306,5 +309,18 @@ const char* mlstm_status_string(int status) {
 }
 
 const char* mlstm_last_error(void) { return g_last_error; }
+
+int mlstm_device_status(void* stream) {
+  int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
+  if (st != MLSTM_OK) return st;
+  unsigned int flag = 0;
+  st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
+  if (st != MLSTM_OK) return st;
+  if (flag) {
+    snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
+    return MLSTM_ERR_TIMEOUT;
+  }
+  return MLSTM_OK;
+}
 
 }  // extern "C"

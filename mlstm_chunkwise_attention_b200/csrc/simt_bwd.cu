@@ -28,7 +28,7 @@ template <typename TIO, typename TS, bool EXPV>
 __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ dh, const float* __restrict__ b,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
-    TS* __restrict__ dC, float* __restrict__ dn, int T, int L, int NC, int dqk, int dhv,
+    float* __restrict__ dC, float* __restrict__ dn, int T, int L, int NC, int dqk, int dhv,
     float scale) {
   __shared__ float sQ[32][64];
   __shared__ float sD[32][64];
@@ -45,12 +45,11 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
   float nacc = 0.f;
 
   for (int c = NC - 1; c >= 0; --c) {
-    TS* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
+    float* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        Gc[(size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] = from_f32<TS>(acc[i][j]);
+      for (int j = 0; j < 4; ++j) Gc[(size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] = acc[i][j];
     if (own_n) dn[((size_t)bh * NC + c) * dqk + i0 + tid] = nacc;
     if (c == 0) break;
 
@@ -109,7 +108,7 @@ cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream
   dim3 grid(p.BH, p.dqk / 64, p.dhv / 64), block(256);
 #define MLSTM_STATE_BWD(TIO, TS, E)                                                             \
   state_bwd_simt_kernel<TIO, TS, E><<<grid, block, 0, s>>>(                                     \
-      (const TIO*)a.q, (const TIO*)a.dh, a.b, a.m, a.inv_den, a.da, (TS*)a.dC, a.dn, p.T, p.L, \
+      (const TIO*)a.q, (const TIO*)a.dh, a.b, a.m, a.inv_den, a.da, a.dC, a.dn, p.T, p.L,       \
       p.NC, p.dqk, p.dhv, p.scale)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_STATE_BWD(bf16, bf16, true);
@@ -206,7 +205,7 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
     const TIO* __restrict__ dh, const float* __restrict__ b, const float* __restrict__ li,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
     const TS* __restrict__ C, const float* __restrict__ n, TIO* __restrict__ dq,
-    float* __restrict__ pq, int T, int L, int NC, int dqk, int dhv, float scale) {
+    float* __restrict__ pq, int T, int L, int NC, int dqk, int dhv, float scale, size_t plane) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -222,13 +221,13 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
   zero44(acc);
 
   if (c > 0) {  // alpha_t (C_{c-1} dnum_t + da_t n_{c-1})
-    const TS* Cc = C + ((size_t)bh * NC + c) * dqk * dhv;
+    const size_t cbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dhv; x0 += 32) {
       __syncthreads();
       for (int e = tid; e < 64 * 32; e += 256) {
         const int r = e >> 5, x = e & 31, t = t0 + r;
         S.a[x * kP + r] = t < len ? to_f32(dh[(tok0 + t) * dhv + x0 + x]) * S.tinv[r] : 0.f;
-        S.bt[x * kP + r] = to_f32(Cc[(size_t)(i0 + r) * dhv + x0 + x]);
+        S.bt[x * kP + r] = StatePlanes<TS>::load(C, plane, cbase + (size_t)(i0 + r) * dhv + x0 + x);
       }
       __syncthreads();
       mac44(acc, S.a, kP, S.bt, kP, 32, ty, tx);
@@ -304,7 +303,7 @@ __global__ void __launch_bounds__(256) dk_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ v,
     const TIO* __restrict__ dh, const float* __restrict__ b, const float* __restrict__ li,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
-    const TS* __restrict__ dC, const float* __restrict__ dn, TIO* __restrict__ dk,
+    const float* __restrict__ dC, const float* __restrict__ dn, TIO* __restrict__ dk,
     float* __restrict__ pk, int T, int L, int NC, int dqk, int dhv, float scale) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
@@ -322,13 +321,13 @@ __global__ void __launch_bounds__(256) dk_simt_kernel(
   zero44(acc);
 
   if (c < NC - 1) {  // w_s (dC_c v_s + dn_c)
-    const TS* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
+    const float* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dhv; x0 += 32) {
       __syncthreads();
       for (int e = tid; e < 64 * 32; e += 256) {
         const int r = e >> 5, x = e & 31, s = s0 + r;
         S.a[x * kP + r] = s < len ? to_f32(v[(tok0 + s) * dhv + x0 + x]) : 0.f;
-        S.bt[x * kP + r] = to_f32(Gc[(size_t)(i0 + r) * dhv + x0 + x]);
+        S.bt[x * kP + r] = Gc[(size_t)(i0 + r) * dhv + x0 + x];
       }
       __syncthreads();
       mac44(acc, S.a, kP, S.bt, kP, 32, ty, tx);
@@ -401,7 +400,7 @@ template <typename TIO, typename TS, bool EXPV>
 __global__ void __launch_bounds__(256) dv_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ dh,
     const float* __restrict__ b, const float* __restrict__ li, const float* __restrict__ m,
-    const float* __restrict__ inv_den, const TS* __restrict__ dC, TIO* __restrict__ dv, int T,
+    const float* __restrict__ inv_den, const float* __restrict__ dC, TIO* __restrict__ dv, int T,
     int L, int NC, int dqk, int dhv, float scale) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
@@ -419,7 +418,7 @@ __global__ void __launch_bounds__(256) dv_simt_kernel(
   zero44(acc);
 
   if (c < NC - 1) {  // w_s dC_c^T k_s
-    const TS* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
+    const float* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dqk; x0 += 32) {
       __syncthreads();
       for (int e = tid; e < 64 * 32; e += 256) {
@@ -428,7 +427,7 @@ __global__ void __launch_bounds__(256) dv_simt_kernel(
       }
       for (int e = tid; e < 32 * 64; e += 256) {
         const int x = e >> 6, col = e & 63;
-        S.w[x * 64 + col] = to_f32(Gc[(size_t)(x0 + x) * dhv + j0 + col]);
+        S.w[x * 64 + col] = Gc[(size_t)(x0 + x) * dhv + j0 + col];
       }
       __syncthreads();
       mac44(acc, S.a, kP, S.w, 64, 32, ty, tx);
@@ -493,7 +492,7 @@ static cudaError_t dq_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dq_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, (const TIO*)a.dh, a.b, a.li, a.m,
       a.inv_den, a.da, (const TS*)a.C, a.n, (TIO*)a.dq, a.pq, p.T, p.L, p.NC, p.dqk, p.dhv,
-      p.scale);
+      p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv);
   return cudaGetLastError();
 }
 
@@ -506,7 +505,7 @@ static cudaError_t dk_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH * p.NC, (p.L + 63) / 64, p.dqk / 64);
   dk_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, (const TIO*)a.dh, a.b, a.li, a.m,
-      a.inv_den, a.da, (const TS*)a.dC, a.dn, (TIO*)a.dk, a.pk, p.T, p.L, p.NC, p.dqk, p.dhv,
+      a.inv_den, a.da, a.dC, a.dn, (TIO*)a.dk, a.pk, p.T, p.L, p.NC, p.dqk, p.dhv,
       p.scale);
   return cudaGetLastError();
 }
@@ -520,7 +519,7 @@ static cudaError_t dv_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH * p.NC, (p.L + 63) / 64, p.dhv / 64);
   dv_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.dh, a.b, a.li, a.m, a.inv_den,
-      (const TS*)a.dC, (TIO*)a.dv, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale);
+      a.dC, (TIO*)a.dv, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale);
   return cudaGetLastError();
 }
 

@@ -22,7 +22,7 @@ template <typename TIO, typename TS, bool EXPV>
 __global__ void __launch_bounds__(256) state_fwd_simt_kernel(
     const TIO* __restrict__ k, const TIO* __restrict__ v, const float* __restrict__ b,
     const float* __restrict__ li, const float* __restrict__ m, TS* __restrict__ C,
-    float* __restrict__ n, int T, int L, int NC, int dqk, int dhv) {
+    float* __restrict__ n, int T, int L, int NC, int dqk, int dhv, size_t plane, bool keep_lo) {
   __shared__ float sK[32][64];
   __shared__ float sV[32][64];
   __shared__ float sw[32];
@@ -38,12 +38,13 @@ __global__ void __launch_bounds__(256) state_fwd_simt_kernel(
   float nacc = 0.f;
 
   for (int c = 0; c < NC; ++c) {
-    TS* Cc = C + ((size_t)bh * NC + c) * dqk * dhv;
+    const size_t cbase = ((size_t)bh * NC + c) * dqk * dhv;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        Cc[(size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] = from_f32<TS>(acc[i][j]);
+        StatePlanes<TS>::store(C, plane, cbase + (size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j,
+                               acc[i][j], keep_lo);
     if (own_n) n[((size_t)bh * NC + c) * dqk + i0 + tid] = nacc;
     if (c == NC - 1) break;  // no state leaves the last chunk
 
@@ -92,10 +93,11 @@ __global__ void __launch_bounds__(256) state_fwd_simt_kernel(
 
 cudaError_t launch_state_fwd_simt(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   dim3 grid(p.BH, p.dqk / 64, p.dhv / 64), block(256);
+  const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
 #define MLSTM_STATE_FWD(TIO, TS, E)                                                              \
   state_fwd_simt_kernel<TIO, TS, E><<<grid, block, 0, s>>>((const TIO*)a.k, (const TIO*)a.v, a.b, \
                                                            a.li, a.m, (TS*)a.C, a.n, p.T, p.L,  \
-                                                           p.NC, p.dqk, p.dhv)
+                                                           p.NC, p.dqk, p.dhv, plane, a.keep_lo)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_STATE_FWD(bf16, bf16, true);
     else MLSTM_STATE_FWD(bf16, bf16, false);
@@ -129,7 +131,8 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ v,
     const float* __restrict__ b, const float* __restrict__ li, const float* __restrict__ m,
     const TS* __restrict__ C, const float* __restrict__ n, TIO* __restrict__ h,
-    float* __restrict__ abar_out, int T, int L, int NC, int dqk, int dhv, float scale) {
+    float* __restrict__ abar_out, int T, int L, int NC, int dqk, int dhv, float scale,
+    size_t plane, bool use_lo) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   OutSmem& S = *reinterpret_cast<OutSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
 
   // inter-chunk term
   if (c > 0) {
-    const TS* Cc = C + ((size_t)bh * NC + c) * dqk * dhv;
+    const size_t cbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int kk0 = 0; kk0 < dqk; kk0 += 32) {
       __syncthreads();
       for (int e = tid; e < 64 * 32; e += 256) {
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
       }
       for (int e = tid; e < 32 * 64; e += 256) {
         const int x = e >> 6, col = e & 63;
-        S.v[x * 64 + col] = to_f32(Cc[(size_t)(kk0 + x) * dhv + j0 + col]);
+        S.v[x * 64 + col] = StatePlanes<TS>::load(C, plane, cbase + (size_t)(kk0 + x) * dhv + j0 + col, use_lo);
       }
       __syncthreads();
 #pragma unroll 4
@@ -296,6 +299,7 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
 cudaError_t launch_output_fwd_simt(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   dim3 grid(p.BH * p.NC, (p.L + 63) / 64, p.dhv / 64), block(256);
   const size_t smem = sizeof(OutSmem);
+  const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
   cudaError_t e = cudaSuccess;
 #define MLSTM_OUT_FWD(TIO, TS, E)                                                                \
   do {                                                                                           \
@@ -304,7 +308,7 @@ cudaError_t launch_output_fwd_simt(const Problem& p, const FwdArgs& a, cudaStrea
     if (e != cudaSuccess) return e;                                                              \
     output_fwd_simt_kernel<TIO, TS, E><<<grid, block, smem, s>>>(                                \
         (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, a.b, a.li, a.m, (const TS*)a.C, a.n, \
-        (TIO*)a.h, a.abar, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale);                               \
+        (TIO*)a.h, a.abar, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale, plane, a.keep_lo);             \
   } while (0)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_OUT_FWD(bf16, bf16, true);

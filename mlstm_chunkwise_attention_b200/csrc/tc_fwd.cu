@@ -1,0 +1,378 @@
+// TFLA intra-chunk output kernel (K-c) on the fifth-generation tensor cores.
+//
+// "Tiled Flash Linear Attention: More Efficient Linear RNN and xLSTM Kernels"
+// (TFLA summary page, Approach; arXiv abstract page, Abstract): the second
+// level of sequence parallelism tiles the intra-chunk matmuls along the
+// sequence, so the chunk size is not bounded by on-chip memory.  One CTA owns
+// a 128-row query tile of one chunk and a slice of up to 128 value columns;
+// it walks the 128-row key/value tiles of the chunk up to the diagonal:
+//
+//   S_j  = Q K_j^T                        (tcgen05, bf16 in smem -> fp32 TMEM)
+//   P_j  = S_j * exp(b_t - b_s + log i_s - m_t) / sqrt(d_qk), causal (registers)
+//   O   += P_j V_j                        (tcgen05, P staged to smem in bf16)
+//   O   += (alpha_t Q / sqrt(d_qk)) C_prev (inter-chunk term, same accumulator)
+//   h_t  = O_t / max(|alpha_t q'_t.n_prev + sum_s P_ts|, exp(-m_t))   (mLSTMexp)
+//
+// Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the
+// MMAs (one thread), warps 2..5 own one query row per thread (TMEM lane),
+// turn S into P, and run the epilogue.  Every mbarrier wait is bounded; on a
+// timeout the kernel sets an error flag and winds down.
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace mlstm {
+
+static __device__ unsigned int g_tc_fwd_error;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int DQK, int DV>
+struct OutTcCfg {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int KB = DQK / 64;  // 64-column blocks of Q and K
+  static constexpr int VB = DV / 64;   // 64-column blocks of the V / C slice
+  static constexpr int Q_BYTES = KB * 16384;
+  static constexpr int K_BYTES = KB * 16384;
+  static constexpr int C_BYTES = VB * DQK * 128;
+  static constexpr int KC_BYTES = K_BYTES > C_BYTES ? K_BYTES : C_BYTES;
+  static constexpr int V_BYTES = VB * 16384;
+  static constexpr int P_BYTES = 2 * 16384;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KC = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_KC + KC_BYTES;
+  static constexpr int OFF_P = OFF_V + V_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;  // 16 mbarriers
+  static constexpr int OFF_TMEM = OFF_BAR + 16 * 8;
+  static constexpr int OFF_NVEC = OFF_TMEM + 16;
+  static constexpr int OFF_COLF = OFF_NVEC + DQK * 4;
+  static constexpr uint32_t TMEM_COLS = 256;  // S in [0, 128), O in [128, 128 + DV)
+  static size_t smem_bytes(int L) { return 1024 + OFF_COLF + (size_t)L * 4; }
+};
+
+enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_COUNT };
+
+}  // namespace
+
+template <int DQK, int DV, bool EXPV>
+__global__ void __launch_bounds__(192, 1) output_fwd_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
+    const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
+    const float* __restrict__ gn, bf16* __restrict__ h, float* __restrict__ abar_out, int T, int L,
+    int NC, int BH, int ntq, int dhv, float scale, float log2_scale) {
+  using Cfg = OutTcCfg<DQK, DV>;
+  constexpr int BM = Cfg::BM, BN = Cfg::BN;
+
+  const int per = BH * NC;
+  const int qt = ntq - 1 - (int)(blockIdx.x / per);  // heaviest query tiles first
+  const int rest = (int)(blockIdx.x % per);
+  const int bh = rest / NC, c = rest % NC;
+  const int c0 = c * L;
+  const int len = min(L, T - c0);
+  const int t0 = qt * BM;
+  if (t0 >= len) return;
+  if (*(volatile unsigned int*)&g_tc_fwd_error != 0u) return;  // an earlier CTA gave up
+  const int nkv = qt + 1;
+  const int dv0 = blockIdx.y * DV;
+  const size_t tok0 = (size_t)bh * T + c0;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + Cfg::OFF_Q;
+  uint8_t* sKC = smem + Cfg::OFF_KC;
+  uint8_t* sV = smem + Cfg::OFF_V;
+  uint8_t* sP = smem + Cfg::OFF_P;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
+  float* nvec = reinterpret_cast<float*>(smem + Cfg::OFF_NVEC);
+  float* colf = reinterpret_cast<float*>(smem + Cfg::OFF_COLF);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_COUNT; ++i) {
+      const uint32_t cnt = (i == B_P || i == B_QS) ? 128u : 1u;
+      tc::mbar_init(&bar[i], cnt);
+    }
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  // column factors (log i_s - b_s) log2(e) of every key row this tile needs
+  if (warp >= 2) {
+    const int gt = threadIdx.x - 64;
+    for (int s = gt; s < nkv * BN; s += 128)
+      colf[s] = s < len ? (gli[tok0 + s] - gb[tok0 + s]) * kLog2e : -INFINITY;
+    if (EXPV && c > 0)
+      for (int i = gt; i < DQK; i += 128) nvec[i] = gn[((size_t)bh * NC + c) * DQK + i];
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 128;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      tc::mbar_arrive_expect_tx(&bar[B_Q], Cfg::Q_BYTES);
+      for (int kb = 0; kb < Cfg::KB; ++kb)
+        tc::tma_load_3d(sQ + kb * 16384, &tm_q, &bar[B_Q], kb * 64, c0 + t0, bh);
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (j > 0) ok = tc::mbar_wait(&bar[B_S], (j - 1) & 1, &g_tc_fwd_error);  // K buffer free
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(&bar[B_K], Cfg::K_BYTES);
+        for (int kb = 0; kb < Cfg::KB; ++kb)
+          tc::tma_load_3d(sKC + kb * 16384, &tm_k, &bar[B_K], kb * 64, c0 + j * BN, bh);
+        if (j > 0) ok = tc::mbar_wait(&bar[B_PV], (j - 1) & 1, &g_tc_fwd_error);  // V buffer free
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(&bar[B_V], Cfg::V_BYTES);
+        for (int vb = 0; vb < Cfg::VB; ++vb)
+          tc::tma_load_3d(sV + vb * 16384, &tm_v, &bar[B_V], dv0 + vb * 64, c0 + j * BN, bh);
+      }
+      if (ok && c > 0) {
+        ok = tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, &g_tc_fwd_error);  // last S done: reuse the K buffer
+        if (ok) {
+          tc::mbar_arrive_expect_tx(&bar[B_C], Cfg::C_BYTES);
+          for (int vb = 0; vb < Cfg::VB; ++vb)
+            tc::tma_load_3d(sKC + vb * DQK * 128, &tm_c, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
+        }
+      }
+      // do not leave while a copy this thread issued may still be landing
+      if (ok) {
+        ok = tc::mbar_wait(&bar[B_V], (nkv - 1) & 1, &g_tc_fwd_error);
+        if (ok && c > 0) ok = tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
+      constexpr uint32_t idO = tc::idesc_bf16(BM, DV, false, true);
+      const uint32_t aQ = tc::smem_u32(sQ), aKC = tc::smem_u32(sKC), aV = tc::smem_u32(sV),
+                     aP = tc::smem_u32(sP);
+      ok = tc::mbar_wait(&bar[B_Q], 0, &g_tc_fwd_error);
+      for (int j = 0; j < nkv && ok; ++j) {
+        ok = tc::mbar_wait(&bar[B_K], j & 1, &g_tc_fwd_error);
+        if (!ok) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < DQK / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          tc::mma_bf16_ss(tS, tc::sdesc_sw128(aQ + off, 16, 1024), tc::sdesc_sw128(aKC + off, 16, 1024),
+                          idS, k > 0);
+        }
+        tc::tc_commit(&bar[B_S]);
+        ok = tc::mbar_wait(&bar[B_P], j & 1, &g_tc_fwd_error) && tc::mbar_wait(&bar[B_V], j & 1, &g_tc_fwd_error);
+        if (!ok) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k) {
+          const uint32_t offp = (k >> 2) * 16384 + (k & 3) * 32;
+          tc::mma_bf16_ss(tO, tc::sdesc_sw128(aP + offp, 16, 1024),
+                          tc::sdesc_sw128(aV + k * 2048, 16384, 1024), idO, (j > 0 || k > 0));
+        }
+        tc::tc_commit(&bar[B_PV]);
+      }
+      if (ok && c > 0) {
+        ok = tc::mbar_wait(&bar[B_QS], 0, &g_tc_fwd_error) && tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
+        if (ok) {
+          tc::tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < DQK / 16; ++k) {
+            const uint32_t offq = (k >> 2) * 16384 + (k & 3) * 32;
+            tc::mma_bf16_ss(tO, tc::sdesc_sw128(aQ + offq, 16, 1024),
+                            tc::sdesc_sw128(aKC + k * 2048, DQK * 128, 1024), idO, 1);
+          }
+        }
+      }
+      tc::tc_commit(&bar[B_O]);
+    }
+  } else {
+    // ------------------------------------------------------------ gate rows + epilogue
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row of the tile
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int tl = t0 + row;
+    const bool valid = tl < len;
+    const size_t tok = tok0 + tl;
+    const float bt = valid ? gb[tok] : 0.f;
+    const float mt = (EXPV && valid) ? gm[tok] : 0.f;
+    const float mprev = EXPV ? (c > 0 ? gm[tok0 - 1] : -INFINITY) : 0.f;
+    const float r2 = valid ? (bt - mt) * kLog2e + log2_scale : -INFINITY;
+    const float qfac = (valid && c > 0) ? expf(bt + mprev - mt) * scale : 0.f;
+    const uint32_t aP = tc::smem_u32(sP), aQ = tc::smem_u32(sQ);
+    float rowsum = 0.f;
+
+    for (int j = 0; j < nkv && ok; ++j) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_S], j & 1, &g_tc_fwd_error));
+      if (ok && j > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_PV], (j - 1) & 1, &g_tc_fwd_error));
+      if (!ok) break;
+      tc::tc_fence_after();
+      const bool diag = (j == qt);
+      const float* cf = colf + j * BN;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        float sv[32];
+        tc::tmem_ld32(tS + lane_base + ch * 32, sv);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int s0 = ch * 32 + i;
+          float p0 = sv[i] * tc::ex2(r2 + cf[s0]);
+          float p1 = sv[i + 1] * tc::ex2(r2 + cf[s0 + 1]);
+          if (diag && s0 > row) p0 = 0.f;
+          if (diag && s0 + 1 > row) p1 = 0.f;
+          if (EXPV) rowsum += p0 + p1;
+          pk[i >> 1] = tc::pack_bf16(p0, p1);
+        }
+        const int kb = ch >> 1;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int lc = (ch & 1) * 4 + q4;
+          const uint32_t addr = aP + kb * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * q4]),
+                       "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3])
+                       : "memory");
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bar[B_P]);
+    }
+
+    // inter-chunk operand: scale the query rows by alpha_t / sqrt(d_qk) in place
+    float inter_norm = 0.f;
+    if (ok && c > 0) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_Q], 0, &g_tc_fwd_error));
+      if (ok) {
+#pragma unroll 1
+        for (int kb = 0; kb < Cfg::KB; ++kb) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int pch = (jj + row) & 7;
+            const uint32_t addr = aQ + kb * 16384 + row * 128 + pch * 16;
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(addr));
+            const int col0 = kb * 64 + ((pch ^ (row & 7)) << 3);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+              const float x0 = __bfloat162float(v2.x) * qfac;
+              const float x1 = __bfloat162float(v2.y) * qfac;
+              if (EXPV) inter_norm += x0 * nvec[col0 + 2 * e] + x1 * nvec[col0 + 2 * e + 1];
+              w[e] = tc::pack_bf16(x0, x1);
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
+                         "r"(w[1]), "r"(w[2]), "r"(w[3])
+                         : "memory");
+          }
+        }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bar[B_QS]);
+      }
+    }
+
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_O], 0, &g_tc_fwd_error));
+    if (ok) {
+      tc::tc_fence_after();
+      float inv = 1.f;
+      if (EXPV) {
+        const float a = inter_norm + rowsum;
+        inv = 1.f / fmaxf(fabsf(a), expf(-mt));
+        if (blockIdx.y == 0 && valid) abar_out[tok] = a;
+      }
+      bf16* hrow = h + tok * dhv + dv0;
+#pragma unroll 1
+      for (int ch = 0; ch < DV / 32; ++ch) {
+        float ov[32];
+        tc::tmem_ld32(tO + lane_base + ch * 32, ov);
+        if (valid) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w;
+            w.x = tc::pack_bf16(ov[8 * q4 + 0] * inv, ov[8 * q4 + 1] * inv);
+            w.y = tc::pack_bf16(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv);
+            w.z = tc::pack_bf16(ov[8 * q4 + 4] * inv, ov[8 * q4 + 5] * inv);
+            w.w = tc::pack_bf16(ov[8 * q4 + 6] * inv, ov[8 * q4 + 7] * inv);
+            *reinterpret_cast<uint4*>(hrow + ch * 32 + q4 * 8) = w;
+          }
+        }
+      }
+    }
+  }
+
+  if (!ok) atomicOr(&g_tc_fwd_error, 1u);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+bool output_fwd_tc_supported(const Problem& p) {
+  return p.bf16() && p.L >= 128 && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
+         (p.dhv % 64 == 0);
+}
+
+template <int DQK, int DV, bool EXPV>
+static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  using Cfg = OutTcCfg<DQK, DV>;
+  CUtensorMap tq, tk, tv, tcm;
+  if (!make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tk, a.k, p.dqk, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tv, a.v, p.dhv, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tcm, a.C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
+    return cudaErrorInvalidValue;
+  const size_t smem = Cfg::smem_bytes(p.L);
+  auto kern = output_fwd_tc_kernel<DQK, DV, EXPV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int ntq = p.L / 128;
+  dim3 grid((unsigned)(p.BH * p.NC * ntq), (unsigned)(p.dhv / DV)), block(192);
+  kern<<<grid, block, smem, s>>>(tq, tk, tv, tcm, a.b, a.li, a.m, a.n, (bf16*)a.h, a.abar, p.T,
+                                 p.L, p.NC, p.BH, ntq, p.dhv, p.scale, log2f(p.scale));
+  return cudaGetLastError();
+}
+
+template <int DQK, bool EXPV>
+static cudaError_t launch_out_tc_dv(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV>(p, a, s);
+  return launch_out_tc<DQK, 128, EXPV>(p, a, s);
+}
+
+cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  const bool e = p.exp_variant();
+  switch (p.dqk) {
+    case 64: return e ? launch_out_tc_dv<64, true>(p, a, s) : launch_out_tc_dv<64, false>(p, a, s);
+    case 128: return e ? launch_out_tc_dv<128, true>(p, a, s) : launch_out_tc_dv<128, false>(p, a, s);
+    case 256: return e ? launch_out_tc_dv<256, true>(p, a, s) : launch_out_tc_dv<256, false>(p, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t fetch_tc_fwd_error(unsigned int* flag) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_fwd_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_tc_fwd_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace mlstm

@@ -12,12 +12,13 @@ from mlstm_chunkwise_attention_b200.synthetic import make_inputs
 TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-4}
 
 
-def relerr(got, ref):
+def relerr(got, ref, floor=1e-30):
+    """max|got - ref| / max(max|ref|, floor)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.all(np.isfinite(got)), "non-finite values in the CUDA result"
-    return float(np.max(np.abs(got - ref)) / max(float(np.max(np.abs(ref))), 1e-30))
+    return float(np.max(np.abs(got - ref)) / max(float(np.max(np.abs(ref))), floor))
 
 
 def np64(t):
@@ -32,14 +33,14 @@ def inputs(B, NH, T, d_qk, d_hv, seed, dtype, ig_mean=0.0, fg_mean=3.0, with_dh=
 def gpu_fwd(cpu, chunk, variant):
     dev = {k: v.cuda() for k, v in cpu.items()}
     h, saved = binding.forward(dev["q"], dev["k"], dev["v"], dev["igate"], dev["fgate"], chunk, variant)
-    torch.cuda.synchronize()
+    binding.check_device()  # synchronises; raises if a kernel reported a timeout
     return dev, h, saved
 
 
 def gpu_bwd(dev, h, saved, chunk, variant):
     g = binding.backward(dev["q"], dev["k"], dev["v"], dev["igate"], dev["fgate"], h, dev["dh"],
                          saved, chunk, variant)
-    torch.cuda.synchronize()
+    binding.check_device()
     return g
 
 

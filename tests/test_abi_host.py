@@ -103,7 +103,8 @@ def test_saved_layout_regions(lib):
             assert lay["gate_b_bytes"] == 4 * tok and lay["gate_li_bytes"] == 4 * tok
             assert lay["gate_m_bytes"] == (4 * tok if variant == B.EXP else 0)
             assert lay["norm_bytes"] == (4 * tok if variant == B.EXP else 0)
-            assert lay["state_c_bytes"] == Bn * NH * NC * dqk * dhv * (2 if dtype == B.BF16 else 4)
+            # bf16: hi and lo bf16 planes; fp32: one fp32 plane
+            assert lay["state_c_bytes"] == Bn * NH * NC * dqk * dhv * 4
             assert lay["state_n_bytes"] == (Bn * NH * NC * dqk * 4 if variant == B.EXP else 0)
             regions = sorted((lay[n], lay[n + "_bytes"]) for n in
                              ("gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n"))

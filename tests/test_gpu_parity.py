@@ -42,7 +42,7 @@ SMALL = [
     ("sig_bf16_igate_bias_m10", 1, 2, 512, 64, 64, 64, SIG, BF, -10.0, 4.0),
     ("exp_bf16_igate_bias_m10", 1, 2, 512, 64, 64, 64, EXP, BF, -10.0, 3.0),
     ("exp_bf16_one_partial_chunk", 1, 1, 37, 64, 64, 64, EXP, BF, 0.0, 3.0),
-    ("exp_fp32_t1", 1, 1, 1, 64, 64, 64, EXP, F32, 0.0, 3.0),
+    ("exp_fp32_t1", 1, 1, 1, 64, 64, 64, EXP, F32, -4.0, 3.0),
     ("sig_bf16_chunk4096_ragged", 1, 1, 4500, 64, 64, 4096, SIG, BF, 0.0, 3.0),
     ("exp_bf16_chunk1024", 1, 1, 2048, 128, 128, 1024, EXP, BF, 0.0, 3.0),
     ("exp_fp32_dqk256", 1, 1, 384, 256, 64, 128, EXP, F32, 1.0, 2.0),
@@ -62,8 +62,12 @@ def test_small_forward_backward_all_heads(case):
             ref = oracle_fwd_head(x, L, var)
             assert relerr(np64(h[b, hh]), ref["h"]) <= tol, f"h ({b},{hh})"
             ref_g = oracle_bwd_head(x, var)
+            # a gradient that is exactly zero in the mathematics (the first forget
+            # gate scales the zero initial state) is compared on the scale of the
+            # other gradients of the same head
+            floor = 1e-3 * max(np.max(np.abs(v)) for v in ref_g.values())
             for key, val in ref_g.items():
-                err = relerr(np64(g[key][b, hh]), val)
+                err = relerr(np64(g[key][b, hh]), val, floor=floor)
                 assert err <= tol, f"{key} ({b},{hh}): {err:.3e}"
 
 
@@ -84,6 +88,22 @@ def test_saved_gate_prep_and_states_match_oracle(var):
             np.testing.assert_allclose(np64(sv["m"][hh]), ref["m_row"], rtol=1e-5, atol=1e-4)
             assert relerr(np64(sv["abar"][hh]), ref["abar"]) < 1e-5
             assert relerr(np64(sv["n"][hh]), ref["n_enter"]) < 1e-5
+
+
+def test_saturated_normaliser_has_zero_gradient():
+    """T = 1 with |i q'.k| > 1: h = sign(a) v, so dq, dk and d igate are exactly 0."""
+    cpu = inputs(1, 1, 1, 64, 64, seed=3, dtype=F32)
+    q, k = cpu["q"][0, 0, 0], cpu["k"][0, 0, 0]
+    s = float(q @ k) / 8.0
+    cpu["igate"] = torch.full((1, 1, 1), float(np.log(4.0 / max(abs(s), 1e-3))), dtype=F32)
+    dev, h, saved = gpu_fwd(cpu, 64, EXP)
+    g = gpu_bwd(dev, h, saved, 64, EXP)
+    want_h = np.sign(s) * np64(cpu["v"][0, 0])
+    assert relerr(np64(h[0, 0]), want_h) <= 1e-4
+    scale = float(np.abs(np64(cpu["dh"])).max() * np.abs(np64(cpu["v"])).max())
+    for key in ("dq", "dk", "digate_pre"):
+        assert np.abs(np64(g[key])).max() <= 1e-5 * scale, key
+    assert relerr(np64(g["dv"][0, 0]), np.sign(s) * np64(cpu["dh"][0, 0])) <= 1e-4
 
 
 def _preact(v, T):
@@ -135,7 +155,7 @@ def test_chunk_size_invariance_on_gpu():
     cpu = inputs(1, 2, 1024, 64, 64, seed=8, dtype=F32, with_dh=False)
     outs = [np64(gpu_fwd(cpu, L, EXP)[1]) for L in (64, 128, 256, 512)]
     for o in outs[1:]:
-        assert relerr(o, outs[0]) <= 1e-5
+        assert relerr(o, outs[0]) <= 1e-4
 
 
 def test_repeat_calls_are_deterministic_forward():
