@@ -393,6 +393,88 @@ def recurrent_backward(q, k, v, log_i, log_f, variant, dh):
             "dlog_i": di * i, "dlog_f": df * f, "h": h}
 
 
+def chunkwise_backward(q, k, v, log_i, log_f, variant, L, dh):
+    """Gradients of sum(dh * h) in the chunkwise order, fp64 (no [T, T] matrices).
+
+    Uses the forward's chunk quantities (chunkwise_forward) with the max state
+    held constant (reading 5):
+
+    a4. reverse over chunks: dC_c, the gradient of the state leaving chunk c,
+        dC_{c-1} = beta_c dC_c + sum_{t in c} alpha_t q'_t dnum_t^T and
+        dn_{c-1} = beta_c dn_c + sum_{t in c} alpha_t da_t q'_t;
+    a5. per chunk, with dA_ts = dnum_t . v_s + da_t and D the in-chunk decay:
+        dq'_t = alpha_t (C_{c-1} dnum_t + da_t n_{c-1}) + sum_s dA_ts D_ts k_s,
+        dk_s  = w_s (dC_c v_s + dn_c) + sum_t dA_ts D_ts q'_t,
+        dv_s  = w_s dC_c^T k_s + sum_t D_ts (q'_t . k_s) dnum_t;
+    a6. d log i_s = k_s . dk_s and d log f_r = sum_{t>=r} (q'_t.dq'_t - k_t.dk_t).
+    """
+    q, k, v, log_i, log_f, dh = _as64(q, k, v, log_i, log_f, dh)
+    T, d_qk = q.shape
+    d_hv = v.shape[1]
+    qs = q / np.sqrt(d_qk)
+    f = chunkwise_forward(q, k, v, log_i, log_f, variant, L)
+    exp_variant = variant == EXP
+    NC = -(-T // L)
+    bounds = [(c * L, min((c + 1) * L, T)) for c in range(NC)]
+    b, m_row, g = f["b"], f["m_row"], f["g"]
+    m_state, m_enter = f["m_state"], f["m_enter"]
+    den = f["den"]
+    dnum = dh / den[:, None]
+    if exp_variant:
+        active = np.abs(f["abar"]) > np.exp(-m_row)
+        da = np.where(active, -np.sum(dh * f["h"], axis=1) * np.sign(f["abar"]) / den, 0.0)
+    else:
+        da = np.zeros(T)
+
+    def alpha_of(c, lo, hi):
+        if exp_variant:
+            return np.exp(b[lo:hi] + m_enter[c] - m_row[lo:hi])
+        return np.exp(b[lo:hi])
+
+    # a4: gradient of the state leaving each chunk
+    dC = np.zeros((NC, d_qk, d_hv))
+    dn = np.zeros((NC, d_qk))
+    G = np.zeros((d_qk, d_hv))
+    gn = np.zeros(d_qk)
+    for c in range(NC - 1, -1, -1):
+        dC[c] = G
+        dn[c] = gn
+        lo, hi = bounds[c]
+        beta = np.exp(g[c] + m_enter[c] - m_state[c]) if exp_variant else np.exp(g[c])
+        alpha = alpha_of(c, lo, hi)
+        G = beta * G + (alpha[:, None] * qs[lo:hi]).T @ dnum[lo:hi]
+        gn = beta * gn + (alpha * da[lo:hi]) @ qs[lo:hi]
+
+    # a5: per-chunk gradients
+    dqs = np.zeros((T, d_qk))
+    dk = np.zeros((T, d_qk))
+    dv = np.zeros((T, d_hv))
+    for c, (lo, hi) in enumerate(bounds):
+        sl = slice(lo, hi)
+        n_rows = hi - lo
+        tril = np.tril(np.ones((n_rows, n_rows), dtype=bool))
+        bt, mt = b[sl], m_row[sl]
+        logD = bt[:, None] - bt[None, :] + log_i[sl][None, :] - mt[:, None]
+        D = np.where(tril, np.exp(np.where(tril, logD, 0.0)), 0.0)
+        alpha = alpha_of(c, lo, hi)
+        mk = m_state[c] if exp_variant else 0.0
+        w = np.exp(g[c] - bt + log_i[sl] - mk)
+        dA = dnum[sl] @ v[sl].T + da[sl][:, None]
+        dS = dA * D
+        A = (qs[sl] @ k[sl].T) * D
+        dqs[sl] = dS @ k[sl] + alpha[:, None] * (dnum[sl] @ f["C_enter"][c].T
+                                                  + da[sl][:, None] * f["n_enter"][c][None, :])
+        dk[sl] = dS.T @ qs[sl] + w[:, None] * (v[sl] @ dC[c].T + dn[c][None, :])
+        dv[sl] = A.T @ dnum[sl] + w[:, None] * (k[sl] @ dC[c])
+
+    # a6: gate gradients from the per-token dot products
+    pq = np.einsum("td,td->t", qs, dqs)
+    pk = np.einsum("td,td->t", k, dk)
+    dlog_f = np.cumsum((pq - pk)[::-1])[::-1]
+    return {"dq": dqs / np.sqrt(d_qk), "dk": dk, "dv": dv, "dlog_i": pk, "dlog_f": dlog_f,
+            "h": f["h"], "den": den, "dC_leave": dC}
+
+
 # ---------------------------------------------------------------------------
 # single rows / columns, for sequences too long for the [T, T] matrices
 # ---------------------------------------------------------------------------

@@ -245,6 +245,17 @@ def check_bptt(M, variant, seed=30, ig_mean=0.0):
         assert rel(p[name], r[name]) < 1e-11, name
 
 
+def check_chunkwise_backward(M, variant, T=50, L=16, seed=33):
+    """The chunkwise backward agrees with BPTT, including a ragged last chunk."""
+    q, k, v, ig, fg = rnd(seed, T, 6, 5, -1.0, 2.0)
+    dh = np.random.default_rng(seed + 1).standard_normal((T, 5))
+    li, lf = M.gate_logs(ig, fg, variant)
+    r = M.recurrent_backward(q, k, v, li, lf, variant, dh)
+    cb = M.chunkwise_backward(q, k, v, li, lf, variant, L, dh)
+    for name in ("dq", "dk", "dv", "dlog_i", "dlog_f"):
+        assert rel(cb[name], r[name]) < 1e-10, name
+
+
 def check_identities(M, variant):
     """d log i_s = k_s.dk_s and d log f_r = sum_{t>=r} (q'_t.dq'_t - k_t.dk_t)."""
     T = 32
@@ -286,6 +297,7 @@ ALL_CHECKS = [
     lambda M: check_chunk_states(M, SIG), lambda M: check_chunk_states(M, EXP),
     lambda M: check_bptt(M, SIG), lambda M: check_bptt(M, EXP),
     lambda M: check_identities(M, SIG), lambda M: check_identities(M, EXP),
+    lambda M: check_chunkwise_backward(M, SIG), lambda M: check_chunkwise_backward(M, EXP),
     lambda M: check_rows(M, SIG), lambda M: check_rows(M, EXP),
     lambda M: check_finite_differences(M, SIG), lambda M: check_finite_differences(M, EXP),
 ]
@@ -361,6 +373,12 @@ def test_parallel_backward_equals_bptt(variant, seed, ig_mean):
 
 
 @pytest.mark.parametrize("variant", [SIG, EXP])
+@pytest.mark.parametrize("T,L,seed", [(50, 16, 33), (48, 8, 34), (7, 4, 35), (40, 40, 36), (33, 1, 37)])
+def test_chunkwise_backward_equals_bptt(variant, T, L, seed):
+    check_chunkwise_backward(oracle, variant, T, L, seed)
+
+
+@pytest.mark.parametrize("variant", [SIG, EXP])
 def test_gate_gradient_identities(variant):
     check_identities(oracle, variant)
 
@@ -381,7 +399,8 @@ MUTATIONS = [
      "den[t] = abs(a[t])\n            h[t] = num / den[t]"),
     ("input gate dropped", "C = f_t * C + i_t * np.outer(k[t], v[t])", "C = f_t * C + np.outer(k[t], v[t])"),
     ("decay row off by one", "row[:t] = np.cumsum(log_f[t:0:-1])[::-1]", "row[:t] = np.cumsum(log_f[t - 1::-1])[::-1]"),
-    ("state decay term dropped", "beta = np.exp(g[c] + m_enter[c] - m_state[c])", "beta = np.exp(m_enter[c] - m_state[c])"),
+    ("state decay term dropped", "beta = np.exp(g[c] + m_enter[c] - m_state[c])\n            w =",
+     "beta = np.exp(m_enter[c] - m_state[c])\n            w ="),
     ("state weight sign", "w = np.exp(g[c] - b[sl] + log_i[sl] - m_state[c])", "w = np.exp(g[c] + b[sl] + log_i[sl] - m_state[c])"),
     ("max state missing b", "m_row[sl] = b[sl] + np.maximum(m_prev, u)", "m_row[sl] = np.maximum(m_prev, u)"),
     ("inter-chunk factor missing b", "alpha = np.exp(bt + m_enter[c] - mt) if exp_variant", "alpha = np.exp(m_enter[c] - mt) if exp_variant"),
@@ -392,6 +411,12 @@ MUTATIONS = [
     ("forget chain rule sign", "dfgate = np.asarray(dlog_f) * sigmoid(-np.asarray(fgate_pre", "dfgate = np.asarray(dlog_f) * sigmoid(np.asarray(fgate_pre"),
     ("bptt forget grad uses C_t", "df[t] = np.sum(dC * Cs[t]) + dn @ ns[t]", "df[t] = np.sum(dC * Cs[t + 1]) + dn @ ns[t]"),
     ("column dA misses da", "dA_col = dnum[r:] @ v[r] + da[r:]", "dA_col = dnum[r:] @ v[r]"),
+    ("state gradient misses the decay", "G = beta * G + (alpha[:, None] * qs[lo:hi]).T @ dnum[lo:hi]",
+     "G = G + (alpha[:, None] * qs[lo:hi]).T @ dnum[lo:hi]"),
+    ("dk misses the state gradient", "dk[sl] = dS.T @ qs[sl] + w[:, None] * (v[sl] @ dC[c].T + dn[c][None, :])",
+     "dk[sl] = dS.T @ qs[sl] + w[:, None] * dn[c][None, :]"),
+    ("dv uses the state entering the chunk", "dv[sl] = A.T @ dnum[sl] + w[:, None] * (k[sl] @ dC[c])",
+     "dv[sl] = A.T @ dnum[sl] + w[:, None] * (k[sl] @ dC[c - 1])"),
     ("chunk mask misses diagonal", "tril = np.tril(np.ones((hi - lo, hi - lo), dtype=bool))",
      "tril = np.tril(np.ones((hi - lo, hi - lo), dtype=bool), -1)"),
     ("chunk decay taken at the wrong row", "g = np.array([b[hi - 1] for (_, hi) in bounds])",
