@@ -255,7 +255,8 @@ def workload_config(spec, n):
             "d_hv": spec["d_hv"], "chunk": spec["chunk"], "pass": "fwd+bwd",
             "global_batch": spec["B"] * n, "seq_len": spec["T"],
             "parallelism": f"replicas{n}" if n > 1 else "single",
-            "l2": "no flush: q, k, v, dh are 268 MB each, larger than the 126 MB L2"}
+            "l2": "no flush: q, k, v, dh are %d MB each, larger than the 126 MB L2"
+                  % (spec["B"] * spec["NH"] * spec["T"] * spec["d_qk"] * 2 >> 20)}
 
 
 # ---------------------------------------------------------------------------
@@ -269,12 +270,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B (smaller captures for ncu; the default is the workload's B)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     from mlstm_chunkwise_attention_b200.synthetic import WORKLOADS
     spec = dict(WORKLOADS[WORKLOAD])
+    if args.batch is not None:
+        spec["B"] = args.batch
 
     if args.impl == "reference":
         return run_reference(args, spec)
