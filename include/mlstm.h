@@ -131,6 +131,27 @@ int mlstm_bwd(const void* q, const void* k, const void* v,
               int B, int NH, int T, int d_qk, int d_hv, int chunk,
               int variant, int dtype, void* stream);
 
+/* Allocation-free forward, for callers that cannot call cudaMalloc when they
+ * run the op (a framework that owns every device allocation, a plugin behind
+ * a custom allocator, a launch path where allocating would synchronise).  The
+ * pages have no counterpart: this is a deployment convenience.  It computes
+ * exactly what mlstm_fwd computes with saved == NULL, but its scratch (gate
+ * sums, max states, chunk states) lives in a 32 MiB array compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  The caller passes the inputs and the output h, device pointers as
+ * for mlstm_fwd.  Problems whose scratch (mlstm_fwd_workspace_size) exceeds
+ * 32 MiB return MLSTM_ERR_WORKSPACE before any launch; no saved state is kept,
+ * so there is no backward from this entry point.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  It calls no
+ * cudaMalloc or cudaFree.  All calls share the one array, so calls whose
+ * kernels overlap on the GPU (different streams, or different host threads)
+ * race on it: serialise them. */
+int mlstm_fwd_noalloc(const void* q, const void* k, const void* v,
+                      const void* igate_pre, const void* fgate_pre, void* h,
+                      int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                      int variant, int dtype, void* stream);
+
 /* Synchronise `stream` and report what the kernels enqueued so far found:
  * MLSTM_ERR_TIMEOUT if one of them gave up a bounded wait (its outputs are
  * then invalid; the flag is cleared by this call), MLSTM_ERR_CUDA on a CUDA

@@ -56,6 +56,7 @@ EXPORTS = {
     "mlstm_launch_name": (ctypes.c_char_p, [ctypes.c_int, ctypes.c_int] + _SIZES),
     "mlstm_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "mlstm_device_status": (ctypes.c_int, [_P]),
+    "mlstm_fwd_noalloc": (ctypes.c_int, [_P] * 6 + _SIZES + [_P]),
 }
 
 
@@ -113,6 +114,13 @@ def mlstm_fwd(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_byte
               B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream):
     return load().mlstm_fwd(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_bytes,
                             B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream)
+
+
+def mlstm_fwd_noalloc(q, k, v, igate_pre, fgate_pre, h, B, NH, T, d_qk, d_hv, chunk, variant,
+                      dtype, stream):
+    """Forward whose scratch is a fixed array inside the library (no allocation)."""
+    return load().mlstm_fwd_noalloc(q, k, v, igate_pre, fgate_pre, h, B, NH, T, d_qk, d_hv, chunk,
+                                    variant, dtype, stream)
 
 
 def mlstm_bwd(q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv, digate_pre, dfgate_pre,
