@@ -35,7 +35,9 @@ KERNEL_SOURCES = {
     "gate_prep": "gates.cu", "bwd_token_prep": "gates.cu", "gate_grad": "gates.cu",
     "state_fwd_simt": "simt_fwd.cu", "output_fwd_simt": "simt_fwd.cu",
     "state_bwd_simt": "simt_bwd.cu", "dq_simt": "simt_bwd.cu", "dk_simt": "simt_bwd.cu",
-    "dv_simt": "simt_bwd.cu",
+    "dv_simt": "simt_bwd.cu", "output_fwd_tc": "tc_fwd.cu", "dq_tc": "tc_bwd.cu",
+    "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
+    "state_bwd_tc": "tc_state.cu",
 }
 
 
@@ -54,29 +56,40 @@ def flops_bwd(T, dqk, dhv, L):
 
 
 def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
-    """(flops, bytes) per head for every kernel of the path, algorithmic counts."""
+    """(flops, bytes) per head for every kernel of the path, algorithmic counts.
+
+    Bytes count each tensor once per kernel that must touch it: inputs read,
+    outputs written, chunk states (two bf16 planes = 4 B per element on the
+    bf16 path, the tensor-core forward reads only the hi plane) and the fp32
+    per-token gate arrays.
+    """
     NC = -(-T // L)
-    sb = io_bytes  # states are stored in the I/O dtype
     g = 3 if exp_variant else 2  # per-token gate floats (b, log i [, m])
-    st = NC * dqk * dhv * sb
+    st_full = NC * dqk * dhv * 4            # hi + lo planes (or one fp32 plane)
+    st_hi = NC * dqk * dhv * io_bytes       # hi plane only
     stn = NC * dqk * 4 if exp_variant else 0
     tdd = 2 * T * dqk * dhv
     tok_f = T * 4
-    return {
+    c = {
         "gate_prep": (0, T * 2 * io_bytes + g * tok_f),
-        "state_fwd_simt": (tdd, T * (dqk + dhv) * io_bytes + g * tok_f + st + stn),
-        "output_fwd_simt": (tdd + T * L * (dqk + dhv),
-                            T * (2 * dqk + 2 * dhv) * io_bytes + g * tok_f + st + stn
-                            + (tok_f if exp_variant else 0)),
+        "state_fwd": (tdd, T * (dqk + dhv) * io_bytes + g * tok_f + st_full + stn),
+        "output_fwd": (tdd + T * L * (dqk + dhv),
+                       T * (2 * dqk + 2 * dhv) * io_bytes + g * tok_f + st_hi + stn
+                       + (tok_f if exp_variant else 0)),
         "bwd_token_prep": (0, (T * 2 * dhv * io_bytes + 2 * tok_f + 4 * tok_f) if exp_variant
                            else 3 * tok_f),
-        "state_bwd_simt": (tdd, T * (dqk + dhv) * io_bytes + 4 * tok_f + st + stn),
-        "dq_simt": (tdd + T * L * (dhv + dqk),
-                    T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st + stn),
-        "dk_simt": (tdd + T * L * dqk, T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st + stn),
-        "dv_simt": (tdd + T * L * (dqk + dhv), T * (2 * dqk + 2 * dhv) * io_bytes + 4 * tok_f + st),
+        "state_bwd": (tdd, T * (dqk + dhv) * io_bytes + 4 * tok_f + st_full + stn),
+        "dq": (tdd + T * L * (dhv + dqk), T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st_full + stn),
+        "dk": (tdd + T * L * dqk, T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st_full + stn),
+        "dv": (tdd + T * L * (dqk + dhv), T * (2 * dqk + 2 * dhv) * io_bytes + 4 * tok_f + st_full),
         "gate_grad": (0, T * 4 * io_bytes + 2 * tok_f),
     }
+    out = {}
+    for role, v in c.items():
+        out[role] = v
+        for impl in ("_simt", "_tc"):
+            out[role + impl] = v
+    return out
 
 
 def kernel_bound(name):
