@@ -36,7 +36,7 @@ struct BwdArgs {
   float* da;       // [BH, T] gradient of the stabilised normaliser (EXP)
   float* pq;       // [BH, T] q_t . dq_t
   float* pk;       // [BH, T] k_t . dk_t
-  float* dC;       // [BH, NC, dqk, dhv] gradient of the state leaving each chunk (fp32)
+  void* dC;        // [BH, NC, dqk, dhv] gradient of the state leaving each chunk (planes, see StatePlanes)
   float* dn;       // [BH, NC, dqk]
 };
 
@@ -59,5 +59,10 @@ bool make_tmap_3d_bf16(void* map, const void* base, uint64_t inner, uint64_t mid
 bool output_fwd_tc_supported(const Problem& p);
 cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_fwd_error(unsigned int* flag);
+bool intra_bwd_tc_supported(const Problem& p);
+cudaError_t launch_dq_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dk_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dv_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t fetch_tc_bwd_error(unsigned int* flag);
 
 }  // namespace mlstm

@@ -117,9 +117,15 @@ int bwd_plan(const Problem& p, BwdStep* st) {
   int n = 0;
   st[n++] = {"bwd_token_prep", mlstm::launch_bwd_token_prep};
   st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
-  st[n++] = {"dq_simt", mlstm::launch_dq_simt};
-  st[n++] = {"dk_simt", mlstm::launch_dk_simt};
-  st[n++] = {"dv_simt", mlstm::launch_dv_simt};
+  if (mlstm::intra_bwd_tc_supported(p)) {
+    st[n++] = {"dq_tc", mlstm::launch_dq_tc};
+    st[n++] = {"dk_tc", mlstm::launch_dk_tc};
+    st[n++] = {"dv_tc", mlstm::launch_dv_tc};
+  } else {
+    st[n++] = {"dq_simt", mlstm::launch_dq_simt};
+    st[n++] = {"dk_simt", mlstm::launch_dk_simt};
+    st[n++] = {"dv_simt", mlstm::launch_dv_simt};
+  }
   st[n++] = {"gate_grad", mlstm::launch_gate_grad};
   return n;
 }
@@ -285,7 +291,7 @@ int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre
   a.da = (float*)(ws + W.da);
   a.pq = (float*)(ws + W.pq);
   a.pk = (float*)(ws + W.pk);
-  a.dC = (float*)(ws + W.dC);
+  a.dC = ws + W.dC;
   a.dn = p.exp_variant() ? (float*)(ws + W.dn) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
@@ -313,9 +319,12 @@ const char* mlstm_last_error(void) { return g_last_error; }
 int mlstm_device_status(void* stream) {
   int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
   if (st != MLSTM_OK) return st;
-  unsigned int flag = 0;
+  unsigned int flag = 0, flag_bwd = 0;
   st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
   if (st != MLSTM_OK) return st;
+  st = cuda_status(mlstm::fetch_tc_bwd_error(&flag_bwd), "device error flag");
+  if (st != MLSTM_OK) return st;
+  flag |= flag_bwd;
   if (flag) {
     snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
     return MLSTM_ERR_TIMEOUT;

@@ -28,8 +28,8 @@ template <typename TIO, typename TS, bool EXPV>
 __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ dh, const float* __restrict__ b,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
-    float* __restrict__ dC, float* __restrict__ dn, int T, int L, int NC, int dqk, int dhv,
-    float scale) {
+    TS* __restrict__ dC, float* __restrict__ dn, int T, int L, int NC, int dqk, int dhv,
+    float scale, size_t plane) {
   __shared__ float sQ[32][64];
   __shared__ float sD[32][64];
   __shared__ float fq[32], fn[32];
@@ -45,11 +45,13 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
   float nacc = 0.f;
 
   for (int c = NC - 1; c >= 0; --c) {
-    float* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
+    const size_t gbase = ((size_t)bh * NC + c) * dqk * dhv;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) Gc[(size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] = acc[i][j];
+      for (int j = 0; j < 4; ++j)
+        StatePlanes<TS>::store(dC, plane, gbase + (size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j,
+                               acc[i][j], true);
     if (own_n) dn[((size_t)bh * NC + c) * dqk + i0 + tid] = nacc;
     if (c == 0) break;
 
@@ -108,8 +110,8 @@ cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream
   dim3 grid(p.BH, p.dqk / 64, p.dhv / 64), block(256);
 #define MLSTM_STATE_BWD(TIO, TS, E)                                                             \
   state_bwd_simt_kernel<TIO, TS, E><<<grid, block, 0, s>>>(                                     \
-      (const TIO*)a.q, (const TIO*)a.dh, a.b, a.m, a.inv_den, a.da, a.dC, a.dn, p.T, p.L,       \
-      p.NC, p.dqk, p.dhv, p.scale)
+      (const TIO*)a.q, (const TIO*)a.dh, a.b, a.m, a.inv_den, a.da, (TS*)a.dC, a.dn, p.T, p.L,  \
+      p.NC, p.dqk, p.dhv, p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_STATE_BWD(bf16, bf16, true);
     else MLSTM_STATE_BWD(bf16, bf16, false);
@@ -303,8 +305,8 @@ __global__ void __launch_bounds__(256) dk_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ v,
     const TIO* __restrict__ dh, const float* __restrict__ b, const float* __restrict__ li,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
-    const float* __restrict__ dC, const float* __restrict__ dn, TIO* __restrict__ dk,
-    float* __restrict__ pk, int T, int L, int NC, int dqk, int dhv, float scale) {
+    const TS* __restrict__ dC, const float* __restrict__ dn, TIO* __restrict__ dk,
+    float* __restrict__ pk, int T, int L, int NC, int dqk, int dhv, float scale, size_t plane) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -321,13 +323,13 @@ __global__ void __launch_bounds__(256) dk_simt_kernel(
   zero44(acc);
 
   if (c < NC - 1) {  // w_s (dC_c v_s + dn_c)
-    const float* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
+    const size_t gbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dhv; x0 += 32) {
       __syncthreads();
       for (int e = tid; e < 64 * 32; e += 256) {
         const int r = e >> 5, x = e & 31, s = s0 + r;
         S.a[x * kP + r] = s < len ? to_f32(v[(tok0 + s) * dhv + x0 + x]) : 0.f;
-        S.bt[x * kP + r] = Gc[(size_t)(i0 + r) * dhv + x0 + x];
+        S.bt[x * kP + r] = StatePlanes<TS>::load(dC, plane, gbase + (size_t)(i0 + r) * dhv + x0 + x);
       }
       __syncthreads();
       mac44(acc, S.a, kP, S.bt, kP, 32, ty, tx);
@@ -400,8 +402,8 @@ template <typename TIO, typename TS, bool EXPV>
 __global__ void __launch_bounds__(256) dv_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ dh,
     const float* __restrict__ b, const float* __restrict__ li, const float* __restrict__ m,
-    const float* __restrict__ inv_den, const float* __restrict__ dC, TIO* __restrict__ dv, int T,
-    int L, int NC, int dqk, int dhv, float scale) {
+    const float* __restrict__ inv_den, const TS* __restrict__ dC, TIO* __restrict__ dv, int T,
+    int L, int NC, int dqk, int dhv, float scale, size_t plane) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(256) dv_simt_kernel(
   zero44(acc);
 
   if (c < NC - 1) {  // w_s dC_c^T k_s
-    const float* Gc = dC + ((size_t)bh * NC + c) * dqk * dhv;
+    const size_t gbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dqk; x0 += 32) {
       __syncthreads();
       for (int e = tid; e < 64 * 32; e += 256) {
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(256) dv_simt_kernel(
       }
       for (int e = tid; e < 32 * 64; e += 256) {
         const int x = e >> 6, col = e & 63;
-        S.w[x * 64 + col] = Gc[(size_t)(x0 + x) * dhv + j0 + col];
+        S.w[x * 64 + col] = StatePlanes<TS>::load(dC, plane, gbase + (size_t)(x0 + x) * dhv + j0 + col);
       }
       __syncthreads();
       mac44(acc, S.a, kP, S.w, 64, 32, ty, tx);
@@ -505,8 +507,8 @@ static cudaError_t dk_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH * p.NC, (p.L + 63) / 64, p.dqk / 64);
   dk_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, (const TIO*)a.dh, a.b, a.li, a.m,
-      a.inv_den, a.da, a.dC, a.dn, (TIO*)a.dk, a.pk, p.T, p.L, p.NC, p.dqk, p.dhv,
-      p.scale);
+      a.inv_den, a.da, (const TS*)a.dC, a.dn, (TIO*)a.dk, a.pk, p.T, p.L, p.NC, p.dqk, p.dhv,
+      p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv);
   return cudaGetLastError();
 }
 
@@ -519,7 +521,8 @@ static cudaError_t dv_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH * p.NC, (p.L + 63) / 64, p.dhv / 64);
   dv_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.dh, a.b, a.li, a.m, a.inv_den,
-      a.dC, (TIO*)a.dv, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale);
+      (const TS*)a.dC, (TIO*)a.dv, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale,
+      (size_t)p.BH * p.NC * p.dqk * p.dhv);
   return cudaGetLastError();
 }
 

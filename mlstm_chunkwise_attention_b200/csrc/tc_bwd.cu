@@ -1,0 +1,524 @@
+// Intra-chunk backward kernels (K-d2) on the fifth-generation tensor cores:
+// dq, dk and dv, each a "score, gated transform, accumulate" walk over the
+// 128-token tiles of one chunk, plus the inter-chunk term through the chunk
+// states.  Timed as the training kernels of "Tiled Flash Linear Attention:
+// More Efficient Linear RNN and xLSTM Kernels" (TFLA summary page, Key
+// results); the second-level tiling along the sequence inside a chunk is the
+// one the same page (Approach) describes for the forward pass.
+//
+// With m held constant, dnum_t = dh_t / den_t, da_t the normaliser gradient,
+// D_ts = exp(b_t - b_s + log i_s - m_t) for s <= t inside the chunk:
+//   dq'_t = alpha_t (C_{c-1} dnum_t + da_t n_{c-1}) + sum_s (dh_t.v_s/den_t + da_t) D_ts k_s
+//   dk_s  = w_s (dC_c v_s + dn_c)                  + sum_t (dh_t.v_s/den_t + da_t) D_ts q'_t
+//   dv_s  = w_s dC_c^T k_s                         + sum_t D_ts (q'_t.k_s) dh_t / den_t
+// One CTA owns a 128-token row tile R (query rows for dq, key rows for dk and
+// dv) and a slice of up to 128 output columns:
+//   X  = A_R B_j^T      score tile (dq: dH V^T, dk: V dH^T, dv: K Q^T)
+//   Y  = transform(X)   gates, mask and normaliser terms, bf16 to smem
+//   Acc += Y E_j        (dq: E = K, dk: E = Q, dv: E = dH)
+// The inter-chunk term Acc = A_R G (G the chunk state or its gradient, split
+// into hi and lo bf16 planes so the product keeps about 16 mantissa bits) is
+// computed first and rescaled per row in TMEM.  Warp roles: warp 0 TMA,
+// warp 1 MMA (one thread), warps 2..5 one tile row per thread.  Every wait is
+// bounded; on a timeout the kernel raises an error flag and winds down.
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace mlstm {
+
+static __device__ unsigned int g_tc_bwd_error;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+enum { KDQ = 0, KDK = 1, KDV = 2 };
+
+template <int D1, int D2S, bool G_MN>
+struct BwdTcCfg {
+  static constexpr int STAGES = 2;
+  static constexpr int SLOT = 16384;  // one 128 x 64 bf16 block
+  static constexpr int STAGE_BYTES = 3 * SLOT;
+  static constexpr int NKB = D1 / 64;  // K-blocks of the score GEMM and the inter GEMM
+  static constexpr int EB = D2S / 64;  // 64-column blocks of E and of the output slice
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_E = STAGES * STAGE_BYTES;
+  static constexpr int OFF_Y = OFF_E + EB * SLOT;
+  static constexpr int OFF_BAR = OFF_Y + 2 * SLOT;
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_RV = OFF_TMEM + 16;
+  static constexpr int OFF_PF = OFF_RV + D2S * 4;  // partner factors, 2 x L floats
+  static constexpr uint32_t TMEM_COLS = 512;       // X buffers [0,128), [128,256); Acc [256, 256+D2S)
+  static constexpr uint32_t G_BYTES = G_MN ? (uint32_t)EB * 8192u : (uint32_t)D2S * 128u;
+  static size_t smem_bytes(int L) { return 1024 + OFF_PF + (size_t)2 * L * 4; }
+};
+
+enum {
+  BB_FULL0 = 0, BB_FULL1, BB_EMPTY0, BB_EMPTY1, BB_EFULL, BB_X0, BB_X1, BB_Y, BB_YE, BB_INTER,
+  BB_ACC, BB_DONE, BB_COUNT
+};
+
+}  // namespace
+
+struct BwdTcParams {
+  const float *b, *li, *m, *inv_den, *da;
+  const float* rowvec;  // dq: n_{c-1} [BH, NC, dqk]; dk: dn_c [BH, NC, dqk]; dv: unused
+  const bf16* dot_src;  // dq: q; dk: k (the per-token dot product with the result)
+  bf16* out;            // dq, dk or dv [BH, T, d_out]
+  float* pdot;          // dq: pq; dk: pk (atomically accumulated)
+  int T, L, NC, BH, ntq, d_out, dqk;
+  float scale, log2_scale;
+};
+
+template <int KIND, int D1, int D2S, bool G_MN, bool EXPV>
+__global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmGhi,
+    const __grid_constant__ CUtensorMap tmGlo, const BwdTcParams P) {
+  using Cfg = BwdTcCfg<D1, D2S, G_MN>;
+  constexpr bool R_IS_QUERY = (KIND == KDQ);
+
+  const int per = P.BH * P.NC;
+  // heaviest row tiles first: dq tiles near the chunk end, dk/dv tiles near its start
+  const int order = (int)(blockIdx.x / per);
+  const int it_tile = R_IS_QUERY ? P.ntq - 1 - order : order;
+  const int rest = (int)(blockIdx.x % per);
+  const int bh = rest / P.NC, c = rest % P.NC;
+  const int c0 = c * P.L;
+  const int len = min(P.L, P.T - c0);
+  const int nt_len = (len + 127) / 128;  // tiles holding rows of this chunk
+  const int r0 = it_tile * 128;
+  if (r0 >= len) return;
+  if (*(volatile unsigned int*)&g_tc_bwd_error != 0u) return;
+  const int col0 = blockIdx.y * D2S;
+  const size_t tok0 = (size_t)bh * P.T + c0;
+  // partner tiles: dq: 0..it_tile; dk, dv: it_tile..nt_len-1
+  const int pj0 = R_IS_QUERY ? 0 : it_tile;
+  const int np = R_IS_QUERY ? it_tile + 1 : nt_len - it_tile;
+  const bool has_inter = R_IS_QUERY ? (c > 0) : (c < P.NC - 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* ring = smem + Cfg::OFF_RING;
+  uint8_t* sE = smem + Cfg::OFF_E;
+  uint8_t* sY = smem + Cfg::OFF_Y;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
+  float* rowvec = reinterpret_cast<float*>(smem + Cfg::OFF_RV);
+  float* pfC = reinterpret_cast<float*>(smem + Cfg::OFF_PF);  // partner exponent term
+  float* pfE = pfC + P.L;                                      // partner additive term (dk)
+  const volatile unsigned int* abort_flag = &g_tc_bwd_error;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < BB_COUNT; ++i) {
+      const uint32_t cnt = (i == BB_Y || i == BB_ACC) ? 128u : 1u;
+      tc::mbar_init(&bar[i], cnt);
+    }
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  // partner factors of every partner row this tile meets, and the inter row vector
+  {
+    const int pbase = pj0 * 128;
+    for (int pi = threadIdx.x; pi < np * 128; pi += blockDim.x) {
+      const int p = pbase + pi;
+      const bool ok = p < len;
+      float cexp = -INFINITY, eadd = 0.f;
+      if (ok) {
+        if (R_IS_QUERY) {
+          cexp = (P.li[tok0 + p] - P.b[tok0 + p]) * kLog2e;
+        } else {
+          const float mt = EXPV ? P.m[tok0 + p] : 0.f;
+          const float invd = EXPV ? P.inv_den[tok0 + p] : 1.f;
+          cexp = (P.b[tok0 + p] - mt) * kLog2e + log2f(invd);
+          if (KIND == KDK && EXPV) eadd = P.da[tok0 + p] / invd;
+        }
+      }
+      pfC[pi] = cexp;
+      pfE[pi] = eadd;
+    }
+    if (KIND != KDV && EXPV && has_inter)
+      for (int i = threadIdx.x; i < D2S; i += blockDim.x)
+        rowvec[i] = P.rowvec[((size_t)bh * P.NC + c) * P.dqk + col0 + i];
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tX0 = tmem, tAcc = tmem + 256;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmA);
+      tc::prefetch_tmap(&tmB);
+      tc::prefetch_tmap(&tmE);
+      uint32_t it = 0;
+      auto acquire = [&](uint32_t bytes) -> uint8_t* {
+        const uint32_t st = it & 1, ph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&bar[BB_EMPTY0 + st], ph ^ 1, abort_flag)) return nullptr;
+        tc::mbar_arrive_expect_tx(&bar[BB_FULL0 + st], bytes);
+        return ring + st * Cfg::STAGE_BYTES;
+      };
+      if (has_inter) {
+        const int gz = bh * P.NC + c;
+        for (int kb = 0; kb < Cfg::NKB && ok; ++kb) {
+          uint8_t* stg = acquire(Cfg::SLOT + 2 * Cfg::G_BYTES);
+          if (!stg) { ok = false; break; }
+          uint64_t* fb = &bar[BB_FULL0 + (it & 1)];
+          tc::tma_load_3d(stg, &tmA, fb, kb * 64, c0 + r0, bh);
+          if (G_MN) {  // G rows = contraction (d_qk block kb), columns = output slice
+            for (int eb = 0; eb < Cfg::EB; ++eb) {
+              tc::tma_load_3d(stg + Cfg::SLOT + eb * 8192, &tmGhi, fb, col0 + eb * 64, kb * 64, gz);
+              tc::tma_load_3d(stg + 2 * Cfg::SLOT + eb * 8192, &tmGlo, fb, col0 + eb * 64, kb * 64, gz);
+            }
+          } else {  // G rows = output slice, columns = contraction (d_hv block kb)
+            tc::tma_load_3d(stg + Cfg::SLOT, &tmGhi, fb, kb * 64, col0, gz);
+            tc::tma_load_3d(stg + 2 * Cfg::SLOT, &tmGlo, fb, kb * 64, col0, gz);
+          }
+          ++it;
+        }
+      }
+      for (int jj = 0; jj < np && ok; ++jj) {
+        const int prow = c0 + (pj0 + jj) * 128;
+        for (int kb = 0; kb < Cfg::NKB; ++kb) {
+          uint8_t* stg = acquire(2 * Cfg::SLOT);
+          if (!stg) { ok = false; break; }
+          uint64_t* fb = &bar[BB_FULL0 + (it & 1)];
+          tc::tma_load_3d(stg, &tmA, fb, kb * 64, c0 + r0, bh);
+          tc::tma_load_3d(stg + Cfg::SLOT, &tmB, fb, kb * 64, prow, bh);
+          ++it;
+        }
+        if (!ok) break;
+        if (jj > 0) ok = tc::mbar_wait(&bar[BB_YE], (jj - 1) & 1, abort_flag);  // E buffer free
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(&bar[BB_EFULL], Cfg::EB * Cfg::SLOT);
+        for (int eb = 0; eb < Cfg::EB; ++eb)
+          tc::tma_load_3d(sE + eb * Cfg::SLOT, &tmE, &bar[BB_EFULL], col0 + eb * 64, prow, bh);
+      }
+      // stay until the last copies this thread issued have landed
+      if (ok) ok = tc::mbar_wait(&bar[BB_EFULL], (np - 1) & 1, abort_flag);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idX = tc::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idAcc = tc::idesc_bf16(128, D2S, false, true);
+      constexpr uint32_t idG = tc::idesc_bf16(128, D2S, false, G_MN);
+      const uint32_t aRing = tc::smem_u32(ring), aE = tc::smem_u32(sE), aY = tc::smem_u32(sY);
+      uint32_t it = 0;
+      auto wait_full = [&]() -> bool {
+        return tc::mbar_wait(&bar[BB_FULL0 + (it & 1)], (it >> 1) & 1, abort_flag);
+      };
+      if (has_inter) {
+        for (int kb = 0; kb < Cfg::NKB && ok; ++kb) {
+          ok = wait_full();
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t st = aRing + (it & 1) * Cfg::STAGE_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t a = tc::sdesc_sw128(st + k * 32, 16, 1024);
+            uint64_t ghi, glo;
+            if (G_MN) {
+              ghi = tc::sdesc_sw128(st + Cfg::SLOT + k * 2048, 8192, 1024);
+              glo = tc::sdesc_sw128(st + 2 * Cfg::SLOT + k * 2048, 8192, 1024);
+            } else {
+              ghi = tc::sdesc_sw128(st + Cfg::SLOT + k * 32, 16, 1024);
+              glo = tc::sdesc_sw128(st + 2 * Cfg::SLOT + k * 32, 16, 1024);
+            }
+            tc::mma_bf16_ss(tAcc, a, ghi, idG, (kb > 0 || k > 0));
+            tc::mma_bf16_ss(tAcc, a, glo, idG, 1);
+          }
+          tc::tc_commit(&bar[BB_EMPTY0 + (it & 1)]);
+          ++it;
+        }
+        tc::tc_commit(&bar[BB_INTER]);
+      }
+      auto issue_score = [&](int jj) -> bool {
+        const uint32_t tX = tX0 + (jj & 1) * 128;
+        for (int kb = 0; kb < Cfg::NKB; ++kb) {
+          if (!wait_full()) return false;
+          tc::tc_fence_after();
+          const uint32_t st = aRing + (it & 1) * Cfg::STAGE_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16_ss(tX, tc::sdesc_sw128(st + k * 32, 16, 1024),
+                            tc::sdesc_sw128(st + Cfg::SLOT + k * 32, 16, 1024), idX, (kb > 0 || k > 0));
+          tc::tc_commit(&bar[BB_EMPTY0 + (it & 1)]);
+          ++it;
+        }
+        tc::tc_commit(&bar[BB_X0 + (jj & 1)]);
+        return true;
+      };
+      if (ok) ok = issue_score(0);
+      for (int jj = 0; jj < np && ok; ++jj) {
+        // the other X buffer was last read by the transform of jj - 1, awaited below
+        if (jj + 1 < np) ok = issue_score(jj + 1);
+        if (!ok) break;
+        ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag) &&
+             tc::mbar_wait(&bar[BB_EFULL], jj & 1, abort_flag);
+        if (ok && jj == 0 && has_inter) ok = tc::mbar_wait(&bar[BB_ACC], 0, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t offy = (k >> 2) * Cfg::SLOT + (k & 3) * 32;
+          tc::mma_bf16_ss(tAcc, tc::sdesc_sw128(aY + offy, 16, 1024),
+                          tc::sdesc_sw128(aE + k * 2048, Cfg::SLOT, 1024), idAcc,
+                          (has_inter || jj > 0 || k > 0));
+        }
+        tc::tc_commit(&bar[BB_YE]);
+      }
+      tc::tc_commit(&bar[BB_DONE]);
+    }
+  } else {
+    // ------------------------------------------------------------ tile rows
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int rl = r0 + row;
+    const bool valid = rl < len;
+    const size_t tok = tok0 + rl;
+    const unsigned full = 0xffffffffu;
+    // row-side factors
+    float Rexp = -INFINITY, eRow = 0.f, rs = 0.f, rvc = 0.f;
+    if (valid) {
+      const float bt = P.b[tok];
+      if (R_IS_QUERY) {
+        const float mt = EXPV ? P.m[tok] : 0.f;
+        const float invd = EXPV ? P.inv_den[tok] : 1.f;
+        const float dat = EXPV ? P.da[tok] : 0.f;
+        Rexp = (bt - mt) * kLog2e + log2f(invd);
+        eRow = dat / invd;
+        const float mprev = EXPV ? (c > 0 ? P.m[tok0 - 1] : -INFINITY) : 0.f;
+        const float alpha = c > 0 ? expf(bt + mprev - mt) : 0.f;
+        rs = alpha * invd;
+        rvc = alpha * dat;
+      } else {
+        const float lis = P.li[tok];
+        Rexp = (lis - bt) * kLog2e + P.log2_scale;
+        const int last = len - 1;
+        const float g = P.b[tok0 + last];
+        const float mc = EXPV ? P.m[tok0 + last] : 0.f;
+        rs = expf(g - bt + lis - mc);
+        rvc = rs;
+      }
+    }
+    const uint32_t aY = tc::smem_u32(sY);
+
+    if (has_inter) {
+      ok = __all_sync(full, tc::mbar_wait(&bar[BB_INTER], 0, abort_flag));
+      if (ok) {
+        tc::tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < D2S / 32; ++ch) {
+          float v[32];
+          tc::tmem_ld32(tAcc + lane_base + ch * 32, v);
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float x = rs * v[i];
+            if (KIND != KDV && EXPV) x += rvc * rowvec[ch * 32 + i];
+            w[i] = __float_as_uint(x);
+          }
+          tc::tmem_st32(tAcc + lane_base + ch * 32, w);
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bar[BB_ACC]);
+      }
+    }
+
+    for (int jj = 0; jj < np && ok; ++jj) {
+      ok = __all_sync(full, tc::mbar_wait(&bar[BB_X0 + (jj & 1)], (jj >> 1) & 1, abort_flag));
+      if (ok && jj > 0) ok = __all_sync(full, tc::mbar_wait(&bar[BB_YE], (jj - 1) & 1, abort_flag));
+      if (!ok) break;
+      tc::tc_fence_after();
+      const bool diag = (pj0 + jj) == it_tile;
+      const float* pc = pfC + jj * 128;
+      const float* pe = pfE + jj * 128;
+      const uint32_t tX = tX0 + (jj & 1) * 128;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float x[32];
+        tc::tmem_ld32(tX + lane_base + ch * 32, x);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float y[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int p = ch * 32 + i + u;
+            float add = 0.f;
+            if (KIND == KDQ) add = eRow;
+            if (KIND == KDK) add = pe[p];
+            float val = (x[i + u] + add) * tc::ex2(Rexp + pc[p]);
+            const bool masked = R_IS_QUERY ? (diag && p > row) : (diag && p < row);
+            y[u] = masked ? 0.f : val;
+          }
+          pk[i >> 1] = tc::pack_bf16(y[0], y[1]);
+        }
+        const int kb = ch >> 1;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int lc = (ch & 1) * 4 + q4;
+          const uint32_t addr = aY + kb * Cfg::SLOT + row * 128 + ((lc ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * q4]),
+                       "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3])
+                       : "memory");
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bar[BB_Y]);
+    }
+
+    if (ok) ok = __all_sync(full, tc::mbar_wait(&bar[BB_DONE], 0, abort_flag));
+    if (ok) {
+      tc::tc_fence_after();
+      const float fin = (KIND == KDQ) ? P.scale : 1.f;
+      bf16* orow = P.out + tok * P.d_out + col0;
+      const bf16* drow = (KIND != KDV) ? P.dot_src + tok * P.dqk + col0 : nullptr;
+      float dot = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < D2S / 32; ++ch) {
+        float v[32];
+        tc::tmem_ld32(tAcc + lane_base + ch * 32, v);
+        if (valid) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float g[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = v[8 * q4 + e] * fin;
+            if (KIND != KDV) {
+              const uint4 src = *reinterpret_cast<const uint4*>(drow + ch * 32 + q4 * 8);
+              const uint32_t sw[4] = {src.x, src.y, src.z, src.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&sw[e]);
+                dot = fmaf(__bfloat162float(s2.x), g[2 * e], dot);
+                dot = fmaf(__bfloat162float(s2.y), g[2 * e + 1], dot);
+              }
+            }
+            uint4 w;
+            w.x = tc::pack_bf16(g[0], g[1]);
+            w.y = tc::pack_bf16(g[2], g[3]);
+            w.z = tc::pack_bf16(g[4], g[5]);
+            w.w = tc::pack_bf16(g[6], g[7]);
+            *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = w;
+          }
+        }
+      }
+      if (KIND != KDV && valid) atomicAdd(&P.pdot[tok], dot);
+    }
+  }
+
+  if (!ok) atomicOr(&g_tc_bwd_error, 1u);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+bool intra_bwd_tc_supported(const Problem& p) {
+  return p.bf16() && p.L >= 128 && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
+         (p.dhv == 64 || p.dhv == 128 || p.dhv == 256 || p.dhv == 512);
+}
+
+template <int KIND, int D1, int D2S, bool G_MN, bool EXPV>
+static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  using Cfg = BwdTcCfg<D1, D2S, G_MN>;
+  const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
+  const bf16* C = (const bf16*)a.C;
+  const bf16* dC = (const bf16*)a.dC;
+  CUtensorMap tA, tB, tE, tGh, tGl;
+  bool okm = true;
+  const uint64_t BHNC = (uint64_t)p.BH * p.NC;
+  if (KIND == KDQ) {
+    okm &= make_tmap_3d_bf16(&tA, a.dh, p.dhv, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tB, a.v, p.dhv, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tE, a.k, p.dqk, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tGh, C, p.dhv, p.dqk, BHNC, 64, D2S);
+    okm &= make_tmap_3d_bf16(&tGl, C + plane, p.dhv, p.dqk, BHNC, 64, D2S);
+  } else if (KIND == KDK) {
+    okm &= make_tmap_3d_bf16(&tA, a.v, p.dhv, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tB, a.dh, p.dhv, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tE, a.q, p.dqk, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tGh, dC, p.dhv, p.dqk, BHNC, 64, D2S);
+    okm &= make_tmap_3d_bf16(&tGl, dC + plane, p.dhv, p.dqk, BHNC, 64, D2S);
+  } else {
+    okm &= make_tmap_3d_bf16(&tA, a.k, p.dqk, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tB, a.q, p.dqk, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tE, a.dh, p.dhv, p.T, p.BH, 64, 128);
+    okm &= make_tmap_3d_bf16(&tGh, dC, p.dhv, p.dqk, BHNC, 64, 64);
+    okm &= make_tmap_3d_bf16(&tGl, dC + plane, p.dhv, p.dqk, BHNC, 64, 64);
+  }
+  if (!okm) return cudaErrorInvalidValue;
+  BwdTcParams P;
+  P.b = a.b; P.li = a.li; P.m = a.m; P.inv_den = a.inv_den; P.da = a.da;
+  P.rowvec = (KIND == KDQ) ? a.n : a.dn;
+  P.dot_src = (const bf16*)((KIND == KDQ) ? a.q : a.k);
+  P.out = (bf16*)((KIND == KDQ) ? a.dq : (KIND == KDK) ? a.dk : a.dv);
+  P.pdot = (KIND == KDQ) ? a.pq : a.pk;
+  P.T = p.T; P.L = p.L; P.NC = p.NC; P.BH = p.BH; P.ntq = p.L / 128;
+  P.d_out = (KIND == KDV) ? p.dhv : p.dqk;
+  P.dqk = p.dqk;
+  P.scale = p.scale;
+  P.log2_scale = log2f(p.scale);
+  const size_t smem = Cfg::smem_bytes(p.L);
+  auto kern = intra_bwd_tc_kernel<KIND, D1, D2S, G_MN, EXPV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)(p.BH * p.NC * P.ntq), (unsigned)(P.d_out / D2S)), block(192);
+  kern<<<grid, block, smem, s>>>(tA, tB, tE, tGh, tGl, P);
+  return cudaGetLastError();
+}
+
+template <int KIND, bool EXPV>
+static cudaError_t dispatch_kind(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  constexpr bool GMN = (KIND == KDV);
+  const int d1 = (KIND == KDV) ? p.dqk : p.dhv;
+  const int dout = (KIND == KDV) ? p.dhv : p.dqk;
+  const bool wide = dout >= 128;
+#define MLSTM_BWD_TC_D1(D1)                                                                \
+  if (d1 == D1) return wide ? launch_kind<KIND, D1, 128, GMN, EXPV>(p, a, s)               \
+                            : launch_kind<KIND, D1, 64, GMN, EXPV>(p, a, s);
+  MLSTM_BWD_TC_D1(64)
+  MLSTM_BWD_TC_D1(128)
+  MLSTM_BWD_TC_D1(256)
+  MLSTM_BWD_TC_D1(512)
+#undef MLSTM_BWD_TC_D1
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_dq_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  return p.exp_variant() ? dispatch_kind<KDQ, true>(p, a, s) : dispatch_kind<KDQ, false>(p, a, s);
+}
+cudaError_t launch_dk_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  return p.exp_variant() ? dispatch_kind<KDK, true>(p, a, s) : dispatch_kind<KDK, false>(p, a, s);
+}
+cudaError_t launch_dv_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  return p.exp_variant() ? dispatch_kind<KDV, true>(p, a, s) : dispatch_kind<KDV, false>(p, a, s);
+}
+
+cudaError_t fetch_tc_bwd_error(unsigned int* flag) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_bwd_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_tc_bwd_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace mlstm
