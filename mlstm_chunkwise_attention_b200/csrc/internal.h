@@ -64,5 +64,9 @@ cudaError_t launch_dq_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dk_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dv_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_bwd_error(unsigned int* flag);
+bool state_tc_supported(const Problem& p);
+cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t fetch_tc_state_error(unsigned int* flag);
 
 }  // namespace mlstm

@@ -104,7 +104,10 @@ constexpr int kMaxSteps = 8;
 int fwd_plan(const Problem& p, FwdStep* st) {
   int n = 0;
   st[n++] = {"gate_prep", mlstm::launch_gate_prep};
-  st[n++] = {"state_fwd_simt", mlstm::launch_state_fwd_simt};
+  if (mlstm::state_tc_supported(p))
+    st[n++] = {"state_fwd_tc", mlstm::launch_state_fwd_tc};
+  else
+    st[n++] = {"state_fwd_simt", mlstm::launch_state_fwd_simt};
   if (mlstm::output_fwd_tc_supported(p))
     st[n++] = {"output_fwd_tc", mlstm::launch_output_fwd_tc};
   else
@@ -116,7 +119,10 @@ int bwd_plan(const Problem& p, BwdStep* st) {
   (void)p;
   int n = 0;
   st[n++] = {"bwd_token_prep", mlstm::launch_bwd_token_prep};
-  st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
+  if (mlstm::state_tc_supported(p))
+    st[n++] = {"state_bwd_tc", mlstm::launch_state_bwd_tc};
+  else
+    st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
   if (mlstm::intra_bwd_tc_supported(p)) {
     st[n++] = {"dq_tc", mlstm::launch_dq_tc};
     st[n++] = {"dk_tc", mlstm::launch_dk_tc};
@@ -319,12 +325,14 @@ const char* mlstm_last_error(void) { return g_last_error; }
 int mlstm_device_status(void* stream) {
   int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
   if (st != MLSTM_OK) return st;
-  unsigned int flag = 0, flag_bwd = 0;
+  unsigned int flag = 0, flag_bwd = 0, flag_state = 0;
   st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_bwd_error(&flag_bwd), "device error flag");
   if (st != MLSTM_OK) return st;
-  flag |= flag_bwd;
+  st = cuda_status(mlstm::fetch_tc_state_error(&flag_state), "device error flag");
+  if (st != MLSTM_OK) return st;
+  flag |= flag_bwd | flag_state;
   if (flag) {
     snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
     return MLSTM_ERR_TIMEOUT;

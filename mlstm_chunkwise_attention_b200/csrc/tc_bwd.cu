@@ -303,11 +303,17 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
         rvc = alpha * dat;
       } else {
         const float lis = P.li[tok];
-        Rexp = (lis - bt) * kLog2e + P.log2_scale;
+        // dk rounds exactly the bf16 values the dq kernel rounds (same terms in the same
+        // order); 1/sqrt(d_qk) is applied in its epilogue instead.  Then the row sums of
+        // the rounded dS tile (q.dq) and its column sums (k.dk) cancel over the sequence
+        // as they do in exact arithmetic, which the forget-gate gradient (a reverse cumsum
+        // of q.dq - k.dk) needs.
+        Rexp = (lis - bt) * kLog2e + (KIND == KDV ? P.log2_scale : 0.f);
         const int last = len - 1;
         const float g = P.b[tok0 + last];
         const float mc = EXPV ? P.m[tok0 + last] : 0.f;
         rs = expf(g - bt + lis - mc);
+        if (KIND == KDK) rs /= P.scale;
         rvc = rs;
       }
     }
@@ -358,7 +364,9 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
             float add = 0.f;
             if (KIND == KDQ) add = eRow;
             if (KIND == KDK) add = pe[p];
-            float val = (x[i + u] + add) * tc::ex2(Rexp + pc[p]);
+            // t-side term first, then the s-side term, in every kernel
+            const float ex = R_IS_QUERY ? (Rexp + pc[p]) : (pc[p] + Rexp);
+            float val = (x[i + u] + add) * tc::ex2(ex);
             const bool masked = R_IS_QUERY ? (diag && p > row) : (diag && p < row);
             y[u] = masked ? 0.f : val;
           }
@@ -382,7 +390,7 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
     if (ok) ok = __all_sync(full, tc::mbar_wait(&bar[BB_DONE], 0, abort_flag));
     if (ok) {
       tc::tc_fence_after();
-      const float fin = (KIND == KDQ) ? P.scale : 1.f;
+      const float fin = (KIND == KDV) ? 1.f : P.scale;
       bf16* orow = P.out + tok * P.d_out + col0;
       const bf16* drow = (KIND != KDV) ? P.dot_src + tok * P.dqk + col0 : nullptr;
       float dot = 0.f;

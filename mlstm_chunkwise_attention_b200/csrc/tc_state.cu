@@ -1,0 +1,379 @@
+// Chunk-state recurrences on the fifth-generation tensor cores: the forward
+// inter-chunk states (K-b) and the backward state gradients (K-d1).
+//
+// "Tiled Flash Linear Attention: More Efficient Linear RNN and xLSTM Kernels"
+// (TFLA summary page, Problem; arXiv abstract page, Abstract): the chunkwise
+// form materialises the state at every chunk boundary.
+//   forward:  C_{c+1} = beta_c C_c + K_c^T diag(w) V_c,   w_s = exp(g_c - b_s + log i_s - m_c)
+//             n_{c+1} = beta_c n_c + K_c^T w                               (mLSTMexp)
+//   backward: G_{c-1} = beta_c G_c + Q_c^T diag(u) dH_c,  u_t = alpha_t / (sqrt(d_qk) den_t)
+//             gn_{c-1} = beta_c gn_c + Q_c^T (alpha_t da_t / sqrt(d_qk))    (mLSTMexp)
+// with beta_c = exp(g_c + m_{c-1} - m_c).  The forward stores the state
+// entering every chunk, the backward the gradient of the state leaving it,
+// both as hi/lo bf16 planes (hi + lo keeps about 16 mantissa bits).
+//
+// One CTA owns a 128-row (d_qk) by 64-column (d_hv) tile of the state and
+// walks the chunks in order; the fp32 running state lives in registers of the
+// four epilogue warps (one state row per thread).  Each chunk is streamed in
+// 64-token sub-tiles through a TMA ring; two warps scale the value-side
+// operand by the per-token weight and split it into hi and lo bf16 tiles, so
+// the contraction K^T (w V) keeps fp32-level accuracy (two MMAs per step).
+// Warp roles: 0 TMA, 1 MMA + TMEM, 2..3 scaling, 4..7 epilogue.
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace mlstm {
+
+static __device__ unsigned int g_tc_state_error;
+
+namespace {
+
+template <int NV>
+struct StateTcCfg {
+  static constexpr int STAGES = 2;
+  static constexpr int SUB = 64;                 // tokens per sub-tile (the MMA K extent)
+  static constexpr int A_BYTES = 2 * 8192;       // 64 tokens x 128 state rows, two 64-row blocks
+  static constexpr int B_BYTES = (NV / 64) * 8192;
+  static constexpr int BN_BYTES = 2048;          // 16 x 64 K-major tile of the normaliser column
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_BHI = OFF_A + A_BYTES;
+  static constexpr int OFF_BLO = OFF_BHI + B_BYTES;
+  static constexpr int OFF_NHI = OFF_BLO + B_BYTES;
+  static constexpr int OFF_NLO = OFF_NHI + BN_BYTES;
+  static constexpr int STAGE_BYTES = OFF_NLO + BN_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr size_t SMEM = 1024 + OFF_TMEM + 16;
+  static constexpr uint32_t TMEM_COLS = 256;     // U in [0, NV), normaliser column block at [NV, NV + 16)
+};
+
+enum { SB_FULL0 = 0, SB_SCALED0 = 2, SB_EMPTY0 = 4, SB_U = 6, SB_UFREE = 7, SB_COUNT = 8 };
+
+}  // namespace
+
+struct StateTcParams {
+  const float *b, *li, *m, *inv_den, *da;
+  bf16* out;      // hi plane; the lo plane follows after `plane` elements
+  float* nout;    // [BH, NC, dqk] normaliser state (forward) or its gradient (backward)
+  size_t plane;
+  int T, L, NC, dqk, dhv;
+  float scale;
+};
+
+template <bool BWD, bool EXPV, int NV>
+__global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                          const __grid_constant__ CUtensorMap tmB,
+                                                          const StateTcParams P) {
+  using Cfg = StateTcCfg<NV>;
+  constexpr int SUB = Cfg::SUB;
+  if (*(volatile unsigned int*)&g_tc_state_error != 0u) return;
+  // value-column tiles vary fastest so the CTAs sharing one head's key rows run together
+  const int dv0 = blockIdx.x * NV, dk0 = blockIdx.y * 128, bh = blockIdx.z;
+  const bool with_n = EXPV && blockIdx.x == 0;
+  const size_t tokh = (size_t)bh * P.T;
+  const int NC = P.NC;
+  const int nsteps = NC - 1;  // chunks whose contribution is needed
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
+  const volatile unsigned int* abort_flag = &g_tc_state_error;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SB_COUNT; ++i) {
+      uint32_t cnt = 1;
+      if (i == SB_SCALED0 || i == SB_SCALED0 + 1) cnt = 64;
+      if (i == SB_UFREE) cnt = 128;
+      tc::mbar_init(&bar[i], cnt);
+    }
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  // rows 1..15 of the normaliser-column tiles stay zero
+  for (int i = threadIdx.x; i < Cfg::STAGES * 2 * Cfg::BN_BYTES / 4; i += blockDim.x) {
+    const int st = i / (2 * Cfg::BN_BYTES / 4), r = i % (2 * Cfg::BN_BYTES / 4);
+    reinterpret_cast<uint32_t*>(smem + st * Cfg::STAGE_BYTES + Cfg::OFF_NHI)[r] = 0u;
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tU = tmem, tN = tmem + NV;
+  bool ok = true;
+
+  auto chunk_of = [&](int u) { return BWD ? NC - 1 - u : u; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int u = 0; u < nsteps && ok; ++u) {
+        const int c = chunk_of(u), c0 = c * P.L, len = min(P.L, P.T - c0);
+        for (int q = 0; q * SUB < len; ++q, ++it) {
+          const uint32_t st = it % Cfg::STAGES, ph = (it / Cfg::STAGES) & 1;
+          ok = tc::mbar_wait(&bar[SB_EMPTY0 + st], ph ^ 1, abort_flag);
+          if (!ok) break;
+          uint8_t* stg = smem + st * Cfg::STAGE_BYTES;
+          tc::mbar_arrive_expect_tx(&bar[SB_FULL0 + st], Cfg::A_BYTES + Cfg::B_BYTES);
+          for (int h = 0; h < 2; ++h)
+            tc::tma_load_3d(stg + Cfg::OFF_A + h * 8192, &tmA, &bar[SB_FULL0 + st], dk0 + h * 64,
+                            c0 + q * SUB, bh);
+          for (int h = 0; h < NV / 64; ++h)
+            tc::tma_load_3d(stg + Cfg::OFF_BHI + h * 8192, &tmB, &bar[SB_FULL0 + st], dv0 + h * 64,
+                            c0 + q * SUB, bh);
+        }
+      }
+      // wait for the last loads this thread issued
+      if (ok && it > 0) {
+        const uint32_t last = it - 1;
+        ok = tc::mbar_wait(&bar[SB_FULL0 + last % Cfg::STAGES], (last / Cfg::STAGES) & 1, abort_flag);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idU = tc::idesc_bf16(128, NV, true, true);
+      constexpr uint32_t idN = tc::idesc_bf16(128, 16, true, false);
+      const uint32_t base = tc::smem_u32(smem);
+      uint32_t it = 0;
+      for (int u = 0; u < nsteps && ok; ++u) {
+        const int c = chunk_of(u), c0 = c * P.L, len = min(P.L, P.T - c0);
+        if (u > 0) ok = tc::mbar_wait(&bar[SB_UFREE], (u - 1) & 1, abort_flag);  // U read out
+        if (!ok) break;
+        for (int q = 0; q * SUB < len; ++q, ++it) {
+          const uint32_t st = it % Cfg::STAGES, ph = (it / Cfg::STAGES) & 1;
+          ok = tc::mbar_wait(&bar[SB_FULL0 + st], ph, abort_flag) &&
+               tc::mbar_wait(&bar[SB_SCALED0 + st], ph, abort_flag);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t sa = base + st * Cfg::STAGE_BYTES;
+#pragma unroll
+          for (int k = 0; k < SUB / 16; ++k) {
+            const uint64_t a = tc::sdesc_sw128(sa + Cfg::OFF_A + k * 2048, 8192, 1024);
+            const uint64_t bhi = tc::sdesc_sw128(sa + Cfg::OFF_BHI + k * 2048, 8192, 1024);
+            const uint64_t blo = tc::sdesc_sw128(sa + Cfg::OFF_BLO + k * 2048, 8192, 1024);
+            tc::mma_bf16_ss(tU, a, bhi, idU, (q > 0 || k > 0));
+            tc::mma_bf16_ss(tU, a, blo, idU, 1);
+            if (with_n) {
+              const uint64_t nhi = tc::sdesc_sw128(sa + Cfg::OFF_NHI + k * 32, 16, 1024);
+              const uint64_t nlo = tc::sdesc_sw128(sa + Cfg::OFF_NLO + k * 32, 16, 1024);
+              tc::mma_bf16_ss(tN, a, nhi, idN, (q > 0 || k > 0));
+              tc::mma_bf16_ss(tN, a, nlo, idN, 1);
+            }
+          }
+          tc::tc_commit(&bar[SB_EMPTY0 + st]);
+        }
+        if (!ok) break;
+        tc::tc_commit(&bar[SB_U]);
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ scaling (one token row per thread)
+    const int r = threadIdx.x - 64;  // 0..63
+    uint32_t it = 0;
+    for (int u = 0; u < nsteps && ok; ++u) {
+      const int c = chunk_of(u), c0 = c * P.L, len = min(P.L, P.T - c0);
+      const size_t ct = tokh + c0;
+      float g = 0.f, mc = 0.f, mprev = 0.f;
+      if (!BWD) {
+        g = P.b[ct + len - 1];
+        mc = EXPV ? P.m[ct + len - 1] : 0.f;
+      } else {
+        mprev = EXPV ? (c > 0 ? P.m[ct - 1] : -INFINITY) : 0.f;
+      }
+      for (int q = 0; q * SUB < len; ++q, ++it) {
+        const uint32_t st = it % Cfg::STAGES, ph = (it / Cfg::STAGES) & 1;
+        const int s = q * SUB + r;
+        float wv = 0.f, wn = 0.f;
+        if (s < len) {
+          const size_t t = ct + s;
+          if (!BWD) {
+            wv = expf(g - P.b[t] + P.li[t] - mc);
+            wn = wv;
+          } else {
+            const float mt = EXPV ? P.m[t] : 0.f;
+            const float alpha = expf(P.b[t] + mprev - mt) * P.scale;
+            wv = alpha * (EXPV ? P.inv_den[t] : 1.f);
+            wn = EXPV ? alpha * P.da[t] : 0.f;
+          }
+        }
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_FULL0 + st], ph, abort_flag));
+        if (!ok) break;
+        uint8_t* stg = smem + st * Cfg::STAGE_BYTES;
+#pragma unroll
+        for (int h = 0; h < NV / 64; ++h) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int pch = (jj + r) & 7;
+            const uint32_t off = h * 8192 + r * 128 + pch * 16;
+            uint4 raw = *reinterpret_cast<const uint4*>(stg + Cfg::OFF_BHI + off);
+            uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w}, hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 x2 = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+              const float y0 = __bfloat162float(x2.x) * wv, y1 = __bfloat162float(x2.y) * wv;
+              const bf16 h0 = __float2bfloat16_rn(y0), h1 = __float2bfloat16_rn(y1);
+              hi[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+              lo[e] = tc::pack_bf16(y0 - __bfloat162float(h0), y1 - __bfloat162float(h1));
+            }
+            *reinterpret_cast<uint4*>(stg + Cfg::OFF_BHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(stg + Cfg::OFF_BLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+        if (with_n) {  // row 0 of the K-major normaliser tile: element s at byte 2 s
+          const bf16 nh = __float2bfloat16_rn(wn);
+          const bf16 nl = __float2bfloat16_rn(wn - __bfloat162float(nh));
+          reinterpret_cast<bf16*>(stg + Cfg::OFF_NHI)[r] = nh;
+          reinterpret_cast<bf16*>(stg + Cfg::OFF_NLO)[r] = nl;
+        }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bar[SB_SCALED0 + st]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: running state rows
+    const int i = 32 * (warp & 3) + lane;  // state row within the tile (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const bool valid = dk0 + i < P.dqk;
+    float S[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) S[j] = 0.f;
+    float sn = 0.f;
+    for (int u = 0; u <= nsteps; ++u) {
+      const int c = chunk_of(u);
+      // store the state at this chunk boundary
+      if (valid) {
+        const size_t row = (((size_t)bh * NC + c) * P.dqk + dk0 + i) * P.dhv + dv0;
+#pragma unroll
+        for (int j = 0; j < NV; j += 8) {
+          uint4 vh, vl;
+          uint32_t* ph = reinterpret_cast<uint32_t*>(&vh);
+          uint32_t* pl = reinterpret_cast<uint32_t*>(&vl);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = S[j + 2 * e], x1 = S[j + 2 * e + 1];
+            const bf16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+            ph[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+            pl[e] = tc::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+          }
+          *reinterpret_cast<uint4*>(P.out + row + j) = vh;
+          *reinterpret_cast<uint4*>(P.out + P.plane + row + j) = vl;
+        }
+        if (with_n) P.nout[((size_t)bh * NC + c) * P.dqk + dk0 + i] = sn;
+      }
+      if (u == nsteps) break;
+      const int c0 = c * P.L, len = min(P.L, P.T - c0);
+      const size_t ct = tokh + c0;
+      const float g = P.b[ct + len - 1];
+      float beta;
+      if (EXPV) {
+        const float mc = P.m[ct + len - 1];
+        const float mp = c > 0 ? P.m[ct - 1] : -INFINITY;
+        beta = c > 0 ? expf(g + mp - mc) : 0.f;
+      } else {
+        beta = expf(g);
+      }
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_U], u & 1, abort_flag));
+      if (!ok) break;
+      tc::tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < NV / 32; ++ch) {
+        float v[32];
+        tc::tmem_ld32(tU + lane_base + ch * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) S[ch * 32 + e] = fmaf(beta, S[ch * 32 + e], v[e]);
+      }
+      if (with_n) {
+        float v[32];
+        tc::tmem_ld32(tN + lane_base, v);  // reads the 16-column block and 16 unused columns
+        sn = fmaf(beta, sn, v[0]);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bar[SB_UFREE]);
+    }
+  }
+
+  if (!ok) atomicOr(&g_tc_state_error, 1u);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+bool state_tc_supported(const Problem& p) {
+  return p.bf16() && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) && (p.dhv % 64 == 0);
+}
+
+template <bool BWD, bool EXPV, int NV>
+static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* B, bf16* out,
+                                   float* nout, const float* b, const float* li, const float* m,
+                                   const float* inv_den, const float* da, cudaStream_t s) {
+  using Cfg = StateTcCfg<NV>;
+  CUtensorMap tA, tB;
+  const uint32_t dkbox = p.dqk >= 64 ? 64 : p.dqk;
+  if (!make_tmap_3d_bf16(&tA, A, p.dqk, p.T, p.BH, dkbox, 64) ||
+      !make_tmap_3d_bf16(&tB, B, p.dhv, p.T, p.BH, 64, 64))
+    return cudaErrorInvalidValue;
+  StateTcParams P;
+  P.b = b; P.li = li; P.m = m; P.inv_den = inv_den; P.da = da;
+  P.out = out; P.nout = nout;
+  P.plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
+  P.T = p.T; P.L = p.L; P.NC = p.NC; P.dqk = p.dqk; P.dhv = p.dhv;
+  P.scale = p.scale;
+  auto kern = state_tc_kernel<BWD, EXPV, NV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)(p.dhv / NV), (unsigned)((p.dqk + 127) / 128), (unsigned)p.BH), block(256);
+  kern<<<grid, block, Cfg::SMEM, s>>>(tA, tB, P);
+  return cudaGetLastError();
+}
+
+// 64 value columns per CTA keep the fp32 running state (64 registers per
+// thread) inside the 128-register budget of two CTAs per SM.
+template <bool BWD, bool EXPV>
+static cudaError_t launch_state_tc_nv(const Problem& p, const void* A, const void* B, bf16* out,
+                                      float* nout, const float* b, const float* li, const float* m,
+                                      const float* inv_den, const float* da, cudaStream_t s) {
+  return launch_state_tc<BWD, EXPV, 64>(p, A, B, out, nout, b, li, m, inv_den, da, s);
+}
+
+cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  if (p.exp_variant())
+    return launch_state_tc_nv<false, true>(p, a.k, a.v, (bf16*)a.C, a.n, a.b, a.li, a.m, nullptr,
+                                           nullptr, s);
+  return launch_state_tc_nv<false, false>(p, a.k, a.v, (bf16*)a.C, a.n, a.b, a.li, a.m, nullptr,
+                                          nullptr, s);
+}
+
+cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  if (p.exp_variant())
+    return launch_state_tc_nv<true, true>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
+                                          a.inv_den, a.da, s);
+  return launch_state_tc_nv<true, false>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
+                                         a.inv_den, a.da, s);
+}
+
+cudaError_t fetch_tc_state_error(unsigned int* flag) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_state_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_tc_state_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace mlstm
