@@ -120,41 +120,58 @@ cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s)
 // K-d0: per token, 1/den_t and the gradient of the stabilised normaliser,
 // da_t = -(dh_t . h_t) sign(a~_t) / den_t when |a~_t| > exp(-m_t), else 0
 // (den_t = max(|a~_t|, exp(-m_t)), h_t = num_t / den_t).  Also zeroes the
-// per-token dot-product accumulators.  One warp per token.
+// per-token dot-product accumulators.  Groups of LPT lanes own one token and
+// read its rows with 16-byte loads; warps stride over the tokens.
 // ---------------------------------------------------------------------------
 template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(256) bwd_token_prep_kernel(
     const TIO* __restrict__ h, const TIO* __restrict__ dh, const float* __restrict__ abar,
     const float* __restrict__ m, float* __restrict__ inv_den, float* __restrict__ da,
     float* __restrict__ pq, float* __restrict__ pk, long long ntok, int dhv) {
-  const long long tok = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  constexpr int VEC = 16 / sizeof(TIO);  // elements per 16-byte load
   const int lane = threadIdx.x & 31;
-  if (tok >= ntok) return;
-  if (lane == 0) {
-    pq[tok] = 0.f;
-    pk[tok] = 0.f;
-  }
-  if (!EXPV) {
-    if (lane == 0) inv_den[tok] = 1.f;
-    return;
-  }
-  float dot = 0.f;
-  const TIO* hr = h + tok * dhv;
-  const TIO* dr = dh + tok * dhv;
-  for (int j = lane; j < dhv; j += 32) dot += to_f32(hr[j]) * to_f32(dr[j]);
-  dot = warp_sum(dot);
-  if (lane == 0) {
-    const float a = abar[tok];
-    const float floor_ = expf(-m[tok]);
-    const float den = fmaxf(fabsf(a), floor_);
-    inv_den[tok] = 1.f / den;
-    da[tok] = fabsf(a) > floor_ ? -dot * copysignf(1.f, a) / den : 0.f;
+  const int lpt = min(32, dhv / VEC);    // lanes per token (a power of two)
+  const int tpw = 32 / lpt;              // tokens per warp step
+  const int sub = lane / lpt, sl = lane % lpt;
+  const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long base = warp_id * tpw; base < ntok; base += nwarps * tpw) {
+    const long long tok = base + sub;
+    const bool valid = tok < ntok;
+    float dot = 0.f;
+    if (EXPV && valid) {
+      const TIO* hr = h + tok * dhv;
+      const TIO* dr = dh + tok * dhv;
+      for (int j = sl * VEC; j < dhv; j += lpt * VEC) {
+        const uint4 hv = *reinterpret_cast<const uint4*>(hr + j);
+        const uint4 dv = *reinterpret_cast<const uint4*>(dr + j);
+        const TIO* he = reinterpret_cast<const TIO*>(&hv);
+        const TIO* de = reinterpret_cast<const TIO*>(&dv);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) dot = fmaf(to_f32(he[e]), to_f32(de[e]), dot);
+      }
+    }
+    for (int o = lpt >> 1; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (valid && sl == 0) {
+      pq[tok] = 0.f;
+      pk[tok] = 0.f;
+      if (EXPV) {
+        const float a = abar[tok];
+        const float floor_ = expf(-m[tok]);
+        const float den = fmaxf(fabsf(a), floor_);
+        inv_den[tok] = 1.f / den;
+        da[tok] = fabsf(a) > floor_ ? -dot * copysignf(1.f, a) / den : 0.f;
+      } else {
+        inv_den[tok] = 1.f;
+      }
+    }
   }
 }
 
 cudaError_t launch_bwd_token_prep(const Problem& p, const BwdArgs& a, cudaStream_t s) {
   const long long ntok = (long long)p.BH * p.T;
-  dim3 block(256), grid((unsigned)((ntok + 7) / 8));
+  const long long want = (ntok + 15) / 16;  // blocks of 8 warps, ~2 tokens per warp
+  dim3 block(256), grid((unsigned)(want < 148LL * 16 ? want : 148LL * 16));
   if (p.bf16()) {
     if (p.exp_variant())
       bwd_token_prep_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.h, (const bf16*)a.dh, a.abar, a.m, a.inv_den, a.da, a.pq, a.pk, ntok, p.dhv);

@@ -34,29 +34,32 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 enum { KDQ = 0, KDK = 1, KDV = 2 };
 
-template <int D1, int D2S, bool G_MN>
+// NXBUF score buffers in TMEM: 1 when every row tile has a single partner tile
+// (chunk 128), so the CTA fits in 256 TMEM columns and ~99 KB of shared memory
+// and two CTAs share an SM; 2 otherwise (the next score overlaps the transform).
+template <int D1, int D2S, bool G_MN, int NXBUF>
 struct BwdTcCfg {
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = NXBUF == 1 ? 2 : 4;
   static constexpr int SLOT = 16384;  // one 128 x 64 bf16 block
-  static constexpr int STAGE_BYTES = 3 * SLOT;
+  static constexpr int STAGE_BYTES = 2 * SLOT;
   static constexpr int NKB = D1 / 64;  // K-blocks of the score GEMM and the inter GEMM
   static constexpr int EB = D2S / 64;  // 64-column blocks of E and of the output slice
   static constexpr int OFF_RING = 0;
-  static constexpr int OFF_E = STAGES * STAGE_BYTES;
-  static constexpr int OFF_Y = OFF_E + EB * SLOT;
+  static constexpr int OFF_Y = STAGES * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_Y + 2 * SLOT;
   static constexpr int NBAR = 16;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_RV = OFF_TMEM + 16;
   static constexpr int OFF_PF = OFF_RV + D2S * 4;  // partner factors, 2 x L floats
-  static constexpr uint32_t TMEM_COLS = 512;       // X buffers [0,128), [128,256); Acc [256, 256+D2S)
+  static constexpr uint32_t TMEM_COLS = NXBUF == 1 ? 256 : 512;  // X buffers, then Acc
+  static constexpr uint32_t ACC_COL = NXBUF * 128;
   static constexpr uint32_t G_BYTES = G_MN ? (uint32_t)EB * 8192u : (uint32_t)D2S * 128u;
+  static constexpr uint32_t E_BYTES = (uint32_t)EB * SLOT;
   static size_t smem_bytes(int L) { return 1024 + OFF_PF + (size_t)2 * L * 4; }
 };
 
 enum {
-  BB_FULL0 = 0, BB_FULL1, BB_EMPTY0, BB_EMPTY1, BB_EFULL, BB_X0, BB_X1, BB_Y, BB_YE, BB_INTER,
-  BB_ACC, BB_DONE, BB_COUNT
+  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_YE, BB_INTER, BB_ACC, BB_DONE, BB_COUNT
 };
 
 }  // namespace
@@ -71,13 +74,14 @@ struct BwdTcParams {
   float scale, log2_scale;
 };
 
-template <int KIND, int D1, int D2S, bool G_MN, bool EXPV>
-__global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
+template <int KIND, int D1, int D2S, bool G_MN, bool EXPV, int NXBUF>
+__global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmGhi,
     const __grid_constant__ CUtensorMap tmGlo, const BwdTcParams P) {
-  using Cfg = BwdTcCfg<D1, D2S, G_MN>;
+  using Cfg = BwdTcCfg<D1, D2S, G_MN, NXBUF>;
   constexpr bool R_IS_QUERY = (KIND == KDQ);
+  constexpr int ST = Cfg::STAGES;
 
   const int per = P.BH * P.NC;
   // heaviest row tiles first: dq tiles near the chunk end, dk/dv tiles near its start
@@ -102,7 +106,6 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem + Cfg::OFF_RING;
-  uint8_t* sE = smem + Cfg::OFF_E;
   uint8_t* sY = smem + Cfg::OFF_Y;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
@@ -151,60 +154,70 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tX0 = tmem, tAcc = tmem + 256;
+  const uint32_t tX0 = tmem, tAcc = tmem + Cfg::ACC_COL;
   bool ok = true;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Every operand goes through one ring, in the order the MMA thread consumes it:
+    // inter (A, G_hi), (A, G_lo) per K-block; score(0); then per partner jj:
+    // score(jj + 1) if any, E(jj).
     if (lane == 0) {
       tc::prefetch_tmap(&tmA);
       tc::prefetch_tmap(&tmB);
       tc::prefetch_tmap(&tmE);
       uint32_t it = 0;
-      auto acquire = [&](uint32_t bytes) -> uint8_t* {
-        const uint32_t st = it & 1, ph = (it >> 1) & 1;
+      auto acquire = [&](uint32_t bytes, uint64_t*& fb) -> uint8_t* {
+        const uint32_t st = it % ST, ph = (it / ST) & 1;
         if (!tc::mbar_wait(&bar[BB_EMPTY0 + st], ph ^ 1, abort_flag)) return nullptr;
-        tc::mbar_arrive_expect_tx(&bar[BB_FULL0 + st], bytes);
+        fb = &bar[BB_FULL0 + st];
+        tc::mbar_arrive_expect_tx(fb, bytes);
+        ++it;
         return ring + st * Cfg::STAGE_BYTES;
+      };
+      auto load_score = [&](int jj) -> bool {
+        const int prow = c0 + (pj0 + jj) * 128;
+        for (int kb = 0; kb < Cfg::NKB; ++kb) {
+          uint64_t* fb;
+          uint8_t* stg = acquire(2 * Cfg::SLOT, fb);
+          if (!stg) return false;
+          tc::tma_load_3d(stg, &tmA, fb, kb * 64, c0 + r0, bh);
+          tc::tma_load_3d(stg + Cfg::SLOT, &tmB, fb, kb * 64, prow, bh);
+        }
+        return true;
       };
       if (has_inter) {
         const int gz = bh * P.NC + c;
         for (int kb = 0; kb < Cfg::NKB && ok; ++kb) {
-          uint8_t* stg = acquire(Cfg::SLOT + 2 * Cfg::G_BYTES);
-          if (!stg) { ok = false; break; }
-          uint64_t* fb = &bar[BB_FULL0 + (it & 1)];
-          tc::tma_load_3d(stg, &tmA, fb, kb * 64, c0 + r0, bh);
-          if (G_MN) {  // G rows = contraction (d_qk block kb), columns = output slice
-            for (int eb = 0; eb < Cfg::EB; ++eb) {
-              tc::tma_load_3d(stg + Cfg::SLOT + eb * 8192, &tmGhi, fb, col0 + eb * 64, kb * 64, gz);
-              tc::tma_load_3d(stg + 2 * Cfg::SLOT + eb * 8192, &tmGlo, fb, col0 + eb * 64, kb * 64, gz);
+          for (int half = 0; half < 2 && ok; ++half) {
+            const CUtensorMap* tg = half == 0 ? &tmGhi : &tmGlo;
+            uint64_t* fb;
+            uint8_t* stg = acquire(Cfg::SLOT + Cfg::G_BYTES, fb);
+            if (!stg) { ok = false; break; }
+            tc::tma_load_3d(stg, &tmA, fb, kb * 64, c0 + r0, bh);
+            if (G_MN) {  // G rows = contraction (d_qk block kb), columns = output slice
+              for (int eb = 0; eb < Cfg::EB; ++eb)
+                tc::tma_load_3d(stg + Cfg::SLOT + eb * 8192, tg, fb, col0 + eb * 64, kb * 64, gz);
+            } else {  // G rows = output slice, columns = contraction (d_hv block kb)
+              tc::tma_load_3d(stg + Cfg::SLOT, tg, fb, kb * 64, col0, gz);
             }
-          } else {  // G rows = output slice, columns = contraction (d_hv block kb)
-            tc::tma_load_3d(stg + Cfg::SLOT, &tmGhi, fb, kb * 64, col0, gz);
-            tc::tma_load_3d(stg + 2 * Cfg::SLOT, &tmGlo, fb, kb * 64, col0, gz);
           }
-          ++it;
         }
       }
+      if (ok) ok = load_score(0);
       for (int jj = 0; jj < np && ok; ++jj) {
+        if (jj + 1 < np) ok = load_score(jj + 1);
+        if (!ok) break;
+        uint64_t* fb;
+        uint8_t* stg = acquire(Cfg::E_BYTES, fb);
+        if (!stg) { ok = false; break; }
         const int prow = c0 + (pj0 + jj) * 128;
-        for (int kb = 0; kb < Cfg::NKB; ++kb) {
-          uint8_t* stg = acquire(2 * Cfg::SLOT);
-          if (!stg) { ok = false; break; }
-          uint64_t* fb = &bar[BB_FULL0 + (it & 1)];
-          tc::tma_load_3d(stg, &tmA, fb, kb * 64, c0 + r0, bh);
-          tc::tma_load_3d(stg + Cfg::SLOT, &tmB, fb, kb * 64, prow, bh);
-          ++it;
-        }
-        if (!ok) break;
-        if (jj > 0) ok = tc::mbar_wait(&bar[BB_YE], (jj - 1) & 1, abort_flag);  // E buffer free
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bar[BB_EFULL], Cfg::EB * Cfg::SLOT);
         for (int eb = 0; eb < Cfg::EB; ++eb)
-          tc::tma_load_3d(sE + eb * Cfg::SLOT, &tmE, &bar[BB_EFULL], col0 + eb * 64, prow, bh);
+          tc::tma_load_3d(stg + eb * Cfg::SLOT, &tmE, fb, col0 + eb * 64, prow, bh);
       }
       // stay until the last copies this thread issued have landed
-      if (ok) ok = tc::mbar_wait(&bar[BB_EFULL], (np - 1) & 1, abort_flag);
+      if (ok && it > 0)
+        ok = tc::mbar_wait(&bar[BB_FULL0 + (it - 1) % ST], ((it - 1) / ST) & 1, abort_flag);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -212,69 +225,69 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
       constexpr uint32_t idX = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idAcc = tc::idesc_bf16(128, D2S, false, true);
       constexpr uint32_t idG = tc::idesc_bf16(128, D2S, false, G_MN);
-      const uint32_t aRing = tc::smem_u32(ring), aE = tc::smem_u32(sE), aY = tc::smem_u32(sY);
+      const uint32_t aRing = tc::smem_u32(ring), aY = tc::smem_u32(sY);
       uint32_t it = 0;
-      auto wait_full = [&]() -> bool {
-        return tc::mbar_wait(&bar[BB_FULL0 + (it & 1)], (it >> 1) & 1, abort_flag);
+      // wait for the next ring entry; returns its shared address (0 on timeout)
+      auto next_stage = [&]() -> uint32_t {
+        const uint32_t st = it % ST;
+        if (!tc::mbar_wait(&bar[BB_FULL0 + st], (it / ST) & 1, abort_flag)) return 0u;
+        tc::tc_fence_after();
+        return aRing + st * Cfg::STAGE_BYTES;
+      };
+      auto release = [&]() {
+        tc::tc_commit(&bar[BB_EMPTY0 + (it % ST)]);
+        ++it;
       };
       if (has_inter) {
         for (int kb = 0; kb < Cfg::NKB && ok; ++kb) {
-          ok = wait_full();
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t st = aRing + (it & 1) * Cfg::STAGE_BYTES;
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t st = next_stage();
+            if (!st) { ok = false; break; }
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t a = tc::sdesc_sw128(st + k * 32, 16, 1024);
-            uint64_t ghi, glo;
-            if (G_MN) {
-              ghi = tc::sdesc_sw128(st + Cfg::SLOT + k * 2048, 8192, 1024);
-              glo = tc::sdesc_sw128(st + 2 * Cfg::SLOT + k * 2048, 8192, 1024);
-            } else {
-              ghi = tc::sdesc_sw128(st + Cfg::SLOT + k * 32, 16, 1024);
-              glo = tc::sdesc_sw128(st + 2 * Cfg::SLOT + k * 32, 16, 1024);
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t a = tc::sdesc_sw128(st + k * 32, 16, 1024);
+              const uint64_t g = G_MN ? tc::sdesc_sw128(st + Cfg::SLOT + k * 2048, 8192, 1024)
+                                      : tc::sdesc_sw128(st + Cfg::SLOT + k * 32, 16, 1024);
+              tc::mma_bf16_ss(tAcc, a, g, idG, (kb > 0 || half > 0 || k > 0));
             }
-            tc::mma_bf16_ss(tAcc, a, ghi, idG, (kb > 0 || k > 0));
-            tc::mma_bf16_ss(tAcc, a, glo, idG, 1);
+            release();
           }
-          tc::tc_commit(&bar[BB_EMPTY0 + (it & 1)]);
-          ++it;
         }
         tc::tc_commit(&bar[BB_INTER]);
       }
       auto issue_score = [&](int jj) -> bool {
-        const uint32_t tX = tX0 + (jj & 1) * 128;
+        const uint32_t tX = tX0 + (jj % NXBUF) * 128;
         for (int kb = 0; kb < Cfg::NKB; ++kb) {
-          if (!wait_full()) return false;
-          tc::tc_fence_after();
-          const uint32_t st = aRing + (it & 1) * Cfg::STAGE_BYTES;
+          const uint32_t st = next_stage();
+          if (!st) return false;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc::mma_bf16_ss(tX, tc::sdesc_sw128(st + k * 32, 16, 1024),
                             tc::sdesc_sw128(st + Cfg::SLOT + k * 32, 16, 1024), idX, (kb > 0 || k > 0));
-          tc::tc_commit(&bar[BB_EMPTY0 + (it & 1)]);
-          ++it;
+          release();
         }
-        tc::tc_commit(&bar[BB_X0 + (jj & 1)]);
+        tc::tc_commit(&bar[BB_X0 + (jj % NXBUF)]);
         return true;
       };
       if (ok) ok = issue_score(0);
       for (int jj = 0; jj < np && ok; ++jj) {
-        // the other X buffer was last read by the transform of jj - 1, awaited below
-        if (jj + 1 < np) ok = issue_score(jj + 1);
-        if (!ok) break;
-        ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag) &&
-             tc::mbar_wait(&bar[BB_EFULL], jj & 1, abort_flag);
+        // one X buffer: the next score waits until the transform has read this one;
+        // two buffers: the other one was released by the transform of jj - 1
+        if (NXBUF == 1) ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag);
+        if (ok && jj + 1 < np) ok = issue_score(jj + 1);
+        if (ok && NXBUF != 1) ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag);
         if (ok && jj == 0 && has_inter) ok = tc::mbar_wait(&bar[BB_ACC], 0, abort_flag);
         if (!ok) break;
-        tc::tc_fence_after();
+        const uint32_t st = next_stage();  // E(jj)
+        if (!st) { ok = false; break; }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t offy = (k >> 2) * Cfg::SLOT + (k & 3) * 32;
           tc::mma_bf16_ss(tAcc, tc::sdesc_sw128(aY + offy, 16, 1024),
-                          tc::sdesc_sw128(aE + k * 2048, Cfg::SLOT, 1024), idAcc,
+                          tc::sdesc_sw128(st + k * 2048, Cfg::SLOT, 1024), idAcc,
                           (has_inter || jj > 0 || k > 0));
         }
+        release();
         tc::tc_commit(&bar[BB_YE]);
       }
       tc::tc_commit(&bar[BB_DONE]);
@@ -342,14 +355,14 @@ __global__ void __launch_bounds__(192, 1) intra_bwd_tc_kernel(
     }
 
     for (int jj = 0; jj < np && ok; ++jj) {
-      ok = __all_sync(full, tc::mbar_wait(&bar[BB_X0 + (jj & 1)], (jj >> 1) & 1, abort_flag));
+      ok = __all_sync(full, tc::mbar_wait(&bar[BB_X0 + (jj % NXBUF)], (jj / NXBUF) & 1, abort_flag));
       if (ok && jj > 0) ok = __all_sync(full, tc::mbar_wait(&bar[BB_YE], (jj - 1) & 1, abort_flag));
       if (!ok) break;
       tc::tc_fence_after();
       const bool diag = (pj0 + jj) == it_tile;
       const float* pc = pfC + jj * 128;
       const float* pe = pfE + jj * 128;
-      const uint32_t tX = tX0 + (jj & 1) * 128;
+      const uint32_t tX = tX0 + (jj % NXBUF) * 128;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         float x[32];
@@ -446,9 +459,9 @@ bool intra_bwd_tc_supported(const Problem& p) {
          (p.dhv == 64 || p.dhv == 128 || p.dhv == 256 || p.dhv == 512);
 }
 
-template <int KIND, int D1, int D2S, bool G_MN, bool EXPV>
+template <int KIND, int D1, int D2S, bool G_MN, bool EXPV, int NXBUF>
 static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t s) {
-  using Cfg = BwdTcCfg<D1, D2S, G_MN>;
+  using Cfg = BwdTcCfg<D1, D2S, G_MN, NXBUF>;
   const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
   const bf16* C = (const bf16*)a.C;
   const bf16* dC = (const bf16*)a.dC;
@@ -487,7 +500,7 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   P.scale = p.scale;
   P.log2_scale = log2f(p.scale);
   const size_t smem = Cfg::smem_bytes(p.L);
-  auto kern = intra_bwd_tc_kernel<KIND, D1, D2S, G_MN, EXPV>;
+  auto kern = intra_bwd_tc_kernel<KIND, D1, D2S, G_MN, EXPV, NXBUF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(p.BH * p.NC * P.ntq), (unsigned)(P.d_out / D2S)), block(192);
@@ -501,9 +514,14 @@ static cudaError_t dispatch_kind(const Problem& p, const BwdArgs& a, cudaStream_
   const int d1 = (KIND == KDV) ? p.dqk : p.dhv;
   const int dout = (KIND == KDV) ? p.dhv : p.dqk;
   const bool wide = dout >= 128;
-#define MLSTM_BWD_TC_D1(D1)                                                                \
-  if (d1 == D1) return wide ? launch_kind<KIND, D1, 128, GMN, EXPV>(p, a, s)               \
-                            : launch_kind<KIND, D1, 64, GMN, EXPV>(p, a, s);
+#define MLSTM_BWD_TC_D1(D1)                                                                  \
+  if (d1 == D1) {                                                                            \
+    if (p.L == 128)                                                                          \
+      return wide ? launch_kind<KIND, D1, 128, GMN, EXPV, 1>(p, a, s)                        \
+                  : launch_kind<KIND, D1, 64, GMN, EXPV, 1>(p, a, s);                        \
+    return wide ? launch_kind<KIND, D1, 128, GMN, EXPV, 2>(p, a, s)                          \
+                : launch_kind<KIND, D1, 64, GMN, EXPV, 2>(p, a, s);                          \
+  }
   MLSTM_BWD_TC_D1(64)
   MLSTM_BWD_TC_D1(128)
   MLSTM_BWD_TC_D1(256)

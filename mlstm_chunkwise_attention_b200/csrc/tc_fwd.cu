@@ -29,7 +29,10 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int DQK, int DV>
+// ALIAS (chunk 128, one key tile per query tile): P is written into the K
+// buffer once S is done and C is loaded into the V buffer once PV is done, so
+// the CTA needs 96 KB of shared memory (at d 128) and two CTAs fit on an SM.
+template <int DQK, int DV, bool ALIAS = false>
 struct OutTcCfg {
   static constexpr int BM = 128, BN = 128;
   static constexpr int KB = DQK / 64;  // 64-column blocks of Q and K
@@ -37,13 +40,16 @@ struct OutTcCfg {
   static constexpr int Q_BYTES = KB * 16384;
   static constexpr int K_BYTES = KB * 16384;
   static constexpr int C_BYTES = VB * DQK * 128;
-  static constexpr int KC_BYTES = K_BYTES > C_BYTES ? K_BYTES : C_BYTES;
-  static constexpr int V_BYTES = VB * 16384;
-  static constexpr int P_BYTES = 2 * 16384;
+  static constexpr int P_TILE = 2 * 16384;
+  static constexpr int KC_BYTES = ALIAS ? (K_BYTES > P_TILE ? K_BYTES : P_TILE)
+                                        : (K_BYTES > C_BYTES ? K_BYTES : C_BYTES);
+  static constexpr int V_BYTES = VB * 16384;  // one V tile: the bytes its TMA loads deliver
+  static constexpr int V_REGION = ALIAS ? (V_BYTES > C_BYTES ? V_BYTES : C_BYTES) : V_BYTES;
+  static constexpr int P_BYTES = ALIAS ? 0 : 2 * 16384;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KC = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_KC + KC_BYTES;
-  static constexpr int OFF_P = OFF_V + V_BYTES;
+  static constexpr int OFF_P = OFF_V + V_REGION;
   static constexpr int OFF_BAR = OFF_P + P_BYTES;  // 16 mbarriers
   static constexpr int OFF_TMEM = OFF_BAR + 16 * 8;
   static constexpr int OFF_NVEC = OFF_TMEM + 16;
@@ -56,14 +62,14 @@ enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_COUNT };
 
 }  // namespace
 
-template <int DQK, int DV, bool EXPV>
-__global__ void __launch_bounds__(192, 1) output_fwd_tc_kernel(
+template <int DQK, int DV, bool EXPV, bool ALIAS>
+__global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
     const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
     const float* __restrict__ gn, bf16* __restrict__ h, float* __restrict__ abar_out, int T, int L,
     int NC, int BH, int ntq, int dhv, float scale, float log2_scale) {
-  using Cfg = OutTcCfg<DQK, DV>;
+  using Cfg = OutTcCfg<DQK, DV, ALIAS>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN;
 
   const int per = BH * NC;
@@ -85,7 +91,8 @@ __global__ void __launch_bounds__(192, 1) output_fwd_tc_kernel(
   uint8_t* sQ = smem + Cfg::OFF_Q;
   uint8_t* sKC = smem + Cfg::OFF_KC;
   uint8_t* sV = smem + Cfg::OFF_V;
-  uint8_t* sP = smem + Cfg::OFF_P;
+  uint8_t* sP = ALIAS ? smem + Cfg::OFF_KC : smem + Cfg::OFF_P;   // P tile
+  uint8_t* sC = ALIAS ? smem + Cfg::OFF_V : smem + Cfg::OFF_KC;    // C_prev tile
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
   float* nvec = reinterpret_cast<float*>(smem + Cfg::OFF_NVEC);
@@ -141,11 +148,13 @@ __global__ void __launch_bounds__(192, 1) output_fwd_tc_kernel(
           tc::tma_load_3d(sV + vb * 16384, &tm_v, &bar[B_V], dv0 + vb * 64, c0 + j * BN, bh);
       }
       if (ok && c > 0) {
-        ok = tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, &g_tc_fwd_error);  // last S done: reuse the K buffer
+        // C goes where K was once the last S is done, or (ALIAS) where V was once PV is done
+        ok = ALIAS ? tc::mbar_wait(&bar[B_PV], (nkv - 1) & 1, &g_tc_fwd_error)
+                   : tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, &g_tc_fwd_error);
         if (ok) {
           tc::mbar_arrive_expect_tx(&bar[B_C], Cfg::C_BYTES);
           for (int vb = 0; vb < Cfg::VB; ++vb)
-            tc::tma_load_3d(sKC + vb * DQK * 128, &tm_c, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
+            tc::tma_load_3d(sC + vb * DQK * 128, &tm_c, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
         }
       }
       // do not leave while a copy this thread issued may still be landing
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(192, 1) output_fwd_tc_kernel(
       constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(BM, DV, false, true);
       const uint32_t aQ = tc::smem_u32(sQ), aKC = tc::smem_u32(sKC), aV = tc::smem_u32(sV),
-                     aP = tc::smem_u32(sP);
+                     aP = tc::smem_u32(sP), aC = tc::smem_u32(sC);
       ok = tc::mbar_wait(&bar[B_Q], 0, &g_tc_fwd_error);
       for (int j = 0; j < nkv && ok; ++j) {
         ok = tc::mbar_wait(&bar[B_K], j & 1, &g_tc_fwd_error);
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(192, 1) output_fwd_tc_kernel(
           for (int k = 0; k < DQK / 16; ++k) {
             const uint32_t offq = (k >> 2) * 16384 + (k & 3) * 32;
             tc::mma_bf16_ss(tO, tc::sdesc_sw128(aQ + offq, 16, 1024),
-                            tc::sdesc_sw128(aKC + k * 2048, DQK * 128, 1024), idO, 1);
+                            tc::sdesc_sw128(aC + k * 2048, DQK * 128, 1024), idO, 1);
           }
         }
       }
@@ -332,9 +341,9 @@ bool output_fwd_tc_supported(const Problem& p) {
          (p.dhv % 64 == 0);
 }
 
-template <int DQK, int DV, bool EXPV>
+template <int DQK, int DV, bool EXPV, bool ALIAS>
 static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
-  using Cfg = OutTcCfg<DQK, DV>;
+  using Cfg = OutTcCfg<DQK, DV, ALIAS>;
   CUtensorMap tq, tk, tv, tcm;
   if (!make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tk, a.k, p.dqk, p.T, p.BH, 64, 128) ||
@@ -342,7 +351,7 @@ static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_
       !make_tmap_3d_bf16(&tcm, a.C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
     return cudaErrorInvalidValue;
   const size_t smem = Cfg::smem_bytes(p.L);
-  auto kern = output_fwd_tc_kernel<DQK, DV, EXPV>;
+  auto kern = output_fwd_tc_kernel<DQK, DV, EXPV, ALIAS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int ntq = p.L / 128;
@@ -354,8 +363,12 @@ static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_
 
 template <int DQK, bool EXPV>
 static cudaError_t launch_out_tc_dv(const Problem& p, const FwdArgs& a, cudaStream_t s) {
-  if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV>(p, a, s);
-  return launch_out_tc<DQK, 128, EXPV>(p, a, s);
+  if (p.L == 128) {
+    if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV, true>(p, a, s);
+    return launch_out_tc<DQK, 128, EXPV, true>(p, a, s);
+  }
+  if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV, false>(p, a, s);
+  return launch_out_tc<DQK, 128, EXPV, false>(p, a, s);
 }
 
 cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {

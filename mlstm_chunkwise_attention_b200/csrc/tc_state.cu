@@ -31,7 +31,7 @@ namespace {
 
 template <int NV>
 struct StateTcCfg {
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = 3;
   static constexpr int SUB = 64;                 // tokens per sub-tile (the MMA K extent)
   static constexpr int A_BYTES = 2 * 8192;       // 64 tokens x 128 state rows, two 64-row blocks
   static constexpr int B_BYTES = (NV / 64) * 8192;
@@ -46,10 +46,12 @@ struct StateTcCfg {
   static constexpr int NBAR = 16;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr size_t SMEM = 1024 + OFF_TMEM + 16;
-  static constexpr uint32_t TMEM_COLS = 256;     // U in [0, NV), normaliser column block at [NV, NV + 16)
+  // two U buffers: U_b in [128 b, 128 b + NV), its normaliser column block at
+  // [128 b + NV, 128 b + NV + 16); the MMA of chunk c+1 overlaps the epilogue of c
+  static constexpr uint32_t TMEM_COLS = 256;
 };
 
-enum { SB_FULL0 = 0, SB_SCALED0 = 2, SB_EMPTY0 = 4, SB_U = 6, SB_UFREE = 7, SB_COUNT = 8 };
+enum { SB_FULL0 = 0, SB_SCALED0 = 3, SB_EMPTY0 = 6, SB_U0 = 9, SB_UFREE0 = 11, SB_COUNT = 13 };
 
 }  // namespace
 
@@ -87,8 +89,8 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < SB_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == SB_SCALED0 || i == SB_SCALED0 + 1) cnt = 64;
-      if (i == SB_UFREE) cnt = 128;
+      if (i >= SB_SCALED0 && i < SB_SCALED0 + Cfg::STAGES) cnt = 64;
+      if (i == SB_UFREE0 || i == SB_UFREE0 + 1) cnt = 128;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tU = tmem, tN = tmem + NV;
+  const uint32_t tU0 = tmem;
   bool ok = true;
 
   auto chunk_of = [&](int u) { return BWD ? NC - 1 - u : u; };
@@ -147,7 +149,10 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
       uint32_t it = 0;
       for (int u = 0; u < nsteps && ok; ++u) {
         const int c = chunk_of(u), c0 = c * P.L, len = min(P.L, P.T - c0);
-        if (u > 0) ok = tc::mbar_wait(&bar[SB_UFREE], (u - 1) & 1, abort_flag);  // U read out
+        const int ub = u & 1;
+        const uint32_t tU = tU0 + ub * 128, tN = tU + NV;
+        // buffer ub was last read by the epilogue of step u - 2
+        ok = tc::mbar_wait(&bar[SB_UFREE0 + ub], ((u >> 1) & 1) ^ 1, abort_flag);
         if (!ok) break;
         for (int q = 0; q * SUB < len; ++q, ++it) {
           const uint32_t st = it % Cfg::STAGES, ph = (it / Cfg::STAGES) & 1;
@@ -173,39 +178,49 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
           tc::tc_commit(&bar[SB_EMPTY0 + st]);
         }
         if (!ok) break;
-        tc::tc_commit(&bar[SB_U]);
+        tc::tc_commit(&bar[SB_U0 + ub]);
       }
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ scaling (one token row per thread)
+    // The weights of the next sub-tile are computed before this one is waited
+    // for, so their global loads overlap the TMA wait and the scaling work.
     const int r = threadIdx.x - 64;  // 0..63
-    uint32_t it = 0;
-    for (int u = 0; u < nsteps && ok; ++u) {
+    auto weights = [&](int u, int q, float& wv, float& wn) {
+      wv = 0.f;
+      wn = 0.f;
+      if (u >= nsteps) return;
       const int c = chunk_of(u), c0 = c * P.L, len = min(P.L, P.T - c0);
-      const size_t ct = tokh + c0;
-      float g = 0.f, mc = 0.f, mprev = 0.f;
+      const int s = q * SUB + r;
+      if (s >= len) return;
+      const size_t ct = tokh + c0, t = ct + s;
       if (!BWD) {
-        g = P.b[ct + len - 1];
-        mc = EXPV ? P.m[ct + len - 1] : 0.f;
+        const float g = P.b[ct + len - 1];
+        const float mc = EXPV ? P.m[ct + len - 1] : 0.f;
+        wv = expf(g - P.b[t] + P.li[t] - mc);
+        wn = wv;
       } else {
-        mprev = EXPV ? (c > 0 ? P.m[ct - 1] : -INFINITY) : 0.f;
+        const float mprev = EXPV ? (c > 0 ? P.m[ct - 1] : -INFINITY) : 0.f;
+        const float mt = EXPV ? P.m[t] : 0.f;
+        const float alpha = expf(P.b[t] + mprev - mt) * P.scale;
+        wv = alpha * (EXPV ? P.inv_den[t] : 1.f);
+        wn = EXPV ? alpha * P.da[t] : 0.f;
       }
-      for (int q = 0; q * SUB < len; ++q, ++it) {
+    };
+    auto nsub = [&](int u) {
+      const int c = chunk_of(u), len = min(P.L, P.T - c * P.L);
+      return (len + SUB - 1) / SUB;
+    };
+    uint32_t it = 0;
+    float wv_next, wn_next;
+    weights(0, 0, wv_next, wn_next);
+    for (int u = 0; u < nsteps && ok; ++u) {
+      const int ns = nsub(u);
+      for (int q = 0; q < ns; ++q, ++it) {
         const uint32_t st = it % Cfg::STAGES, ph = (it / Cfg::STAGES) & 1;
-        const int s = q * SUB + r;
-        float wv = 0.f, wn = 0.f;
-        if (s < len) {
-          const size_t t = ct + s;
-          if (!BWD) {
-            wv = expf(g - P.b[t] + P.li[t] - mc);
-            wn = wv;
-          } else {
-            const float mt = EXPV ? P.m[t] : 0.f;
-            const float alpha = expf(P.b[t] + mprev - mt) * P.scale;
-            wv = alpha * (EXPV ? P.inv_den[t] : 1.f);
-            wn = EXPV ? alpha * P.da[t] : 0.f;
-          }
-        }
+        const float wv = wv_next, wn = wn_next;
+        if (q + 1 < ns) weights(u, q + 1, wv_next, wn_next);
+        else weights(u + 1, 0, wv_next, wn_next);
         ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_FULL0 + st], ph, abort_flag));
         if (!ok) break;
         uint8_t* stg = smem + st * Cfg::STAGE_BYTES;
@@ -282,7 +297,9 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
       } else {
         beta = expf(g);
       }
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_U], u & 1, abort_flag));
+      const int ub = u & 1;
+      const uint32_t tU = tU0 + ub * 128, tN = tU + NV;
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_U0 + ub], (u >> 1) & 1, abort_flag));
       if (!ok) break;
       tc::tc_fence_after();
 #pragma unroll
@@ -298,7 +315,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         sn = fmaf(beta, sn, v[0]);
       }
       tc::tc_fence_before();
-      tc::mbar_arrive(&bar[SB_UFREE]);
+      tc::mbar_arrive(&bar[SB_UFREE0 + ub]);
     }
   }
 

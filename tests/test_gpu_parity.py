@@ -222,3 +222,45 @@ def test_full_headline_exp_b8h32_t4096_fwd_bwd():
 @pytest.mark.parametrize("var", [SIG, EXP])
 def test_full_training_b4h16_t8192_d256(var):
     _full("train_b4h16_t8192_d256_c256", variant=var, heads_fwd=2, heads_bwd=1)
+
+
+def test_full_long_context_sig_b1h8_t65536():
+    """T = 65536, d_qk 256, d_hv 512, chunk 1024: second-level tiling inside the chunk."""
+    _full("sig_long_b1h8_t65536_c1024", heads_fwd=1, heads_bwd=1)
+
+
+@pytest.mark.parametrize("var", [SIG, EXP])
+@pytest.mark.parametrize("L", [64, 128, 256, 512, 1024])
+def test_sweep_t16384_d128(var, L):
+    """Chunk-size sweep at T = 16384, d 128 (the sweep's per-head shape), whole heads."""
+    cpu = inputs(1, 4, 16384, 128, 128, seed=3000 + L + var, dtype=BF, ig_mean=0.0, fg_mean=3.0)
+    dev, h, saved = gpu_fwd(cpu, L, var)
+    g = gpu_bwd(dev, h, saved, L, var)
+    for hh in (0, 3):
+        x = head64(cpu, 0, hh)
+        assert relerr(np64(h[0, hh]), oracle_fwd_head(x, L, var)["h"]) <= 1e-2
+        li, lf = oracle.gate_logs(x["igate"], x["fgate"], var)
+        cb = oracle.chunkwise_backward(x["q"], x["k"], x["v"], li, lf, var, L, x["dh"])
+        di, df = oracle.preact_grads(cb["dlog_i"], cb["dlog_f"], x["igate"], x["fgate"], var)
+        ref_g = {"dq": cb["dq"], "dk": cb["dk"], "dv": cb["dv"], "digate_pre": di, "dfgate_pre": df}
+        floor = 1e-3 * max(np.max(np.abs(v)) for v in ref_g.values())
+        for key, val in ref_g.items():
+            err = relerr(np64(g[key][0, hh]), val, floor=floor)
+            assert err <= 1e-2, f"{key} L={L} head {hh}: {err:.3e}"
+
+
+def test_sweep_igate_bias_minus10():
+    """The -10 input-gate bias distribution at chunk 512."""
+    for var in (SIG, EXP):
+        cpu = inputs(1, 2, 8192, 128, 128, seed=3100 + var, dtype=BF, ig_mean=-10.0, fg_mean=3.0)
+        dev, h, saved = gpu_fwd(cpu, 512, var)
+        g = gpu_bwd(dev, h, saved, 512, var)
+        x = head64(cpu, 0, 1)
+        assert relerr(np64(h[0, 1]), oracle_fwd_head(x, 512, var)["h"]) <= 1e-2
+        li, lf = oracle.gate_logs(x["igate"], x["fgate"], var)
+        cb = oracle.chunkwise_backward(x["q"], x["k"], x["v"], li, lf, var, 512, x["dh"])
+        di, df = oracle.preact_grads(cb["dlog_i"], cb["dlog_f"], x["igate"], x["fgate"], var)
+        floor = 1e-3 * max(np.max(np.abs(v)) for v in (cb["dq"], cb["dk"], cb["dv"], di, df))
+        for key, val in (("dq", cb["dq"]), ("dk", cb["dk"]), ("dv", cb["dv"]),
+                         ("digate_pre", di), ("dfgate_pre", df)):
+            assert relerr(np64(g[key][0, 1]), val, floor=floor) <= 1e-2, key
