@@ -31,7 +31,7 @@ namespace {
 
 template <int NV>
 struct StateTcCfg {
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 2;
   static constexpr int SUB = 64;                 // tokens per sub-tile (the MMA K extent)
   static constexpr int A_BYTES = 2 * 8192;       // 64 tokens x 128 state rows, two 64-row blocks
   static constexpr int B_BYTES = (NV / 64) * 8192;
@@ -42,7 +42,11 @@ struct StateTcCfg {
   static constexpr int OFF_NHI = OFF_BLO + B_BYTES;
   static constexpr int OFF_NLO = OFF_NHI + BN_BYTES;
   static constexpr int STAGE_BYTES = OFF_NLO + BN_BYTES;
-  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  // staging tile of one chunk boundary for the TMA stores: hi then lo plane,
+  // each 128 rows x NV columns in the 128-byte-swizzled layout
+  static constexpr int OFF_STG = STAGES * STAGE_BYTES;
+  static constexpr int STG_PLANE = (NV / 64) * 16384;
+  static constexpr int OFF_BAR = OFF_STG + 2 * STG_PLANE;
   static constexpr int NBAR = 16;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr size_t SMEM = 1024 + OFF_TMEM + 16;
@@ -51,7 +55,10 @@ struct StateTcCfg {
   static constexpr uint32_t TMEM_COLS = 256;
 };
 
-enum { SB_FULL0 = 0, SB_SCALED0 = 3, SB_EMPTY0 = 6, SB_U0 = 9, SB_UFREE0 = 11, SB_COUNT = 13 };
+enum {
+  SB_FULL0 = 0, SB_SCALED0 = 3, SB_EMPTY0 = 6, SB_U0 = 9, SB_UFREE0 = 11, SB_STG_FULL = 13,
+  SB_STG_FREE = 14, SB_COUNT = 15
+};
 
 }  // namespace
 
@@ -67,6 +74,8 @@ struct StateTcParams {
 template <bool BWD, bool EXPV, int NV>
 __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                           const __grid_constant__ CUtensorMap tmB,
+                                                          const __grid_constant__ CUtensorMap tmOhi,
+                                                          const __grid_constant__ CUtensorMap tmOlo,
                                                           const StateTcParams P) {
   using Cfg = StateTcCfg<NV>;
   constexpr int SUB = Cfg::SUB;
@@ -90,7 +99,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
     for (int i = 0; i < SB_COUNT; ++i) {
       uint32_t cnt = 1;
       if (i >= SB_SCALED0 && i < SB_SCALED0 + Cfg::STAGES) cnt = 64;
-      if (i == SB_UFREE0 || i == SB_UFREE0 + 1) cnt = 128;
+      if (i == SB_UFREE0 || i == SB_UFREE0 + 1 || i == SB_STG_FULL) cnt = 128;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -265,9 +274,13 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
     float sn = 0.f;
     for (int u = 0; u <= nsteps; ++u) {
       const int c = chunk_of(u);
-      // store the state at this chunk boundary
-      if (valid) {
-        const size_t row = (((size_t)bh * NC + c) * P.dqk + dk0 + i) * P.dhv + dv0;
+      // store the state at this chunk boundary: rows into the swizzled staging
+      // tile, then one TMA store per plane issued by thread 0 of the epilogue
+      if (u > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_STG_FREE], (u - 1) & 1, abort_flag));
+      if (!ok) break;
+      {
+        uint8_t* stg_hi = smem + Cfg::OFF_STG;
+        uint8_t* stg_lo = stg_hi + Cfg::STG_PLANE;
 #pragma unroll
         for (int j = 0; j < NV; j += 8) {
           uint4 vh, vl;
@@ -280,10 +293,29 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
             ph[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
             pl[e] = tc::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
           }
-          *reinterpret_cast<uint4*>(P.out + row + j) = vh;
-          *reinterpret_cast<uint4*>(P.out + P.plane + row + j) = vl;
+          const int blk = j >> 6, lc = (j & 63) >> 3;
+          const uint32_t off = blk * 16384 + i * 128 + ((lc ^ (i & 7)) << 4);
+          *reinterpret_cast<uint4*>(stg_hi + off) = vh;
+          *reinterpret_cast<uint4*>(stg_lo + off) = vl;
         }
-        if (with_n) P.nout[((size_t)bh * NC + c) * P.dqk + dk0 + i] = sn;
+        if (valid && with_n) P.nout[((size_t)bh * NC + c) * P.dqk + dk0 + i] = sn;
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bar[SB_STG_FULL]);
+        if (i == 0) {
+          ok = tc::mbar_wait(&bar[SB_STG_FULL], u & 1, abort_flag);
+          if (ok) {
+            const int z = bh * NC + c;
+            for (int blk = 0; blk < NV / 64; ++blk) {
+              tc::tma_store_3d(&tmOhi, stg_hi + blk * 16384, dv0 + blk * 64, dk0, z);
+              tc::tma_store_3d(&tmOlo, stg_lo + blk * 16384, dv0 + blk * 64, dk0, z);
+            }
+            tc::bulk_commit_group();
+            tc::bulk_wait_read_all();
+            tc::mbar_arrive(&bar[SB_STG_FREE]);
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
       }
       if (u == nsteps) break;
       const int c0 = c * P.L, len = min(P.L, P.T - c0);
@@ -319,6 +351,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
     }
   }
 
+  if (warp >= 4 && threadIdx.x == 128) tc::bulk_wait_all();  // this thread's TMA stores are done
   if (!ok) atomicOr(&g_tc_state_error, 1u);
   tc::tc_fence_before();
   __syncthreads();
@@ -342,10 +375,13 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
                                    float* nout, const float* b, const float* li, const float* m,
                                    const float* inv_den, const float* da, cudaStream_t s) {
   using Cfg = StateTcCfg<NV>;
-  CUtensorMap tA, tB;
-  const uint32_t dkbox = p.dqk >= 64 ? 64 : p.dqk;
-  if (!make_tmap_3d_bf16(&tA, A, p.dqk, p.T, p.BH, dkbox, 64) ||
-      !make_tmap_3d_bf16(&tB, B, p.dhv, p.T, p.BH, 64, 64))
+  CUtensorMap tA, tB, tOh, tOl;
+  const uint64_t plane = (uint64_t)p.BH * p.NC * p.dqk * p.dhv;
+  const uint64_t BHNC = (uint64_t)p.BH * p.NC;
+  if (!make_tmap_3d_bf16(&tA, A, p.dqk, p.T, p.BH, 64, 64) ||
+      !make_tmap_3d_bf16(&tB, B, p.dhv, p.T, p.BH, 64, 64) ||
+      !make_tmap_3d_bf16(&tOh, out, p.dhv, p.dqk, BHNC, 64, 128) ||
+      !make_tmap_3d_bf16(&tOl, out + plane, p.dhv, p.dqk, BHNC, 64, 128))
     return cudaErrorInvalidValue;
   StateTcParams P;
   P.b = b; P.li = li; P.m = m; P.inv_den = inv_den; P.da = da;
@@ -357,7 +393,7 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(p.dhv / NV), (unsigned)((p.dqk + 127) / 128), (unsigned)p.BH), block(256);
-  kern<<<grid, block, Cfg::SMEM, s>>>(tA, tB, P);
+  kern<<<grid, block, Cfg::SMEM, s>>>(tA, tB, tOh, tOl, P);
   return cudaGetLastError();
 }
 
