@@ -59,7 +59,7 @@ struct BwdTcCfg {
 };
 
 enum {
-  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_YE, BB_INTER, BB_ACC, BB_DONE, BB_COUNT
+  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_YE, BB_INTER, BB_ACC, BB_DONE, BB_STG, BB_COUNT
 };
 
 }  // namespace
@@ -78,7 +78,8 @@ template <int KIND, int D1, int D2S, bool G_MN, bool EXPV, int NXBUF>
 __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmGhi,
-    const __grid_constant__ CUtensorMap tmGlo, const BwdTcParams P) {
+    const __grid_constant__ CUtensorMap tmGlo, const __grid_constant__ CUtensorMap tmOut,
+    const BwdTcParams P) {
   using Cfg = BwdTcCfg<D1, D2S, G_MN, NXBUF>;
   constexpr bool R_IS_QUERY = (KIND == KDQ);
   constexpr int ST = Cfg::STAGES;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < BB_COUNT; ++i) {
-      const uint32_t cnt = (i == BB_Y || i == BB_ACC) ? 128u : 1u;
+      const uint32_t cnt = (i == BB_Y || i == BB_ACC || i == BB_STG) ? 128u : 1u;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -402,41 +403,51 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
 
     if (ok) ok = __all_sync(full, tc::mbar_wait(&bar[BB_DONE], 0, abort_flag));
     if (ok) {
+      // the result tile goes through the (now idle) Y tile and one TMA store per
+      // 64-column block; rows past the sequence end are clipped by the TMA unit
       tc::tc_fence_after();
       const float fin = (KIND == KDV) ? 1.f : P.scale;
-      bf16* orow = P.out + tok * P.d_out + col0;
       const bf16* drow = (KIND != KDV) ? P.dot_src + tok * P.dqk + col0 : nullptr;
       float dot = 0.f;
 #pragma unroll 1
       for (int ch = 0; ch < D2S / 32; ++ch) {
         float v[32];
         tc::tmem_ld32(tAcc + lane_base + ch * 32, v);
-        if (valid) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            float g[8];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float g[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = v[8 * q4 + e] * fin;
-            if (KIND != KDV) {
-              const uint4 src = *reinterpret_cast<const uint4*>(drow + ch * 32 + q4 * 8);
-              const uint32_t sw[4] = {src.x, src.y, src.z, src.w};
+          for (int e = 0; e < 8; ++e) g[e] = v[8 * q4 + e] * fin;
+          if (KIND != KDV && valid) {
+            const uint4 src = *reinterpret_cast<const uint4*>(drow + ch * 32 + q4 * 8);
+            const uint32_t sw[4] = {src.x, src.y, src.z, src.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&sw[e]);
-                dot = fmaf(__bfloat162float(s2.x), g[2 * e], dot);
-                dot = fmaf(__bfloat162float(s2.y), g[2 * e + 1], dot);
-              }
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&sw[e]);
+              dot = fmaf(__bfloat162float(s2.x), g[2 * e], dot);
+              dot = fmaf(__bfloat162float(s2.y), g[2 * e + 1], dot);
             }
-            uint4 w;
-            w.x = tc::pack_bf16(g[0], g[1]);
-            w.y = tc::pack_bf16(g[2], g[3]);
-            w.z = tc::pack_bf16(g[4], g[5]);
-            w.w = tc::pack_bf16(g[6], g[7]);
-            *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = w;
           }
+          const int col = ch * 32 + q4 * 8, blk = col >> 6, lc = (col & 63) >> 3;
+          const uint32_t addr = aY + blk * Cfg::SLOT + row * 128 + ((lc ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(tc::pack_bf16(g[0], g[1])), "r"(tc::pack_bf16(g[2], g[3])),
+                       "r"(tc::pack_bf16(g[4], g[5])), "r"(tc::pack_bf16(g[6], g[7]))
+                       : "memory");
         }
       }
       if (KIND != KDV && valid) atomicAdd(&P.pdot[tok], dot);
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[BB_STG]);
+      if (row == 0) {
+        ok = tc::mbar_wait(&bar[BB_STG], 0, abort_flag);
+        if (ok) {
+          for (int blk = 0; blk < Cfg::EB; ++blk)
+            tc::tma_store_3d(&tmOut, sY + blk * Cfg::SLOT, col0 + blk * 64, c0 + r0, bh);
+          tc::bulk_commit_group();
+          tc::bulk_wait_all();
+        }
+      }
     }
   }
 
@@ -465,7 +476,7 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
   const bf16* C = (const bf16*)a.C;
   const bf16* dC = (const bf16*)a.dC;
-  CUtensorMap tA, tB, tE, tGh, tGl;
+  CUtensorMap tA, tB, tE, tGh, tGl, tO;
   bool okm = true;
   const uint64_t BHNC = (uint64_t)p.BH * p.NC;
   if (KIND == KDQ) {
@@ -487,6 +498,11 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
     okm &= make_tmap_3d_bf16(&tGh, dC, p.dhv, p.dqk, BHNC, 64, 64);
     okm &= make_tmap_3d_bf16(&tGl, dC + plane, p.dhv, p.dqk, BHNC, 64, 64);
   }
+  {
+    void* outp = (KIND == KDQ) ? a.dq : (KIND == KDK) ? a.dk : a.dv;
+    const int dout = (KIND == KDV) ? p.dhv : p.dqk;
+    okm &= make_tmap_3d_bf16(&tO, outp, dout, p.T, p.BH, 64, 128);
+  }
   if (!okm) return cudaErrorInvalidValue;
   BwdTcParams P;
   P.b = a.b; P.li = a.li; P.m = a.m; P.inv_den = a.inv_den; P.da = a.da;
@@ -504,7 +520,7 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(p.BH * p.NC * P.ntq), (unsigned)(P.d_out / D2S)), block(192);
-  kern<<<grid, block, smem, s>>>(tA, tB, tE, tGh, tGl, P);
+  kern<<<grid, block, smem, s>>>(tA, tB, tE, tGh, tGl, tO, P);
   return cudaGetLastError();
 }
 

@@ -58,7 +58,7 @@ struct OutTcCfg {
   static size_t smem_bytes(int L) { return 1024 + OFF_COLF + (size_t)L * 4; }
 };
 
-enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_COUNT };
+enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_STG, B_COUNT };
 
 }  // namespace
 
@@ -66,7 +66,7 @@ template <int DQK, int DV, bool EXPV, bool ALIAS>
 __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-    const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
+    const __grid_constant__ CUtensorMap tm_h, const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
     const float* __restrict__ gn, bf16* __restrict__ h, float* __restrict__ abar_out, int T, int L,
     int NC, int BH, int ntq, int dhv, float scale, float log2_scale) {
   using Cfg = OutTcCfg<DQK, DV, ALIAS>;
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
-      const uint32_t cnt = (i == B_P || i == B_QS) ? 128u : 1u;
+      const uint32_t cnt = (i == B_P || i == B_QS || i == B_STG) ? 128u : 1u;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -302,21 +302,32 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
         inv = 1.f / fmaxf(fabsf(a), expf(-mt));
         if (blockIdx.y == 0 && valid) abar_out[tok] = a;
       }
-      bf16* hrow = h + tok * dhv + dv0;
+      // h goes through the (now idle) P tile and one TMA store per 64-column block
 #pragma unroll 1
       for (int ch = 0; ch < DV / 32; ++ch) {
         float ov[32];
         tc::tmem_ld32(tO + lane_base + ch * 32, ov);
-        if (valid) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 w;
-            w.x = tc::pack_bf16(ov[8 * q4 + 0] * inv, ov[8 * q4 + 1] * inv);
-            w.y = tc::pack_bf16(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv);
-            w.z = tc::pack_bf16(ov[8 * q4 + 4] * inv, ov[8 * q4 + 5] * inv);
-            w.w = tc::pack_bf16(ov[8 * q4 + 6] * inv, ov[8 * q4 + 7] * inv);
-            *reinterpret_cast<uint4*>(hrow + ch * 32 + q4 * 8) = w;
-          }
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int col = ch * 32 + q4 * 8, blk = col >> 6, lc = (col & 63) >> 3;
+          const uint32_t addr = aP + blk * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(tc::pack_bf16(ov[8 * q4 + 0] * inv, ov[8 * q4 + 1] * inv)),
+                       "r"(tc::pack_bf16(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv)),
+                       "r"(tc::pack_bf16(ov[8 * q4 + 4] * inv, ov[8 * q4 + 5] * inv)),
+                       "r"(tc::pack_bf16(ov[8 * q4 + 6] * inv, ov[8 * q4 + 7] * inv))
+                       : "memory");
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[B_STG]);
+      if (row == 0) {
+        ok = tc::mbar_wait(&bar[B_STG], 0, &g_tc_fwd_error);
+        if (ok) {
+          for (int blk = 0; blk < DV / 64; ++blk)
+            tc::tma_store_3d(&tm_h, sP + blk * 16384, dv0 + blk * 64, c0 + t0, bh);
+          tc::bulk_commit_group();
+          tc::bulk_wait_all();
         }
       }
     }
@@ -344,8 +355,9 @@ bool output_fwd_tc_supported(const Problem& p) {
 template <int DQK, int DV, bool EXPV, bool ALIAS>
 static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   using Cfg = OutTcCfg<DQK, DV, ALIAS>;
-  CUtensorMap tq, tk, tv, tcm;
-  if (!make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
+  CUtensorMap tq, tk, tv, tcm, th;
+  if (!make_tmap_3d_bf16(&th, a.h, p.dhv, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tk, a.k, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tv, a.v, p.dhv, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tcm, a.C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
@@ -356,7 +368,7 @@ static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_
   if (e != cudaSuccess) return e;
   const int ntq = p.L / 128;
   dim3 grid((unsigned)(p.BH * p.NC * ntq), (unsigned)(p.dhv / DV)), block(192);
-  kern<<<grid, block, smem, s>>>(tq, tk, tv, tcm, a.b, a.li, a.m, a.n, (bf16*)a.h, a.abar, p.T,
+  kern<<<grid, block, smem, s>>>(tq, tk, tv, tcm, th, a.b, a.li, a.m, a.n, (bf16*)a.h, a.abar, p.T,
                                  p.L, p.NC, p.BH, ntq, p.dhv, p.scale, log2f(p.scale));
   return cudaGetLastError();
 }
