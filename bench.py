@@ -262,6 +262,83 @@ def run_reference(args, spec):
     return 0
 
 
+def run_sweep(args):
+    """Forward chunk-size / sequence-length sweep at B8 H32 d128 (one JSON line per point).
+
+    Each point times mlstm_fwd with CUDA events over `--steps` calls (after
+    `--warmup`), per kernel through the library's timing hook; reports
+    forward TFLOP/s, tokens/s, and the output kernel's TFLOP/s as a share of
+    the measured dense bf16 peak.
+    """
+    import torch
+    from mlstm_chunkwise_attention_b200 import binding
+    from mlstm_chunkwise_attention_b200.synthetic import SWEEP_CHUNK, SWEEP_SEED, SWEEP_T, make_inputs
+    peaks = load_peaks()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    B, NH, d = 8, 32, 128
+    Ts = [int(t) for t in args.sweep_t.split(",")] if args.sweep_t else list(SWEEP_T)
+    Ls = [int(c) for c in args.sweep_chunk.split(",")] if args.sweep_chunk else list(SWEEP_CHUNK)
+    for T in Ts:
+        for (var, igm, label) in ((0, 0.0, "sig"), (1, 0.0, "exp"), (1, -10.0, "exp_igate_bias_m10")):
+            cpu = make_inputs(B, NH, T, d, d, seed=SWEEP_SEED, igate_mean=igm, fgate_mean=3.0,
+                              dtype=torch.bfloat16)
+            x = {k: v.to(dev) for k, v in cpu.items()}
+            del cpu
+            h = torch.empty_like(x["v"])
+            for L in Ls:
+                sizes = binding.problem_sizes(x["q"], x["v"], L, var)
+                saved = torch.empty(binding.mlstm_saved_size(*sizes), dtype=torch.uint8, device=dev)
+                nf = binding.mlstm_fwd_launch_count(*sizes)
+                names = [binding.mlstm_launch_name(0, i, *sizes) for i in range(nf)]
+                evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nf)] for _ in range(args.steps)]
+                for row in evs:
+                    for e in row:
+                        e.record(stream)
+                torch.cuda.synchronize(dev)
+                arrs = [(ctypes.c_void_p * (2 * nf))(*[e.cuda_event for e in row]) for row in evs]
+
+                def call(ev=None):
+                    if ev is not None:
+                        binding.mlstm_set_timing_events(ev, 2 * nf)
+                    st = binding.mlstm_fwd(x["q"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(),
+                                           x["igate"].data_ptr(), x["fgate"].data_ptr(), h.data_ptr(),
+                                           saved.data_ptr(), None, 0, *sizes, sh)
+                    binding.mlstm_set_timing_events(None, 0)
+                    if st != 0:
+                        raise binding.MLSTMError(st, "mlstm_fwd")
+
+                for _ in range(args.warmup):
+                    call()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize(dev)
+                e0.record(stream)
+                for i in range(args.steps):
+                    call(arrs[i])
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                binding.check_device()
+                ms = e0.elapsed_time(e1) / args.steps
+                kms = {n: sum(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs) / args.steps
+                       for i, n in enumerate(names)}
+                flops = B * NH * flops_fwd(T, d, d, L)
+                out_name = [n for n in names if n.startswith("output_fwd")][0]
+                out_fl = B * NH * kernel_costs(T, d, d, L, var == 1, 2)["output_fwd"][0]
+                print(json.dumps({
+                    "sweep": "fwd_b8h32_d128", "cell": label, "T": T, "chunk": L,
+                    "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": B * T / ms * 1e3,
+                    "kernel_ms": kms, "output_kernel": out_name,
+                    "output_tflops": out_fl / kms[out_name] / 1e9,
+                    "output_pct_bf16_peak": 100 * out_fl / kms[out_name] / 1e9 / peaks["bf16_tflops"],
+                }), flush=True)
+                del saved
+            del x, h
+            torch.cuda.empty_cache()
+    return 0
+
+
 def workload_config(spec, n):
     return {"workload": WORKLOAD, "cell": "mLSTMexp" if spec["variant"] == 1 else "mLSTMsig",
             "B": spec["B"], "NH": spec["NH"], "T": spec["T"], "d_qk": spec["d_qk"],
@@ -283,6 +360,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="forward chunk/sequence sweep at B8 H32 d128 instead of the headline step")
+    ap.add_argument("--sweep-t", default=None, help="comma list of T for --sweep")
+    ap.add_argument("--sweep-chunk", default=None, help="comma list of chunk sizes for --sweep")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (smaller captures for ncu; the default is the workload's B)")
     args = ap.parse_args()
@@ -296,6 +377,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, spec)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch
     import torch.distributed as dist
