@@ -37,6 +37,7 @@ KERNEL_SOURCES = {
     "state_bwd_simt": "simt_bwd.cu", "dq_simt": "simt_bwd.cu", "dk_simt": "simt_bwd.cu",
     "dv_simt": "simt_bwd.cu", "output_fwd_tc": "tc_fwd.cu", "dq_tc": "tc_bwd.cu",
     "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
+    "output_fwd_xl": "tc_fwd_xl.cu",
     "state_bwd_tc": "tc_state.cu",
 }
 
@@ -87,7 +88,7 @@ def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
     out = {}
     for role, v in c.items():
         out[role] = v
-        for impl in ("_simt", "_tc"):
+        for impl in ("_simt", "_tc", "_xl"):
             out[role + impl] = v
     return out
 
@@ -96,7 +97,7 @@ def kernel_bound(name):
     """Which roofline bounds a kernel of this implementation."""
     if name.endswith("_simt"):
         return "alu"
-    if name.endswith("_tc"):
+    if name.endswith("_tc") or name.endswith("_xl"):
         return "tensor"
     return "hbm"
 
@@ -277,11 +278,15 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
     sh = ctypes.c_void_p(stream.cuda_stream)
-    B, NH, d = 8, 32, 128
+    B, NH, d = args.sweep_batch, 32, 128
     Ts = [int(t) for t in args.sweep_t.split(",")] if args.sweep_t else list(SWEEP_T)
     Ls = [int(c) for c in args.sweep_chunk.split(",")] if args.sweep_chunk else list(SWEEP_CHUNK)
+    cells = ((0, 0.0, "sig"), (1, 0.0, "exp"), (1, -10.0, "exp_igate_bias_m10"))
+    if args.sweep_cells:
+        keep = args.sweep_cells.split(",")
+        cells = tuple(c for c in cells if c[2] in keep)
     for T in Ts:
-        for (var, igm, label) in ((0, 0.0, "sig"), (1, 0.0, "exp"), (1, -10.0, "exp_igate_bias_m10")):
+        for (var, igm, label) in cells:
             cpu = make_inputs(B, NH, T, d, d, seed=SWEEP_SEED, igate_mean=igm, fgate_mean=3.0,
                               dtype=torch.bfloat16)
             x = {k: v.to(dev) for k, v in cpu.items()}
@@ -327,7 +332,7 @@ def run_sweep(args):
                 out_name = [n for n in names if n.startswith("output_fwd")][0]
                 out_fl = B * NH * kernel_costs(T, d, d, L, var == 1, 2)["output_fwd"][0]
                 print(json.dumps({
-                    "sweep": "fwd_b8h32_d128", "cell": label, "T": T, "chunk": L,
+                    "sweep": f"fwd_b{B}h32_d128", "cell": label, "T": T, "chunk": L,
                     "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": B * T / ms * 1e3,
                     "kernel_ms": kms, "output_kernel": out_name,
                     "output_tflops": out_fl / kms[out_name] / 1e9,
@@ -364,6 +369,10 @@ def main():
                     help="forward chunk/sequence sweep at B8 H32 d128 instead of the headline step")
     ap.add_argument("--sweep-t", default=None, help="comma list of T for --sweep")
     ap.add_argument("--sweep-chunk", default=None, help="comma list of chunk sizes for --sweep")
+    ap.add_argument("--sweep-batch", type=int, default=8,
+                    help="B for --sweep (smaller for ncu captures; the sweep workload is B8)")
+    ap.add_argument("--sweep-cells", default=None,
+                    help="comma subset of sig,exp,exp_igate_bias_m10 for --sweep")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (smaller captures for ncu; the default is the workload's B)")
     args = ap.parse_args()

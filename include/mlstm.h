@@ -79,10 +79,17 @@ typedef enum {
  *            plane.  bf16 path: two bf16 planes back to back, hi = bf16(C)
  *            then lo = bf16(C - hi), so hi + lo keeps about 16 mantissa bits
  *            for the backward pass
- *   state_n  float [BH, NC, d_qk]  EXP: normaliser state entering each chunk */
+ *   state_n  float [BH, NC, d_qk]  EXP: normaliser state entering each chunk
+ *   tile_table  float [BH, NC, 5 chunk + max(32, chunk / 32)]  bf16 with
+ *            chunk >= 256 only: per-chunk gate factors of the large-chunk
+ *            output kernel (row exponents, inter-chunk row factors, the
+ *            normaliser floor exp(-m_t), key exponents, per-32-key column
+ *            factors and their block maxima).  Forward scratch; the backward
+ *            does not read it. */
 typedef struct {
-  size_t gate_b, gate_li, gate_m, norm, state_c, state_n;
-  size_t gate_b_bytes, gate_li_bytes, gate_m_bytes, norm_bytes, state_c_bytes, state_n_bytes;
+  size_t gate_b, gate_li, gate_m, norm, state_c, state_n, tile_table;
+  size_t gate_b_bytes, gate_li_bytes, gate_m_bytes, norm_bytes, state_c_bytes, state_n_bytes,
+      tile_table_bytes;
   size_t total;
 } mlstm_saved_layout_t;
 

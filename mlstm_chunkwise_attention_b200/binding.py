@@ -34,9 +34,9 @@ class MLSTMError(RuntimeError):
 
 class SavedLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
-        "gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n",
+        "gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n", "tile_table",
         "gate_b_bytes", "gate_li_bytes", "gate_m_bytes", "norm_bytes", "state_c_bytes",
-        "state_n_bytes", "total")]
+        "state_n_bytes", "tile_table_bytes", "total")]
 
 
 _SIZES = [ctypes.c_int] * 8  # B, NH, T, d_qk, d_hv, chunk, variant, dtype

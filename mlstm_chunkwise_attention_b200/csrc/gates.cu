@@ -19,10 +19,48 @@ namespace mlstm {
 // run of rows.  The chunk recurrence is an inclusive warp scan of the affine
 // max-plus maps x -> max(x + g_c, u_c).
 // ---------------------------------------------------------------------------
+// Per-chunk gate tables of the large-chunk output kernel (layout in
+// internal.h).  With R_t + CC_s = log2 D_ts / sqrt(d_qk) for s <= t, the decay
+// factor separates as exp2(R_t + MU_j) * KP_s over a block j of 32 keys that
+// lies wholly before row t; both factors are at most 1, because the max state
+// m_t bounds every b_t - b_s + log i_s with s <= t (SIG: log i <= 0, b falls).
+// One warp handles one block of 32 keys, so MU_j is a warp max.
+template <bool EXPV>
+__device__ void write_xl_tables(const float* b, const float* li, const float* m, float* xt,
+                                size_t base, int T, int L, int NC, float scale,
+                                float log2_scale) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int stride = xl_table_stride(L), bpc = L / 32;
+  for (int blk = warp; blk < NC * bpc; blk += nwarps) {
+    const int c = blk / bpc, r = (blk % bpc) * 32 + lane;
+    const int t = c * L + r;
+    const bool valid = t < T;
+    float R = -INFINITY, QF = 0.f, FL = 1.f, CC = -INFINITY;
+    if (valid) {
+      const float bt = b[base + t];
+      const float mt = EXPV ? m[base + t] : 0.f;
+      R = (bt - mt) * kLog2e + log2_scale;
+      if (c > 0) QF = expf(bt + (EXPV ? m[base + (size_t)c * L - 1] : 0.f) - mt) * scale;
+      if (EXPV) FL = expf(-mt);
+      CC = (li[base + t] - bt) * kLog2e;
+    }
+    const float mu = warp_max(CC);
+    float* tb = xt + ((size_t)blockIdx.x * NC + c) * (size_t)stride;
+    tb[r] = R;
+    tb[L + r] = QF;
+    tb[2 * L + r] = FL;
+    tb[3 * L + r] = CC;
+    tb[4 * L + r] = valid ? exp2f(CC - mu) : 0.f;
+    if (lane == 0) tb[5 * L + r / 32] = mu;
+  }
+}
+
 template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(256) gate_prep_kernel(
     const TIO* __restrict__ ig, const TIO* __restrict__ fg, float* __restrict__ b_out,
-    float* __restrict__ li_out, float* __restrict__ m_out, int T, int L, int NC) {
+    float* __restrict__ li_out, float* __restrict__ m_out, float* __restrict__ xt, int T, int L,
+    int NC, float scale, float log2_scale) {
   extern __shared__ float smem[];
   float* sg = smem;       // g_c  (chunk decay)
   float* su = smem + NC;  // u_c, then m_c
@@ -68,7 +106,13 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
       }
     }
   }
-  if (!EXPV) return;
+  if (!EXPV) {
+    if (xt != nullptr) {
+      __syncthreads();
+      write_xl_tables<false>(b_out, li_out, m_out, xt, base, T, L, NC, scale, log2_scale);
+    }
+    return;
+  }
   __syncthreads();
   if (warp == 0) {
     float carry = -INFINITY;
@@ -97,6 +141,10 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
     const size_t idx = base + t;
     m_out[idx] = b_out[idx] + fmaxf(mprev, m_out[idx]);
   }
+  if (xt != nullptr) {
+    __syncthreads();
+    write_xl_tables<true>(b_out, li_out, m_out, xt, base, T, L, NC, scale, log2_scale);
+  }
 }
 
 cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s) {
@@ -104,14 +152,14 @@ cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH), block(256);
   if (p.bf16()) {
     if (p.exp_variant())
-      gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+      gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
     else
-      gate_prep_kernel<bf16, false><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+      gate_prep_kernel<bf16, false><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
   } else {
     if (p.exp_variant())
-      gate_prep_kernel<float, true><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+      gate_prep_kernel<float, true><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
     else
-      gate_prep_kernel<float, false><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, p.T, p.L, p.NC);
+      gate_prep_kernel<float, false><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
   }
   return cudaGetLastError();
 }

@@ -23,7 +23,20 @@ struct FwdArgs {
   void* C;                   // [BH, NC, dqk, dhv] state entering each chunk (planes, see StatePlanes)
   float* n;                  // [BH, NC, dqk]
   bool keep_lo;              // write the low plane of bf16 states (needed by the backward)
+  float* xt;                 // per-chunk gate tables of the large-chunk output kernel, or null
 };
+
+// Per-chunk gate tables, [BH, NC, xl_table_stride(L)] floats, written by
+// gate_prep when FwdArgs::xt is set.  For token t (row) or s (key) of chunk c:
+//   R  [0, L)    (b_t - m_t) log2 e + log2(1/sqrt(d_qk))    (m_t = 0 for SIG)
+//   QF [L, 2L)   exp(b_t + m_{c-1} - m_t) / sqrt(d_qk)       (0 in the first chunk)
+//   FL [2L, 3L)  exp(-m_t) (EXP; 1 for SIG)
+//   CC [3L, 4L)  (log i_s - b_s) log2 e
+//   KP [4L, 5L)  exp2(CC_s - MU_{s/32})
+//   MU [5L, ..)  max of CC over each block of 32 keys
+// Past the end of the sequence: R = CC = MU = -inf, QF = KP = 0, FL = 1.
+// Every block of a chunk starts 16-byte aligned (L is a multiple of 128).
+__host__ __device__ inline int xl_table_stride(int L) { return 5 * L + (L / 32 > 32 ? L / 32 : 32); }
 
 // Device pointers of one backward call.
 struct BwdArgs {
@@ -59,6 +72,9 @@ bool make_tmap_3d_bf16(void* map, const void* base, uint64_t inner, uint64_t mid
 bool output_fwd_tc_supported(const Problem& p);
 cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_fwd_error(unsigned int* flag);
+bool output_fwd_xl_supported(const Problem& p);
+cudaError_t launch_output_fwd_xl(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t fetch_tc_fwd_xl_error(unsigned int* flag);
 bool intra_bwd_tc_supported(const Problem& p);
 cudaError_t launch_dq_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dk_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);

@@ -54,6 +54,9 @@ void saved_layout(const Problem& p, mlstm_saved_layout_t* L) {
   // bf16 path: hi and lo bf16 planes; fp32 path: one fp32 plane
   L->state_c_bytes = (size_t)p.BH * p.NC * p.dqk * p.dhv * (p.bf16() ? 2 * state_elem : state_elem);
   L->state_n_bytes = p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0;
+  L->tile_table_bytes = mlstm::output_fwd_xl_supported(p)
+                            ? (size_t)p.BH * p.NC * mlstm::xl_table_stride(p.L) * 4
+                            : 0;
   size_t off = 0;
   L->gate_b = off;  off = align256(off + L->gate_b_bytes);
   L->gate_li = off; off = align256(off + L->gate_li_bytes);
@@ -61,6 +64,7 @@ void saved_layout(const Problem& p, mlstm_saved_layout_t* L) {
   L->norm = off;    off = align256(off + L->norm_bytes);
   L->state_c = off; off = align256(off + L->state_c_bytes);
   L->state_n = off; off = align256(off + L->state_n_bytes);
+  L->tile_table = off; off = align256(off + L->tile_table_bytes);
   L->total = off;
 }
 
@@ -108,7 +112,9 @@ int fwd_plan(const Problem& p, FwdStep* st) {
     st[n++] = {"state_fwd_tc", mlstm::launch_state_fwd_tc};
   else
     st[n++] = {"state_fwd_simt", mlstm::launch_state_fwd_simt};
-  if (mlstm::output_fwd_tc_supported(p))
+  if (mlstm::output_fwd_xl_supported(p))
+    st[n++] = {"output_fwd_xl", mlstm::launch_output_fwd_xl};
+  else if (mlstm::output_fwd_tc_supported(p))
     st[n++] = {"output_fwd_tc", mlstm::launch_output_fwd_tc};
   else
     st[n++] = {"output_fwd_simt", mlstm::launch_output_fwd_simt};
@@ -253,6 +259,7 @@ int mlstm_fwd(const void* q, const void* k, const void* v, const void* igate_pre
   a.C = base + L.state_c;
   a.n = p.exp_variant() ? (float*)(base + L.state_n) : nullptr;
   a.keep_lo = saved != nullptr;
+  a.xt = L.tile_table_bytes ? (float*)(base + L.tile_table) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_fwd");
@@ -325,14 +332,16 @@ const char* mlstm_last_error(void) { return g_last_error; }
 int mlstm_device_status(void* stream) {
   int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
   if (st != MLSTM_OK) return st;
-  unsigned int flag = 0, flag_bwd = 0, flag_state = 0;
+  unsigned int flag = 0, flag_bwd = 0, flag_state = 0, flag_xl = 0;
   st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_bwd_error(&flag_bwd), "device error flag");
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_state_error(&flag_state), "device error flag");
   if (st != MLSTM_OK) return st;
-  flag |= flag_bwd | flag_state;
+  st = cuda_status(mlstm::fetch_tc_fwd_xl_error(&flag_xl), "device error flag");
+  if (st != MLSTM_OK) return st;
+  flag |= flag_bwd | flag_state | flag_xl;
   if (flag) {
     snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
     return MLSTM_ERR_TIMEOUT;

@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   const int nt_len = (len + 127) / 128;  // tiles holding rows of this chunk
   const int r0 = it_tile * 128;
   if (r0 >= len) return;
-  if (*(volatile unsigned int*)&g_tc_bwd_error != 0u) return;
+  // an earlier CTA gave up: the whole block leaves together
+  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_bwd_error != 0u)) return;
   const int col0 = blockIdx.y * D2S;
   const size_t tok0 = (size_t)bh * P.T + c0;
   // partner tiles: dq: 0..it_tile; dk, dv: it_tile..nt_len-1

@@ -80,7 +80,8 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
   const int len = min(L, T - c0);
   const int t0 = qt * BM;
   if (t0 >= len) return;
-  if (*(volatile unsigned int*)&g_tc_fwd_error != 0u) return;  // an earlier CTA gave up
+  // an earlier CTA gave up: the whole block leaves together
+  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_fwd_error != 0u)) return;
   const int nkv = qt + 1;
   const int dv0 = blockIdx.y * DV;
   const size_t tok0 = (size_t)bh * T + c0;

@@ -1,0 +1,551 @@
+// TFLA intra-chunk output kernel for large chunks (chunk >= 256): the second
+// level of tiling walks 128-token key tiles inside the chunk ("Tiled Flash
+// Linear Attention: More Efficient Linear RNN and xLSTM Kernels", TFLA summary
+// page, Approach; arXiv abstract page, Abstract).  Same mathematics as the
+// chunk-128 kernel (tc_fwd.cu):
+//   S_j = Q K_j^T;  P_ts = S_ts D_ts / sqrt(d_qk),  D_ts = exp(b_t - b_s + log i_s - m_t) (s <= t)
+//   O  = (alpha_t Q / sqrt(d_qk)) C_prev + sum_j P_j V_j;   h_t = O_t / den_t.
+//
+// Organisation (one persistent CTA per SM, work items = (query tile, head,
+// chunk, value block), heaviest query tiles first):
+//  * warp 0 streams Q tiles (double-buffered) and, per step, one key/value
+//    stage (K_j, V_j and the key tile's gate factors) or the chunk's entering
+//    state C_prev through a two-stage ring, all by TMA / bulk copies;
+//  * warp 1 issues tcgen05.mma: S_{g+1} before P_g V_g, so the tensor core
+//    computes the next score tile while the gate transform runs;
+//  * warps 2-9 (two warpgroups, one per 64-key half of a tile) turn S into P
+//    in TMEM in place (bf16, two per column), and P V reads P straight from
+//    TMEM.  The inter-chunk term is one more step of the same kind: the
+//    transform writes alpha_t q_t / sqrt(d_qk) into the S buffer and the
+//    tensor core multiplies it by C_prev, so it lands in the same
+//    accumulator O;
+//  * O is double-buffered in TMEM; the epilogue of an item (normalise,
+//    store h) runs after the first step of the next item.
+// Gate factors come from per-chunk tables written by gate_prep: off-diagonal
+// 32-key blocks use the separable form exp2(R_t + MU) * KP_s (one exp per row
+// and block), the diagonal block of the diagonal tile the per-element
+// exp2(R_t + CC_s) with the causal mask, and blocks above the diagonal are 0.
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace mlstm {
+
+static __device__ unsigned int g_tc_fwd_xl_error;
+
+namespace {
+
+template <int DQK, int DV>
+struct XlCfg {
+  static constexpr int KB = DQK / 64, VB = DV / 64;
+  static constexpr int NQ = DQK <= 128 ? 2 : 1;  // Q buffers
+  static constexpr int NS = DQK <= 128 ? 2 : 1;  // ring stages
+  static constexpr int Q_BYTES = KB * 16384;
+  static constexpr int K_BYTES = KB * 16384;
+  static constexpr int V_BYTES = VB * 16384;
+  static constexpr int C_BYTES = VB * DQK * 128;
+  static constexpr int STAGE = K_BYTES + V_BYTES;
+  static constexpr int ROWAUX = 3 * 512 + DQK * 4;  // R, QF, FL of 128 rows; n_{c-1}
+  static constexpr int COLAUX = 1152;               // CC, KP of 128 keys; 4 block maxima
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
+  static constexpr int OFF_ROW = OFF_RING + NS * STAGE;
+  static constexpr int OFF_COL = OFF_ROW + NQ * ROWAUX;
+  static constexpr int OFF_XS = OFF_COL + NS * COLAUX;  // [2 O buffers][2 halves][128] floats
+  static constexpr int OFF_BAR = OFF_XS + 2 * 2 * 128 * 4;
+  static constexpr int OFF_TMEM = OFF_BAR + 24 * 8;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;         // S0 [0,128) S1 [128,256) O0, O1 from 256
+  static_assert(C_BYTES <= STAGE, "C_prev must fit one ring stage");
+  static_assert(NQ == 2 || NS == 1, "the S look-ahead needs a second Q buffer");
+  static_assert(256 + 2 * DV <= 512, "two O buffers must fit TMEM");
+};
+
+enum {
+  X_QF0 = 0,   // Q (+ row factors) full, per Q buffer
+  X_QE0 = 2,   // Q buffer free: MMA commit + 256 transform threads
+  X_KVF0 = 4,  // ring stage full
+  X_KVE0 = 6,  // ring stage free (MMA commit)
+  X_SF0 = 8,   // S buffer written (MMA commit), per S buffer
+  X_PF0 = 10,  // P half written (128 threads), [S buffer][half]
+  X_OF0 = 14,  // O complete (MMA commit), per O buffer
+  X_OE0 = 16,  // O read out (256 threads), per O buffer
+  X_XS0 = 18,  // normaliser partials exchanged (256 threads), per O buffer
+  X_COUNT = 20
+};
+
+constexpr int kXlThreads = 320;
+
+struct XlItem {
+  int qt, bh, c, vb, t0, len, nkv;
+  bool pseudo;  // the chunk has a C_prev step (c > 0)
+};
+
+__device__ __forceinline__ bool xl_item(int k, int BH, int NC, int NVB, int ntq, int T, int L,
+                                        XlItem& it) {
+  const int per = BH * NC * NVB;
+  it.qt = ntq - 1 - k / per;
+  int r = k % per;
+  it.vb = r % NVB;
+  r /= NVB;
+  it.c = r % NC;
+  it.bh = r / NC;
+  it.t0 = it.qt * 128;
+  it.len = min(L, T - it.c * L);
+  it.nkv = it.qt + 1;
+  it.pseudo = it.c > 0;
+  return it.t0 < it.len;
+}
+
+__device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB, int ntq, int T,
+                                       int L, XlItem& it) {
+  for (; k < total; k += gridDim.x)
+    if (xl_item(k, BH, NC, NVB, ntq, T, L, it)) return k;
+  return total;
+}
+
+}  // namespace
+
+template <int DQK, int DV, bool EXPV>
+__global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
+    const float* __restrict__ tab, const float* __restrict__ gn, bf16* __restrict__ hout,
+    float* __restrict__ abar_out, int T, int L, int NC, int BH, int NVB, int ntq, int total,
+    int tstride, int dhv) {
+  using Cfg = XlCfg<DQK, DV>;
+  constexpr int NQ = Cfg::NQ, NS = Cfg::NS;
+  // an earlier CTA gave up: the whole block leaves together
+  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_fwd_xl_error != 0u)) return;
+  const volatile unsigned int* abort_flag = &g_tc_fwd_xl_error;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
+  float* xs = reinterpret_cast<float*>(smem + Cfg::OFF_XS);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < X_COUNT; ++i) {
+      uint32_t cnt = 1;
+      if (i == X_QE0 || i == X_QE0 + 1) cnt = 257;
+      if (i >= X_PF0 && i < X_PF0 + 4) cnt = 128;
+      if (i >= X_OE0 && i < X_XS0 + 2) cnt = 256;
+      tc::mbar_init(&bar[i], cnt);
+    }
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      tc::prefetch_tmap(&tm_c);
+      int it = 0, g = 0;
+      for (int k = blockIdx.x; k < total && ok; k += gridDim.x) {
+        XlItem I;
+        if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
+        const int qb = it % NQ;
+        ok = tc::mbar_wait(&bar[X_QE0 + qb], ((it / NQ) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        const float* tb = tab + ((size_t)I.bh * NC + I.c) * tstride;
+        const bool nv = EXPV && I.pseudo;
+        uint64_t* qf = &bar[X_QF0 + qb];
+        tc::mbar_arrive_expect_tx(qf, Cfg::Q_BYTES + 1536 + (nv ? DQK * 4 : 0));
+        uint8_t* sq = smem + Cfg::OFF_Q + qb * Cfg::Q_BYTES;
+        for (int kb = 0; kb < Cfg::KB; ++kb)
+          tc::tma_load_3d(sq + kb * 16384, &tm_q, qf, kb * 64, I.c * L + I.t0, I.bh);
+        uint8_t* rp = smem + Cfg::OFF_ROW + qb * Cfg::ROWAUX;
+        tc::bulk_load(rp, tb + I.t0, 512, qf);
+        tc::bulk_load(rp + 512, tb + L + I.t0, 512, qf);
+        tc::bulk_load(rp + 1024, tb + 2 * L + I.t0, 512, qf);
+        if (nv) tc::bulk_load(rp + 1536, gn + ((size_t)I.bh * NC + I.c) * DQK, DQK * 4, qf);
+        const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
+        for (int s = 0; s < nsteps && ok; ++s, ++g) {
+          const int st = g % NS;
+          ok = tc::mbar_wait(&bar[X_KVE0 + st], ((g / NS) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          uint64_t* full = &bar[X_KVF0 + st];
+          uint8_t* stg = smem + Cfg::OFF_RING + st * Cfg::STAGE;
+          if (I.pseudo && s == 0) {
+            tc::mbar_arrive_expect_tx(full, Cfg::C_BYTES);
+            for (int v = 0; v < Cfg::VB; ++v)
+              tc::tma_load_3d(stg + v * DQK * 128, &tm_c, full, I.vb * DV + v * 64, 0, I.bh * NC + I.c);
+          } else {
+            const int j = s - (I.pseudo ? 1 : 0);
+            const int row0 = I.c * L + j * 128;
+            tc::mbar_arrive_expect_tx(full, Cfg::STAGE + 1040);
+            for (int kb = 0; kb < Cfg::KB; ++kb)
+              tc::tma_load_3d(stg + kb * 16384, &tm_k, full, kb * 64, row0, I.bh);
+            for (int v = 0; v < Cfg::VB; ++v)
+              tc::tma_load_3d(stg + Cfg::K_BYTES + v * 16384, &tm_v, full, I.vb * DV + v * 64, row0, I.bh);
+            uint8_t* cp = smem + Cfg::OFF_COL + st * Cfg::COLAUX;
+            tc::bulk_load(cp, tb + 3 * L + j * 128, 512, full);
+            tc::bulk_load(cp + 512, tb + 4 * L + j * 128, 512, full);
+            tc::bulk_load(cp + 1024, tb + 5 * L + j * 4, 16, full);
+          }
+        }
+        ++it;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idO = tc::idesc_bf16(128, DV, false, true);
+      const uint32_t aQ0 = tc::smem_u32(smem + Cfg::OFF_Q), aR0 = tc::smem_u32(smem + Cfg::OFF_RING);
+
+      // score step s of item I (its it-th item, global step g): S_j = Q K_j^T,
+      // or for the C_prev step only a commit, which tells the transform the S
+      // buffer's last reader (P V of step g - 2) is done
+      auto issue_s = [&](const XlItem& I, int it, int s, int g) -> bool {
+        const int sb = g & 1;
+        if (I.pseudo && s == 0) {
+          tc::tc_commit(&bar[X_SF0 + sb]);
+          return true;
+        }
+        const int qb = it % NQ, st = g % NS;
+        if (!tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag)) return false;
+        if (!tc::mbar_wait(&bar[X_KVF0 + st], (g / NS) & 1, abort_flag)) return false;
+        tc::tc_fence_after();
+        const uint32_t aQ = aQ0 + qb * Cfg::Q_BYTES, aK = aR0 + st * Cfg::STAGE;
+#pragma unroll
+        for (int k = 0; k < DQK / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          tc::mma_bf16_ss(tmem + sb * 128, tc::sdesc_sw128(aQ + off, 16, 1024),
+                          tc::sdesc_sw128(aK + off, 16, 1024), idS, k > 0);
+        }
+        tc::tc_commit(&bar[X_SF0 + sb]);
+        return true;
+      };
+      // accumulate step s into O: P_j V_j, or (alpha q / sqrt(d_qk)) C_prev,
+      // A read from the two P halves in TMEM
+      auto issue_pv = [&](const XlItem& I, int it, int s, int g) -> bool {
+        const int sb = g & 1, st = g % NS, ob = it & 1;
+        const uint32_t tO = tmem + 256 + ob * DV, tP = tmem + sb * 128;
+        if (s == 0 && !tc::mbar_wait(&bar[X_OE0 + ob], ((it >> 1) & 1) ^ 1, abort_flag)) return false;
+        const uint32_t aS = aR0 + st * Cfg::STAGE;
+        const bool pseudo = I.pseudo && s == 0;
+        for (int h = 0; h < 2; ++h) {
+          if (!tc::mbar_wait(&bar[X_PF0 + 2 * sb + h], (g >> 1) & 1, abort_flag)) return false;
+          tc::tc_fence_after();
+          if (pseudo) {
+#pragma unroll
+            for (int kk = 0; kk < DQK / 32; ++kk) {
+              const int k = h * (DQK / 32) + kk;  // 16 rows of C_prev
+              tc::mma_bf16_ts(tO, tP + 64 * h + 8 * kk,
+                              tc::sdesc_sw128(aS + k * 2048, DQK * 128, 1024), idO, k > 0);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int k = 4 * h + kk;  // 16 keys of the tile
+              tc::mma_bf16_ts(tO, tP + 64 * h + 8 * kk,
+                              tc::sdesc_sw128(aS + Cfg::K_BYTES + k * 2048, 16384, 1024), idO,
+                              (s > 0 || k > 0));
+            }
+          }
+        }
+        tc::tc_commit(&bar[X_KVE0 + st]);
+        return true;
+      };
+
+      XlItem I, N;
+      int k = xl_next(blockIdx.x, total, BH, NC, NVB, ntq, T, L, I);
+      int it = 0, g = 0;
+      if (k < total) ok = issue_s(I, 0, 0, 0);
+      while (k < total && ok) {
+        const int kn = xl_next(k + gridDim.x, total, BH, NC, NVB, ntq, T, L, N);
+        const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
+        for (int s = 0; s < nsteps && ok; ++s, ++g) {
+          const bool last = s + 1 == nsteps;
+          if (NS > 1) {
+            if (!last) ok = issue_s(I, it, s + 1, g + 1);
+            else if (kn < total) ok = issue_s(N, it + 1, 0, g + 1);
+            if (!ok) break;
+          }
+          ok = issue_pv(I, it, s, g);
+          if (!ok) break;
+          if (last) {
+            tc::tc_commit(&bar[X_QE0 + it % NQ]);
+            tc::tc_commit(&bar[X_OF0 + (it & 1)]);
+          }
+          if (NS == 1) {
+            if (!last) ok = issue_s(I, it, s + 1, g + 1);
+            else if (kn < total) ok = issue_s(N, it + 1, 0, g + 1);
+          }
+        }
+        ++it;
+        k = kn;
+        I = N;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ gate transform + epilogue
+    const int h = (warp - 2) >> 2;  // 64-key half of each tile this warpgroup owns
+    const int qr = warp & 3;        // TMEM lane quarter = 32-row block of the tile
+    const int row = 32 * qr + lane;
+    const uint32_t lb = (uint32_t)(32 * qr) << 16;
+    const unsigned full = 0xffffffffu;
+    int it = 0, g = 0;
+
+    // epilogue of one item: normalise O and store h
+    struct Pending {
+      int ob, par, vb, col0;
+      bool valid;
+      size_t tok;
+      float fl, part;
+    } pe{};
+    bool pend = false;
+    auto epilogue = [&](const Pending& e) -> bool {
+      float inv = 1.f;
+      if (EXPV) {
+        // den_t = max(|a_t|, exp(-m_t)), a_t the sum of both halves' shares
+        float* x = xs + e.ob * 256;
+        x[h * 128 + row] = e.part;
+        tc::mbar_arrive(&bar[X_XS0 + e.ob]);
+        if (!__all_sync(full, tc::mbar_wait(&bar[X_XS0 + e.ob], e.par, abort_flag))) return false;
+        const float a = e.part + x[(1 - h) * 128 + row];
+        inv = 1.f / fmaxf(fabsf(a), e.fl);
+        if (h == 0 && e.vb == 0 && e.valid) abar_out[e.tok] = a;
+      }
+      if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + e.ob], e.par, abort_flag))) return false;
+      tc::tc_fence_after();
+      const uint32_t tO = tmem + 256 + e.ob * DV + lb + h * (DV / 2);
+      uint4* dst = reinterpret_cast<uint4*>(hout + e.tok * (size_t)dhv + e.col0);
+#pragma unroll
+      for (int q = 0; q < DV / 64; ++q) {
+        uint32_t o[32];
+        tc::tmem_ld32_async(tO + 32 * q, o);
+        tc::tmem_wait_ld(o);
+        if (q == DV / 64 - 1) {
+          tc::tc_fence_before();
+          tc::mbar_arrive(&bar[X_OE0 + e.ob]);
+        }
+        if (e.valid) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            const uint32_t* r = &o[8 * c8];
+            uint4 w;
+            w.x = tc::pack_bf16(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
+            w.y = tc::pack_bf16(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
+            w.z = tc::pack_bf16(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
+            w.w = tc::pack_bf16(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
+            dst[4 * q + c8] = w;
+          }
+        }
+      }
+      return true;
+    };
+
+    for (int k = blockIdx.x; k < total && ok; k += gridDim.x) {
+      XlItem I;
+      if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
+      const int qb = it % NQ;
+      ok = __all_sync(full, tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag));
+      if (!ok) break;
+      const float* rp = reinterpret_cast<const float*>(smem + Cfg::OFF_ROW + qb * Cfg::ROWAUX);
+      const float R = rp[row], QFt = rp[128 + row], FLt = rp[256 + row];
+      uint64_t part2 = tc::f2_make(0.f, 0.f);  // EXP: this half's share of the normaliser
+      const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
+      for (int s = 0; s < nsteps && ok; ++s, ++g) {
+        const int sb = g & 1, st = g % NS;
+        ok = __all_sync(full, tc::mbar_wait(&bar[X_SF0 + sb], (g >> 1) & 1, abort_flag));
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint32_t tS = tmem + sb * 128 + lb + 64 * h;
+        if (I.pseudo && s == 0) {
+          // alpha_t q_t / sqrt(d_qk), this half's d_qk / 2 columns, into the S buffer
+          const uint8_t* sq = smem + Cfg::OFF_Q + qb * Cfg::Q_BYTES;
+          const float* nvec = rp + 384;
+          constexpr int NCH = DQK / 16;  // 16-byte chunks in half a row
+#pragma unroll
+          for (int grp = 0; grp < NCH / 4; ++grp) {  // 32 columns -> 16 TMEM columns
+            uint32_t w[16];
+#pragma unroll
+            for (int cq = 0; cq < 4; ++cq) {
+              const int ci = 4 * grp + cq;
+              const int gc = h * NCH + ci, kb = gc >> 3, lc = gc & 7;
+              const uint32_t addr = tc::smem_u32(sq) + kb * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
+              uint32_t q4[4];
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(q4[0]), "=r"(q4[1]), "=r"(q4[2]), "=r"(q4[3])
+                           : "r"(addr));
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&q4[e]);
+                const float x0 = __bfloat162float(v2.x) * QFt, x1 = __bfloat162float(v2.y) * QFt;
+                if (EXPV) {
+                  const float2 n2 = *reinterpret_cast<const float2*>(nvec + gc * 8 + 2 * e);
+                  part2 = tc::f2_add(part2, tc::f2_mul(tc::f2_make(x0, x1), tc::f2_make(n2.x, n2.y)));
+                }
+                w[cq * 4 + e] = tc::pack_bf16(x0, x1);
+              }
+            }
+            tc::tmem_st16_async(tS + 16 * grp, w);
+          }
+        } else {
+          const int j = s - (I.pseudo ? 1 : 0);
+          const bool diag = j == I.qt;
+          const float* cp = reinterpret_cast<const float*>(smem + Cfg::OFF_COL + st * Cfg::COLAUX);
+          uint32_t sa[32], sb2[32];
+          tc::tmem_ld32_async(tS, sa);
+          tc::tmem_ld32_async(tS + 32, sb2);
+          tc::tmem_wait_ld(sa);
+          tc::reg_fence(sb2);
+#pragma unroll
+          for (int cl = 0; cl < 2; ++cl) {
+            const int cc = 2 * h + cl;  // 32-key block of the tile
+            const uint32_t* sv = cl == 0 ? sa : sb2;
+            uint32_t w[16];
+            if (!diag || cc < qr) {
+              // the whole block lies before this row: separable factors
+              const float rho = tc::ex2(R + cp[256 + cc]);
+              const uint64_t rho2 = tc::f2_make(rho, rho);
+              const float* kp = cp + 128 + 32 * cc;
+#pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                const float4 k4 = *reinterpret_cast<const float4*>(kp + e);
+                const uint64_t p0 = tc::f2_mul(
+                    tc::f2_mul(tc::f2_make(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                               tc::f2_make(k4.x, k4.y)), rho2);
+                const uint64_t p1 = tc::f2_mul(
+                    tc::f2_mul(tc::f2_make(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
+                               tc::f2_make(k4.z, k4.w)), rho2);
+                if (EXPV) part2 = tc::f2_add(part2, tc::f2_add(p0, p1));
+                const float2 a0 = tc::f2_split(p0), a1 = tc::f2_split(p1);
+                w[e / 2] = tc::pack_bf16(a0.x, a0.y);
+                w[e / 2 + 1] = tc::pack_bf16(a1.x, a1.y);
+              }
+            } else if (cc == qr) {
+              // the block holding this row: per-element decay and causal mask
+              const float* ccv = cp + 32 * cc;
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float p[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  const int key = 32 * cc + e + u;
+                  p[u] = key <= row ? __uint_as_float(sv[e + u]) * tc::ex2(R + ccv[e + u]) : 0.f;
+                }
+                if (EXPV) part2 = tc::f2_add(part2, tc::f2_make(p[0], p[1]));
+                w[e / 2] = tc::pack_bf16(p[0], p[1]);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) w[e] = 0u;
+            }
+            tc::tmem_st16_async(tS + 16 * cl, w);
+          }
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bar[X_PF0 + 2 * sb + h]);
+        if (s == 0) {
+          tc::mbar_arrive(&bar[X_QE0 + qb]);
+          if (pend) {
+            ok = epilogue(pe);
+            pend = false;
+          }
+        }
+      }
+      if (!ok) break;
+      const float2 pf = tc::f2_split(part2);
+      pe.ob = it & 1;
+      pe.par = (it >> 1) & 1;
+      pe.vb = I.vb;
+      pe.col0 = I.vb * DV + h * (DV / 2);
+      pe.valid = I.t0 + row < I.len;
+      pe.tok = (size_t)I.bh * T + (size_t)I.c * L + I.t0 + row;
+      pe.fl = FLt;
+      pe.part = pf.x + pf.y;
+      pend = true;
+      ++it;
+    }
+    if (ok && pend) ok = epilogue(pe);
+  }
+
+  if (!ok) atomicOr(&g_tc_fwd_xl_error, 1u);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+template <int DQK, int DV, bool EXPV>
+static cudaError_t launch_out_xl(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  using Cfg = XlCfg<DQK, DV>;
+  if (a.xt == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv, tcm;
+  if (!make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tk, a.k, p.dqk, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tv, a.v, p.dhv, p.T, p.BH, 64, 128) ||
+      !make_tmap_3d_bf16(&tcm, a.C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
+    return cudaErrorInvalidValue;
+  // at least 120 KB, so no second CTA shares the SM (each holds all 512 TMEM columns)
+  const int smem = Cfg::SMEM > 120 * 1024 ? Cfg::SMEM : 120 * 1024;
+  auto kern = output_fwd_xl_kernel<DQK, DV, EXPV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int ntq = p.L / 128, nvb = p.dhv / DV;
+  const long long total = (long long)ntq * p.BH * p.NC * nvb;
+  if (total >= (1LL << 31)) return cudaErrorInvalidValue;
+  const int grid = (int)(total < nsm ? total : nsm);
+  kern<<<grid, kXlThreads, smem, s>>>(tq, tk, tv, tcm, a.xt, a.n, (bf16*)a.h, a.abar, p.T, p.L,
+                                      p.NC, p.BH, nvb, ntq, (int)total, xl_table_stride(p.L),
+                                      p.dhv);
+  return cudaGetLastError();
+}
+
+bool output_fwd_xl_supported(const Problem& p) {
+  return p.bf16() && p.L >= 256 && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
+         (p.dhv == 64 || p.dhv % 128 == 0);
+}
+
+cudaError_t launch_output_fwd_xl(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  const bool e = p.exp_variant();
+#define MLSTM_XL(DQK)                                                                       \
+  if (p.dqk == DQK) {                                                                       \
+    if (p.dhv == 64) return e ? launch_out_xl<DQK, 64, true>(p, a, s) : launch_out_xl<DQK, 64, false>(p, a, s); \
+    return e ? launch_out_xl<DQK, 128, true>(p, a, s) : launch_out_xl<DQK, 128, false>(p, a, s); \
+  }
+  MLSTM_XL(64)
+  MLSTM_XL(128)
+  MLSTM_XL(256)
+#undef MLSTM_XL
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t fetch_tc_fwd_xl_error(unsigned int* flag) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_fwd_xl_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_tc_fwd_xl_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace mlstm

@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
                                                           const StateTcParams P) {
   using Cfg = StateTcCfg<NV>;
   constexpr int SUB = Cfg::SUB;
-  if (*(volatile unsigned int*)&g_tc_state_error != 0u) return;
+  // an earlier CTA gave up: the whole block leaves together
+  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_state_error != 0u)) return;
   // value-column tiles vary fastest so the CTAs sharing one head's key rows run together
   const int dv0 = blockIdx.x * NV, dk0 = blockIdx.y * 128, bh = blockIdx.z;
   const bool with_n = EXPV && blockIdx.x == 0;

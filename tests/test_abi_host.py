@@ -93,10 +93,11 @@ def test_empty_problem_is_a_noop(lib):
         assert lib.mlstm_fwd_launch_count(*sizes(**kw)) == 0
 
 
-def test_saved_layout_regions(lib):
+@pytest.mark.parametrize("L", [128, 512])
+def test_saved_layout_regions(lib, L):
     for variant in (B.SIG, B.EXP):
         for dtype in (B.BF16, B.FP32):
-            Bn, NH, T, dqk, dhv, L = 2, 3, 300, 128, 256, 128
+            Bn, NH, T, dqk, dhv = 2, 3, 300, 128, 256
             lay = B.mlstm_saved_layout(Bn, NH, T, dqk, dhv, L, variant, dtype)
             NC = (T + L - 1) // L
             tok = Bn * NH * T
@@ -106,8 +107,14 @@ def test_saved_layout_regions(lib):
             # bf16: hi and lo bf16 planes; fp32: one fp32 plane
             assert lay["state_c_bytes"] == Bn * NH * NC * dqk * dhv * 4
             assert lay["state_n_bytes"] == (Bn * NH * NC * dqk * 4 if variant == B.EXP else 0)
+            # per-chunk gate tables of the large-chunk bf16 output kernel:
+            # 5 L floats + max(32, L / 32) block maxima per chunk
+            xl = dtype == B.BF16 and L >= 256
+            assert lay["tile_table_bytes"] == (Bn * NH * NC * (5 * L + max(32, L // 32)) * 4
+                                               if xl else 0)
             regions = sorted((lay[n], lay[n + "_bytes"]) for n in
-                             ("gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n"))
+                             ("gate_b", "gate_li", "gate_m", "norm", "state_c", "state_n",
+                              "tile_table"))
             end = 0
             for off, nb in regions:
                 assert off % 256 == 0 and off >= end

@@ -45,6 +45,8 @@ SMALL = [
     ("exp_fp32_t1", 1, 1, 1, 64, 64, 64, EXP, F32, -4.0, 3.0),
     ("sig_bf16_chunk4096_ragged", 1, 1, 4500, 64, 64, 4096, SIG, BF, 0.0, 3.0),
     ("exp_bf16_chunk1024", 1, 1, 2048, 128, 128, 1024, EXP, BF, 0.0, 3.0),
+    ("exp_bf16_dqk256_dhv64_chunk512_ragged", 1, 2, 1000, 256, 64, 512, EXP, BF, 0.0, 3.0),
+    ("sig_bf16_dqk64_dhv128_chunk256_ragged", 1, 2, 600, 64, 128, 256, SIG, BF, -2.0, 3.0),
     ("exp_fp32_dqk256", 1, 1, 384, 256, 64, 128, EXP, F32, 1.0, 2.0),
 ]
 
