@@ -7,10 +7,12 @@
 //   O  = (alpha_t Q / sqrt(d_qk)) C_prev + sum_j P_j V_j;   h_t = O_t / den_t.
 //
 // Organisation (one persistent CTA per SM, work items = (query tile, head,
-// chunk, value block), heaviest query tiles first):
-//  * warp 0 streams Q tiles (double-buffered) and, per step, one key/value
-//    stage (K_j, V_j and the key tile's gate factors) or the chunk's entering
-//    state C_prev through a two-stage ring, all by TMA / bulk copies;
+// chunk, value block), taken in balanced pairs of query tiles):
+//  * warp 0 streams Q tiles (double-buffered) and, per step, K_j or the
+//    chunk's entering state C_prev through a ring whose stages free as soon
+//    as their score product is done; warp 10 streams V_j with the key
+//    tile's gate factors through a second ring (TMA and bulk copies, no
+//    multicast);
 //  * warp 1 issues tcgen05.mma: S_{g+1} before P_g V_g, so the tensor core
 //    computes the next score tile while the gate transform runs;
 //  * warps 2-9 (two warpgroups, one per 64-key half of a tile) turn S into P
@@ -39,57 +41,73 @@ template <int DQK, int DV>
 struct XlCfg {
   static constexpr int KB = DQK / 64, VB = DV / 64;
   static constexpr int NQ = DQK <= 128 ? 2 : 1;  // Q buffers
-  static constexpr int NS = DQK <= 128 ? 2 : 1;  // ring stages
+  // K ring (K tiles, and C_prev for the inter-chunk step); V ring (V tiles,
+  // each with its key tile's gate factors)
+  static constexpr int NK = DQK == 64 ? 4 : (DQK == 128 ? 2 : 1);
+  static constexpr int NV = DQK == 64 ? (DV == 64 ? 4 : 3) : (DQK == 128 ? (DV == 64 ? 4 : 2) : 2);
+  // the next S is issued before the current P V when the next Q and K can be resident
+  static constexpr bool LOOK = NQ == 2 && NK >= 2;
   static constexpr int Q_BYTES = KB * 16384;
   static constexpr int K_BYTES = KB * 16384;
   static constexpr int V_BYTES = VB * 16384;
   static constexpr int C_BYTES = VB * DQK * 128;
-  static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int ROWAUX = 3 * 512 + DQK * 4;  // R, QF, FL of 128 rows; n_{c-1}
-  static constexpr int COLAUX = 1152;               // CC, KP of 128 keys; 4 block maxima
+  static constexpr int COLAUX = 1040;               // CC, KP of 128 keys; 4 block maxima
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
-  static constexpr int OFF_ROW = OFF_RING + NS * STAGE;
+  static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * K_BYTES;
+  static constexpr int OFF_ROW = OFF_V + NV * V_BYTES;
   static constexpr int OFF_COL = OFF_ROW + NQ * ROWAUX;
-  static constexpr int OFF_XS = OFF_COL + NS * COLAUX;  // [2 O buffers][2 halves][128] floats
+  static constexpr int OFF_XS = OFF_COL + NV * COLAUX;  // [2 O buffers][2 halves][128] floats
   static constexpr int OFF_BAR = OFF_XS + 2 * 2 * 128 * 4;
-  static constexpr int OFF_TMEM = OFF_BAR + 24 * 8;
+  static constexpr int OFF_TMEM = OFF_BAR + 64 * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;         // S0 [0,128) S1 [128,256) O0, O1 from 256
-  static_assert(C_BYTES <= STAGE, "C_prev must fit one ring stage");
-  static_assert(NQ == 2 || NS == 1, "the S look-ahead needs a second Q buffer");
+  static_assert(C_BYTES <= K_BYTES, "C_prev must fit one K stage");
+  static_assert(NK <= 4 && NV <= 8, "barrier slots");
   static_assert(256 + 2 * DV <= 512, "two O buffers must fit TMEM");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 enum {
   X_QF0 = 0,   // Q (+ row factors) full, per Q buffer
   X_QE0 = 2,   // Q buffer free: MMA commit + 256 transform threads
-  X_KVF0 = 4,  // ring stage full
-  X_KVE0 = 6,  // ring stage free (MMA commit)
-  X_SF0 = 8,   // S buffer written (MMA commit), per S buffer
-  X_PF0 = 10,  // P half written (128 threads), [S buffer][half]
-  X_OF0 = 14,  // O complete (MMA commit), per O buffer
-  X_OE0 = 16,  // O read out (256 threads), per O buffer
-  X_XS0 = 18,  // normaliser partials exchanged (256 threads), per O buffer
-  X_COUNT = 20
+  X_KF0 = 4,   // K stage full (K tile or C_prev)
+  X_KE0 = 8,   // K stage free (MMA commit after the S or inter-chunk product)
+  X_VF0 = 12,  // V stage full (V tile + its key tile's gate factors)
+  X_VE0 = 20,  // V stage free (MMA commit after P V)
+  X_SF0 = 28,  // S buffer written (MMA commit), per S buffer
+  X_PF0 = 30,  // P written (256 threads, each having seen its step's V / C_prev), per S buffer
+  X_OF0 = 34,  // O complete (MMA commit), per O buffer
+  X_OE0 = 36,  // O read out (256 threads), per O buffer
+  X_XS0 = 38,  // normaliser partials exchanged (256 threads), per O buffer
+  X_COUNT = 40
 };
 
-constexpr int kXlThreads = 320;
+constexpr int kXlThreads = 352;  // K producer, MMA, 8 transform warps, V producer
 
 struct XlItem {
   int qt, bh, c, vb, t0, len, nkv;
   bool pseudo;  // the chunk has a C_prev step (c > 0)
 };
 
+// Work items come in pairs: query tiles ntq-1-p and p of one (head, chunk,
+// value block), so every pair holds ntq + 1 key tiles and a static split of
+// pairs over the CTAs is balanced.  Pair index fastest varies the pair inside
+// a chunk, so the CTAs running at one time cover few chunks and their K / V
+// tiles stay in L2 for every query tile that reads them.  Item k is half k & 1
+// of pair k >> 1; a CTA walks pairs blockIdx.x, blockIdx.x + gridDim.x, ...
 __device__ __forceinline__ bool xl_item(int k, int BH, int NC, int NVB, int ntq, int T, int L,
                                         XlItem& it) {
-  const int per = BH * NC * NVB;
-  it.qt = ntq - 1 - k / per;
-  int r = k % per;
+  const int half_ntq = ntq >> 1;
+  int r = k >> 1;
+  const int pi = r % half_ntq;
+  r /= half_ntq;
   it.vb = r % NVB;
   r /= NVB;
   it.c = r % NC;
   it.bh = r / NC;
+  it.qt = (k & 1) ? pi : ntq - 1 - pi;
   it.t0 = it.qt * 128;
   it.len = min(L, T - it.c * L);
   it.nkv = it.qt + 1;
@@ -97,9 +115,12 @@ __device__ __forceinline__ bool xl_item(int k, int BH, int NC, int NVB, int ntq,
   return it.t0 < it.len;
 }
 
+__device__ __forceinline__ int xl_first() { return 2 * blockIdx.x; }
+__device__ __forceinline__ int xl_succ(int k) { return (k & 1) ? k + 2 * gridDim.x - 1 : k + 1; }
+
 __device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB, int ntq, int T,
                                        int L, XlItem& it) {
-  for (; k < total; k += gridDim.x)
+  for (; k < total; k = xl_succ(k))
     if (xl_item(k, BH, NC, NVB, ntq, T, L, it)) return k;
   return total;
 }
@@ -114,7 +135,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     float* __restrict__ abar_out, int T, int L, int NC, int BH, int NVB, int ntq, int total,
     int tstride, int dhv) {
   using Cfg = XlCfg<DQK, DV>;
-  constexpr int NQ = Cfg::NQ, NS = Cfg::NS;
+  constexpr int NQ = Cfg::NQ, NK = Cfg::NK, NV = Cfg::NV;
   // an earlier CTA gave up: the whole block leaves together
   if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_fwd_xl_error != 0u)) return;
   const volatile unsigned int* abort_flag = &g_tc_fwd_xl_error;
@@ -131,7 +152,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     for (int i = 0; i < X_COUNT; ++i) {
       uint32_t cnt = 1;
       if (i == X_QE0 || i == X_QE0 + 1) cnt = 257;
-      if (i >= X_PF0 && i < X_PF0 + 4) cnt = 128;
+      if (i >= X_PF0 && i < X_PF0 + 4) cnt = 256;
       if (i >= X_OE0 && i < X_XS0 + 2) cnt = 256;
       tc::mbar_init(&bar[i], cnt);
     }
@@ -148,142 +169,202 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
   bool ok = true;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tc::prefetch_tmap(&tm_q);
-      tc::prefetch_tmap(&tm_k);
-      tc::prefetch_tmap(&tm_v);
-      tc::prefetch_tmap(&tm_c);
+    // ------------------------------------------------------------ Q / K / C_prev producer
+    // The whole warp walks the schedule (warp-uniform values); lane 0 issues.
+    {
+      const unsigned full = 0xffffffffu;
+      const bool leader = lane == 0;
+      if (leader) {
+        tc::prefetch_tmap(&tm_q);
+        tc::prefetch_tmap(&tm_k);
+        tc::prefetch_tmap(&tm_c);
+      }
       int it = 0, g = 0;
-      for (int k = blockIdx.x; k < total && ok; k += gridDim.x) {
+      for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
         XlItem I;
         if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
         const int qb = it % NQ;
-        ok = tc::mbar_wait(&bar[X_QE0 + qb], ((it / NQ) & 1) ^ 1, abort_flag);
+        ok = __all_sync(full, tc::mbar_wait(&bar[X_QE0 + qb], ((it / NQ) & 1) ^ 1, abort_flag));
         if (!ok) break;
         const float* tb = tab + ((size_t)I.bh * NC + I.c) * tstride;
         const bool nv = EXPV && I.pseudo;
-        uint64_t* qf = &bar[X_QF0 + qb];
-        tc::mbar_arrive_expect_tx(qf, Cfg::Q_BYTES + 1536 + (nv ? DQK * 4 : 0));
-        uint8_t* sq = smem + Cfg::OFF_Q + qb * Cfg::Q_BYTES;
-        for (int kb = 0; kb < Cfg::KB; ++kb)
-          tc::tma_load_3d(sq + kb * 16384, &tm_q, qf, kb * 64, I.c * L + I.t0, I.bh);
-        uint8_t* rp = smem + Cfg::OFF_ROW + qb * Cfg::ROWAUX;
-        tc::bulk_load(rp, tb + I.t0, 512, qf);
-        tc::bulk_load(rp + 512, tb + L + I.t0, 512, qf);
-        tc::bulk_load(rp + 1024, tb + 2 * L + I.t0, 512, qf);
-        if (nv) tc::bulk_load(rp + 1536, gn + ((size_t)I.bh * NC + I.c) * DQK, DQK * 4, qf);
+        if (leader) {
+          uint64_t* qf = &bar[X_QF0 + qb];
+          tc::mbar_arrive_expect_tx(qf, Cfg::Q_BYTES + 1536 + (nv ? DQK * 4 : 0));
+          uint8_t* sq = smem + Cfg::OFF_Q + qb * Cfg::Q_BYTES;
+          for (int kb = 0; kb < Cfg::KB; ++kb)
+            tc::tma_load_3d(sq + kb * 16384, &tm_q, qf, kb * 64, I.c * L + I.t0, I.bh);
+          uint8_t* rp = smem + Cfg::OFF_ROW + qb * Cfg::ROWAUX;
+          tc::bulk_load(rp, tb + I.t0, 512, qf);
+          tc::bulk_load(rp + 512, tb + L + I.t0, 512, qf);
+          tc::bulk_load(rp + 1024, tb + 2 * L + I.t0, 512, qf);
+          if (nv) tc::bulk_load(rp + 1536, gn + ((size_t)I.bh * NC + I.c) * DQK, DQK * 4, qf);
+        }
         const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
         for (int s = 0; s < nsteps && ok; ++s, ++g) {
-          const int st = g % NS;
-          ok = tc::mbar_wait(&bar[X_KVE0 + st], ((g / NS) & 1) ^ 1, abort_flag);
+          const int kst = g % NK;
+          ok = __all_sync(full, tc::mbar_wait(&bar[X_KE0 + kst], ((g / NK) & 1) ^ 1, abort_flag));
           if (!ok) break;
-          uint64_t* full = &bar[X_KVF0 + st];
-          uint8_t* stg = smem + Cfg::OFF_RING + st * Cfg::STAGE;
+          uint64_t* kf = &bar[X_KF0 + kst];
+          uint8_t* ks = smem + Cfg::OFF_K + kst * Cfg::K_BYTES;
           if (I.pseudo && s == 0) {
-            tc::mbar_arrive_expect_tx(full, Cfg::C_BYTES);
-            for (int v = 0; v < Cfg::VB; ++v)
-              tc::tma_load_3d(stg + v * DQK * 128, &tm_c, full, I.vb * DV + v * 64, 0, I.bh * NC + I.c);
+            if (leader) {
+              tc::mbar_arrive_expect_tx(kf, Cfg::C_BYTES);
+              for (int v = 0; v < Cfg::VB; ++v)
+                tc::tma_load_3d(ks + v * DQK * 128, &tm_c, kf, I.vb * DV + v * 64, 0, I.bh * NC + I.c);
+            }
           } else {
             const int j = s - (I.pseudo ? 1 : 0);
-            const int row0 = I.c * L + j * 128;
-            tc::mbar_arrive_expect_tx(full, Cfg::STAGE + 1040);
-            for (int kb = 0; kb < Cfg::KB; ++kb)
-              tc::tma_load_3d(stg + kb * 16384, &tm_k, full, kb * 64, row0, I.bh);
-            for (int v = 0; v < Cfg::VB; ++v)
-              tc::tma_load_3d(stg + Cfg::K_BYTES + v * 16384, &tm_v, full, I.vb * DV + v * 64, row0, I.bh);
-            uint8_t* cp = smem + Cfg::OFF_COL + st * Cfg::COLAUX;
-            tc::bulk_load(cp, tb + 3 * L + j * 128, 512, full);
-            tc::bulk_load(cp + 512, tb + 4 * L + j * 128, 512, full);
-            tc::bulk_load(cp + 1024, tb + 5 * L + j * 4, 16, full);
+            if (leader) {
+              tc::mbar_arrive_expect_tx(kf, Cfg::K_BYTES);
+              for (int kb = 0; kb < Cfg::KB; ++kb)
+                tc::tma_load_3d(ks + kb * 16384, &tm_k, kf, kb * 64, I.c * L + j * 128, I.bh);
+            }
           }
         }
         ++it;
       }
     }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ V producer
+    // Per key tile the V tile and the tile's gate factors (CC, KP of its 128
+    // keys and the four 32-key block maxima).
+    {
+      const unsigned full = 0xffffffffu;
+      const bool leader = lane == 0;
+      if (leader) tc::prefetch_tmap(&tm_v);
+      int gv = 0;
+      for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
+        XlItem I;
+        if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
+        const float* tb = tab + ((size_t)I.bh * NC + I.c) * tstride;
+        for (int j = 0; j < I.nkv && ok; ++j, ++gv) {
+          const int st = gv % NV;
+          ok = __all_sync(full, tc::mbar_wait(&bar[X_VE0 + st], ((gv / NV) & 1) ^ 1, abort_flag));
+          if (!ok) break;
+          if (leader) {
+            uint64_t* vf = &bar[X_VF0 + st];
+            uint8_t* vs = smem + Cfg::OFF_V + st * Cfg::V_BYTES;
+            uint8_t* cp = smem + Cfg::OFF_COL + st * Cfg::COLAUX;
+            tc::mbar_arrive_expect_tx(vf, Cfg::V_BYTES + Cfg::COLAUX);
+            for (int v = 0; v < Cfg::VB; ++v)
+              tc::tma_load_3d(vs + v * 16384, &tm_v, vf, I.vb * DV + v * 64, I.c * L + j * 128, I.bh);
+            tc::bulk_load(cp, tb + 3 * L + j * 128, 512, vf);
+            tc::bulk_load(cp + 512, tb + 4 * L + j * 128, 512, vf);
+            tc::bulk_load(cp + 1024, tb + 5 * L + j * 4, 16, vf);
+          }
+        }
+      }
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks the schedule and waits; lane 0 issues the MMAs and
+    // their commits (a commit tracks the MMAs of the thread that issues it).
+    {
+      const unsigned full = 0xffffffffu;
+      const bool leader = lane == 0;
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(128, DV, false, true);
-      const uint32_t aQ0 = tc::smem_u32(smem + Cfg::OFF_Q), aR0 = tc::smem_u32(smem + Cfg::OFF_RING);
+      const uint32_t aQ0 = tc::smem_u32(smem + Cfg::OFF_Q), aK0 = tc::smem_u32(smem + Cfg::OFF_K),
+                     aV0 = tc::smem_u32(smem + Cfg::OFF_V);
 
       // score step s of item I (its it-th item, global step g): S_j = Q K_j^T,
-      // or for the C_prev step only a commit, which tells the transform the S
-      // buffer's last reader (P V of step g - 2) is done
+      // then the K stage is free; for the C_prev step only a commit, which
+      // tells the transform the S buffer's last reader (P V of step g - 2) is done
       auto issue_s = [&](const XlItem& I, int it, int s, int g) -> bool {
         const int sb = g & 1;
         if (I.pseudo && s == 0) {
-          tc::tc_commit(&bar[X_SF0 + sb]);
+          if (leader) tc::tc_commit(&bar[X_SF0 + sb]);
+          __syncwarp();
           return true;
         }
-        const int qb = it % NQ, st = g % NS;
-        if (!tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag)) return false;
-        if (!tc::mbar_wait(&bar[X_KVF0 + st], (g / NS) & 1, abort_flag)) return false;
+        const int qb = it % NQ, kst = g % NK;
+        // every barrier check costs the tensor pipe a drain, so the Q buffer is
+        // checked only before the item's first score product
+        if (s == (I.pseudo ? 1 : 0) &&
+            !__all_sync(full, tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag)))
+          return false;
+        if (!__all_sync(full, tc::mbar_wait(&bar[X_KF0 + kst], (g / NK) & 1, abort_flag))) return false;
         tc::tc_fence_after();
-        const uint32_t aQ = aQ0 + qb * Cfg::Q_BYTES, aK = aR0 + st * Cfg::STAGE;
+        const uint32_t aQ = aQ0 + qb * Cfg::Q_BYTES, aK = aK0 + kst * Cfg::K_BYTES;
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < DQK / 16; ++k) {
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          tc::mma_bf16_ss(tmem + sb * 128, tc::sdesc_sw128(aQ + off, 16, 1024),
-                          tc::sdesc_sw128(aK + off, 16, 1024), idS, k > 0);
+          for (int k = 0; k < DQK / 16; ++k) {
+            const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+            tc::mma_bf16_ss(tmem + sb * 128, tc::sdesc_sw128(aQ + off, 16, 1024),
+                            tc::sdesc_sw128(aK + off, 16, 1024), idS, k > 0);
+          }
+          tc::tc_commit(&bar[X_SF0 + sb]);
+          tc::tc_commit(&bar[X_KE0 + kst]);
         }
-        tc::tc_commit(&bar[X_SF0 + sb]);
+        __syncwarp();
         return true;
       };
-      // accumulate step s into O: P_j V_j, or (alpha q / sqrt(d_qk)) C_prev,
-      // A read from the two P halves in TMEM
-      auto issue_pv = [&](const XlItem& I, int it, int s, int g) -> bool {
-        const int sb = g & 1, st = g % NS, ob = it & 1;
+      // accumulate step s into O: P_j V_j (V stage of real step gv),
+      // or (alpha q / sqrt(d_qk)) C_prev (K stage of step g); A is read from
+      // P in TMEM.  The transform threads see V / C_prev arrive before they
+      // signal P, so one barrier check covers the whole product.
+      auto issue_pv = [&](const XlItem& I, int it, int s, int g, int gv) -> bool {
+        const int sb = g & 1, ob = it & 1;
         const uint32_t tO = tmem + 256 + ob * DV, tP = tmem + sb * 128;
-        if (s == 0 && !tc::mbar_wait(&bar[X_OE0 + ob], ((it >> 1) & 1) ^ 1, abort_flag)) return false;
-        const uint32_t aS = aR0 + st * Cfg::STAGE;
-        const bool pseudo = I.pseudo && s == 0;
-        for (int h = 0; h < 2; ++h) {
-          if (!tc::mbar_wait(&bar[X_PF0 + 2 * sb + h], (g >> 1) & 1, abort_flag)) return false;
-          tc::tc_fence_after();
-          if (pseudo) {
+        if (s == 0 && !__all_sync(full, tc::mbar_wait(&bar[X_OE0 + ob], ((it >> 1) & 1) ^ 1, abort_flag)))
+          return false;
+        if (!__all_sync(full, tc::mbar_wait(&bar[X_PF0 + sb], (g >> 1) & 1, abort_flag))) return false;
+        tc::tc_fence_after();
+        if (I.pseudo && s == 0) {
+          const int kst = g % NK;
+          const uint32_t aC = aK0 + kst * Cfg::K_BYTES;
+          if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < DQK / 32; ++kk) {
-              const int k = h * (DQK / 32) + kk;  // 16 rows of C_prev
-              tc::mma_bf16_ts(tO, tP + 64 * h + 8 * kk,
-                              tc::sdesc_sw128(aS + k * 2048, DQK * 128, 1024), idO, k > 0);
+            for (int k = 0; k < DQK / 16; ++k) {  // 16 rows of C_prev
+              const int h = k / (DQK / 32), kk = k % (DQK / 32);
+              tc::mma_bf16_ts(tO, tP + 64 * h + 8 * kk, tc::sdesc_sw128(aC + k * 2048, DQK * 128, 1024),
+                              idO, k > 0);
             }
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int k = 4 * h + kk;  // 16 keys of the tile
-              tc::mma_bf16_ts(tO, tP + 64 * h + 8 * kk,
-                              tc::sdesc_sw128(aS + Cfg::K_BYTES + k * 2048, 16384, 1024), idO,
-                              (s > 0 || k > 0));
-            }
+            tc::tc_commit(&bar[X_KE0 + kst]);
           }
+          __syncwarp();
+          return true;
         }
-        tc::tc_commit(&bar[X_KVE0 + st]);
+        if (leader) {
+          const int vst = gv % NV;
+          const uint32_t aV = aV0 + vst * Cfg::V_BYTES;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // 16 keys per step; keys 64 h .. of P live at column 64 h
+            tc::mma_bf16_ts(tO, tP + 64 * (k >> 2) + 8 * (k & 3),
+                            tc::sdesc_sw128(aV + k * 2048, 16384, 1024), idO, (s > 0 || k > 0));
+          tc::tc_commit(&bar[X_VE0 + vst]);
+        }
+        __syncwarp();
         return true;
       };
 
       XlItem I, N;
-      int k = xl_next(blockIdx.x, total, BH, NC, NVB, ntq, T, L, I);
-      int it = 0, g = 0;
+      int k = xl_next(xl_first(), total, BH, NC, NVB, ntq, T, L, I);
+      int it = 0, g = 0, gv = 0;
       if (k < total) ok = issue_s(I, 0, 0, 0);
       while (k < total && ok) {
-        const int kn = xl_next(k + gridDim.x, total, BH, NC, NVB, ntq, T, L, N);
+        const int kn = xl_next(xl_succ(k), total, BH, NC, NVB, ntq, T, L, N);
         const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
         for (int s = 0; s < nsteps && ok; ++s, ++g) {
           const bool last = s + 1 == nsteps;
-          if (NS > 1) {
+          // the look-ahead S goes before this step's P V when the next Q and K
+          // stages can be resident at the same time; otherwise after it
+          if (Cfg::LOOK) {
             if (!last) ok = issue_s(I, it, s + 1, g + 1);
             else if (kn < total) ok = issue_s(N, it + 1, 0, g + 1);
             if (!ok) break;
           }
-          ok = issue_pv(I, it, s, g);
+          const bool real = !(I.pseudo && s == 0);
+          ok = issue_pv(I, it, s, g, gv);
           if (!ok) break;
-          if (last) {
+          if (real) ++gv;
+          if (last && leader) {
             tc::tc_commit(&bar[X_QE0 + it % NQ]);
             tc::tc_commit(&bar[X_OF0 + (it & 1)]);
           }
-          if (NS == 1) {
+          __syncwarp();
+          if (!Cfg::LOOK) {
             if (!last) ok = issue_s(I, it, s + 1, g + 1);
             else if (kn < total) ok = issue_s(N, it + 1, 0, g + 1);
           }
@@ -300,7 +381,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     const int row = 32 * qr + lane;
     const uint32_t lb = (uint32_t)(32 * qr) << 16;
     const unsigned full = 0xffffffffu;
-    int it = 0, g = 0;
+    int it = 0, g = 0, gv = 0;
 
     // epilogue of one item: normalise O and store h
     struct Pending {
@@ -351,7 +432,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       return true;
     };
 
-    for (int k = blockIdx.x; k < total && ok; k += gridDim.x) {
+    for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
       XlItem I;
       if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
       const int qb = it % NQ;
@@ -362,7 +443,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       uint64_t part2 = tc::f2_make(0.f, 0.f);  // EXP: this half's share of the normaliser
       const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
       for (int s = 0; s < nsteps && ok; ++s, ++g) {
-        const int sb = g & 1, st = g % NS;
+        const int sb = g & 1;
         ok = __all_sync(full, tc::mbar_wait(&bar[X_SF0 + sb], (g >> 1) & 1, abort_flag));
         if (!ok) break;
         tc::tc_fence_after();
@@ -397,10 +478,19 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
             }
             tc::tmem_st16_async(tS + 16 * grp, w);
           }
+          // P signals the MMA thread that C_prev has landed as well
+          ok = __all_sync(full, tc::mbar_wait(&bar[X_KF0 + g % NK], (g / NK) & 1, abort_flag));
+          if (!ok) break;
         } else {
           const int j = s - (I.pseudo ? 1 : 0);
           const bool diag = j == I.qt;
-          const float* cp = reinterpret_cast<const float*>(smem + Cfg::OFF_COL + st * Cfg::COLAUX);
+          const int vst = gv % NV, vpar = (gv / NV) & 1;
+          ++gv;
+          // the key tile's gate factors, which arrive with its V tile; seeing
+          // them also tells the MMA thread (through P) that V has landed
+          ok = __all_sync(full, tc::mbar_wait(&bar[X_VF0 + vst], vpar, abort_flag));
+          if (!ok) break;
+          const float* cp = reinterpret_cast<const float*>(smem + Cfg::OFF_COL + vst * Cfg::COLAUX);
           uint32_t sa[32], sb2[32];
           tc::tmem_ld32_async(tS, sa);
           tc::tmem_ld32_async(tS + 32, sb2);
@@ -453,7 +543,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
-        tc::mbar_arrive(&bar[X_PF0 + 2 * sb + h]);
+        tc::mbar_arrive(&bar[X_PF0 + sb]);
         if (s == 0) {
           tc::mbar_arrive(&bar[X_QE0 + qb]);
           if (pend) {
@@ -512,10 +602,11 @@ static cudaError_t launch_out_xl(const Problem& p, const FwdArgs& a, cudaStream_
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const int ntq = p.L / 128, nvb = p.dhv / DV;
+  const int ntq = p.L / 128, nvb = p.dhv / DV;  // ntq is even: L >= 256 is a power of two
   const long long total = (long long)ntq * p.BH * p.NC * nvb;
-  if (total >= (1LL << 31)) return cudaErrorInvalidValue;
-  const int grid = (int)(total < nsm ? total : nsm);
+  if (total >= (1LL << 30)) return cudaErrorInvalidValue;
+  const long long pairs = total / 2;
+  const int grid = (int)(pairs < nsm ? pairs : nsm);
   kern<<<grid, kXlThreads, smem, s>>>(tq, tk, tv, tcm, a.xt, a.n, (bf16*)a.h, a.abar, p.T, p.L,
                                       p.NC, p.BH, nvb, ntq, (int)total, xl_table_stride(p.L),
                                       p.dhv);
