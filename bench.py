@@ -331,17 +331,77 @@ def run_sweep(args):
                 flops = B * NH * flops_fwd(T, d, d, L)
                 out_name = [n for n in names if n.startswith("output_fwd")][0]
                 out_fl = B * NH * kernel_costs(T, d, d, L, var == 1, 2)["output_fwd"][0]
-                print(json.dumps({
+                line = {
                     "sweep": f"fwd_b{B}h32_d128", "cell": label, "T": T, "chunk": L,
                     "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": B * T / ms * 1e3,
                     "kernel_ms": kms, "output_kernel": out_name,
                     "output_tflops": out_fl / kms[out_name] / 1e9,
                     "output_pct_bf16_peak": 100 * out_fl / kms[out_name] / 1e9 / peaks["bf16_tflops"],
-                }), flush=True)
+                }
+                if args.sweep_bwd:
+                    line.update(sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev,
+                                                B, NH, T, d, L, var, peaks))
+                print(json.dumps(line), flush=True)
                 del saved
             del x, h
             torch.cuda.empty_cache()
     return 0
+
+
+def sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev, B, NH, T, d, L, var, peaks):
+    """Backward at one sweep point: mlstm_bwd timed like the forward, per kernel.
+
+    Reports backward TFLOP/s (algorithmic count 8 T d^2 + T L 5 d per head) and
+    the intra-chunk kernels' (dq, dk, dv) combined TFLOP/s against the dense
+    bf16 peak.  Inputs: the point's forward outputs and an upstream dh ~ N(0,1).
+    """
+    import torch
+    g = torch.Generator(device="cpu").manual_seed(7)
+    dh = torch.randn(x["v"].shape, generator=g).to(device=dev, dtype=x["v"].dtype)
+    dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+    dig, dfg = torch.empty_like(x["igate"]), torch.empty_like(x["fgate"])
+    ws = torch.empty(binding.mlstm_bwd_workspace_size(*sizes), dtype=torch.uint8, device=dev)
+    nb = binding.mlstm_bwd_launch_count(*sizes)
+    names = [binding.mlstm_launch_name(1, i, *sizes) for i in range(nb)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nb)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    arrs = [(ctypes.c_void_p * (2 * nb))(*[e.cuda_event for e in row]) for row in evs]
+
+    def call(ev=None):
+        if ev is not None:
+            binding.mlstm_set_timing_events(ev, 2 * nb)
+        st = binding.mlstm_bwd(x["q"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(),
+                               x["igate"].data_ptr(), x["fgate"].data_ptr(), h.data_ptr(),
+                               dh.data_ptr(), saved.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), dig.data_ptr(), dfg.data_ptr(), ws.data_ptr(),
+                               ws.numel(), *sizes, sh)
+        binding.mlstm_set_timing_events(None, 0)
+        if st != 0:
+            raise binding.MLSTMError(st, "mlstm_bwd")
+
+    for _ in range(args.warmup):
+        call()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i in range(args.steps):
+        call(arrs[i])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    binding.check_device()
+    ms = e0.elapsed_time(e1) / args.steps
+    kms = {n: sum(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs) / args.steps
+           for i, n in enumerate(names)}
+    costs = kernel_costs(T, d, d, L, var == 1, 2)
+    intra = [n for n in names if n.split("_")[0] in ("dq", "dk", "dv")]
+    intra_fl = B * NH * sum(costs[n][0] for n in intra)
+    intra_ms = sum(kms[n] for n in intra)
+    return {"bwd_ms": ms, "bwd_tflops": B * NH * flops_bwd(T, d, d, L) / ms / 1e9,
+            "bwd_kernel_ms": kms, "bwd_intra_tflops": intra_fl / intra_ms / 1e9,
+            "bwd_intra_pct_bf16_peak": 100 * intra_fl / intra_ms / 1e9 / peaks["bf16_tflops"]}
 
 
 def workload_config(spec, n):
@@ -373,6 +433,8 @@ def main():
                     help="B for --sweep (smaller for ncu captures; the sweep workload is B8)")
     ap.add_argument("--sweep-cells", default=None,
                     help="comma subset of sig,exp,exp_igate_bias_m10 for --sweep")
+    ap.add_argument("--sweep-bwd", action="store_true",
+                    help="also time the backward at every --sweep point")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (smaller captures for ncu; the default is the workload's B)")
     args = ap.parse_args()
