@@ -59,7 +59,9 @@ struct XlCfg {
   static constexpr int OFF_ROW = OFF_V + NV * V_BYTES;
   static constexpr int OFF_COL = OFF_ROW + NQ * ROWAUX;
   static constexpr int OFF_XS = OFF_COL + NV * COLAUX;  // [2 O buffers][2 halves][128] floats
-  static constexpr int OFF_BAR = OFF_XS + 2 * 2 * 128 * 4;
+  static constexpr int OFF_STG = OFF_XS + 2 * 2 * 128 * 4;  // per transform warp: 16 rows of h
+  static constexpr int STG_WARP = 16 * DV;                     // 16 rows x DV / 2 bf16
+  static constexpr int OFF_BAR = OFF_STG + 8 * STG_WARP;
   static constexpr int OFF_TMEM = OFF_BAR + 64 * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;         // S0 [0,128) S1 [128,256) O0, O1 from 256
@@ -126,6 +128,84 @@ __device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB
 }
 
 }  // namespace
+
+// Epilogue of one SIG work item (no normaliser, h = O) for the transform
+// thread of row 32 qr + lane and key half h: read O out of TMEM, freeing it
+// for the next item's products, and store h through a staging slot so each
+// store instruction writes whole row segments.  Kept out of line so its
+// registers do not count against the gate transform it is called from.
+// (EXP keeps its epilogue inline with direct stores: there the staging cost
+// more in transform registers than it saved in store traffic, measured.)
+template <int DQK, int DV, bool EXPV>
+__device__ __noinline__ bool xl_epilogue(int it, int vb, int nvalid, size_t tok, float fl, float part,
+                                         int h, int qr, int lane, uint32_t tmem, uint8_t* smem,
+                                         bf16* __restrict__ hout, float* __restrict__ abar_out,
+                                         int dhv, const volatile unsigned int* abort_flag) {
+  using Cfg = XlCfg<DQK, DV>;
+  const unsigned full = 0xffffffffu;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  const int warp = 2 + 4 * h + ((qr + 2) & 3);
+  const uint32_t lb = (uint32_t)(32 * qr) << 16;
+  const int ob = it & 1, par = (it >> 1) & 1;
+  (void)fl;
+  (void)part;
+  (void)abar_out;
+  if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + ob], par, abort_flag))) return false;
+  tc::tc_fence_after();
+  const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 2);
+  // this thread's DV / 2 columns as CPR 16-byte chunks, read 32 columns at a time
+  constexpr int CPR = DV / 16, RPI = 32 / CPR;
+  uint4 w[CPR];
+#pragma unroll
+  for (int q = 0; q < DV / 64; ++q) {
+    uint32_t o[32];
+    tc::tmem_ld32_async(tO + 32 * q, o);
+    tc::tmem_wait_ld(o);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const uint32_t* r = &o[8 * c4];
+      uint4& d = w[4 * q + c4];
+      d.x = tc::pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
+      d.y = tc::pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
+      d.z = tc::pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
+      d.w = tc::pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
+    }
+  }
+  tc::tc_fence_before();
+  tc::mbar_arrive(&bar[X_OE0 + ob]);
+  // Each thread owns one row, so direct stores would touch 32 lines per
+  // warp instruction.  Rows go through a swizzled 16-row staging slot
+  // instead and leave as RPI whole row segments per instruction.
+  const uint32_t stg = tc::smem_u32(smem + Cfg::OFF_STG + (warp - 2) * Cfg::STG_WARP);
+#pragma unroll
+  for (int rnd = 0; rnd < 2; ++rnd) {
+    if ((lane >> 4) == rnd) {
+      const int r = lane & 15;
+#pragma unroll
+      for (int c = 0; c < CPR; ++c)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         stg + r * (CPR * 16) + ((c ^ (r & (CPR - 1))) << 4)),
+                     "r"(w[c].x), "r"(w[c].y), "r"(w[c].z), "r"(w[c].w)
+                     : "memory");
+    }
+    __syncwarp();
+#pragma unroll
+    for (int kk = 0; kk < 16 / RPI; ++kk) {
+      const int rr = kk * RPI + lane / CPR, c = lane % CPR;
+      uint4 v;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(stg + rr * (CPR * 16) + ((c ^ (rr & (CPR - 1))) << 4))
+                   : "memory");
+      const int rw = 16 * rnd + rr;  // row within this warp's 32
+      if (rw < nvalid)
+        *reinterpret_cast<uint4*>(hout + (tok - lane + rw) * (size_t)dhv + vb * DV +
+                                  h * (DV / 2) + 8 * c) = v;
+    }
+    __syncwarp();
+  }
+  return true;
+}
 
 template <int DQK, int DV, bool EXPV>
 __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
@@ -384,29 +464,32 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     int it = 0, g = 0, gv = 0;
 
     // epilogue of one item: normalise O and store h
+    // what the deferred epilogue of an item needs (kept small: it is live
+    // through the next item's first step)
     struct Pending {
-      int ob, par, vb, col0;
-      bool valid;
-      size_t tok;
+      int it, vb, nvalid;  // item counter; value block; rows of this warp's 32 in the sequence
+      size_t tok;          // token of this thread's row
       float fl, part;
     } pe{};
     bool pend = false;
     auto epilogue = [&](const Pending& e) -> bool {
-      float inv = 1.f;
-      if (EXPV) {
-        // den_t = max(|a_t|, exp(-m_t)), a_t the sum of both halves' shares
-        float* x = xs + e.ob * 256;
-        x[h * 128 + row] = e.part;
-        tc::mbar_arrive(&bar[X_XS0 + e.ob]);
-        if (!__all_sync(full, tc::mbar_wait(&bar[X_XS0 + e.ob], e.par, abort_flag))) return false;
-        const float a = e.part + x[(1 - h) * 128 + row];
-        inv = 1.f / fmaxf(fabsf(a), e.fl);
-        if (h == 0 && e.vb == 0 && e.valid) abar_out[e.tok] = a;
-      }
-      if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + e.ob], e.par, abort_flag))) return false;
+      if (!EXPV)
+        return xl_epilogue<DQK, DV, EXPV>(e.it, e.vb, e.nvalid, e.tok, e.fl, e.part, h, qr, lane, tmem,
+                                          smem, hout, abar_out, dhv, abort_flag);
+      // EXP: den_t = max(|a_t|, exp(-m_t)), a_t the sum of both halves' shares
+      const int ob = e.it & 1, par = (e.it >> 1) & 1;
+      const bool valid = lane < e.nvalid;
+      float* x = xs + ob * 256;
+      x[h * 128 + row] = e.part;
+      tc::mbar_arrive(&bar[X_XS0 + ob]);
+      if (!__all_sync(full, tc::mbar_wait(&bar[X_XS0 + ob], par, abort_flag))) return false;
+      const float a = e.part + x[(1 - h) * 128 + row];
+      const float inv = 1.f / fmaxf(fabsf(a), e.fl);
+      if (h == 0 && e.vb == 0 && valid) abar_out[e.tok] = a;
+      if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + ob], par, abort_flag))) return false;
       tc::tc_fence_after();
-      const uint32_t tO = tmem + 256 + e.ob * DV + lb + h * (DV / 2);
-      uint4* dst = reinterpret_cast<uint4*>(hout + e.tok * (size_t)dhv + e.col0);
+      const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 2);
+      uint4* dst = reinterpret_cast<uint4*>(hout + e.tok * (size_t)dhv + e.vb * DV + h * (DV / 2));
 #pragma unroll
       for (int q = 0; q < DV / 64; ++q) {
         uint32_t o[32];
@@ -414,9 +497,9 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
         tc::tmem_wait_ld(o);
         if (q == DV / 64 - 1) {
           tc::tc_fence_before();
-          tc::mbar_arrive(&bar[X_OE0 + e.ob]);
+          tc::mbar_arrive(&bar[X_OE0 + ob]);
         }
-        if (e.valid) {
+        if (valid) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
             const uint32_t* r = &o[8 * c8];
@@ -554,12 +637,10 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       }
       if (!ok) break;
       const float2 pf = tc::f2_split(part2);
-      pe.ob = it & 1;
-      pe.par = (it >> 1) & 1;
+      pe.it = it;
       pe.vb = I.vb;
-      pe.col0 = I.vb * DV + h * (DV / 2);
-      pe.valid = I.t0 + row < I.len;
       pe.tok = (size_t)I.bh * T + (size_t)I.c * L + I.t0 + row;
+      pe.nvalid = min(32, max(0, I.len - (I.t0 + 32 * qr)));
       pe.fl = FLt;
       pe.part = pf.x + pf.y;
       pend = true;
