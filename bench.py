@@ -348,6 +348,75 @@ def run_sweep(args):
     return 0
 
 
+# RetNet chunk_fwd / chunk_fwdbwd times (ms) on one A100 80GB at B8, 32 heads,
+# head dim 128 (flash-linear-attention README, RetNet vs FlashAttention-2
+# timing table; units not printed, read as ms).  Context only: other hardware.
+RETNET_A100_MS = {128: (0.185344, 1.591296), 256: (0.219136, 1.596928), 512: (0.397312, 1.603584),
+                  1024: (0.747520, 3.089408), 2048: (1.403904, 6.059008), 4096: (2.755072, 11.938816),
+                  8192: (5.491712, 23.952385), 16384: (10.870784, 48.745472)}
+
+
+def run_retnet(args):
+    """Retention (RetNet decays gamma_h = 1 - 2^(-5-h)) through the SIG kernels.
+
+    B8 H32 d128 bf16 at the sequence lengths of the pages' A100 table; per T the
+    forward and forward+backward are timed (CUDA events, mean of --steps after
+    --warmup) at every chunk in 128..1024 not above T, and the fastest chunk of
+    each pass is reported.  One JSON line per T.
+    """
+    import torch
+    from mlstm_chunkwise_attention_b200 import binding
+    from mlstm_chunkwise_attention_b200.synthetic import make_inputs
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    B, NH, d = 8, 32, 128
+    gamma = binding.retnet_decays(NH)
+    Ts = [int(t) for t in args.sweep_t.split(",")] if args.sweep_t else sorted(RETNET_A100_MS)
+    for T in Ts:
+        cpu = make_inputs(B, NH, T, d, d, seed=11, igate_mean=0.0, fgate_mean=3.0,
+                          dtype=torch.bfloat16, with_dh=True)
+        x = {k: v.to(dev) for k, v in cpu.items()}
+        del cpu
+        ig, fg, _ = binding.retention_gates(gamma, B, T, torch.bfloat16, dev)
+        best = {}
+        for L in [c for c in (128, 256, 512, 1024) if c <= max(T, 128)]:
+            def fwd():
+                return binding.forward(x["q"], x["k"], x["v"], ig, fg, L, binding.SIG,
+                                       keep_saved=True)
+
+            def fwdbwd():
+                h, saved = fwd()
+                binding.backward(x["q"], x["k"], x["v"], ig, fg, h, x["dh"], saved, L, binding.SIG)
+
+            for name, fn in (("fwd", fwd), ("fwdbwd", fwdbwd)):
+                for _ in range(args.warmup):
+                    fn()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize(dev)
+                e0.record(stream)
+                for _ in range(args.steps):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                binding.check_device()
+                ms = e0.elapsed_time(e1) / args.steps
+                if name not in best or ms < best[name][0]:
+                    best[name] = (ms, L)
+        ref = RETNET_A100_MS.get(T)
+        print(json.dumps({
+            "retnet": "b8h32_d128_bf16", "T": T,
+            "fwd_ms": best["fwd"][0], "fwd_chunk": best["fwd"][1],
+            "fwd_tflops": B * NH * flops_fwd(T, d, d, best["fwd"][1]) / best["fwd"][0] / 1e9,
+            "fwdbwd_ms": best["fwdbwd"][0], "fwdbwd_chunk": best["fwdbwd"][1],
+            "tokens_per_s_fwdbwd": B * T / best["fwdbwd"][0] * 1e3,
+            "a100_chunk_fwd_ms": ref[0] if ref else None,
+            "a100_chunk_fwdbwd_ms": ref[1] if ref else None,
+        }), flush=True)
+        del x
+        torch.cuda.empty_cache()
+    return 0
+
+
 def sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev, B, NH, T, d, L, var, peaks):
     """Backward at one sweep point: mlstm_bwd timed like the forward, per kernel.
 
@@ -435,6 +504,9 @@ def main():
                     help="comma subset of sig,exp,exp_igate_bias_m10 for --sweep")
     ap.add_argument("--sweep-bwd", action="store_true",
                     help="also time the backward at every --sweep point")
+    ap.add_argument("--retnet", action="store_true",
+                    help="retention (RetNet decays) through the SIG kernels at B8 H32 d128, "
+                         "T from --sweep-t or the 128..16384 list")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (smaller captures for ncu; the default is the workload's B)")
     args = ap.parse_args()
@@ -450,6 +522,8 @@ def main():
         return run_reference(args, spec)
     if args.sweep:
         return run_sweep(args)
+    if args.retnet:
+        return run_retnet(args)
 
     import torch
     import torch.distributed as dist
