@@ -488,6 +488,7 @@ def workload_config(spec, n):
 # ---------------------------------------------------------------------------
 
 def main():
+    global WORKLOAD
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -509,14 +510,23 @@ def main():
                          "T from --sweep-t or the 128..16384 list")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (smaller captures for ncu; the default is the workload's B)")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["exp_b8h32_t4096_d128_c128", "train_b4h16_t8192_d256_c256",
+                             "sig_long_b1h8_t65536_c1024"],
+                    help="bf16 workload of the fwd+bwd step (default: the headline)")
+    ap.add_argument("--variant", choices=["sig", "exp"], default=None,
+                    help="override the workload's cell variant")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     from mlstm_chunkwise_attention_b200.synthetic import WORKLOADS
+    WORKLOAD = args.workload
     spec = dict(WORKLOADS[WORKLOAD])
     if args.batch is not None:
         spec["B"] = args.batch
+    if args.variant is not None:
+        spec["variant"] = 0 if args.variant == "sig" else 1
 
     if args.impl == "reference":
         return run_reference(args, spec)

@@ -163,6 +163,30 @@ def recurrent_forward_stabilised(q, k, v, log_i, log_f):
     return {"h": h, "m": m_all, "abar": abar}
 
 
+def recurrent_step(C, n, m, q, k, v, igate_pre, fgate_pre, variant):
+    """One token of the recurrence from the state of the previous token (FusedRecurrent
+    form of the flash-linear-attention README; readings 1 and 2).
+
+    SIG: C' = f C + i k v^T, h = C'^T q' (n and m are carried unchanged).
+    EXP: m' = max(log f + m, log i), C' = exp(log f + m - m') C + exp(log i - m') k v^T,
+    n' likewise, h = C'^T q' / max(|n' . q'|, exp(-m')).
+    The zero state is C = 0, n = 0, m = -inf.  Returns (h, C', n', m').
+    """
+    C, n, q, k, v = _as64(C, n, q, k, v)
+    log_i, log_f = gate_logs(np.float64(igate_pre), np.float64(fgate_pre), variant)
+    qs = q / np.sqrt(q.shape[0])
+    if variant == SIG:
+        C = np.exp(log_f) * C + np.exp(log_i) * np.outer(k, v)
+        return C.T @ qs, C, n, m
+    m_new = max(log_f + m, log_i)
+    decay = np.exp(log_f + m - m_new)
+    inp = np.exp(log_i - m_new)
+    C = decay * C + inp * np.outer(k, v)
+    n = decay * n + inp * k
+    h = (C.T @ qs) / max(abs(n @ qs), np.exp(-m_new))
+    return h, C, n, m_new
+
+
 # ---------------------------------------------------------------------------
 # parallel (quadratic) form
 # ---------------------------------------------------------------------------
@@ -298,6 +322,9 @@ def chunkwise_forward(q, k, v, log_i, log_f, variant, L):
         "h": h, "b": b, "g": g, "log_i": log_i.copy(), "m_row": m_row,
         "m_state": m_state, "m_enter": m_enter, "C_enter": C_enter,
         "n_enter": n_enter, "abar": abar, "den": den,
+        # state after the last row (EXP: scaled by exp(-m_T)), what a step-by-step
+        # continuation of the sequence starts from
+        "C_final": C, "n_final": n, "m_final": m_state[-1] if exp_variant else 0.0,
     }
 
 

@@ -133,6 +133,27 @@ def check_single_token(M):
                                i1 * s * v[0] / max(abs(i1 * s), 1.0), rtol=1e-14)
 
 
+def check_steps(M, variant, seed=51):
+    """Stepping token by token from the zero state reproduces the recurrent forms (which
+    the closed forms above pin), and the chunkwise form's final state is the state after
+    the last step, with a ragged last chunk."""
+    q, k, v, ig, fg = rnd(seed, 23, 4, 5, 3.0)
+    C, n, m = np.zeros((4, 5)), np.zeros(4), -np.inf
+    hs = []
+    for t in range(23):
+        h, C, n, m = M.recurrent_step(C, n, m, q[t], k[t], v[t], ig[t], fg[t], variant)
+        hs.append(h)
+    li, lf = M.gate_logs(ig, fg, variant)
+    ref = (M.recurrent_forward(q, k, v, li, lf, SIG)["h"] if variant == SIG
+           else M.recurrent_forward_stabilised(q, k, v, li, lf)["h"])
+    np.testing.assert_allclose(np.array(hs), ref, rtol=1e-11, atol=1e-13)
+    cw = M.chunkwise_forward(q, k, v, li, lf, variant, 7)
+    np.testing.assert_allclose(cw["C_final"], C, rtol=1e-11, atol=1e-13)
+    if variant == EXP:
+        np.testing.assert_allclose(cw["n_final"], n, rtol=1e-11, atol=1e-13)
+        assert abs(cw["m_final"] - m) < 1e-12
+
+
 def check_parallel_vs_recurrent(M, variant, seed=5, ig_mean=0.0, fg_mean=3.0):
     q, k, v, ig, fg = rnd(seed, 40, 8, 6, ig_mean, fg_mean)
     li, lf = M.gate_logs(ig, fg, variant)
@@ -300,12 +321,18 @@ ALL_CHECKS = [
     lambda M: check_chunkwise_backward(M, SIG), lambda M: check_chunkwise_backward(M, EXP),
     lambda M: check_rows(M, SIG), lambda M: check_rows(M, EXP),
     lambda M: check_finite_differences(M, SIG), lambda M: check_finite_differences(M, EXP),
+    lambda M: check_steps(M, SIG), lambda M: check_steps(M, EXP),
 ]
 
 
 # ---------------------------------------------------------------------------
 # the pins, on the real oracle
 # ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("variant", [SIG, EXP])
+def test_steps_and_final_state(variant):
+    check_steps(oracle, variant)
+
 
 def test_hand_worked_cases():
     check_hand_cases(oracle)
@@ -405,6 +432,10 @@ MUTATIONS = [
     ("max state missing b", "m_row[sl] = b[sl] + np.maximum(m_prev, u)", "m_row[sl] = np.maximum(m_prev, u)"),
     ("inter-chunk factor missing b", "alpha = np.exp(bt + m_enter[c] - mt) if exp_variant", "alpha = np.exp(m_enter[c] - mt) if exp_variant"),
     ("stabilised floor 1", "max(abs(abar[t]), np.exp(-m_new))", "max(abs(abar[t]), 1.0)"),
+    ("step decay dropped", "C = decay * C + inp * np.outer(k, v)\n    n = decay * n + inp * k\n    h = (C.T",
+     "C = C + inp * np.outer(k, v)\n    n = decay * n + inp * k\n    h = (C.T"),
+    ("step floor 1", "h = (C.T @ qs) / max(abs(n @ qs), np.exp(-m_new))", "h = (C.T @ qs) / max(abs(n @ qs), 1.0)"),
+    ("final state one chunk early", '"C_final": C, "n_final"', '"C_final": C_enter[-1], "n_final"'),
     ("dk transposed", "dk = dS.T @ qs", "dk = dS @ qs"),
     ("dlog_f summed on the wrong axis", "dlog_f = np.tril(excl).sum(axis=0)", "dlog_f = np.tril(excl).sum(axis=1)"),
     ("da sign", "da = np.where(active, -np.sum(dh * h, axis=1)", "da = np.where(active, np.sum(dh * h, axis=1)"),
