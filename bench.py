@@ -417,6 +417,83 @@ def run_retnet(args):
     return 0
 
 
+def run_decode(args):
+    """One-token steps (generation) at B8 H32 d128 bf16, both cells.
+
+    Times --steps replays of a CUDA graph of 100 consecutive mlstm_step calls
+    (state ping-pong, CUDA events), and reports tokens/s and the step kernel's
+    HBM roofline: every step reads and writes the fp32 state (C, and n for
+    EXP) once and touches q, k, v, h and the gates.  Also times the hand-off
+    from a T = 4096 chunk-128 forward (mlstm_final_state).
+    """
+    import torch
+    from mlstm_chunkwise_attention_b200 import binding
+    from mlstm_chunkwise_attention_b200.synthetic import make_inputs
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    B, NH, d, T, L = 8, 32, 128, 4096, 128
+    for var, label in ((0, "sig"), (1, "exp")):
+        cpu = make_inputs(B, NH, T, d, d, seed=13, igate_mean=-2.0, fgate_mean=3.0,
+                          dtype=torch.bfloat16, with_dh=False)
+        x = {k: v.to(dev) for k, v in cpu.items()}
+        _, saved = binding.forward(x["q"], x["k"], x["v"], x["igate"], x["fgate"], L, var)
+        state = binding.final_state(x["k"], x["v"], saved, L, var)
+        other = torch.empty_like(state)
+        tok = {k: v[:, :, -1].contiguous() for k, v in x.items()}
+        h = torch.empty((B, NH, d), dtype=torch.bfloat16, device=dev)
+
+        def steps(n):
+            nonlocal state, other
+            for _ in range(n):
+                binding.step(tok["q"], tok["k"], tok["v"], tok["igate"], tok["fgate"], state, other,
+                             var, h=h)
+                state, other = other, state
+
+        steps(100 * args.warmup)
+        torch.cuda.synchronize(dev)
+        # 100 steps captured once in a CUDA graph (an even count: the state
+        # buffers end where they started), so the device time is measured
+        # without the host's per-call overhead
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            steps(100)
+        for _ in range(args.warmup):
+            graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        binding.check_device()
+        ms = e0.elapsed_time(e1) / (100 * args.steps)
+        del graph
+        st_bytes = B * NH * (d * d * 4 + (d * 4 if var == 1 else 0))
+        step_bytes = 2 * st_bytes + B * NH * (4 * d * 2 + 2 * 2) + (B * NH * 4 * 2 if var == 1 else 0)
+        # hand-off from the prefill: mlstm_final_state
+        for _ in range(args.warmup):
+            binding.final_state(x["k"], x["v"], saved, L, var, state=other)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            binding.final_state(x["k"], x["v"], saved, L, var, state=other)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        achieved = step_bytes / ms / 1e6
+        print(json.dumps({
+            "decode": "b8h32_d128_bf16", "cell": label, "ms_per_step": ms,
+            "tokens_per_s": B / ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "bytes_per_step": step_bytes},
+            "final_state_ms": f0.elapsed_time(f1) / args.steps,
+        }), flush=True)
+        del x, saved, state, other
+        torch.cuda.empty_cache()
+    return 0
+
+
 def sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev, B, NH, T, d, L, var, peaks):
     """Backward at one sweep point: mlstm_bwd timed like the forward, per kernel.
 
@@ -508,6 +585,8 @@ def main():
     ap.add_argument("--retnet", action="store_true",
                     help="retention (RetNet decays) through the SIG kernels at B8 H32 d128, "
                          "T from --sweep-t or the 128..16384 list")
+    ap.add_argument("--decode", action="store_true",
+                    help="one-token steps (generation) at B8 H32 d128, and the prefill hand-off")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (smaller captures for ncu; the default is the workload's B)")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -534,6 +613,8 @@ def main():
         return run_sweep(args)
     if args.retnet:
         return run_retnet(args)
+    if args.decode:
+        return run_decode(args)
 
     import torch
     import torch.distributed as dist

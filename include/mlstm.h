@@ -159,6 +159,54 @@ int mlstm_fwd_noalloc(const void* q, const void* k, const void* v,
                       int B, int NH, int T, int d_qk, int d_hv, int chunk,
                       int variant, int dtype, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Recurrent form: one token at a time, and the hand-off from a chunkwise
+ * forward to it.  "flash-linear-attention" README, the FusedRecurrent form
+ * (O(T), states on chip); "Tiled Flash Linear Attention", TFLA summary page,
+ * Approach (the mLSTM recurrence, exponential or sigmoid input gate, sigmoid
+ * forget gate, normaliser and max state for mLSTMexp).
+ *
+ * State buffer (device memory owned by the caller), per head, fp32, 256-byte
+ * aligned regions of size mlstm_state_size():
+ *   C [B*NH, d_qk, d_hv]  at offset 0; for EXP scaled by exp(-m)
+ *   n [B*NH, d_qk]        EXP only, next 256-byte boundary after C
+ *   m [B*NH]              EXP only, next 256-byte boundary after n
+ * The zero state (no token seen) is C = 0, n = 0, m = -inf.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of a state buffer (0 on an argument error). */
+size_t mlstm_state_size(int B, int NH, int d_qk, int d_hv, int variant);
+
+/* Write the zero state into `state` (enqueued on `stream`).  Errors:
+ * MLSTM_ERR_INVALID (NULL or misaligned state), MLSTM_ERR_UNSUPPORTED,
+ * MLSTM_ERR_CUDA. */
+int mlstm_state_zero(void* state, int B, int NH, int d_qk, int d_hv, int variant, void* stream);
+
+/* State after the last token of a sequence that mlstm_fwd processed with
+ * the same sizes, from its `saved` buffer (the state entering the last
+ * chunk, gate cumsums and max states) and its k, v: C_T = beta C_enter +
+ * sum_s w_s k_s v_s^T over the last chunk, n likewise, m_T the last max
+ * state.  Writes `state` (layout above); reads k, v, saved.  T = 0 writes
+ * the zero state.  Errors as mlstm_fwd. */
+int mlstm_final_state(const void* k, const void* v, const void* saved, void* state,
+                      int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                      int variant, int dtype, void* stream);
+
+/* One token of the recurrence for every head.  q, k [B, NH, d_qk] and
+ * v [B, NH, d_hv] in the I/O dtype; igate_pre, fgate_pre [B, NH] in the I/O
+ * dtype; h [B, NH, d_hv] out in the I/O dtype.  Reads state_in, writes
+ * state_out; the two must not overlap (MLSTM_ERR_INVALID), callers
+ * alternate two buffers.
+ *   SIG: C' = f C + i k v^T, h = C'^T q / sqrt(d_qk)
+ *   EXP: m' = max(log f + m, i~), C' = exp(log f + m - m') C + exp(i~ - m') k v^T,
+ *        n' likewise, h = C'^T q' / max(|n' . q'|, exp(-m'))
+ * with f = sigmoid(f~), i = sigmoid(i~) (SIG).  Arithmetic in fp32.
+ * Errors: MLSTM_ERR_INVALID (NULL, misaligned or overlapping buffers),
+ * MLSTM_ERR_UNSUPPORTED (sizes outside the chunkwise path's), MLSTM_ERR_CUDA. */
+int mlstm_step(const void* q, const void* k, const void* v, const void* igate_pre,
+               const void* fgate_pre, void* h, const void* state_in, void* state_out,
+               int B, int NH, int d_qk, int d_hv, int variant, int dtype, void* stream);
+
 /* Synchronise `stream` and report what the kernels enqueued so far found:
  * MLSTM_ERR_TIMEOUT if one of them gave up a bounded wait (its outputs are
  * then invalid; the flag is cleared by this call), MLSTM_ERR_CUDA on a CUDA

@@ -17,6 +17,8 @@ BF16 = 0
 FP32 = 1
 
 STATUS_OK = 0
+STATUS_INVALID = 1
+STATUS_UNSUPPORTED = 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmlstm.so")
@@ -57,6 +59,10 @@ EXPORTS = {
     "mlstm_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "mlstm_device_status": (ctypes.c_int, [_P]),
     "mlstm_fwd_noalloc": (ctypes.c_int, [_P] * 6 + _SIZES + [_P]),
+    "mlstm_state_size": (ctypes.c_size_t, [ctypes.c_int] * 5),
+    "mlstm_state_zero": (ctypes.c_int, [_P] + [ctypes.c_int] * 5 + [_P]),
+    "mlstm_final_state": (ctypes.c_int, [_P] * 4 + _SIZES + [_P]),
+    "mlstm_step": (ctypes.c_int, [_P] * 8 + [ctypes.c_int] * 6 + [_P]),
 }
 
 
@@ -242,6 +248,69 @@ def backward(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, *, wor
     if st != STATUS_OK:
         raise MLSTMError(st, "mlstm_bwd")
     return out
+
+
+# ---------------------------------------------------------------------------
+# Recurrent form: state buffers, hand-off from a forward pass, one-token steps
+# ---------------------------------------------------------------------------
+
+def state_views(state, B, NH, d_qk, d_hv, variant):
+    """C [B, NH, d_qk, d_hv] and, for EXP, n [B, NH, d_qk] and m [B, NH] views of a state
+    buffer (layout in include/mlstm.h)."""
+    import torch
+    BH = B * NH
+    c_bytes = BH * d_qk * d_hv * 4
+    out = {"C": state[:c_bytes].view(torch.float32).view(B, NH, d_qk, d_hv), "n": None, "m": None}
+    if variant == EXP:
+        off = (c_bytes + 255) // 256 * 256
+        out["n"] = state[off: off + BH * d_qk * 4].view(torch.float32).view(B, NH, d_qk)
+        off = (off + BH * d_qk * 4 + 255) // 256 * 256
+        out["m"] = state[off: off + BH * 4].view(torch.float32).view(B, NH)
+    return out
+
+
+def new_state(B, NH, d_qk, d_hv, variant, device, stream=None):
+    """A zero state (C = 0, n = 0, m = -inf) in a fresh uint8 buffer."""
+    import torch
+    nbytes = load().mlstm_state_size(B, NH, d_qk, d_hv, variant)
+    if nbytes == 0:
+        raise MLSTMError(STATUS_UNSUPPORTED, "mlstm_state_size")
+    state = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    st = load().mlstm_state_zero(state.data_ptr(), B, NH, d_qk, d_hv, variant, _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_state_zero")
+    return state
+
+
+def final_state(k, v, saved, chunk, variant, *, state=None, stream=None):
+    """State after the last token of a forward that kept ``saved`` (same sizes)."""
+    import torch
+    B, NH, T, d_qk = k.shape
+    d_hv = v.shape[-1]
+    if state is None:
+        state = torch.empty(load().mlstm_state_size(B, NH, d_qk, d_hv, variant), dtype=torch.uint8,
+                            device=k.device)
+    st = load().mlstm_final_state(k.data_ptr(), v.data_ptr(), saved.data_ptr(), state.data_ptr(),
+                                  *problem_sizes(k, v, chunk, variant), _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_final_state")
+    return state
+
+
+def step(q, k, v, igate_pre, fgate_pre, state_in, state_out, variant, *, h=None, stream=None):
+    """One token: q, k [B, NH, d_qk], v [B, NH, d_hv], gates [B, NH]; returns h [B, NH, d_hv]."""
+    import torch
+    _check({"q": q, "k": k, "v": v, "igate_pre": igate_pre, "fgate_pre": fgate_pre}, q.dtype)
+    B, NH, d_qk = q.shape
+    d_hv = v.shape[-1]
+    if h is None:
+        h = torch.empty((B, NH, d_hv), dtype=q.dtype, device=q.device)
+    st = load().mlstm_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
+                           fgate_pre.data_ptr(), h.data_ptr(), state_in.data_ptr(), state_out.data_ptr(),
+                           B, NH, d_qk, d_hv, int(variant), _dtype_code(q), _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_step")
+    return h
 
 
 # ---------------------------------------------------------------------------

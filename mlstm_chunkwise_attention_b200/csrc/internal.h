@@ -85,4 +85,14 @@ cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t
 cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_state_error(unsigned int* flag);
 
+// recurrent-form kernels (recurrent.cu)
+cudaError_t launch_final_state(const Problem& p, const void* k, const void* v, const float* b,
+                               const float* li, const float* m, const void* C, const float* n,
+                               float* Cout, float* nout, float* mout, cudaStream_t s);
+cudaError_t launch_step(const Problem& p, const void* q, const void* k, const void* v,
+                        const void* ig, const void* fg, void* h, const float* Cin, const float* nin,
+                        const float* min_, float* Cout, float* nout, float* mout, cudaStream_t s);
+cudaError_t launch_state_zero(int BH, int dqk, int dhv, bool exp_variant, float* C, float* n, float* m,
+                              cudaStream_t s);
+
 }  // namespace mlstm

@@ -315,6 +315,107 @@ int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre
   return run_plan(steps, n, p, a, s);
 }
 
+}  // extern "C"
+
+namespace {
+
+struct StateLayout {
+  size_t C, n, m, total;
+};
+
+// Recurrent state of one call: C [BH, d_qk, d_hv], then (EXP) n [BH, d_qk] and m [BH],
+// fp32, 256-byte aligned regions.
+StateLayout state_layout(int BH, int dqk, int dhv, bool exp_variant) {
+  StateLayout L;
+  L.C = 0;
+  size_t off = align256((size_t)BH * dqk * dhv * 4);
+  L.n = off;
+  if (exp_variant) off = align256(off + (size_t)BH * dqk * 4);
+  L.m = off;
+  if (exp_variant) off = align256(off + (size_t)BH * 4);
+  L.total = off;
+  return L;
+}
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + bytes && y < x + bytes;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mlstm_state_size(int B, int NH, int d_qk, int d_hv, int variant) {
+  if (check_sizes(B, NH, 1, d_qk, d_hv, 64, variant, MLSTM_FP32) != MLSTM_OK) return 0;
+  return state_layout(B * NH, d_qk, d_hv, variant == MLSTM_EXP).total;
+}
+
+int mlstm_state_zero(void* state, int B, int NH, int d_qk, int d_hv, int variant, void* stream) {
+  int st = check_sizes(B, NH, 1, d_qk, d_hv, 64, variant, MLSTM_FP32);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (!state || misaligned(state)) return MLSTM_ERR_INVALID;
+  const bool e = variant == MLSTM_EXP;
+  const StateLayout L = state_layout(B * NH, d_qk, d_hv, e);
+  char* base = (char*)state;
+  return cuda_status(mlstm::launch_state_zero(B * NH, d_qk, d_hv, e, (float*)(base + L.C),
+                                              (float*)(base + L.n), (float*)(base + L.m),
+                                              (cudaStream_t)stream),
+                     "state_zero");
+}
+
+int mlstm_final_state(const void* k, const void* v, const void* saved, void* state, int B, int NH,
+                      int T, int d_qk, int d_hv, int chunk, int variant, int dtype, void* stream) {
+  int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (T == 0) return mlstm_state_zero(state, B, NH, d_qk, d_hv, variant, stream);
+  if (!k || !v || !saved || !state) return MLSTM_ERR_INVALID;
+  if (misaligned(k) || misaligned(v) || misaligned(saved) || misaligned(state)) return MLSTM_ERR_INVALID;
+  const Problem p = make_problem(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
+  mlstm_saved_layout_t L;
+  saved_layout(p, &L);
+  const StateLayout S = state_layout(p.BH, d_qk, d_hv, p.exp_variant());
+  const char* sv = (const char*)saved;
+  char* out = (char*)state;
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_final_state");
+  if (st != MLSTM_OK) return st;
+  return cuda_status(
+      mlstm::launch_final_state(p, k, v, (const float*)(sv + L.gate_b), (const float*)(sv + L.gate_li),
+                                p.exp_variant() ? (const float*)(sv + L.gate_m) : nullptr,
+                                sv + L.state_c,
+                                p.exp_variant() ? (const float*)(sv + L.state_n) : nullptr,
+                                (float*)(out + S.C), (float*)(out + S.n), (float*)(out + S.m),
+                                (cudaStream_t)stream),
+      "final_state");
+}
+
+int mlstm_step(const void* q, const void* k, const void* v, const void* igate_pre,
+               const void* fgate_pre, void* h, const void* state_in, void* state_out, int B,
+               int NH, int d_qk, int d_hv, int variant, int dtype, void* stream) {
+  int st = check_sizes(B, NH, 1, d_qk, d_hv, 64, variant, dtype);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (!q || !k || !v || !igate_pre || !fgate_pre || !h || !state_in || !state_out)
+    return MLSTM_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, h, state_in, state_out};
+  for (const void* ptr : ptrs)
+    if (misaligned(ptr)) return MLSTM_ERR_INVALID;
+  const Problem p = make_problem(B, NH, 1, d_qk, d_hv, 64, variant, dtype);
+  const StateLayout S = state_layout(p.BH, d_qk, d_hv, p.exp_variant());
+  if (overlaps(state_in, state_out, S.total)) return MLSTM_ERR_INVALID;
+  const char* si = (const char*)state_in;
+  char* so = (char*)state_out;
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_step");
+  if (st != MLSTM_OK) return st;
+  return cuda_status(
+      mlstm::launch_step(p, q, k, v, igate_pre, fgate_pre, h, (const float*)(si + S.C),
+                         (const float*)(si + S.n), (const float*)(si + S.m), (float*)(so + S.C),
+                         (float*)(so + S.n), (float*)(so + S.m), (cudaStream_t)stream),
+      "step");
+}
+
 const char* mlstm_status_string(int status) {
   switch (status) {
     case MLSTM_OK: return "ok";

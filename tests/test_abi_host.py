@@ -129,3 +129,31 @@ def test_status_strings(lib):
     for code in range(6):
         assert B.mlstm_status_string(code)
     assert B.mlstm_status_string(99) == "unknown status"
+
+
+def test_state_layout_and_argument_errors(lib):
+    """Recurrent-state entry points: sizes, and argument errors returned before any launch."""
+    for variant in (B.SIG, B.EXP):
+        nb = lib.mlstm_state_size(2, 3, 128, 64, variant)
+        c = 2 * 3 * 128 * 64 * 4
+        if variant == B.SIG:
+            assert nb == c
+        else:  # C, then n and m on 256-byte boundaries
+            n_off = (c + 255) // 256 * 256
+            m_off = (n_off + 6 * 128 * 4 + 255) // 256 * 256
+            assert nb == (m_off + 6 * 4 + 255) // 256 * 256
+    assert lib.mlstm_state_size(2, 3, 100, 64, B.EXP) == 0  # unsupported d_qk
+    fake, other = 0x10000, 0x20000  # aligned addresses, never dereferenced
+    nb = lib.mlstm_state_size(1, 2, 64, 64, B.EXP)
+    args = (fake, fake, fake, fake, fake, fake)
+    # overlapping state_in / state_out
+    assert lib.mlstm_step(*args, fake, fake + 256, 1, 2, 64, 64, B.EXP, B.BF16, None) == B.STATUS_INVALID
+    assert nb > 256
+    # NULL state
+    assert lib.mlstm_step(*args, None, other, 1, 2, 64, 64, B.EXP, B.BF16, None) == B.STATUS_INVALID
+    # misaligned
+    assert lib.mlstm_state_zero(fake + 4, 1, 2, 64, 64, B.EXP, None) == B.STATUS_INVALID
+    # empty problems are no-ops
+    assert lib.mlstm_state_zero(None, 0, 2, 64, 64, B.EXP, None) == 0
+    assert lib.mlstm_step(*[None] * 8, 0, 2, 64, 64, B.SIG, B.BF16, None) == 0
+    assert lib.mlstm_final_state(None, None, None, None, 0, 2, 5, 64, 64, 64, B.SIG, B.BF16, None) == 0
