@@ -34,9 +34,10 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 enum { KDQ = 0, KDK = 1, KDV = 2 };
 
-// NXBUF score buffers in TMEM: 1 when every row tile has a single partner tile
-// (chunk 128), so the CTA fits in 256 TMEM columns and ~99 KB of shared memory
-// and two CTAs share an SM; 2 otherwise (the next score overlaps the transform).
+// NXBUF score buffers in TMEM: 1 up to chunk 1024, so the CTA fits in 256 TMEM
+// columns and ~100-108 KB of shared memory and two CTAs share an SM (one CTA's
+// serial phases overlap the other's tiles); 2 for longer chunks, where only one
+// CTA fits and the next score overlaps the transform instead.
 template <int D1, int D2S, bool G_MN, int NXBUF>
 struct BwdTcCfg {
   static constexpr int STAGES = NXBUF == 1 ? 2 : 4;
@@ -127,30 +128,6 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tc::tmem_relinquish();
-  }
-  // partner factors of every partner row this tile meets, and the inter row vector
-  {
-    const int pbase = pj0 * 128;
-    for (int pi = threadIdx.x; pi < np * 128; pi += blockDim.x) {
-      const int p = pbase + pi;
-      const bool ok = p < len;
-      float cexp = -INFINITY, eadd = 0.f;
-      if (ok) {
-        if (R_IS_QUERY) {
-          cexp = (P.li[tok0 + p] - P.b[tok0 + p]) * kLog2e;
-        } else {
-          const float mt = EXPV ? P.m[tok0 + p] : 0.f;
-          const float invd = EXPV ? P.inv_den[tok0 + p] : 1.f;
-          cexp = (P.b[tok0 + p] - mt) * kLog2e + log2f(invd);
-          if (KIND == KDK && EXPV) eadd = P.da[tok0 + p] / invd;
-        }
-      }
-      pfC[pi] = cexp;
-      pfE[pi] = eadd;
-    }
-    if (KIND != KDV && EXPV && has_inter)
-      for (int i = threadIdx.x; i < D2S; i += blockDim.x)
-        rowvec[i] = P.rowvec[((size_t)bh * P.NC + c) * P.dqk + col0 + i];
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -296,6 +273,31 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     }
   } else {
     // ------------------------------------------------------------ tile rows
+    // Partner factors of every partner row this tile meets, and the inter row vector,
+    // loaded by the four transform warps while the producer already streams operands.
+    {
+      const int pbase = pj0 * 128;
+      for (int pi = threadIdx.x - 64; pi < np * 128; pi += 128) {
+        const int p = pbase + pi;
+        float cexp = -INFINITY, eadd = 0.f;
+        if (p < len) {
+          if (R_IS_QUERY) {
+            cexp = (P.li[tok0 + p] - P.b[tok0 + p]) * kLog2e;
+          } else {
+            const float mt = EXPV ? P.m[tok0 + p] : 0.f;
+            const float invd = EXPV ? P.inv_den[tok0 + p] : 1.f;
+            cexp = (P.b[tok0 + p] - mt) * kLog2e + log2f(invd);
+            if (KIND == KDK && EXPV) eadd = P.da[tok0 + p] / invd;
+          }
+        }
+        pfC[pi] = cexp;
+        pfE[pi] = eadd;
+      }
+      if (KIND != KDV && EXPV && has_inter)
+        for (int i = threadIdx.x - 64; i < D2S; i += 128)
+          rowvec[i] = P.rowvec[((size_t)bh * P.NC + c) * P.dqk + col0 + i];
+      tc::named_bar_sync(1, 128);
+    }
     const int row = 32 * (warp & 3) + lane;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int rl = r0 + row;
@@ -531,9 +533,12 @@ static cudaError_t dispatch_kind(const Problem& p, const BwdArgs& a, cudaStream_
   const int d1 = (KIND == KDV) ? p.dqk : p.dhv;
   const int dout = (KIND == KDV) ? p.dhv : p.dqk;
   const bool wide = dout >= 128;
+  // One score buffer (256 TMEM columns) lets two CTAs share an SM, so one CTA's
+  // prologue, inter term and epilogue overlap the other's tiles; that needs both
+  // CTAs' shared memory (about 100 KB plus 8 bytes per chunk token) to fit.
 #define MLSTM_BWD_TC_D1(D1)                                                                  \
   if (d1 == D1) {                                                                            \
-    if (p.L == 128)                                                                          \
+    if (p.L <= 1024)                                                                         \
       return wide ? launch_kind<KIND, D1, 128, GMN, EXPV, 1>(p, a, s)                        \
                   : launch_kind<KIND, D1, 64, GMN, EXPV, 1>(p, a, s);                        \
     return wide ? launch_kind<KIND, D1, 128, GMN, EXPV, 2>(p, a, s)                          \
