@@ -37,26 +37,30 @@ enum { KDQ = 0, KDK = 1, KDV = 2 };
 // NXBUF score buffers in TMEM: 1 up to chunk 1024, so the CTA fits in 256 TMEM
 // columns and ~100-108 KB of shared memory and two CTAs share an SM (one CTA's
 // serial phases overlap the other's tiles); 2 for longer chunks, where only one
-// CTA fits and the next score overlaps the transform instead.
+// CTA fits and the next score overlaps the transform instead.  The transformed
+// tile Y is written back over its score as packed bf16 and read from TMEM by the
+// accumulate product, so shared memory holds only the operand ring.
 template <int D1, int D2S, bool G_MN, int NXBUF>
 struct BwdTcCfg {
-  static constexpr int STAGES = NXBUF == 1 ? 2 : 4;
+  static constexpr int STAGES = NXBUF == 1 ? 3 : 4;
   static constexpr int SLOT = 16384;  // one 128 x 64 bf16 block
   static constexpr int STAGE_BYTES = 2 * SLOT;
   static constexpr int NKB = D1 / 64;  // K-blocks of the score GEMM and the inter GEMM
   static constexpr int EB = D2S / 64;  // 64-column blocks of E and of the output slice
-  static constexpr int OFF_RING = 0;
-  static constexpr int OFF_Y = STAGES * STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_Y + 2 * SLOT;
+  static constexpr int OFF_RING = 0;   // ring stage 0 also stages the result tile at the end
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
   static constexpr int NBAR = 16;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_RV = OFF_TMEM + 16;
-  static constexpr int OFF_PF = OFF_RV + D2S * 4;  // partner factors, 2 x L floats
+  static constexpr int OFF_PW = OFF_RV + D2S * 4;   // per-warp partner factors, 4 x 128 floats
+  static constexpr int OFF_PF = OFF_PW + 4 * 128 * 4;  // partner factors: 2 x L, then L / 32 (>= 4)
   static constexpr uint32_t TMEM_COLS = NXBUF == 1 ? 256 : 512;  // X buffers, then Acc
   static constexpr uint32_t ACC_COL = NXBUF * 128;
   static constexpr uint32_t G_BYTES = G_MN ? (uint32_t)EB * 8192u : (uint32_t)D2S * 128u;
   static constexpr uint32_t E_BYTES = (uint32_t)EB * SLOT;
-  static size_t smem_bytes(int L) { return 1024 + OFF_PF + (size_t)2 * L * 4; }
+  static size_t smem_bytes(int L) {
+    return 1024 + OFF_PF + ((size_t)2 * L + (L / 32 > 4 ? L / 32 : 4)) * 4;
+  }
 };
 
 enum {
@@ -71,7 +75,7 @@ struct BwdTcParams {
   const bf16* dot_src;  // dq: q; dk: k (the per-token dot product with the result)
   bf16* out;            // dq, dk or dv [BH, T, d_out]
   float* pdot;          // dq: pq; dk: pk (atomically accumulated)
-  int T, L, NC, BH, ntq, d_out, dqk;
+  int T, L, NC, BH, ntq, nsl, d_out, dqk;  // nsl: output column slices of D2S
   float scale, log2_scale;
 };
 
@@ -85,11 +89,13 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   constexpr bool R_IS_QUERY = (KIND == KDQ);
   constexpr int ST = Cfg::STAGES;
 
-  const int per = P.BH * P.NC;
-  // heaviest row tiles first: dq tiles near the chunk end, dk/dv tiles near its start
-  const int order = (int)(blockIdx.x / per);
+  // The row tiles (and output column slices) of one chunk are consecutive CTAs, so
+  // the partner tiles they all stream stay in L2 between them; inside a chunk the
+  // heaviest tiles go first (dq tiles near the chunk end, dk/dv tiles near its start).
+  const int slice = (int)(blockIdx.x % P.nsl);
+  const int order = (int)((blockIdx.x / P.nsl) % P.ntq);
   const int it_tile = R_IS_QUERY ? P.ntq - 1 - order : order;
-  const int rest = (int)(blockIdx.x % per);
+  const int rest = (int)(blockIdx.x / P.nsl / P.ntq);
   const int bh = rest / P.NC, c = rest % P.NC;
   const int c0 = c * P.L;
   const int len = min(P.L, P.T - c0);
@@ -98,7 +104,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   if (r0 >= len) return;
   // an earlier CTA gave up: the whole block leaves together
   if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_bwd_error != 0u)) return;
-  const int col0 = blockIdx.y * D2S;
+  const int col0 = slice * D2S;
   const size_t tok0 = (size_t)bh * P.T + c0;
   // partner tiles: dq: 0..it_tile; dk, dv: it_tile..nt_len-1
   const int pj0 = R_IS_QUERY ? 0 : it_tile;
@@ -109,12 +115,14 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem + Cfg::OFF_RING;
-  uint8_t* sY = smem + Cfg::OFF_Y;
+  uint8_t* sOut = ring;  // result staging tile, once every product is done
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
   float* rowvec = reinterpret_cast<float*>(smem + Cfg::OFF_RV);
   float* pfC = reinterpret_cast<float*>(smem + Cfg::OFF_PF);  // partner exponent term
-  float* pfE = pfC + P.L;                                      // partner additive term (dk)
+  float* pfE = pfC + P.L;  // partner additive term (dk) or separable key factor (dq)
+  float* pfM = pfE + P.L;  // dq: stabiliser of every 32-key partner block
+  float* pfW = reinterpret_cast<float*>(smem + Cfg::OFF_PW);  // dk, dv: this warp's partner factors
   const volatile unsigned int* abort_flag = &g_tc_bwd_error;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,7 +148,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     // ------------------------------------------------------------ producer
     // Every operand goes through one ring, in the order the MMA thread consumes it:
     // inter (A, G_hi), (A, G_lo) per K-block; score(0); then per partner jj:
-    // score(jj + 1) if any, E(jj).
+    // E(jj), score(jj + 1) with one score buffer, score(jj + 1), E(jj) with two.
     if (lane == 0) {
       tc::prefetch_tmap(&tmA);
       tc::prefetch_tmap(&tmB);
@@ -183,16 +191,24 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
           }
         }
       }
-      if (ok) ok = load_score(0);
-      for (int jj = 0; jj < np && ok; ++jj) {
-        if (jj + 1 < np) ok = load_score(jj + 1);
-        if (!ok) break;
+      auto load_e = [&](int jj) -> bool {
         uint64_t* fb;
         uint8_t* stg = acquire(Cfg::E_BYTES, fb);
-        if (!stg) { ok = false; break; }
+        if (!stg) return false;
         const int prow = c0 + (pj0 + jj) * 128;
         for (int eb = 0; eb < Cfg::EB; ++eb)
           tc::tma_load_3d(stg + eb * Cfg::SLOT, &tmE, fb, col0 + eb * 64, prow, bh);
+        return true;
+      };
+      if (ok) ok = load_score(0);
+      for (int jj = 0; jj < np && ok; ++jj) {
+        if (NXBUF == 1) {
+          ok = load_e(jj);
+          if (ok && jj + 1 < np) ok = load_score(jj + 1);
+        } else {
+          if (jj + 1 < np) ok = load_score(jj + 1);
+          if (ok) ok = load_e(jj);
+        }
       }
       // stay until the last copies this thread issued have landed
       if (ok && it > 0)
@@ -204,7 +220,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
       constexpr uint32_t idX = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idAcc = tc::idesc_bf16(128, D2S, false, true);
       constexpr uint32_t idG = tc::idesc_bf16(128, D2S, false, G_MN);
-      const uint32_t aRing = tc::smem_u32(ring), aY = tc::smem_u32(sY);
+      const uint32_t aRing = tc::smem_u32(ring);
       uint32_t it = 0;
       // wait for the next ring entry; returns its shared address (0 on timeout)
       auto next_stage = [&]() -> uint32_t {
@@ -248,26 +264,30 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         tc::tc_commit(&bar[BB_X0 + (jj % NXBUF)]);
         return true;
       };
+      // Acc += Y E_jj, Y read from TMEM (packed bf16 over its score, 16 partners per
+      // 8 columns).  MMAs of this thread run in issue order, so a later score may
+      // overwrite the columns this product reads.
+      auto issue_acc = [&](int jj) -> bool {
+        const uint32_t st = next_stage();  // E(jj)
+        if (!st) return false;
+        const uint32_t tY = tX0 + (jj % NXBUF) * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          tc::mma_bf16_ts(tAcc, tY + 8 * k, tc::sdesc_sw128(st + k * 2048, Cfg::SLOT, 1024), idAcc,
+                          (has_inter || jj > 0 || k > 0));
+        release();
+        return true;
+      };
       if (ok) ok = issue_score(0);
       for (int jj = 0; jj < np && ok; ++jj) {
-        // one X buffer: the next score waits until the transform has read this one;
-        // two buffers: the other one was released by the transform of jj - 1
-        if (NXBUF == 1) ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag);
-        if (ok && jj + 1 < np) ok = issue_score(jj + 1);
-        if (ok && NXBUF != 1) ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag);
+        // one X buffer: the next score follows this accumulate (it overwrites Y);
+        // two buffers: the next score goes to the buffer the accumulate of jj - 1 read
+        if (NXBUF != 1 && jj + 1 < np) ok = issue_score(jj + 1);
+        if (ok) ok = tc::mbar_wait(&bar[BB_Y], jj & 1, abort_flag);
         if (ok && jj == 0 && has_inter) ok = tc::mbar_wait(&bar[BB_ACC], 0, abort_flag);
-        if (!ok) break;
-        const uint32_t st = next_stage();  // E(jj)
-        if (!st) { ok = false; break; }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t offy = (k >> 2) * Cfg::SLOT + (k & 3) * 32;
-          tc::mma_bf16_ss(tAcc, tc::sdesc_sw128(aY + offy, 16, 1024),
-                          tc::sdesc_sw128(st + k * 2048, Cfg::SLOT, 1024), idAcc,
-                          (has_inter || jj > 0 || k > 0));
-        }
-        release();
-        tc::tc_commit(&bar[BB_YE]);
+        if (ok) tc::tc_fence_after();
+        if (ok) ok = issue_acc(jj);
+        if (ok && NXBUF == 1 && jj + 1 < np) ok = issue_score(jj + 1);
       }
       tc::tc_commit(&bar[BB_DONE]);
     }
@@ -297,6 +317,21 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         for (int i = threadIdx.x - 64; i < D2S; i += 128)
           rowvec[i] = P.rowvec[((size_t)bh * P.NC + c) * P.dqk + col0 + i];
       tc::named_bar_sync(1, 128);
+      if (R_IS_QUERY) {
+        // Off-diagonal tiles split the decay: 2^(A_t + B_s) = 2^(A_t + M) 2^(B_s - M), with
+        // M the largest key term B_s of the key's 32-block (so the key factor is <= 1 and
+        // the row factor is at most the row's 1 / den).  One warp per block.
+        for (int blk = warp - 2; blk < np * 4; blk += 4) {
+          const float v = pfC[blk * 32 + lane];
+          float mx = v;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (mx == -INFINITY) mx = 0.f;  // a block wholly past the sequence end
+          if (lane == 0) pfM[blk] = mx;
+          pfE[blk * 32 + lane] = tc::ex2(v - mx);
+        }
+        tc::named_bar_sync(1, 128);
+      }
     }
     const int row = 32 * (warp & 3) + lane;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -334,7 +369,17 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         rvc = rs;
       }
     }
-    const uint32_t aY = tc::smem_u32(sY);
+    // dk, dv: this warp's 32 rows are one key block; its stabiliser M (the same value the
+    // dq kernel takes for the block) and the row's separable factor 2^(B_s - M)
+    float Mrow = 0.f, grow = 0.f;
+    if (!R_IS_QUERY) {
+      float mx = Rexp;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, o));
+      Mrow = mx == -INFINITY ? 0.f : mx;
+      grow = tc::ex2(Rexp - Mrow);
+    }
+    const uint32_t aOut = tc::smem_u32(sOut);
 
     if (has_inter) {
       ok = __all_sync(full, tc::mbar_wait(&bar[BB_INTER], 0, abort_flag));
@@ -360,55 +405,92 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
 
     for (int jj = 0; jj < np && ok; ++jj) {
       ok = __all_sync(full, tc::mbar_wait(&bar[BB_X0 + (jj % NXBUF)], (jj / NXBUF) & 1, abort_flag));
-      if (ok && jj > 0) ok = __all_sync(full, tc::mbar_wait(&bar[BB_YE], (jj - 1) & 1, abort_flag));
       if (!ok) break;
       tc::tc_fence_after();
       const bool diag = (pj0 + jj) == it_tile;
       const float* pc = pfC + jj * 128;
       const float* pe = pfE + jj * 128;
       const uint32_t tX = tX0 + (jj % NXBUF) * 128;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        float x[32];
-        tc::tmem_ld32(tX + lane_base + ch * 32, x);
-        uint32_t pk[16];
+      float* fw = pfW + (warp & 3) * 128;
+      if (!diag && !R_IS_QUERY) {
+        // partner factors 2^(A_t + M) of this warp's key block (t-side term first, as in dq)
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float y[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int p = ch * 32 + i + u;
-            float add = 0.f;
-            if (KIND == KDQ) add = eRow;
-            if (KIND == KDK) add = pe[p];
-            // t-side term first, then the s-side term, in every kernel
-            const float ex = R_IS_QUERY ? (Rexp + pc[p]) : (pc[p] + Rexp);
-            float val = (x[i + u] + add) * tc::ex2(ex);
-            const bool masked = R_IS_QUERY ? (diag && p > row) : (diag && p < row);
-            y[u] = masked ? 0.f : val;
-          }
-          pk[i >> 1] = tc::pack_bf16(y[0], y[1]);
-        }
-        const int kb = ch >> 1;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int lc = (ch & 1) * 4 + q4;
-          const uint32_t addr = aY + kb * Cfg::SLOT + row * 128 + ((lc ^ (row & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * q4]),
-                       "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3])
-                       : "memory");
-        }
+        for (int u = 0; u < 4; ++u) fw[lane + 32 * u] = tc::ex2(pc[lane + 32 * u] + Mrow);
+        __syncwarp();
       }
-      tc::fence_proxy_async_smem();
+      // one 32-column chunk: gates, mask and normaliser terms, packed bf16 into TMEM
+      // columns [16 ch, 16 ch + 16) of the score buffer (columns already read)
+      auto transform_chunk = [&](const uint32_t (&xr)[32], int ch) {
+        uint32_t pk[16];
+        if (diag) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float y[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int p = ch * 32 + i + u;
+              float add = 0.f;
+              if (KIND == KDQ) add = eRow;
+              if (KIND == KDK) add = pe[p];
+              // t-side term first, then the s-side term, in every kernel
+              const float ex = R_IS_QUERY ? (Rexp + pc[p]) : (pc[p] + Rexp);
+              const float val = (__uint_as_float(xr[i + u]) + add) * tc::ex2(ex);
+              const bool masked = R_IS_QUERY ? (p > row) : (p < row);
+              y[u] = masked ? 0.f : val;
+            }
+            pk[i >> 1] = tc::pack_bf16(y[0], y[1]);
+          }
+        } else {
+          // y = ((x + e) f) g with f the t-side and g the s-side factor: the same fp32
+          // operations, so the same bf16 values, in the dq and dk kernels
+          const float fq = R_IS_QUERY ? tc::ex2(Rexp + pfM[jj * 4 + ch]) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const int p = ch * 32 + i;
+            const float4 g4 = *reinterpret_cast<const float4*>((R_IS_QUERY ? pe : fw) + p);
+            float4 e4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (KIND == KDK) e4 = *reinterpret_cast<const float4*>(pe + p);
+            const float gv[4] = {g4.x, g4.y, g4.z, g4.w}, ev[4] = {e4.x, e4.y, e4.z, e4.w};
+            float y[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float xv = __uint_as_float(xr[i + u]);
+              if (KIND == KDQ) y[u] = ((xv + eRow) * fq) * gv[u];
+              else if (KIND == KDK) y[u] = ((xv + ev[u]) * gv[u]) * grow;
+              else y[u] = (xv * gv[u]) * grow;
+            }
+            pk[i >> 1] = tc::pack_bf16(y[0], y[1]);
+            pk[(i >> 1) + 1] = tc::pack_bf16(y[2], y[3]);
+          }
+        }
+        tc::tmem_st16_async(tX + lane_base + 16 * ch, pk);
+      };
+      // the next chunk's TMEM load is in flight while this one is transformed
+      uint32_t xa[32], xb[32];
+      tc::tmem_ld32_async(tX + lane_base, xa);
+      tc::tmem_wait_ld(xa);
+      tc::tmem_ld32_async(tX + lane_base + 32, xb);
+      transform_chunk(xa, 0);
+      tc::tmem_wait_ld(xb);
+      tc::tmem_ld32_async(tX + lane_base + 64, xa);
+      transform_chunk(xb, 1);
+      tc::tmem_wait_ld(xa);
+      tc::tmem_ld32_async(tX + lane_base + 96, xb);
+      transform_chunk(xa, 2);
+      tc::tmem_wait_ld(xb);
+      transform_chunk(xb, 3);
+      tc::tmem_wait_st();
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[BB_Y]);
     }
 
     if (ok) ok = __all_sync(full, tc::mbar_wait(&bar[BB_DONE], 0, abort_flag));
     if (ok) {
-      // the result tile goes through the (now idle) Y tile and one TMA store per
-      // 64-column block; rows past the sequence end are clipped by the TMA unit
+      // the result tile goes through the (now idle) first ring stage and one TMA store
+      // per 64-column block; rows past the sequence end are clipped by the TMA unit
       tc::tc_fence_after();
+      tc::fence_proxy_async_smem();
       const float fin = (KIND == KDV) ? 1.f : P.scale;
       const bf16* drow = (KIND != KDV) ? P.dot_src + tok * P.dqk + col0 : nullptr;
       float dot = 0.f;
@@ -432,7 +514,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
             }
           }
           const int col = ch * 32 + q4 * 8, blk = col >> 6, lc = (col & 63) >> 3;
-          const uint32_t addr = aY + blk * Cfg::SLOT + row * 128 + ((lc ^ (row & 7)) << 4);
+          const uint32_t addr = aOut + blk * Cfg::SLOT + row * 128 + ((lc ^ (row & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
                        "r"(tc::pack_bf16(g[0], g[1])), "r"(tc::pack_bf16(g[2], g[3])),
                        "r"(tc::pack_bf16(g[4], g[5])), "r"(tc::pack_bf16(g[6], g[7]))
@@ -446,7 +528,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         ok = tc::mbar_wait(&bar[BB_STG], 0, abort_flag);
         if (ok) {
           for (int blk = 0; blk < Cfg::EB; ++blk)
-            tc::tma_store_3d(&tmOut, sY + blk * Cfg::SLOT, col0 + blk * 64, c0 + r0, bh);
+            tc::tma_store_3d(&tmOut, sOut + blk * Cfg::SLOT, col0 + blk * 64, c0 + r0, bh);
           tc::bulk_commit_group();
           tc::bulk_wait_all();
         }
@@ -522,7 +604,8 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   auto kern = intra_bwd_tc_kernel<KIND, D1, D2S, G_MN, EXPV, NXBUF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(p.BH * p.NC * P.ntq), (unsigned)(P.d_out / D2S)), block(192);
+  P.nsl = P.d_out / D2S;
+  dim3 grid((unsigned)(p.BH * p.NC * P.ntq * P.nsl)), block(192);
   kern<<<grid, block, smem, s>>>(tA, tB, tE, tGh, tGl, tO, P);
   return cudaGetLastError();
 }
