@@ -296,22 +296,36 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     // Partner factors of every partner row this tile meets, and the inter row vector,
     // loaded by the four transform warps while the producer already streams operands.
     {
-      const int pbase = pj0 * 128;
-      for (int pi = threadIdx.x - 64; pi < np * 128; pi += 128) {
-        const int p = pbase + pi;
-        float cexp = -INFINITY, eadd = 0.f;
-        if (p < len) {
-          if (R_IS_QUERY) {
-            cexp = (P.li[tok0 + p] - P.b[tok0 + p]) * kLog2e;
-          } else {
-            const float mt = EXPV ? P.m[tok0 + p] : 0.f;
-            const float invd = EXPV ? P.inv_den[tok0 + p] : 1.f;
-            cexp = (P.b[tok0 + p] - mt) * kLog2e + log2f(invd);
-            if (KIND == KDK && EXPV) eadd = P.da[tok0 + p] / invd;
-          }
+      // eight partners per thread at a time: all their loads issue before any store
+      const int pbase = pj0 * 128, npart = np * 128;
+      for (int pi0 = threadIdx.x - 64; pi0 < npart; pi0 += 8 * 128) {
+        float g0[8], g1[8], g2[8], g3[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int pi = pi0 + u * 128, p = pbase + pi;
+          const bool in = pi < npart && p < len;
+          const size_t t = tok0 + (in ? p : 0);
+          g0[u] = in ? P.b[t] : 0.f;
+          g1[u] = in ? (R_IS_QUERY ? P.li[t] : (EXPV ? P.m[t] : 0.f)) : 0.f;
+          g2[u] = (in && !R_IS_QUERY && EXPV) ? P.inv_den[t] : 1.f;
+          g3[u] = (in && KIND == KDK && EXPV) ? P.da[t] : 0.f;
         }
-        pfC[pi] = cexp;
-        pfE[pi] = eadd;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int pi = pi0 + u * 128, p = pbase + pi;
+          if (pi >= npart) break;
+          float cexp = -INFINITY, eadd = 0.f;
+          if (p < len) {
+            if (R_IS_QUERY) {
+              cexp = (g1[u] - g0[u]) * kLog2e;
+            } else {
+              cexp = (g0[u] - g1[u]) * kLog2e + log2f(g2[u]);
+              if (KIND == KDK && EXPV) eadd = g3[u] / g2[u];
+            }
+          }
+          pfC[pi] = cexp;
+          pfE[pi] = eadd;
+        }
       }
       if (KIND != KDV && EXPV && has_inter)
         for (int i = threadIdx.x - 64; i < D2S; i += 128)
@@ -412,7 +426,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
       const float* pe = pfE + jj * 128;
       const uint32_t tX = tX0 + (jj % NXBUF) * 128;
       float* fw = pfW + (warp & 3) * 128;
-      if (!diag && !R_IS_QUERY) {
+      if (!R_IS_QUERY) {
         // partner factors 2^(A_t + M) of this warp's key block (t-side term first, as in dq)
         __syncwarp();
 #pragma unroll
@@ -422,8 +436,19 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
       // one 32-column chunk: gates, mask and normaliser terms, packed bf16 into TMEM
       // columns [16 ch, 16 ch + 16) of the score buffer (columns already read)
       auto transform_chunk = [&](const uint32_t (&xr)[32], int ch) {
+        // 32 x 32 sub-blocks: the warp's row block against column block ch.  On the
+        // diagonal tile, the diagonal sub-block takes every element's own exponent and
+        // the causal mask, the sub-blocks on the far side of it are zero, and the rest
+        // use the separable form like every other tile (dq and dk classify each
+        // (query block, key block) pair alike).
+        const int wb = warp & 3;
+        const bool own = diag && ch == wb;
+        const bool zero = diag && (R_IS_QUERY ? ch > wb : ch < wb);
         uint32_t pk[16];
-        if (diag) {
+        if (zero) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = 0u;
+        } else if (own) {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             float y[2];
@@ -443,25 +468,33 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
           }
         } else {
           // y = ((x + e) f) g with f the t-side and g the s-side factor: the same fp32
-          // operations, so the same bf16 values, in the dq and dk kernels
+          // operations (two lanes at a time, each rounded as alone), so the same bf16
+          // values, in the dq and dk kernels
           const float fq = R_IS_QUERY ? tc::ex2(Rexp + pfM[jj * 4 + ch]) : 0.f;
+          const uint64_t e2 = tc::f2_make(eRow, eRow), fq2 = tc::f2_make(fq, fq),
+                         g2r = tc::f2_make(grow, grow);
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
             const int p = ch * 32 + i;
             const float4 g4 = *reinterpret_cast<const float4*>((R_IS_QUERY ? pe : fw) + p);
             float4 e4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (KIND == KDK) e4 = *reinterpret_cast<const float4*>(pe + p);
-            const float gv[4] = {g4.x, g4.y, g4.z, g4.w}, ev[4] = {e4.x, e4.y, e4.z, e4.w};
-            float y[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float xv = __uint_as_float(xr[i + u]);
-              if (KIND == KDQ) y[u] = ((xv + eRow) * fq) * gv[u];
-              else if (KIND == KDK) y[u] = ((xv + ev[u]) * gv[u]) * grow;
-              else y[u] = (xv * gv[u]) * grow;
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t x2 = tc::f2_make(__uint_as_float(xr[i + 2 * h]), __uint_as_float(xr[i + 2 * h + 1]));
+              const uint64_t gv = h ? tc::f2_make(g4.z, g4.w) : tc::f2_make(g4.x, g4.y);
+              uint64_t y2;
+              if (KIND == KDQ) {
+                y2 = tc::f2_mul(tc::f2_mul(tc::f2_add(x2, e2), fq2), gv);
+              } else if (KIND == KDK) {
+                const uint64_t ev = h ? tc::f2_make(e4.z, e4.w) : tc::f2_make(e4.x, e4.y);
+                y2 = tc::f2_mul(tc::f2_mul(tc::f2_add(x2, ev), gv), g2r);
+              } else {
+                y2 = tc::f2_mul(tc::f2_mul(x2, gv), g2r);
+              }
+              const float2 yy = tc::f2_split(y2);
+              pk[(i >> 1) + h] = tc::pack_bf16(yy.x, yy.y);
             }
-            pk[i >> 1] = tc::pack_bf16(y[0], y[1]);
-            pk[(i >> 1) + 1] = tc::pack_bf16(y[2], y[3]);
           }
         }
         tc::tmem_st16_async(tX + lane_base + 16 * ch, pk);
