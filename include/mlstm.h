@@ -207,6 +207,43 @@ int mlstm_step(const void* q, const void* k, const void* v, const void* igate_pr
                const void* fgate_pre, void* h, const void* state_in, void* state_out,
                int B, int NH, int d_qk, int d_hv, int variant, int dtype, void* stream);
 
+/* The chunkwise forward of a sequence that continues from a state, for
+ * chaining calls (a long prompt in pieces, or a prompt after generated
+ * tokens).  Same arguments, layouts, ownership and errors as mlstm_fwd, plus:
+ *   state_in   the state before the first token (layout above), read; NULL:
+ *              the zero state, which makes this call mlstm_fwd.
+ *   state_out  the state after the last token, written; NULL: not wanted.
+ * With the recurrence above started from state_in, h is the same as for the
+ * whole sequence: inside, the state enters the first chunk like any chunk's
+ * state (its C and n, and m as the first chunk's m_{c-1}), and state_out is
+ * mlstm_final_state's result.  state_in and state_out must not overlap
+ * (MLSTM_ERR_INVALID).  T = 0 copies state_in (or the zero state) to
+ * state_out.  The saved buffer of such a call is for mlstm_bwd_state with the
+ * same state_in. */
+int mlstm_fwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
+                    const void* fgate_pre, void* h, void* saved, void* workspace,
+                    size_t workspace_bytes, const void* state_in, void* state_out, int B, int NH,
+                    int T, int d_qk, int d_hv, int chunk, int variant, int dtype, void* stream);
+
+/* The backward of mlstm_fwd_state, with the initial state held constant (its
+ * max state m, like every max state, carries no gradient).  Same arguments,
+ * layouts and errors as mlstm_bwd, plus:
+ *   state_in   the state the forward started from (NULL: the zero state).
+ *   dstate_in  gradient of the loss with respect to state_in's C and (EXP) n,
+ *              written into those regions of a state-layout buffer (its m
+ *              region is not written); NULL: not wanted.  It is one more step
+ *              of the state-gradient recurrence: beta_0 dC_0 + Q_0^T diag(u)
+ *              dH_0 over the first chunk.
+ * state_in and dstate_in must not overlap (MLSTM_ERR_INVALID).  The gradient
+ * of a loss that also reads state_out is not supported here: such a loss
+ * contributes through a later call's dstate_in only. */
+int mlstm_bwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
+                    const void* fgate_pre, const void* h, const void* dh, const void* saved,
+                    const void* state_in, void* dstate_in, void* dq, void* dk, void* dv,
+                    void* digate_pre, void* dfgate_pre, void* workspace, size_t workspace_bytes,
+                    int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype,
+                    void* stream);
+
 /* Synchronise `stream` and report what the kernels enqueued so far found:
  * MLSTM_ERR_TIMEOUT if one of them gave up a bounded wait (its outputs are
  * then invalid; the flag is cleared by this call), MLSTM_ERR_CUDA on a CUDA

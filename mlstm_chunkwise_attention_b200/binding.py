@@ -63,6 +63,8 @@ EXPORTS = {
     "mlstm_state_zero": (ctypes.c_int, [_P] + [ctypes.c_int] * 5 + [_P]),
     "mlstm_final_state": (ctypes.c_int, [_P] * 4 + _SIZES + [_P]),
     "mlstm_step": (ctypes.c_int, [_P] * 8 + [ctypes.c_int] * 6 + [_P]),
+    "mlstm_fwd_state": (ctypes.c_int, [_P] * 7 + [_P, ctypes.c_size_t, _P, _P] + _SIZES + [_P]),
+    "mlstm_bwd_state": (ctypes.c_int, [_P] * 15 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
 }
 
 
@@ -134,6 +136,21 @@ def mlstm_bwd(q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv, digate_pr
     return load().mlstm_bwd(q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv, digate_pre,
                             dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
                             variant, dtype, stream)
+
+
+def mlstm_fwd_state(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_bytes,
+                    state_in, state_out, B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream):
+    return load().mlstm_fwd_state(q, k, v, igate_pre, fgate_pre, h, saved, workspace,
+                                  workspace_bytes, state_in, state_out, B, NH, T, d_qk, d_hv, chunk,
+                                  variant, dtype, stream)
+
+
+def mlstm_bwd_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in, dq, dk, dv,
+                    digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
+                    variant, dtype, stream):
+    return load().mlstm_bwd_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in,
+                                  dq, dk, dv, digate_pre, dfgate_pre, workspace, workspace_bytes, B,
+                                  NH, T, d_qk, d_hv, chunk, variant, dtype, stream)
 
 
 def mlstm_status_string(status):
@@ -295,6 +312,68 @@ def final_state(k, v, saved, chunk, variant, *, state=None, stream=None):
     if st != STATUS_OK:
         raise MLSTMError(st, "mlstm_final_state")
     return state
+
+
+def forward_state(q, k, v, igate_pre, fgate_pre, chunk, variant, state_in=None, *,
+                  keep_saved=True, stream=None):
+    """Chunkwise forward continuing from ``state_in`` (None: the zero state).
+
+    Returns (h, saved, state_out): state_out is a fresh state buffer holding the state
+    after the last token; saved (None when keep_saved is False) is for backward_state.
+    """
+    import torch
+    _check({"q": q, "k": k, "v": v, "igate_pre": igate_pre, "fgate_pre": fgate_pre}, q.dtype)
+    sizes = problem_sizes(q, v, chunk, variant)
+    B, NH, T, d_qk, d_hv = sizes[:5]
+    h = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    state_out = torch.empty(load().mlstm_state_size(B, NH, d_qk, d_hv, variant), dtype=torch.uint8,
+                            device=q.device)
+    saved = ws = None
+    if keep_saved:
+        saved = torch.empty(max(mlstm_saved_size(*sizes), 1), dtype=torch.uint8, device=q.device)
+    else:
+        ws = torch.empty(max(mlstm_fwd_workspace_size(*sizes), 1), dtype=torch.uint8,
+                         device=q.device)
+    st = mlstm_fwd_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
+                         fgate_pre.data_ptr(), h.data_ptr(),
+                         saved.data_ptr() if saved is not None else None,
+                         ws.data_ptr() if ws is not None else None,
+                         ws.numel() if ws is not None else 0,
+                         state_in.data_ptr() if state_in is not None else None,
+                         state_out.data_ptr(), *sizes, _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_fwd_state")
+    return h, saved, state_out
+
+
+def backward_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, state_in=None, *,
+                   want_dstate=True, stream=None):
+    """Gradients of sum(dh * h) for a forward_state call, the initial state held constant.
+
+    Returns the dict of ``backward`` plus "dstate_in" (a state-layout buffer whose C and,
+    for EXP, n regions hold the gradient with respect to state_in) when want_dstate.
+    """
+    import torch
+    _check({"q": q, "k": k, "v": v, "igate_pre": igate_pre, "fgate_pre": fgate_pre, "h": h,
+            "dh": dh}, q.dtype)
+    sizes = problem_sizes(q, v, chunk, variant)
+    B, NH, T, d_qk, d_hv = sizes[:5]
+    out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "digate_pre": torch.empty_like(igate_pre), "dfgate_pre": torch.empty_like(fgate_pre)}
+    if want_dstate:
+        out["dstate_in"] = torch.zeros(load().mlstm_state_size(B, NH, d_qk, d_hv, variant),
+                                       dtype=torch.uint8, device=q.device)
+    ws = torch.empty(max(mlstm_bwd_workspace_size(*sizes), 1), dtype=torch.uint8, device=q.device)
+    st = mlstm_bwd_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
+                         fgate_pre.data_ptr(), h.data_ptr(), dh.data_ptr(), saved.data_ptr(),
+                         state_in.data_ptr() if state_in is not None else None,
+                         out["dstate_in"].data_ptr() if want_dstate else None,
+                         out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr(),
+                         out["digate_pre"].data_ptr(), out["dfgate_pre"].data_ptr(),
+                         ws.data_ptr(), ws.numel(), *sizes, _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_bwd_state")
+    return out
 
 
 def step(q, k, v, igate_pre, fgate_pre, state_in, state_out, variant, *, h=None, stream=None):

@@ -28,7 +28,7 @@ namespace mlstm {
 template <bool EXPV>
 __device__ void write_xl_tables(const float* b, const float* li, const float* m, float* xt,
                                 size_t base, int T, int L, int NC, float scale,
-                                float log2_scale) {
+                                float log2_scale, bool has_init, const float* m0) {
   constexpr float kLog2e = 1.4426950408889634f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int stride = xl_table_stride(L), bpc = L / 32;
@@ -41,7 +41,8 @@ __device__ void write_xl_tables(const float* b, const float* li, const float* m,
       const float bt = b[base + t];
       const float mt = EXPV ? m[base + t] : 0.f;
       R = (bt - mt) * kLog2e + log2_scale;
-      if (c > 0) QF = expf(bt + (EXPV ? m[base + (size_t)c * L - 1] : 0.f) - mt) * scale;
+      if (c > 0 || has_init)
+        QF = expf(bt + (EXPV ? chunk_mprev(m, base + (size_t)c * L, c, m0, blockIdx.x) : 0.f) - mt) * scale;
       if (EXPV) FL = expf(-mt);
       CC = (li[base + t] - bt) * kLog2e;
     }
@@ -60,7 +61,7 @@ template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(256) gate_prep_kernel(
     const TIO* __restrict__ ig, const TIO* __restrict__ fg, float* __restrict__ b_out,
     float* __restrict__ li_out, float* __restrict__ m_out, float* __restrict__ xt, int T, int L,
-    int NC, float scale, float log2_scale) {
+    int NC, float scale, float log2_scale, bool has_init, const float* __restrict__ m0) {
   extern __shared__ float smem[];
   float* sg = smem;       // g_c  (chunk decay)
   float* su = smem + NC;  // u_c, then m_c
@@ -109,13 +110,15 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
   if (!EXPV) {
     if (xt != nullptr) {
       __syncthreads();
-      write_xl_tables<false>(b_out, li_out, m_out, xt, base, T, L, NC, scale, log2_scale);
+      write_xl_tables<false>(b_out, li_out, m_out, xt, base, T, L, NC, scale, log2_scale, has_init, m0);
     }
     return;
   }
   __syncthreads();
+  // the max state before the first chunk: the initial state's, -inf without one
+  const float m_init = m0 != nullptr ? m0[blockIdx.x] : -INFINITY;
   if (warp == 0) {
-    float carry = -INFINITY;
+    float carry = m_init;
     for (int cb = 0; cb < NC; cb += 32) {
       const int c = cb + lane;
       float g = c < NC ? sg[c] : 0.f;
@@ -137,13 +140,13 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
   __syncthreads();
   for (int t = threadIdx.x; t < T; t += blockDim.x) {
     const int c = t / L;
-    const float mprev = c > 0 ? su[c - 1] : -INFINITY;
+    const float mprev = c > 0 ? su[c - 1] : m_init;
     const size_t idx = base + t;
     m_out[idx] = b_out[idx] + fmaxf(mprev, m_out[idx]);
   }
   if (xt != nullptr) {
     __syncthreads();
-    write_xl_tables<true>(b_out, li_out, m_out, xt, base, T, L, NC, scale, log2_scale);
+    write_xl_tables<true>(b_out, li_out, m_out, xt, base, T, L, NC, scale, log2_scale, has_init, m0);
   }
 }
 
@@ -152,14 +155,14 @@ cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH), block(256);
   if (p.bf16()) {
     if (p.exp_variant())
-      gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
+      gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale), a.init.on(), a.init.on() && p.exp_variant() ? a.init.m : nullptr);
     else
-      gate_prep_kernel<bf16, false><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
+      gate_prep_kernel<bf16, false><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale), a.init.on(), a.init.on() && p.exp_variant() ? a.init.m : nullptr);
   } else {
     if (p.exp_variant())
-      gate_prep_kernel<float, true><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
+      gate_prep_kernel<float, true><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale), a.init.on(), a.init.on() && p.exp_variant() ? a.init.m : nullptr);
     else
-      gate_prep_kernel<float, false><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale));
+      gate_prep_kernel<float, false><<<grid, block, smem, s>>>((const float*)a.ig, (const float*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale), a.init.on(), a.init.on() && p.exp_variant() ? a.init.m : nullptr);
   }
   return cudaGetLastError();
 }

@@ -15,6 +15,23 @@ struct Problem {
   bool bf16() const { return dtype == 0; }
 };
 
+// The state a sequence starts from, in the recurrent-state layout (fp32):
+// C [BH, dqk, dhv], n [BH, dqk] and m [BH] (n and m for mLSTMexp only), the
+// stabilised form whose true state is exp(m) (C, n).  C == nullptr: the zero
+// state (m = -inf), which every kernel then treats as "no state enters the
+// first chunk".
+struct InitState {
+  const float *C = nullptr, *n = nullptr, *m = nullptr;
+  __host__ __device__ bool on() const { return C != nullptr; }
+};
+
+// m_{c-1} as chunk c sees it (mLSTMexp): the max state at the previous chunk's
+// last row, or the initial state's for the first chunk (-inf without one).
+__device__ __forceinline__ float chunk_mprev(const float* m, size_t tok_first, int c, const float* m0,
+                                             int bh) {
+  return c > 0 ? m[tok_first - 1] : (m0 != nullptr ? m0[bh] : -__int_as_float(0x7f800000));
+}
+
 // Device pointers of one forward call.
 struct FwdArgs {
   const void *q, *k, *v, *ig, *fg;
@@ -24,6 +41,7 @@ struct FwdArgs {
   float* n;                  // [BH, NC, dqk]
   bool keep_lo;              // write the low plane of bf16 states (needed by the backward)
   float* xt;                 // per-chunk gate tables of the large-chunk output kernel, or null
+  InitState init;            // the state entering the first chunk
 };
 
 // Per-chunk gate tables, [BH, NC, xl_table_stride(L)] floats, written by
@@ -51,6 +69,9 @@ struct BwdArgs {
   float* pk;       // [BH, T] k_t . dk_t
   void* dC;        // [BH, NC, dqk, dhv] gradient of the state leaving each chunk (planes, see StatePlanes)
   float* dn;       // [BH, NC, dqk]
+  InitState init;  // the state the forward started from (held constant)
+  float* dC0;      // gradient of the initial state: C [BH, dqk, dhv] (null: not wanted)
+  float* dn0;      // and n [BH, dqk] (mLSTMexp)
 };
 
 // gate kernels (gates.cu)
@@ -88,7 +109,8 @@ cudaError_t fetch_tc_state_error(unsigned int* flag);
 // recurrent-form kernels (recurrent.cu)
 cudaError_t launch_final_state(const Problem& p, const void* k, const void* v, const float* b,
                                const float* li, const float* m, const void* C, const float* n,
-                               float* Cout, float* nout, float* mout, cudaStream_t s);
+                               const InitState& init, float* Cout, float* nout, float* mout,
+                               cudaStream_t s);
 cudaError_t launch_step(const Problem& p, const void* q, const void* k, const void* v,
                         const void* ig, const void* fg, void* h, const float* Cin, const float* nin,
                         const float* min_, float* Cout, float* nout, float* mout, cudaStream_t s);

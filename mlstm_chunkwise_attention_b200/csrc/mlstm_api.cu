@@ -88,6 +88,43 @@ BwdLayout bwd_layout(const Problem& p) {
 
 bool misaligned(const void* ptr) { return ((uintptr_t)ptr & 15) != 0; }
 
+struct StateLayout {
+  size_t C, n, m, total;
+};
+
+// Recurrent state of one call: C [BH, d_qk, d_hv], then (EXP) n [BH, d_qk] and m [BH],
+// fp32, 256-byte aligned regions.
+StateLayout state_layout(int BH, int dqk, int dhv, bool exp_variant) {
+  StateLayout L;
+  L.C = 0;
+  size_t off = align256((size_t)BH * dqk * dhv * 4);
+  L.n = off;
+  if (exp_variant) off = align256(off + (size_t)BH * dqk * 4);
+  L.m = off;
+  if (exp_variant) off = align256(off + (size_t)BH * 4);
+  L.total = off;
+  return L;
+}
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + bytes && y < x + bytes;
+}
+
+// The initial state held in a recurrent-state buffer (null: the zero state).
+mlstm::InitState init_from(const void* state, const Problem& p) {
+  mlstm::InitState in;
+  if (!state) return in;
+  const StateLayout S = state_layout(p.BH, p.dqk, p.dhv, p.exp_variant());
+  const char* base = (const char*)state;
+  in.C = (const float*)(base + S.C);
+  if (p.exp_variant()) {
+    in.n = (const float*)(base + S.n);
+    in.m = (const float*)(base + S.m);
+  }
+  return in;
+}
+
 int cuda_status(cudaError_t e, const char* where) {
   if (e == cudaSuccess) return MLSTM_OK;
   snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
@@ -230,13 +267,27 @@ int mlstm_set_timing_events(void* const* events, int count) {
   return MLSTM_OK;
 }
 
-int mlstm_fwd(const void* q, const void* k, const void* v, const void* igate_pre,
-              const void* fgate_pre, void* h, void* saved, void* workspace,
-              size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
-              int variant, int dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
+             const void* fgate_pre, void* h, void* saved, void* workspace, size_t workspace_bytes,
+             const void* state_in, void* state_out, int B, int NH, int T, int d_qk, int d_hv,
+             int chunk, int variant, int dtype, void* stream) {
   int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
   if (st != MLSTM_OK) return st;
-  if ((long long)B * NH * T == 0) return MLSTM_OK;
+  if (misaligned(state_in) || misaligned(state_out)) return MLSTM_ERR_INVALID;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  const StateLayout SL = state_layout(B * NH, d_qk, d_hv, variant == MLSTM_EXP);
+  if (state_in && state_out && overlaps(state_in, state_out, SL.total)) return MLSTM_ERR_INVALID;
+  if (T == 0) {  // the final state is the initial one
+    if (!state_out) return MLSTM_OK;
+    if (!state_in) return mlstm_state_zero(state_out, B, NH, d_qk, d_hv, variant, stream);
+    return cuda_status(cudaMemcpyAsync(state_out, state_in, SL.total, cudaMemcpyDeviceToDevice,
+                                       (cudaStream_t)stream),
+                       "state copy");
+  }
   if (!q || !k || !v || !igate_pre || !fgate_pre || !h) return MLSTM_ERR_INVALID;
   if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(h) ||
       misaligned(igate_pre) || misaligned(fgate_pre) || misaligned(saved) ||
@@ -258,25 +309,63 @@ int mlstm_fwd(const void* q, const void* k, const void* v, const void* igate_pre
   a.abar = p.exp_variant() ? (float*)(base + L.norm) : nullptr;
   a.C = base + L.state_c;
   a.n = p.exp_variant() ? (float*)(base + L.state_n) : nullptr;
-  a.keep_lo = saved != nullptr;
+  a.keep_lo = saved != nullptr || state_out != nullptr;  // the final state reads both planes
   a.xt = L.tile_table_bytes ? (float*)(base + L.tile_table) : nullptr;
+  a.init = init_from(state_in, p);
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_fwd");
   if (st != MLSTM_OK) return st;
   FwdStep steps[kMaxSteps];
   const int n = fwd_plan(p, steps);
-  return run_plan(steps, n, p, a, s);
+  st = run_plan(steps, n, p, a, s);
+  if (st != MLSTM_OK || !state_out) return st;
+  char* out = (char*)state_out;
+  return cuda_status(mlstm::launch_final_state(p, k, v, a.b, a.li, a.m, a.C, a.n, a.init,
+                                               (float*)(out + SL.C), (float*)(out + SL.n),
+                                               (float*)(out + SL.m), s),
+                     "final_state");
 }
 
-int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre,
-              const void* fgate_pre, const void* h, const void* dh, const void* saved, void* dq,
-              void* dk, void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
+}  // namespace
+
+extern "C" {
+
+int mlstm_fwd(const void* q, const void* k, const void* v, const void* igate_pre,
+              const void* fgate_pre, void* h, void* saved, void* workspace,
               size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
               int variant, int dtype, void* stream) {
+  return fwd_impl(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_bytes, nullptr,
+                  nullptr, B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream);
+}
+
+int mlstm_fwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
+                    const void* fgate_pre, void* h, void* saved, void* workspace,
+                    size_t workspace_bytes, const void* state_in, void* state_out, int B, int NH,
+                    int T, int d_qk, int d_hv, int chunk, int variant, int dtype, void* stream) {
+  return fwd_impl(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspace_bytes, state_in,
+                  state_out, B, NH, T, d_qk, d_hv, chunk, variant, dtype, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
+             const void* fgate_pre, const void* h, const void* dh, const void* saved,
+             const void* state_in, void* dstate_in, void* dq, void* dk, void* dv, void* digate_pre,
+             void* dfgate_pre, void* workspace, size_t workspace_bytes, int B, int NH, int T,
+             int d_qk, int d_hv, int chunk, int variant, int dtype, void* stream) {
   int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
   if (st != MLSTM_OK) return st;
-  if ((long long)B * NH * T == 0) return MLSTM_OK;
+  if (misaligned(state_in) || misaligned(dstate_in)) return MLSTM_ERR_INVALID;
+  const StateLayout SL = state_layout(B * NH, d_qk, d_hv, variant == MLSTM_EXP);
+  if (dstate_in && state_in && overlaps(state_in, dstate_in, SL.total)) return MLSTM_ERR_INVALID;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (T == 0) {  // nothing reads the initial state: its gradient is zero
+    if (!dstate_in) return MLSTM_OK;
+    return cuda_status(cudaMemsetAsync(dstate_in, 0, SL.total, (cudaStream_t)stream), "memset");
+  }
   if (!q || !k || !v || !igate_pre || !fgate_pre || !h || !dh || !saved || !dq || !dk || !dv ||
       !digate_pre || !dfgate_pre)
     return MLSTM_ERR_INVALID;
@@ -306,6 +395,9 @@ int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre
   a.pk = (float*)(ws + W.pk);
   a.dC = ws + W.dC;
   a.dn = p.exp_variant() ? (float*)(ws + W.dn) : nullptr;
+  a.init = init_from(state_in, p);
+  a.dC0 = dstate_in ? (float*)((char*)dstate_in + SL.C) : nullptr;
+  a.dn0 = (dstate_in && p.exp_variant()) ? (float*)((char*)dstate_in + SL.n) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_bwd");
@@ -315,34 +407,32 @@ int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre
   return run_plan(steps, n, p, a, s);
 }
 
-}  // extern "C"
-
-namespace {
-
-struct StateLayout {
-  size_t C, n, m, total;
-};
-
-// Recurrent state of one call: C [BH, d_qk, d_hv], then (EXP) n [BH, d_qk] and m [BH],
-// fp32, 256-byte aligned regions.
-StateLayout state_layout(int BH, int dqk, int dhv, bool exp_variant) {
-  StateLayout L;
-  L.C = 0;
-  size_t off = align256((size_t)BH * dqk * dhv * 4);
-  L.n = off;
-  if (exp_variant) off = align256(off + (size_t)BH * dqk * 4);
-  L.m = off;
-  if (exp_variant) off = align256(off + (size_t)BH * 4);
-  L.total = off;
-  return L;
-}
-
-bool overlaps(const void* a, const void* b, size_t bytes) {
-  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
-  return x < y + bytes && y < x + bytes;
-}
-
 }  // namespace
+
+extern "C" {
+
+int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre,
+              const void* fgate_pre, const void* h, const void* dh, const void* saved, void* dq,
+              void* dk, void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
+              size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
+              int variant, int dtype, void* stream) {
+  return bwd_impl(q, k, v, igate_pre, fgate_pre, h, dh, saved, nullptr, nullptr, dq, dk, dv,
+                  digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
+                  variant, dtype, stream);
+}
+
+int mlstm_bwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
+                    const void* fgate_pre, const void* h, const void* dh, const void* saved,
+                    const void* state_in, void* dstate_in, void* dq, void* dk, void* dv,
+                    void* digate_pre, void* dfgate_pre, void* workspace, size_t workspace_bytes,
+                    int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype,
+                    void* stream) {
+  return bwd_impl(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in, dq, dk, dv,
+                  digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
+                  variant, dtype, stream);
+}
+
+}  // extern "C"
 
 extern "C" {
 
@@ -386,7 +476,8 @@ int mlstm_final_state(const void* k, const void* v, const void* saved, void* sta
                                 p.exp_variant() ? (const float*)(sv + L.gate_m) : nullptr,
                                 sv + L.state_c,
                                 p.exp_variant() ? (const float*)(sv + L.state_n) : nullptr,
-                                (float*)(out + S.C), (float*)(out + S.n), (float*)(out + S.m),
+                                mlstm::InitState{}, (float*)(out + S.C), (float*)(out + S.n),
+                                (float*)(out + S.m),
                                 (cudaStream_t)stream),
       "final_state");
 }

@@ -26,7 +26,8 @@ __global__ void __launch_bounds__(256) final_state_kernel(
     const TIO* __restrict__ k, const TIO* __restrict__ v, const float* __restrict__ b,
     const float* __restrict__ li, const float* __restrict__ m, const TS* __restrict__ C,
     const float* __restrict__ n, size_t plane, float* __restrict__ Cout,
-    float* __restrict__ nout, float* __restrict__ mout, int T, int L, int NC, int dhv) {
+    float* __restrict__ nout, float* __restrict__ mout, int T, int L, int NC, int dhv,
+    bool has_init, const float* __restrict__ m0) {
   __shared__ float ks[kTok][DQK];
   __shared__ float vs[kTok][64];
   __shared__ float ws[kTok];
@@ -36,8 +37,10 @@ __global__ void __launch_bounds__(256) final_state_kernel(
   const size_t tok0 = (size_t)bh * T;
   const float g = b[tok0 + T - 1];
   const float mT = EXPV ? m[tok0 + T - 1] : 0.f;
-  const float menter = EXPV ? (c > 0 ? m[tok0 + lo - 1] : kNegInf) : 0.f;
-  const float beta = c > 0 ? expf(g + menter - mT) : 0.f;
+  // a state enters the last chunk: an earlier chunk's, or the initial state
+  const bool has_prev = c > 0 || has_init;
+  const float menter = EXPV ? chunk_mprev(m, tok0 + lo, c, m0, bh) : 0.f;
+  const float beta = has_prev ? expf(g + menter - mT) : 0.f;
   constexpr int R = DQK / 4;
   float acc[R];
 #pragma unroll
@@ -70,13 +73,13 @@ __global__ void __launch_bounds__(256) final_state_kernel(
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int i = rg + 4 * r;
-      const float prev = c > 0 ? StatePlanes<TS>::load(C, plane, cbase + (size_t)i * dhv + j) : 0.f;
+      const float prev = has_prev ? StatePlanes<TS>::load(C, plane, cbase + (size_t)i * dhv + j) : 0.f;
       Cout[((size_t)bh * DQK + i) * dhv + j] = beta * prev + acc[r];
     }
   }
   if (EXPV && blockIdx.x == 0) {
     if (tid < DQK) {
-      const float prev = c > 0 ? n[((size_t)bh * NC + c) * DQK + tid] : 0.f;
+      const float prev = has_prev ? n[((size_t)bh * NC + c) * DQK + tid] : 0.f;
       nout[(size_t)bh * DQK + tid] = beta * prev + nacc;
     }
     if (tid == 0) mout[bh] = mT;
@@ -187,13 +190,15 @@ __global__ void fill_neg_inf_kernel(float* __restrict__ m, int count) {
 
 cudaError_t launch_final_state(const Problem& p, const void* k, const void* v, const float* b,
                                const float* li, const float* m, const void* C, const float* n,
-                               float* Cout, float* nout, float* mout, cudaStream_t s) {
+                               const InitState& init, float* Cout, float* nout, float* mout,
+                               cudaStream_t s) {
+  const float* m0 = (init.on() && p.exp_variant()) ? init.m : nullptr;
   const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
   dim3 grid((unsigned)((p.dhv + 63) / 64), (unsigned)p.BH), block(256);
 #define MLSTM_FS(TIO, TS, E, D)                                                                     \
   final_state_kernel<TIO, TS, E, D><<<grid, block, 0, s>>>((const TIO*)k, (const TIO*)v, b, li, m, \
                                                           (const TS*)C, n, plane, Cout, nout, mout, \
-                                                          p.T, p.L, p.NC, p.dhv)
+                                                          p.T, p.L, p.NC, p.dhv, init.on(), m0)
 #define MLSTM_FS_D(TIO, TS, E)                       \
   if (p.dqk == 64) MLSTM_FS(TIO, TS, E, 64);         \
   else if (p.dqk == 128) MLSTM_FS(TIO, TS, E, 128);  \

@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ dh, const float* __restrict__ b,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
     TS* __restrict__ dC, float* __restrict__ dn, int T, int L, int NC, int dqk, int dhv,
-    float scale, size_t plane) {
+    float scale, size_t plane, const float* __restrict__ m0, float* __restrict__ d0,
+    float* __restrict__ dn0) {
   __shared__ float sQ[32][64];
   __shared__ float sD[32][64];
   __shared__ float fq[32], fn[32];
@@ -53,12 +54,12 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
         StatePlanes<TS>::store(dC, plane, gbase + (size_t)(i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j,
                                acc[i][j], true);
     if (own_n) dn[((size_t)bh * NC + c) * dqk + i0 + tid] = nacc;
-    if (c == 0) break;
+    if (c == 0 && d0 == nullptr) break;  // the first chunk's contribution: the initial state's gradient
 
     const int c0 = c * L, len = min(L, T - c0), last = c0 + len - 1;
     const float g = b[tokh + last];
     const float mc = EXPV ? m[tokh + last] : 0.f;
-    const float mprev = EXPV ? m[tokh + c0 - 1] : 0.f;
+    const float mprev = EXPV ? chunk_mprev(m, tokh + c0, c, m0, bh) : 0.f;
     const float beta = expf(g + mprev - mc);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -104,6 +105,13 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
         for (int r = 0; r < 32; ++r) nacc = fmaf(sQ[r][tid], fn[r], nacc);
     }
   }
+  if (d0 != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d0[((size_t)bh * dqk + i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] = acc[i][j];
+    if (own_n) dn0[(size_t)bh * dqk + i0 + tid] = nacc;
+  }
 }
 
 cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream_t s) {
@@ -111,7 +119,8 @@ cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream
 #define MLSTM_STATE_BWD(TIO, TS, E)                                                             \
   state_bwd_simt_kernel<TIO, TS, E><<<grid, block, 0, s>>>(                                     \
       (const TIO*)a.q, (const TIO*)a.dh, a.b, a.m, a.inv_den, a.da, (TS*)a.dC, a.dn, p.T, p.L,  \
-      p.NC, p.dqk, p.dhv, p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv)
+      p.NC, p.dqk, p.dhv, p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv,                     \
+      a.init.on() ? a.init.m : nullptr, a.dC0, a.dn0)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_STATE_BWD(bf16, bf16, true);
     else MLSTM_STATE_BWD(bf16, bf16, false);
@@ -207,7 +216,8 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
     const TIO* __restrict__ dh, const float* __restrict__ b, const float* __restrict__ li,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
     const TS* __restrict__ C, const float* __restrict__ n, TIO* __restrict__ dq,
-    float* __restrict__ pq, int T, int L, int NC, int dqk, int dhv, float scale, size_t plane) {
+    float* __restrict__ pq, int T, int L, int NC, int dqk, int dhv, float scale, size_t plane,
+    bool has_init, const float* __restrict__ m0) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -217,12 +227,13 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
   const int i0 = blockIdx.z * 64;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const size_t tok0 = (size_t)bh * T + c0;
-  const float mprev = EXPV ? (c > 0 ? m[(size_t)bh * T + c0 - 1] : -INFINITY) : 0.f;
-  load_row_factors<EXPV>(S, b, m, inv_den, da, tok0, t0, len, mprev, c > 0);
+  const float mprev = EXPV ? chunk_mprev(m, (size_t)bh * T + c0, c, m0, bh) : 0.f;
+  const bool has_prev = c > 0 || has_init;  // a state enters this chunk
+  load_row_factors<EXPV>(S, b, m, inv_den, da, tok0, t0, len, mprev, has_prev);
   float acc[4][4];
   zero44(acc);
 
-  if (c > 0) {  // alpha_t (C_{c-1} dnum_t + da_t n_{c-1})
+  if (has_prev) {  // alpha_t (C_{c-1} dnum_t + da_t n_{c-1})
     const size_t cbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dhv; x0 += 32) {
       __syncthreads();
@@ -494,7 +505,7 @@ static cudaError_t dq_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dq_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, (const TIO*)a.dh, a.b, a.li, a.m,
       a.inv_den, a.da, (const TS*)a.C, a.n, (TIO*)a.dq, a.pq, p.T, p.L, p.NC, p.dqk, p.dhv,
-      p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv);
+      p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv, a.init.on(), a.init.on() ? a.init.m : nullptr);
   return cudaGetLastError();
 }
 

@@ -22,7 +22,8 @@ template <typename TIO, typename TS, bool EXPV>
 __global__ void __launch_bounds__(256) state_fwd_simt_kernel(
     const TIO* __restrict__ k, const TIO* __restrict__ v, const float* __restrict__ b,
     const float* __restrict__ li, const float* __restrict__ m, TS* __restrict__ C,
-    float* __restrict__ n, int T, int L, int NC, int dqk, int dhv, size_t plane, bool keep_lo) {
+    float* __restrict__ n, int T, int L, int NC, int dqk, int dhv, size_t plane, bool keep_lo,
+    InitState init) {
   __shared__ float sK[32][64];
   __shared__ float sV[32][64];
   __shared__ float sw[32];
@@ -30,12 +31,15 @@ __global__ void __launch_bounds__(256) state_fwd_simt_kernel(
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const size_t tok0 = (size_t)bh * T;
   const bool own_n = EXPV && blockIdx.z == 0 && tid < 64;
+  // the state entering the first chunk: the initial state, or zero
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  float nacc = 0.f;
+    for (int j = 0; j < 4; ++j)
+      acc[i][j] = init.on() ? init.C[((size_t)bh * dqk + i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] : 0.f;
+  float nacc = (own_n && init.on()) ? init.n[(size_t)bh * dqk + i0 + tid] : 0.f;
+  const float* m0 = init.on() ? init.m : nullptr;
 
   for (int c = 0; c < NC; ++c) {
     const size_t cbase = ((size_t)bh * NC + c) * dqk * dhv;
@@ -51,8 +55,8 @@ __global__ void __launch_bounds__(256) state_fwd_simt_kernel(
     const int c0 = c * L, len = min(L, T - c0), last = c0 + len - 1;
     const float g = b[tok0 + last];
     const float mc = EXPV ? m[tok0 + last] : 0.f;
-    const float mprev = EXPV ? (c > 0 ? m[tok0 + c0 - 1] : -INFINITY) : 0.f;
-    const float beta = c == 0 ? 0.f : expf(g + mprev - mc);
+    const float mprev = EXPV ? chunk_mprev(m, tok0 + c0, c, m0, bh) : 0.f;
+    const float beta = (c == 0 && !init.on()) ? 0.f : expf(g + mprev - mc);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -97,7 +101,7 @@ cudaError_t launch_state_fwd_simt(const Problem& p, const FwdArgs& a, cudaStream
 #define MLSTM_STATE_FWD(TIO, TS, E)                                                              \
   state_fwd_simt_kernel<TIO, TS, E><<<grid, block, 0, s>>>((const TIO*)a.k, (const TIO*)a.v, a.b, \
                                                            a.li, a.m, (TS*)a.C, a.n, p.T, p.L,  \
-                                                           p.NC, p.dqk, p.dhv, plane, a.keep_lo)
+                                                           p.NC, p.dqk, p.dhv, plane, a.keep_lo, a.init)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_STATE_FWD(bf16, bf16, true);
     else MLSTM_STATE_FWD(bf16, bf16, false);
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
     const float* __restrict__ b, const float* __restrict__ li, const float* __restrict__ m,
     const TS* __restrict__ C, const float* __restrict__ n, TIO* __restrict__ h,
     float* __restrict__ abar_out, int T, int L, int NC, int dqk, int dhv, float scale,
-    size_t plane, bool use_lo) {
+    size_t plane, bool use_lo, bool has_init, const float* __restrict__ m0) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   OutSmem& S = *reinterpret_cast<OutSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -142,7 +146,8 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
   const int j0 = blockIdx.z * 64;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const size_t tok0 = (size_t)bh * T + c0;  // first token of the chunk
-  const float mprev = EXPV ? (c > 0 ? m[(size_t)bh * T + c0 - 1] : -INFINITY) : 0.f;
+  const float mprev = EXPV ? chunk_mprev(m, (size_t)bh * T + c0, c, m0, bh) : 0.f;
+  const bool has_prev = c > 0 || has_init;  // a state enters this chunk
 
   if (tid < 64) {
     const int t = t0 + tid;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
     const float mt = (EXPV && ok) ? m[tok0 + t] : 0.f;
     S.bt[tid] = bt;
     S.mt[tid] = mt;
-    S.alpha[tid] = (ok && c > 0) ? expf(bt + mprev - mt) : 0.f;
+    S.alpha[tid] = (ok && has_prev) ? expf(bt + mprev - mt) : 0.f;
     S.rowsum[tid] = 0.f;
     S.ainter[tid] = 0.f;
   }
@@ -162,7 +167,7 @@ __global__ void __launch_bounds__(256) output_fwd_simt_kernel(
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
   // inter-chunk term
-  if (c > 0) {
+  if (has_prev) {
     const size_t cbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int kk0 = 0; kk0 < dqk; kk0 += 32) {
       __syncthreads();
@@ -308,7 +313,8 @@ cudaError_t launch_output_fwd_simt(const Problem& p, const FwdArgs& a, cudaStrea
     if (e != cudaSuccess) return e;                                                              \
     output_fwd_simt_kernel<TIO, TS, E><<<grid, block, smem, s>>>(                                \
         (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, a.b, a.li, a.m, (const TS*)a.C, a.n, \
-        (TIO*)a.h, a.abar, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale, plane, a.keep_lo);             \
+        (TIO*)a.h, a.abar, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale, plane, a.keep_lo,             \
+        a.init.on(), a.init.on() ? a.init.m : nullptr);                                          \
   } while (0)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_OUT_FWD(bf16, bf16, true);

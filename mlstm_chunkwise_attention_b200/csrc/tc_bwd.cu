@@ -76,6 +76,8 @@ struct BwdTcParams {
   bf16* out;            // dq, dk or dv [BH, T, d_out]
   float* pdot;          // dq: pq; dk: pk (atomically accumulated)
   int T, L, NC, BH, ntq, nsl, d_out, dqk;  // nsl: output column slices of D2S
+  bool m0set;                              // the forward started from an initial state
+  const float* m0;                         // its max state (mLSTMexp), else null
   float scale, log2_scale;
 };
 
@@ -109,7 +111,8 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   // partner tiles: dq: 0..it_tile; dk, dv: it_tile..nt_len-1
   const int pj0 = R_IS_QUERY ? 0 : it_tile;
   const int np = R_IS_QUERY ? it_tile + 1 : nt_len - it_tile;
-  const bool has_inter = R_IS_QUERY ? (c > 0) : (c < P.NC - 1);
+  // a state enters the chunk (dq: c > 0 or an initial state), one leaves it (dk, dv)
+  const bool has_inter = R_IS_QUERY ? (c > 0 || P.m0set) : (c < P.NC - 1);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -363,8 +366,8 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         const float dat = EXPV ? P.da[tok] : 0.f;
         Rexp = (bt - mt) * kLog2e + log2f(invd);
         eRow = dat / invd;
-        const float mprev = EXPV ? (c > 0 ? P.m[tok0 - 1] : -INFINITY) : 0.f;
-        const float alpha = c > 0 ? expf(bt + mprev - mt) : 0.f;
+        const float mprev = EXPV ? chunk_mprev(P.m, tok0, c, P.m0, bh) : 0.f;
+        const float alpha = has_inter ? expf(bt + mprev - mt) : 0.f;
         rs = alpha * invd;
         rvc = alpha * dat;
       } else {
@@ -626,6 +629,8 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   P.b = a.b; P.li = a.li; P.m = a.m; P.inv_den = a.inv_den; P.da = a.da;
   P.rowvec = (KIND == KDQ) ? a.n : a.dn;
   P.dot_src = (const bf16*)((KIND == KDQ) ? a.q : a.k);
+  P.m0set = a.init.on();
+  P.m0 = (a.init.on() && p.exp_variant()) ? a.init.m : nullptr;
   P.out = (bf16*)((KIND == KDQ) ? a.dq : (KIND == KDK) ? a.dk : a.dv);
   P.pdot = (KIND == KDQ) ? a.pq : a.pk;
   P.T = p.T; P.L = p.L; P.NC = p.NC; P.BH = p.BH; P.ntq = p.L / 128;

@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
     const __grid_constant__ CUtensorMap tm_h, const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
     const float* __restrict__ gn, bf16* __restrict__ h, float* __restrict__ abar_out, int T, int L,
-    int NC, int BH, int ntq, int dhv, float scale, float log2_scale) {
+    int NC, int BH, int ntq, int dhv, float scale, float log2_scale, bool has_init,
+    const float* __restrict__ m0) {
   using Cfg = OutTcCfg<DQK, DV, ALIAS>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN;
 
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
   const int nkv = qt + 1;
   const int dv0 = blockIdx.y * DV;
   const size_t tok0 = (size_t)bh * T + c0;
+  const bool has_prev = c > 0 || has_init;  // a state enters this chunk
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     const int gt = threadIdx.x - 64;
     for (int s = gt; s < nkv * BN; s += 128)
       colf[s] = s < len ? (gli[tok0 + s] - gb[tok0 + s]) * kLog2e : -INFINITY;
-    if (EXPV && c > 0)
+    if (EXPV && has_prev)
       for (int i = gt; i < DQK; i += 128) nvec[i] = gn[((size_t)bh * NC + c) * DQK + i];
   }
   tc::tc_fence_before();
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
         for (int vb = 0; vb < Cfg::VB; ++vb)
           tc::tma_load_3d(sV + vb * 16384, &tm_v, &bar[B_V], dv0 + vb * 64, c0 + j * BN, bh);
       }
-      if (ok && c > 0) {
+      if (ok && has_prev) {
         // C goes where K was once the last S is done, or (ALIAS) where V was once PV is done
         ok = ALIAS ? tc::mbar_wait(&bar[B_PV], (nkv - 1) & 1, &g_tc_fwd_error)
                    : tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, &g_tc_fwd_error);
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       // do not leave while a copy this thread issued may still be landing
       if (ok) {
         ok = tc::mbar_wait(&bar[B_V], (nkv - 1) & 1, &g_tc_fwd_error);
-        if (ok && c > 0) ok = tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
+        if (ok && has_prev) ok = tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
       }
     }
   } else if (warp == 1) {
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
         }
         tc::tc_commit(&bar[B_PV]);
       }
-      if (ok && c > 0) {
+      if (ok && has_prev) {
         ok = tc::mbar_wait(&bar[B_QS], 0, &g_tc_fwd_error) && tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
         if (ok) {
           tc::tc_fence_after();
@@ -217,9 +219,9 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     const size_t tok = tok0 + tl;
     const float bt = valid ? gb[tok] : 0.f;
     const float mt = (EXPV && valid) ? gm[tok] : 0.f;
-    const float mprev = EXPV ? (c > 0 ? gm[tok0 - 1] : -INFINITY) : 0.f;
+    const float mprev = EXPV ? chunk_mprev(gm, tok0, c, m0, bh) : 0.f;
     const float r2 = valid ? (bt - mt) * kLog2e + log2_scale : -INFINITY;
-    const float qfac = (valid && c > 0) ? expf(bt + mprev - mt) * scale : 0.f;
+    const float qfac = (valid && has_prev) ? expf(bt + mprev - mt) * scale : 0.f;
     const uint32_t aP = tc::smem_u32(sP), aQ = tc::smem_u32(sQ);
     float rowsum = 0.f;
 
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
 
     // inter-chunk operand: scale the query rows by alpha_t / sqrt(d_qk) in place
     float inter_norm = 0.f;
-    if (ok && c > 0) {
+    if (ok && has_prev) {
       ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_Q], 0, &g_tc_fwd_error));
       if (ok) {
 #pragma unroll 1
@@ -370,7 +372,8 @@ static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_
   const int ntq = p.L / 128;
   dim3 grid((unsigned)(p.BH * p.NC * ntq), (unsigned)(p.dhv / DV)), block(192);
   kern<<<grid, block, smem, s>>>(tq, tk, tv, tcm, th, a.b, a.li, a.m, a.n, (bf16*)a.h, a.abar, p.T,
-                                 p.L, p.NC, p.BH, ntq, p.dhv, p.scale, log2f(p.scale));
+                                 p.L, p.NC, p.BH, ntq, p.dhv, p.scale, log2f(p.scale), a.init.on(),
+                                 a.init.on() ? a.init.m : nullptr);
   return cudaGetLastError();
 }
 

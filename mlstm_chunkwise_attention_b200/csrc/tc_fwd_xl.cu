@@ -90,7 +90,7 @@ constexpr int kXlThreads = 352;  // K producer, MMA, 8 transform warps, V produc
 
 struct XlItem {
   int qt, bh, c, vb, t0, len, nkv;
-  bool pseudo;  // the chunk has a C_prev step (c > 0)
+  bool pseudo;  // a state enters the chunk: it has a C_prev step (c > 0, or an initial state)
 };
 
 // Work items come in pairs: query tiles ntq-1-p and p of one (head, chunk,
@@ -100,7 +100,7 @@ struct XlItem {
 // tiles stay in L2 for every query tile that reads them.  Item k is half k & 1
 // of pair k >> 1; a CTA walks pairs blockIdx.x, blockIdx.x + gridDim.x, ...
 __device__ __forceinline__ bool xl_item(int k, int BH, int NC, int NVB, int ntq, int T, int L,
-                                        XlItem& it) {
+                                        bool init, XlItem& it) {
   const int half_ntq = ntq >> 1;
   int r = k >> 1;
   const int pi = r % half_ntq;
@@ -113,7 +113,7 @@ __device__ __forceinline__ bool xl_item(int k, int BH, int NC, int NVB, int ntq,
   it.t0 = it.qt * 128;
   it.len = min(L, T - it.c * L);
   it.nkv = it.qt + 1;
-  it.pseudo = it.c > 0;
+  it.pseudo = it.c > 0 || init;
   return it.t0 < it.len;
 }
 
@@ -121,9 +121,9 @@ __device__ __forceinline__ int xl_first() { return 2 * blockIdx.x; }
 __device__ __forceinline__ int xl_succ(int k) { return (k & 1) ? k + 2 * gridDim.x - 1 : k + 1; }
 
 __device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB, int ntq, int T,
-                                       int L, XlItem& it) {
+                                       int L, bool init, XlItem& it) {
   for (; k < total; k = xl_succ(k))
-    if (xl_item(k, BH, NC, NVB, ntq, T, L, it)) return k;
+    if (xl_item(k, BH, NC, NVB, ntq, T, L, init, it)) return k;
   return total;
 }
 
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
     const float* __restrict__ tab, const float* __restrict__ gn, bf16* __restrict__ hout,
     float* __restrict__ abar_out, int T, int L, int NC, int BH, int NVB, int ntq, int total,
-    int tstride, int dhv) {
+    int tstride, int dhv, bool has_init) {
   using Cfg = XlCfg<DQK, DV>;
   constexpr int NQ = Cfg::NQ, NK = Cfg::NK, NV = Cfg::NV;
   // an earlier CTA gave up: the whole block leaves together
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       int it = 0, g = 0;
       for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
         XlItem I;
-        if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
+        if (!xl_item(k, BH, NC, NVB, ntq, T, L, has_init, I)) continue;
         const int qb = it % NQ;
         ok = __all_sync(full, tc::mbar_wait(&bar[X_QE0 + qb], ((it / NQ) & 1) ^ 1, abort_flag));
         if (!ok) break;
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       int gv = 0;
       for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
         XlItem I;
-        if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
+        if (!xl_item(k, BH, NC, NVB, ntq, T, L, has_init, I)) continue;
         const float* tb = tab + ((size_t)I.bh * NC + I.c) * tstride;
         for (int j = 0; j < I.nkv && ok; ++j, ++gv) {
           const int st = gv % NV;
@@ -420,11 +420,11 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       };
 
       XlItem I, N;
-      int k = xl_next(xl_first(), total, BH, NC, NVB, ntq, T, L, I);
+      int k = xl_next(xl_first(), total, BH, NC, NVB, ntq, T, L, has_init, I);
       int it = 0, g = 0, gv = 0;
       if (k < total) ok = issue_s(I, 0, 0, 0);
       while (k < total && ok) {
-        const int kn = xl_next(xl_succ(k), total, BH, NC, NVB, ntq, T, L, N);
+        const int kn = xl_next(xl_succ(k), total, BH, NC, NVB, ntq, T, L, has_init, N);
         const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
         for (int s = 0; s < nsteps && ok; ++s, ++g) {
           const bool last = s + 1 == nsteps;
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
 
     for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
       XlItem I;
-      if (!xl_item(k, BH, NC, NVB, ntq, T, L, I)) continue;
+      if (!xl_item(k, BH, NC, NVB, ntq, T, L, has_init, I)) continue;
       const int qb = it % NQ;
       ok = __all_sync(full, tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag));
       if (!ok) break;
@@ -690,7 +690,7 @@ static cudaError_t launch_out_xl(const Problem& p, const FwdArgs& a, cudaStream_
   const int grid = (int)(pairs < nsm ? pairs : nsm);
   kern<<<grid, kXlThreads, smem, s>>>(tq, tk, tv, tcm, a.xt, a.n, (bf16*)a.h, a.abar, p.T, p.L,
                                       p.NC, p.BH, nvb, ntq, (int)total, xl_table_stride(p.L),
-                                      p.dhv);
+                                      p.dhv, a.init.on());
   return cudaGetLastError();
 }
 

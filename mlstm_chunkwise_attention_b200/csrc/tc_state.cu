@@ -69,6 +69,8 @@ struct StateTcParams {
   size_t plane;
   int T, L, NC, dqk, dhv;
   float scale;
+  InitState init;   // forward: the state entering chunk 0; both: its max state m0
+  float *d0, *dn0;  // backward: gradient of the initial state (C, n), fp32, or null
 };
 
 template <bool BWD, bool EXPV, int NV>
@@ -86,7 +88,10 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   const bool with_n = EXPV && blockIdx.x == 0;
   const size_t tokh = (size_t)bh * P.T;
   const int NC = P.NC;
-  const int nsteps = NC - 1;  // chunks whose contribution is needed
+  // chunks whose contribution is needed: all but the last (forward) or the first
+  // (backward), and the backward's first too when the initial state's gradient is wanted
+  const int nsteps = NC - 1 + ((BWD && P.d0 != nullptr) ? 1 : 0);
+  const float* m0 = P.init.on() ? P.init.m : nullptr;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         wv = expf(g - P.b[t] + P.li[t] - mc);
         wn = wv;
       } else {
-        const float mprev = EXPV ? (c > 0 ? P.m[ct - 1] : -INFINITY) : 0.f;
+        const float mprev = EXPV ? chunk_mprev(P.m, ct, c, m0, bh) : 0.f;
         const float mt = EXPV ? P.m[t] : 0.f;
         const float alpha = expf(P.b[t] + mprev - mt) * P.scale;
         wv = alpha * (EXPV ? P.inv_den[t] : 1.f);
@@ -269,11 +274,14 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
     const int i = 32 * (warp & 3) + lane;  // state row within the tile (TMEM lane)
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const bool valid = dk0 + i < P.dqk;
+    // the running state: the forward starts from the initial state (zero without one)
     float S[NV];
+    const bool from_init = !BWD && P.init.on() && valid;
 #pragma unroll
-    for (int j = 0; j < NV; ++j) S[j] = 0.f;
-    float sn = 0.f;
-    for (int u = 0; u <= nsteps; ++u) {
+    for (int j = 0; j < NV; ++j)
+      S[j] = from_init ? P.init.C[((size_t)bh * P.dqk + dk0 + i) * P.dhv + dv0 + j] : 0.f;
+    float sn = (from_init && with_n) ? P.init.n[(size_t)bh * P.dqk + dk0 + i] : 0.f;
+    for (int u = 0; u < NC; ++u) {
       const int c = chunk_of(u);
       // store the state at this chunk boundary: rows into the swizzled staging
       // tile, then one TMA store per plane issued by thread 0 of the epilogue
@@ -318,15 +326,15 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
-      if (u == nsteps) break;
+      if (u == nsteps) break;  // the state leaving this chunk is not needed
       const int c0 = c * P.L, len = min(P.L, P.T - c0);
       const size_t ct = tokh + c0;
       const float g = P.b[ct + len - 1];
       float beta;
       if (EXPV) {
         const float mc = P.m[ct + len - 1];
-        const float mp = c > 0 ? P.m[ct - 1] : -INFINITY;
-        beta = c > 0 ? expf(g + mp - mc) : 0.f;
+        const float mp = chunk_mprev(P.m, ct, c, m0, bh);
+        beta = (c > 0 || m0 != nullptr) ? expf(g + mp - mc) : 0.f;
       } else {
         beta = expf(g);
       }
@@ -349,6 +357,14 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[SB_UFREE0 + ub]);
+    }
+    // backward with the initial state's gradient: after the first chunk's contribution
+    // the running state is the gradient of the state entering it
+    if (BWD && P.d0 != nullptr && ok && valid) {
+      float4* dst = reinterpret_cast<float4*>(P.d0 + ((size_t)bh * P.dqk + dk0 + i) * P.dhv + dv0);
+#pragma unroll
+      for (int j = 0; j < NV; j += 4) dst[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+      if (with_n) P.dn0[(size_t)bh * P.dqk + dk0 + i] = sn;
     }
   }
 
@@ -374,7 +390,8 @@ bool state_tc_supported(const Problem& p) {
 template <bool BWD, bool EXPV, int NV>
 static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* B, bf16* out,
                                    float* nout, const float* b, const float* li, const float* m,
-                                   const float* inv_den, const float* da, cudaStream_t s) {
+                                   const float* inv_den, const float* da, const InitState& init,
+                                   float* d0, float* dn0, cudaStream_t s) {
   using Cfg = StateTcCfg<NV>;
   CUtensorMap tA, tB, tOh, tOl;
   const uint64_t plane = (uint64_t)p.BH * p.NC * p.dqk * p.dhv;
@@ -390,6 +407,9 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
   P.plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
   P.T = p.T; P.L = p.L; P.NC = p.NC; P.dqk = p.dqk; P.dhv = p.dhv;
   P.scale = p.scale;
+  P.init = init;
+  P.d0 = d0;
+  P.dn0 = dn0;
   auto kern = state_tc_kernel<BWD, EXPV, NV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
@@ -403,24 +423,25 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
 template <bool BWD, bool EXPV>
 static cudaError_t launch_state_tc_nv(const Problem& p, const void* A, const void* B, bf16* out,
                                       float* nout, const float* b, const float* li, const float* m,
-                                      const float* inv_den, const float* da, cudaStream_t s) {
-  return launch_state_tc<BWD, EXPV, 64>(p, A, B, out, nout, b, li, m, inv_den, da, s);
+                                      const float* inv_den, const float* da, const InitState& init,
+                                      float* d0, float* dn0, cudaStream_t s) {
+  return launch_state_tc<BWD, EXPV, 64>(p, A, B, out, nout, b, li, m, inv_den, da, init, d0, dn0, s);
 }
 
 cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   if (p.exp_variant())
     return launch_state_tc_nv<false, true>(p, a.k, a.v, (bf16*)a.C, a.n, a.b, a.li, a.m, nullptr,
-                                           nullptr, s);
+                                           nullptr, a.init, nullptr, nullptr, s);
   return launch_state_tc_nv<false, false>(p, a.k, a.v, (bf16*)a.C, a.n, a.b, a.li, a.m, nullptr,
-                                          nullptr, s);
+                                          nullptr, a.init, nullptr, nullptr, s);
 }
 
 cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
   if (p.exp_variant())
     return launch_state_tc_nv<true, true>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
-                                          a.inv_den, a.da, s);
+                                          a.inv_den, a.da, a.init, a.dC0, a.dn0, s);
   return launch_state_tc_nv<true, false>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
-                                         a.inv_den, a.da, s);
+                                         a.inv_den, a.da, a.init, a.dC0, a.dn0, s);
 }
 
 cudaError_t fetch_tc_state_error(unsigned int* flag) {

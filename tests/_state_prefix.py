@@ -1,0 +1,86 @@
+"""A recurrent state written as a prefix of tokens (test construction, fp64).
+
+Starting the mLSTM recurrence from a state (C, n, m) is the same as running it
+from the zero state over d_qk extra tokens placed first, whose only effect on
+every later token is to leave exactly that state behind:
+  token j = 0 .. d_qk - 1:  k_j = e_j (unit vector), q_j = 0, log f_j = 0,
+  so after them the unstabilised state is C = sum_j i_j e_j v_j^T (row j is
+  i_j v_j) and n = sum_j i_j e_j (entry j is i_j).
+  SIG (no normaliser): i_j = 1/2, v_j = 2 C[j].
+  EXP: the stabilised state (C~, n~, m) stands for exp(m) (C~, n~); with
+  i_j = exp(m) n~_j (so n~ > 0 is needed) and v_j = C~[j] / n~_j.
+Their own outputs are zero (q = 0) and dropped.  Later tokens then see the
+state decayed by their own forget gates, as in the recurrence started from it,
+so the oracle's forward and backward over the longer sequence give the
+expected values of a call that starts from a state, with no new oracle code;
+test_state_prefix.py pins the construction against the oracle's own
+one-token step.
+"""
+
+import numpy as np
+
+import oracle
+
+
+def prefix(C, n, m, variant):
+    """q, k, v, log_i, log_f of the d_qk prefix tokens for the state (C, n, m) of one head."""
+    C = np.asarray(C, dtype=np.float64)
+    d_qk, _ = C.shape
+    k = np.eye(d_qk)
+    q = np.zeros((d_qk, d_qk))
+    log_f = np.zeros(d_qk)
+    if variant == oracle.SIG:
+        log_i = np.full(d_qk, np.log(0.5))
+        v = 2.0 * C
+    else:
+        n = np.asarray(n, dtype=np.float64)
+        assert np.all(n > 0), "the construction needs a positive normaliser state"
+        log_i = float(m) + np.log(n)
+        v = C / n[:, None]
+    return q, k, v, log_i, log_f
+
+
+def extend(pre, q, k, v, log_i, log_f):
+    """The prefix followed by the real tokens."""
+    return tuple(np.concatenate([np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)])
+                 for a, b in zip(pre, (q, k, v, log_i, log_f)))
+
+
+def state_grads(pre, dk_pre, dv_pre, m, variant):
+    """Gradient of the loss with respect to the stabilised state (C~, n~), from the
+    prefix tokens' dk, dv (m held constant).
+
+    Row j of the true C is i_j v_j, so dL/dC_true[j] = dv_j / i_j; entry j of the
+    true n is i_j (k_j = e_j enters C and n), so dk_j[j] = i_j (dC_true[j] . v_j +
+    dn_true[j]).  The stabilised state is exp(-m) times the true one, so its
+    gradient is exp(m) times the true gradient (exp(m) = 1 for SIG).
+    """
+    _, _, v, log_i, _ = pre
+    i = np.exp(log_i)
+    dC_true = dv_pre / i[:, None]
+    scale = 1.0 if variant == oracle.SIG else float(np.exp(m))
+    dC = scale * dC_true
+    dn = None
+    if variant == oracle.EXP:
+        diag = np.diagonal(dk_pre)
+        dn_true = diag / i - np.sum(dC_true * v, axis=1)
+        dn = scale * dn_true
+    return dC, dn
+
+
+def true_state(C, n, m, variant):
+    """exp(m) (C, n): the unstabilised state (SIG: C itself)."""
+    if variant == oracle.SIG:
+        return np.asarray(C, dtype=np.float64), None
+    s = float(np.exp(m))
+    return s * np.asarray(C, dtype=np.float64), s * np.asarray(n, dtype=np.float64)
+
+
+def random_state(rng, d_qk, d_hv, variant, scale=0.3):
+    """A state of one head: C ~ N(0, scale^2), n~ in [0.5, 2) (EXP), m ~ N(0, 1) (EXP)."""
+    C = rng.standard_normal((d_qk, d_hv)) * scale
+    if variant == oracle.SIG:
+        return C, None, 0.0
+    n = rng.uniform(0.5, 2.0, d_qk)
+    m = float(rng.standard_normal())
+    return C, n, m

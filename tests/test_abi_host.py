@@ -157,3 +157,26 @@ def test_state_layout_and_argument_errors(lib):
     assert lib.mlstm_state_zero(None, 0, 2, 64, 64, B.EXP, None) == 0
     assert lib.mlstm_step(*[None] * 8, 0, 2, 64, 64, B.SIG, B.BF16, None) == 0
     assert lib.mlstm_final_state(None, None, None, None, 0, 2, 5, 64, 64, 64, B.SIG, B.BF16, None) == 0
+
+
+def test_chunkwise_state_entry_points_argument_errors(lib):
+    """mlstm_fwd_state / mlstm_bwd_state: argument errors are returned before any launch."""
+    fake, other = 0x10000, 0x20000  # aligned addresses, never dereferenced
+    sizes = (1, 2, 256, 64, 64, 64, B.EXP, B.BF16)
+    fwd_in = (fake,) * 6 + (fake, None, 0)  # q k v ig fg h, saved, workspace, bytes
+    # overlapping initial and final states
+    assert lib.mlstm_fwd_state(*fwd_in, fake, fake + 256, *sizes, None) == B.STATUS_INVALID
+    # misaligned states
+    assert lib.mlstm_fwd_state(*fwd_in, fake + 8, other, *sizes, None) == B.STATUS_INVALID
+    assert lib.mlstm_fwd_state(*fwd_in, fake, other + 4, *sizes, None) == B.STATUS_INVALID
+    # unsupported sizes come first
+    assert lib.mlstm_fwd_state(*fwd_in, fake, other, 1, 2, 256, 100, 64, 64, B.EXP, B.BF16,
+                               None) == B.STATUS_UNSUPPORTED
+    bwd_in = (fake,) * 8  # q k v ig fg h dh saved
+    outs = (fake,) * 5 + (fake, 1 << 30)  # dq dk dv dig dfg, workspace, bytes
+    assert lib.mlstm_bwd_state(*bwd_in, fake, fake + 512, *outs, *sizes, None) == B.STATUS_INVALID
+    assert lib.mlstm_bwd_state(*bwd_in, fake, other + 4, *outs, *sizes, None) == B.STATUS_INVALID
+    # empty problems are no-ops
+    assert lib.mlstm_fwd_state(*[None] * 8, 0, None, None, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16,
+                               None) == 0
+    assert lib.mlstm_bwd_state(*[None] * 16, 0, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16, None) == 0
