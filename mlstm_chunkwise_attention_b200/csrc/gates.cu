@@ -189,6 +189,9 @@ __global__ void __launch_bounds__(256) bwd_token_prep_kernel(
   for (long long base = warp_id * tpw; base < ntok; base += nwarps * tpw) {
     const long long tok = base + sub;
     const bool valid = tok < ntok;
+    // the token's normaliser and max state load alongside its rows, not after the dot product
+    const float a = (EXPV && valid && sl == 0) ? abar[tok] : 0.f;
+    const float mtok = (EXPV && valid && sl == 0) ? m[tok] : 0.f;
     float dot = 0.f;
     if (EXPV && valid) {
       const TIO* hr = h + tok * dhv;
@@ -207,8 +210,7 @@ __global__ void __launch_bounds__(256) bwd_token_prep_kernel(
       pq[tok] = 0.f;
       pk[tok] = 0.f;
       if (EXPV) {
-        const float a = abar[tok];
-        const float floor_ = expf(-m[tok]);
+        const float floor_ = expf(-mtok);
         const float den = fmaxf(fabsf(a), floor_);
         inv_den[tok] = 1.f / den;
         da[tok] = fabsf(a) > floor_ ? -dot * copysignf(1.f, a) / den : 0.f;
