@@ -124,6 +124,17 @@ def source_sha(kernel):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def reduce_max(v, world, device):
+    """The largest of every rank's v (one all-reduce; v itself when world == 1)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def committed_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -678,11 +689,7 @@ def main():
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     # ---- device-timed region: inputs resident in HBM
     for _ in range(args.warmup):

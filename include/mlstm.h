@@ -218,8 +218,9 @@ int mlstm_step(const void* q, const void* k, const void* v, const void* igate_pr
  * state (its C and n, and m as the first chunk's m_{c-1}), and state_out is
  * mlstm_final_state's result.  state_in and state_out must not overlap
  * (MLSTM_ERR_INVALID).  T = 0 copies state_in (or the zero state) to
- * state_out.  The saved buffer of such a call is for mlstm_bwd_state with the
- * same state_in. */
+ * state_out.  h may be NULL when state_out is not: the state-only pass (gate
+ * preprocessing, chunk states and the final state, no output kernel).  The
+ * saved buffer of such a call is for mlstm_bwd_state with the same state_in. */
 int mlstm_fwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
                     const void* fgate_pre, void* h, void* saved, void* workspace,
                     size_t workspace_bytes, const void* state_in, void* state_out, int B, int NH,
@@ -243,6 +244,35 @@ int mlstm_bwd_state(const void* q, const void* k, const void* v, const void* iga
                     void* digate_pre, void* dfgate_pre, void* workspace, size_t workspace_bytes,
                     int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype,
                     void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Sequence segments.  A sequence split into consecutive segments (one per
+ * GPU, say) is processed exactly by: the state-only pass of every segment from
+ * the zero state (mlstm_fwd_state with h = NULL), each segment's total log
+ * forget gate (mlstm_log_decay), an exchange of both, the state entering every
+ * segment by chaining the earlier segments' states (mlstm_state_chain), and a
+ * forward of every segment from that state.  "Tiled Flash Linear Attention",
+ * TFLA summary page, Problem and Approach (states at chunk boundaries carry
+ * everything a later chunk needs, so they can cross a device boundary too).
+ * ------------------------------------------------------------------------- */
+
+/* log_decay [B*NH] (fp32, written) = sum over the T tokens of
+ * log sigmoid(fgate_pre) for every head; fgate_pre [B, NH, T] in the I/O
+ * dtype.  T = 0 writes zeros.  Errors: MLSTM_ERR_INVALID (NULL or misaligned
+ * pointer), MLSTM_ERR_UNSUPPORTED, MLSTM_ERR_CUDA. */
+int mlstm_log_decay(const void* fgate_pre, float* log_decay, int B, int NH, int T, int dtype,
+                    void* stream);
+
+/* state_out = the state after segment b when b starts from state_a, given
+ * state_b (b's final state from the zero state) and b's log_decay:
+ * unstabilised, exp(G_b) (state a) + (state b); for mLSTMexp the stabilised
+ * form with m = max(G_b + m_a, m_b) (the max-state recurrence unrolled over
+ * the segment).  All three buffers in the state layout above, fp32;
+ * state_out must not overlap state_a or state_b (MLSTM_ERR_INVALID). */
+int mlstm_state_chain(const void* state_a, const void* state_b, const float* log_decay_b,
+                      void* state_out, int B, int NH, int d_qk, int d_hv, int variant,
+                      void* stream);
+
 
 /* Synchronise `stream` and report what the kernels enqueued so far found:
  * MLSTM_ERR_TIMEOUT if one of them gave up a bounded wait (its outputs are

@@ -65,6 +65,8 @@ EXPORTS = {
     "mlstm_step": (ctypes.c_int, [_P] * 8 + [ctypes.c_int] * 6 + [_P]),
     "mlstm_fwd_state": (ctypes.c_int, [_P] * 7 + [_P, ctypes.c_size_t, _P, _P] + _SIZES + [_P]),
     "mlstm_bwd_state": (ctypes.c_int, [_P] * 15 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
+    "mlstm_log_decay": (ctypes.c_int, [_P, _P] + [ctypes.c_int] * 4 + [_P]),
+    "mlstm_state_chain": (ctypes.c_int, [_P] * 4 + [ctypes.c_int] * 5 + [_P]),
 }
 
 
@@ -315,17 +317,18 @@ def final_state(k, v, saved, chunk, variant, *, state=None, stream=None):
 
 
 def forward_state(q, k, v, igate_pre, fgate_pre, chunk, variant, state_in=None, *,
-                  keep_saved=True, stream=None):
+                  keep_saved=True, want_h=True, stream=None):
     """Chunkwise forward continuing from ``state_in`` (None: the zero state).
 
     Returns (h, saved, state_out): state_out is a fresh state buffer holding the state
-    after the last token; saved (None when keep_saved is False) is for backward_state.
+    after the last token; saved (None when keep_saved is False) is for backward_state;
+    h is None when want_h is False (the state-only pass).
     """
     import torch
     _check({"q": q, "k": k, "v": v, "igate_pre": igate_pre, "fgate_pre": fgate_pre}, q.dtype)
     sizes = problem_sizes(q, v, chunk, variant)
     B, NH, T, d_qk, d_hv = sizes[:5]
-    h = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    h = torch.empty(v.shape, dtype=q.dtype, device=q.device) if want_h else None
     state_out = torch.empty(load().mlstm_state_size(B, NH, d_qk, d_hv, variant), dtype=torch.uint8,
                             device=q.device)
     saved = ws = None
@@ -335,7 +338,7 @@ def forward_state(q, k, v, igate_pre, fgate_pre, chunk, variant, state_in=None, 
         ws = torch.empty(max(mlstm_fwd_workspace_size(*sizes), 1), dtype=torch.uint8,
                          device=q.device)
     st = mlstm_fwd_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
-                         fgate_pre.data_ptr(), h.data_ptr(),
+                         fgate_pre.data_ptr(), h.data_ptr() if h is not None else None,
                          saved.data_ptr() if saved is not None else None,
                          ws.data_ptr() if ws is not None else None,
                          ws.numel() if ws is not None else 0,
@@ -344,6 +347,32 @@ def forward_state(q, k, v, igate_pre, fgate_pre, chunk, variant, state_in=None, 
     if st != STATUS_OK:
         raise MLSTMError(st, "mlstm_fwd_state")
     return h, saved, state_out
+
+
+def log_decay(fgate_pre, *, stream=None):
+    """sum_t log sigmoid(fgate_pre) per head: float32 [B, NH]."""
+    import torch
+    B, NH, T = fgate_pre.shape
+    out = torch.empty((B, NH), dtype=torch.float32, device=fgate_pre.device)
+    st = load().mlstm_log_decay(fgate_pre.data_ptr(), out.data_ptr(), B, NH, T,
+                                _dtype_code(fgate_pre), _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_log_decay")
+    return out
+
+
+def state_chain(state_a, state_b, log_decay_b, B, NH, d_qk, d_hv, variant, *, out=None,
+                stream=None):
+    """The state after segment b when it starts from state_a (see include/mlstm.h)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(state_a)
+    st = load().mlstm_state_chain(state_a.data_ptr(), state_b.data_ptr(), log_decay_b.data_ptr(),
+                                  out.data_ptr(), B, NH, d_qk, d_hv, variant,
+                                  _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_state_chain")
+    return out
 
 
 def backward_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, state_in=None, *,

@@ -116,5 +116,10 @@ cudaError_t launch_step(const Problem& p, const void* q, const void* k, const vo
                         const float* min_, float* Cout, float* nout, float* mout, cudaStream_t s);
 cudaError_t launch_state_zero(int BH, int dqk, int dhv, bool exp_variant, float* C, float* n, float* m,
                               cudaStream_t s);
+cudaError_t launch_log_decay(const Problem& p, const void* fg, float* G, cudaStream_t s);
+cudaError_t launch_state_chain(int BH, int dqk, int dhv, bool exp_variant, const float* Ca,
+                               const float* na, const float* ma, const float* Cb, const float* nb,
+                               const float* mb, const float* G, float* Co, float* no, float* mo,
+                               cudaStream_t s);
 
 }  // namespace mlstm

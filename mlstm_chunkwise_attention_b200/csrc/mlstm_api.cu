@@ -288,7 +288,8 @@ int fwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
                                        (cudaStream_t)stream),
                        "state copy");
   }
-  if (!q || !k || !v || !igate_pre || !fgate_pre || !h) return MLSTM_ERR_INVALID;
+  // h == NULL with a state_out: the state-only pass (no output kernel)
+  if (!q || !k || !v || !igate_pre || !fgate_pre || (!h && !state_out)) return MLSTM_ERR_INVALID;
   if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(h) ||
       misaligned(igate_pre) || misaligned(fgate_pre) || misaligned(saved) ||
       misaligned(workspace))
@@ -318,7 +319,7 @@ int fwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   if (st != MLSTM_OK) return st;
   FwdStep steps[kMaxSteps];
   const int n = fwd_plan(p, steps);
-  st = run_plan(steps, n, p, a, s);
+  st = run_plan(steps, h ? n : n - 1, p, a, s);  // the output kernel is the plan's last step
   if (st != MLSTM_OK || !state_out) return st;
   char* out = (char*)state_out;
   return cuda_status(mlstm::launch_final_state(p, k, v, a.b, a.li, a.m, a.C, a.n, a.init,
@@ -505,6 +506,52 @@ int mlstm_step(const void* q, const void* k, const void* v, const void* igate_pr
                          (const float*)(si + S.n), (const float*)(si + S.m), (float*)(so + S.C),
                          (float*)(so + S.n), (float*)(so + S.m), (cudaStream_t)stream),
       "step");
+}
+
+int mlstm_log_decay(const void* fgate_pre, float* log_decay, int B, int NH, int T, int dtype,
+                    void* stream) {
+  int st = check_sizes(B, NH, T, 64, 64, 64, MLSTM_SIG, dtype);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (!log_decay || misaligned(log_decay) || (T > 0 && (!fgate_pre || misaligned(fgate_pre))))
+    return MLSTM_ERR_INVALID;
+  if (T == 0)
+    return cuda_status(cudaMemsetAsync(log_decay, 0, (size_t)B * NH * sizeof(float),
+                                       (cudaStream_t)stream),
+                       "memset");
+  const Problem p = make_problem(B, NH, T, 64, 64, 64, MLSTM_SIG, dtype);
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_log_decay");
+  if (st != MLSTM_OK) return st;
+  return cuda_status(mlstm::launch_log_decay(p, fgate_pre, log_decay, (cudaStream_t)stream),
+                     "log_decay");
+}
+
+int mlstm_state_chain(const void* state_a, const void* state_b, const float* log_decay_b,
+                      void* state_out, int B, int NH, int d_qk, int d_hv, int variant,
+                      void* stream) {
+  int st = check_sizes(B, NH, 1, d_qk, d_hv, 64, variant, MLSTM_FP32);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (!state_a || !state_b || !log_decay_b || !state_out) return MLSTM_ERR_INVALID;
+  const void* ptrs[] = {state_a, state_b, log_decay_b, state_out};
+  for (const void* ptr : ptrs)
+    if (misaligned(ptr)) return MLSTM_ERR_INVALID;
+  const bool e = variant == MLSTM_EXP;
+  const StateLayout S = state_layout(B * NH, d_qk, d_hv, e);
+  if (overlaps(state_out, state_a, S.total) || overlaps(state_out, state_b, S.total))
+    return MLSTM_ERR_INVALID;
+  const char* pa = (const char*)state_a;
+  const char* pb = (const char*)state_b;
+  char* po = (char*)state_out;
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_state_chain");
+  if (st != MLSTM_OK) return st;
+  return cuda_status(
+      mlstm::launch_state_chain(B * NH, d_qk, d_hv, e, (const float*)(pa + S.C),
+                                (const float*)(pa + S.n), (const float*)(pa + S.m),
+                                (const float*)(pb + S.C), (const float*)(pb + S.n),
+                                (const float*)(pb + S.m), log_decay_b, (float*)(po + S.C),
+                                (float*)(po + S.n), (float*)(po + S.m), (cudaStream_t)stream),
+      "state_chain");
 }
 
 const char* mlstm_status_string(int status) {

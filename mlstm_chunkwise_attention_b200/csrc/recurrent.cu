@@ -182,6 +182,61 @@ __global__ void fill_neg_inf_kernel(float* __restrict__ m, int count) {
   if (i < count) m[i] = kNegInf;
 }
 
+// Total log forget gate of a segment, per head: G = sum_t log sigmoid(f~_t).  One CTA
+// per head; each thread sums a strided share, then a block reduction.
+template <typename TIO>
+__global__ void __launch_bounds__(256) log_decay_kernel(const TIO* __restrict__ fg,
+                                                        float* __restrict__ G, int T) {
+  __shared__ float part[8];
+  const size_t base = (size_t)blockIdx.x * T;
+  float acc = 0.f;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) acc += log_sigmoid(to_f32(fg[base + t]));
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float g = 0.f;
+    for (int w = 0; w < 8; ++w) g += part[w];
+    G[blockIdx.x] = g;
+  }
+}
+
+// The state after segment b when b starts from state a instead of the zero state:
+// the true state is exp(G_b) (state a) + (state b), G_b the segment's total log
+// forget gate.  mLSTMexp keeps the stabilised form: m = max(G_b + m_a, m_b), the
+// max-state recurrence unrolled over the segment, and C~ = exp(G_b + m_a - m) C~_a
+// + exp(m_b - m) C~_b (n~ likewise).  One CTA per head.
+template <bool EXPV>
+__global__ void __launch_bounds__(256) state_chain_kernel(
+    const float* __restrict__ Ca, const float* __restrict__ na, const float* __restrict__ ma,
+    const float* __restrict__ Cb, const float* __restrict__ nb, const float* __restrict__ mb,
+    const float* __restrict__ G, float* __restrict__ Co, float* __restrict__ no,
+    float* __restrict__ mo, int dqk, int dhv) {
+  const int bh = blockIdx.x;
+  const float g = G[bh];
+  float fa = expf(g), fb = 1.f;
+  if (EXPV) {
+    const float x = g + ma[bh], y = mb[bh];
+    const float m = fmaxf(x, y);
+    // both -inf: two zero states, and the result is the zero state
+    fa = m == kNegInf ? 0.f : expf(x - m);
+    fb = m == kNegInf ? 0.f : expf(y - m);
+    if (threadIdx.x == 0) mo[bh] = m;
+  }
+  const size_t n4 = (size_t)dqk * dhv / 4, off = (size_t)bh * dqk * dhv / 4;
+  const float4* a4 = reinterpret_cast<const float4*>(Ca) + off;
+  const float4* b4 = reinterpret_cast<const float4*>(Cb) + off;
+  float4* o4 = reinterpret_cast<float4*>(Co) + off;
+  for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 a = a4[i], b = b4[i];
+    o4[i] = make_float4(fmaf(fa, a.x, fb * b.x), fmaf(fa, a.y, fb * b.y), fmaf(fa, a.z, fb * b.z),
+                        fmaf(fa, a.w, fb * b.w));
+  }
+  if (EXPV)
+    for (int i = threadIdx.x; i < dqk; i += blockDim.x)
+      no[(size_t)bh * dqk + i] = fmaf(fa, na[(size_t)bh * dqk + i], fb * nb[(size_t)bh * dqk + i]);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -239,6 +294,25 @@ cudaError_t launch_state_zero(int BH, int dqk, int dhv, bool exp_variant, float*
   e = cudaMemsetAsync(n, 0, (size_t)BH * dqk * sizeof(float), s);
   if (e != cudaSuccess) return e;
   fill_neg_inf_kernel<<<(BH + 255) / 256, 256, 0, s>>>(m, BH);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_log_decay(const Problem& p, const void* fg, float* G, cudaStream_t s) {
+  if (p.bf16())
+    log_decay_kernel<bf16><<<p.BH, 256, 0, s>>>((const bf16*)fg, G, p.T);
+  else
+    log_decay_kernel<float><<<p.BH, 256, 0, s>>>((const float*)fg, G, p.T);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_chain(int BH, int dqk, int dhv, bool exp_variant, const float* Ca,
+                               const float* na, const float* ma, const float* Cb, const float* nb,
+                               const float* mb, const float* G, float* Co, float* no, float* mo,
+                               cudaStream_t s) {
+  if (exp_variant)
+    state_chain_kernel<true><<<BH, 256, 0, s>>>(Ca, na, ma, Cb, nb, mb, G, Co, no, mo, dqk, dhv);
+  else
+    state_chain_kernel<false><<<BH, 256, 0, s>>>(Ca, na, ma, Cb, nb, mb, G, Co, no, mo, dqk, dhv);
   return cudaGetLastError();
 }
 

@@ -180,3 +180,18 @@ def test_chunkwise_state_entry_points_argument_errors(lib):
     assert lib.mlstm_fwd_state(*[None] * 8, 0, None, None, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16,
                                None) == 0
     assert lib.mlstm_bwd_state(*[None] * 16, 0, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16, None) == 0
+
+
+def test_segment_entry_points_argument_errors(lib):
+    """mlstm_log_decay / mlstm_state_chain: argument errors before any launch."""
+    fake, other, third = 0x10000, 0x40000, 0x80000  # aligned, never dereferenced
+    assert lib.mlstm_log_decay(fake, None, 1, 2, 100, B.BF16, None) == B.STATUS_INVALID
+    assert lib.mlstm_log_decay(fake + 2, other, 1, 2, 100, B.BF16, None) == B.STATUS_INVALID
+    assert lib.mlstm_log_decay(fake, other, 1, 2, 100, 7, None) == B.STATUS_INVALID
+    assert lib.mlstm_log_decay(None, None, 0, 2, 100, B.BF16, None) == 0
+    # the output must not overlap either input
+    assert lib.mlstm_state_chain(fake, other, third, fake + 256, 1, 2, 64, 64, B.EXP, None) == B.STATUS_INVALID
+    assert lib.mlstm_state_chain(fake, other, third, other, 1, 2, 64, 64, B.SIG, None) == B.STATUS_INVALID
+    assert lib.mlstm_state_chain(fake, other, None, third, 1, 2, 64, 64, B.SIG, None) == B.STATUS_INVALID
+    assert lib.mlstm_state_chain(fake, other, third, third + 4, 1, 2, 64, 64, B.SIG, None) == B.STATUS_INVALID
+    assert lib.mlstm_state_chain(fake, other, third, 0x100000, 1, 2, 100, 64, B.SIG, None) == B.STATUS_UNSUPPORTED
