@@ -235,15 +235,23 @@ int mlstm_fwd_state(const void* q, const void* k, const void* v, const void* iga
  *              region is not written); NULL: not wanted.  It is one more step
  *              of the state-gradient recurrence: beta_0 dC_0 + Q_0^T diag(u)
  *              dH_0 over the first chunk.
- * state_in and dstate_in must not overlap (MLSTM_ERR_INVALID).  The gradient
- * of a loss that also reads state_out is not supported here: such a loss
- * contributes through a later call's dstate_in only. */
+ *   dstate_out gradient of the loss with respect to the final state's C and
+ *              (EXP) n (state layout, read; its m region is ignored), for a loss
+ *              that also reads state_out, e.g. through a later call's
+ *              dstate_in; NULL: none.  It starts the state-gradient recurrence
+ *              (the gradient of the state leaving the last chunk), gives dk and
+ *              dv an inter-chunk term in the last chunk, and adds
+ *              <dC_T, C_T> + <dn_T, n_T> to every forget-gate gradient (the
+ *              final state reads every key before it); the final state is
+ *              rebuilt from `saved` in the workspace.
+ * dstate_in must not overlap state_in or dstate_out (MLSTM_ERR_INVALID).
+ * With T = 0 the gradient with respect to the initial state is dstate_out. */
 int mlstm_bwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
                     const void* fgate_pre, const void* h, const void* dh, const void* saved,
-                    const void* state_in, void* dstate_in, void* dq, void* dk, void* dv,
-                    void* digate_pre, void* dfgate_pre, void* workspace, size_t workspace_bytes,
-                    int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype,
-                    void* stream);
+                    const void* state_in, void* dstate_in, const void* dstate_out, void* dq,
+                    void* dk, void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
+                    size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                    int variant, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Sequence segments.  A sequence split into consecutive segments (one per

@@ -64,7 +64,7 @@ EXPORTS = {
     "mlstm_final_state": (ctypes.c_int, [_P] * 4 + _SIZES + [_P]),
     "mlstm_step": (ctypes.c_int, [_P] * 8 + [ctypes.c_int] * 6 + [_P]),
     "mlstm_fwd_state": (ctypes.c_int, [_P] * 7 + [_P, ctypes.c_size_t, _P, _P] + _SIZES + [_P]),
-    "mlstm_bwd_state": (ctypes.c_int, [_P] * 15 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
+    "mlstm_bwd_state": (ctypes.c_int, [_P] * 16 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
     "mlstm_log_decay": (ctypes.c_int, [_P, _P] + [ctypes.c_int] * 4 + [_P]),
     "mlstm_state_chain": (ctypes.c_int, [_P] * 4 + [ctypes.c_int] * 5 + [_P]),
 }
@@ -147,12 +147,13 @@ def mlstm_fwd_state(q, k, v, igate_pre, fgate_pre, h, saved, workspace, workspac
                                   variant, dtype, stream)
 
 
-def mlstm_bwd_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in, dq, dk, dv,
-                    digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
-                    variant, dtype, stream):
+def mlstm_bwd_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in, dstate_out,
+                    dq, dk, dv, digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk,
+                    d_hv, chunk, variant, dtype, stream):
     return load().mlstm_bwd_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in,
-                                  dq, dk, dv, digate_pre, dfgate_pre, workspace, workspace_bytes, B,
-                                  NH, T, d_qk, d_hv, chunk, variant, dtype, stream)
+                                  dstate_out, dq, dk, dv, digate_pre, dfgate_pre, workspace,
+                                  workspace_bytes, B, NH, T, d_qk, d_hv, chunk, variant, dtype,
+                                  stream)
 
 
 def mlstm_status_string(status):
@@ -376,8 +377,9 @@ def state_chain(state_a, state_b, log_decay_b, B, NH, d_qk, d_hv, variant, *, ou
 
 
 def backward_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, state_in=None, *,
-                   want_dstate=True, stream=None):
-    """Gradients of sum(dh * h) for a forward_state call, the initial state held constant.
+                   dstate_out=None, want_dstate=True, stream=None):
+    """Gradients of sum(dh * h) (+ <dstate_out, final state> when dstate_out, a state-layout
+    buffer, is given) for a forward_state call, the initial state held constant.
 
     Returns the dict of ``backward`` plus "dstate_in" (a state-layout buffer whose C and,
     for EXP, n regions hold the gradient with respect to state_in) when want_dstate.
@@ -397,6 +399,7 @@ def backward_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, 
                          fgate_pre.data_ptr(), h.data_ptr(), dh.data_ptr(), saved.data_ptr(),
                          state_in.data_ptr() if state_in is not None else None,
                          out["dstate_in"].data_ptr() if want_dstate else None,
+                         dstate_out.data_ptr() if dstate_out is not None else None,
                          out["dq"].data_ptr(), out["dk"].data_ptr(), out["dv"].data_ptr(),
                          out["digate_pre"].data_ptr(), out["dfgate_pre"].data_ptr(),
                          ws.data_ptr(), ws.numel(), *sizes, _stream_handle(stream))

@@ -251,7 +251,8 @@ cudaError_t launch_bwd_token_prep(const Problem& p, const BwdArgs& a, cudaStream
 template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(1024) gate_grad_kernel(
     const TIO* __restrict__ ig, const TIO* __restrict__ fg, const float* __restrict__ pq,
-    const float* __restrict__ pk, TIO* __restrict__ dig, TIO* __restrict__ dfg, int T) {
+    const float* __restrict__ pk, TIO* __restrict__ dig, TIO* __restrict__ dfg, int T,
+    const float* __restrict__ fdot) {
   __shared__ float s_tot[32];
   const size_t base = (size_t)blockIdx.x * T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -268,7 +269,9 @@ __global__ void __launch_bounds__(1024) gate_grad_kernel(
     s_tot[lane] = incl - x;  // sum of the later segments
   }
   __syncthreads();
-  float carry = s_tot[warp];
+  // a loss on the final state adds <dC_T, C_T> + <dn_T, n_T> to every d log f_r: the
+  // final state is one more row after the last token, and it reads every key
+  float carry = s_tot[warp] + (fdot != nullptr ? fdot[blockIdx.x] : 0.f);
   for (int e = se; e > sb; e -= 32) {
     const int t = e - 32 + lane;
     const bool valid = t >= sb;
@@ -290,14 +293,14 @@ cudaError_t launch_gate_grad(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH), block(1024);
   if (p.bf16()) {
     if (p.exp_variant())
-      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T);
+      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot);
     else
-      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T);
+      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot);
   } else {
     if (p.exp_variant())
-      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T);
+      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot);
     else
-      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T);
+      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot);
   }
   return cudaGetLastError();
 }

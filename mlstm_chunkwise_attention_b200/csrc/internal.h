@@ -72,6 +72,9 @@ struct BwdArgs {
   InitState init;  // the state the forward started from (held constant)
   float* dC0;      // gradient of the initial state: C [BH, dqk, dhv] (null: not wanted)
   float* dn0;      // and n [BH, dqk] (mLSTMexp)
+  const float* dCT;  // gradient with respect to the final state: C [BH, dqk, dhv] (null: none)
+  const float* dnT;  // and n [BH, dqk] (mLSTMexp)
+  float* fdot;       // [BH] <dC_T, C_T> + <dn_T, n_T>, added to every forget-gate gradient
 };
 
 // gate kernels (gates.cu)
@@ -117,6 +120,9 @@ cudaError_t launch_step(const Problem& p, const void* q, const void* k, const vo
 cudaError_t launch_state_zero(int BH, int dqk, int dhv, bool exp_variant, float* C, float* n, float* m,
                               cudaStream_t s);
 cudaError_t launch_log_decay(const Problem& p, const void* fg, float* G, cudaStream_t s);
+cudaError_t launch_state_dot(int BH, int dqk, int dhv, bool exp_variant, const float* Ca,
+                             const float* na, const float* Cb, const float* nb, float* out,
+                             cudaStream_t s);
 cudaError_t launch_state_chain(int BH, int dqk, int dhv, bool exp_variant, const float* Ca,
                                const float* na, const float* ma, const float* Cb, const float* nb,
                                const float* mb, const float* G, float* Co, float* no, float* mo,

@@ -68,26 +68,6 @@ void saved_layout(const Problem& p, mlstm_saved_layout_t* L) {
   L->total = off;
 }
 
-struct BwdLayout {
-  size_t inv_den, da, pq, pk, dC, dn, total;
-};
-
-BwdLayout bwd_layout(const Problem& p) {
-  BwdLayout L;
-  const size_t tok = (size_t)p.BH * p.T;
-  size_t off = 0;
-  L.inv_den = off; off = align256(off + tok * 4);
-  L.da = off;      off = align256(off + tok * 4);
-  L.pq = off;      off = align256(off + tok * 4);
-  L.pk = off;      off = align256(off + tok * 4);
-  L.dC = off;      off = align256(off + (size_t)p.BH * p.NC * p.dqk * p.dhv * 4);
-  L.dn = off;      off = align256(off + (p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0));
-  L.total = off;
-  return L;
-}
-
-bool misaligned(const void* ptr) { return ((uintptr_t)ptr & 15) != 0; }
-
 struct StateLayout {
   size_t C, n, m, total;
 };
@@ -124,6 +104,30 @@ mlstm::InitState init_from(const void* state, const Problem& p) {
   }
   return in;
 }
+
+struct BwdLayout {
+  size_t inv_den, da, pq, pk, dC, dn, fstate, fdot, total;
+};
+
+BwdLayout bwd_layout(const Problem& p) {
+  BwdLayout L;
+  const size_t tok = (size_t)p.BH * p.T;
+  size_t off = 0;
+  L.inv_den = off; off = align256(off + tok * 4);
+  L.da = off;      off = align256(off + tok * 4);
+  L.pq = off;      off = align256(off + tok * 4);
+  L.pk = off;      off = align256(off + tok * 4);
+  L.dC = off;      off = align256(off + (size_t)p.BH * p.NC * p.dqk * p.dhv * 4);
+  L.dn = off;      off = align256(off + (p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0));
+  // the final state, rebuilt when the loss has a term on it, and its dot product with that term
+  L.fstate = off;  off = align256(off + state_layout(p.BH, p.dqk, p.dhv, p.exp_variant()).total);
+  L.fdot = off;    off = align256(off + (size_t)p.BH * 4);
+  L.total = off;
+  return L;
+}
+
+bool misaligned(const void* ptr) { return ((uintptr_t)ptr & 15) != 0; }
+
 
 int cuda_status(cudaError_t e, const char* where) {
   if (e == cudaSuccess) return MLSTM_OK;
@@ -354,17 +358,24 @@ namespace {
 
 int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
              const void* fgate_pre, const void* h, const void* dh, const void* saved,
-             const void* state_in, void* dstate_in, void* dq, void* dk, void* dv, void* digate_pre,
-             void* dfgate_pre, void* workspace, size_t workspace_bytes, int B, int NH, int T,
-             int d_qk, int d_hv, int chunk, int variant, int dtype, void* stream) {
+             const void* state_in, void* dstate_in, const void* dstate_out, void* dq, void* dk,
+             void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
+             size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
+             int variant, int dtype, void* stream) {
   int st = check_sizes(B, NH, T, d_qk, d_hv, chunk, variant, dtype);
   if (st != MLSTM_OK) return st;
-  if (misaligned(state_in) || misaligned(dstate_in)) return MLSTM_ERR_INVALID;
+  if (misaligned(state_in) || misaligned(dstate_in) || misaligned(dstate_out)) return MLSTM_ERR_INVALID;
   const StateLayout SL = state_layout(B * NH, d_qk, d_hv, variant == MLSTM_EXP);
-  if (dstate_in && state_in && overlaps(state_in, dstate_in, SL.total)) return MLSTM_ERR_INVALID;
+  if (dstate_in && ((state_in && overlaps(state_in, dstate_in, SL.total)) ||
+                    (dstate_out && overlaps(dstate_out, dstate_in, SL.total))))
+    return MLSTM_ERR_INVALID;
   if ((long long)B * NH == 0) return MLSTM_OK;
-  if (T == 0) {  // nothing reads the initial state: its gradient is zero
+  if (T == 0) {  // the final state is the initial one
     if (!dstate_in) return MLSTM_OK;
+    if (dstate_out)
+      return cuda_status(cudaMemcpyAsync(dstate_in, dstate_out, SL.total, cudaMemcpyDeviceToDevice,
+                                         (cudaStream_t)stream),
+                         "state copy");
     return cuda_status(cudaMemsetAsync(dstate_in, 0, SL.total, (cudaStream_t)stream), "memset");
   }
   if (!q || !k || !v || !igate_pre || !fgate_pre || !h || !dh || !saved || !dq || !dk || !dv ||
@@ -399,10 +410,27 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   a.init = init_from(state_in, p);
   a.dC0 = dstate_in ? (float*)((char*)dstate_in + SL.C) : nullptr;
   a.dn0 = (dstate_in && p.exp_variant()) ? (float*)((char*)dstate_in + SL.n) : nullptr;
+  a.dCT = dstate_out ? (const float*)((const char*)dstate_out + SL.C) : nullptr;
+  a.dnT = (dstate_out && p.exp_variant()) ? (const float*)((const char*)dstate_out + SL.n) : nullptr;
+  a.fdot = dstate_out ? (float*)(ws + W.fdot) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_bwd");
   if (st != MLSTM_OK) return st;
+  if (dstate_out) {
+    // the final state (from the saved buffer) and its dot product with its gradient
+    float* fs = (float*)(ws + W.fstate);
+    const float* fC = fs + SL.C / 4;
+    const float* fn = fs + SL.n / 4;
+    st = cuda_status(mlstm::launch_final_state(p, k, v, a.b, a.li, a.m, a.C, a.n, a.init,
+                                               fs + SL.C / 4, fs + SL.n / 4, fs + SL.m / 4, s),
+                     "final_state");
+    if (st != MLSTM_OK) return st;
+    st = cuda_status(mlstm::launch_state_dot(p.BH, p.dqk, p.dhv, p.exp_variant(), a.dCT, a.dnT, fC,
+                                             fn, a.fdot, s),
+                     "state_dot");
+    if (st != MLSTM_OK) return st;
+  }
   BwdStep steps[kMaxSteps];
   const int n = bwd_plan(p, steps);
   return run_plan(steps, n, p, a, s);
@@ -417,20 +445,20 @@ int mlstm_bwd(const void* q, const void* k, const void* v, const void* igate_pre
               void* dk, void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
               size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
               int variant, int dtype, void* stream) {
-  return bwd_impl(q, k, v, igate_pre, fgate_pre, h, dh, saved, nullptr, nullptr, dq, dk, dv,
-                  digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
-                  variant, dtype, stream);
+  return bwd_impl(q, k, v, igate_pre, fgate_pre, h, dh, saved, nullptr, nullptr, nullptr, dq, dk,
+                  dv, digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv,
+                  chunk, variant, dtype, stream);
 }
 
 int mlstm_bwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
                     const void* fgate_pre, const void* h, const void* dh, const void* saved,
-                    const void* state_in, void* dstate_in, void* dq, void* dk, void* dv,
-                    void* digate_pre, void* dfgate_pre, void* workspace, size_t workspace_bytes,
-                    int B, int NH, int T, int d_qk, int d_hv, int chunk, int variant, int dtype,
-                    void* stream) {
-  return bwd_impl(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in, dq, dk, dv,
-                  digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv, chunk,
-                  variant, dtype, stream);
+                    const void* state_in, void* dstate_in, const void* dstate_out, void* dq,
+                    void* dk, void* dv, void* digate_pre, void* dfgate_pre, void* workspace,
+                    size_t workspace_bytes, int B, int NH, int T, int d_qk, int d_hv, int chunk,
+                    int variant, int dtype, void* stream) {
+  return bwd_impl(q, k, v, igate_pre, fgate_pre, h, dh, saved, state_in, dstate_in, dstate_out, dq,
+                  dk, dv, digate_pre, dfgate_pre, workspace, workspace_bytes, B, NH, T, d_qk, d_hv,
+                  chunk, variant, dtype, stream);
 }
 
 }  // extern "C"

@@ -237,6 +237,36 @@ __global__ void __launch_bounds__(256) state_chain_kernel(
       no[(size_t)bh * dqk + i] = fmaf(fa, na[(size_t)bh * dqk + i], fb * nb[(size_t)bh * dqk + i]);
 }
 
+// out[bh] = <C_a, C_b> + <n_a, n_b> over one head's state (n for mLSTMexp only).
+template <bool EXPV>
+__global__ void __launch_bounds__(256) state_dot_kernel(const float* __restrict__ Ca,
+                                                        const float* __restrict__ na,
+                                                        const float* __restrict__ Cb,
+                                                        const float* __restrict__ nb,
+                                                        float* __restrict__ out, int dqk, int dhv) {
+  __shared__ float part[8];
+  const int bh = blockIdx.x;
+  const size_t n4 = (size_t)dqk * dhv / 4, off = (size_t)bh * dqk * dhv / 4;
+  const float4* a4 = reinterpret_cast<const float4*>(Ca) + off;
+  const float4* b4 = reinterpret_cast<const float4*>(Cb) + off;
+  float acc = 0.f;
+  for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 a = a4[i], b = b4[i];
+    acc = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+  }
+  if (EXPV)
+    for (int i = threadIdx.x; i < dqk; i += blockDim.x)
+      acc = fmaf(na[(size_t)bh * dqk + i], nb[(size_t)bh * dqk + i], acc);
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += part[w];
+    out[bh] = t;
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -313,6 +343,16 @@ cudaError_t launch_state_chain(int BH, int dqk, int dhv, bool exp_variant, const
     state_chain_kernel<true><<<BH, 256, 0, s>>>(Ca, na, ma, Cb, nb, mb, G, Co, no, mo, dqk, dhv);
   else
     state_chain_kernel<false><<<BH, 256, 0, s>>>(Ca, na, ma, Cb, nb, mb, G, Co, no, mo, dqk, dhv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_dot(int BH, int dqk, int dhv, bool exp_variant, const float* Ca,
+                             const float* na, const float* Cb, const float* nb, float* out,
+                             cudaStream_t s) {
+  if (exp_variant)
+    state_dot_kernel<true><<<BH, 256, 0, s>>>(Ca, na, Cb, nb, out, dqk, dhv);
+  else
+    state_dot_kernel<false><<<BH, 256, 0, s>>>(Ca, na, Cb, nb, out, dqk, dhv);
   return cudaGetLastError();
 }
 

@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
     TS* __restrict__ dC, float* __restrict__ dn, int T, int L, int NC, int dqk, int dhv,
     float scale, size_t plane, const float* __restrict__ m0, float* __restrict__ d0,
-    float* __restrict__ dn0) {
+    float* __restrict__ dn0, const float* __restrict__ dT, const float* __restrict__ dnT) {
   __shared__ float sQ[32][64];
   __shared__ float sD[32][64];
   __shared__ float fq[32], fn[32];
@@ -38,12 +38,14 @@ __global__ void __launch_bounds__(256) state_bwd_simt_kernel(
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const size_t tokh = (size_t)bh * T;
   const bool own_n = EXPV && blockIdx.z == 0 && tid < 64;
+  // the gradient of the state leaving the last chunk: the final state's, or zero
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  float nacc = 0.f;
+    for (int j = 0; j < 4; ++j)
+      acc[i][j] = dT ? dT[((size_t)bh * dqk + i0 + ty * 4 + i) * dhv + j0 + tx * 4 + j] : 0.f;
+  float nacc = (own_n && dT) ? dnT[(size_t)bh * dqk + i0 + tid] : 0.f;
 
   for (int c = NC - 1; c >= 0; --c) {
     const size_t gbase = ((size_t)bh * NC + c) * dqk * dhv;
@@ -120,7 +122,7 @@ cudaError_t launch_state_bwd_simt(const Problem& p, const BwdArgs& a, cudaStream
   state_bwd_simt_kernel<TIO, TS, E><<<grid, block, 0, s>>>(                                     \
       (const TIO*)a.q, (const TIO*)a.dh, a.b, a.m, a.inv_den, a.da, (TS*)a.dC, a.dn, p.T, p.L,  \
       p.NC, p.dqk, p.dhv, p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv,                     \
-      a.init.on() ? a.init.m : nullptr, a.dC0, a.dn0)
+      a.init.on() ? a.init.m : nullptr, a.dC0, a.dn0, a.dCT, a.dnT)
   if (p.bf16()) {
     if (p.exp_variant()) MLSTM_STATE_BWD(bf16, bf16, true);
     else MLSTM_STATE_BWD(bf16, bf16, false);
@@ -317,7 +319,8 @@ __global__ void __launch_bounds__(256) dk_simt_kernel(
     const TIO* __restrict__ dh, const float* __restrict__ b, const float* __restrict__ li,
     const float* __restrict__ m, const float* __restrict__ inv_den, const float* __restrict__ da,
     const TS* __restrict__ dC, const float* __restrict__ dn, TIO* __restrict__ dk,
-    float* __restrict__ pk, int T, int L, int NC, int dqk, int dhv, float scale, size_t plane) {
+    float* __restrict__ pk, int T, int L, int NC, int dqk, int dhv, float scale, size_t plane,
+    bool dfin) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -333,7 +336,7 @@ __global__ void __launch_bounds__(256) dk_simt_kernel(
   float acc[4][4];
   zero44(acc);
 
-  if (c < NC - 1) {  // w_s (dC_c v_s + dn_c)
+  if (c < NC - 1 || dfin) {  // w_s (dC_c v_s + dn_c)
     const size_t gbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dhv; x0 += 32) {
       __syncthreads();
@@ -414,7 +417,7 @@ __global__ void __launch_bounds__(256) dv_simt_kernel(
     const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ dh,
     const float* __restrict__ b, const float* __restrict__ li, const float* __restrict__ m,
     const float* __restrict__ inv_den, const TS* __restrict__ dC, TIO* __restrict__ dv, int T,
-    int L, int NC, int dqk, int dhv, float scale, size_t plane) {
+    int L, int NC, int dqk, int dhv, float scale, size_t plane, bool dfin) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& S = *reinterpret_cast<BwdSmem*>(smem_raw);
   const int bh = blockIdx.x / NC, c = blockIdx.x % NC;
@@ -430,7 +433,7 @@ __global__ void __launch_bounds__(256) dv_simt_kernel(
   float acc[4][4];
   zero44(acc);
 
-  if (c < NC - 1) {  // w_s dC_c^T k_s
+  if (c < NC - 1 || dfin) {  // w_s dC_c^T k_s
     const size_t gbase = ((size_t)bh * NC + c) * dqk * dhv;
     for (int x0 = 0; x0 < dqk; x0 += 32) {
       __syncthreads();
@@ -519,7 +522,7 @@ static cudaError_t dk_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dk_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.v, (const TIO*)a.dh, a.b, a.li, a.m,
       a.inv_den, a.da, (const TS*)a.dC, a.dn, (TIO*)a.dk, a.pk, p.T, p.L, p.NC, p.dqk, p.dhv,
-      p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv);
+      p.scale, (size_t)p.BH * p.NC * p.dqk * p.dhv, a.dCT != nullptr);
   return cudaGetLastError();
 }
 
@@ -533,7 +536,7 @@ static cudaError_t dv_launch(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dv_simt_kernel<TIO, TS, E><<<grid, 256, smem, s>>>(
       (const TIO*)a.q, (const TIO*)a.k, (const TIO*)a.dh, a.b, a.li, a.m, a.inv_den,
       (const TS*)a.dC, (TIO*)a.dv, p.T, p.L, p.NC, p.dqk, p.dhv, p.scale,
-      (size_t)p.BH * p.NC * p.dqk * p.dhv);
+      (size_t)p.BH * p.NC * p.dqk * p.dhv, a.dCT != nullptr);
   return cudaGetLastError();
 }
 

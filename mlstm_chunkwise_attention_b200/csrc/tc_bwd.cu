@@ -77,6 +77,7 @@ struct BwdTcParams {
   float* pdot;          // dq: pq; dk: pk (atomically accumulated)
   int T, L, NC, BH, ntq, nsl, d_out, dqk;  // nsl: output column slices of D2S
   bool m0set;                              // the forward started from an initial state
+  bool dfin;                               // the final state has a gradient (dk, dv)
   const float* m0;                         // its max state (mLSTMexp), else null
   float scale, log2_scale;
 };
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   const int pj0 = R_IS_QUERY ? 0 : it_tile;
   const int np = R_IS_QUERY ? it_tile + 1 : nt_len - it_tile;
   // a state enters the chunk (dq: c > 0 or an initial state), one leaves it (dk, dv)
-  const bool has_inter = R_IS_QUERY ? (c > 0 || P.m0set) : (c < P.NC - 1);
+  const bool has_inter = R_IS_QUERY ? (c > 0 || P.m0set) : (c < P.NC - 1 || P.dfin);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -630,6 +631,7 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   P.rowvec = (KIND == KDQ) ? a.n : a.dn;
   P.dot_src = (const bf16*)((KIND == KDQ) ? a.q : a.k);
   P.m0set = a.init.on();
+  P.dfin = a.dCT != nullptr;
   P.m0 = (a.init.on() && p.exp_variant()) ? a.init.m : nullptr;
   P.out = (bf16*)((KIND == KDQ) ? a.dq : (KIND == KDK) ? a.dk : a.dv);
   P.pdot = (KIND == KDQ) ? a.pq : a.pk;

@@ -71,6 +71,7 @@ struct StateTcParams {
   float scale;
   InitState init;   // forward: the state entering chunk 0; both: its max state m0
   float *d0, *dn0;  // backward: gradient of the initial state (C, n), fp32, or null
+  const float *dT, *dnT;  // backward: gradient of the final state (C, n), fp32, or null
 };
 
 template <bool BWD, bool EXPV, int NV>
@@ -275,12 +276,15 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const bool valid = dk0 + i < P.dqk;
     // the running state: the forward starts from the initial state (zero without one)
+    // (the backward from the final state's gradient, if one is given)
     float S[NV];
-    const bool from_init = !BWD && P.init.on() && valid;
+    const float* S0 = BWD ? P.dT : P.init.C;
+    const float* n0 = BWD ? P.dnT : P.init.n;
+    const bool from_init = S0 != nullptr && valid;
 #pragma unroll
     for (int j = 0; j < NV; ++j)
-      S[j] = from_init ? P.init.C[((size_t)bh * P.dqk + dk0 + i) * P.dhv + dv0 + j] : 0.f;
-    float sn = (from_init && with_n) ? P.init.n[(size_t)bh * P.dqk + dk0 + i] : 0.f;
+      S[j] = from_init ? S0[((size_t)bh * P.dqk + dk0 + i) * P.dhv + dv0 + j] : 0.f;
+    float sn = (from_init && with_n) ? n0[(size_t)bh * P.dqk + dk0 + i] : 0.f;
     for (int u = 0; u < NC; ++u) {
       const int c = chunk_of(u);
       // store the state at this chunk boundary: rows into the swizzled staging
@@ -391,7 +395,8 @@ template <bool BWD, bool EXPV, int NV>
 static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* B, bf16* out,
                                    float* nout, const float* b, const float* li, const float* m,
                                    const float* inv_den, const float* da, const InitState& init,
-                                   float* d0, float* dn0, cudaStream_t s) {
+                                   float* d0, float* dn0, const float* dT, const float* dnT,
+                                   cudaStream_t s) {
   using Cfg = StateTcCfg<NV>;
   CUtensorMap tA, tB, tOh, tOl;
   const uint64_t plane = (uint64_t)p.BH * p.NC * p.dqk * p.dhv;
@@ -410,6 +415,8 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
   P.init = init;
   P.d0 = d0;
   P.dn0 = dn0;
+  P.dT = dT;
+  P.dnT = dnT;
   auto kern = state_tc_kernel<BWD, EXPV, NV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
@@ -424,24 +431,26 @@ template <bool BWD, bool EXPV>
 static cudaError_t launch_state_tc_nv(const Problem& p, const void* A, const void* B, bf16* out,
                                       float* nout, const float* b, const float* li, const float* m,
                                       const float* inv_den, const float* da, const InitState& init,
-                                      float* d0, float* dn0, cudaStream_t s) {
-  return launch_state_tc<BWD, EXPV, 64>(p, A, B, out, nout, b, li, m, inv_den, da, init, d0, dn0, s);
+                                      float* d0, float* dn0, const float* dT, const float* dnT,
+                                      cudaStream_t s) {
+  return launch_state_tc<BWD, EXPV, 64>(p, A, B, out, nout, b, li, m, inv_den, da, init, d0, dn0,
+                                        dT, dnT, s);
 }
 
 cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   if (p.exp_variant())
     return launch_state_tc_nv<false, true>(p, a.k, a.v, (bf16*)a.C, a.n, a.b, a.li, a.m, nullptr,
-                                           nullptr, a.init, nullptr, nullptr, s);
+                                           nullptr, a.init, nullptr, nullptr, nullptr, nullptr, s);
   return launch_state_tc_nv<false, false>(p, a.k, a.v, (bf16*)a.C, a.n, a.b, a.li, a.m, nullptr,
-                                          nullptr, a.init, nullptr, nullptr, s);
+                                          nullptr, a.init, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
   if (p.exp_variant())
     return launch_state_tc_nv<true, true>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
-                                          a.inv_den, a.da, a.init, a.dC0, a.dn0, s);
+                                          a.inv_den, a.da, a.init, a.dC0, a.dn0, a.dCT, a.dnT, s);
   return launch_state_tc_nv<true, false>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
-                                         a.inv_den, a.da, a.init, a.dC0, a.dn0, s);
+                                         a.inv_den, a.da, a.init, a.dC0, a.dn0, a.dCT, a.dnT, s);
 }
 
 cudaError_t fetch_tc_state_error(unsigned int* flag) {

@@ -84,3 +84,24 @@ def random_state(rng, d_qk, d_hv, variant, scale=0.3):
     n = rng.uniform(0.5, 2.0, d_qk)
     m = float(rng.standard_normal())
     return C, n, m
+
+
+def final_state_term_grads(q, k, v, log_i, log_f, W, w):
+    """Gradients of <W, C_T> + <w, n_T> (unstabilised final state after the last token)
+    with respect to k, v, log i and log f, in closed form (fp64); q does not enter.
+
+    With D_s = exp(sum_{r > s} log f_r + log i_s) the decay from token s to the end,
+    C_T = sum_s D_s k_s v_s^T and n_T = sum_s D_s k_s, so with l_s = D_s (k_s^T W v_s + k_s.w):
+    dk_s = D_s (W v_s + w), dv_s = D_s W^T k_s, d log i_s = l_s, d log f_r = sum_{s < r} l_s.
+    """
+    k, v, log_i, log_f = (np.asarray(a, dtype=np.float64) for a in (k, v, log_i, log_f))
+    T = k.shape[0]
+    after = np.concatenate([np.cumsum(log_f[::-1])[::-1][1:], [0.0]])  # sum_{r > s} log f_r
+    D = np.exp(after + log_i)
+    Wv = v @ W.T                                   # row s: W v_s
+    lam = D * (np.sum(k * Wv, axis=1) + (k @ w if w is not None else 0.0))
+    dk = D[:, None] * (Wv + (w[None, :] if w is not None else 0.0))
+    dv = D[:, None] * (k @ W)
+    dlog_f = np.concatenate([[0.0], np.cumsum(lam)[:-1]])
+    return {"dq": np.zeros_like(np.asarray(q, dtype=np.float64)), "dk": dk, "dv": dv,
+            "dlog_i": lam, "dlog_f": dlog_f}

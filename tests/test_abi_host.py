@@ -174,12 +174,13 @@ def test_chunkwise_state_entry_points_argument_errors(lib):
                                None) == B.STATUS_UNSUPPORTED
     bwd_in = (fake,) * 8  # q k v ig fg h dh saved
     outs = (fake,) * 5 + (fake, 1 << 30)  # dq dk dv dig dfg, workspace, bytes
-    assert lib.mlstm_bwd_state(*bwd_in, fake, fake + 512, *outs, *sizes, None) == B.STATUS_INVALID
-    assert lib.mlstm_bwd_state(*bwd_in, fake, other + 4, *outs, *sizes, None) == B.STATUS_INVALID
+    assert lib.mlstm_bwd_state(*bwd_in, fake, fake + 512, None, *outs, *sizes, None) == B.STATUS_INVALID
+    assert lib.mlstm_bwd_state(*bwd_in, fake, other + 4, None, *outs, *sizes, None) == B.STATUS_INVALID
+    assert lib.mlstm_bwd_state(*bwd_in, fake, other, other + 256, *outs, *sizes, None) == B.STATUS_INVALID
     # empty problems are no-ops
     assert lib.mlstm_fwd_state(*[None] * 8, 0, None, None, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16,
                                None) == 0
-    assert lib.mlstm_bwd_state(*[None] * 16, 0, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16, None) == 0
+    assert lib.mlstm_bwd_state(*[None] * 17, 0, 0, 2, 256, 64, 64, 64, B.SIG, B.BF16, None) == 0
 
 
 def test_segment_entry_points_argument_errors(lib):

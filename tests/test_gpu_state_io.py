@@ -132,3 +132,39 @@ def test_chained_calls_equal_one_call(variant, case):
         assert relerr(got_C, ref_C) <= tol, f"final C head {hh}"
         if variant == EXP:
             assert relerr(got_n, ref_n) <= tol, f"final n head {hh}"
+
+
+@pytest.mark.parametrize("variant", [SIG, EXP], ids=["sig", "exp"])
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_gradient_through_the_final_state(variant, case):
+    """Backward of a loss on the final state alone (dh = 0): the gradients of
+    <dC~_T, C~_T> + <dn~_T, n~_T> with m_T held constant, i.e. of <W, C_T> + <w, n_T> for
+    the unstabilised state with W = exp(-m_T) dC~_T, against their closed form
+    (tests/_state_prefix.py, pinned by finite differences in test_state_prefix.py)."""
+    from _state_prefix import final_state_term_grads
+    name, dt, d, L, T = case
+    B, NH = 1, 2
+    cpu = inputs(B, NH, T, d, d, seed=74, dtype=dt, ig_mean=-2.0)
+    dev = {k: v.cuda() for k, v in cpu.items()}
+    rng = np.random.default_rng(75)
+    douts = [random_state(rng, d, d, variant, scale=1.0) for _ in range(B * NH)]
+    d_out = _device_state(douts, B, NH, d, d, variant)
+    h, saved, _ = binding.forward_state(dev["q"], dev["k"], dev["v"], dev["igate"], dev["fgate"],
+                                        L, variant)
+    zero_dh = torch.zeros_like(dev["dh"])
+    g = binding.backward_state(dev["q"], dev["k"], dev["v"], dev["igate"], dev["fgate"], h, zero_dh,
+                               saved, L, variant, dstate_out=d_out)
+    binding.check_device()
+    tol = TOL[dt]
+    assert float(g["dq"].abs().max()) == 0.0
+    for hh in range(NH):
+        q, k, v, li, lf, ig, fg, _ = _head(cpu, hh, variant)
+        m_T = oracle.chunkwise_forward(q, k, v, li, lf, variant, L)["m_final"]
+        dC, dn, _ = douts[hh]
+        s = float(np.exp(-m_T)) if variant == EXP else 1.0
+        ref = final_state_term_grads(q, k, v, li, lf, s * dC, s * dn if variant == EXP else None)
+        di, df = oracle.preact_grads(ref["dlog_i"], ref["dlog_f"], ig, fg, variant)
+        want = {"dk": ref["dk"], "dv": ref["dv"], "digate_pre": di, "dfgate_pre": df}
+        for key, r in want.items():
+            err = relerr(np64(g[key][0, hh]), r)
+            assert err <= tol, f"{key} head {hh}: {err:.3e}"

@@ -94,3 +94,42 @@ def test_prefix_state_gradient_matches_finite_differences(variant):
             nmi[j] -= eps
             fd = (loss(C, npl) - loss(C, nmi)) / (2 * eps)
             assert abs(fd - dn[j]) <= 1e-6 * max(1.0, abs(fd)), (j, fd, dn[j])
+
+
+@pytest.mark.parametrize("variant", [SIG, EXP], ids=["sig", "exp"])
+def test_final_state_term_gradients_match_finite_differences(variant):
+    """The closed form in _state_prefix.final_state_term_grads against central finite
+    differences of <W, C_T> + <w, n_T> over the oracle's unstabilised recurrence."""
+    from _state_prefix import final_state_term_grads
+    rng = np.random.default_rng(13)
+    d_qk, d_hv, T = 5, 4, 11
+    q, k, v, ig, fg = _tokens(rng, T, d_qk, d_hv, variant)
+    W = rng.standard_normal((d_qk, d_hv))
+    w = rng.standard_normal(d_qk) if variant == EXP else None
+
+    def loss(k_, v_, ig_, fg_):
+        li, lf = oracle.gate_logs(ig_, fg_, variant)
+        C, n = oracle.recurrent_forward(q, k_, v_, li, lf, variant, state_steps=(T,))["states"][T]
+        return float(np.sum(W * C) + (w @ n if w is not None else 0.0))
+
+    li, lf = oracle.gate_logs(ig, fg, variant)
+    g = final_state_term_grads(q, k, v, li, lf, W, w)
+    di, df = oracle.preact_grads(g["dlog_i"], g["dlog_f"], ig, fg, variant)
+    eps = 1e-6
+
+    def fd(arr, idx, which):
+        a, b = arr.copy(), arr.copy()
+        a[idx] += eps
+        b[idx] -= eps
+        args_a = {"k": k, "v": v, "ig": ig, "fg": fg, which: a}
+        args_b = {"k": k, "v": v, "ig": ig, "fg": fg, which: b}
+        return (loss(args_a["k"], args_a["v"], args_a["ig"], args_a["fg"])
+                - loss(args_b["k"], args_b["v"], args_b["ig"], args_b["fg"])) / (2 * eps)
+
+    for idx in [(0, 1), (6, 3), (10, 0)]:
+        assert abs(fd(k, idx, "k") - g["dk"][idx]) <= 1e-6 * max(1.0, abs(g["dk"][idx]))
+    for idx in [(2, 2), (9, 1)]:
+        assert abs(fd(v, idx, "v") - g["dv"][idx]) <= 1e-6 * max(1.0, abs(g["dv"][idx]))
+    for t in (0, 5, 10):
+        assert abs(fd(ig, t, "ig") - di[t]) <= 1e-6 * max(1.0, abs(di[t]))
+        assert abs(fd(fg, t, "fg") - df[t]) <= 1e-6 * max(1.0, abs(df[t]))
