@@ -245,7 +245,10 @@ int mlstm_fwd_state(const void* q, const void* k, const void* v, const void* iga
  *              final state reads every key before it); the final state is
  *              rebuilt from `saved` in the workspace.
  * dstate_in must not overlap state_in or dstate_out (MLSTM_ERR_INVALID).
- * With T = 0 the gradient with respect to the initial state is dstate_out. */
+ * With T = 0 the gradient with respect to the initial state is dstate_out.
+ * dq, dk, dv, digate_pre and dfgate_pre may all be NULL when dstate_in is not:
+ * the state-gradient-only pass (per-token normaliser terms and the state
+ * recurrence, no intra-chunk or gate kernels). */
 int mlstm_bwd_state(const void* q, const void* k, const void* v, const void* igate_pre,
                     const void* fgate_pre, const void* h, const void* dh, const void* saved,
                     const void* state_in, void* dstate_in, const void* dstate_out, void* dq,
@@ -280,6 +283,22 @@ int mlstm_log_decay(const void* fgate_pre, float* log_decay, int B, int NH, int 
 int mlstm_state_chain(const void* state_a, const void* state_b, const float* log_decay_b,
                       void* state_out, int B, int NH, int d_qk, int d_hv, int variant,
                       void* stream);
+
+/* The backward of chained segments.  For segment b, given
+ *   dstate_local  the gradient with respect to b's initial state from b's own
+ *                 outputs (mlstm_bwd_state with dstate_in and the five
+ *                 gradient outputs NULL: the state-gradient-only pass),
+ *   dstate_out    the gradient with respect to b's final state,
+ *   state_in, state_out  the states entering and leaving b (their m), and b's
+ *                 log_decay,
+ * dstate_in = dstate_local + f dstate_out with f = exp(G_b + m_in - m_out)
+ * (exp(G_b) for mLSTMsig): the state map through b is S_out = f S_in + (b's
+ * own state) in the stabilised form, the max states held constant.  C and
+ * (EXP) n regions of state-layout buffers; dstate_in must not overlap
+ * dstate_local or dstate_out (MLSTM_ERR_INVALID). */
+int mlstm_dstate_chain(const void* dstate_local, const void* dstate_out, const void* state_in,
+                       const void* state_out, const float* log_decay, void* dstate_in, int B,
+                       int NH, int d_qk, int d_hv, int variant, void* stream);
 
 
 /* Synchronise `stream` and report what the kernels enqueued so far found:

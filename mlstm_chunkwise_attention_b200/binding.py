@@ -67,6 +67,7 @@ EXPORTS = {
     "mlstm_bwd_state": (ctypes.c_int, [_P] * 16 + [_P, ctypes.c_size_t] + _SIZES + [_P]),
     "mlstm_log_decay": (ctypes.c_int, [_P, _P] + [ctypes.c_int] * 4 + [_P]),
     "mlstm_state_chain": (ctypes.c_int, [_P] * 4 + [ctypes.c_int] * 5 + [_P]),
+    "mlstm_dstate_chain": (ctypes.c_int, [_P] * 6 + [ctypes.c_int] * 5 + [_P]),
 }
 
 
@@ -374,6 +375,40 @@ def state_chain(state_a, state_b, log_decay_b, B, NH, d_qk, d_hv, variant, *, ou
     if st != STATUS_OK:
         raise MLSTMError(st, "mlstm_state_chain")
     return out
+
+
+def dstate_chain(dstate_local, dstate_out, state_in, state_out, log_decay_b, B, NH, d_qk, d_hv,
+                 variant, *, out=None, stream=None):
+    """Gradient with respect to segment b's initial state (see include/mlstm.h)."""
+    import torch
+    if out is None:
+        out = torch.zeros_like(dstate_local)
+    st = load().mlstm_dstate_chain(dstate_local.data_ptr(), dstate_out.data_ptr(),
+                                   state_in.data_ptr(), state_out.data_ptr(), log_decay_b.data_ptr(),
+                                   out.data_ptr(), B, NH, d_qk, d_hv, variant,
+                                   _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_dstate_chain")
+    return out
+
+
+def state_gradient(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, state_in=None, *,
+                   stream=None):
+    """The state-gradient-only pass: gradient of sum(dh * h) with respect to state_in."""
+    import torch
+    sizes = problem_sizes(q, v, chunk, variant)
+    B, NH, T, d_qk, d_hv = sizes[:5]
+    dstate = torch.zeros(load().mlstm_state_size(B, NH, d_qk, d_hv, variant), dtype=torch.uint8,
+                         device=q.device)
+    ws = torch.empty(max(mlstm_bwd_workspace_size(*sizes), 1), dtype=torch.uint8, device=q.device)
+    st = mlstm_bwd_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), igate_pre.data_ptr(),
+                         fgate_pre.data_ptr(), h.data_ptr(), dh.data_ptr(), saved.data_ptr(),
+                         state_in.data_ptr() if state_in is not None else None, dstate.data_ptr(),
+                         None, None, None, None, None, None, ws.data_ptr(), ws.numel(), *sizes,
+                         _stream_handle(stream))
+    if st != STATUS_OK:
+        raise MLSTMError(st, "mlstm_bwd_state")
+    return dstate
 
 
 def backward_state(q, k, v, igate_pre, fgate_pre, h, dh, saved, chunk, variant, state_in=None, *,

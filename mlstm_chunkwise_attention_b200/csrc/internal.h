@@ -120,6 +120,10 @@ cudaError_t launch_step(const Problem& p, const void* q, const void* k, const vo
 cudaError_t launch_state_zero(int BH, int dqk, int dhv, bool exp_variant, float* C, float* n, float* m,
                               cudaStream_t s);
 cudaError_t launch_log_decay(const Problem& p, const void* fg, float* G, cudaStream_t s);
+cudaError_t launch_dstate_chain(int BH, int dqk, int dhv, bool exp_variant, const float* Cl,
+                                const float* nl, const float* Cd, const float* nd,
+                                const float* m_in, const float* m_out, const float* G, float* Co,
+                                float* no, cudaStream_t s);
 cudaError_t launch_state_dot(int BH, int dqk, int dhv, bool exp_variant, const float* Ca,
                              const float* na, const float* Cb, const float* nb, float* out,
                              cudaStream_t s);

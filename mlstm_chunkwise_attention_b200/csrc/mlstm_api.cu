@@ -378,8 +378,10 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
                          "state copy");
     return cuda_status(cudaMemsetAsync(dstate_in, 0, SL.total, (cudaStream_t)stream), "memset");
   }
-  if (!q || !k || !v || !igate_pre || !fgate_pre || !h || !dh || !saved || !dq || !dk || !dv ||
-      !digate_pre || !dfgate_pre)
+  // all five outputs NULL with a dstate_in: the state-gradient-only pass
+  const bool grads = dq || dk || dv || digate_pre || dfgate_pre;
+  if (!q || !k || !v || !igate_pre || !fgate_pre || !h || !dh || !saved ||
+      (grads && (!dq || !dk || !dv || !digate_pre || !dfgate_pre)) || (!grads && !dstate_in))
     return MLSTM_ERR_INVALID;
   const void* ptrs[] = {q, k, v, igate_pre, fgate_pre, h, dh, saved, dq, dk, dv,
                         digate_pre, dfgate_pre, workspace};
@@ -433,7 +435,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   }
   BwdStep steps[kMaxSteps];
   const int n = bwd_plan(p, steps);
-  return run_plan(steps, n, p, a, s);
+  // the state-gradient-only pass: bwd_token_prep and the state recurrence (the plan's first
+  // two steps) give dstate_in
+  return run_plan(steps, grads ? n : 2, p, a, s);
 }
 
 }  // namespace
@@ -580,6 +584,37 @@ int mlstm_state_chain(const void* state_a, const void* state_b, const float* log
                                 (const float*)(pb + S.m), log_decay_b, (float*)(po + S.C),
                                 (float*)(po + S.n), (float*)(po + S.m), (cudaStream_t)stream),
       "state_chain");
+}
+
+int mlstm_dstate_chain(const void* dstate_local, const void* dstate_out, const void* state_in,
+                       const void* state_out, const float* log_decay, void* dstate_in, int B,
+                       int NH, int d_qk, int d_hv, int variant, void* stream) {
+  int st = check_sizes(B, NH, 1, d_qk, d_hv, 64, variant, MLSTM_FP32);
+  if (st != MLSTM_OK) return st;
+  if ((long long)B * NH == 0) return MLSTM_OK;
+  if (!dstate_local || !dstate_out || !state_in || !state_out || !log_decay || !dstate_in)
+    return MLSTM_ERR_INVALID;
+  const void* ptrs[] = {dstate_local, dstate_out, state_in, state_out, log_decay, dstate_in};
+  for (const void* ptr : ptrs)
+    if (misaligned(ptr)) return MLSTM_ERR_INVALID;
+  const bool e = variant == MLSTM_EXP;
+  const StateLayout S = state_layout(B * NH, d_qk, d_hv, e);
+  if (overlaps(dstate_in, dstate_local, S.total) || overlaps(dstate_in, dstate_out, S.total))
+    return MLSTM_ERR_INVALID;
+  const char* pl = (const char*)dstate_local;
+  const char* pd = (const char*)dstate_out;
+  const char* pi = (const char*)state_in;
+  const char* po = (const char*)state_out;
+  char* pr = (char*)dstate_in;
+  st = cuda_status(cudaPeekAtLastError(), "before mlstm_dstate_chain");
+  if (st != MLSTM_OK) return st;
+  return cuda_status(
+      mlstm::launch_dstate_chain(B * NH, d_qk, d_hv, e, (const float*)(pl + S.C),
+                                 (const float*)(pl + S.n), (const float*)(pd + S.C),
+                                 (const float*)(pd + S.n), (const float*)(pi + S.m),
+                                 (const float*)(po + S.m), log_decay, (float*)(pr + S.C),
+                                 (float*)(pr + S.n), (cudaStream_t)stream),
+      "dstate_chain");
 }
 
 const char* mlstm_status_string(int status) {

@@ -237,6 +237,38 @@ __global__ void __launch_bounds__(256) state_chain_kernel(
       no[(size_t)bh * dqk + i] = fmaf(fa, na[(size_t)bh * dqk + i], fb * nb[(size_t)bh * dqk + i]);
 }
 
+// Gradient with respect to the state entering segment b: its own share (g_local, from the
+// segment's outputs) plus the gradient with respect to the state leaving b carried back
+// through the segment.  The state map through b is S_out = exp(G_b + m_in - m_out) S_in +
+// (b's own state) in the stabilised form, so the carried share is that factor times the
+// leaving state's gradient (C and n; the max states are held constant).
+template <bool EXPV>
+__global__ void __launch_bounds__(256) dstate_chain_kernel(
+    const float* __restrict__ Cl, const float* __restrict__ nl, const float* __restrict__ Cd,
+    const float* __restrict__ nd, const float* __restrict__ m_in, const float* __restrict__ m_out,
+    const float* __restrict__ G, float* __restrict__ Co, float* __restrict__ no, int dqk,
+    int dhv) {
+  const int bh = blockIdx.x;
+  float f;
+  if (EXPV) {
+    const float x = G[bh] + m_in[bh], y = m_out[bh];
+    f = x == kNegInf ? 0.f : expf(x - y);
+  } else {
+    f = expf(G[bh]);
+  }
+  const size_t n4 = (size_t)dqk * dhv / 4, off = (size_t)bh * dqk * dhv / 4;
+  const float4* l4 = reinterpret_cast<const float4*>(Cl) + off;
+  const float4* d4 = reinterpret_cast<const float4*>(Cd) + off;
+  float4* o4 = reinterpret_cast<float4*>(Co) + off;
+  for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 a = l4[i], b = d4[i];
+    o4[i] = make_float4(fmaf(f, b.x, a.x), fmaf(f, b.y, a.y), fmaf(f, b.z, a.z), fmaf(f, b.w, a.w));
+  }
+  if (EXPV)
+    for (int i = threadIdx.x; i < dqk; i += blockDim.x)
+      no[(size_t)bh * dqk + i] = fmaf(f, nd[(size_t)bh * dqk + i], nl[(size_t)bh * dqk + i]);
+}
+
 // out[bh] = <C_a, C_b> + <n_a, n_b> over one head's state (n for mLSTMexp only).
 template <bool EXPV>
 __global__ void __launch_bounds__(256) state_dot_kernel(const float* __restrict__ Ca,
@@ -353,6 +385,17 @@ cudaError_t launch_state_dot(int BH, int dqk, int dhv, bool exp_variant, const f
     state_dot_kernel<true><<<BH, 256, 0, s>>>(Ca, na, Cb, nb, out, dqk, dhv);
   else
     state_dot_kernel<false><<<BH, 256, 0, s>>>(Ca, na, Cb, nb, out, dqk, dhv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dstate_chain(int BH, int dqk, int dhv, bool exp_variant, const float* Cl,
+                                const float* nl, const float* Cd, const float* nd,
+                                const float* m_in, const float* m_out, const float* G, float* Co,
+                                float* no, cudaStream_t s) {
+  if (exp_variant)
+    dstate_chain_kernel<true><<<BH, 256, 0, s>>>(Cl, nl, Cd, nd, m_in, m_out, G, Co, no, dqk, dhv);
+  else
+    dstate_chain_kernel<false><<<BH, 256, 0, s>>>(Cl, nl, Cd, nd, m_in, m_out, G, Co, no, dqk, dhv);
   return cudaGetLastError();
 }
 

@@ -3,12 +3,12 @@
 Starting the mLSTM recurrence from a state (C, n, m) is the same as running it
 from the zero state over d_qk extra tokens placed first, whose only effect on
 every later token is to leave exactly that state behind:
-  token j = 0 .. d_qk - 1:  k_j = e_j (unit vector), q_j = 0, log f_j = 0,
-  so after them the unstabilised state is C = sum_j i_j e_j v_j^T (row j is
-  i_j v_j) and n = sum_j i_j e_j (entry j is i_j).
-  SIG (no normaliser): i_j = 1/2, v_j = 2 C[j].
+  token j = 0 .. d_qk - 1:  k_j = s_j e_j (s_j = +-1, e_j a unit vector), q_j = 0,
+  log f_j = 0, so after them the unstabilised state is C = sum_j i_j k_j v_j^T
+  (row j is s_j i_j v_j) and n = sum_j i_j k_j (entry j is s_j i_j).
+  SIG (no normaliser): s_j = 1, i_j = 1/2, v_j = 2 C[j].
   EXP: the stabilised state (C~, n~, m) stands for exp(m) (C~, n~); with
-  i_j = exp(m) n~_j (so n~ > 0 is needed) and v_j = C~[j] / n~_j.
+  s_j = sign(n~_j), i_j = exp(m) |n~_j| (n~_j != 0 is needed) and v_j = C~[j] / n~_j.
 Their own outputs are zero (q = 0) and dropped.  Later tokens then see the
 state decayed by their own forget gates, as in the recurrence started from it,
 so the oracle's forward and backward over the longer sequence give the
@@ -34,8 +34,9 @@ def prefix(C, n, m, variant):
         v = 2.0 * C
     else:
         n = np.asarray(n, dtype=np.float64)
-        assert np.all(n > 0), "the construction needs a positive normaliser state"
-        log_i = float(m) + np.log(n)
+        assert np.all(n != 0), "the construction needs a normaliser state without zeros"
+        k = np.diag(np.sign(n))
+        log_i = float(m) + np.log(np.abs(n))
         v = C / n[:, None]
     return q, k, v, log_i, log_f
 
@@ -50,14 +51,15 @@ def state_grads(pre, dk_pre, dv_pre, m, variant):
     """Gradient of the loss with respect to the stabilised state (C~, n~), from the
     prefix tokens' dk, dv (m held constant).
 
-    Row j of the true C is i_j v_j, so dL/dC_true[j] = dv_j / i_j; entry j of the
-    true n is i_j (k_j = e_j enters C and n), so dk_j[j] = i_j (dC_true[j] . v_j +
-    dn_true[j]).  The stabilised state is exp(-m) times the true one, so its
+    Row j of the true C is s_j i_j v_j, so dL/dC_true[j] = dv_j / (s_j i_j); entry j of
+    the true n is s_j i_j (k_j = s_j e_j enters C and n through its entry j), so
+    dk_j[j] = i_j (dC_true[j] . v_j + dn_true[j]).  The stabilised state is exp(-m) times the true one, so its
     gradient is exp(m) times the true gradient (exp(m) = 1 for SIG).
     """
-    _, _, v, log_i, _ = pre
+    _, k, v, log_i, _ = pre
     i = np.exp(log_i)
-    dC_true = dv_pre / i[:, None]
+    sgn = np.diagonal(k)
+    dC_true = dv_pre / (sgn * i)[:, None]
     scale = 1.0 if variant == oracle.SIG else float(np.exp(m))
     dC = scale * dC_true
     dn = None

@@ -196,3 +196,22 @@ def test_segment_entry_points_argument_errors(lib):
     assert lib.mlstm_state_chain(fake, other, None, third, 1, 2, 64, 64, B.SIG, None) == B.STATUS_INVALID
     assert lib.mlstm_state_chain(fake, other, third, third + 4, 1, 2, 64, 64, B.SIG, None) == B.STATUS_INVALID
     assert lib.mlstm_state_chain(fake, other, third, 0x100000, 1, 2, 100, 64, B.SIG, None) == B.STATUS_UNSUPPORTED
+
+
+def test_backward_chain_argument_errors(lib):
+    """mlstm_dstate_chain and the state-gradient-only pass: argument errors before any launch."""
+    a, b, c, d, g, o = (0x10000 * (i + 1) for i in range(6))  # aligned, never dereferenced
+    sz = (1, 2, 64, 64, B.EXP, None)
+    assert lib.mlstm_dstate_chain(a, b, c, d, None, o, *sz) == B.STATUS_INVALID
+    assert lib.mlstm_dstate_chain(a, b, c, d, g, a + 256, *sz) == B.STATUS_INVALID  # overlaps dstate_local
+    assert lib.mlstm_dstate_chain(a, b, c, d, g, b, *sz) == B.STATUS_INVALID        # overlaps dstate_out
+    assert lib.mlstm_dstate_chain(a, b, c, d, g, o + 8, *sz) == B.STATUS_INVALID
+    assert lib.mlstm_dstate_chain(None, None, None, None, None, None, 0, 2, 64, 64, B.EXP, None) == 0
+    # state-gradient-only pass: all five gradient outputs NULL needs a dstate_in
+    sizes = (1, 2, 256, 64, 64, 64, B.SIG, B.BF16)
+    ins = (a,) * 8
+    assert lib.mlstm_bwd_state(*ins, None, None, None, None, None, None, None, None, b, 1 << 30,
+                               *sizes, None) == B.STATUS_INVALID
+    # some but not all of the five outputs
+    assert lib.mlstm_bwd_state(*ins, None, c, None, d, None, None, None, None, b, 1 << 30,
+                               *sizes, None) == B.STATUS_INVALID

@@ -6,8 +6,8 @@
   (compared as unstabilised states);
 * the sequence-parallel protocol of seqpar.py with its segments run one after
   the other in this process (no cross-process exchange: the gathered lists are
-  the local ones): the outputs of every segment against the oracle over the
-  whole sequence.
+  the local ones): the outputs of every segment, and the gradients of every
+  segment's tokens, against the oracle over the whole sequence.
 """
 
 import numpy as np
@@ -72,27 +72,43 @@ def test_state_chain(variant):
             assert relerr(got_n, ref_n) <= TOL[F32], f"n head {hh}"
 
 
+def _run_segments(cpu, L, variant, P, with_backward):
+    """The protocol of seqpar.py with its P segments run one after the other here."""
+    dev = {k: v.cuda() for k, v in cpu.items()}
+    T = dev["q"].shape[2]
+    bounds = [round(T * r / P) for r in range(P + 1)]
+    segs = [{k: x[:, :, bounds[r]:bounds[r + 1]].contiguous() for k, x in dev.items()}
+            for r in range(P)]
+    ops = seqpar.DeviceOps()
+    B, NH, _, d = dev["q"].shape
+    sizes = (B, NH, d, dev["v"].shape[-1])
+    local = [ops.local_state(s, L, variant) for s in segs]
+    decays = [g for _, g in local]
+    chained = seqpar.chain_states([s for s, _ in local], decays, sizes, variant, ops)
+    parts = []
+    for r in range(P):
+        h, saved = ops.forward_from(segs[r], L, variant, chained[r], keep_saved=with_backward)
+        parts.append(seqpar.Segment(h=h, state_in=chained[r], states=chained, decays=decays,
+                                    saved=saved, index=r))
+    grads = None
+    if with_backward:
+        dls = [ops.local_dstate(segs[r], segs[r]["dh"], parts[r], L, variant) for r in range(P)]
+        grads = []
+        for r in range(P):
+            dout = seqpar.final_state_gradient(r, dls, chained, decays, sizes, variant, ops)
+            grads.append(ops.backward_from(segs[r], segs[r]["dh"], parts[r], L, variant, dout))
+    binding.check_device()
+    return bounds, parts, grads
+
+
 @pytest.mark.parametrize("variant", [SIG, EXP], ids=["sig", "exp"])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_segments_in_sequence_equal_one_call(variant, case):
     name, dt, d, L, T, P = case
     B, NH = 1, 2
     cpu = inputs(B, NH, T, d, d, seed=83, dtype=dt, ig_mean=-2.0, with_dh=False)
-    dev = {k: v.cuda() for k, v in cpu.items()}
-    bounds = [round(T * r / P) for r in range(P + 1)]
-    segs = [{k: x[:, :, bounds[r]:bounds[r + 1]].contiguous() for k, x in dev.items()}
-            for r in range(P)]
-    ops = seqpar.DeviceOps()
-    local = [ops.local_state(s, L, variant) for s in segs]
-    states, decays = [s for s, _ in local], [g for _, g in local]
-    sizes = (B, NH, d, d)
-    hs = []
-    for r in range(P):
-        state_in = seqpar.incoming_state(r, states, decays, sizes, variant, ops)
-        h, _ = ops.forward_from(segs[r], L, variant, state_in, keep_saved=False)
-        hs.append(h)
-    binding.check_device()
-    h_all = torch.cat(hs, dim=2)
+    bounds, parts, _ = _run_segments(cpu, L, variant, P, with_backward=False)
+    h_all = torch.cat([p.h for p in parts], dim=2)
     for hh in range(NH):
         x = {k: np64(v[0, hh]) for k, v in cpu.items()}
         li, lf = oracle.gate_logs(x["igate"], x["fgate"], variant)
@@ -100,3 +116,23 @@ def test_segments_in_sequence_equal_one_call(variant, case):
         for r in range(P):
             sl = slice(bounds[r], bounds[r + 1])
             assert relerr(np64(h_all[0, hh, sl]), ref[sl]) <= TOL[dt], f"segment {r} head {hh}"
+
+
+@pytest.mark.parametrize("variant", [SIG, EXP], ids=["sig", "exp"])
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_segment_backward_equals_one_call(variant, case):
+    """The sequence-parallel backward (each segment's own initial-state share, carried
+    back to the earlier segments as their final-state gradients) against the oracle's
+    backward over the whole sequence."""
+    name, dt, d, L, T, P = case
+    B, NH = 1, 2
+    cpu = inputs(B, NH, T, d, d, seed=84, dtype=dt, ig_mean=-2.0)
+    bounds, _, grads = _run_segments(cpu, L, variant, P, with_backward=True)
+    got = {k: torch.cat([g[k] for g in grads], dim=2) for k in grads[0]}
+    ref = oracle.backward_heads(np64(cpu["q"]), np64(cpu["k"]), np64(cpu["v"]), np64(cpu["igate"]),
+                                np64(cpu["fgate"]), variant, np64(cpu["dh"]))
+    names = {"dq": "dq", "dk": "dk", "dv": "dv", "digate_pre": "digate", "dfgate_pre": "dfgate"}
+    for key, rk in names.items():
+        for hh in range(NH):
+            err = relerr(np64(got[key][0, hh]), ref[rk][0, hh])
+            assert err <= TOL[dt], f"{key} head {hh}: {err:.3e}"

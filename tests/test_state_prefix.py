@@ -46,6 +46,8 @@ def test_prefix_reproduces_steps_from_state(variant):
     rng = np.random.default_rng(11)
     d_qk, d_hv, T = 8, 6, 13
     C, n, m = random_state(rng, d_qk, d_hv, variant)
+    if variant == EXP:
+        n = n * np.array([1, -1, -1, 1, 1, -1, 1, -1])
     q, k, v, ig, fg = _tokens(rng, T, d_qk, d_hv, variant)
     h_ref, C_T, n_T, m_T = _steps(C.copy(), None if n is None else n.copy(), m, q, k, v, ig, fg,
                                   variant)
@@ -67,6 +69,8 @@ def test_prefix_state_gradient_matches_finite_differences(variant):
     rng = np.random.default_rng(12)
     d_qk, d_hv, T = 6, 5, 9
     C, n, m = random_state(rng, d_qk, d_hv, variant)
+    if variant == EXP:
+        n = n * np.array([1, -1, 1, -1, -1, 1])  # the construction takes either sign
     q, k, v, ig, fg = _tokens(rng, T, d_qk, d_hv, variant)
     dh = rng.standard_normal((T, d_hv))
     li, lf = oracle.gate_logs(ig, fg, variant)
