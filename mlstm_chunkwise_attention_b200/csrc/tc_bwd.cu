@@ -64,7 +64,7 @@ struct BwdTcCfg {
 };
 
 enum {
-  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_YE, BB_INTER, BB_ACC, BB_DONE, BB_STG, BB_COUNT
+  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_INTER, BB_ACC, BB_DONE, BB_STG, BB_COUNT
 };
 
 }  // namespace
