@@ -38,7 +38,7 @@ KERNEL_SOURCES = {
     "dv_simt": "simt_bwd.cu", "output_fwd_tc": "tc_fwd.cu", "dq_tc": "tc_bwd.cu",
     "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
     "output_fwd_xl": "tc_fwd_xl.cu",
-    "state_bwd_tc": "tc_state.cu",
+    "state_bwd_tc": "tc_state.cu", "dkv_walk_tc": "tc_bwd_walk.cu",
 }
 
 
@@ -84,6 +84,12 @@ def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
         "dk": (tdd + T * L * dqk, T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st_full + stn),
         "dv": (tdd + T * L * (dqk + dhv), T * (2 * dqk + 2 * dhv) * io_bytes + 4 * tok_f + st_full),
         "gate_grad": (0, T * 4 * io_bytes + 2 * tok_f),
+        # state gradients, dk and dv in one pass: the state-gradient recurrence and the
+        # dk, dv contractions; q, k, v, dh read once, dk, dv and k.dk written, the state
+        # gradients never leave the chip
+        "dkv_walk": (3 * tdd + T * L * (2 * dqk + dhv),
+                     T * (3 * dqk + 3 * dhv) * io_bytes
+                     + (g + (2 if exp_variant else 0) + 1) * tok_f),
     }
     out = {}
     for role, v in c.items():

@@ -162,14 +162,22 @@ int fwd_plan(const Problem& p, FwdStep* st) {
   return n;
 }
 
-int bwd_plan(const Problem& p, BwdStep* st) {
-  (void)p;
+// grads false: the state-gradient-only pass (token prep and the state recurrence).
+int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
   int n = 0;
   st[n++] = {"bwd_token_prep", mlstm::launch_bwd_token_prep};
+  if (grads && mlstm::bwd_walk_supported(p)) {
+    // one pass per head over its chunks in reverse gives the state gradients, dk and dv
+    st[n++] = {"dkv_walk_tc", mlstm::launch_bwd_walk};
+    st[n++] = {"dq_tc", mlstm::launch_dq_tc};
+    st[n++] = {"gate_grad", mlstm::launch_gate_grad};
+    return n;
+  }
   if (mlstm::state_tc_supported(p))
     st[n++] = {"state_bwd_tc", mlstm::launch_state_bwd_tc};
   else
     st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
+  if (!grads) return n;
   if (mlstm::intra_bwd_tc_supported(p)) {
     st[n++] = {"dq_tc", mlstm::launch_dq_tc};
     st[n++] = {"dk_tc", mlstm::launch_dk_tc};
@@ -434,10 +442,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
     if (st != MLSTM_OK) return st;
   }
   BwdStep steps[kMaxSteps];
-  const int n = bwd_plan(p, steps);
-  // the state-gradient-only pass: bwd_token_prep and the state recurrence (the plan's first
-  // two steps) give dstate_in
-  return run_plan(steps, grads ? n : 2, p, a, s);
+  const int n = bwd_plan(p, steps, grads);
+  return run_plan(steps, n, p, a, s);
 }
 
 }  // namespace
@@ -634,7 +640,7 @@ const char* mlstm_last_error(void) { return g_last_error; }
 int mlstm_device_status(void* stream) {
   int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
   if (st != MLSTM_OK) return st;
-  unsigned int flag = 0, flag_bwd = 0, flag_state = 0, flag_xl = 0;
+  unsigned int flag = 0, flag_bwd = 0, flag_state = 0, flag_xl = 0, flag_walk = 0;
   st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_bwd_error(&flag_bwd), "device error flag");
@@ -643,7 +649,9 @@ int mlstm_device_status(void* stream) {
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_fwd_xl_error(&flag_xl), "device error flag");
   if (st != MLSTM_OK) return st;
-  flag |= flag_bwd | flag_state | flag_xl;
+  st = cuda_status(mlstm::fetch_tc_walk_error(&flag_walk), "device error flag");
+  if (st != MLSTM_OK) return st;
+  flag |= flag_bwd | flag_state | flag_xl | flag_walk;
   if (flag) {
     snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
     return MLSTM_ERR_TIMEOUT;

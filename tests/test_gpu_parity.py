@@ -48,6 +48,9 @@ SMALL = [
     ("exp_bf16_dqk256_dhv64_chunk512_ragged", 1, 2, 1000, 256, 64, 512, EXP, BF, 0.0, 3.0),
     ("sig_bf16_dqk64_dhv128_chunk256_ragged", 1, 2, 600, 64, 128, 256, SIG, BF, -2.0, 3.0),
     ("exp_fp32_dqk256", 1, 1, 384, 256, 64, 128, EXP, F32, 1.0, 2.0),
+    ("exp_bf16_chunk128_d128_ragged", 2, 2, 700, 128, 128, 128, EXP, BF, -2.0, 3.0),
+    ("sig_bf16_chunk128_d128_ragged", 1, 3, 1000, 128, 128, 128, SIG, BF, 0.0, 3.0),
+    ("exp_bf16_chunk128_d128_one_partial", 1, 2, 77, 128, 128, 128, EXP, BF, 0.0, 3.0),
 ]
 
 
