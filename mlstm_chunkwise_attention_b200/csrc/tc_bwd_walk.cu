@@ -17,9 +17,9 @@
 // through two mbarriers, so work that does not feed the next product (the dv and
 // dk epilogues, the next chunk's gate factors) runs while the tensor core works:
 //   rows: stage dC -> A | rescale dv inter, dv transform -> B | rescale dk inter,
-//         dk transform -> C | dv out | u dH, dn -> D | dk out, next gate factors
+//         dk transform -> C | u dH -> D | dv out | dk out | next gate factors
 //   MMA:  A: K dC (dv inter), K Q^T | B: Y dH (dv), V dH^T, V dC^T (dk inter) |
-//         C: Y Q (dk) | D: dC += Q^T (u dH)
+//         C: Y Q (dk) | D: dC += Q^T (u dH), Q^T wn (the normaliser's update)
 // The next chunk's K and V tiles load as soon as their buffers are free, Q and
 // dH once the state update has read them.  Every wait is bounded; on a timeout
 // the kernel raises its error flag and winds down.
@@ -47,16 +47,24 @@ struct WalkCfg {
   static constexpr int OFF_F = 6 * TILE;              // per-token factors, NF arrays of 128 floats
   static constexpr int NF = 8;
   static constexpr int OFF_W = OFF_F + NF * 128 * 4;  // per-warp partner factors, 4 x 128
-  static constexpr int OFF_BAR = OFF_W + 4 * 128 * 4;
+  // the normaliser weights as the B operand of the dn product: 16 x 128 K-major bf16 (row 0
+  // the hi, row 1 the lo plane, rows 2..15 zero), two buffers (chunk parity)
+  static constexpr int OFF_WN = OFF_W + 4 * 128 * 4;
+  static constexpr int WN_BYTES = 4096;
+  static constexpr int OFF_BAR = OFF_WN + 2 * WN_BYTES;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * 8;
   static constexpr size_t SMEM = 1024 + OFF_TMEM + 16;
   static constexpr uint32_t TMEM_COLS = 512;  // dC, score / transformed tile, dv, dk
 };
 
 // per-token factor arrays in the OFF_F region (token t of the chunk, or state row j)
-enum { F_PC = 0, F_PE, F_WV, F_WN, F_DN };
-// mbarriers: tile loads (one per tile), rows -> MMA thread, MMA thread -> rows
-enum { BW_Q = 0, BW_K, BW_V, BW_H, BW_R, BW_M, BW_COUNT };
+enum { F_PC = 0, F_PE, F_WV, F_DN };
+// mbarriers: tile loads (one per tile); rows -> MMA thread (hand-overs A, B, C; and D on
+// its own barrier, since the rows signal C and D back to back); MMA thread -> rows (the
+// products after A, B, C; and the state update on its own barrier, which can complete
+// before the rows wait for C's products).  Each barrier's phases strictly alternate
+// with its waiter, so parity waits cannot alias.
+enum { BW_Q = 0, BW_K, BW_V, BW_H, BW_R, BW_D, BW_M, BW_S, BW_COUNT };
 
 __device__ __forceinline__ uint32_t sw_off(int row, int col) {
   // byte offset of (row, col) in a [128 rows x 128 cols] bf16 tile of two swizzled blocks
@@ -118,7 +126,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < BW_COUNT; ++i) tc::mbar_init(&bar[i], i == BW_R ? 128u : 1u);
+    for (int i = 0; i < BW_COUNT; ++i) tc::mbar_init(&bar[i], (i == BW_R || i == BW_D) ? 128u : 1u);
     tc::fence_mbar_init();
   }
   if (warp == 1) {
@@ -138,14 +146,16 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       constexpr uint32_t idKK = tc::idesc_bf16(128, 128, false, false);  // A, B K-major
       constexpr uint32_t idKM = tc::idesc_bf16(128, 128, false, true);   // B MN-major
       constexpr uint32_t idMM = tc::idesc_bf16(128, 128, true, true);    // A, B MN-major
+      constexpr uint32_t idN = tc::idesc_bf16(128, 16, true, false);     // A MN-major, N = 16
       const uint32_t aQ = tc::smem_u32(sQ), aK = tc::smem_u32(sK), aV = tc::smem_u32(sV),
-                     aH = tc::smem_u32(sH), aG = tc::smem_u32(sG), aGl = aG + Cfg::TILE;
+                     aH = tc::smem_u32(sH), aG = tc::smem_u32(sG), aGl = aG + Cfg::TILE,
+                     aWN = tc::smem_u32(smem + Cfg::OFF_WN);
       // K-step k (16 elements) of a K-major tile, or of an MN-major tile (rows = K)
       auto kmaj = [](uint32_t base, int k) {
         return tc::sdesc_sw128(base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
       };
       auto mnmaj = [](uint32_t base, int k) { return tc::sdesc_sw128(base + k * 2048, 16384, 1024); };
-      uint32_t nr = 0;  // row hand-overs consumed
+      uint32_t nr = 0;  // row hand-overs A, B, C consumed
       auto wait_rows = [&]() -> bool {
         const bool w = tc::mbar_wait(&bar[BW_R], nr & 1, abort_flag);
         ++nr;
@@ -195,7 +205,8 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         tc::tc_commit(&bar[BW_M]);
         // D (u dH staged, hi plane over dH, lo plane over dC's): dC_{c-1} = beta_c dC_c (the
         // rows scaled it) + Q^T (u dH)
-        ok = wait_rows();
+        ok = tc::mbar_wait(&bar[BW_D], it & 1, abort_flag);
+        tc::tc_fence_after();
         if (!ok) break;
         if (c > 0 || P.d0 != nullptr) {
 #pragma unroll
@@ -203,8 +214,16 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
             tc::mma_bf16_ss(tDC, mnmaj(aQ, k), mnmaj(aH, k), idMM, 1);
             tc::mma_bf16_ss(tDC, mnmaj(aQ, k), mnmaj(aGl, k), idMM, 1);
           }
+          if (EXPV) {  // columns 0 and 1 of the score buffer: Q^T wn (hi, lo)
+            const uint32_t wn = aWN + (it & 1) * Cfg::WN_BYTES;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              tc::mma_bf16_ss(tX, mnmaj(aQ, k),
+                              tc::sdesc_sw128(wn + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), idN,
+                              k > 0);
+          }
         }
-        tc::tc_commit(&bar[BW_M]);
+        tc::tc_commit(&bar[BW_S]);
       }
       if (!ok) atomicOr(&g_tc_walk_error, 1u);
     }
@@ -214,7 +233,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const unsigned full = 0xffffffffu;
     const bool issuer = row == 0;  // issues the TMA loads and stores
-    uint32_t nm = 0;               // MMA hand-overs consumed
+    uint32_t nm = 0, ns = 0;       // product hand-overs (A, B, C) and state updates consumed
     auto wait_mma = [&]() -> bool {
       const bool w = __all_sync(full, tc::mbar_wait(&bar[BW_M], nm & 1, abort_flag));
       ++nm;
@@ -222,12 +241,19 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       tc::tc_fence_after();
       return w;
     };
-    // this thread's TMEM stores and shared-memory writes, then the hand-over to the MMA thread
-    auto signal = [&]() {
+    auto wait_state = [&]() -> bool {
+      const bool w = __all_sync(full, tc::mbar_wait(&bar[BW_S], ns & 1, abort_flag));
+      ++ns;
+      if (!w && lane == 0) atomicOr(&g_tc_walk_error, 1u);
+      tc::tc_fence_after();
+      return w;
+    };
+    // this thread's TMEM stores and shared-memory writes, then a hand-over to the MMA thread
+    auto signal = [&](int b) {
       tc::tmem_wait_st();
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
-      tc::mbar_arrive(&bar[BW_R]);
+      tc::mbar_arrive(&bar[b]);
     };
     auto load_tile = [&](int b, uint8_t* dst, const CUtensorMap* tm, int c) {
       tc::mbar_arrive_expect_tx(&bar[b], Cfg::TILE);
@@ -240,33 +266,66 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       tc::bulk_commit_group();
     };
 
-    // Gate factors of chunk c: partner factors of this row as a query (the dk and dv
-    // transforms), its state-update weights, and the chunk's scalars.
-    struct Gates { float g, mc, beta, bt, lis; int len; };
-    auto gate_factors = [&](int c) -> Gates {
-      Gates G;
-      const int c0 = c * 128;
-      G.len = min(128, P.T - c0);
+    // Gate values of chunk c (this row's token, the chunk's last token, the previous
+    // chunk's max state), loaded a chunk ahead of their use.
+    struct GateIn { float g, mc, mprev, bt, lis, mt, invd, dat; };
+    auto gate_load = [&](int c) -> GateIn {
+      GateIn I;
+      const int c0 = c * 128, len = min(128, P.T - c0);
       const size_t tok0 = (size_t)bh * P.T + c0;
-      const bool in = row < G.len;
+      const bool in = row < len;
       const size_t t = tok0 + (in ? row : 0);
-      G.g = P.b[tok0 + G.len - 1];
-      G.mc = EXPV ? P.m[tok0 + G.len - 1] : 0.f;
-      const float mprev = EXPV ? chunk_mprev(P.m, tok0, c, P.m0, bh) : 0.f;
-      G.bt = in ? P.b[t] : 0.f;
-      G.lis = in ? P.li[t] : 0.f;
-      const float mt = (in && EXPV) ? P.m[t] : 0.f;
-      const float invd = (in && EXPV) ? P.inv_den[t] : 1.f;
-      const float dat = (in && EXPV) ? P.da[t] : 0.f;
-      if (EXPV) G.beta = (c > 0 || P.m0 != nullptr) ? expf(G.g + mprev - G.mc) : 0.f;
-      else G.beta = expf(G.g);
-      F[F_PC * 128 + row] = in ? (G.bt - mt) * kLog2e + log2f(invd) : -INFINITY;
-      F[F_PE * 128 + row] = (EXPV && in) ? dat / invd : 0.f;
+      I.g = P.b[tok0 + len - 1];
+      I.mc = EXPV ? P.m[tok0 + len - 1] : 0.f;
+      I.mprev = EXPV ? chunk_mprev(P.m, tok0, c, P.m0, bh) : 0.f;
+      I.bt = in ? P.b[t] : 0.f;
+      I.lis = in ? P.li[t] : 0.f;
+      I.mt = (in && EXPV) ? P.m[t] : 0.f;
+      I.invd = (in && EXPV) ? P.inv_den[t] : 1.f;
+      I.dat = (in && EXPV) ? P.da[t] : 0.f;
+      return I;
+    };
+    // Gate factors of chunk c: partner factors of this row as a query (the dk and dv
+    // transforms), its state-update weights (u in shared memory, wn as the hi and lo rows of
+    // the dn product's operand), and the chunk's scalars.
+    struct Gates { float g, mc, beta, bt, lis; int len; };
+    auto gate_factors = [&](int c, const GateIn& I) -> Gates {
+      Gates G;
+      G.len = min(128, P.T - c * 128);
+      const bool in = row < G.len;
+      G.g = I.g;
+      G.mc = I.mc;
+      G.bt = I.bt;
+      G.lis = I.lis;
+      if (EXPV) G.beta = (c > 0 || P.m0 != nullptr) ? expf(I.g + I.mprev - I.mc) : 0.f;
+      else G.beta = expf(I.g);
+      F[F_PC * 128 + row] = in ? (I.bt - I.mt) * kLog2e + log2f(I.invd) : -INFINITY;
+      F[F_PE * 128 + row] = (EXPV && in) ? I.dat / I.invd : 0.f;
       // exp(-inf) = 0 in the first chunk of an mLSTMexp sequence without an initial state
-      const float alpha = in ? expf(G.bt + mprev - mt) * P.scale : 0.f;
-      F[F_WV * 128 + row] = alpha * invd;
-      F[F_WN * 128 + row] = EXPV ? alpha * dat : 0.f;
+      const float alpha = in ? expf(I.bt + I.mprev - I.mt) * P.scale : 0.f;
+      F[F_WV * 128 + row] = alpha * I.invd;
+      if (EXPV) {
+        const float wn = alpha * I.dat;
+        const bf16 hi = __float2bfloat16_rn(wn);
+        const bf16 lo = __float2bfloat16_rn(wn - __bfloat162float(hi));
+        // K-major 128-byte swizzle: token t of row r at block t / 64, chunk (t % 64) / 8 ^ r
+        uint8_t* wt = smem + Cfg::OFF_WN + ((NC - 1 - c) & 1) * Cfg::WN_BYTES + (row >> 6) * 2048 +
+                      (row & 7) * 2;
+        *reinterpret_cast<bf16*>(wt + (((row & 63) >> 3) << 4)) = hi;
+        *reinterpret_cast<bf16*>(wt + 128 + ((((row & 63) >> 3) ^ 1) << 4)) = lo;
+      }
       return G;
+    };
+    // columns 0 and 1 of the score buffer after a state update: the normaliser's increment
+    auto dn_increment = [&]() -> float {
+      uint32_t r0, r1;
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
+          "tcgen05.wait::ld.sync.aligned;"
+          : "=r"(r0), "=r"(r1)
+          : "r"(tX + lane_base)
+          : "memory");
+      return __uint_as_float(r0) + __uint_as_float(r1);
     };
     // Rescale an inter-term accumulator row in TMEM: x = rs x (+ rs dn[col] for dk, mLSTMexp).
     auto rescale = [&](uint32_t tA, float rs, bool with_dn) {
@@ -473,7 +532,11 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       if (EXPV && P.dnT) dn = P.dnT[(size_t)bh * 128 + row];
       if (EXPV) F[F_DN * 128 + row] = dn;
     }
-    Gates cur = gate_factors(NC - 1);
+    if (EXPV)
+      for (int i = row; i < 2 * Cfg::WN_BYTES / 16; i += 128)
+        reinterpret_cast<uint4*>(smem + Cfg::OFF_WN)[i] = make_uint4(0u, 0u, 0u, 0u);
+    ok = rows_and(ok);  // the zeroing is done before any row writes its weights
+    Gates cur = gate_factors(NC - 1, gate_load(NC - 1));
     ok = rows_and(ok);
 
     for (int it = 0; it < NC && ok; ++it) {
@@ -481,7 +544,11 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       if (it > 0) {
         // the previous chunk's state update is done: Q and dH are free for this chunk's
         // tiles, and the staging planes once the dk store has read its tile
-        ok = wait_mma();
+        ok = wait_state();
+        if (EXPV) {
+          dn += dn_increment();       // dn_c
+          F[F_DN * 128 + row] = dn;   // read by this chunk's dk rescale
+        }
         if (issuer && ok) {
           load_tile(BW_Q, sQ, &tmQ, c);
           load_tile(BW_H, sH, &tmH, c);
@@ -490,11 +557,14 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         ok = rows_and(ok);
         if (!ok) break;
       }
+      // the next chunk's gate values, in flight while this chunk runs
+      GateIn nxt;
+      if (c > 0) nxt = gate_load(c - 1);
       const bool valid = row < cur.len;
       // ---- A: stage dC_c (hi, lo), scale it by beta_c in TMEM
       stage_dc(cur.beta);
       if (EXPV) dn *= cur.beta;
-      signal();
+      signal(BW_R);
       // row-side factors of this key row (the dk and dv kernels' conventions)
       float rs_v = 0.f, rs_k = 0.f, Rk = -INFINITY, Rv = -INFINITY;
       if (valid) {
@@ -507,20 +577,14 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       ok = wait_mma();
       rescale(tAV, rs_v, false);
       transform(false, Rv);
-      signal();
+      signal(BW_R);
       // ---- C: dk inter rescaled (+ dn_c), dk transform
       ok = wait_mma() && ok;
       rescale(tAK, rs_k, true);
       transform(true, Rk);
-      signal();
-      // ---- dv out, staged over V (its products are done), while dk accumulates
-      epilogue(tAV, 1.f, sV, false);
-      tc::fence_proxy_async_smem();
-      ok = rows_and(ok);
-      if (!ok) break;
-      if (issuer) store_tile(&tmDV, sV, c);
-      // ---- D: u dH (hi over dH, lo over dC's lo plane) and the normaliser's update
-      ok = wait_mma();
+      signal(BW_R);
+      // ---- D: u dH, hi plane over dH and lo plane over dC's lo plane (their products are
+      // done), so the state update runs while the outputs are written
       const bool update = c > 0 || P.d0 != nullptr;
       if (update) {
         const float wv = F[F_WV * 128 + row];
@@ -541,23 +605,16 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
           *reinterpret_cast<uint4*>(sH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sG + Cfg::TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        if (EXPV) {
-          // dn_{c-1} = beta_c dn_c (scaled above) + sum_t q_t[j] wn_t
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-          const float* wn = F + F_WN * 128;
-#pragma unroll 8
-          for (int t = 0; t < 128; t += 4) {
-            a0 = fmaf(__bfloat162float(*reinterpret_cast<const bf16*>(sQ + sw_off(t, row))), wn[t], a0);
-            a1 = fmaf(__bfloat162float(*reinterpret_cast<const bf16*>(sQ + sw_off(t + 1, row))), wn[t + 1], a1);
-            a2 = fmaf(__bfloat162float(*reinterpret_cast<const bf16*>(sQ + sw_off(t + 2, row))), wn[t + 2], a2);
-            a3 = fmaf(__bfloat162float(*reinterpret_cast<const bf16*>(sQ + sw_off(t + 3, row))), wn[t + 3], a3);
-          }
-          dn += (a0 + a1) + (a2 + a3);
-          F[F_DN * 128 + row] = dn;  // read by the next chunk's dk rescale
-        }
       }
-      signal();
-      // ---- dk out, staged over dC's hi plane, with k . dk from the K tile
+      signal(BW_D);
+      // ---- dv out, staged over V (its products are done)
+      epilogue(tAV, 1.f, sV, false);
+      tc::fence_proxy_async_smem();
+      ok = rows_and(ok);
+      if (!ok) break;
+      if (issuer) store_tile(&tmDV, sV, c);
+      // ---- dk out once dk is accumulated, staged over dC's hi plane, with k . dk from K
+      ok = wait_mma();
       const float dot = epilogue(tAK, P.scale, sG, true);
       if (valid) P.pk[(size_t)bh * P.T + (size_t)c * 128 + row] = dot;
       tc::fence_proxy_async_smem();
@@ -573,13 +630,14 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       }
       // ---- the next chunk's gate factors, while the state update runs
       if (c > 0) {
-        cur = gate_factors(c - 1);
+        cur = gate_factors(c - 1, nxt);
         ok = rows_and(ok);
       }
     }
     // the last state update
-    if (ok) ok = wait_mma();
+    if (ok) ok = wait_state();
     if (ok && P.d0 != nullptr) {
+      if (EXPV) dn += dn_increment();
       for (int cb = 0; cb < 4; ++cb) {
         float x[32];
         tc::tmem_ld32(tDC + lane_base + 32 * cb, x);
