@@ -17,9 +17,9 @@
 // through two mbarriers, so work that does not feed the next product (the dv and
 // dk epilogues, the next chunk's gate factors) runs while the tensor core works:
 //   rows: stage dC -> A | rescale dv inter, dv transform -> B | rescale dk inter,
-//         dk transform -> C | u dH -> D | dv out | dk out | next gate factors
-//   MMA:  A: K dC (dv inter), K Q^T | B: Y dH (dv), V dH^T, V dC^T (dk inter) |
-//         C: Y Q (dk) | D: dC += Q^T (u dH), Q^T wn (the normaliser's update)
+//         dk transform -> C | u dH, dn increment -> D | dv out | dk out | next gates
+//   MMA:  K Q^T (dv score) | A: K dC (dv inter) | V dC^T (dk inter) | B: Y dH (dv),
+//         V dH^T (dk score) | C: Y Q (dk), Q^T wn (dn increment) | D: dC += Q^T (u dH)
 // The next chunk's K and V tiles load as soon as their buffers are free, Q and
 // dH once the state update has read them.  Every wait is bounded; on a timeout
 // the kernel raises its error flag and winds down.
@@ -169,58 +169,63 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       };
       for (int it = 0; it < NC && ok; ++it) {
         const int c = NC - 1 - it;
-        // A (dC staged): dv inter K dC (hi + lo planes), then the dv score K Q^T
-        ok = wait_tile(BW_K, it) && wait_rows();
+        // the dv score K Q^T (the score buffer is free: the rows read the previous chunk's
+        // dn increment before they handed over its state update)
+        ok = wait_tile(BW_K, it) && wait_tile(BW_Q, it);
+        if (!ok) break;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tX, kmaj(aK, k), kmaj(aQ, k), idKK, k > 0);
+        // A (dC staged): dv inter K dC (hi + lo planes)
+        ok = wait_rows();
         if (!ok) break;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           tc::mma_bf16_ss(tAV, kmaj(aK, k), mnmaj(aG, k), idKM, k > 0);
           tc::mma_bf16_ss(tAV, kmaj(aK, k), mnmaj(aGl, k), idKM, 1);
         }
-        ok = wait_tile(BW_Q, it);
-        if (!ok) break;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tX, kmaj(aK, k), kmaj(aQ, k), idKK, k > 0);
         tc::tc_commit(&bar[BW_M]);
-        // B (dv transform in TMEM): dv += Y dH; dk score V dH^T; dk inter V dC^T (hi + lo)
-        ok = wait_rows() && wait_tile(BW_H, it);
-        if (!ok) break;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tAV, tX + 8 * k, mnmaj(aH, k), idKM, 1);
+        // the dk inter V dC^T (hi + lo) while the rows transform the dv score
         ok = wait_tile(BW_V, it);
         if (!ok) break;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tX, kmaj(aV, k), kmaj(aH, k), idKK, k > 0);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           tc::mma_bf16_ss(tAK, kmaj(aV, k), kmaj(aG, k), idKK, k > 0);
           tc::mma_bf16_ss(tAK, kmaj(aV, k), kmaj(aGl, k), idKK, 1);
         }
-        tc::tc_commit(&bar[BW_M]);
-        // C (dk transform in TMEM): dk += Y Q
-        ok = wait_rows();
+        // B (dv transform in TMEM): dv += Y dH, then the dk score V dH^T over Y
+        ok = wait_rows() && wait_tile(BW_H, it);
         if (!ok) break;
 #pragma unroll
+        for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tAV, tX + 8 * k, mnmaj(aH, k), idKM, 1);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tX, kmaj(aV, k), kmaj(aH, k), idKK, k > 0);
+        tc::tc_commit(&bar[BW_M]);
+        // C (dk transform in TMEM): dk += Y Q; then the normaliser's increment Q^T wn (hi, lo)
+        // into columns 0 and 1 of the score buffer
+        ok = wait_rows();
+        if (!ok) break;
+        const bool update = c > 0 || P.d0 != nullptr;
+#pragma unroll
         for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tAK, tX + 8 * k, mnmaj(aQ, k), idKM, 1);
+        if (EXPV && update) {
+          const uint32_t wn = aWN + (it & 1) * Cfg::WN_BYTES;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc::mma_bf16_ss(tX, mnmaj(aQ, k),
+                            tc::sdesc_sw128(wn + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), idN,
+                            k > 0);
+        }
         tc::tc_commit(&bar[BW_M]);
         // D (u dH staged, hi plane over dH, lo plane over dC's): dC_{c-1} = beta_c dC_c (the
         // rows scaled it) + Q^T (u dH)
         ok = tc::mbar_wait(&bar[BW_D], it & 1, abort_flag);
         tc::tc_fence_after();
         if (!ok) break;
-        if (c > 0 || P.d0 != nullptr) {
+        if (update) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             tc::mma_bf16_ss(tDC, mnmaj(aQ, k), mnmaj(aH, k), idMM, 1);
             tc::mma_bf16_ss(tDC, mnmaj(aQ, k), mnmaj(aGl, k), idMM, 1);
-          }
-          if (EXPV) {  // columns 0 and 1 of the score buffer: Q^T wn (hi, lo)
-            const uint32_t wn = aWN + (it & 1) * Cfg::WN_BYTES;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              tc::mma_bf16_ss(tX, mnmaj(aQ, k),
-                              tc::sdesc_sw128(wn + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), idN,
-                              k > 0);
           }
         }
         tc::tc_commit(&bar[BW_S]);
@@ -545,10 +550,6 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         // the previous chunk's state update is done: Q and dH are free for this chunk's
         // tiles, and the staging planes once the dk store has read its tile
         ok = wait_state();
-        if (EXPV) {
-          dn += dn_increment();       // dn_c
-          F[F_DN * 128 + row] = dn;   // read by this chunk's dk rescale
-        }
         if (issuer && ok) {
           load_tile(BW_Q, sQ, &tmQ, c);
           load_tile(BW_H, sH, &tmH, c);
@@ -606,6 +607,14 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
           *reinterpret_cast<uint4*>(sG + Cfg::TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
+      // dk accumulated and the normaliser's increment in the score buffer, which the next
+      // chunk's dv score overwrites once the state update has been handed over
+      ok = wait_mma() && ok;
+      if (EXPV && update) {
+        dn += dn_increment();       // dn_{c-1}
+        F[F_DN * 128 + row] = dn;   // read by the next chunk's dk rescale (every row's dk
+                                    // rescale of this chunk is done: the products waited for it)
+      }
       signal(BW_D);
       // ---- dv out, staged over V (its products are done)
       epilogue(tAV, 1.f, sV, false);
@@ -613,8 +622,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       ok = rows_and(ok);
       if (!ok) break;
       if (issuer) store_tile(&tmDV, sV, c);
-      // ---- dk out once dk is accumulated, staged over dC's hi plane, with k . dk from K
-      ok = wait_mma();
+      // ---- dk out, staged over dC's hi plane, with k . dk from the K tile
       const float dot = epilogue(tAK, P.scale, sG, true);
       if (valid) P.pk[(size_t)bh * P.T + (size_t)c * 128 + row] = dot;
       tc::fence_proxy_async_smem();
@@ -637,7 +645,6 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
     // the last state update
     if (ok) ok = wait_state();
     if (ok && P.d0 != nullptr) {
-      if (EXPV) dn += dn_increment();
       for (int cb = 0; cb < 4; ++cb) {
         float x[32];
         tc::tmem_ld32(tDC + lane_base + 32 * cb, x);
