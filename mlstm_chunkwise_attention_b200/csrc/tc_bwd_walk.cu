@@ -11,9 +11,10 @@
 // are read once for all three products.  "Tiled Flash Linear Attention" (TFLA
 // summary page, Problem: materialised chunk states cost IO; Approach).
 //
-// Roles: one thread (warp 1) issues the MMAs; four row warps (one key row or one
-// state row per thread, the TMEM lane) transform, rescale and store, and one of
-// their threads issues the TMA loads and stores.  Rows and MMA thread hand over
+// Roles: one thread (warp 0) issues the MMAs; eight row warps transform, rescale
+// and store, two per TMEM lane quarter: a thread owns one key row, token row or
+// state row (its TMEM lane) and one half of the columns.  One row thread issues
+// the TMA loads and stores.  Rows and MMA thread hand over
 // through two mbarriers, so work that does not feed the next product (the dv and
 // dk epilogues, the next chunk's gate factors) runs while the tensor core works:
 //   rows: stage dC -> A | rescale dv inter, dv transform -> B | rescale dk inter,
@@ -46,10 +47,10 @@ struct WalkCfg {
   static constexpr int OFF_G = 4 * TILE;
   static constexpr int OFF_F = 6 * TILE;              // per-token factors, NF arrays of 128 floats
   static constexpr int NF = 8;
-  static constexpr int OFF_W = OFF_F + NF * 128 * 4;  // per-warp partner factors, 4 x 128
+  static constexpr int OFF_W = OFF_F + NF * 128 * 4;  // per-warp partner factors, 8 x 128
   // the normaliser weights as the B operand of the dn product: 16 x 128 K-major bf16 (row 0
   // the hi, row 1 the lo plane, rows 2..15 zero), two buffers (chunk parity)
-  static constexpr int OFF_WN = OFF_W + 4 * 128 * 4;
+  static constexpr int OFF_WN = OFF_W + 8 * 128 * 4;
   static constexpr int WN_BYTES = 4096;
   static constexpr int OFF_BAR = OFF_WN + 2 * WN_BYTES;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * 8;
@@ -58,7 +59,7 @@ struct WalkCfg {
 };
 
 // per-token factor arrays in the OFF_F region (token t of the chunk, or state row j)
-enum { F_PC = 0, F_PE, F_WV, F_DN };
+enum { F_PC = 0, F_PE, F_WV, F_DN, F_DOT };
 // mbarriers: tile loads (one per tile); rows -> MMA thread (hand-overs A, B, C; and D on
 // its own barrier, since the rows signal C and D back to back); MMA thread -> rows (the
 // products after A, B, C; and the state update on its own barrier, which can complete
@@ -72,13 +73,13 @@ __device__ __forceinline__ uint32_t sw_off(int row, int col) {
                     (col & 7) * 2);
 }
 
-// AND of v over the 128 threads of the row warps (named barrier 1).
+// AND of v over the 256 threads of the row warps (named barrier 1).
 __device__ __forceinline__ bool rows_and(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -104,7 +105,7 @@ struct WalkParams {
 };
 
 template <bool EXPV>
-__global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
+__global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmH,
     const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
@@ -126,10 +127,10 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < BW_COUNT; ++i) tc::mbar_init(&bar[i], (i == BW_R || i == BW_D) ? 128u : 1u);
+    for (int i = 0; i < BW_COUNT; ++i) tc::mbar_init(&bar[i], (i == BW_R || i == BW_D) ? 256u : 1u);
     tc::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 0) {
     tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tc::tmem_relinquish();
   }
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
   const uint32_t tDC = tmem, tX = tmem + 128, tAV = tmem + 256, tAK = tmem + 384;
   bool ok = true;
 
-  if (warp == 1) {
+  if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idKK = tc::idesc_bf16(128, 128, false, false);  // A, B K-major
@@ -232,12 +233,15 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       }
       if (!ok) atomicOr(&g_tc_walk_error, 1u);
     }
-  } else if (warp >= 2) {
+  } else {
     // ------------------------------------------------------------ rows
     const int row = 32 * (warp & 3) + lane;  // TMEM lane: key row s, token t or state row j
+    const int half = (warp - 1) >> 2;        // columns [64 half, 64 half + 64)
+    const int cb0 = 2 * half;                // its two 32-column chunks
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const unsigned full = 0xffffffffu;
-    const bool issuer = row == 0;  // issues the TMA loads and stores
+    const bool lead = half == 0;             // writes the per-row factors
+    const bool issuer = row == 0 && lead;    // issues the TMA loads and stores
     uint32_t nm = 0, ns = 0;       // product hand-overs (A, B, C) and state updates consumed
     auto wait_mma = [&]() -> bool {
       const bool w = __all_sync(full, tc::mbar_wait(&bar[BW_M], nm & 1, abort_flag));
@@ -304,6 +308,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       G.lis = I.lis;
       if (EXPV) G.beta = (c > 0 || P.m0 != nullptr) ? expf(I.g + I.mprev - I.mc) : 0.f;
       else G.beta = expf(I.g);
+      if (!lead) return G;
       F[F_PC * 128 + row] = in ? (I.bt - I.mt) * kLog2e + log2f(I.invd) : -INFINITY;
       F[F_PE * 128 + row] = (EXPV && in) ? I.dat / I.invd : 0.f;
       // exp(-inf) = 0 in the first chunk of an mLSTMexp sequence without an initial state
@@ -345,18 +350,12 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         tc::tmem_st32_async(tA + lane_base + 32 * cb, w);
       };
       uint32_t xa[32], xb[32];
-      tc::tmem_ld32_async(tA + lane_base, xa);
+      tc::tmem_ld32_async(tA + lane_base + 32 * cb0, xa);
       tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tA + lane_base + 32, xb);
-      one(xa, 0);
+      tc::tmem_ld32_async(tA + lane_base + 32 * cb0 + 32, xb);
+      one(xa, cb0);
       tc::tmem_wait_ld(xb);
-      tc::tmem_ld32_async(tA + lane_base + 64, xa);
-      one(xb, 1);
-      tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tA + lane_base + 96, xb);
-      one(xa, 2);
-      tc::tmem_wait_ld(xb);
-      one(xb, 3);
+      one(xb, cb0 + 1);
     };
 
     // The dk or dv transform of this key row (R: its row factor), written over the score
@@ -370,10 +369,10 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, o));
       const float Mrow = mx == -INFINITY ? 0.f : mx;
       const float grow = tc::ex2(R - Mrow);
-      float* fw = fwv + (warp & 3) * 128;
+      float* fw = fwv + (warp - 1) * 128;
       __syncwarp();
 #pragma unroll
-      for (int u = 0; u < 4; ++u) fw[lane + 32 * u] = tc::ex2(F[F_PC * 128 + lane + 32 * u] + Mrow);
+      for (int u = cb0; u < cb0 + 2; ++u) fw[lane + 32 * u] = tc::ex2(F[F_PC * 128 + lane + 32 * u] + Mrow);
       __syncwarp();
       const float* pc = F + F_PC * 128;
       const float* pe = F + F_PE * 128;
@@ -424,18 +423,12 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         tc::tmem_st16_async(tX + lane_base + 16 * ch, pk);
       };
       uint32_t xa[32], xb[32];
-      tc::tmem_ld32_async(tX + lane_base, xa);
+      tc::tmem_ld32_async(tX + lane_base + 32 * cb0, xa);
       tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tX + lane_base + 32, xb);
-      one(xa, 0);
+      tc::tmem_ld32_async(tX + lane_base + 32 * cb0 + 32, xb);
+      one(xa, cb0);
       tc::tmem_wait_ld(xb);
-      tc::tmem_ld32_async(tX + lane_base + 64, xa);
-      one(xb, 1);
-      tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tX + lane_base + 96, xb);
-      one(xa, 2);
-      tc::tmem_wait_ld(xb);
-      one(xb, 3);
+      one(xb, cb0 + 1);
     };
 
     // An output row: TMEM x fin, packed to bf16 into a staging tile (swizzled as the TMA
@@ -466,18 +459,12 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         }
       };
       uint32_t xa[32], xb[32];
-      tc::tmem_ld32_async(tA + lane_base, xa);
+      tc::tmem_ld32_async(tA + lane_base + 32 * cb0, xa);
       tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tA + lane_base + 32, xb);
-      one(xa, 0);
+      tc::tmem_ld32_async(tA + lane_base + 32 * cb0 + 32, xb);
+      one(xa, cb0);
       tc::tmem_wait_ld(xb);
-      tc::tmem_ld32_async(tA + lane_base + 64, xa);
-      one(xb, 1);
-      tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tA + lane_base + 96, xb);
-      one(xa, 2);
-      tc::tmem_wait_ld(xb);
-      one(xb, 3);
+      one(xb, cb0 + 1);
       return dsum;
     };
 
@@ -505,18 +492,12 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
         tc::tmem_st32_async(tDC + lane_base + 32 * cb, w);
       };
       uint32_t xa[32], xb[32];
-      tc::tmem_ld32_async(tDC + lane_base, xa);
+      tc::tmem_ld32_async(tDC + lane_base + 32 * cb0, xa);
       tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tDC + lane_base + 32, xb);
-      one(xa, 0);
+      tc::tmem_ld32_async(tDC + lane_base + 32 * cb0 + 32, xb);
+      one(xa, cb0);
       tc::tmem_wait_ld(xb);
-      tc::tmem_ld32_async(tDC + lane_base + 64, xa);
-      one(xb, 1);
-      tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tDC + lane_base + 96, xb);
-      one(xa, 2);
-      tc::tmem_wait_ld(xb);
-      one(xb, 3);
+      one(xb, cb0 + 1);
     };
     // ---- prologue: the last chunk's tiles, the final state's gradient (or zero), gates
     if (issuer) {
@@ -528,17 +509,17 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
     float dn = 0.f;  // dn_c, the normaliser part of the state gradient (mLSTMexp), row j
     {
       uint32_t w[32];
-      for (int cb = 0; cb < 4; ++cb) {
+      for (int cb = cb0; cb < cb0 + 2; ++cb) {
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           w[e] = __float_as_uint(P.dCT ? P.dCT[((size_t)bh * 128 + row) * 128 + 32 * cb + e] : 0.f);
         tc::tmem_st32(tDC + lane_base + 32 * cb, w);
       }
       if (EXPV && P.dnT) dn = P.dnT[(size_t)bh * 128 + row];
-      if (EXPV) F[F_DN * 128 + row] = dn;
+      if (EXPV && lead) F[F_DN * 128 + row] = dn;
     }
     if (EXPV)
-      for (int i = row; i < 2 * Cfg::WN_BYTES / 16; i += 128)
+      for (int i = row + 128 * half; i < 2 * Cfg::WN_BYTES / 16; i += 256)
         reinterpret_cast<uint4*>(smem + Cfg::OFF_WN)[i] = make_uint4(0u, 0u, 0u, 0u);
     ok = rows_and(ok);  // the zeroing is done before any row writes its weights
     Gates cur = gate_factors(NC - 1, gate_load(NC - 1));
@@ -590,7 +571,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       if (update) {
         const float wv = F[F_WV * 128 + row];
 #pragma unroll 4
-        for (int col = 0; col < 128; col += 8) {
+        for (int col = 64 * half; col < 64 * half + 64; col += 8) {
           const uint32_t off = sw_off(row, col);
           const uint4 raw = *reinterpret_cast<const uint4*>(sH + off);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -611,9 +592,10 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       // chunk's dv score overwrites once the state update has been handed over
       ok = wait_mma() && ok;
       if (EXPV && update) {
-        dn += dn_increment();       // dn_{c-1}
-        F[F_DN * 128 + row] = dn;   // read by the next chunk's dk rescale (every row's dk
-                                    // rescale of this chunk is done: the products waited for it)
+        dn += dn_increment();  // dn_{c-1}
+        // read by the next chunk's dk rescale (every row's dk rescale of this chunk is
+        // done: the products waited for it)
+        if (lead) F[F_DN * 128 + row] = dn;
       }
       signal(BW_D);
       // ---- dv out, staged over V (its products are done)
@@ -624,10 +606,11 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
       if (issuer) store_tile(&tmDV, sV, c);
       // ---- dk out, staged over dC's hi plane, with k . dk from the K tile
       const float dot = epilogue(tAK, P.scale, sG, true);
-      if (valid) P.pk[(size_t)bh * P.T + (size_t)c * 128 + row] = dot;
+      if (!lead) F[F_DOT * 128 + row] = dot;  // this half's share of k . dk
       tc::fence_proxy_async_smem();
       ok = rows_and(ok);
       if (!ok) break;
+      if (lead && valid) P.pk[(size_t)bh * P.T + (size_t)c * 128 + row] = dot + F[F_DOT * 128 + row];
       if (issuer) {
         store_tile(&tmDK, sG, c);
         if (c > 0) {
@@ -645,14 +628,14 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
     // the last state update
     if (ok) ok = wait_state();
     if (ok && P.d0 != nullptr) {
-      for (int cb = 0; cb < 4; ++cb) {
+      for (int cb = cb0; cb < cb0 + 2; ++cb) {
         float x[32];
         tc::tmem_ld32(tDC + lane_base + 32 * cb, x);
         float4* dst = reinterpret_cast<float4*>(P.d0 + ((size_t)bh * 128 + row) * 128 + 32 * cb);
 #pragma unroll
         for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
       }
-      if (EXPV) P.dn0[(size_t)bh * 128 + row] = dn;
+      if (EXPV && lead) P.dn0[(size_t)bh * 128 + row] = dn;
     }
     if (issuer) tc::bulk_wait_all();
     if (!ok) atomicOr(&g_tc_walk_error, 1u);
@@ -660,7 +643,7 @@ __global__ void __launch_bounds__(192, 1) bwd_walk_kernel(
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
@@ -698,7 +681,7 @@ static cudaError_t launch_walk(const Problem& p, const BwdArgs& a, cudaStream_t 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)WalkCfg::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)p.BH, 192, WalkCfg::SMEM, s>>>(tQ, tK, tV, tH, tDK, tDV, P);
+  kern<<<(unsigned)p.BH, 288, WalkCfg::SMEM, s>>>(tQ, tK, tV, tH, tDK, tDV, P);
   return cudaGetLastError();
 }
 
