@@ -515,8 +515,9 @@ def sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev, B, NH, T
     """Backward at one sweep point: mlstm_bwd timed like the forward, per kernel.
 
     Reports backward TFLOP/s (algorithmic count 8 T d^2 + T L 5 d per head) and
-    the intra-chunk kernels' (dq, dk, dv) combined TFLOP/s against the dense
-    bf16 peak.  Inputs: the point's forward outputs and an upstream dh ~ N(0,1).
+    the intra-chunk kernels' (dq, dk, dv; at chunk 128 with d 128 dq and the walker,
+    whose count includes the state-gradient products) combined TFLOP/s against the
+    dense bf16 peak.  Inputs: the point's forward outputs and an upstream dh ~ N(0,1).
     """
     import torch
     g = torch.Generator(device="cpu").manual_seed(7)
@@ -559,7 +560,7 @@ def sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev, B, NH, T
     kms = {n: sum(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs) / args.steps
            for i, n in enumerate(names)}
     costs = kernel_costs(T, d, d, L, var == 1, 2)
-    intra = [n for n in names if n.split("_")[0] in ("dq", "dk", "dv")]
+    intra = [n for n in names if n.split("_")[0] in ("dq", "dk", "dv", "dkv")]
     intra_fl = B * NH * sum(costs[n][0] for n in intra)
     intra_ms = sum(kms[n] for n in intra)
     return {"bwd_ms": ms, "bwd_tflops": B * NH * flops_bwd(T, d, d, L) / ms / 1e9,
