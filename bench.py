@@ -38,7 +38,7 @@ KERNEL_SOURCES = {
     "dv_simt": "simt_bwd.cu", "output_fwd_tc": "tc_fwd.cu", "dq_tc": "tc_bwd.cu",
     "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
     "output_fwd_xl": "tc_fwd_xl.cu",
-    "state_bwd_tc": "tc_state.cu", "dkv_walk_tc": "tc_bwd_walk.cu",
+    "state_bwd_tc": "tc_state.cu", "dkv_walk_tc": "tc_bwd_walk.cu", "fwd_walk_tc": "tc_fwd_walk.cu",
 }
 
 
@@ -87,6 +87,11 @@ def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
         # state gradients, dk and dv in one pass: the state-gradient recurrence and the
         # dk, dv contractions; q, k, v, dh read once, dk, dv and k.dk written, the state
         # gradients never leave the chip
+        # the states and the outputs in one pass: q, k, v read once, h, the states (both
+        # planes, the backward reads them) and the normaliser written
+        "fwd_walk": (2 * tdd + T * L * (dqk + dhv),
+                     T * (2 * dqk + 2 * dhv) * io_bytes + g * tok_f + st_full + stn
+                     + (tok_f if exp_variant else 0)),
         "dkv_walk": (3 * tdd + T * L * (2 * dqk + dhv),
                      T * (3 * dqk + 3 * dhv) * io_bytes
                      + (g + (2 if exp_variant else 0) + 1) * tok_f),

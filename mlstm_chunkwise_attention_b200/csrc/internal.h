@@ -111,6 +111,9 @@ cudaError_t fetch_tc_state_error(unsigned int* flag);
 bool bwd_walk_supported(const Problem& p);
 cudaError_t launch_bwd_walk(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_walk_error(unsigned int* flag);
+bool fwd_walk_supported(const Problem& p);
+cudaError_t launch_fwd_walk(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t fetch_tc_fwalk_error(unsigned int* flag);
 
 // recurrent-form kernels (recurrent.cu)
 cudaError_t launch_final_state(const Problem& p, const void* k, const void* v, const float* b,

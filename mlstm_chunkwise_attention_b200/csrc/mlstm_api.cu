@@ -146,9 +146,15 @@ struct BwdStep { const char* name; BwdLauncher fn; };
 constexpr int kMaxSteps = 8;
 
 // The kernels each pass enqueues, in order.
-int fwd_plan(const Problem& p, FwdStep* st) {
+// want_h false: the state-only pass (the plan without its last step, the output kernel).
+int fwd_plan(const Problem& p, FwdStep* st, bool want_h = true) {
   int n = 0;
   st[n++] = {"gate_prep", mlstm::launch_gate_prep};
+  if (want_h && mlstm::fwd_walk_supported(p)) {
+    // one pass per head over its chunks gives the states and the outputs
+    st[n++] = {"fwd_walk_tc", mlstm::launch_fwd_walk};
+    return n;
+  }
   if (mlstm::state_tc_supported(p))
     st[n++] = {"state_fwd_tc", mlstm::launch_state_fwd_tc};
   else
@@ -330,7 +336,7 @@ int fwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_fwd");
   if (st != MLSTM_OK) return st;
   FwdStep steps[kMaxSteps];
-  const int n = fwd_plan(p, steps);
+  const int n = fwd_plan(p, steps, h != nullptr);
   st = run_plan(steps, h ? n : n - 1, p, a, s);  // the output kernel is the plan's last step
   if (st != MLSTM_OK || !state_out) return st;
   char* out = (char*)state_out;
@@ -640,7 +646,7 @@ const char* mlstm_last_error(void) { return g_last_error; }
 int mlstm_device_status(void* stream) {
   int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
   if (st != MLSTM_OK) return st;
-  unsigned int flag = 0, flag_bwd = 0, flag_state = 0, flag_xl = 0, flag_walk = 0;
+  unsigned int flag = 0, flag_bwd = 0, flag_state = 0, flag_xl = 0, flag_walk = 0, flag_fwalk = 0;
   st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_bwd_error(&flag_bwd), "device error flag");
@@ -651,7 +657,9 @@ int mlstm_device_status(void* stream) {
   if (st != MLSTM_OK) return st;
   st = cuda_status(mlstm::fetch_tc_walk_error(&flag_walk), "device error flag");
   if (st != MLSTM_OK) return st;
-  flag |= flag_bwd | flag_state | flag_xl | flag_walk;
+  st = cuda_status(mlstm::fetch_tc_fwalk_error(&flag_fwalk), "device error flag");
+  if (st != MLSTM_OK) return st;
+  flag |= flag_bwd | flag_state | flag_xl | flag_walk | flag_fwalk;
   if (flag) {
     snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
     return MLSTM_ERR_TIMEOUT;

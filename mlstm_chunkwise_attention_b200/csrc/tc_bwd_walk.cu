@@ -27,6 +27,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "walk_common.cuh"
 
 namespace mlstm {
 
@@ -67,30 +68,9 @@ enum { F_PC = 0, F_PE, F_WV, F_DN, F_DOT };
 // with its waiter, so parity waits cannot alias.
 enum { BW_Q = 0, BW_K, BW_V, BW_H, BW_R, BW_D, BW_M, BW_S, BW_COUNT };
 
-__device__ __forceinline__ uint32_t sw_off(int row, int col) {
-  // byte offset of (row, col) in a [128 rows x 128 cols] bf16 tile of two swizzled blocks
-  return (uint32_t)((col >> 6) * 16384 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
-                    (col & 7) * 2);
-}
-
-// AND of v over the 256 threads of the row warps (named barrier 1).
-__device__ __forceinline__ bool rows_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v)
-      : "memory");
-  return r != 0;
-}
-
-// Wait until every bulk store group of this thread but the newest has read its source.
-__device__ __forceinline__ void bulk_wait_read_but_one() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
+using walk::sw_off;
+constexpr auto rows_and = walk::rows_and<256>;
+using walk::bulk_wait_read_but_one;
 
 }  // namespace
 
@@ -318,24 +298,17 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
         const float wn = alpha * I.dat;
         const bf16 hi = __float2bfloat16_rn(wn);
         const bf16 lo = __float2bfloat16_rn(wn - __bfloat162float(hi));
-        // K-major 128-byte swizzle: token t of row r at block t / 64, chunk (t % 64) / 8 ^ r
-        uint8_t* wt = smem + Cfg::OFF_WN + ((NC - 1 - c) & 1) * Cfg::WN_BYTES + (row >> 6) * 2048 +
-                      (row & 7) * 2;
-        *reinterpret_cast<bf16*>(wt + (((row & 63) >> 3) << 4)) = hi;
-        *reinterpret_cast<bf16*>(wt + 128 + ((((row & 63) >> 3) ^ 1) << 4)) = lo;
+        uint8_t* wt = smem + Cfg::OFF_WN + ((NC - 1 - c) & 1) * Cfg::WN_BYTES;
+        *reinterpret_cast<bf16*>(wt + walk::n16_off(0, row)) = hi;
+        *reinterpret_cast<bf16*>(wt + walk::n16_off(1, row)) = lo;
       }
       return G;
     };
-    // columns 0 and 1 of the score buffer after a state update: the normaliser's increment
+    // columns 0 and 1 of the score buffer after the dk accumulate: the normaliser's increment
     auto dn_increment = [&]() -> float {
-      uint32_t r0, r1;
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
-          "tcgen05.wait::ld.sync.aligned;"
-          : "=r"(r0), "=r"(r1)
-          : "r"(tX + lane_base)
-          : "memory");
-      return __uint_as_float(r0) + __uint_as_float(r1);
+      float a, b;
+      walk::tmem_ld2(tX + lane_base, a, b);
+      return a + b;
     };
     // Rescale an inter-term accumulator row in TMEM: x = rs x (+ rs dn[col] for dk, mLSTMexp).
     auto rescale = [&](uint32_t tA, float rs, bool with_dn) {
