@@ -11,7 +11,8 @@
 //   h_t = O_t / max(|alpha_t q_t.n_c / sqrt(d_qk) + sum_s P_ts|, exp(-m_t))  (mLSTMexp)
 // as the chunk-128 output kernel of tc_fwd.cu does, then updates
 //   C_{c+1} = beta_c C_c + K^T diag(w) V,  n_{c+1} = beta_c n_c + K^T w
-// on the tensor core, w_s = exp(g_c - b_s + log i_s - m_c).  The states never
+// on the tensor core, w_s = exp(g_c - b_s + log i_s - m_c), as (diag(w) K)^T V so
+// that the update does not wait for P V to finish reading V.  The states never
 // make a round trip through HBM between the two halves of the forward, and q,
 // k, v are read once.  "Tiled Flash Linear Attention" (TFLA summary page,
 // Problem: materialised chunk states cost IO; Approach).
@@ -19,10 +20,12 @@
 // Roles: one thread (warp 0) issues the MMAs; eight row warps, two per TMEM lane
 // quarter, each own one token or state row (the TMEM lane) and half of its
 // columns; one row thread issues the TMA loads and stores.  Hand-overs:
-//   rows: stage C_c -> A | P transform, inter rescale -> B | w V -> D | h out,
+//   rows: stage C_c -> A | P transform, inter rescale -> B | w K -> D | h out,
 //         next gate factors
-//   MMA:  Q K^T | A: Q C_c (hi), Q n_c (hi, lo) | B: P V | D: C += K^T (w V) (hi, lo),
-//         K^T w (hi, lo)
+//   MMA:  Q K^T, K^T w (hi, lo) | A: Q C_c (hi), Q n_c (hi, lo) | B: P V |
+//         D: C += (w K)^T V (hi, lo)
+// The next chunk's gate factors (and w as the n-update operand) are written before the
+// hand-over D, so the n update can start as soon as the next chunk's tiles land.
 // Two K/V buffer sets alternate between chunks; the set a chunk does not use
 // holds its C staging, and takes the next chunk's K and V as soon as the inter
 // product and the saved-state store have read it.  Every wait is bounded; on a
@@ -42,7 +45,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 using walk::sw_off;
 using walk::TILE;
 
-// Shared memory: Q tile; two K/V sets (K at +0, V at +TILE); the w V lo plane;
+// Shared memory: Q tile; two K/V sets (K at +0, V at +TILE); the w K lo plane;
 // per-token factors; the N = 16 operand tiles of n (one) and w (two, by chunk parity).
 struct FwalkCfg {
   static constexpr int OFF_Q = 0;
@@ -56,10 +59,12 @@ struct FwalkCfg {
   static constexpr int OFF_BAR = OFF_WT + 2 * N16_BYTES;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * 8;
   static constexpr size_t SMEM = 1024 + OFF_TMEM + 16;
-  static constexpr uint32_t TMEM_COLS = 512;  // C, S / P, O, q.n (16), K^T w (16)
+  static constexpr uint32_t TMEM_COLS = 512;  // C, S / P, O, q.n (16), K^T w (2 x 16)
 };
 
-enum { F_CF = 0, F_RS0, F_RS1 };
+// the key factors of chunk c in F_CF0 + (c & 1) (written a chunk ahead), the two halves'
+// row-sum shares
+enum { F_CF0 = 0, F_CF1, F_RS0, F_RS1 };
 // mbarriers: Q tile, K/V sets, rows -> MMA (A, B), rows -> MMA (D), MMA -> rows
 // (after A, B), state update done.  Each barrier's phases alternate with its waiter.
 enum { BF_Q = 0, BF_KV0, BF_KV1, BF_R, BF_D, BF_M, BF_S, BF_COUNT };
@@ -111,6 +116,8 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // K^T w of chunk c goes to tNU + 16 (c & 1): the rows read the previous chunk's after its
+  // state update, which may come after this chunk's first products
   const uint32_t tC = tmem, tS = tmem + 128, tO = tmem + 256, tN = tmem + 384, tNU = tmem + 400;
   bool ok = true;
 
@@ -150,9 +157,19 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         if (!ok) break;
 #pragma unroll
         for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tS, kmaj(aQ, k), kmaj(aK, k), idKK, k > 0);
+        // the n increment K^T w (hi, lo): w of chunk c was written before the previous
+        // chunk's hand-over D (in the prologue for the first chunk, so after A there)
+        auto n_update = [&]() {
+          const uint32_t wt = aWT + (c & 1) * Cfg::N16_BYTES;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc::mma_bf16_ss(tNU + 16 * (c & 1), mnmaj(aK, k), n16(wt, k), idNM, k > 0);
+        };
+        if (EXPV && c > 0 && c + 1 < NC) n_update();
         // A (C_c staged): O = Q C_c (hi plane); Q n_c (hi, lo) into the two q.n columns
         ok = wait_rows();
         if (!ok) break;
+        if (EXPV && c == 0 && c + 1 < NC) n_update();
 #pragma unroll
         for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tO, kmaj(aQ, k), mnmaj(aG, k), idKM, k > 0);
         if (EXPV) {
@@ -166,20 +183,15 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
 #pragma unroll
         for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tO, tS + 8 * k, mnmaj(aV, k), idKM, 1);
         tc::tc_commit(&bar[BF_M]);
-        // D (w V staged: hi plane over V, lo plane apart): C_{c+1} = beta_c C_c (the rows
-        // scaled it) + K^T (w V); K^T w (hi, lo) into the two n-update columns
+        // D (w K staged: hi plane over K, lo plane apart): C_{c+1} = beta_c C_c (the rows
+        // scaled it) + (w K)^T V, while P V runs
         ok = wait_bar(BF_D, c & 1);
         if (!ok) break;
         if (c + 1 < NC) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             tc::mma_bf16_ss(tC, mnmaj(aK, k), mnmaj(aV, k), idMM, 1);
-            tc::mma_bf16_ss(tC, mnmaj(aK, k), mnmaj(aWL, k), idMM, 1);
-          }
-          if (EXPV) {
-            const uint32_t wt = aWT + (c & 1) * Cfg::N16_BYTES;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tNU, mnmaj(aK, k), n16(wt, k), idNM, k > 0);
+            tc::mma_bf16_ss(tC, mnmaj(aWL, k), mnmaj(aV, k), idMM, 1);
           }
         }
         tc::tc_commit(&bar[BF_S]);
@@ -269,7 +281,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
       G.w = in ? expf(I.g - I.bt + I.lit - I.mc) : 0.f;
       G.mt = I.mt;
       if (lead) {
-        F[F_CF * 128 + row] = in ? (I.lit - I.bt) * kLog2e : -INFINITY;
+        F[(F_CF0 + (c & 1)) * 128 + row] = in ? (I.lit - I.bt) * kLog2e : -INFINITY;
         if (EXPV) {
           uint8_t* wt = smem + Cfg::OFF_WT + (c & 1) * Cfg::N16_BYTES;
           const bf16 hi = __float2bfloat16_rn(G.w);
@@ -321,10 +333,10 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     // P of this query row over this half's keys, written over S in TMEM as packed bf16:
     // p = s 2^(r2 + cf_s), zero past the diagonal (the chunk-128 output kernel's form).
     // Returns the half's share of the row sum.
-    auto transform = [&](float r2) -> float {
+    auto transform = [&](float r2, int c) -> float {
       float rs = 0.f;
       const int qd = warp & 3;
-      const float* cf = F + F_CF * 128;
+      const float* cf = F + (F_CF0 + (c & 1)) * 128;
       auto one = [&](const uint32_t (&xr)[32], int ch) {
         uint32_t pk[16];
         if (ch > qd) {
@@ -406,7 +418,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         ok = wait_state();
         if (EXPV) {
           float a, b;
-          walk::tmem_ld2(tNU + lane_base, a, b);
+          walk::tmem_ld2(tNU + 16 * ((c - 1) & 1) + lane_base, a, b);
           n += a + b;  // n_c = beta_{c-1} n_{c-1} (scaled below, a chunk ago) + K^T w
         }
         if (issuer && ok) {
@@ -448,7 +460,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
       // ---- B: P over this half's keys and its row-sum share, the inter term scaled by qfac,
       // q.n
       ok = wait_mma();
-      const float rs = transform(cur.r2);
+      const float rs = transform(cur.r2, c);
       rescale(cur.qfac);
       float inter_norm = 0.f;
       if (EXPV) {
@@ -464,14 +476,18 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         tc::bulk_wait_read_all();
         load_kv(c + 1);
       }
-      // ---- D: w V (hi plane over V, lo plane apart) once P V has read V
-      ok = wait_mma() && ok;
+      // ---- the next chunk's gate factors (its key factors in the other buffer, its w as the
+      // n-update operand), before the hand-over D that the next n update follows
+      Gates nxtG = cur;
+      if (c + 1 < NC) nxtG = gate_factors(c + 1, nxt);
+      // ---- D: w K (hi plane over K, lo plane apart): the score, inter and n-update products
+      // that read K are done (waited for above)
       if (c + 1 < NC) {
-        uint8_t* sV = set_of(c) + TILE;
+        uint8_t* sK = set_of(c);
 #pragma unroll 4
         for (int col = 64 * half; col < 64 * half + 64; col += 8) {
           const uint32_t off = sw_off(row, col);
-          const uint4 raw = *reinterpret_cast<const uint4*>(sV + off);
+          const uint4 raw = *reinterpret_cast<const uint4*>(sK + off);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t hi[4], lo[4];
 #pragma unroll
@@ -482,14 +498,15 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
             hi[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
             lo[e] = tc::pack_bf16(y0 - __bfloat162float(h0), y1 - __bfloat162float(h1));
           }
-          *reinterpret_cast<uint4*>(sV + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sK + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sWL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
       signal(BF_D);
-      ok = rows_and(ok);  // both halves' row sums are in shared memory
+      // ---- h = O / den once P V is done, staged over Q (its products are done)
+      ok = wait_mma() && ok;
+      ok = rows_and(ok);  // and both halves' row sums are in shared memory
       if (!ok) break;
-      // ---- h = O / den, staged over Q (its products are done)
       float inv = 1.f;
       if (EXPV) {
         const float a = inter_norm + (F[F_RS0 * 128 + row] + F[F_RS1 * 128 + row]);
@@ -505,11 +522,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         tc::tma_store_3d(&tmH, sQ + 16384, 64, c * 128, bh);
         tc::bulk_commit_group();
       }
-      // ---- the next chunk's gate factors, while the state update runs
-      if (c + 1 < NC) {
-        cur = gate_factors(c + 1, nxt);
-        ok = rows_and(ok);
-      }
+      cur = nxtG;
     }
     // the last chunk's hand-over: every product has completed
     if (ok) ok = wait_state();
