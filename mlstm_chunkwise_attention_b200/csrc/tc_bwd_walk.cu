@@ -314,11 +314,25 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
     auto rescale = [&](uint32_t tA, float rs, bool with_dn) {
       auto one = [&](const uint32_t (&x)[32], int cb) {
         uint32_t w[32];
+        if (EXPV && with_dn) {  // rs (x + dn[col]), two lanes per f32x2 operation
+          const uint64_t r2 = tc::f2_make(rs, rs);
+          const float4* dn4 = reinterpret_cast<const float4*>(F + F_DN * 128 + 32 * cb);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float y = rs * __uint_as_float(x[e]);
-          if (EXPV && with_dn) y += rs * F[F_DN * 128 + 32 * cb + e];
-          w[e] = __float_as_uint(y);
+          for (int e = 0; e < 32; e += 4) {
+            const float4 d = dn4[e / 4];
+            const float2 y0 = tc::f2_split(tc::f2_mul(
+                tc::f2_add(tc::f2_make(__uint_as_float(x[e]), __uint_as_float(x[e + 1])),
+                           tc::f2_make(d.x, d.y)), r2));
+            const float2 y1 = tc::f2_split(tc::f2_mul(
+                tc::f2_add(tc::f2_make(__uint_as_float(x[e + 2]), __uint_as_float(x[e + 3])),
+                           tc::f2_make(d.z, d.w)), r2));
+            w[e] = __float_as_uint(y0.x);
+            w[e + 1] = __float_as_uint(y0.y);
+            w[e + 2] = __float_as_uint(y1.x);
+            w[e + 3] = __float_as_uint(y1.y);
+          }
+        } else {
+          walk::scale32(x, rs, w);
         }
         tc::tmem_st32_async(tA + lane_base + 32 * cb, w);
       };
@@ -450,18 +464,14 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
         for (int e = 0; e < 32; e += 8) {
           uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float x0 = __uint_as_float(x[e + 2 * u]), x1 = __uint_as_float(x[e + 2 * u + 1]);
-            const bf16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-            hi[u] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lo[u] = tc::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-          }
+          for (int u = 0; u < 4; ++u)
+            walk::split_hi_lo(__uint_as_float(x[e + 2 * u]), __uint_as_float(x[e + 2 * u + 1]), hi[u],
+                              lo[u]);
           const uint32_t off = sw_off(row, 32 * cb + e);
           *reinterpret_cast<uint4*>(sG + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sG + Cfg::TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(beta * __uint_as_float(x[e]));
+        walk::scale32(x, beta, w);
         tc::tmem_st32_async(tDC + lane_base + 32 * cb, w);
       };
       uint32_t xa[32], xb[32];
@@ -550,13 +560,8 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-            const float y0 = __bfloat162float(x2.x) * wv, y1 = __bfloat162float(x2.y) * wv;
-            const bf16 h0 = __float2bfloat16_rn(y0), h1 = __float2bfloat16_rn(y1);
-            hi[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lo[e] = tc::pack_bf16(y0 - __bfloat162float(h0), y1 - __bfloat162float(h1));
-          }
+          for (int e = 0; e < 4; ++e)
+            walk::split_hi_lo(walk::bf16_lo(w[e]) * wv, walk::bf16_hi(w[e]) * wv, hi[e], lo[e]);
           *reinterpret_cast<uint4*>(sH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sG + Cfg::TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }

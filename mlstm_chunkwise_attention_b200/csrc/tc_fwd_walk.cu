@@ -314,18 +314,14 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         for (int e = 0; e < 32; e += 8) {
           uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float x0 = __uint_as_float(x[e + 2 * u]), x1 = __uint_as_float(x[e + 2 * u + 1]);
-            const bf16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-            hi[u] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lo[u] = tc::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-          }
+          for (int u = 0; u < 4; ++u)
+            walk::split_hi_lo(__uint_as_float(x[e + 2 * u]), __uint_as_float(x[e + 2 * u + 1]), hi[u],
+                              lo[u]);
           const uint32_t off = sw_off(row, 32 * cb + e);
           *reinterpret_cast<uint4*>(stg + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(stg + TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(beta * __uint_as_float(x[e]));
+        walk::scale32(x, beta, w);
         tc::tmem_st32_async(tC + lane_base + 32 * cb, w);
       };
       MLSTM_WALK_PIPE(tC, one)
@@ -365,8 +361,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     auto rescale = [&](float f) {
       auto one = [&](const uint32_t (&x)[32], int cb) {
         uint32_t w[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(f * __uint_as_float(x[e]));
+        walk::scale32(x, f, w);
         tc::tmem_st32_async(tO + lane_base + 32 * cb, w);
       };
       MLSTM_WALK_PIPE(tO, one)
@@ -491,13 +486,8 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-            const float y0 = __bfloat162float(x2.x) * cur.w, y1 = __bfloat162float(x2.y) * cur.w;
-            const bf16 h0 = __float2bfloat16_rn(y0), h1 = __float2bfloat16_rn(y1);
-            hi[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lo[e] = tc::pack_bf16(y0 - __bfloat162float(h0), y1 - __bfloat162float(h1));
-          }
+          for (int e = 0; e < 4; ++e)
+            walk::split_hi_lo(walk::bf16_lo(w[e]) * cur.w, walk::bf16_hi(w[e]) * cur.w, hi[e], lo[e]);
           *reinterpret_cast<uint4*>(sK + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sWL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }

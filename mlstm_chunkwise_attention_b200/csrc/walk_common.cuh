@@ -5,6 +5,8 @@
 
 #include <stdint.h>
 
+#include "tc_common.cuh"
+
 namespace mlstm {
 namespace walk {
 
@@ -55,6 +57,31 @@ __device__ __forceinline__ void tmem_ld2(uint32_t taddr, float& a, float& b) {
 __device__ __forceinline__ uint32_t n16_off(int r, int t) {
   return (uint32_t)((t >> 6) * 2048 + r * 128 + ((((t & 63) >> 3) ^ r) << 4) + (t & 7) * 2);
 }
+
+// A pair of fp32 values as hi = bf16(x) and lo = bf16(x - hi), each a packed bf16x2 word
+// (first value in the low half); hi + lo keeps about 16 mantissa bits.  One packed
+// conversion per plane; the hi halves are widened back by a shift and a mask.
+__device__ __forceinline__ void split_hi_lo(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = tc::pack_bf16(x0, x1);
+  const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+  lo = tc::pack_bf16(x0 - h0, x1 - h1);
+}
+
+// w = f x over 32 fp32 values held as raw bits, two lanes per f32x2 multiply.
+__device__ __forceinline__ void scale32(const uint32_t (&x)[32], float f, uint32_t (&w)[32]) {
+  const uint64_t f2 = tc::f2_make(f, f);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float2 y =
+        tc::f2_split(tc::f2_mul(tc::f2_make(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), f2));
+    w[e] = __float_as_uint(y.x);
+    w[e + 1] = __float_as_uint(y.y);
+  }
+}
+
+// The two bf16 values of a packed word as fp32.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 }  // namespace walk
 }  // namespace mlstm
