@@ -52,7 +52,7 @@ struct FwalkCfg {
   static constexpr int OFF_SET0 = TILE, OFF_SET1 = 3 * TILE;
   static constexpr int OFF_WL = 5 * TILE;
   static constexpr int OFF_F = 6 * TILE;                // NF arrays of 128 floats
-  static constexpr int NF = 4;
+  static constexpr int NF = 8;
   static constexpr int OFF_NT = OFF_F + NF * 128 * 4;   // 1024-aligned: 16 x 128 bf16 K-major
   static constexpr int N16_BYTES = 4096;
   static constexpr int OFF_WT = OFF_NT + N16_BYTES;     // two buffers
@@ -62,9 +62,10 @@ struct FwalkCfg {
   static constexpr uint32_t TMEM_COLS = 512;  // C, S / P, O, q.n (16), K^T w (2 x 16)
 };
 
-// the key factors of chunk c in F_CF0 + (c & 1) (written a chunk ahead), the two halves'
-// row-sum shares
-enum { F_CF0 = 0, F_CF1, F_RS0, F_RS1 };
+// Per chunk (buffer c & 1, written a chunk ahead): the key factors cf_s = (log i_s - b_s)
+// log2 e, their maxima M over each 32-key block (F_MB, 4 per buffer) and 2^(cf_s - M);
+// the two halves' row-sum shares.
+enum { F_CF0 = 0, F_CF1, F_KP0, F_KP1, F_RS0, F_RS1, F_MB };
 // mbarriers: Q tile, K/V sets, rows -> MMA (A, B), rows -> MMA (D), MMA -> rows
 // (after A, B), state update done.  Each barrier's phases alternate with its waiter.
 enum { BF_Q = 0, BF_KV0, BF_KV1, BF_R, BF_D, BF_M, BF_S, BF_COUNT };
@@ -281,7 +282,16 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
       G.w = in ? expf(I.g - I.bt + I.lit - I.mc) : 0.f;
       G.mt = I.mt;
       if (lead) {
-        F[(F_CF0 + (c & 1)) * 128 + row] = in ? (I.lit - I.bt) * kLog2e : -INFINITY;
+        // this warp's 32 rows are one key block: its largest key factor (0 for a block wholly
+        // past the end) and the separable key factor 2^(cf_s - M) <= 1
+        const float cf = in ? (I.lit - I.bt) * kLog2e : -INFINITY;
+        float mx = cf;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, o));
+        if (mx == -INFINITY) mx = 0.f;
+        F[(F_CF0 + (c & 1)) * 128 + row] = cf;
+        F[(F_KP0 + (c & 1)) * 128 + row] = tc::ex2(cf - mx);
+        if (lane == 0) F[F_MB * 128 + 4 * (c & 1) + (warp & 3)] = mx;
         if (EXPV) {
           uint8_t* wt = smem + Cfg::OFF_WT + (c & 1) * Cfg::N16_BYTES;
           const bf16 hi = __float2bfloat16_rn(G.w);
@@ -327,29 +337,54 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
       MLSTM_WALK_PIPE(tC, one)
     };
     // P of this query row over this half's keys, written over S in TMEM as packed bf16:
-    // p = s 2^(r2 + cf_s), zero past the diagonal (the chunk-128 output kernel's form).
-    // Returns the half's share of the row sum.
+    // p = s 2^(r2 + cf_s), zero past the diagonal.  The 32-key blocks left of the diagonal
+    // take the separable form s 2^(cf_s - M) 2^(r2 + M) (M: the block's largest cf, so
+    // both factors are at most 1: every key there precedes the query); the diagonal block
+    // takes each element's own exponent and the causal mask.  Returns the half's share of
+    // the row sum.
     auto transform = [&](float r2, int c) -> float {
       float rs = 0.f;
       const int qd = warp & 3;
       const float* cf = F + (F_CF0 + (c & 1)) * 128;
+      const float* kp = F + (F_KP0 + (c & 1)) * 128;
+      const float* mb = F + F_MB * 128 + 4 * (c & 1);
       auto one = [&](const uint32_t (&xr)[32], int ch) {
         uint32_t pk[16];
         if (ch > qd) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = 0u;
-        } else {
+        } else if (ch == qd) {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const int s0 = ch * 32 + i;
             float p0 = __uint_as_float(xr[i]) * tc::ex2(r2 + cf[s0]);
             float p1 = __uint_as_float(xr[i + 1]) * tc::ex2(r2 + cf[s0 + 1]);
-            if (ch == qd) {
-              if (s0 > row) p0 = 0.f;
-              if (s0 + 1 > row) p1 = 0.f;
-            }
+            if (s0 > row) p0 = 0.f;
+            if (s0 + 1 > row) p1 = 0.f;
             if (EXPV) rs += p0 + p1;
             pk[i >> 1] = tc::pack_bf16(p0, p1);
+          }
+        } else {
+          const float f = tc::ex2(r2 + mb[ch]);
+          const uint64_t f2 = tc::f2_make(f, f);
+          uint64_t acc = tc::f2_make(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 g4 = *reinterpret_cast<const float4*>(kp + ch * 32 + i);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t x2 =
+                  tc::f2_make(__uint_as_float(xr[i + 2 * h]), __uint_as_float(xr[i + 2 * h + 1]));
+              const uint64_t g2 = h ? tc::f2_make(g4.z, g4.w) : tc::f2_make(g4.x, g4.y);
+              const uint64_t p2 = tc::f2_mul(tc::f2_mul(x2, g2), f2);
+              if (EXPV) acc = tc::f2_add(acc, p2);
+              const float2 pp = tc::f2_split(p2);
+              pk[(i >> 1) + h] = tc::pack_bf16(pp.x, pp.y);
+            }
+          }
+          if (EXPV) {
+            const float2 a = tc::f2_split(acc);
+            rs += a.x + a.y;
           }
         }
         tc::tmem_st16_async(tS + lane_base + 16 * ch, pk);
@@ -369,14 +404,14 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     // h = O / den of this row, packed to bf16 into the staging tile.
     auto epilogue = [&](float inv, uint8_t* stg) {
       auto one = [&](const uint32_t (&x)[32], int cb) {
+        uint32_t g[32];
+        walk::scale32(x, inv, g);
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
-          float g[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) g[u] = __uint_as_float(x[e + u]) * inv;
+          auto f = [&](int u) { return __uint_as_float(g[e + u]); };
           *reinterpret_cast<uint4*>(stg + sw_off(row, 32 * cb + e)) =
-              make_uint4(tc::pack_bf16(g[0], g[1]), tc::pack_bf16(g[2], g[3]),
-                         tc::pack_bf16(g[4], g[5]), tc::pack_bf16(g[6], g[7]));
+              make_uint4(tc::pack_bf16(f(0), f(1)), tc::pack_bf16(f(2), f(3)),
+                         tc::pack_bf16(f(4), f(5)), tc::pack_bf16(f(6), f(7)));
         }
       };
       MLSTM_WALK_PIPE(tO, one)
