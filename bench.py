@@ -557,8 +557,14 @@ def sweep_bwd_point(args, binding, x, h, saved, sizes, sh, stream, dev, B, NH, T
     torch.cuda.synchronize(dev)
     e0.record(stream)
     for i in range(args.steps):
-        call(arrs[i])
+        call()
     e1.record(stream)
+    torch.cuda.synchronize(dev)
+    # per-kernel times: the same calls with every kernel on the caller's stream, each alone
+    binding.mlstm_set_serial_launches(True)
+    for i in range(args.steps):
+        call(arrs[i])
+    binding.mlstm_set_serial_launches(False)
     torch.cuda.synchronize(dev)
     binding.check_device()
     ms = e0.elapsed_time(e1) / args.steps
@@ -728,12 +734,19 @@ def main():
     barrier()
     start.record(stream)
     for i in range(args.steps):
-        step(x, fwd_evs[i], bwd_evs[i])
+        step(x)
     end.record(stream)
     barrier()
     clk = clocks.stop()
     ms = start.elapsed_time(end)
     ms_max = max_over_ranks(ms)
+    # per-kernel times: the same steps once more with every kernel on the caller's stream
+    # (the timed steps overlap dq with the backward walker), each kernel bracketed alone
+    binding.mlstm_set_serial_launches(True)
+    for i in range(args.steps):
+        step(x, fwd_evs[i], bwd_evs[i])
+    binding.mlstm_set_serial_launches(False)
+    barrier()
     per_kernel = {n: 0.0 for n in names}
     for fe, be in ev_keep:
         for i in range(nf):
@@ -818,6 +831,8 @@ def main():
         "config": workload_config(spec, world),
         "tokens_per_s": tokens_s, "pct_bf16_peak": 100.0 * tflops / (world * peaks["bf16_tflops"]),
         "kernel_ms": per_kernel,
+        "kernel_ms_mode": "each kernel alone (mlstm_set_serial_launches); the timed steps run "
+                          "dq alongside the backward walker where the plan has one",
         "roofline": roofline,
         "cpu_baseline": cpu_base,
         "e2e": {"value": e2e_tflops, "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -129,7 +129,13 @@ int mlstm_fwd(const void* q, const void* k, const void* v,
  * mlstm_fwd on the same inputs (required, not NULL).  Writes dq, dk, dv and
  * the preactivation gradients digate_pre, dfgate_pre.  The timed training
  * kernels of the TFLA summary page (Key results) are this forward plus this
- * backward. */
+ * backward.  On the bf16 path with chunk 128 and d_qk = d_hv = 128 one kernel
+ * runs on a high-priority stream of the calling thread, forked from `stream`
+ * after the kernels before it and joined back before the last one, so that
+ * dq can use the SMs it leaves idle; all work is ordered after what `stream`
+ * held at the call and before what it receives later.  That stream and its two
+ * events are created on the thread's first such call on a device (make it
+ * before any stream capture) and kept until the process exits. */
 int mlstm_bwd(const void* q, const void* k, const void* v,
               const void* igate_pre, const void* fgate_pre,
               const void* h, const void* dh, const void* saved,
@@ -326,10 +332,17 @@ int mlstm_bwd_launch_count(int B, int NH, int T, int d_qk, int d_hv, int chunk,
 const char* mlstm_launch_name(int pass, int index, int B, int NH, int T, int d_qk,
                               int d_hv, int chunk, int variant, int dtype);
 
+/* Run every kernel of the calling thread's later calls on their own stream
+ * (serial != 0), or let mlstm_bwd run one kernel on its side stream again
+ * (0, the default).  The results are the same either way; the serial order
+ * times each kernel alone.  Returns MLSTM_OK. */
+int mlstm_set_serial_launches(int serial);
+
 /* Per-kernel timing hook for the calling thread.  While set (count > 0),
  * every mlstm_fwd / mlstm_bwd call records events[2i] (a cudaEvent_t passed
- * as void*) on its stream just before its i-th kernel and events[2i+1] just
- * after it, for i < count/2; kernels beyond that are not bracketed.  The
+ * as void*) on the stream its i-th kernel runs on just before that kernel and
+ * events[2i+1] just after it, for i < count/2; kernels beyond that are not
+ * bracketed.  The
  * array is borrowed, not copied: it must stay valid until the hook is
  * cleared with (NULL, 0).  Returns MLSTM_ERR_INVALID for count < 0 or a NULL
  * array with count > 0. */

@@ -57,6 +57,7 @@ EXPORTS = {
     "mlstm_last_error": (ctypes.c_char_p, []),
     "mlstm_launch_name": (ctypes.c_char_p, [ctypes.c_int, ctypes.c_int] + _SIZES),
     "mlstm_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
+    "mlstm_set_serial_launches": (ctypes.c_int, [ctypes.c_int]),
     "mlstm_device_status": (ctypes.c_int, [_P]),
     "mlstm_fwd_noalloc": (ctypes.c_int, [_P] * 6 + _SIZES + [_P]),
     "mlstm_state_size": (ctypes.c_size_t, [ctypes.c_int] * 5),
@@ -183,6 +184,12 @@ def mlstm_launch_name(pass_, index, *sizes):
 def mlstm_set_timing_events(events, count):
     """events: a ctypes array of void* (cudaEvent_t handles), or None."""
     return load().mlstm_set_timing_events(events, count)
+
+
+def mlstm_set_serial_launches(serial):
+    """True: every kernel of this thread's later calls on the caller's stream (for timing
+    each kernel alone); False (the default): the backward may overlap two of them."""
+    return load().mlstm_set_serial_launches(1 if serial else 0)
 
 
 # --------------------------------------------------------------------------

@@ -141,9 +141,43 @@ thread_local int g_nevents = 0;
 
 typedef cudaError_t (*FwdLauncher)(const Problem&, const mlstm::FwdArgs&, cudaStream_t);
 typedef cudaError_t (*BwdLauncher)(const Problem&, const mlstm::BwdArgs&, cudaStream_t);
-struct FwdStep { const char* name; FwdLauncher fn; };
-struct BwdStep { const char* name; BwdLauncher fn; };
+// side: the step runs on the calling thread's high-priority side stream, forked from the
+// caller's stream after the steps before it, while the following steps continue on the
+// caller's stream; join: the caller's stream waits for the side work before this step.
+struct FwdStep { const char* name; FwdLauncher fn; bool side = false, join = false; };
+struct BwdStep { const char* name; BwdLauncher fn; bool side = false, join = false; };
 constexpr int kMaxSteps = 8;
+
+// The side stream and fork / join events of the calling thread on the current device,
+// created on its first use there (a call that forks must not be the first one made during
+// a stream capture) and kept until the process exits.  Per thread: one thread enqueues its
+// calls in order, so reusing the events is safe; a capture of the caller's stream takes
+// the side stream in through the fork event.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+thread_local SideStream g_side[kMaxSideDevices];
+thread_local bool g_serial = false;  // mlstm_set_serial_launches: every step on the caller's stream
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  SideStream& r = g_side[dev];
+  if (r.stream == nullptr) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&r.stream, cudaStreamNonBlocking, greatest)) != cudaSuccess)
+      return e;
+  }
+  *out = &r;
+  return cudaSuccess;
+}
 
 // The kernels each pass enqueues, in order.
 // want_h false: the state-only pass (the plan without its last step, the output kernel).
@@ -173,10 +207,12 @@ int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
   int n = 0;
   st[n++] = {"bwd_token_prep", mlstm::launch_bwd_token_prep};
   if (grads && mlstm::bwd_walk_supported(p)) {
-    // one pass per head over its chunks in reverse gives the state gradients, dk and dv
-    st[n++] = {"dkv_walk_tc", mlstm::launch_bwd_walk};
+    // one pass per head over its chunks in reverse gives the state gradients, dk and dv; it
+    // runs on the high-priority side stream with dq alongside, whose CTAs take the SMs the
+    // walker's last wave (one CTA per SM and head) leaves idle
+    st[n++] = {"dkv_walk_tc", mlstm::launch_bwd_walk, true, false};
     st[n++] = {"dq_tc", mlstm::launch_dq_tc};
-    st[n++] = {"gate_grad", mlstm::launch_gate_grad};
+    st[n++] = {"gate_grad", mlstm::launch_gate_grad, false, true};
     return n;
   }
   if (mlstm::state_tc_supported(p))
@@ -199,17 +235,39 @@ int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
 
 template <typename Step, typename Args>
 int run_plan(const Step* steps, int n, const Problem& p, const Args& a, cudaStream_t s) {
+  SideStream* side = nullptr;
+  bool forked = false;
   for (int i = 0; i < n; ++i) {
+    cudaStream_t si = s;
+    if (steps[i].join && forked) {
+      int st = cuda_status(cudaEventRecord(side->join, side->stream), "side join");
+      if (st == MLSTM_OK) st = cuda_status(cudaStreamWaitEvent(s, side->join, 0), "side join");
+      if (st != MLSTM_OK) return st;
+      forked = false;
+    }
+    if (steps[i].side && !g_serial) {
+      int st = cuda_status(side_stream(&side), "side stream");
+      if (st == MLSTM_OK) st = cuda_status(cudaEventRecord(side->fork, s), "side fork");
+      if (st == MLSTM_OK) st = cuda_status(cudaStreamWaitEvent(side->stream, side->fork, 0), "side fork");
+      if (st != MLSTM_OK) return st;
+      si = side->stream;
+      forked = true;
+    }
     if (g_events && 2 * i + 1 < g_nevents) {
-      int st = cuda_status(cudaEventRecord((cudaEvent_t)g_events[2 * i], s), "event record");
+      int st = cuda_status(cudaEventRecord((cudaEvent_t)g_events[2 * i], si), "event record");
       if (st != MLSTM_OK) return st;
     }
-    int st = cuda_status(steps[i].fn(p, a, s), steps[i].name);
+    int st = cuda_status(steps[i].fn(p, a, si), steps[i].name);
     if (st != MLSTM_OK) return st;
     if (g_events && 2 * i + 1 < g_nevents) {
-      st = cuda_status(cudaEventRecord((cudaEvent_t)g_events[2 * i + 1], s), "event record");
+      st = cuda_status(cudaEventRecord((cudaEvent_t)g_events[2 * i + 1], si), "event record");
       if (st != MLSTM_OK) return st;
     }
+  }
+  if (forked) {  // a plan whose side work no later step joined: join at its end
+    int st = cuda_status(cudaEventRecord(side->join, side->stream), "side join");
+    if (st == MLSTM_OK) st = cuda_status(cudaStreamWaitEvent(s, side->join, 0), "side join");
+    if (st != MLSTM_OK) return st;
   }
   return MLSTM_OK;
 }
@@ -276,6 +334,11 @@ const char* mlstm_launch_name(int pass, int index, int B, int NH, int T, int d_q
     return index < n ? steps[index].name : "";
   }
   return "";
+}
+
+int mlstm_set_serial_launches(int serial) {
+  g_serial = serial != 0;
+  return MLSTM_OK;
 }
 
 int mlstm_set_timing_events(void* const* events, int count) {

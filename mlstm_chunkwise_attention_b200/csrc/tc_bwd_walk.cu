@@ -424,11 +424,13 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
     auto epilogue = [&](uint32_t tA, float fin, uint8_t* stg, bool dot) -> float {
       float dsum = 0.f;
       auto one = [&](const uint32_t (&x)[32], int cb) {
+        uint32_t g[32];
+        walk::scale32(x, fin, g);
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
           float gq[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) gq[u] = __uint_as_float(x[e + u]) * fin;
+          for (int u = 0; u < 8; ++u) gq[u] = __uint_as_float(g[e + u]);
           const uint32_t off = sw_off(row, 32 * cb + e);
           if (dot) {
             const uint4 src = *reinterpret_cast<const uint4*>(sK + off);

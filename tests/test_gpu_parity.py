@@ -269,3 +269,19 @@ def test_sweep_igate_bias_minus10():
         for key, val in (("dq", cb["dq"]), ("dk", cb["dk"]), ("dv", cb["dv"]),
                          ("digate_pre", di), ("dfgate_pre", df)):
             assert relerr(np64(g[key][0, 1]), val, floor=floor) <= 1e-2, key
+
+
+@pytest.mark.parametrize("var", [SIG, EXP], ids=["sig", "exp"])
+def test_backward_same_bits_with_serial_launches(var):
+    """The backward walker overlaps dq on a side stream; with every kernel on the caller's
+    stream (mlstm_set_serial_launches) the gradients are bit-identical."""
+    cpu = inputs(2, 3, 777, 128, 128, seed=4242 + var, dtype=BF, ig_mean=-2.0, fg_mean=3.0)
+    dev, h, saved = gpu_fwd(cpu, 128, var)
+    g1 = gpu_bwd(dev, h, saved, 128, var)
+    binding.mlstm_set_serial_launches(True)
+    try:
+        g2 = gpu_bwd(dev, h, saved, 128, var)
+    finally:
+        binding.mlstm_set_serial_launches(False)
+    for key in g1:
+        assert torch.equal(g1[key], g2[key]), key
