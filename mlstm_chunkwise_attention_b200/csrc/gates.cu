@@ -172,7 +172,8 @@ cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s)
 // da_t = -(dh_t . h_t) sign(a~_t) / den_t when |a~_t| > exp(-m_t), else 0
 // (den_t = max(|a~_t|, exp(-m_t)), h_t = num_t / den_t).  Also zeroes the
 // per-token dot-product accumulators.  Groups of LPT lanes own one token and
-// read its rows with 16-byte loads; warps stride over the tokens.
+// read its rows with 16-byte loads, at least two of each row per lane so that
+// several are in flight; warps stride over the tokens.
 // ---------------------------------------------------------------------------
 template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(256) bwd_token_prep_kernel(
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(256) bwd_token_prep_kernel(
     float* __restrict__ pq, float* __restrict__ pk, long long ntok, int dhv) {
   constexpr int VEC = 16 / sizeof(TIO);  // elements per 16-byte load
   const int lane = threadIdx.x & 31;
-  const int lpt = min(32, dhv / VEC);    // lanes per token (a power of two)
+  const int lpt = max(1, min(32, dhv / VEC) / 2);  // lanes per token (a power of two)
   const int tpw = 32 / lpt;              // tokens per warp step
   const int sub = lane / lpt, sl = lane % lpt;
   const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(256) bwd_token_prep_kernel(
     if (EXPV && valid) {
       const TIO* hr = h + tok * dhv;
       const TIO* dr = dh + tok * dhv;
+#pragma unroll 2
       for (int j = sl * VEC; j < dhv; j += lpt * VEC) {
         const uint4 hv = *reinterpret_cast<const uint4*>(hr + j);
         const uint4 dv = *reinterpret_cast<const uint4*>(dr + j);
