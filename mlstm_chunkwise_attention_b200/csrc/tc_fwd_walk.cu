@@ -443,17 +443,18 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
 
     for (int c = 0; c < NC && ok; ++c) {
       if (c > 0) {
-        // the previous chunk's state update is done: C_c is in TMEM, the Q tile is free once
-        // the previous h store has read it
+        // the Q tile is free once the previous h store has read it (the products that read
+        // Q were waited for before that store): its load need not wait for the state update
+        if (issuer) {
+          tc::bulk_wait_read_all();
+          load_q(c);
+        }
+        // the previous chunk's state update is done: C_c is in TMEM
         ok = wait_state();
         if (EXPV) {
           float a, b;
           walk::tmem_ld2(tNU + 16 * ((c - 1) & 1) + lane_base, a, b);
           n += a + b;  // n_c = beta_{c-1} n_{c-1} (scaled below, a chunk ago) + K^T w
-        }
-        if (issuer && ok) {
-          tc::bulk_wait_read_all();
-          load_q(c);
         }
         ok = rows_and(ok);
         if (!ok) break;
@@ -487,6 +488,11 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         tc::tma_store_3d(&tmClo, stg + TILE + 16384, 64, 0, z);
         tc::bulk_commit_group();
       }
+      // ---- the next chunk's gate factors (its key factors in the other buffer, its w as the
+      // n-update operand), while the first products run; written before the hand-over D that
+      // the next n update follows
+      Gates nxtG = cur;
+      if (c + 1 < NC) nxtG = gate_factors(c + 1, nxt);
       // ---- B: P over this half's keys and its row-sum share, the inter term scaled by qfac,
       // q.n
       ok = wait_mma();
@@ -506,10 +512,6 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         tc::bulk_wait_read_all();
         load_kv(c + 1);
       }
-      // ---- the next chunk's gate factors (its key factors in the other buffer, its w as the
-      // n-update operand), before the hand-over D that the next n update follows
-      Gates nxtG = cur;
-      if (c + 1 < NC) nxtG = gate_factors(c + 1, nxt);
       // ---- D: w K (hi plane over K, lo plane apart): the score, inter and n-update products
       // that read K are done (waited for above)
       if (c + 1 < NC) {
