@@ -60,7 +60,9 @@ struct WalkCfg {
 };
 
 // per-token factor arrays in the OFF_F region (token t of the chunk, or state row j)
-enum { F_PC = 0, F_PE, F_WV, F_DN, F_DOT };
+// (the partner factors and state-update weights of the chunk with walk index it are in
+// buffer it & 1: the next chunk's are written while this chunk's are still read)
+enum { F_PC0 = 0, F_PC1, F_PE0, F_PE1, F_WV0, F_WV1, F_DN, F_DOT };
 // mbarriers: tile loads (one per tile); rows -> MMA thread (hand-overs A, B, C; and D on
 // its own barrier, since the rows signal C and D back to back); MMA thread -> rows (the
 // products after A, B, C; and the state update on its own barrier, which can complete
@@ -289,11 +291,12 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       if (EXPV) G.beta = (c > 0 || P.m0 != nullptr) ? expf(I.g + I.mprev - I.mc) : 0.f;
       else G.beta = expf(I.g);
       if (!lead) return G;
-      F[F_PC * 128 + row] = in ? (I.bt - I.mt) * kLog2e + log2f(I.invd) : -INFINITY;
-      F[F_PE * 128 + row] = (EXPV && in) ? I.dat / I.invd : 0.f;
+      const int fb = (NC - 1 - c) & 1;
+      F[(F_PC0 + fb) * 128 + row] = in ? (I.bt - I.mt) * kLog2e + log2f(I.invd) : -INFINITY;
+      F[(F_PE0 + fb) * 128 + row] = (EXPV && in) ? I.dat / I.invd : 0.f;
       // exp(-inf) = 0 in the first chunk of an mLSTMexp sequence without an initial state
       const float alpha = in ? expf(I.bt + I.mprev - I.mt) * P.scale : 0.f;
-      F[F_WV * 128 + row] = alpha * I.invd;
+      F[(F_WV0 + fb) * 128 + row] = alpha * I.invd;
       if (EXPV) {
         const float wn = alpha * I.dat;
         const bf16 hi = __float2bfloat16_rn(wn);
@@ -350,7 +353,8 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
     // the dk and dv kernels of tc_bwd.cu on a diagonal tile: sub-blocks left of the
     // diagonal are zero, the diagonal one takes every element's own exponent and the
     // causal mask, the others the separable form ((x + e) f_t) g_s.
-    auto transform = [&](bool is_dk, float R) {
+    auto transform = [&](bool is_dk, float R, int fb) {
+      const float* pc = F + (F_PC0 + fb) * 128;
       float mx = R;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, o));
@@ -359,10 +363,9 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       float* fw = fwv + (warp - 1) * 128;
       __syncwarp();
 #pragma unroll
-      for (int u = cb0; u < cb0 + 2; ++u) fw[lane + 32 * u] = tc::ex2(F[F_PC * 128 + lane + 32 * u] + Mrow);
+      for (int u = cb0; u < cb0 + 2; ++u) fw[lane + 32 * u] = tc::ex2(pc[lane + 32 * u] + Mrow);
       __syncwarp();
-      const float* pc = F + F_PC * 128;
-      const float* pe = F + F_PE * 128;
+      const float* pe = F + (F_PE0 + fb) * 128;
       const int wb = warp & 3;
       auto one = [&](const uint32_t (&xr)[32], int ch) {
         uint32_t pk[16];
@@ -532,6 +535,9 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       stage_dc(cur.beta);
       if (EXPV) dn *= cur.beta;
       signal(BW_R);
+      // the next chunk's gate factors (the other factor buffer) while the first products run
+      Gates nxtG = cur;
+      if (c > 0) nxtG = gate_factors(c - 1, nxt);
       // row-side factors of this key row (the dk and dv kernels' conventions)
       float rs_v = 0.f, rs_k = 0.f, Rk = -INFINITY, Rv = -INFINITY;
       if (valid) {
@@ -543,18 +549,18 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       // ---- B: dv inter rescaled, dv transform
       ok = wait_mma();
       rescale(tAV, rs_v, false);
-      transform(false, Rv);
+      transform(false, Rv, it & 1);
       signal(BW_R);
       // ---- C: dk inter rescaled (+ dn_c), dk transform
       ok = wait_mma() && ok;
       rescale(tAK, rs_k, true);
-      transform(true, Rk);
+      transform(true, Rk, it & 1);
       signal(BW_R);
       // ---- D: u dH, hi plane over dH and lo plane over dC's lo plane (their products are
       // done), so the state update runs while the outputs are written
       const bool update = c > 0 || P.d0 != nullptr;
       if (update) {
-        const float wv = F[F_WV * 128 + row];
+        const float wv = F[(F_WV0 + (it & 1)) * 128 + row];
 #pragma unroll 4
         for (int col = 64 * half; col < 64 * half + 64; col += 8) {
           const uint32_t off = sw_off(row, col);
@@ -599,11 +605,7 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
           load_tile(BW_V, sV, &tmV, c - 1);
         }
       }
-      // ---- the next chunk's gate factors, while the state update runs
-      if (c > 0) {
-        cur = gate_factors(c - 1, nxt);
-        ok = rows_and(ok);
-      }
+      cur = nxtG;
     }
     // the last state update
     if (ok) ok = wait_state();
