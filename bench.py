@@ -351,8 +351,11 @@ def run_sweep(args):
                 kms = {n: sum(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs) / args.steps
                        for i, n in enumerate(names)}
                 flops = B * NH * flops_fwd(T, d, d, L)
-                out_name = [n for n in names if n.startswith("output_fwd")][0]
-                out_fl = B * NH * kernel_costs(T, d, d, L, var == 1, 2)["output_fwd"][0]
+                # the output kernel, or the forward walker (states and outputs in one pass,
+                # counted with the state products)
+                out_name = [n for n in names if n.startswith(("output_fwd", "fwd_walk"))][0]
+                role = "fwd_walk" if out_name.startswith("fwd_walk") else "output_fwd"
+                out_fl = B * NH * kernel_costs(T, d, d, L, var == 1, 2)[role][0]
                 line = {
                     "sweep": f"fwd_b{B}h32_d128", "cell": label, "T": T, "chunk": L,
                     "ms": ms, "tflops": flops / ms / 1e9, "tokens_per_s": B * T / ms * 1e3,
