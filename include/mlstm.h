@@ -116,7 +116,9 @@ size_t mlstm_bwd_workspace_size(int B, int NH, int T, int d_qk, int d_hv,
  * those of the chunkwise form: gate preprocessing, the inter-chunk state
  * recurrence, then the tiled intra-chunk outputs fused with the inter-chunk
  * term q' C_prev and the normaliser (TFLA summary page, Approach; arXiv
- * abstract page, Abstract). */
+ * abstract page, Abstract).  On the bf16 path with chunk 128 and d_qk = d_hv
+ * = 128 the recurrence and the outputs run in one kernel that carries each
+ * head's state through its chunks on chip; the saved regions are the same. */
 int mlstm_fwd(const void* q, const void* k, const void* v,
               const void* igate_pre, const void* fgate_pre,
               void* h, void* saved,

@@ -51,6 +51,9 @@ SMALL = [
     ("exp_bf16_chunk128_d128_ragged", 2, 2, 700, 128, 128, 128, EXP, BF, -2.0, 3.0),
     ("sig_bf16_chunk128_d128_ragged", 1, 3, 1000, 128, 128, 128, SIG, BF, 0.0, 3.0),
     ("exp_bf16_chunk128_d128_one_partial", 1, 2, 77, 128, 128, 128, EXP, BF, 0.0, 3.0),
+    ("exp_bf16_chunk128_d128_t1", 1, 2, 1, 128, 128, 128, EXP, BF, -1.0, 3.0),
+    ("sig_bf16_chunk128_d128_t128_one_full", 1, 2, 128, 128, 128, 128, SIG, BF, 0.0, 3.0),
+    ("exp_bf16_chunk128_d128_t129_one_token_tail", 2, 1, 129, 128, 128, 128, EXP, BF, -2.0, 3.0),
 ]
 
 
