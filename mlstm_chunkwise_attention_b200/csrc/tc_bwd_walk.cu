@@ -14,11 +14,12 @@
 // Roles: one thread (warp 0) issues the MMAs; eight row warps transform, rescale
 // and store, two per TMEM lane quarter: a thread owns one key row, token row or
 // state row (its TMEM lane) and one half of the columns.  One row thread issues
-// the TMA loads and stores.  Rows and MMA thread hand over
-// through two mbarriers, so work that does not feed the next product (the dv and
-// dk epilogues, the next chunk's gate factors) runs while the tensor core works:
-//   rows: stage dC -> A | rescale dv inter, dv transform -> B | rescale dk inter,
-//         dk transform -> C | u dH, dn increment -> D | dv out | dk out | next gates
+// the TMA loads and stores.  Rows and MMA thread hand over through mbarriers
+// (four hand-overs each way per chunk), so work that does not feed the next product
+// (the next chunk's gate factors, the dv and dk epilogues) runs while the tensor
+// core works:
+//   rows: stage dC -> A, next gates | rescale dv inter, dv transform -> B | rescale
+//         dk inter, dk transform -> C | u dH, dn increment -> D | dv out | dk out
 //   MMA:  K Q^T (dv score) | A: K dC (dv inter) | V dC^T (dk inter) | B: Y dH (dv),
 //         V dH^T (dk score) | C: Y Q (dk), Q^T wn (dn increment) | D: dC += Q^T (u dH)
 // The next chunk's K and V tiles load as soon as their buffers are free, Q and
@@ -43,7 +44,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 //   V: v, then the dv staging tile;  H: dh, then u dH (hi plane);
 //   G: dC hi plane, then the dk staging tile;  G + TILE: dC lo plane, then u dH lo.
 struct WalkCfg {
-  static constexpr int TILE = 32768;
+  static constexpr int TILE = walk::TILE;
   static constexpr int OFF_Q = 0, OFF_K = TILE, OFF_V = 2 * TILE, OFF_H = 3 * TILE;
   static constexpr int OFF_G = 4 * TILE;
   static constexpr int OFF_F = 6 * TILE;              // per-token factors, NF arrays of 128 floats

@@ -20,12 +20,13 @@
 // Roles: one thread (warp 0) issues the MMAs; eight row warps, two per TMEM lane
 // quarter, each own one token or state row (the TMEM lane) and half of its
 // columns; one row thread issues the TMA loads and stores.  Hand-overs:
-//   rows: stage C_c -> A | P transform, inter rescale -> B | w K -> D | h out,
-//         next gate factors
+//   rows: stage C_c -> A, next gate factors | P transform, inter rescale -> B |
+//         w K -> D | h out
 //   MMA:  Q K^T, K^T w (hi, lo) | A: Q C_c (hi), Q n_c (hi, lo) | B: P V |
 //         D: C += (w K)^T V (hi, lo)
-// The next chunk's gate factors (and w as the n-update operand) are written before the
-// hand-over D, so the n update can start as soon as the next chunk's tiles land.
+// The next chunk's gate factors (and w as the n-update operand) are written while the
+// first products run, before the hand-over D, so the next chunk's n update can start as
+// soon as its tiles land.
 // Two K/V buffer sets alternate between chunks; the set a chunk does not use
 // holds its C staging, and takes the next chunk's K and V as soon as the inter
 // product and the saved-state store have read it.  Every wait is bounded; on a
