@@ -215,3 +215,25 @@ def test_backward_chain_argument_errors(lib):
     # some but not all of the five outputs
     assert lib.mlstm_bwd_state(*ins, None, c, None, d, None, None, None, None, b, 1 << 30,
                                *sizes, None) == B.STATUS_INVALID
+
+
+def _plan(pass_, sizes):
+    n = (B.mlstm_fwd_launch_count if pass_ == 0 else B.mlstm_bwd_launch_count)(*sizes)
+    return [B.mlstm_launch_name(pass_, i, *sizes) for i in range(n)]
+
+
+@pytest.mark.parametrize("variant", [B.SIG, B.EXP], ids=["sig", "exp"])
+def test_launch_plans_choose_the_walkers_on_their_shape(lib, variant):
+    """bf16, chunk 128, d_qk = d_hv = 128: the forward walker replaces the state and output
+    kernels, the backward walker the state-gradient, dk and dv kernels (dq stays); any other
+    chunk, head dim or dtype keeps the separate kernels."""
+    walk = (2, 4, 1000, 128, 128, 128, variant, B.BF16)
+    assert _plan(0, walk) == ["gate_prep", "fwd_walk_tc"]
+    assert _plan(1, walk) == ["bwd_token_prep", "dkv_walk_tc", "dq_tc", "gate_grad"]
+    for other in [(2, 4, 1000, 128, 128, 256, variant, B.BF16),
+                  (2, 4, 1000, 64, 128, 128, variant, B.BF16),
+                  (2, 4, 1000, 128, 256, 128, variant, B.BF16),
+                  (2, 4, 1000, 128, 128, 128, variant, B.FP32)]:
+        names = _plan(0, other) + _plan(1, other)
+        assert not any("walk" in n for n in names), (other, names)
+        assert any(n.startswith("state_fwd") for n in names) and any(n.startswith("dk_") for n in names)
