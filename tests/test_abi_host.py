@@ -237,3 +237,11 @@ def test_launch_plans_choose_the_walkers_on_their_shape(lib, variant):
         names = _plan(0, other) + _plan(1, other)
         assert not any("walk" in n for n in names), (other, names)
         assert any(n.startswith("state_fwd") for n in names) and any(n.startswith("dk_") for n in names)
+
+
+def test_serial_launch_switch_needs_no_device(lib):
+    """mlstm_set_serial_launches only sets a per-thread flag: no CUDA call, always MLSTM_OK."""
+    assert lib.mlstm_set_serial_launches(1) == 0
+    assert lib.mlstm_set_serial_launches(0) == 0
+    assert lib.mlstm_set_serial_launches(7) == 0
+    assert lib.mlstm_set_serial_launches(0) == 0
