@@ -391,18 +391,18 @@ def run_retnet(args):
     """
     import torch
     from mlstm_chunkwise_attention_b200 import binding
-    from mlstm_chunkwise_attention_b200.synthetic import make_inputs
+    from mlstm_chunkwise_attention_b200.synthetic import make_inputs, retention_gates, retnet_decays
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
     B, NH, d = 8, 32, 128
-    gamma = binding.retnet_decays(NH)
+    gamma = retnet_decays(NH)
     Ts = [int(t) for t in args.sweep_t.split(",")] if args.sweep_t else sorted(RETNET_A100_MS)
     for T in Ts:
         cpu = make_inputs(B, NH, T, d, d, seed=11, igate_mean=0.0, fgate_mean=3.0,
                           dtype=torch.bfloat16, with_dh=True)
         x = {k: v.to(dev) for k, v in cpu.items()}
         del cpu
-        ig, fg, _ = binding.retention_gates(gamma, B, T, torch.bfloat16, dev)
+        ig, fg = retention_gates(gamma, B, T, torch.bfloat16, dev)
         best = {}
         for L in [c for c in (128, 256, 512, 1024) if c <= max(T, 128)]:
             def fwd():

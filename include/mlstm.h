@@ -158,8 +158,15 @@ int mlstm_bwd(const void* q, const void* k, const void* v,
  * 32 MiB return MLSTM_ERR_WORKSPACE before any launch; no saved state is kept,
  * so there is no backward from this entry point.  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture.  It calls no
- * cudaMalloc or cudaFree.  All calls share the one array, so calls whose
+ * current.  Under CUDA's default lazy module loading, that lookup is what
+ * places the 32 MiB array on the device, and the first launch of each kernel
+ * loads that kernel's code; either may allocate device memory and synchronise.
+ * So make one warm-up call with the same sizes, variant and dtype on each
+ * device before any region that must not allocate and before any stream
+ * capture.  After it, calls of that configuration allocate nothing: the entry
+ * point calls no cudaMalloc, cudaFree or allocating library routine.  The
+ * cached address is per device ordinal and is not refreshed after
+ * cudaDeviceReset.  All calls share the one array, so calls whose
  * kernels overlap on the GPU (different streams, or different host threads)
  * race on it: serialise them. */
 int mlstm_fwd_noalloc(const void* q, const void* k, const void* v,
@@ -309,11 +316,27 @@ int mlstm_dstate_chain(const void* dstate_local, const void* dstate_out, const v
                        int NH, int d_qk, int d_hv, int variant, void* stream);
 
 
-/* Synchronise `stream` and report what the kernels enqueued so far found:
- * MLSTM_ERR_TIMEOUT if one of them gave up a bounded wait (its outputs are
- * then invalid; the flag is cleared by this call), MLSTM_ERR_CUDA on a CUDA
- * error, else MLSTM_OK.  This is the one call that blocks. */
+/* Synchronise `stream` and report what the kernels of this device found:
+ * MLSTM_ERR_TIMEOUT if a tensor-core kernel launched on the current device
+ * gave up a bounded wait (2 s) since the previous mlstm_device_status call on
+ * that device (the outputs of that launch are invalid), MLSTM_ERR_CUDA on a
+ * CUDA error, else MLSTM_OK.  Each failure is reported once.  A failure stays
+ * within its own launch: each launch carries its own abort epoch, so the
+ * launches after a failed one run normally whether or not this call is made
+ * in between.  The call reads the kernels' failure flags without clearing
+ * them, so it does not disturb kernels running on other streams; a failure of
+ * a launch on another stream of the same device is reported too.  This is the
+ * one call that blocks. */
 int mlstm_device_status(void* stream);
+
+/* Self-test of the failure report: enqueue one tiny kernel whose bounded wait
+ * (on a barrier that nothing completes) runs out after 2 s, as a tensor-core
+ * kernel's wait would if a hand-over never came.  The kernel then raises its
+ * launch's failure flag and returns; it faults nothing and the context stays
+ * usable.  The next mlstm_device_status on this device returns
+ * MLSTM_ERR_TIMEOUT.  Not part of the mLSTM computation (the pages have no
+ * counterpart); for tests of the error path. */
+int mlstm_selftest_timeout(void* stream);
 
 /* Static text for a status code. */
 const char* mlstm_status_string(int status);

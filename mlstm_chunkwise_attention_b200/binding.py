@@ -59,6 +59,7 @@ EXPORTS = {
     "mlstm_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     "mlstm_set_serial_launches": (ctypes.c_int, [ctypes.c_int]),
     "mlstm_device_status": (ctypes.c_int, [_P]),
+    "mlstm_selftest_timeout": (ctypes.c_int, [_P]),
     "mlstm_fwd_noalloc": (ctypes.c_int, [_P] * 6 + _SIZES + [_P]),
     "mlstm_state_size": (ctypes.c_size_t, [ctypes.c_int] * 5),
     "mlstm_state_zero": (ctypes.c_int, [_P] + [ctypes.c_int] * 5 + [_P]),
@@ -164,6 +165,10 @@ def mlstm_status_string(status):
 
 def mlstm_device_status(stream=None):
     return load().mlstm_device_status(stream)
+
+
+def mlstm_selftest_timeout(stream=None):
+    return load().mlstm_selftest_timeout(stream)
 
 
 def check_device(stream=None):
@@ -464,51 +469,6 @@ def step(q, k, v, igate_pre, fgate_pre, state_in, state_out, variant, *, h=None,
     if st != STATUS_OK:
         raise MLSTMError(st, "mlstm_step")
     return h
-
-
-# ---------------------------------------------------------------------------
-# Retention (RetNet): a constant per-head decay through the SIG kernels
-# ---------------------------------------------------------------------------
-
-#: input-gate preactivation that makes log sigmoid(i~) = 0 to fp32 rounding
-RETENTION_IGATE = 30.0
-
-
-def retnet_decays(num_heads):
-    """RetNet's per-head decay schedule gamma_h = 1 - 2^(-5 - h)."""
-    import torch
-    return 1.0 - torch.pow(2.0, -5.0 - torch.arange(num_heads, dtype=torch.float64))
-
-
-def retention_gates(gamma, B, T, dtype, device):
-    """Gate preactivations that turn mLSTMsig into retention.
-
-    With i~ = RETENTION_IGATE and f~_h = logit(gamma_h), the SIG cell computes
-    h_t = sum_{s <= t} gamma_h^(t - s) (q_t . k_s / sqrt(d_qk)) v_s.  The
-    preactivations are stored in the I/O dtype, so the decay actually applied
-    is sigmoid(dtype(logit gamma_h)); it is returned as ``gamma_eff`` (fp64,
-    per head).
-    """
-    import torch
-    g = torch.as_tensor(gamma, dtype=torch.float64).cpu()
-    NH = g.numel()
-    fg_h = (torch.log(g) - torch.log1p(-g)).to(dtype)
-    gamma_eff = torch.sigmoid(fg_h.double())
-    fg = fg_h.view(1, NH, 1).expand(B, NH, T).contiguous().to(device)
-    ig = torch.full((B, NH, T), RETENTION_IGATE, dtype=dtype, device=device)
-    return ig, fg, gamma_eff
-
-
-def retention(q, k, v, gamma, chunk, *, keep_saved=False, stream=None):
-    """RetNet retention with decay gamma[h] per head, on the mLSTMsig kernels.
-
-    Returns (h, saved, gates); ``gates`` = (igate_pre, fgate_pre, gamma_eff),
-    which ``backward`` needs together with ``saved`` (keep_saved=True).
-    """
-    B, NH, T, _ = q.shape
-    ig, fg, gamma_eff = retention_gates(gamma, B, T, q.dtype, q.device)
-    h, saved = forward(q, k, v, ig, fg, chunk, SIG, keep_saved=keep_saved, stream=stream)
-    return h, saved, (ig, fg, gamma_eff)
 
 
 def saved_views(saved, q, v, chunk, variant):

@@ -90,12 +90,19 @@ cudaError_t launch_dq_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dk_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dv_simt(const Problem& p, const BwdArgs& a, cudaStream_t s);
 
+// Abort epoch for the next launch of a tensor-core kernel: a process-wide launch
+// counter, never 0 (see tc::Abort).  Each kernel family keeps a device flag that
+// holds the epoch of its last launch that gave up; fetch_tc_*_error read it
+// without clearing it.
+unsigned int next_epoch();
+
 // tensor-core kernels (tc_*.cu) and their host helpers (tmap.cu)
 bool make_tmap_3d_bf16(void* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
                        uint32_t box_inner, uint32_t box_mid);
 bool output_fwd_tc_supported(const Problem& p);
 cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_fwd_error(unsigned int* flag);
+cudaError_t launch_selftest_timeout(cudaStream_t s);
 bool output_fwd_xl_supported(const Problem& p);
 cudaError_t launch_output_fwd_xl(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_fwd_xl_error(unsigned int* flag);

@@ -5,6 +5,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "internal.h"
 #include "mlstm.h"
 
@@ -273,6 +276,17 @@ int run_plan(const Step* steps, int n, const Problem& p, const Args& a, cudaStre
 }
 
 }  // namespace
+
+namespace mlstm {
+
+unsigned int next_epoch() {
+  static std::atomic<unsigned int> counter{0};
+  unsigned int e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+  while (e == 0u) e = counter.fetch_add(1, std::memory_order_relaxed) + 1;  // 0 means "no failure"
+  return e;
+}
+
+}  // namespace mlstm
 
 extern "C" {
 
@@ -706,28 +720,54 @@ const char* mlstm_status_string(int status) {
 
 const char* mlstm_last_error(void) { return g_last_error; }
 
+}  // extern "C"
+
+namespace {
+// Failures already reported, per device and kernel family: the flag values
+// mlstm_device_status saw last.  A flag holds the epoch of the last launch of
+// its family that gave up, so a value that differs from the last one seen is a
+// failure not yet reported.
+constexpr int kFlagDevices = 64, kFlagFamilies = 6;
+std::mutex g_flag_mu;
+unsigned int g_flag_seen[kFlagDevices][kFlagFamilies] = {};
+}  // namespace
+
+extern "C" {
+
 int mlstm_device_status(void* stream) {
   int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
   if (st != MLSTM_OK) return st;
-  unsigned int flag = 0, flag_bwd = 0, flag_state = 0, flag_xl = 0, flag_walk = 0, flag_fwalk = 0;
-  st = cuda_status(mlstm::fetch_tc_fwd_error(&flag), "device error flag");
+  int dev = 0;
+  st = cuda_status(cudaGetDevice(&dev), "device");
   if (st != MLSTM_OK) return st;
-  st = cuda_status(mlstm::fetch_tc_bwd_error(&flag_bwd), "device error flag");
-  if (st != MLSTM_OK) return st;
-  st = cuda_status(mlstm::fetch_tc_state_error(&flag_state), "device error flag");
-  if (st != MLSTM_OK) return st;
-  st = cuda_status(mlstm::fetch_tc_fwd_xl_error(&flag_xl), "device error flag");
-  if (st != MLSTM_OK) return st;
-  st = cuda_status(mlstm::fetch_tc_walk_error(&flag_walk), "device error flag");
-  if (st != MLSTM_OK) return st;
-  st = cuda_status(mlstm::fetch_tc_fwalk_error(&flag_fwalk), "device error flag");
-  if (st != MLSTM_OK) return st;
-  flag |= flag_bwd | flag_state | flag_xl | flag_walk | flag_fwalk;
-  if (flag) {
+  if (dev < 0 || dev >= kFlagDevices) return MLSTM_ERR_UNSUPPORTED;
+  // read every flag before deciding anything; nothing is cleared
+  typedef cudaError_t (*Fetch)(unsigned int*);
+  const Fetch fetch[kFlagFamilies] = {mlstm::fetch_tc_fwd_error,    mlstm::fetch_tc_bwd_error,
+                                      mlstm::fetch_tc_state_error,  mlstm::fetch_tc_fwd_xl_error,
+                                      mlstm::fetch_tc_walk_error,   mlstm::fetch_tc_fwalk_error};
+  unsigned int flag[kFlagFamilies] = {};
+  for (int i = 0; i < kFlagFamilies; ++i) {
+    st = cuda_status(fetch[i](&flag[i]), "device error flag");
+    if (st != MLSTM_OK) return st;
+  }
+  bool fresh = false;
+  {
+    std::lock_guard<std::mutex> lock(g_flag_mu);
+    for (int i = 0; i < kFlagFamilies; ++i) {
+      if (flag[i] != g_flag_seen[dev][i]) fresh = true;
+      g_flag_seen[dev][i] = flag[i];
+    }
+  }
+  if (fresh) {
     snprintf(g_last_error, sizeof(g_last_error), "a tensor-core kernel timed out waiting");
     return MLSTM_ERR_TIMEOUT;
   }
   return MLSTM_OK;
+}
+
+int mlstm_selftest_timeout(void* stream) {
+  return cuda_status(mlstm::launch_selftest_timeout((cudaStream_t)stream), "selftest_timeout");
 }
 
 }  // extern "C"

@@ -80,6 +80,7 @@ struct BwdTcParams {
   bool dfin;                               // the final state has a gradient (dk, dv)
   const float* m0;                         // its max state (mLSTMexp), else null
   float scale, log2_scale;
+  unsigned int epoch;  // this launch's abort epoch
 };
 
 template <int KIND, int D1, int D2S, bool G_MN, bool EXPV, int NXBUF>
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     const __grid_constant__ CUtensorMap tmGlo, const __grid_constant__ CUtensorMap tmOut,
     const BwdTcParams P) {
   using Cfg = BwdTcCfg<D1, D2S, G_MN, NXBUF>;
+  const tc::Abort abort_flag{&g_tc_bwd_error, P.epoch};
   constexpr bool R_IS_QUERY = (KIND == KDQ);
   constexpr int ST = Cfg::STAGES;
 
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   const int r0 = it_tile * 128;
   if (r0 >= len) return;
   // an earlier CTA gave up: the whole block leaves together
-  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_bwd_error != 0u)) return;
+  if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
   const int col0 = slice * D2S;
   const size_t tok0 = (size_t)bh * P.T + c0;
   // partner tiles: dq: 0..it_tile; dk, dv: it_tile..nt_len-1
@@ -127,7 +129,6 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   float* pfE = pfC + P.L;  // partner additive term (dk) or separable key factor (dq)
   float* pfM = pfE + P.L;  // dq: stabiliser of every 32-key partner block
   float* pfW = reinterpret_cast<float*>(smem + Cfg::OFF_PW);  // dk, dv: this warp's partner factors
-  const volatile unsigned int* abort_flag = &g_tc_bwd_error;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -573,7 +574,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     }
   }
 
-  if (!ok) atomicOr(&g_tc_bwd_error, 1u);
+  if (!ok) abort_flag.raise();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -640,6 +641,7 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   P.dqk = p.dqk;
   P.scale = p.scale;
   P.log2_scale = log2f(p.scale);
+  P.epoch = next_epoch();
   const size_t smem = Cfg::smem_bytes(p.L);
   auto kern = intra_bwd_tc_kernel<KIND, D1, D2S, G_MN, EXPV, NXBUF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -686,10 +688,7 @@ cudaError_t launch_dv_tc(const Problem& p, const BwdArgs& a, cudaStream_t s) {
 }
 
 cudaError_t fetch_tc_bwd_error(unsigned int* flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_bwd_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_bwd_error, &zero, sizeof(unsigned int));
+  return cudaMemcpyFromSymbol(flag, g_tc_bwd_error, sizeof(unsigned int));
 }
 
 }  // namespace mlstm

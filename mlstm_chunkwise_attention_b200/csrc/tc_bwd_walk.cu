@@ -85,6 +85,7 @@ struct WalkParams {
   float *d0, *dn0;         // gradient of the initial state, or null
   int T, NC;
   float scale, log2_scale;
+  unsigned int epoch;  // this launch's abort epoch
 };
 
 template <bool EXPV>
@@ -94,7 +95,8 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
     const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
     const WalkParams P) {
   using Cfg = WalkCfg;
-  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_walk_error != 0u)) return;
+  const tc::Abort abort_flag{&g_tc_walk_error, P.epoch};
+  if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
   const int bh = blockIdx.x;
   const int NC = P.NC;
   extern __shared__ uint8_t smem_raw[];
@@ -106,7 +108,6 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
   float* fwv = reinterpret_cast<float*>(smem + Cfg::OFF_W);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
-  const volatile unsigned int* abort_flag = &g_tc_walk_error;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
         }
         tc::tc_commit(&bar[BW_S]);
       }
-      if (!ok) atomicOr(&g_tc_walk_error, 1u);
+      if (!ok) abort_flag.raise();
     }
   } else {
     // ------------------------------------------------------------ rows
@@ -229,14 +230,14 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
     auto wait_mma = [&]() -> bool {
       const bool w = __all_sync(full, tc::mbar_wait(&bar[BW_M], nm & 1, abort_flag));
       ++nm;
-      if (!w && lane == 0) atomicOr(&g_tc_walk_error, 1u);
+      if (!w && lane == 0) abort_flag.raise();
       tc::tc_fence_after();
       return w;
     };
     auto wait_state = [&]() -> bool {
       const bool w = __all_sync(full, tc::mbar_wait(&bar[BW_S], ns & 1, abort_flag));
       ++ns;
-      if (!w && lane == 0) atomicOr(&g_tc_walk_error, 1u);
+      if (!w && lane == 0) abort_flag.raise();
       tc::tc_fence_after();
       return w;
     };
@@ -621,7 +622,7 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       if (EXPV && lead) P.dn0[(size_t)bh * 128 + row] = dn;
     }
     if (issuer) tc::bulk_wait_all();
-    if (!ok) atomicOr(&g_tc_walk_error, 1u);
+    if (!ok) abort_flag.raise();
   }
 
   tc::tc_fence_before();
@@ -660,6 +661,7 @@ static cudaError_t launch_walk(const Problem& p, const BwdArgs& a, cudaStream_t 
   P.T = p.T; P.NC = p.NC;
   P.scale = p.scale;
   P.log2_scale = log2f(p.scale);
+  P.epoch = next_epoch();
   auto kern = bwd_walk_kernel<EXPV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)WalkCfg::SMEM);
@@ -673,10 +675,7 @@ cudaError_t launch_bwd_walk(const Problem& p, const BwdArgs& a, cudaStream_t s) 
 }
 
 cudaError_t fetch_tc_walk_error(unsigned int* flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_walk_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_walk_error, &zero, sizeof(unsigned int));
+  return cudaMemcpyFromSymbol(flag, g_tc_walk_error, sizeof(unsigned int));
 }
 
 }  // namespace mlstm

@@ -62,22 +62,49 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The abort state of one kernel launch.  Every launch of a tensor-core kernel
+// gets an epoch from the host (a launch counter, never 0).  A CTA that gives
+// up writes its launch's epoch into its kernel family's flag; waits give up
+// early, and CTAs that start later skip their work, only while the flag holds
+// their own launch's epoch.  A failed launch therefore never silences a later
+// one, and nobody has to clear the flag: the host reads it to report the
+// failure (mlstm_device_status).
+struct Abort {
+  unsigned int* flag;
+  unsigned int epoch;
+  __device__ __forceinline__ bool raised() const {
+    return *reinterpret_cast<volatile unsigned int*>(flag) == epoch;
+  }
+  __device__ __forceinline__ void raise() const { atomicExch(flag, epoch); }
+};
+
 // Wait for the phase with the given parity to complete.  Returns false on
-// timeout, or early when *abort (a kernel's error flag) has been raised by any
+// timeout, or early when this launch's abort flag has been raised by any
 // thread of the grid, so one stuck CTA does not make every other CTA wait out
 // its own timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile unsigned int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1; i != 0; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {
-      if (*abort != 0u) return false;
+      if (abort.raised()) return false;
       if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
     }
   }
   return false;
+}
+
+// Wind-down after a failure: wait, for at most kDrainTimeoutNs and whatever the
+// abort flag says, for a phase that copies or products this thread issued
+// complete, so they do not land in shared memory or TMEM after the CTA has
+// freed them.  Returns false if the phase did not complete in time.
+constexpr uint64_t kDrainTimeoutNs = 20000000ull;
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() - t0 > kDrainTimeoutNs) return false;
+  return true;
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

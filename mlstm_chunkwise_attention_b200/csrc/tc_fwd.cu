@@ -69,8 +69,9 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_h, const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
     const float* __restrict__ gn, bf16* __restrict__ h, float* __restrict__ abar_out, int T, int L,
     int NC, int BH, int ntq, int dhv, float scale, float log2_scale, bool has_init,
-    const float* __restrict__ m0) {
+    const float* __restrict__ m0, unsigned int epoch) {
   using Cfg = OutTcCfg<DQK, DV, ALIAS>;
+  const tc::Abort abort_flag{&g_tc_fwd_error, epoch};
   constexpr int BM = Cfg::BM, BN = Cfg::BN;
 
   const int per = BH * NC;
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
   const int t0 = qt * BM;
   if (t0 >= len) return;
   // an earlier CTA gave up: the whole block leaves together
-  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_fwd_error != 0u)) return;
+  if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
   const int nkv = qt + 1;
   const int dv0 = blockIdx.y * DV;
   const size_t tok0 = (size_t)bh * T + c0;
@@ -139,12 +140,12 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       for (int kb = 0; kb < Cfg::KB; ++kb)
         tc::tma_load_3d(sQ + kb * 16384, &tm_q, &bar[B_Q], kb * 64, c0 + t0, bh);
       for (int j = 0; j < nkv && ok; ++j) {
-        if (j > 0) ok = tc::mbar_wait(&bar[B_S], (j - 1) & 1, &g_tc_fwd_error);  // K buffer free
+        if (j > 0) ok = tc::mbar_wait(&bar[B_S], (j - 1) & 1, abort_flag);  // K buffer free
         if (!ok) break;
         tc::mbar_arrive_expect_tx(&bar[B_K], Cfg::K_BYTES);
         for (int kb = 0; kb < Cfg::KB; ++kb)
           tc::tma_load_3d(sKC + kb * 16384, &tm_k, &bar[B_K], kb * 64, c0 + j * BN, bh);
-        if (j > 0) ok = tc::mbar_wait(&bar[B_PV], (j - 1) & 1, &g_tc_fwd_error);  // V buffer free
+        if (j > 0) ok = tc::mbar_wait(&bar[B_PV], (j - 1) & 1, abort_flag);  // V buffer free
         if (!ok) break;
         tc::mbar_arrive_expect_tx(&bar[B_V], Cfg::V_BYTES);
         for (int vb = 0; vb < Cfg::VB; ++vb)
@@ -152,8 +153,8 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       }
       if (ok && has_prev) {
         // C goes where K was once the last S is done, or (ALIAS) where V was once PV is done
-        ok = ALIAS ? tc::mbar_wait(&bar[B_PV], (nkv - 1) & 1, &g_tc_fwd_error)
-                   : tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, &g_tc_fwd_error);
+        ok = ALIAS ? tc::mbar_wait(&bar[B_PV], (nkv - 1) & 1, abort_flag)
+                   : tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, abort_flag);
         if (ok) {
           tc::mbar_arrive_expect_tx(&bar[B_C], Cfg::C_BYTES);
           for (int vb = 0; vb < Cfg::VB; ++vb)
@@ -162,8 +163,8 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       }
       // do not leave while a copy this thread issued may still be landing
       if (ok) {
-        ok = tc::mbar_wait(&bar[B_V], (nkv - 1) & 1, &g_tc_fwd_error);
-        if (ok && has_prev) ok = tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
+        ok = tc::mbar_wait(&bar[B_V], (nkv - 1) & 1, abort_flag);
+        if (ok && has_prev) ok = tc::mbar_wait(&bar[B_C], 0, abort_flag);
       }
     }
   } else if (warp == 1) {
@@ -173,9 +174,9 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       constexpr uint32_t idO = tc::idesc_bf16(BM, DV, false, true);
       const uint32_t aQ = tc::smem_u32(sQ), aKC = tc::smem_u32(sKC), aV = tc::smem_u32(sV),
                      aP = tc::smem_u32(sP), aC = tc::smem_u32(sC);
-      ok = tc::mbar_wait(&bar[B_Q], 0, &g_tc_fwd_error);
+      ok = tc::mbar_wait(&bar[B_Q], 0, abort_flag);
       for (int j = 0; j < nkv && ok; ++j) {
-        ok = tc::mbar_wait(&bar[B_K], j & 1, &g_tc_fwd_error);
+        ok = tc::mbar_wait(&bar[B_K], j & 1, abort_flag);
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
                           idS, k > 0);
         }
         tc::tc_commit(&bar[B_S]);
-        ok = tc::mbar_wait(&bar[B_P], j & 1, &g_tc_fwd_error) && tc::mbar_wait(&bar[B_V], j & 1, &g_tc_fwd_error);
+        ok = tc::mbar_wait(&bar[B_P], j & 1, abort_flag) && tc::mbar_wait(&bar[B_V], j & 1, abort_flag);
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
         tc::tc_commit(&bar[B_PV]);
       }
       if (ok && has_prev) {
-        ok = tc::mbar_wait(&bar[B_QS], 0, &g_tc_fwd_error) && tc::mbar_wait(&bar[B_C], 0, &g_tc_fwd_error);
+        ok = tc::mbar_wait(&bar[B_QS], 0, abort_flag) && tc::mbar_wait(&bar[B_C], 0, abort_flag);
         if (ok) {
           tc::tc_fence_after();
 #pragma unroll
@@ -226,8 +227,8 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     float rowsum = 0.f;
 
     for (int j = 0; j < nkv && ok; ++j) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_S], j & 1, &g_tc_fwd_error));
-      if (ok && j > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_PV], (j - 1) & 1, &g_tc_fwd_error));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_S], j & 1, abort_flag));
+      if (ok && j > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_PV], (j - 1) & 1, abort_flag));
       if (!ok) break;
       tc::tc_fence_after();
       const bool diag = (j == qt);
@@ -265,7 +266,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     // inter-chunk operand: scale the query rows by alpha_t / sqrt(d_qk) in place
     float inter_norm = 0.f;
     if (ok && has_prev) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_Q], 0, &g_tc_fwd_error));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_Q], 0, abort_flag));
       if (ok) {
 #pragma unroll 1
         for (int kb = 0; kb < Cfg::KB; ++kb) {
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       }
     }
 
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_O], 0, &g_tc_fwd_error));
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_O], 0, abort_flag));
     if (ok) {
       tc::tc_fence_after();
       float inv = 1.f;
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bar[B_STG]);
       if (row == 0) {
-        ok = tc::mbar_wait(&bar[B_STG], 0, &g_tc_fwd_error);
+        ok = tc::mbar_wait(&bar[B_STG], 0, abort_flag);
         if (ok) {
           for (int blk = 0; blk < DV / 64; ++blk)
             tc::tma_store_3d(&tm_h, sP + blk * 16384, dv0 + blk * 64, c0 + t0, bh);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     }
   }
 
-  if (!ok) atomicOr(&g_tc_fwd_error, 1u);
+  if (!ok) abort_flag.raise();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -373,7 +374,7 @@ static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_
   dim3 grid((unsigned)(p.BH * p.NC * ntq), (unsigned)(p.dhv / DV)), block(192);
   kern<<<grid, block, smem, s>>>(tq, tk, tv, tcm, th, a.b, a.li, a.m, a.n, (bf16*)a.h, a.abar, p.T,
                                  p.L, p.NC, p.BH, ntq, p.dhv, p.scale, log2f(p.scale), a.init.on(),
-                                 a.init.on() ? a.init.m : nullptr);
+                                 a.init.on() ? a.init.m : nullptr, next_epoch());
   return cudaGetLastError();
 }
 
@@ -397,11 +398,24 @@ cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_
   }
 }
 
+// Self-test of the failure report: one thread waits on an mbarrier that nothing
+// completes, its bounded wait runs out, and it raises its launch's flag in this
+// kernel family, as a chunk-128 output CTA whose hand-over never came would.
+__global__ void selftest_timeout_kernel(unsigned int epoch) {
+  __shared__ uint64_t bar;
+  const tc::Abort abort_flag{&g_tc_fwd_error, epoch};
+  tc::mbar_init(&bar, 1);
+  tc::fence_mbar_init();
+  if (!tc::mbar_wait(&bar, 0, abort_flag)) abort_flag.raise();
+}
+
+cudaError_t launch_selftest_timeout(cudaStream_t s) {
+  selftest_timeout_kernel<<<1, 1, 0, s>>>(next_epoch());
+  return cudaGetLastError();
+}
+
 cudaError_t fetch_tc_fwd_error(unsigned int* flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_fwd_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_fwd_error, &zero, sizeof(unsigned int));
+  return cudaMemcpyFromSymbol(flag, g_tc_fwd_error, sizeof(unsigned int));
 }
 
 }  // namespace mlstm

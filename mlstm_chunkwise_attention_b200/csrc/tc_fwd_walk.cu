@@ -80,6 +80,7 @@ struct FwalkParams {
   InitState init;           // the state entering the first chunk (C null: zero)
   int T, NC;
   float scale, log2_scale;
+  unsigned int epoch;  // this launch's abort epoch
 };
 
 template <bool EXPV>
@@ -89,7 +90,8 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     const __grid_constant__ CUtensorMap tmChi, const __grid_constant__ CUtensorMap tmClo,
     const FwalkParams P) {
   using Cfg = FwalkCfg;
-  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_fwalk_error != 0u)) return;
+  const tc::Abort abort_flag{&g_tc_fwalk_error, P.epoch};
+  if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
   const int bh = blockIdx.x;
   const int NC = P.NC;
   extern __shared__ uint8_t smem_raw[];
@@ -100,7 +102,6 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
   float* F = reinterpret_cast<float*>(smem + Cfg::OFF_F);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
-  const volatile unsigned int* abort_flag = &g_tc_fwalk_error;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the K/V set of chunk c, and the set holding its C staging (hi plane, lo plane at +TILE)
   auto set_of = [&](int c) { return smem + ((c & 1) ? Cfg::OFF_SET1 : Cfg::OFF_SET0); };
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         }
         tc::tc_commit(&bar[BF_S]);
       }
-      if (!ok) atomicOr(&g_tc_fwalk_error, 1u);
+      if (!ok) abort_flag.raise();
     }
   } else {
     // ------------------------------------------------------------ rows
@@ -216,14 +217,14 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     auto wait_mma = [&]() -> bool {
       const bool w = __all_sync(full, tc::mbar_wait(&bar[BF_M], nm & 1, abort_flag));
       ++nm;
-      if (!w && lane == 0) atomicOr(&g_tc_fwalk_error, 1u);
+      if (!w && lane == 0) abort_flag.raise();
       tc::tc_fence_after();
       return w;
     };
     auto wait_state = [&]() -> bool {
       const bool w = __all_sync(full, tc::mbar_wait(&bar[BF_S], ns & 1, abort_flag));
       ++ns;
-      if (!w && lane == 0) atomicOr(&g_tc_fwalk_error, 1u);
+      if (!w && lane == 0) abort_flag.raise();
       tc::tc_fence_after();
       return w;
     };
@@ -555,7 +556,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     // the last chunk's hand-over: every product has completed
     if (ok) ok = wait_state();
     if (issuer) tc::bulk_wait_all();
-    if (!ok) atomicOr(&g_tc_fwalk_error, 1u);
+    if (!ok) abort_flag.raise();
   }
 
   tc::tc_fence_before();
@@ -596,6 +597,7 @@ static cudaError_t launch_fwalk(const Problem& p, const FwdArgs& a, cudaStream_t
   P.T = p.T; P.NC = p.NC;
   P.scale = p.scale;
   P.log2_scale = log2f(p.scale);
+  P.epoch = next_epoch();
   auto kern = fwd_walk_kernel<EXPV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)FwalkCfg::SMEM);
@@ -609,10 +611,7 @@ cudaError_t launch_fwd_walk(const Problem& p, const FwdArgs& a, cudaStream_t s) 
 }
 
 cudaError_t fetch_tc_fwalk_error(unsigned int* flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_fwalk_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_fwalk_error, &zero, sizeof(unsigned int));
+  return cudaMemcpyFromSymbol(flag, g_tc_fwalk_error, sizeof(unsigned int));
 }
 
 }  // namespace mlstm

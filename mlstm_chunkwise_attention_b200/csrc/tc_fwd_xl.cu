@@ -140,7 +140,7 @@ template <int DQK, int DV, bool EXPV>
 __device__ __noinline__ bool xl_epilogue(int it, int vb, int nvalid, size_t tok, float fl, float part,
                                          int h, int qr, int lane, uint32_t tmem, uint8_t* smem,
                                          bf16* __restrict__ hout, float* __restrict__ abar_out,
-                                         int dhv, const volatile unsigned int* abort_flag) {
+                                         int dhv, const tc::Abort& abort_flag) {
   using Cfg = XlCfg<DQK, DV>;
   const unsigned full = 0xffffffffu;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
@@ -213,12 +213,12 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
     const float* __restrict__ tab, const float* __restrict__ gn, bf16* __restrict__ hout,
     float* __restrict__ abar_out, int T, int L, int NC, int BH, int NVB, int ntq, int total,
-    int tstride, int dhv, bool has_init) {
+    int tstride, int dhv, bool has_init, unsigned int epoch) {
   using Cfg = XlCfg<DQK, DV>;
+  const tc::Abort abort_flag{&g_tc_fwd_xl_error, epoch};
   constexpr int NQ = Cfg::NQ, NK = Cfg::NK, NV = Cfg::NV;
   // an earlier CTA gave up: the whole block leaves together
-  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_fwd_xl_error != 0u)) return;
-  const volatile unsigned int* abort_flag = &g_tc_fwd_xl_error;
+  if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     if (ok && pend) ok = epilogue(pe);
   }
 
-  if (!ok) atomicOr(&g_tc_fwd_xl_error, 1u);
+  if (!ok) abort_flag.raise();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -690,7 +690,7 @@ static cudaError_t launch_out_xl(const Problem& p, const FwdArgs& a, cudaStream_
   const int grid = (int)(pairs < nsm ? pairs : nsm);
   kern<<<grid, kXlThreads, smem, s>>>(tq, tk, tv, tcm, a.xt, a.n, (bf16*)a.h, a.abar, p.T, p.L,
                                       p.NC, p.BH, nvb, ntq, (int)total, xl_table_stride(p.L),
-                                      p.dhv, a.init.on());
+                                      p.dhv, a.init.on(), next_epoch());
   return cudaGetLastError();
 }
 
@@ -714,10 +714,7 @@ cudaError_t launch_output_fwd_xl(const Problem& p, const FwdArgs& a, cudaStream_
 }
 
 cudaError_t fetch_tc_fwd_xl_error(unsigned int* flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_fwd_xl_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_fwd_xl_error, &zero, sizeof(unsigned int));
+  return cudaMemcpyFromSymbol(flag, g_tc_fwd_xl_error, sizeof(unsigned int));
 }
 
 }  // namespace mlstm

@@ -72,6 +72,7 @@ struct StateTcParams {
   InitState init;   // forward: the state entering chunk 0; both: its max state m0
   float *d0, *dn0;  // backward: gradient of the initial state (C, n), fp32, or null
   const float *dT, *dnT;  // backward: gradient of the final state (C, n), fp32, or null
+  unsigned int epoch;     // this launch's abort epoch
 };
 
 template <bool BWD, bool EXPV, int NV>
@@ -81,9 +82,10 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tmOlo,
                                                           const StateTcParams P) {
   using Cfg = StateTcCfg<NV>;
+  const tc::Abort abort_flag{&g_tc_state_error, P.epoch};
   constexpr int SUB = Cfg::SUB;
   // an earlier CTA gave up: the whole block leaves together
-  if (__syncthreads_or(threadIdx.x == 0 && *(volatile unsigned int*)&g_tc_state_error != 0u)) return;
+  if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
   // value-column tiles vary fastest so the CTAs sharing one head's key rows run together
   const int dv0 = blockIdx.x * NV, dk0 = blockIdx.y * 128, bh = blockIdx.z;
   const bool with_n = EXPV && blockIdx.x == 0;
@@ -99,7 +101,6 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
-  const volatile unsigned int* abort_flag = &g_tc_state_error;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -373,7 +374,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   }
 
   if (warp >= 4 && threadIdx.x == 128) tc::bulk_wait_all();  // this thread's TMA stores are done
-  if (!ok) atomicOr(&g_tc_state_error, 1u);
+  if (!ok) abort_flag.raise();
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -417,6 +418,7 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
   P.dn0 = dn0;
   P.dT = dT;
   P.dnT = dnT;
+  P.epoch = next_epoch();
   auto kern = state_tc_kernel<BWD, EXPV, NV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
@@ -454,10 +456,7 @@ cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t
 }
 
 cudaError_t fetch_tc_state_error(unsigned int* flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_state_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_tc_state_error, &zero, sizeof(unsigned int));
+  return cudaMemcpyFromSymbol(flag, g_tc_state_error, sizeof(unsigned int));
 }
 
 }  // namespace mlstm

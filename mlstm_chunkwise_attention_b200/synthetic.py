@@ -91,3 +91,31 @@ def sample_rows(T, n, seed, chunk=None):
         rows.update({min(chunk - 1, T - 1), min(chunk, T - 1)})
     rows.update(torch.randint(0, T, (max(n - len(rows), 0),), generator=g).tolist())
     return sorted(rows)
+
+
+# ---------------------------------------------------------------------------
+# Retention (RetNet) inputs: constant gates that make mLSTMsig a retention
+# ---------------------------------------------------------------------------
+
+#: input-gate preactivation whose log-sigmoid is 0 to fp32 rounding (input gate 1)
+RETENTION_IGATE = 30.0
+
+
+def retnet_decays(num_heads):
+    """RetNet's per-head decay schedule gamma_h = 1 - 2^(-5 - h), fp64."""
+    return 1.0 - torch.pow(2.0, -5.0 - torch.arange(num_heads, dtype=torch.float64))
+
+
+def retention_gates(gamma, B, T, dtype, device):
+    """Gate preactivations [B, NH, T] for a retention with decay gamma[h] per head.
+
+    The input gate is RETENTION_IGATE everywhere and the forget gate of head h is
+    logit(gamma_h), both rounded to the I/O dtype; the decay the mLSTMsig cell then
+    applies is the sigmoid of that rounded forget preactivation.
+    """
+    g = torch.as_tensor(gamma, dtype=torch.float64).cpu()
+    NH = g.numel()
+    fg_h = (torch.log(g) - torch.log1p(-g)).to(dtype)
+    fg = fg_h.view(1, NH, 1).expand(B, NH, T).contiguous().to(device)
+    ig = torch.full((B, NH, T), RETENTION_IGATE, dtype=dtype, device=device)
+    return ig, fg

@@ -563,23 +563,6 @@ def parallel_backward_rows(q, k, v, log_i, log_f, variant, dh, h, a, den, rows):
 # batched helpers ([B, NH, T, d] arrays, heads independent)
 # ---------------------------------------------------------------------------
 
-def forward_heads(q, k, v, igate_pre, fgate_pre, variant, L=None, form="chunkwise"):
-    """Run one forward form on every (b, h) head; returns h [B, NH, T, d_hv]."""
-    B, NH, T, _ = q.shape
-    out = np.empty(v.shape, dtype=np.float64)
-    for bb in range(B):
-        for hh in range(NH):
-            li, lf = gate_logs(igate_pre[bb, hh], fgate_pre[bb, hh], variant)
-            args = (q[bb, hh], k[bb, hh], v[bb, hh], li, lf)
-            if form == "chunkwise":
-                out[bb, hh] = chunkwise_forward(*args, variant, L)["h"]
-            elif form == "parallel":
-                out[bb, hh] = parallel_forward(*args, variant)["h"]
-            else:
-                out[bb, hh] = recurrent_forward(*args, variant)["h"]
-    return out
-
-
 def backward_heads(q, k, v, igate_pre, fgate_pre, variant, dh):
     """Parallel-form backward on every head, returning preactivation gradients."""
     res = {n: np.empty(x.shape, dtype=np.float64) for n, x in

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from mlstm_chunkwise_attention_b200 import binding
-from mlstm_chunkwise_attention_b200.synthetic import WORKLOADS, sample_heads
+from mlstm_chunkwise_attention_b200.synthetic import WORKLOADS, sample_heads, sample_rows
 from _parity import (TOL, gpu_bwd, gpu_fwd, head64, inputs, np64, oracle_bwd_head,
                      oracle_fwd_head, relerr)
 
@@ -77,6 +77,45 @@ def test_small_forward_backward_all_heads(case):
             for key, val in ref_g.items():
                 err = relerr(np64(g[key][b, hh]), val, floor=floor)
                 assert err <= tol, f"{key} ({b},{hh}): {err:.3e}"
+
+
+# mLSTMexp with large positive input-gate preactivations, on every tensor-core path:
+# exp(i~) far above 1 stresses the max state, the separable decay factors and the
+# hi/lo state planes.  name, B, NH, T, d_qk, d_hv, chunk, igate mean, igate std,
+# spike value (every 53rd token from token 11 on), forget mean
+BIG_IGATE = [
+    ("exp_walkers_chunk128_d128", 2, 2, 700, 128, 128, 128, 8.0, 2.0, None, 3.0),
+    ("exp_walkers_chunk128_d128_spikes40", 1, 2, 640, 128, 128, 128, 0.0, 1.0, 40.0, 3.0),
+    ("exp_chunk128_dqk256_dhv512", 1, 2, 300, 256, 512, 128, 8.0, 2.0, None, 3.0),
+    ("exp_chunk128_dqk64_dhv64_spikes40", 1, 2, 400, 64, 64, 128, 0.0, 1.0, 40.0, 3.0),
+    ("exp_xl_chunk256_ragged", 1, 2, 700, 128, 128, 256, 8.0, 2.0, None, 3.0),
+    ("exp_xl_chunk256_spikes40", 1, 2, 600, 64, 128, 256, 0.0, 1.0, 40.0, 3.0),
+    ("exp_xl_chunk1024", 1, 2, 2048, 128, 128, 1024, 8.0, 2.0, None, 3.0),
+    ("exp_xl_chunk1024_spikes40", 1, 1, 1500, 128, 128, 1024, 0.0, 1.0, 40.0, 3.0),
+    ("exp_chunk64_d128", 1, 2, 500, 128, 128, 64, 8.0, 2.0, None, 3.0),
+    ("exp_chunk64_d64_spikes40", 1, 2, 333, 64, 64, 64, 0.0, 1.0, 40.0, 3.0),
+]
+
+
+@pytest.mark.parametrize("case", BIG_IGATE, ids=[c[0] for c in BIG_IGATE])
+def test_exp_large_input_gates_all_heads(case):
+    name, Bn, NH, T, dqk, dhv, L, igm, igs, spike, fgm = case
+    cpu = inputs(Bn, NH, T, dqk, dhv, seed=zlib.crc32(name.encode()) % 10000, dtype=BF,
+                 ig_mean=igm, fg_mean=fgm, igate_std=igs)
+    if spike is not None:
+        cpu["igate"][..., 11::53] = spike
+    dev, h, saved = gpu_fwd(cpu, L, EXP)
+    g = gpu_bwd(dev, h, saved, L, EXP)
+    for b in range(Bn):
+        for hh in range(NH):
+            x = head64(cpu, b, hh)
+            ref = oracle_fwd_head(x, L, EXP)
+            assert relerr(np64(h[b, hh]), ref["h"]) <= 1e-2, f"h ({b},{hh})"
+            ref_g = oracle_bwd_head(x, EXP)
+            floor = 1e-3 * max(np.max(np.abs(v)) for v in ref_g.values())
+            for key, val in ref_g.items():
+                err = relerr(np64(g[key][b, hh]), val, floor=floor)
+                assert err <= 1e-2, f"{key} ({b},{hh}): {err:.3e}"
 
 
 @pytest.mark.parametrize("var", [SIG, EXP])
@@ -225,6 +264,44 @@ def _full(name, variant=None, heads_fwd=2, heads_bwd=1):
 
 def test_full_headline_exp_b8h32_t4096_fwd_bwd():
     _full("exp_b8h32_t4096_d128_c128", heads_fwd=3, heads_bwd=2)
+
+
+def test_full_headline_every_head_sampled_rows():
+    """Every one of the 256 heads of the headline workload (the walkers run one CTA per
+    head in more than one wave) on sampled rows: h and dq on rows spread over the
+    sequence, dk, dv and d igate on columns of the last chunk, each from its own row or
+    column of the oracle's parallel form."""
+    spec = WORKLOADS["exp_b8h32_t4096_d128_c128"]
+    T, L, var = spec["T"], spec["chunk"], spec["variant"]
+    cpu = inputs(spec["B"], spec["NH"], T, spec["d_qk"], spec["d_hv"], seed=spec["seed"], dtype=BF,
+                 ig_mean=spec["igate_mean"], fg_mean=spec["fgate_mean"])
+    dev, h, saved = gpu_fwd(cpu, L, var)
+    g = gpu_bwd(dev, h, saved, L, var)
+    rows = sample_rows(T, 6, spec["seed"], chunk=L)
+    cols = [T - L, T - 70, T - 1]
+    tail = list(range(T - L, T))
+    need = sorted(set(rows) | set(tail))
+    for b in range(spec["B"]):
+        for hh in range(spec["NH"]):
+            x = head64(cpu, b, hh)
+            li, lf = oracle.gate_logs(x["igate"], x["fgate"], var)
+            fr = oracle.parallel_forward_rows(x["q"], x["k"], x["v"], li, lf, var, need)
+            hf = np.zeros((T, spec["d_hv"]))
+            af, df = np.zeros(T), np.ones(T)
+            hf[need], af[need], df[need] = fr["h"], fr["a"], fr["den"]
+            assert relerr(np64(h[b, hh])[rows], hf[rows]) <= 1e-2, f"h ({b},{hh})"
+            # dq of row r reads only row r of the forward
+            br = oracle.parallel_backward_rows(x["q"], x["k"], x["v"], li, lf, var, x["dh"], hf, af,
+                                               df, rows)
+            assert relerr(np64(g["dq"][b, hh])[rows], br["dq"]) <= 1e-2, f"dq ({b},{hh})"
+            # dk, dv, d log i of column s read the forward rows t >= s (all in `tail`)
+            bc = oracle.parallel_backward_rows(x["q"], x["k"], x["v"], li, lf, var, x["dh"], hf, af,
+                                               df, cols)
+            di, _ = oracle.preact_grads(bc["dlog_i"], np.zeros(len(cols)), x["igate"][cols],
+                                        x["fgate"][cols], var)
+            for key, val in (("dk", bc["dk"]), ("dv", bc["dv"]), ("digate_pre", di)):
+                err = relerr(np64(g[key][b, hh])[cols], val)
+                assert err <= 1e-2, f"{key} ({b},{hh}): {err:.3e}"
 
 
 @pytest.mark.parametrize("var", [SIG, EXP])

@@ -12,7 +12,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mlstm_chunkwise_attention_b200 import binding
+from mlstm_chunkwise_attention_b200.synthetic import retention_gates, retnet_decays
 from _parity import TOL, inputs, np64, relerr
 
 pytestmark = pytest.mark.gpu
@@ -44,9 +46,12 @@ def test_retention_matches_closed_form(case):
     B, NH, d = 1, 4, 128 if dt == BF else 64
     cpu = inputs(B, NH, T, d, d, seed=41, dtype=dt)
     dev = {k: v.cuda() for k, v in cpu.items()}
-    gamma = binding.retnet_decays(NH)
-    h, saved, (ig, fg, gamma_eff) = binding.retention(dev["q"], dev["k"], dev["v"], gamma, L,
-                                                       keep_saved=True)
+    gamma = retnet_decays(NH)
+    ig, fg = retention_gates(gamma, B, T, dt, "cuda")
+    # the decay the kernels apply: the sigmoid of the stored forget preactivation
+    gamma_eff = oracle.sigmoid(fg[0, :, 0].double().cpu().numpy())
+    h, saved = binding.forward(dev["q"], dev["k"], dev["v"], ig, fg, L, binding.SIG,
+                               keep_saved=True)
     g = binding.backward(dev["q"], dev["k"], dev["v"], ig, fg, h, dev["dh"], saved, L, binding.SIG)
     binding.check_device()
     tol = TOL[dt]
