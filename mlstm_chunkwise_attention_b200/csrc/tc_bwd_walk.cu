@@ -181,22 +181,24 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
         ok = wait_rows() && wait_tile(BW_H, it);
         if (!ok) break;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tAV, tX + 8 * k, mnmaj(aH, k), idKM, 1);
+        for (int k = 0; k < 8; ++k)  // keys 64 h .. 64 h + 63 of Y live at column 64 h
+          tc::mma_bf16_ts(tAV, tX + 64 * (k >> 2) + 8 * (k & 3), mnmaj(aH, k), idKM, 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tX, kmaj(aV, k), kmaj(aH, k), idKK, k > 0);
         tc::tc_commit(&bar[BW_M]);
         // C (dk transform in TMEM): dk += Y Q; then the normaliser's increment Q^T wn (hi, lo)
-        // into columns 0 and 1 of the score buffer
+        // into columns 32 and 33 of the score buffer (Y lives in columns 0..31 and 64..95)
         ok = wait_rows();
         if (!ok) break;
         const bool update = c > 0 || P.d0 != nullptr;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tAK, tX + 8 * k, mnmaj(aQ, k), idKM, 1);
+        for (int k = 0; k < 8; ++k)
+          tc::mma_bf16_ts(tAK, tX + 64 * (k >> 2) + 8 * (k & 3), mnmaj(aQ, k), idKM, 1);
         if (EXPV && update) {
           const uint32_t wn = aWN + (it & 1) * Cfg::WN_BYTES;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            tc::mma_bf16_ss(tX, mnmaj(aQ, k),
+            tc::mma_bf16_ss(tX + 32, mnmaj(aQ, k),
                             tc::sdesc_sw128(wn + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), idN,
                             k > 0);
         }
@@ -309,10 +311,10 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       }
       return G;
     };
-    // columns 0 and 1 of the score buffer after the dk accumulate: the normaliser's increment
+    // columns 32 and 33 of the score buffer after the dk accumulate: the normaliser's increment
     auto dn_increment = [&]() -> float {
       float a, b;
-      walk::tmem_ld2(tX + lane_base, a, b);
+      walk::tmem_ld2(tX + 32 + lane_base, a, b);
       return a + b;
     };
     // Rescale an inter-term accumulator row in TMEM: x = rs x (+ rs dn[col] for dk, mLSTMexp).
@@ -412,7 +414,9 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
             }
           }
         }
-        tc::tmem_st16_async(tX + lane_base + 16 * ch, pk);
+        // packed into this half's own columns [64 half, 64 half + 32): the other warp of the
+        // lane quarter may still be reading its fp32 scores in [64 (1 - half), ...)
+        tc::tmem_st16_async(tX + lane_base + 32 * cb0 + 16 * (ch - cb0), pk);
       };
       uint32_t xa[32], xb[32];
       tc::tmem_ld32_async(tX + lane_base + 32 * cb0, xa);

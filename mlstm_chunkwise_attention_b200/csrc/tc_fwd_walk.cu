@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         ok = wait_rows();
         if (!ok) break;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) tc::mma_bf16_ts(tO, tS + 8 * k, mnmaj(aV, k), idKM, 1);
+        for (int k = 0; k < 8; ++k)  // keys 64 h .. 64 h + 63 of P live at column 64 h
+          tc::mma_bf16_ts(tO, tS + 64 * (k >> 2) + 8 * (k & 3), mnmaj(aV, k), idKM, 1);
         tc::tc_commit(&bar[BF_M]);
         // D (w K staged: hi plane over K, lo plane apart): C_{c+1} = beta_c C_c (the rows
         // scaled it) + (w K)^T V, while P V runs
@@ -389,7 +390,9 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
             rs += a.x + a.y;
           }
         }
-        tc::tmem_st16_async(tS + lane_base + 16 * ch, pk);
+        // packed into this half's own columns [64 half, 64 half + 32): the other warp of the
+        // lane quarter may still be reading its fp32 scores in [64 (1 - half), ...)
+        tc::tmem_st16_async(tS + lane_base + 32 * cb0 + 16 * (ch - cb0), pk);
       };
       MLSTM_WALK_PIPE(tS, one)
       return rs;
