@@ -17,7 +17,11 @@ namespace mlstm {
 // recurrence m_c = max(g_c + m_{c-1}, g_c + max_{s in c}(log i_s - b_s)).
 // One CTA per (b, h); each warp owns whole chunks, each lane a contiguous
 // run of rows.  The chunk recurrence is an inclusive warp scan of the affine
-// max-plus maps x -> max(x + g_c, u_c).
+// max-plus maps x -> max(x + g_c, u_c).  The sums run in fp64 and are rounded
+// once to fp32: b reaches tens in magnitude over a long chunk, and fp32
+// partial sums would carry an error of many fp32 ulps of it into every decay
+// exp(b_t - b_s + ...) and into the normaliser, where it is amplified when the
+// normaliser nearly cancels.
 // ---------------------------------------------------------------------------
 // Per-chunk gate tables of the large-chunk output kernel (layout in
 // internal.h).  With R_t + CC_s = log2 D_ts / sqrt(d_qk) for s <= t, the decay
@@ -74,36 +78,36 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
     const int len = min(L, T - c0);
     const int per = (len + 31) / 32;
     const int r0 = min(lane * per, len), r1 = min(r0 + per, len);
-    float seg = 0.f;
-    for (int r = r0; r < r1; ++r) seg += log_sigmoid(to_f32(fg[base + c0 + r]));
-    const float incl = warp_incl_sum(seg);
-    float run = incl - seg;
-    float umax = -INFINITY;
+    double seg = 0.0;
+    for (int r = r0; r < r1; ++r) seg += (double)log_sigmoid(to_f32(fg[base + c0 + r]));
+    const double incl = warp_incl_sum(seg);
+    double run = incl - seg;
+    double umax = -INFINITY;
     for (int r = r0; r < r1; ++r) {
       const size_t idx = base + c0 + r;
-      run += log_sigmoid(to_f32(fg[idx]));
+      run += (double)log_sigmoid(to_f32(fg[idx]));
       const float x = to_f32(ig[idx]);
       const float li = EXPV ? x : log_sigmoid(x);
-      b_out[idx] = run;
+      b_out[idx] = (float)run;
       li_out[idx] = li;
       if (EXPV) {
-        umax = fmaxf(umax, li - run);
-        m_out[idx] = umax;
+        umax = fmax(umax, (double)li - run);
+        m_out[idx] = (float)umax;
       }
     }
     if (EXPV) {
-      const float pm = warp_incl_max(umax);
+      const float pm = warp_incl_max((float)umax);
       float excl = __shfl_up_sync(full, pm, 1);
       if (lane == 0) excl = -INFINITY;
       for (int r = r0; r < r1; ++r) {
         const size_t idx = base + c0 + r;
         m_out[idx] = fmaxf(m_out[idx], excl);
       }
-      const float g = __shfl_sync(full, incl, 31);
-      const float tot = __shfl_sync(full, pm, 31);
+      const double g = __shfl_sync(full, incl, 31);
+      const double tot = __shfl_sync(full, (double)pm, 31);
       if (lane == 0) {
-        sg[c] = g;
-        su[c] = g + tot;
+        sg[c] = (float)g;
+        su[c] = (float)(g + tot);
       }
     }
   }
@@ -118,22 +122,22 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
   // the max state before the first chunk: the initial state's, -inf without one
   const float m_init = m0 != nullptr ? m0[blockIdx.x] : -INFINITY;
   if (warp == 0) {
-    float carry = m_init;
+    double carry = m_init;
     for (int cb = 0; cb < NC; cb += 32) {
       const int c = cb + lane;
-      float g = c < NC ? sg[c] : 0.f;
-      float u = c < NC ? su[c] : -INFINITY;
+      double g = c < NC ? (double)sg[c] : 0.0;
+      double u = c < NC ? (double)su[c] : -INFINITY;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const float g2 = __shfl_up_sync(full, g, o);
-        const float u2 = __shfl_up_sync(full, u, o);
+        const double g2 = __shfl_up_sync(full, g, o);
+        const double u2 = __shfl_up_sync(full, u, o);
         if (lane >= o) {
-          u = fmaxf(u2 + g, u);
+          u = fmax(u2 + g, u);
           g = g2 + g;
         }
       }
-      const float mc = fmaxf(carry + g, u);
-      if (c < NC) su[c] = mc;
+      const double mc = fmax(carry + g, u);
+      if (c < NC) su[c] = (float)mc;
       carry = __shfl_sync(full, mc, 31);
     }
   }

@@ -187,17 +187,18 @@ __global__ void fill_neg_inf_kernel(float* __restrict__ m, int count) {
 template <typename TIO>
 __global__ void __launch_bounds__(256) log_decay_kernel(const TIO* __restrict__ fg,
                                                         float* __restrict__ G, int T) {
-  __shared__ float part[8];
+  // summed in fp64, like the in-chunk cumsums of gate_prep, and rounded once
+  __shared__ double part[8];
   const size_t base = (size_t)blockIdx.x * T;
-  float acc = 0.f;
-  for (int t = threadIdx.x; t < T; t += blockDim.x) acc += log_sigmoid(to_f32(fg[base + t]));
+  double acc = 0.0;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) acc += (double)log_sigmoid(to_f32(fg[base + t]));
   acc = warp_sum(acc);
   if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
   __syncthreads();
   if (threadIdx.x == 0) {
-    float g = 0.f;
+    double g = 0.0;
     for (int w = 0; w < 8; ++w) g += part[w];
-    G[blockIdx.x] = g;
+    G[blockIdx.x] = (float)g;
   }
 }
 

@@ -18,9 +18,12 @@
 //   Acc += Y E_j        (dq: E = K, dk: E = Q, dv: E = dH)
 // The inter-chunk term Acc = A_R G (G the chunk state or its gradient, split
 // into hi and lo bf16 planes so the product keeps about 16 mantissa bits) is
-// computed first and rescaled per row in TMEM.  Warp roles: warp 0 TMA,
-// warp 1 MMA (one thread), warps 2..5 one tile row per thread.  Every wait is
-// bounded; on a timeout the kernel raises an error flag and winds down.
+// computed first and rescaled per row in TMEM.  A 64-token chunk is one
+// half-filled 128-row tile with one partner: its score product has N = 64,
+// the accumulate contracts over 64 partners, and the result leaves through a
+// 64-row store.  Warp roles: warp 0 TMA, warp 1 MMA (one thread), warps 2..5
+// one tile row per thread.  Every wait is bounded; on a timeout the kernel
+// raises an error flag and winds down.
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -53,13 +56,15 @@ struct BwdTcCfg {
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_RV = OFF_TMEM + 16;
   static constexpr int OFF_PW = OFF_RV + D2S * 4;   // per-warp partner factors, 4 x 128 floats
-  static constexpr int OFF_PF = OFF_PW + 4 * 128 * 4;  // partner factors: 2 x L, then L / 32 (>= 4)
+  static constexpr int OFF_PF = OFF_PW + 4 * 128 * 4;  // partner factors: 2 x PL, then PL / 32 (>= 4)
   static constexpr uint32_t TMEM_COLS = NXBUF == 1 ? 256 : 512;  // X buffers, then Acc
   static constexpr uint32_t ACC_COL = NXBUF * 128;
   static constexpr uint32_t G_BYTES = G_MN ? (uint32_t)EB * 8192u : (uint32_t)D2S * 128u;
   static constexpr uint32_t E_BYTES = (uint32_t)EB * SLOT;
+  // PL = max(L, 128): a 64-token chunk still loads one whole 128-row partner tile
   static size_t smem_bytes(int L) {
-    return 1024 + OFF_PF + ((size_t)2 * L + (L / 32 > 4 ? L / 32 : 4)) * 4;
+    const size_t PL = L < 128 ? 128 : (size_t)L;
+    return 1024 + OFF_PF + (2 * PL + (PL / 32 > 4 ? PL / 32 : 4)) * 4;
   }
 };
 
@@ -105,6 +110,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   const int c0 = c * P.L;
   const int len = min(P.L, P.T - c0);
   const int nt_len = (len + 127) / 128;  // tiles holding rows of this chunk
+  const int NP = P.L < 128 ? P.L : 128;  // partners per partner tile (64 for a 64-token chunk)
   const int r0 = it_tile * 128;
   if (r0 >= len) return;
   // an earlier CTA gave up: the whole block leaves together
@@ -126,8 +132,9 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
   float* rowvec = reinterpret_cast<float*>(smem + Cfg::OFF_RV);
   float* pfC = reinterpret_cast<float*>(smem + Cfg::OFF_PF);  // partner exponent term
-  float* pfE = pfC + P.L;  // partner additive term (dk) or separable key factor (dq)
-  float* pfM = pfE + P.L;  // dq: stabiliser of every 32-key partner block
+  const int PL = P.L < 128 ? 128 : P.L;  // partner slots: whole 128-row partner tiles
+  float* pfE = pfC + PL;  // partner additive term (dk) or separable key factor (dq)
+  float* pfM = pfE + PL;  // dq: stabiliser of every 32-key partner block
   float* pfW = reinterpret_cast<float*>(smem + Cfg::OFF_PW);  // dk, dv: this warp's partner factors
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -222,7 +229,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idX = tc::idesc_bf16(128, 128, false, false);
+      const uint32_t idX = tc::idesc_bf16(128, NP, false, false);
       constexpr uint32_t idAcc = tc::idesc_bf16(128, D2S, false, true);
       constexpr uint32_t idG = tc::idesc_bf16(128, D2S, false, G_MN);
       const uint32_t aRing = tc::smem_u32(ring);
@@ -278,8 +285,9 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         const uint32_t tY = tX0 + (jj % NXBUF) * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc::mma_bf16_ts(tAcc, tY + 8 * k, tc::sdesc_sw128(st + k * 2048, Cfg::SLOT, 1024), idAcc,
-                          (has_inter || jj > 0 || k > 0));
+          if (16 * k < NP)
+            tc::mma_bf16_ts(tAcc, tY + 8 * k, tc::sdesc_sw128(st + k * 2048, Cfg::SLOT, 1024), idAcc,
+                            (has_inter || jj > 0 || k > 0));
         release();
         return true;
       };
@@ -356,6 +364,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int rl = r0 + row;
     const bool valid = rl < len;
+    const int nch = NP / 32;  // 32-column chunks of a score tile
     const size_t tok = tok0 + rl;
     const unsigned full = 0xffffffffu;
     // row-side factors
@@ -511,13 +520,17 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
       tc::tmem_ld32_async(tX + lane_base + 32, xb);
       transform_chunk(xa, 0);
       tc::tmem_wait_ld(xb);
-      tc::tmem_ld32_async(tX + lane_base + 64, xa);
-      transform_chunk(xb, 1);
-      tc::tmem_wait_ld(xa);
-      tc::tmem_ld32_async(tX + lane_base + 96, xb);
-      transform_chunk(xa, 2);
-      tc::tmem_wait_ld(xb);
-      transform_chunk(xb, 3);
+      if (nch > 2) {
+        tc::tmem_ld32_async(tX + lane_base + 64, xa);
+        transform_chunk(xb, 1);
+        tc::tmem_wait_ld(xa);
+        tc::tmem_ld32_async(tX + lane_base + 96, xb);
+        transform_chunk(xa, 2);
+        tc::tmem_wait_ld(xb);
+        transform_chunk(xb, 3);
+      } else {
+        transform_chunk(xb, 1);
+      }
       tc::tmem_wait_st();
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[BB_Y]);
@@ -589,7 +602,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
 // ---------------------------------------------------------------------------
 
 bool intra_bwd_tc_supported(const Problem& p) {
-  return p.bf16() && p.L >= 128 && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
+  return p.bf16() && p.L >= 64 && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
          (p.dhv == 64 || p.dhv == 128 || p.dhv == 256 || p.dhv == 512);
 }
 
@@ -624,7 +637,8 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   {
     void* outp = (KIND == KDQ) ? a.dq : (KIND == KDK) ? a.dk : a.dv;
     const int dout = (KIND == KDV) ? p.dhv : p.dqk;
-    okm &= make_tmap_3d_bf16(&tO, outp, dout, p.T, p.BH, 64, 128);
+    // one 64-row store per block for a 64-token chunk, so the next chunk's rows stay untouched
+    okm &= make_tmap_3d_bf16(&tO, outp, dout, p.T, p.BH, 64, p.L < 128 ? (uint32_t)p.L : 128u);
   }
   if (!okm) return cudaErrorInvalidValue;
   BwdTcParams P;
@@ -636,7 +650,7 @@ static cudaError_t launch_kind(const Problem& p, const BwdArgs& a, cudaStream_t 
   P.m0 = (a.init.on() && p.exp_variant()) ? a.init.m : nullptr;
   P.out = (bf16*)((KIND == KDQ) ? a.dq : (KIND == KDK) ? a.dk : a.dv);
   P.pdot = (KIND == KDQ) ? a.pq : a.pk;
-  P.T = p.T; P.L = p.L; P.NC = p.NC; P.BH = p.BH; P.ntq = p.L / 128;
+  P.T = p.T; P.L = p.L; P.NC = p.NC; P.BH = p.BH; P.ntq = p.L < 128 ? 1 : p.L / 128;
   P.d_out = (KIND == KDV) ? p.dhv : p.dqk;
   P.dqk = p.dqk;
   P.scale = p.scale;

@@ -1,17 +1,22 @@
-// TFLA intra-chunk output kernel (K-c) on the fifth-generation tensor cores.
-//
+// TFLA intra-chunk output kernel (K-c) on the fifth-generation tensor cores,
+// for chunks that fit one 128-row tile (chunk 64 and 128): the single-level
+// ("limit_chunk") form, where one tile holds a whole chunk's queries and keys.
 // "Tiled Flash Linear Attention: More Efficient Linear RNN and xLSTM Kernels"
-// (TFLA summary page, Approach; arXiv abstract page, Abstract): the second
-// level of sequence parallelism tiles the intra-chunk matmuls along the
-// sequence, so the chunk size is not bounded by on-chip memory.  One CTA owns
-// a 128-row query tile of one chunk and a slice of up to 128 value columns;
-// it walks the 128-row key/value tiles of the chunk up to the diagonal:
+// (TFLA summary page, Approach and Measured effects; arXiv abstract page,
+// Abstract).  One CTA owns one chunk and a slice of up to 128 value columns:
 //
-//   S_j  = Q K_j^T                        (tcgen05, bf16 in smem -> fp32 TMEM)
-//   P_j  = S_j * exp(b_t - b_s + log i_s - m_t) / sqrt(d_qk), causal (registers)
-//   O   += P_j V_j                        (tcgen05, P staged to smem in bf16)
-//   O   += (alpha_t Q / sqrt(d_qk)) C_prev (inter-chunk term, same accumulator)
+//   S    = Q K^T                          (tcgen05, bf16 in smem -> fp32 TMEM)
+//   P    = S * exp(b_t - b_s + log i_s - m_t) / sqrt(d_qk), causal (registers)
+//   O    = P V                            (tcgen05, P staged to smem in bf16)
+//   O   += (alpha_t Q / sqrt(d_qk)) C_prev (inter-chunk term, hi and lo planes)
 //   h_t  = O_t / max(|alpha_t q'_t.n_prev + sum_s P_ts|, exp(-m_t))   (mLSTMexp)
+//
+// A 64-token chunk occupies the first 64 rows of the tile: the score product
+// has N = 64 keys, P V contracts over 64 keys, rows 64..127 compute nothing
+// that is kept, and h leaves through a 64-row store.  The state entering the
+// chunk is multiplied in both of its bf16 planes (hi + lo keeps about 16
+// mantissa bits): where the normaliser nearly cancels, h = O / den amplifies
+// the rounding of the inter-chunk term.
 //
 // Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the
 // MMAs (one thread), warps 2..5 own one query row per thread (TMEM lane),
@@ -29,62 +34,54 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// ALIAS (chunk 128, one key tile per query tile): P is written into the K
-// buffer once S is done and C is loaded into the V buffer once PV is done, so
-// the CTA needs 96 KB of shared memory (at d 128) and two CTAs fit on an SM.
-template <int DQK, int DV, bool ALIAS = false>
+// Shared memory, 96 KB at d 128 so two CTAs fit on an SM: the K region takes
+// K, then P once S is done, then the lo plane of C_prev once P V is done; the
+// V region takes V, then the hi plane of C_prev, then the h staging tile.
+template <int DQK, int DV>
 struct OutTcCfg {
-  static constexpr int BM = 128, BN = 128;
   static constexpr int KB = DQK / 64;  // 64-column blocks of Q and K
   static constexpr int VB = DV / 64;   // 64-column blocks of the V / C slice
   static constexpr int Q_BYTES = KB * 16384;
   static constexpr int K_BYTES = KB * 16384;
   static constexpr int C_BYTES = VB * DQK * 128;
   static constexpr int P_TILE = 2 * 16384;
-  static constexpr int KC_BYTES = ALIAS ? (K_BYTES > P_TILE ? K_BYTES : P_TILE)
-                                        : (K_BYTES > C_BYTES ? K_BYTES : C_BYTES);
+  static constexpr int KC_BYTES = K_BYTES > P_TILE ? K_BYTES : P_TILE;
   static constexpr int V_BYTES = VB * 16384;  // one V tile: the bytes its TMA loads deliver
-  static constexpr int V_REGION = ALIAS ? (V_BYTES > C_BYTES ? V_BYTES : C_BYTES) : V_BYTES;
-  static constexpr int P_BYTES = ALIAS ? 0 : 2 * 16384;
+  static constexpr int V_REGION = V_BYTES > C_BYTES ? V_BYTES : C_BYTES;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KC = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_KC + KC_BYTES;
-  static constexpr int OFF_P = OFF_V + V_REGION;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;  // 16 mbarriers
+  static constexpr int OFF_BAR = OFF_V + V_REGION;  // 16 mbarriers
   static constexpr int OFF_TMEM = OFF_BAR + 16 * 8;
   static constexpr int OFF_NVEC = OFF_TMEM + 16;
   static constexpr int OFF_COLF = OFF_NVEC + DQK * 4;
+  static constexpr size_t SMEM = 1024 + OFF_COLF + 128 * 4;
   static constexpr uint32_t TMEM_COLS = 256;  // S in [0, 128), O in [128, 128 + DV)
-  static size_t smem_bytes(int L) { return 1024 + OFF_COLF + (size_t)L * 4; }
+  static_assert(C_BYTES <= KC_BYTES, "the lo plane of C_prev must fit the K region");
 };
 
 enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_STG, B_COUNT };
 
 }  // namespace
 
-template <int DQK, int DV, bool EXPV, bool ALIAS>
-__global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
+template <int DQK, int DV, bool EXPV>
+__global__ void __launch_bounds__(192, 2) output_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-    const __grid_constant__ CUtensorMap tm_h, const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
-    const float* __restrict__ gn, bf16* __restrict__ h, float* __restrict__ abar_out, int T, int L,
-    int NC, int BH, int ntq, int dhv, float scale, float log2_scale, bool has_init,
-    const float* __restrict__ m0, unsigned int epoch) {
-  using Cfg = OutTcCfg<DQK, DV, ALIAS>;
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_chi,
+    const __grid_constant__ CUtensorMap tm_clo, const __grid_constant__ CUtensorMap tm_h,
+    const float* __restrict__ gb, const float* __restrict__ gli, const float* __restrict__ gm,
+    const float* __restrict__ gn, float* __restrict__ abar_out, int T, int L, int NC, float scale,
+    float log2_scale, bool has_init, const float* __restrict__ m0, unsigned int epoch) {
+  using Cfg = OutTcCfg<DQK, DV>;
   const tc::Abort abort_flag{&g_tc_fwd_error, epoch};
-  constexpr int BM = Cfg::BM, BN = Cfg::BN;
+  // NKEY keys per chunk (64 or 128): the score's N, P V's contraction extent
+  const int NKEY = L < 128 ? L : 128;
 
-  const int per = BH * NC;
-  const int qt = ntq - 1 - (int)(blockIdx.x / per);  // heaviest query tiles first
-  const int rest = (int)(blockIdx.x % per);
-  const int bh = rest / NC, c = rest % NC;
+  const int bh = (int)(blockIdx.x / NC), c = (int)(blockIdx.x % NC);
   const int c0 = c * L;
   const int len = min(L, T - c0);
-  const int t0 = qt * BM;
-  if (t0 >= len) return;
-  // an earlier CTA gave up: the whole block leaves together
+  // an earlier CTA of this launch gave up: the whole block leaves together
   if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
-  const int nkv = qt + 1;
   const int dv0 = blockIdx.y * DV;
   const size_t tok0 = (size_t)bh * T + c0;
   const bool has_prev = c > 0 || has_init;  // a state enters this chunk
@@ -93,10 +90,8 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem + Cfg::OFF_Q;
-  uint8_t* sKC = smem + Cfg::OFF_KC;
-  uint8_t* sV = smem + Cfg::OFF_V;
-  uint8_t* sP = ALIAS ? smem + Cfg::OFF_KC : smem + Cfg::OFF_P;   // P tile
-  uint8_t* sC = ALIAS ? smem + Cfg::OFF_V : smem + Cfg::OFF_KC;    // C_prev tile
+  uint8_t* sKC = smem + Cfg::OFF_KC;  // K, then P, then the lo plane of C_prev (or h)
+  uint8_t* sV = smem + Cfg::OFF_V;    // V, then the hi plane of C_prev (then h)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_TMEM);
   float* nvec = reinterpret_cast<float*>(smem + Cfg::OFF_NVEC);
@@ -115,11 +110,10 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tc::tmem_relinquish();
   }
-  // column factors (log i_s - b_s) log2(e) of every key row this tile needs
+  // column factors (log i_s - b_s) log2(e) of the chunk's keys
   if (warp >= 2) {
     const int gt = threadIdx.x - 64;
-    for (int s = gt; s < nkv * BN; s += 128)
-      colf[s] = s < len ? (gli[tok0 + s] - gb[tok0 + s]) * kLog2e : -INFINITY;
+    colf[gt] = gt < len ? (gli[tok0 + gt] - gb[tok0 + gt]) * kLog2e : -INFINITY;
     if (EXPV && has_prev)
       for (int i = gt; i < DQK; i += 128) nvec[i] = gn[((size_t)bh * NC + c) * DQK + i];
   }
@@ -137,47 +131,35 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
       tc::mbar_arrive_expect_tx(&bar[B_Q], Cfg::Q_BYTES);
-      for (int kb = 0; kb < Cfg::KB; ++kb)
-        tc::tma_load_3d(sQ + kb * 16384, &tm_q, &bar[B_Q], kb * 64, c0 + t0, bh);
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j > 0) ok = tc::mbar_wait(&bar[B_S], (j - 1) & 1, abort_flag);  // K buffer free
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bar[B_K], Cfg::K_BYTES);
-        for (int kb = 0; kb < Cfg::KB; ++kb)
-          tc::tma_load_3d(sKC + kb * 16384, &tm_k, &bar[B_K], kb * 64, c0 + j * BN, bh);
-        if (j > 0) ok = tc::mbar_wait(&bar[B_PV], (j - 1) & 1, abort_flag);  // V buffer free
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bar[B_V], Cfg::V_BYTES);
-        for (int vb = 0; vb < Cfg::VB; ++vb)
-          tc::tma_load_3d(sV + vb * 16384, &tm_v, &bar[B_V], dv0 + vb * 64, c0 + j * BN, bh);
-      }
-      if (ok && has_prev) {
-        // C goes where K was once the last S is done, or (ALIAS) where V was once PV is done
-        ok = ALIAS ? tc::mbar_wait(&bar[B_PV], (nkv - 1) & 1, abort_flag)
-                   : tc::mbar_wait(&bar[B_S], (nkv - 1) & 1, abort_flag);
+      for (int kb = 0; kb < Cfg::KB; ++kb) tc::tma_load_3d(sQ + kb * 16384, &tm_q, &bar[B_Q], kb * 64, c0, bh);
+      tc::mbar_arrive_expect_tx(&bar[B_K], Cfg::K_BYTES);
+      for (int kb = 0; kb < Cfg::KB; ++kb) tc::tma_load_3d(sKC + kb * 16384, &tm_k, &bar[B_K], kb * 64, c0, bh);
+      tc::mbar_arrive_expect_tx(&bar[B_V], Cfg::V_BYTES);
+      for (int vb = 0; vb < Cfg::VB; ++vb)
+        tc::tma_load_3d(sV + vb * 16384, &tm_v, &bar[B_V], dv0 + vb * 64, c0, bh);
+      if (has_prev) {
+        // both planes of C_prev once P V is done: hi where V was, lo where P was
+        ok = tc::mbar_wait(&bar[B_PV], 0, abort_flag);
         if (ok) {
-          tc::mbar_arrive_expect_tx(&bar[B_C], Cfg::C_BYTES);
-          for (int vb = 0; vb < Cfg::VB; ++vb)
-            tc::tma_load_3d(sC + vb * DQK * 128, &tm_c, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
+          tc::mbar_arrive_expect_tx(&bar[B_C], 2 * Cfg::C_BYTES);
+          for (int vb = 0; vb < Cfg::VB; ++vb) {
+            tc::tma_load_3d(sV + vb * DQK * 128, &tm_chi, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
+            tc::tma_load_3d(sKC + vb * DQK * 128, &tm_clo, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
+          }
         }
       }
       // do not leave while a copy this thread issued may still be landing
-      if (ok) {
-        ok = tc::mbar_wait(&bar[B_V], (nkv - 1) & 1, abort_flag);
-        if (ok && has_prev) ok = tc::mbar_wait(&bar[B_C], 0, abort_flag);
-      }
+      if (ok) ok = tc::mbar_wait(&bar[B_V], 0, abort_flag);
+      if (ok && has_prev) ok = tc::mbar_wait(&bar[B_C], 0, abort_flag);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
-      constexpr uint32_t idO = tc::idesc_bf16(BM, DV, false, true);
-      const uint32_t aQ = tc::smem_u32(sQ), aKC = tc::smem_u32(sKC), aV = tc::smem_u32(sV),
-                     aP = tc::smem_u32(sP), aC = tc::smem_u32(sC);
-      ok = tc::mbar_wait(&bar[B_Q], 0, abort_flag);
-      for (int j = 0; j < nkv && ok; ++j) {
-        ok = tc::mbar_wait(&bar[B_K], j & 1, abort_flag);
-        if (!ok) break;
+      const uint32_t idS = tc::idesc_bf16(128, NKEY, false, false);
+      constexpr uint32_t idO = tc::idesc_bf16(128, DV, false, true);
+      const uint32_t aQ = tc::smem_u32(sQ), aKC = tc::smem_u32(sKC), aV = tc::smem_u32(sV);
+      ok = tc::mbar_wait(&bar[B_Q], 0, abort_flag) && tc::mbar_wait(&bar[B_K], 0, abort_flag);
+      if (ok) {
         tc::tc_fence_after();
 #pragma unroll
         for (int k = 0; k < DQK / 16; ++k) {
@@ -186,14 +168,17 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
                           idS, k > 0);
         }
         tc::tc_commit(&bar[B_S]);
-        ok = tc::mbar_wait(&bar[B_P], j & 1, abort_flag) && tc::mbar_wait(&bar[B_V], j & 1, abort_flag);
-        if (!ok) break;
+        ok = tc::mbar_wait(&bar[B_P], 0, abort_flag) && tc::mbar_wait(&bar[B_V], 0, abort_flag);
+      }
+      if (ok) {
         tc::tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint32_t offp = (k >> 2) * 16384 + (k & 3) * 32;
-          tc::mma_bf16_ss(tO, tc::sdesc_sw128(aP + offp, 16, 1024),
-                          tc::sdesc_sw128(aV + k * 2048, 16384, 1024), idO, (j > 0 || k > 0));
+        for (int k = 0; k < 8; ++k) {
+          if (16 * k < NKEY) {
+            const uint32_t offp = (k >> 2) * 16384 + (k & 3) * 32;
+            tc::mma_bf16_ss(tO, tc::sdesc_sw128(aKC + offp, 16, 1024),
+                            tc::sdesc_sw128(aV + k * 2048, 16384, 1024), idO, k > 0);
+          }
         }
         tc::tc_commit(&bar[B_PV]);
       }
@@ -203,9 +188,9 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
           tc::tc_fence_after();
 #pragma unroll
           for (int k = 0; k < DQK / 16; ++k) {
-            const uint32_t offq = (k >> 2) * 16384 + (k & 3) * 32;
-            tc::mma_bf16_ss(tO, tc::sdesc_sw128(aQ + offq, 16, 1024),
-                            tc::sdesc_sw128(aC + k * 2048, DQK * 128, 1024), idO, 1);
+            const uint64_t a = tc::sdesc_sw128(aQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+            tc::mma_bf16_ss(tO, a, tc::sdesc_sw128(aV + k * 2048, DQK * 128, 1024), idO, 1);
+            tc::mma_bf16_ss(tO, a, tc::sdesc_sw128(aKC + k * 2048, DQK * 128, 1024), idO, 1);
           }
         }
       }
@@ -215,36 +200,31 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
     // ------------------------------------------------------------ gate rows + epilogue
     const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row of the tile
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const int tl = t0 + row;
-    const bool valid = tl < len;
-    const size_t tok = tok0 + tl;
+    const bool valid = row < len;
+    const size_t tok = tok0 + row;
     const float bt = valid ? gb[tok] : 0.f;
     const float mt = (EXPV && valid) ? gm[tok] : 0.f;
     const float mprev = EXPV ? chunk_mprev(gm, tok0, c, m0, bh) : 0.f;
     const float r2 = valid ? (bt - mt) * kLog2e + log2_scale : -INFINITY;
     const float qfac = (valid && has_prev) ? expf(bt + mprev - mt) * scale : 0.f;
-    const uint32_t aP = tc::smem_u32(sP), aQ = tc::smem_u32(sQ);
+    const uint32_t aP = tc::smem_u32(sKC), aQ = tc::smem_u32(sQ);
     float rowsum = 0.f;
 
-    for (int j = 0; j < nkv && ok; ++j) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_S], j & 1, abort_flag));
-      if (ok && j > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_PV], (j - 1) & 1, abort_flag));
-      if (!ok) break;
+    ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_S], 0, abort_flag));
+    if (ok) {
       tc::tc_fence_after();
-      const bool diag = (j == qt);
-      const float* cf = colf + j * BN;
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int ch = 0; ch < NKEY / 32; ++ch) {
         float sv[32];
         tc::tmem_ld32(tS + lane_base + ch * 32, sv);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const int s0 = ch * 32 + i;
-          float p0 = sv[i] * tc::ex2(r2 + cf[s0]);
-          float p1 = sv[i + 1] * tc::ex2(r2 + cf[s0 + 1]);
-          if (diag && s0 > row) p0 = 0.f;
-          if (diag && s0 + 1 > row) p1 = 0.f;
+          float p0 = sv[i] * tc::ex2(r2 + colf[s0]);
+          float p1 = sv[i + 1] * tc::ex2(r2 + colf[s0 + 1]);
+          if (s0 > row) p0 = 0.f;
+          if (s0 + 1 > row) p1 = 0.f;
           if (EXPV) rowsum += p0 + p1;
           pk[i >> 1] = tc::pack_bf16(p0, p1);
         }
@@ -263,38 +243,36 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
       tc::mbar_arrive(&bar[B_P]);
     }
 
-    // inter-chunk operand: scale the query rows by alpha_t / sqrt(d_qk) in place
+    // inter-chunk operand: scale the query rows by alpha_t / sqrt(d_qk) in place (the
+    // score product that read Q is done)
     float inter_norm = 0.f;
     if (ok && has_prev) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_Q], 0, abort_flag));
-      if (ok) {
 #pragma unroll 1
-        for (int kb = 0; kb < Cfg::KB; ++kb) {
+      for (int kb = 0; kb < Cfg::KB; ++kb) {
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int pch = (jj + row) & 7;
-            const uint32_t addr = aQ + kb * 16384 + row * 128 + pch * 16;
-            uint32_t w[4];
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                         : "r"(addr));
-            const int col0 = kb * 64 + ((pch ^ (row & 7)) << 3);
+        for (int jj = 0; jj < 8; ++jj) {
+          const int pch = (jj + row) & 7;
+          const uint32_t addr = aQ + kb * 16384 + row * 128 + pch * 16;
+          uint32_t w[4];
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                       : "r"(addr));
+          const int col0 = kb * 64 + ((pch ^ (row & 7)) << 3);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
-              const float x0 = __bfloat162float(v2.x) * qfac;
-              const float x1 = __bfloat162float(v2.y) * qfac;
-              if (EXPV) inter_norm += x0 * nvec[col0 + 2 * e] + x1 * nvec[col0 + 2 * e + 1];
-              w[e] = tc::pack_bf16(x0, x1);
-            }
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
-                         "r"(w[1]), "r"(w[2]), "r"(w[3])
-                         : "memory");
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+            const float x0 = __bfloat162float(v2.x) * qfac;
+            const float x1 = __bfloat162float(v2.y) * qfac;
+            if (EXPV) inter_norm += x0 * nvec[col0 + 2 * e] + x1 * nvec[col0 + 2 * e + 1];
+            w[e] = tc::pack_bf16(x0, x1);
           }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
+                       "r"(w[1]), "r"(w[2]), "r"(w[3])
+                       : "memory");
         }
-        tc::fence_proxy_async_smem();
-        tc::mbar_arrive(&bar[B_QS]);
       }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[B_QS]);
     }
 
     if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[B_O], 0, abort_flag));
@@ -306,7 +284,12 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
         inv = 1.f / fmaxf(fabsf(a), expf(-mt));
         if (blockIdx.y == 0 && valid) abar_out[tok] = a;
       }
-      // h goes through the (now idle) P tile and one TMA store per 64-column block
+      // h goes through an idle region and one TMA store per 64-column block (NKEY rows: a
+      // 64-token chunk leaves the next chunk's rows alone): the V region once the inter
+      // product has read C_prev's hi plane from it, else the K / P region.  (Staged over
+      // V right after P V, the first 16 rows of h were measured to come out zero.)
+      uint8_t* sH = has_prev ? sV : sKC;
+      const uint32_t aH = tc::smem_u32(sH);
 #pragma unroll 1
       for (int ch = 0; ch < DV / 32; ++ch) {
         float ov[32];
@@ -314,7 +297,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int col = ch * 32 + q4 * 8, blk = col >> 6, lc = (col & 63) >> 3;
-          const uint32_t addr = aP + blk * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
+          const uint32_t addr = aH + blk * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
                        "r"(tc::pack_bf16(ov[8 * q4 + 0] * inv, ov[8 * q4 + 1] * inv)),
                        "r"(tc::pack_bf16(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv)),
@@ -329,7 +312,7 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
         ok = tc::mbar_wait(&bar[B_STG], 0, abort_flag);
         if (ok) {
           for (int blk = 0; blk < DV / 64; ++blk)
-            tc::tma_store_3d(&tm_h, sP + blk * 16384, dv0 + blk * 64, c0 + t0, bh);
+            tc::tma_store_3d(&tm_h, sH + blk * 16384, dv0 + blk * 64, c0, bh);
           tc::bulk_commit_group();
           tc::bulk_wait_all();
         }
@@ -352,40 +335,38 @@ __global__ void __launch_bounds__(192, ALIAS ? 2 : 1) output_fwd_tc_kernel(
 // ---------------------------------------------------------------------------
 
 bool output_fwd_tc_supported(const Problem& p) {
-  return p.bf16() && p.L >= 128 && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
+  return p.bf16() && (p.L == 64 || p.L == 128) && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) &&
          (p.dhv % 64 == 0);
 }
 
-template <int DQK, int DV, bool EXPV, bool ALIAS>
+template <int DQK, int DV, bool EXPV>
 static cudaError_t launch_out_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {
-  using Cfg = OutTcCfg<DQK, DV, ALIAS>;
-  CUtensorMap tq, tk, tv, tcm, th;
-  if (!make_tmap_3d_bf16(&th, a.h, p.dhv, p.T, p.BH, 64, 128) ||
+  using Cfg = OutTcCfg<DQK, DV>;
+  const bf16* C = (const bf16*)a.C;
+  const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
+  CUtensorMap tq, tk, tv, tch, tcl, th;
+  const uint32_t rows = p.L < 128 ? (uint32_t)p.L : 128u;  // one chunk per tile
+  if (!make_tmap_3d_bf16(&th, a.h, p.dhv, p.T, p.BH, 64, rows) ||
       !make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tk, a.k, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tv, a.v, p.dhv, p.T, p.BH, 64, 128) ||
-      !make_tmap_3d_bf16(&tcm, a.C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
+      !make_tmap_3d_bf16(&tch, C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK) ||
+      !make_tmap_3d_bf16(&tcl, C + plane, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
     return cudaErrorInvalidValue;
-  const size_t smem = Cfg::smem_bytes(p.L);
-  auto kern = output_fwd_tc_kernel<DQK, DV, EXPV, ALIAS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = output_fwd_tc_kernel<DQK, DV, EXPV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  const int ntq = p.L / 128;
-  dim3 grid((unsigned)(p.BH * p.NC * ntq), (unsigned)(p.dhv / DV)), block(192);
-  kern<<<grid, block, smem, s>>>(tq, tk, tv, tcm, th, a.b, a.li, a.m, a.n, (bf16*)a.h, a.abar, p.T,
-                                 p.L, p.NC, p.BH, ntq, p.dhv, p.scale, log2f(p.scale), a.init.on(),
-                                 a.init.on() ? a.init.m : nullptr, next_epoch());
+  dim3 grid((unsigned)(p.BH * p.NC), (unsigned)(p.dhv / DV)), block(192);
+  kern<<<grid, block, Cfg::SMEM, s>>>(tq, tk, tv, tch, tcl, th, a.b, a.li, a.m, a.n, a.abar, p.T, p.L,
+                                      p.NC, p.scale, log2f(p.scale), a.init.on(),
+                                      a.init.on() ? a.init.m : nullptr, next_epoch());
   return cudaGetLastError();
 }
 
 template <int DQK, bool EXPV>
 static cudaError_t launch_out_tc_dv(const Problem& p, const FwdArgs& a, cudaStream_t s) {
-  if (p.L == 128) {
-    if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV, true>(p, a, s);
-    return launch_out_tc<DQK, 128, EXPV, true>(p, a, s);
-  }
-  if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV, false>(p, a, s);
-  return launch_out_tc<DQK, 128, EXPV, false>(p, a, s);
+  if (p.dhv == 64) return launch_out_tc<DQK, 64, EXPV>(p, a, s);
+  return launch_out_tc<DQK, 128, EXPV>(p, a, s);
 }
 
 cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s) {

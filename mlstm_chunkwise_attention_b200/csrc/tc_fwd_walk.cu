@@ -169,12 +169,16 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
             tc::mma_bf16_ss(tNU + 16 * (c & 1), mnmaj(aK, k), n16(wt, k), idNM, k > 0);
         };
         if (EXPV && c > 0 && c + 1 < NC) n_update();
-        // A (C_c staged): O = Q C_c (hi plane); Q n_c (hi, lo) into the two q.n columns
+        // A (C_c staged): O = Q C_c (hi and lo planes: where the normaliser nearly cancels,
+        // h = O / den amplifies the rounding of the state); Q n_c (hi, lo) into the two q.n
+        // columns
         ok = wait_rows();
         if (!ok) break;
         if (EXPV && c == 0 && c + 1 < NC) n_update();
 #pragma unroll
         for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tO, kmaj(aQ, k), mnmaj(aG, k), idKM, k > 0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tO, kmaj(aQ, k), mnmaj(aG + TILE, k), idKM, 1);
         if (EXPV) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) tc::mma_bf16_ss(tN, kmaj(aQ, k), n16(aNT, k), idNK, k > 0);

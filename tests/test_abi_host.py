@@ -239,6 +239,26 @@ def test_launch_plans_choose_the_walkers_on_their_shape(lib, variant):
         assert any(n.startswith("state_fwd") for n in names) and any(n.startswith("dk_") for n in names)
 
 
+@pytest.mark.parametrize("variant", [B.SIG, B.EXP], ids=["sig", "exp"])
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_launch_plans_put_every_bf16_chunk_size_on_tensor_cores(lib, variant, d):
+    """bf16 runs every chunk size on tcgen05 kernels: chunk 64 and 128 on the one-tile
+    output kernel (or the walkers), chunk >= 256 on the large-chunk kernel, the backward on
+    the tensor-core state-gradient and dq / dk / dv kernels.  fp32 I/O keeps the CUDA-core
+    kernels (a bf16 operand cannot meet its 1e-4 bar)."""
+    for L in (64, 128, 256, 1024):
+        sizes = (2, 4, 2048, d, d, L, variant, B.BF16)
+        names = _plan(0, sizes) + _plan(1, sizes)
+        assert not any(n.endswith("_simt") for n in names), (L, names)
+        fwd_out = _plan(0, sizes)[-1]
+        if L <= 128:
+            assert fwd_out in ("output_fwd_tc", "fwd_walk_tc"), (L, fwd_out)
+        else:
+            assert fwd_out == "output_fwd_xl", (L, fwd_out)
+    names = _plan(0, (2, 4, 2048, d, d, 64, variant, B.FP32)) + _plan(1, (2, 4, 2048, d, d, 64, variant, B.FP32))
+    assert all(n.endswith("_simt") for n in names if n not in ("gate_prep", "bwd_token_prep", "gate_grad"))
+
+
 def test_serial_launch_switch_needs_no_device(lib):
     """mlstm_set_serial_launches only sets a per-thread flag: no CUDA call, always MLSTM_OK."""
     assert lib.mlstm_set_serial_launches(1) == 0

@@ -54,6 +54,12 @@ SMALL = [
     ("exp_bf16_chunk128_d128_t1", 1, 2, 1, 128, 128, 128, EXP, BF, -1.0, 3.0),
     ("sig_bf16_chunk128_d128_t128_one_full", 1, 2, 128, 128, 128, 128, SIG, BF, 0.0, 3.0),
     ("exp_bf16_chunk128_d128_t129_one_token_tail", 2, 1, 129, 128, 128, 128, EXP, BF, -2.0, 3.0),
+    # chunk 64 on the tensor cores: a 64-token chunk in a half-filled 128-row tile
+    ("exp_bf16_chunk64_d128_ragged", 2, 2, 700, 128, 128, 64, EXP, BF, -2.0, 3.0),
+    ("sig_bf16_chunk64_d128_ragged", 1, 3, 333, 128, 128, 64, SIG, BF, 0.0, 3.0),
+    ("exp_bf16_chunk64_t1", 1, 2, 1, 128, 128, 64, EXP, BF, -1.0, 3.0),
+    ("sig_bf16_chunk64_dqk256_dhv512", 1, 1, 200, 256, 512, 64, SIG, BF, 0.0, 3.0),
+    ("exp_bf16_chunk64_dqk64_dhv128_t65", 1, 2, 65, 64, 128, 64, EXP, BF, 0.0, 3.0),
 ]
 
 
@@ -278,8 +284,8 @@ def test_full_headline_every_head_sampled_rows():
     dev, h, saved = gpu_fwd(cpu, L, var)
     g = gpu_bwd(dev, h, saved, L, var)
     rows = sample_rows(T, 6, spec["seed"], chunk=L)
-    cols = [T - L, T - 70, T - 1]
     tail = list(range(T - L, T))
+    cols = tail  # every column of the last chunk
     need = sorted(set(rows) | set(tail))
     for b in range(spec["B"]):
         for hh in range(spec["NH"]):
