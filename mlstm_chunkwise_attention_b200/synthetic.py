@@ -50,12 +50,15 @@ def torch_dtype(name):
 
 
 def make_inputs(B, NH, T, d_qk, d_hv, *, seed, igate_mean=0.0, fgate_mean=3.0,
-                igate_std=1.0, fgate_std=1.0, dtype=torch.bfloat16, with_dh=False):
-    """Draw q, k, v [B,NH,T,d], gate preactivations [B,NH,T] (and dh) on the CPU."""
+                igate_std=1.0, fgate_std=1.0, qk_mean=0.0, dtype=torch.bfloat16, with_dh=False):
+    """Draw q, k, v [B,NH,T,d], gate preactivations [B,NH,T] (and dh) on the CPU.
+
+    q and k are N(qk_mean, 1); everything else as in the module docstring.
+    """
     g = torch.Generator().manual_seed(int(seed))
     out = {}
-    out["q"] = torch.randn(B, NH, T, d_qk, generator=g).to(dtype)
-    out["k"] = torch.randn(B, NH, T, d_qk, generator=g).to(dtype)
+    out["q"] = (torch.randn(B, NH, T, d_qk, generator=g) + qk_mean).to(dtype)
+    out["k"] = (torch.randn(B, NH, T, d_qk, generator=g) + qk_mean).to(dtype)
     out["v"] = torch.randn(B, NH, T, d_hv, generator=g).to(dtype)
     out["igate"] = (torch.randn(B, NH, T, generator=g) * igate_std + igate_mean).to(dtype)
     out["fgate"] = (torch.randn(B, NH, T, generator=g) * fgate_std + fgate_mean).to(dtype)

@@ -36,6 +36,10 @@ Readings taken where the pages are silent (one per item):
 3. No epsilon is added to the normaliser.
 4. On a normaliser tie |a_t| == 1 the constant branch is taken (zero gradient).
 5. The stabiliser carries no gradient (the output does not depend on it).
+6. The backward receives the forward's output h as one of its inputs, in the
+   I/O dtype like q, k, v and the gates.  The normaliser's gradient,
+   da_t = -(dh_t . h_t) sign(a_t) / den_t, is evaluated with that h: the
+   backward functions take it as ``h_in`` (None: the exact fp64 h).
 """
 
 import numpy as np
@@ -342,8 +346,8 @@ def _output_grads(dh, h, a, den, variant, floor=1.0):
     return dnum, da
 
 
-def parallel_backward(q, k, v, log_i, log_f, variant, dh):
-    """Gradients of sum(dh * h) through the parallel form (readings 4, 5).
+def parallel_backward(q, k, v, log_i, log_f, variant, dh, h_in=None):
+    """Gradients of sum(dh * h) through the parallel form (readings 4, 5, 6).
 
     dA_ts = dnum_t . v_s + da_t;  dq'_t = sum_s dA_ts D_ts k_s;
     dk_s = sum_t dA_ts D_ts q'_t;  dv_s = sum_t A_ts dnum_t;
@@ -356,7 +360,8 @@ def parallel_backward(q, k, v, log_i, log_f, variant, dh):
     fwd = parallel_forward(q, k, v, log_i, log_f, variant)
     A = fwd["A"]
     D = np.exp(parallel_log_decay(log_i, log_f))
-    dnum, da = _output_grads(dh, fwd["h"], fwd["a"], fwd["den"], variant)
+    h_used = fwd["h"] if h_in is None else np.asarray(h_in, dtype=np.float64)
+    dnum, da = _output_grads(dh, h_used, fwd["a"], fwd["den"], variant)
     dA = dnum @ v.T + da[:, None]
     dA = np.tril(dA)
     dS = dA * D
@@ -420,7 +425,7 @@ def recurrent_backward(q, k, v, log_i, log_f, variant, dh):
             "dlog_i": di * i, "dlog_f": df * f, "h": h}
 
 
-def chunkwise_backward(q, k, v, log_i, log_f, variant, L, dh):
+def chunkwise_backward(q, k, v, log_i, log_f, variant, L, dh, h_in=None):
     """Gradients of sum(dh * h) in the chunkwise order, fp64 (no [T, T] matrices).
 
     Uses the forward's chunk quantities (chunkwise_forward) with the max state
@@ -449,7 +454,8 @@ def chunkwise_backward(q, k, v, log_i, log_f, variant, L, dh):
     dnum = dh / den[:, None]
     if exp_variant:
         active = np.abs(f["abar"]) > np.exp(-m_row)
-        da = np.where(active, -np.sum(dh * f["h"], axis=1) * np.sign(f["abar"]) / den, 0.0)
+        h_used = f["h"] if h_in is None else np.asarray(h_in, dtype=np.float64)  # reading 6
+        da = np.where(active, -np.sum(dh * h_used, axis=1) * np.sign(f["abar"]) / den, 0.0)
     else:
         da = np.zeros(T)
 

@@ -53,8 +53,18 @@ def oracle_fwd_head(x, chunk, variant):
     return oracle.chunkwise_forward(x["q"], x["k"], x["v"], li, lf, variant, chunk)
 
 
-def oracle_bwd_head(x, variant):
+def io_round(a, dtype):
+    """a rounded to the I/O dtype, as a tensor of that dtype would hold it."""
+    return torch.from_numpy(np.asarray(a, dtype=np.float64)).to(dtype).double().numpy()
+
+
+def oracle_bwd_head(x, variant, dtype=None):
+    """Parallel-form backward of one head.  With dtype (the I/O dtype), the backward's h
+    input is the oracle's own forward output rounded to it, as the boundary passes h."""
     li, lf = oracle.gate_logs(x["igate"], x["fgate"], variant)
-    g = oracle.parallel_backward(x["q"], x["k"], x["v"], li, lf, variant, x["dh"])
+    h_in = None
+    if dtype is not None:
+        h_in = io_round(oracle.parallel_forward(x["q"], x["k"], x["v"], li, lf, variant)["h"], dtype)
+    g = oracle.parallel_backward(x["q"], x["k"], x["v"], li, lf, variant, x["dh"], h_in=h_in)
     di, df = oracle.preact_grads(g["dlog_i"], g["dlog_f"], x["igate"], x["fgate"], variant)
     return {"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "digate_pre": di, "dfgate_pre": df}

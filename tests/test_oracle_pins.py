@@ -481,3 +481,29 @@ def test_unmutated_copy_passes_every_check():
     M = _mutant("SIG = 0", "SIG = 0")
     for check in ALL_CHECKS:
         check(M)
+
+
+@pytest.mark.parametrize("variant", [SIG, EXP])
+def test_backward_forms_agree_for_a_given_h_input(variant):
+    """Reading 6: the backward takes the output h as an input.  For any h_in (here the
+    exact h perturbed by a relative 1e-3), the parallel and chunkwise backward forms use
+    it in the normaliser gradient alike and agree; h_in = the exact h reproduces the
+    default; and for mLSTMsig (no normaliser) h_in changes nothing."""
+    rng = np.random.default_rng(61)
+    T, d, L = 45, 8, 8
+    q, k, v, dh = (rng.standard_normal((T, d)) for _ in range(4))
+    li, lf = oracle.gate_logs(rng.standard_normal(T) - 1.0, rng.standard_normal(T) + 2.0, variant)
+    h = oracle.parallel_forward(q, k, v, li, lf, variant)["h"]
+    h_in = h * (1.0 + 1e-3 * rng.standard_normal(h.shape))
+    p = oracle.parallel_backward(q, k, v, li, lf, variant, dh, h_in=h_in)
+    c = oracle.chunkwise_backward(q, k, v, li, lf, variant, L, dh, h_in=h_in)
+    for key in ("dq", "dk", "dv", "dlog_i", "dlog_f"):
+        np.testing.assert_allclose(c[key], p[key], rtol=1e-9, atol=1e-11)
+    same = oracle.parallel_backward(q, k, v, li, lf, variant, dh, h_in=h)
+    dflt = oracle.parallel_backward(q, k, v, li, lf, variant, dh)
+    for key in ("dq", "dk", "dv", "dlog_i", "dlog_f"):
+        np.testing.assert_array_equal(same[key], dflt[key])
+        if variant == SIG:
+            np.testing.assert_allclose(p[key], dflt[key], rtol=1e-12, atol=1e-14)
+    if variant == EXP:  # the perturbation reaches the gradients through da only
+        assert np.max(np.abs(p["dq"] - dflt["dq"])) > 0
