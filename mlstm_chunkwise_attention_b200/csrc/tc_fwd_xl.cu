@@ -10,13 +10,16 @@
 // chunk, value block), taken in balanced pairs of query tiles):
 //  * warp 0 streams Q tiles (double-buffered) and, per step, K_j or the
 //    chunk's entering state C_prev through a ring whose stages free as soon
-//    as their score product is done; warp 10 streams V_j with the key
+//    as their score product is done; warp 18 streams V_j with the key
 //    tile's gate factors through a second ring (TMA and bulk copies, no
 //    multicast);
 //  * warp 1 issues tcgen05.mma: S_{g+1} before P_g V_g, so the tensor core
 //    computes the next score tile while the gate transform runs;
-//  * warps 2-9 (two warpgroups, one per 64-key half of a tile) turn S into P
-//    in TMEM in place (bf16, two per column), and P V reads P straight from
+//  * warps 2-17 (four warpgroups, one per 32-key block of a tile; four
+//    warps per SM sub-partition, so the latency of one warp's TMEM traffic
+//    and exp2 is hidden by the others) turn S into P in TMEM in place (bf16,
+//    two per column, each block packed into the first half of its own 32
+//    columns, which no other warp reads), and P V reads P straight from
 //    TMEM.  The inter-chunk term is one more step of the same kind: the
 //    transform writes alpha_t q_t / sqrt(d_qk) into the S buffer and the
 //    tensor core multiplies it by C_prev, so it lands in the same
@@ -58,10 +61,10 @@ struct XlCfg {
   static constexpr int OFF_V = OFF_K + NK * K_BYTES;
   static constexpr int OFF_ROW = OFF_V + NV * V_BYTES;
   static constexpr int OFF_COL = OFF_ROW + NQ * ROWAUX;
-  static constexpr int OFF_XS = OFF_COL + NV * COLAUX;  // [2 O buffers][2 halves][128] floats
-  static constexpr int OFF_STG = OFF_XS + 2 * 2 * 128 * 4;  // per transform warp: 16 rows of h
-  static constexpr int STG_WARP = 16 * DV;                     // 16 rows x DV / 2 bf16
-  static constexpr int OFF_BAR = OFF_STG + 8 * STG_WARP;
+  static constexpr int OFF_XS = OFF_COL + NV * COLAUX;  // [2 O buffers][4 key blocks][128] floats
+  static constexpr int OFF_STG = OFF_XS + 2 * 4 * 128 * 4;  // per transform warp: 16 rows of h
+  static constexpr int STG_WARP = 8 * DV;                      // 16 rows x DV / 4 bf16
+  static constexpr int OFF_BAR = OFF_STG + 16 * STG_WARP;
   static constexpr int OFF_TMEM = OFF_BAR + 64 * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;         // S0 [0,128) S1 [128,256) O0, O1 from 256
@@ -86,7 +89,9 @@ enum {
   X_COUNT = 40
 };
 
-constexpr int kXlThreads = 352;  // K producer, MMA, 8 transform warps, V producer
+constexpr int kXlThreads = 608;    // K producer, MMA, 16 transform warps, V producer
+constexpr int kXlTransform = 512;  // transform threads (warps 2..17)
+constexpr int kXlVWarp = 18;       // V producer warp
 
 struct XlItem {
   int qt, bh, c, vb, t0, len, nkv;
@@ -130,7 +135,7 @@ __device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB
 }  // namespace
 
 // Epilogue of one SIG work item (no normaliser, h = O) for the transform
-// thread of row 32 qr + lane and key half h: read O out of TMEM, freeing it
+// thread of row 32 qr + lane and column quarter h (DV / 4 columns): read O out of TMEM, freeing it
 // for the next item's products, and store h through a staging slot so each
 // store instruction writes whole row segments.  Kept out of line so its
 // registers do not count against the gate transform it is called from.
@@ -152,19 +157,22 @@ __device__ __noinline__ bool xl_epilogue(int it, int vb, int nvalid, size_t tok,
   (void)abar_out;
   if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + ob], par, abort_flag))) return false;
   tc::tc_fence_after();
-  const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 2);
-  // this thread's DV / 2 columns as CPR 16-byte chunks, read 32 columns at a time
-  constexpr int CPR = DV / 16, RPI = 32 / CPR;
+  const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 4);
+  // this thread's DV / 4 columns as CPR 16-byte chunks
+  constexpr int CPR = DV / 32, RPI = 32 / CPR;
   uint4 w[CPR];
-#pragma unroll
-  for (int q = 0; q < DV / 64; ++q) {
+  {
     uint32_t o[32];
-    tc::tmem_ld32_async(tO + 32 * q, o);
-    tc::tmem_wait_ld(o);
+    if (DV >= 128) {
+      tc::tmem_ld32_async(tO, o);
+      tc::tmem_wait_ld(o);
+    } else {
+      tc::tmem_ld16(tO, o);
+    }
 #pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
+    for (int c4 = 0; c4 < CPR; ++c4) {
       const uint32_t* r = &o[8 * c4];
-      uint4& d = w[4 * q + c4];
+      uint4& d = w[c4];
       d.x = tc::pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
       d.y = tc::pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
       d.z = tc::pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
@@ -200,7 +208,7 @@ __device__ __noinline__ bool xl_epilogue(int it, int vb, int nvalid, size_t tok,
       const int rw = 16 * rnd + rr;  // row within this warp's 32
       if (rw < nvalid)
         *reinterpret_cast<uint4*>(hout + (tok - lane + rw) * (size_t)dhv + vb * DV +
-                                  h * (DV / 2) + 8 * c) = v;
+                                  h * (DV / 4) + 8 * c) = v;
     }
     __syncwarp();
   }
@@ -231,9 +239,9 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
   if (threadIdx.x == 0) {
     for (int i = 0; i < X_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == X_QE0 || i == X_QE0 + 1) cnt = 257;
-      if (i >= X_PF0 && i < X_PF0 + 4) cnt = 256;
-      if (i >= X_OE0 && i < X_XS0 + 2) cnt = 256;
+      if (i == X_QE0 || i == X_QE0 + 1) cnt = kXlTransform + 1;
+      if (i >= X_PF0 && i < X_PF0 + 4) cnt = kXlTransform;
+      if (i >= X_OE0 && i < X_XS0 + 2) cnt = kXlTransform;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -305,7 +313,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
         ++it;
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == kXlVWarp) {
     // ------------------------------------------------------------ V producer
     // Per key tile the V tile and the tile's gate factors (CC, KP of its 128
     // keys and the four 32-key block maxima).
@@ -397,8 +405,9 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           if (leader) {
 #pragma unroll
             for (int k = 0; k < DQK / 16; ++k) {  // 16 rows of C_prev
-              const int h = k / (DQK / 32), kk = k % (DQK / 32);
-              tc::mma_bf16_ts(tO, tP + 64 * h + 8 * kk, tc::sdesc_sw128(aC + k * 2048, DQK * 128, 1024),
+              // the q elements of block g = k / (DQK / 64) sit packed at column 32 g
+              const int g = k / (DQK / 64), kk = k % (DQK / 64);
+              tc::mma_bf16_ts(tO, tP + 32 * g + 8 * kk, tc::sdesc_sw128(aC + k * 2048, DQK * 128, 1024),
                               idO, k > 0);
             }
             tc::tc_commit(&bar[X_KE0 + kst]);
@@ -410,8 +419,8 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           const int vst = gv % NV;
           const uint32_t aV = aV0 + vst * Cfg::V_BYTES;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)  // 16 keys per step; keys 64 h .. of P live at column 64 h
-            tc::mma_bf16_ts(tO, tP + 64 * (k >> 2) + 8 * (k & 3),
+          for (int k = 0; k < 8; ++k)  // 16 keys per step; keys 32 g .. of P live at column 32 g
+            tc::mma_bf16_ts(tO, tP + 32 * (k >> 1) + 8 * (k & 1),
                             tc::sdesc_sw128(aV + k * 2048, 16384, 1024), idO, (s > 0 || k > 0));
           tc::tc_commit(&bar[X_VE0 + vst]);
         }
@@ -456,7 +465,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     }
   } else {
     // ------------------------------------------------------------ gate transform + epilogue
-    const int h = (warp - 2) >> 2;  // 64-key half of each tile this warpgroup owns
+    const int h = (warp - 2) >> 2;  // this warpgroup's 32-key block of each tile (and DV / 4 h columns)
     const int qr = warp & 3;        // TMEM lane quarter = 32-row block of the tile
     const int row = 32 * qr + lane;
     const uint32_t lb = (uint32_t)(32 * qr) << 16;
@@ -476,40 +485,40 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       if (!EXPV)
         return xl_epilogue<DQK, DV, EXPV>(e.it, e.vb, e.nvalid, e.tok, e.fl, e.part, h, qr, lane, tmem,
                                           smem, hout, abar_out, dhv, abort_flag);
-      // EXP: den_t = max(|a_t|, exp(-m_t)), a_t the sum of both halves' shares
+      // EXP: den_t = max(|a_t|, exp(-m_t)), a_t the sum of the four key blocks' shares (added
+      // in block order, so the four threads of a row agree)
       const int ob = e.it & 1, par = (e.it >> 1) & 1;
       const bool valid = lane < e.nvalid;
-      float* x = xs + ob * 256;
+      float* x = xs + ob * 512;
       x[h * 128 + row] = e.part;
       tc::mbar_arrive(&bar[X_XS0 + ob]);
       if (!__all_sync(full, tc::mbar_wait(&bar[X_XS0 + ob], par, abort_flag))) return false;
-      const float a = e.part + x[(1 - h) * 128 + row];
+      const float a = ((x[row] + x[128 + row]) + x[256 + row]) + x[384 + row];
       const float inv = 1.f / fmaxf(fabsf(a), e.fl);
       if (h == 0 && e.vb == 0 && valid) abar_out[e.tok] = a;
       if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + ob], par, abort_flag))) return false;
       tc::tc_fence_after();
-      const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 2);
-      uint4* dst = reinterpret_cast<uint4*>(hout + e.tok * (size_t)dhv + e.vb * DV + h * (DV / 2));
-#pragma unroll
-      for (int q = 0; q < DV / 64; ++q) {
-        uint32_t o[32];
-        tc::tmem_ld32_async(tO + 32 * q, o);
+      const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 4);
+      uint32_t o[32];
+      if (DV >= 128) {
+        tc::tmem_ld32_async(tO, o);
         tc::tmem_wait_ld(o);
-        if (q == DV / 64 - 1) {
-          tc::tc_fence_before();
-          tc::mbar_arrive(&bar[X_OE0 + ob]);
-        }
-        if (valid) {
+      } else {
+        tc::tmem_ld16(tO, o);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bar[X_OE0 + ob]);
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(hout + e.tok * (size_t)dhv + e.vb * DV + h * (DV / 4));
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            const uint32_t* r = &o[8 * c8];
-            uint4 w;
-            w.x = tc::pack_bf16(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
-            w.y = tc::pack_bf16(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
-            w.z = tc::pack_bf16(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
-            w.w = tc::pack_bf16(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
-            dst[4 * q + c8] = w;
-          }
+        for (int c8 = 0; c8 < DV / 32; ++c8) {
+          const uint32_t* r = &o[8 * c8];
+          uint4 w;
+          w.x = tc::pack_bf16(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
+          w.y = tc::pack_bf16(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
+          w.z = tc::pack_bf16(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
+          w.w = tc::pack_bf16(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
+          dst[c8] = w;
         }
       }
       return true;
@@ -523,43 +532,40 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       if (!ok) break;
       const float* rp = reinterpret_cast<const float*>(smem + Cfg::OFF_ROW + qb * Cfg::ROWAUX);
       const float R = rp[row], QFt = rp[128 + row], FLt = rp[256 + row];
-      uint64_t part2 = tc::f2_make(0.f, 0.f);  // EXP: this half's share of the normaliser
+      uint64_t part2 = tc::f2_make(0.f, 0.f);  // EXP: this block's share of the normaliser
       const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
       for (int s = 0; s < nsteps && ok; ++s, ++g) {
         const int sb = g & 1;
         ok = __all_sync(full, tc::mbar_wait(&bar[X_SF0 + sb], (g >> 1) & 1, abort_flag));
         if (!ok) break;
         tc::tc_fence_after();
-        const uint32_t tS = tmem + sb * 128 + lb + 64 * h;
+        const uint32_t tS = tmem + sb * 128 + lb + 32 * h;
         if (I.pseudo && s == 0) {
-          // alpha_t q_t / sqrt(d_qk), this half's d_qk / 2 columns, into the S buffer
+          // alpha_t q_t / sqrt(d_qk) over this block's d_qk / 4 elements, packed into the S buffer
           const uint8_t* sq = smem + Cfg::OFF_Q + qb * Cfg::Q_BYTES;
           const float* nvec = rp + 384;
-          constexpr int NCH = DQK / 16;  // 16-byte chunks in half a row
+          constexpr int NCH = DQK / 32;  // 16-byte chunks of the block's q elements
+          uint32_t w[16];
 #pragma unroll
-          for (int grp = 0; grp < NCH / 4; ++grp) {  // 32 columns -> 16 TMEM columns
-            uint32_t w[16];
+          for (int ci = 0; ci < NCH; ++ci) {
+            const int gc = h * NCH + ci, kb = gc >> 3, lc = gc & 7;
+            const uint32_t addr = tc::smem_u32(sq) + kb * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
+            uint32_t q4[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(q4[0]), "=r"(q4[1]), "=r"(q4[2]), "=r"(q4[3])
+                         : "r"(addr));
 #pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-              const int ci = 4 * grp + cq;
-              const int gc = h * NCH + ci, kb = gc >> 3, lc = gc & 7;
-              const uint32_t addr = tc::smem_u32(sq) + kb * 16384 + row * 128 + ((lc ^ (row & 7)) << 4);
-              uint32_t q4[4];
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(q4[0]), "=r"(q4[1]), "=r"(q4[2]), "=r"(q4[3])
-                           : "r"(addr));
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&q4[e]);
-                const float x0 = __bfloat162float(v2.x) * QFt, x1 = __bfloat162float(v2.y) * QFt;
-                if (EXPV) {
-                  const float2 n2 = *reinterpret_cast<const float2*>(nvec + gc * 8 + 2 * e);
-                  part2 = tc::f2_add(part2, tc::f2_mul(tc::f2_make(x0, x1), tc::f2_make(n2.x, n2.y)));
-                }
-                w[cq * 4 + e] = tc::pack_bf16(x0, x1);
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&q4[e]);
+              const float x0 = __bfloat162float(v2.x) * QFt, x1 = __bfloat162float(v2.y) * QFt;
+              if (EXPV) {
+                const float2 n2 = *reinterpret_cast<const float2*>(nvec + gc * 8 + 2 * e);
+                part2 = tc::f2_add(part2, tc::f2_mul(tc::f2_make(x0, x1), tc::f2_make(n2.x, n2.y)));
               }
+              w[(ci & 3) * 4 + e] = tc::pack_bf16(x0, x1);
             }
-            tc::tmem_st16_async(tS + 16 * grp, w);
+            if (NCH == 2 && ci == 1) tc::tmem_st8_async(tS, w);
+            if (NCH >= 4 && (ci & 3) == 3) tc::tmem_st16_async(tS + 16 * (ci >> 2), w);
           }
           // P signals the MMA thread that C_prev has landed as well
           ok = __all_sync(full, tc::mbar_wait(&bar[X_KF0 + g % NK], (g / NK) & 1, abort_flag));
@@ -574,55 +580,50 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           ok = __all_sync(full, tc::mbar_wait(&bar[X_VF0 + vst], vpar, abort_flag));
           if (!ok) break;
           const float* cp = reinterpret_cast<const float*>(smem + Cfg::OFF_COL + vst * Cfg::COLAUX);
-          uint32_t sa[32], sb2[32];
-          tc::tmem_ld32_async(tS, sa);
-          tc::tmem_ld32_async(tS + 32, sb2);
-          tc::tmem_wait_ld(sa);
-          tc::reg_fence(sb2);
+          uint32_t sv[32];
+          tc::tmem_ld32_async(tS, sv);
+          tc::tmem_wait_ld(sv);
+          const int cc = h;  // this warp's 32-key block of the tile
+          uint32_t w[16];
+          if (!diag || cc < qr) {
+            // the whole block lies before this row: separable factors
+            const float rho = tc::ex2(R + cp[256 + cc]);
+            const uint64_t rho2 = tc::f2_make(rho, rho);
+            const float* kp = cp + 128 + 32 * cc;
 #pragma unroll
-          for (int cl = 0; cl < 2; ++cl) {
-            const int cc = 2 * h + cl;  // 32-key block of the tile
-            const uint32_t* sv = cl == 0 ? sa : sb2;
-            uint32_t w[16];
-            if (!diag || cc < qr) {
-              // the whole block lies before this row: separable factors
-              const float rho = tc::ex2(R + cp[256 + cc]);
-              const uint64_t rho2 = tc::f2_make(rho, rho);
-              const float* kp = cp + 128 + 32 * cc;
-#pragma unroll
-              for (int e = 0; e < 32; e += 4) {
-                const float4 k4 = *reinterpret_cast<const float4*>(kp + e);
-                const uint64_t p0 = tc::f2_mul(
-                    tc::f2_mul(tc::f2_make(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
-                               tc::f2_make(k4.x, k4.y)), rho2);
-                const uint64_t p1 = tc::f2_mul(
-                    tc::f2_mul(tc::f2_make(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
-                               tc::f2_make(k4.z, k4.w)), rho2);
-                if (EXPV) part2 = tc::f2_add(part2, tc::f2_add(p0, p1));
-                const float2 a0 = tc::f2_split(p0), a1 = tc::f2_split(p1);
-                w[e / 2] = tc::pack_bf16(a0.x, a0.y);
-                w[e / 2 + 1] = tc::pack_bf16(a1.x, a1.y);
-              }
-            } else if (cc == qr) {
-              // the block holding this row: per-element decay and causal mask
-              const float* ccv = cp + 32 * cc;
-#pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                float p[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  const int key = 32 * cc + e + u;
-                  p[u] = key <= row ? __uint_as_float(sv[e + u]) * tc::ex2(R + ccv[e + u]) : 0.f;
-                }
-                if (EXPV) part2 = tc::f2_add(part2, tc::f2_make(p[0], p[1]));
-                w[e / 2] = tc::pack_bf16(p[0], p[1]);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) w[e] = 0u;
+            for (int e = 0; e < 32; e += 4) {
+              const float4 k4 = *reinterpret_cast<const float4*>(kp + e);
+              const uint64_t p0 = tc::f2_mul(
+                  tc::f2_mul(tc::f2_make(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                             tc::f2_make(k4.x, k4.y)), rho2);
+              const uint64_t p1 = tc::f2_mul(
+                  tc::f2_mul(tc::f2_make(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])),
+                             tc::f2_make(k4.z, k4.w)), rho2);
+              if (EXPV) part2 = tc::f2_add(part2, tc::f2_add(p0, p1));
+              const float2 a0 = tc::f2_split(p0), a1 = tc::f2_split(p1);
+              w[e / 2] = tc::pack_bf16(a0.x, a0.y);
+              w[e / 2 + 1] = tc::pack_bf16(a1.x, a1.y);
             }
-            tc::tmem_st16_async(tS + 16 * cl, w);
+          } else if (cc == qr) {
+            // the block holding this row: per-element decay and causal mask
+            const float* ccv = cp + 32 * cc;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float p[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int key = 32 * cc + e + u;
+                p[u] = key <= row ? __uint_as_float(sv[e + u]) * tc::ex2(R + ccv[e + u]) : 0.f;
+              }
+              if (EXPV) part2 = tc::f2_add(part2, tc::f2_make(p[0], p[1]));
+              w[e / 2] = tc::pack_bf16(p[0], p[1]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w[e] = 0u;
           }
+          // packed into the first 16 of this block's own 32 columns
+          tc::tmem_st16_async(tS, w);
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
