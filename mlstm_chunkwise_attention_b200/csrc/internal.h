@@ -99,6 +99,8 @@ unsigned int next_epoch();
 // tensor-core kernels (tc_*.cu) and their host helpers (tmap.cu)
 bool make_tmap_3d_bf16(void* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
                        uint32_t box_inner, uint32_t box_mid);
+bool make_tmap_3d_bf16_rows(void* map, const void* base, uint64_t inner, uint64_t mid,
+                            uint64_t outer, uint32_t box_inner, uint32_t box_mid);
 bool output_fwd_tc_supported(const Problem& p);
 cudaError_t launch_output_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_fwd_error(unsigned int* flag);

@@ -13,7 +13,7 @@
 //    as their score product is done; warp 18 streams V_j with the key
 //    tile's gate factors through a second ring (TMA and bulk copies, no
 //    multicast);
-//  * warp 1 issues tcgen05.mma: S_{g+1} before P_g V_g, so the tensor core
+//  * warp 1 (lane 0 alone) issues tcgen05.mma: S_{g+1} before P_g V_g, so the tensor core
 //    computes the next score tile while the gate transform runs;
 //  * warps 2-17 (four warpgroups, one per 32-key block of a tile; four
 //    warps per SM sub-partition, so the latency of one warp's TMEM traffic
@@ -62,8 +62,9 @@ struct XlCfg {
   static constexpr int OFF_ROW = OFF_V + NV * V_BYTES;
   static constexpr int OFF_COL = OFF_ROW + NQ * ROWAUX;
   static constexpr int OFF_XS = OFF_COL + NV * COLAUX;  // [2 O buffers][4 key blocks][128] floats
-  static constexpr int OFF_STG = OFF_XS + 2 * 4 * 128 * 4;  // per transform warp: 16 rows of h
-  static constexpr int STG_WARP = 8 * DV;                      // 16 rows x DV / 4 bf16
+  // per transform warp: 16 rows of h (DV / 4 bf16 each), 1024-byte aligned for the swizzle
+  static constexpr int OFF_STG = (OFF_XS + 2 * 4 * 128 * 4 + 1023) & ~1023;
+  static constexpr int STG_WARP = 8 * DV;
   static constexpr int OFF_BAR = OFF_STG + 16 * STG_WARP;
   static constexpr int OFF_TMEM = OFF_BAR + 64 * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + alignment slack
@@ -85,8 +86,8 @@ enum {
   X_PF0 = 30,  // P written (256 threads, each having seen its step's V / C_prev), per S buffer
   X_OF0 = 34,  // O complete (MMA commit), per O buffer
   X_OE0 = 36,  // O read out (256 threads), per O buffer
-  X_XS0 = 38,  // normaliser partials exchanged (256 threads), per O buffer
-  X_COUNT = 40
+  X_XS0 = 38,  // normaliser shares exchanged (128 threads), per O buffer and lane quarter
+  X_COUNT = 46
 };
 
 constexpr int kXlThreads = 608;    // K producer, MMA, 16 transform warps, V producer
@@ -134,32 +135,42 @@ __device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB
 
 }  // namespace
 
-// Epilogue of one SIG work item (no normaliser, h = O) for the transform
-// thread of row 32 qr + lane and column quarter h (DV / 4 columns): read O out of TMEM, freeing it
-// for the next item's products, and store h through a staging slot so each
-// store instruction writes whole row segments.  Kept out of line so its
-// registers do not count against the gate transform it is called from.
-// (EXP keeps its epilogue inline with direct stores: there the staging cost
-// more in transform registers than it saved in store traffic, measured.)
+// Epilogue of one work item for the transform thread of row 32 qr + lane and
+// column quarter h (DV / 4 columns): for mLSTMexp the normaliser a_t (the
+// four key blocks' shares, exchanged among the four warps of this TMEM lane
+// quarter only) and 1 / den_t; then O is read out of TMEM, freeing it for the
+// next items' products, and h leaves through this warp's staging slot, 16
+// rows at a time, by TMA stores (the TMA unit clips rows past the sequence
+// end), so the stores cost the load/store unit nothing.  Kept out of line so
+// its registers do not count against the gate transform it is called from.
 template <int DQK, int DV, bool EXPV>
-__device__ __noinline__ bool xl_epilogue(int it, int vb, int nvalid, size_t tok, float fl, float part,
-                                         int h, int qr, int lane, uint32_t tmem, uint8_t* smem,
-                                         bf16* __restrict__ hout, float* __restrict__ abar_out,
-                                         int dhv, const tc::Abort& abort_flag) {
+__device__ __noinline__ bool xl_epilogue(int it, int vb, int y0, int bh, size_t tok, bool valid,
+                                         float fl, float part, int h, int qr, int lane, uint32_t tmem,
+                                         uint8_t* smem, const CUtensorMap* tm_h,
+                                         float* __restrict__ abar_out, const tc::Abort& abort_flag) {
   using Cfg = XlCfg<DQK, DV>;
   const unsigned full = 0xffffffffu;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
-  const int warp = 2 + 4 * h + ((qr + 2) & 3);
+  const int warp = 2 + 4 * h + ((qr + 2) & 3);  // the warp of (h, qr): lane quarter = warp % 4
+  const int row = 32 * qr + lane;
   const uint32_t lb = (uint32_t)(32 * qr) << 16;
   const int ob = it & 1, par = (it >> 1) & 1;
-  (void)fl;
-  (void)part;
-  (void)abar_out;
+  float inv = 1.f;
+  if (EXPV) {
+    // den_t = max(|a_t|, exp(-m_t)), a_t added in block order so the four threads of a row agree
+    float* x = reinterpret_cast<float*>(smem + Cfg::OFF_XS) + ob * 512;
+    x[h * 128 + row] = part;
+    uint64_t* xb = &bar[X_XS0 + 4 * ob + qr];
+    tc::mbar_arrive(xb);
+    if (!__all_sync(full, tc::mbar_wait(xb, par, abort_flag))) return false;
+    const float a = ((x[row] + x[128 + row]) + x[256 + row]) + x[384 + row];
+    inv = 1.f / fmaxf(fabsf(a), fl);
+    if (h == 0 && vb == 0 && valid) abar_out[tok] = a;
+  }
   if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + ob], par, abort_flag))) return false;
   tc::tc_fence_after();
   const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 4);
-  // this thread's DV / 4 columns as CPR 16-byte chunks
-  constexpr int CPR = DV / 32, RPI = 32 / CPR;
+  constexpr int CPR = DV / 32;  // 16-byte chunks of this thread's DV / 4 columns
   uint4 w[CPR];
   {
     uint32_t o[32];
@@ -169,48 +180,41 @@ __device__ __noinline__ bool xl_epilogue(int it, int vb, int nvalid, size_t tok,
     } else {
       tc::tmem_ld16(tO, o);
     }
+    tc::tc_fence_before();
+    tc::mbar_arrive(&bar[X_OE0 + ob]);
 #pragma unroll
     for (int c4 = 0; c4 < CPR; ++c4) {
       const uint32_t* r = &o[8 * c4];
       uint4& d = w[c4];
-      d.x = tc::pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
-      d.y = tc::pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
-      d.z = tc::pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
-      d.w = tc::pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
+      d.x = tc::pack_bf16(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
+      d.y = tc::pack_bf16(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
+      d.z = tc::pack_bf16(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
+      d.w = tc::pack_bf16(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
     }
   }
-  tc::tc_fence_before();
-  tc::mbar_arrive(&bar[X_OE0 + ob]);
-  // Each thread owns one row, so direct stores would touch 32 lines per
-  // warp instruction.  Rows go through a swizzled 16-row staging slot
-  // instead and leave as RPI whole row segments per instruction.
-  const uint32_t stg = tc::smem_u32(smem + Cfg::OFF_STG + (warp - 2) * Cfg::STG_WARP);
+  uint8_t* stg = smem + Cfg::OFF_STG + (warp - 2) * Cfg::STG_WARP;
+  const uint32_t astg = tc::smem_u32(stg);
 #pragma unroll
   for (int rnd = 0; rnd < 2; ++rnd) {
+    if (lane == 0) tc::bulk_wait_read_all();  // the slot's previous store has read it
+    __syncwarp();
     if ((lane >> 4) == rnd) {
+      // row r of the box, its 16-byte chunk c at chunk c ^ (address bits 7.. of the row):
+      // the swizzle of the h tensor map, whose span is one row (DV / 2 bytes)
       const int r = lane & 15;
+      const uint32_t sw = ((uint32_t)(r * CPR * 16) >> 7) & (CPR - 1);
 #pragma unroll
       for (int c = 0; c < CPR; ++c)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         stg + r * (CPR * 16) + ((c ^ (r & (CPR - 1))) << 4)),
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(astg + r * (CPR * 16) + ((c ^ sw) << 4)),
                      "r"(w[c].x), "r"(w[c].y), "r"(w[c].z), "r"(w[c].w)
                      : "memory");
+      tc::fence_proxy_async_smem();
     }
     __syncwarp();
-#pragma unroll
-    for (int kk = 0; kk < 16 / RPI; ++kk) {
-      const int rr = kk * RPI + lane / CPR, c = lane % CPR;
-      uint4 v;
-      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                   : "r"(stg + rr * (CPR * 16) + ((c ^ (rr & (CPR - 1))) << 4))
-                   : "memory");
-      const int rw = 16 * rnd + rr;  // row within this warp's 32
-      if (rw < nvalid)
-        *reinterpret_cast<uint4*>(hout + (tok - lane + rw) * (size_t)dhv + vb * DV +
-                                  h * (DV / 4) + 8 * c) = v;
+    if (lane == 0) {
+      tc::tma_store_3d(tm_h, stg, vb * DV + h * (DV / 4), y0 + 16 * rnd, bh);
+      tc::bulk_commit_group();
     }
-    __syncwarp();
   }
   return true;
 }
@@ -219,7 +223,8 @@ template <int DQK, int DV, bool EXPV>
 __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-    const float* __restrict__ tab, const float* __restrict__ gn, bf16* __restrict__ hout,
+    const __grid_constant__ CUtensorMap tm_h, const float* __restrict__ tab,
+    const float* __restrict__ gn, bf16* __restrict__ hout,
     float* __restrict__ abar_out, int T, int L, int NC, int BH, int NVB, int ntq, int total,
     int tstride, int dhv, bool has_init, unsigned int epoch) {
   using Cfg = XlCfg<DQK, DV>;
@@ -241,7 +246,8 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       uint32_t cnt = 1;
       if (i == X_QE0 || i == X_QE0 + 1) cnt = kXlTransform + 1;
       if (i >= X_PF0 && i < X_PF0 + 4) cnt = kXlTransform;
-      if (i >= X_OE0 && i < X_XS0 + 2) cnt = kXlTransform;
+      if (i >= X_OE0 && i < X_OE0 + 2) cnt = kXlTransform;
+      if (i >= X_XS0 && i < X_XS0 + 8) cnt = kXlTransform / 4;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -346,15 +352,20 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp walks the schedule and waits; lane 0 issues the MMAs and
-    // their commits (a commit tracks the MMAs of the thread that issues it).
-    {
-      const unsigned full = 0xffffffffu;
-      const bool leader = lane == 0;
+    // Lane 0 alone walks the schedule, waits and issues.  tcgen05.mma issue
+    // blocks behind a shallow queue, so every other instruction this thread
+    // runs between two products (warp votes, descriptor arithmetic) is time
+    // the tensor pipe stands idle: the shared-memory descriptors are built
+    // once and advanced by constant offsets (the address field is the low
+    // 14 bits of address / 16, and no offset reaches past the 227 KB of
+    // shared memory, so adding to the descriptor is exact).
+    if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(128, DV, false, true);
       const uint32_t aQ0 = tc::smem_u32(smem + Cfg::OFF_Q), aK0 = tc::smem_u32(smem + Cfg::OFF_K),
                      aV0 = tc::smem_u32(smem + Cfg::OFF_V);
+      const uint64_t dQ0 = tc::sdesc_sw128(aQ0, 16, 1024), dK0 = tc::sdesc_sw128(aK0, 16, 1024),
+                     dV0 = tc::sdesc_sw128(aV0, 16384, 1024), dC0 = tc::sdesc_sw128(aK0, DQK * 128, 1024);
 
       // score step s of item I (its it-th item, global step g): S_j = Q K_j^T,
       // then the K stage is free; for the C_prev step only a commit, which
@@ -362,30 +373,23 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       auto issue_s = [&](const XlItem& I, int it, int s, int g) -> bool {
         const int sb = g & 1;
         if (I.pseudo && s == 0) {
-          if (leader) tc::tc_commit(&bar[X_SF0 + sb]);
-          __syncwarp();
+          tc::tc_commit(&bar[X_SF0 + sb]);
           return true;
         }
         const int qb = it % NQ, kst = g % NK;
-        // every barrier check costs the tensor pipe a drain, so the Q buffer is
-        // checked only before the item's first score product
-        if (s == (I.pseudo ? 1 : 0) &&
-            !__all_sync(full, tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag)))
+        // the Q buffer is checked only before the item's first score product
+        if (s == (I.pseudo ? 1 : 0) && !tc::mbar_wait(&bar[X_QF0 + qb], (it / NQ) & 1, abort_flag))
           return false;
-        if (!__all_sync(full, tc::mbar_wait(&bar[X_KF0 + kst], (g / NK) & 1, abort_flag))) return false;
-        tc::tc_fence_after();
-        const uint32_t aQ = aQ0 + qb * Cfg::Q_BYTES, aK = aK0 + kst * Cfg::K_BYTES;
-        if (leader) {
+        if (!tc::mbar_wait(&bar[X_KF0 + kst], (g / NK) & 1, abort_flag)) return false;
+        const uint64_t dQ = dQ0 + (uint64_t)((qb * Cfg::Q_BYTES) >> 4),
+                       dK = dK0 + (uint64_t)((kst * Cfg::K_BYTES) >> 4);
 #pragma unroll
-          for (int k = 0; k < DQK / 16; ++k) {
-            const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-            tc::mma_bf16_ss(tmem + sb * 128, tc::sdesc_sw128(aQ + off, 16, 1024),
-                            tc::sdesc_sw128(aK + off, 16, 1024), idS, k > 0);
-          }
-          tc::tc_commit(&bar[X_SF0 + sb]);
-          tc::tc_commit(&bar[X_KE0 + kst]);
+        for (int k = 0; k < DQK / 16; ++k) {
+          const uint64_t off = (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4);
+          tc::mma_bf16_ss(tmem + sb * 128, dQ + off, dK + off, idS, k > 0);
         }
-        __syncwarp();
+        tc::tc_commit(&bar[X_SF0 + sb]);
+        tc::tc_commit(&bar[X_KE0 + kst]);
         return true;
       };
       // accumulate step s into O: P_j V_j (V stage of real step gv),
@@ -395,36 +399,27 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       auto issue_pv = [&](const XlItem& I, int it, int s, int g, int gv) -> bool {
         const int sb = g & 1, ob = it & 1;
         const uint32_t tO = tmem + 256 + ob * DV, tP = tmem + sb * 128;
-        if (s == 0 && !__all_sync(full, tc::mbar_wait(&bar[X_OE0 + ob], ((it >> 1) & 1) ^ 1, abort_flag)))
-          return false;
-        if (!__all_sync(full, tc::mbar_wait(&bar[X_PF0 + sb], (g >> 1) & 1, abort_flag))) return false;
+        if (s == 0 && !tc::mbar_wait(&bar[X_OE0 + ob], ((it >> 1) & 1) ^ 1, abort_flag)) return false;
+        if (!tc::mbar_wait(&bar[X_PF0 + sb], (g >> 1) & 1, abort_flag)) return false;
         tc::tc_fence_after();
         if (I.pseudo && s == 0) {
           const int kst = g % NK;
-          const uint32_t aC = aK0 + kst * Cfg::K_BYTES;
-          if (leader) {
+          const uint64_t dC = dC0 + (uint64_t)((kst * Cfg::K_BYTES) >> 4);
 #pragma unroll
-            for (int k = 0; k < DQK / 16; ++k) {  // 16 rows of C_prev
-              // the q elements of block g = k / (DQK / 64) sit packed at column 32 g
-              const int g = k / (DQK / 64), kk = k % (DQK / 64);
-              tc::mma_bf16_ts(tO, tP + 32 * g + 8 * kk, tc::sdesc_sw128(aC + k * 2048, DQK * 128, 1024),
-                              idO, k > 0);
-            }
-            tc::tc_commit(&bar[X_KE0 + kst]);
+          for (int k = 0; k < DQK / 16; ++k) {  // 16 rows of C_prev
+            // the q elements of block b = k / (DQK / 64) sit packed at column 32 b
+            const int b = k / (DQK / 64), kk = k % (DQK / 64);
+            tc::mma_bf16_ts(tO, tP + 32 * b + 8 * kk, dC + (uint64_t)(k * 128), idO, k > 0);
           }
-          __syncwarp();
+          tc::tc_commit(&bar[X_KE0 + kst]);
           return true;
         }
-        if (leader) {
-          const int vst = gv % NV;
-          const uint32_t aV = aV0 + vst * Cfg::V_BYTES;
+        const uint64_t dV = dV0 + (uint64_t)(((gv % NV) * Cfg::V_BYTES) >> 4);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)  // 16 keys per step; keys 32 g .. of P live at column 32 g
-            tc::mma_bf16_ts(tO, tP + 32 * (k >> 1) + 8 * (k & 1),
-                            tc::sdesc_sw128(aV + k * 2048, 16384, 1024), idO, (s > 0 || k > 0));
-          tc::tc_commit(&bar[X_VE0 + vst]);
-        }
-        __syncwarp();
+        for (int k = 0; k < 8; ++k)  // 16 keys per step; keys 32 b .. of P live at column 32 b
+          tc::mma_bf16_ts(tO, tP + 32 * (k >> 1) + 8 * (k & 1), dV + (uint64_t)(k * 128), idO,
+                          (s > 0 || k > 0));
+        tc::tc_commit(&bar[X_VE0 + (gv % NV)]);
         return true;
       };
 
@@ -448,11 +443,10 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           ok = issue_pv(I, it, s, g, gv);
           if (!ok) break;
           if (real) ++gv;
-          if (last && leader) {
+          if (last) {
             tc::tc_commit(&bar[X_QE0 + it % NQ]);
             tc::tc_commit(&bar[X_OF0 + (it & 1)]);
           }
-          __syncwarp();
           if (!Cfg::LOOK) {
             if (!last) ok = issue_s(I, it, s + 1, g + 1);
             else if (kn < total) ok = issue_s(N, it + 1, 0, g + 1);
@@ -472,56 +466,18 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
     const unsigned full = 0xffffffffu;
     int it = 0, g = 0, gv = 0;
 
-    // epilogue of one item: normalise O and store h
     // what the deferred epilogue of an item needs (kept small: it is live
     // through the next item's first step)
     struct Pending {
-      int it, vb, nvalid;  // item counter; value block; rows of this warp's 32 in the sequence
-      size_t tok;          // token of this thread's row
+      int it, vb, y0, bh;  // item counter; value block; token of this warp's first row; head
+      size_t tok;          // token of this thread's row ([BH, T] index)
+      bool valid;          // this thread's row is in the sequence
       float fl, part;
     } pe{};
     bool pend = false;
     auto epilogue = [&](const Pending& e) -> bool {
-      if (!EXPV)
-        return xl_epilogue<DQK, DV, EXPV>(e.it, e.vb, e.nvalid, e.tok, e.fl, e.part, h, qr, lane, tmem,
-                                          smem, hout, abar_out, dhv, abort_flag);
-      // EXP: den_t = max(|a_t|, exp(-m_t)), a_t the sum of the four key blocks' shares (added
-      // in block order, so the four threads of a row agree)
-      const int ob = e.it & 1, par = (e.it >> 1) & 1;
-      const bool valid = lane < e.nvalid;
-      float* x = xs + ob * 512;
-      x[h * 128 + row] = e.part;
-      tc::mbar_arrive(&bar[X_XS0 + ob]);
-      if (!__all_sync(full, tc::mbar_wait(&bar[X_XS0 + ob], par, abort_flag))) return false;
-      const float a = ((x[row] + x[128 + row]) + x[256 + row]) + x[384 + row];
-      const float inv = 1.f / fmaxf(fabsf(a), e.fl);
-      if (h == 0 && e.vb == 0 && valid) abar_out[e.tok] = a;
-      if (!__all_sync(full, tc::mbar_wait(&bar[X_OF0 + ob], par, abort_flag))) return false;
-      tc::tc_fence_after();
-      const uint32_t tO = tmem + 256 + ob * DV + lb + h * (DV / 4);
-      uint32_t o[32];
-      if (DV >= 128) {
-        tc::tmem_ld32_async(tO, o);
-        tc::tmem_wait_ld(o);
-      } else {
-        tc::tmem_ld16(tO, o);
-      }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&bar[X_OE0 + ob]);
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(hout + e.tok * (size_t)dhv + e.vb * DV + h * (DV / 4));
-#pragma unroll
-        for (int c8 = 0; c8 < DV / 32; ++c8) {
-          const uint32_t* r = &o[8 * c8];
-          uint4 w;
-          w.x = tc::pack_bf16(__uint_as_float(r[0]) * inv, __uint_as_float(r[1]) * inv);
-          w.y = tc::pack_bf16(__uint_as_float(r[2]) * inv, __uint_as_float(r[3]) * inv);
-          w.z = tc::pack_bf16(__uint_as_float(r[4]) * inv, __uint_as_float(r[5]) * inv);
-          w.w = tc::pack_bf16(__uint_as_float(r[6]) * inv, __uint_as_float(r[7]) * inv);
-          dst[c8] = w;
-        }
-      }
-      return true;
+      return xl_epilogue<DQK, DV, EXPV>(e.it, e.vb, e.y0, e.bh, e.tok, e.valid, e.fl, e.part, h, qr,
+                                        lane, tmem, smem, &tm_h, abar_out, abort_flag);
     };
 
     for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
@@ -640,14 +596,17 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       const float2 pf = tc::f2_split(part2);
       pe.it = it;
       pe.vb = I.vb;
+      pe.y0 = I.c * L + I.t0 + 32 * qr;
+      pe.bh = I.bh;
       pe.tok = (size_t)I.bh * T + (size_t)I.c * L + I.t0 + row;
-      pe.nvalid = min(32, max(0, I.len - (I.t0 + 32 * qr)));
+      pe.valid = I.t0 + row < I.len;
       pe.fl = FLt;
       pe.part = pf.x + pf.y;
       pend = true;
       ++it;
     }
     if (ok && pend) ok = epilogue(pe);
+    if (lane == 0) tc::bulk_wait_all();  // the h stores have read the staging slot
   }
 
   if (!ok) abort_flag.raise();
@@ -668,8 +627,9 @@ template <int DQK, int DV, bool EXPV>
 static cudaError_t launch_out_xl(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   using Cfg = XlCfg<DQK, DV>;
   if (a.xt == nullptr) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv, tcm;
-  if (!make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
+  CUtensorMap tq, tk, tv, tcm, th;
+  if (!make_tmap_3d_bf16_rows(&th, a.h, p.dhv, p.T, p.BH, DV / 4, 16) ||
+      !make_tmap_3d_bf16(&tq, a.q, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tk, a.k, p.dqk, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tv, a.v, p.dhv, p.T, p.BH, 64, 128) ||
       !make_tmap_3d_bf16(&tcm, a.C, p.dhv, p.dqk, (uint64_t)p.BH * p.NC, 64, DQK))
@@ -689,7 +649,7 @@ static cudaError_t launch_out_xl(const Problem& p, const FwdArgs& a, cudaStream_
   if (total >= (1LL << 30)) return cudaErrorInvalidValue;
   const long long pairs = total / 2;
   const int grid = (int)(pairs < nsm ? pairs : nsm);
-  kern<<<grid, kXlThreads, smem, s>>>(tq, tk, tv, tcm, a.xt, a.n, (bf16*)a.h, a.abar, p.T, p.L,
+  kern<<<grid, kXlThreads, smem, s>>>(tq, tk, tv, tcm, th, a.xt, a.n, (bf16*)a.h, a.abar, p.T, p.L,
                                       p.NC, p.BH, nvb, ntq, (int)total, xl_table_stride(p.L),
                                       p.dhv, a.init.on(), next_epoch());
   return cudaGetLastError();

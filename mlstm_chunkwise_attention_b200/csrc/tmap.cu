@@ -36,4 +36,30 @@ bool make_tmap_3d_bf16(void* map, const void* base, uint64_t inner, uint64_t mid
   return r == CUDA_SUCCESS;
 }
 
+// The same with the swizzle span equal to the box's row (box_inner * 2 bytes:
+// 32, 64 or 128): a box of box_mid rows of box_inner elements, row after row in
+// shared memory, each row's 16-byte chunks permuted by the row index (the
+// staging layout of row-wise epilogues, written without bank conflicts).
+bool make_tmap_3d_bf16_rows(void* map, const void* base, uint64_t inner, uint64_t mid,
+                            uint64_t outer, uint32_t box_inner, uint32_t box_mid) {
+  CUtensorMapSwizzle sw;
+  switch (box_inner * 2) {
+    case 32: sw = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    case 64: sw = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 128: sw = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    default: return false;
+  }
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {box_inner, box_mid, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace mlstm

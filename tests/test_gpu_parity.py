@@ -66,7 +66,7 @@ SMALL = [
 def _compare_all_heads(cpu, h, g, L, var, tol, grad_tol=None):
     """Every element of every head against the oracle; the bar applies per output tensor
     (max|err| over all heads / max|ref| over all heads), tol for h and grad_tol (default
-    tol) for the gradients.  The oracle backward reads h in the I/O dtype, as mlstm_bwd
+    tol; a dict maps a gradient's name, else "default", to its bar) for the gradients.  The oracle backward reads h in the I/O dtype, as mlstm_bwd
     receives it."""
     Bn, NH = cpu["q"].shape[:2]
     worst = {}
@@ -88,6 +88,8 @@ def _compare_all_heads(cpu, h, g, L, var, tol, grad_tol=None):
         floor = 1e-3 * gscale if key != "h" else 1e-30
         err = e / max(r, floor)
         bar = tol if key == "h" or grad_tol is None else grad_tol
+        if isinstance(bar, dict):
+            bar = bar.get(key, bar["default"])
         assert err <= bar, f"{key}: {err:.3e} (largest error in head {at})"
 
 
@@ -136,8 +138,12 @@ def test_exp_large_input_gates_all_heads(case):
     # term dA_ts = dh_t.(v_s - h_t) / den_t cancels down to the last bits of the bf16
     # output h: an fp64 emulation with only h rounded puts the gradients 1e-2 to 5e-2 off
     # the exact ones, and a forward that differs in the last bit of h moves them as much.
-    # h itself is held to 1e-2; the gradients of these inputs to a sanity bound of 1e-1.
-    _compare_all_heads(cpu, h, g, L, EXP, 1e-2, grad_tol=1e-1 if spike is not None else None)
+    # The gate gradients sum such terms over the sequence: moving a random half of the
+    # bf16 h by one ulp moves the oracle's dfgate_pre by up to 0.23 and digate_pre by up
+    # to 0.13 of their largest element in the chunk-128 d64 case.  h itself is held to
+    # 1e-2; dq, dk, dv to a sanity bound of 1e-1, the gate gradients to 0.25.
+    spike_tol = {"default": 1e-1, "digate_pre": 0.25, "dfgate_pre": 0.25}
+    _compare_all_heads(cpu, h, g, L, EXP, 1e-2, grad_tol=spike_tol if spike is not None else None)
 
 
 @pytest.mark.parametrize("var", [SIG, EXP])
