@@ -37,7 +37,8 @@ KERNEL_SOURCES = {
     "state_bwd_simt": "simt_bwd.cu", "dq_simt": "simt_bwd.cu", "dk_simt": "simt_bwd.cu",
     "dv_simt": "simt_bwd.cu", "output_fwd_tc": "tc_fwd.cu", "dq_tc": "tc_bwd.cu",
     "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
-    "output_fwd_xl": "tc_fwd_xl.cu",
+    "output_fwd_xl": "tc_fwd_xl.cu", "bwd_xl_table": "tc_bwd_xl.cu", "dq_xl": "tc_bwd_xl.cu",
+    "dk_xl": "tc_bwd_xl.cu", "dv_xl": "tc_bwd_xl.cu",
     "state_bwd_tc": "tc_state.cu", "dkv_walk_tc": "tc_bwd_walk.cu", "fwd_walk_tc": "tc_fwd_walk.cu",
 }
 
@@ -84,6 +85,8 @@ def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
         "dk": (tdd + T * L * dqk, T * (3 * dqk + 2 * dhv) * io_bytes + 6 * tok_f + st_full + stn),
         "dv": (tdd + T * L * (dqk + dhv), T * (2 * dqk + 2 * dhv) * io_bytes + 4 * tok_f + st_full),
         "gate_grad": (0, T * 4 * io_bytes + 2 * tok_f),
+        # the large-chunk backward's gate table: five per-token arrays in, seven out
+        "bwd_xl_table": (0, 12 * tok_f),
         # state gradients, dk and dv in one pass: the state-gradient recurrence and the
         # dk, dv contractions; q, k, v, dh read once, dk, dv and k.dk written, the state
         # gradients never leave the chip

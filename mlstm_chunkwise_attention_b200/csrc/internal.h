@@ -56,6 +56,19 @@ struct FwdArgs {
 // Every block of a chunk starts 16-byte aligned (L is a multiple of 128).
 __host__ __device__ inline int xl_table_stride(int L) { return 5 * L + (L / 32 > 32 ? L / 32 : 32); }
 
+// Per-chunk gate table of the large-chunk backward, [BH, NC, bwd_xl_table_stride(L)]
+// floats, written by bwd_xl_table.  For token t (query side) or s (key side) of chunk c:
+//   QX [0, L)    (b_t - m_t) log2 e + log2(1/den_t)          (m_t = 0, den_t = 1 for SIG)
+//   QE [L, 2L)   da_t den_t                                   (0 for SIG)
+//   KX [2L, 3L)  (log i_s - b_s) log2 e
+//   KG [3L, 4L)  exp2(KX_s - KM_{s/32})
+//   RQ [4L, 5L)  alpha_t / den_t, alpha_t = exp(b_t + m_{c-1} - m_t)  (0 with no entering state)
+//   RV [5L, 6L)  alpha_t da_t
+//   RK [6L, 7L)  exp(b_last - b_s + log i_s - m_last)  (last: the chunk's last token)
+//   KM [7L, ..)  max of KX over each block of 32 keys (0 for a block wholly past the end)
+// Past the end of the sequence: QX = KX = -inf, QE = KG = RQ = RV = RK = 0.
+__host__ __device__ inline int bwd_xl_table_stride(int L) { return 7 * L + (L / 32 > 32 ? L / 32 : 32); }
+
 // Device pointers of one backward call.
 struct BwdArgs {
   const void *q, *k, *v, *ig, *fg, *h, *dh;
@@ -75,6 +88,7 @@ struct BwdArgs {
   const float* dCT;  // gradient with respect to the final state: C [BH, dqk, dhv] (null: none)
   const float* dnT;  // and n [BH, dqk] (mLSTMexp)
   float* fdot;       // [BH] <dC_T, C_T> + <dn_T, n_T>, added to every forget-gate gradient
+  float* btab;       // per-chunk gate table of the large-chunk backward (null: not used)
 };
 
 // gate kernels (gates.cu)
@@ -112,7 +126,14 @@ bool intra_bwd_tc_supported(const Problem& p);
 cudaError_t launch_dq_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dk_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_dv_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
+// large chunks, d_qk = d_hv = 128, bf16 (tc_bwd_xl.cu): the gate table, then dq, dk, dv
+bool intra_bwd_xl_supported(const Problem& p);
+cudaError_t launch_bwd_xl_table(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dq_xl(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dk_xl(const Problem& p, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_dv_xl(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_bwd_error(unsigned int* flag);
+cudaError_t fetch_tc_bwd_xl_error(unsigned int* flag);
 bool state_tc_supported(const Problem& p);
 cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);

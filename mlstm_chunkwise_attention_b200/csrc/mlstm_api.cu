@@ -109,7 +109,7 @@ mlstm::InitState init_from(const void* state, const Problem& p) {
 }
 
 struct BwdLayout {
-  size_t inv_den, da, pq, pk, dC, dn, fstate, fdot, total;
+  size_t inv_den, da, pq, pk, dC, dn, fstate, fdot, btab, btab_bytes, total;
 };
 
 BwdLayout bwd_layout(const Problem& p) {
@@ -125,6 +125,11 @@ BwdLayout bwd_layout(const Problem& p) {
   // the final state, rebuilt when the loss has a term on it, and its dot product with that term
   L.fstate = off;  off = align256(off + state_layout(p.BH, p.dqk, p.dhv, p.exp_variant()).total);
   L.fdot = off;    off = align256(off + (size_t)p.BH * 4);
+  // the large-chunk backward's per-chunk gate table
+  L.btab_bytes = mlstm::intra_bwd_xl_supported(p)
+                     ? (size_t)p.BH * p.NC * mlstm::bwd_xl_table_stride(p.L) * 4
+                     : 0;
+  L.btab = off;    off = align256(off + L.btab_bytes);
   L.total = off;
   return L;
 }
@@ -223,7 +228,12 @@ int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
   else
     st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
   if (!grads) return n;
-  if (mlstm::intra_bwd_tc_supported(p)) {
+  if (mlstm::intra_bwd_xl_supported(p)) {
+    st[n++] = {"bwd_xl_table", mlstm::launch_bwd_xl_table};
+    st[n++] = {"dq_xl", mlstm::launch_dq_xl};
+    st[n++] = {"dk_xl", mlstm::launch_dk_xl};
+    st[n++] = {"dv_xl", mlstm::launch_dv_xl};
+  } else if (mlstm::intra_bwd_tc_supported(p)) {
     st[n++] = {"dq_tc", mlstm::launch_dq_tc};
     st[n++] = {"dk_tc", mlstm::launch_dk_tc};
     st[n++] = {"dv_tc", mlstm::launch_dv_tc};
@@ -506,6 +516,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   a.dCT = dstate_out ? (const float*)((const char*)dstate_out + SL.C) : nullptr;
   a.dnT = (dstate_out && p.exp_variant()) ? (const float*)((const char*)dstate_out + SL.n) : nullptr;
   a.fdot = dstate_out ? (float*)(ws + W.fdot) : nullptr;
+  a.btab = W.btab_bytes ? (float*)(ws + W.btab) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_bwd");
@@ -727,7 +738,7 @@ namespace {
 // mlstm_device_status saw last.  A flag holds the epoch of the last launch of
 // its family that gave up, so a value that differs from the last one seen is a
 // failure not yet reported.
-constexpr int kFlagDevices = 64, kFlagFamilies = 6;
+constexpr int kFlagDevices = 64, kFlagFamilies = 7;
 std::mutex g_flag_mu;
 unsigned int g_flag_seen[kFlagDevices][kFlagFamilies] = {};
 }  // namespace
@@ -745,7 +756,8 @@ int mlstm_device_status(void* stream) {
   typedef cudaError_t (*Fetch)(unsigned int*);
   const Fetch fetch[kFlagFamilies] = {mlstm::fetch_tc_fwd_error,    mlstm::fetch_tc_bwd_error,
                                       mlstm::fetch_tc_state_error,  mlstm::fetch_tc_fwd_xl_error,
-                                      mlstm::fetch_tc_walk_error,   mlstm::fetch_tc_fwalk_error};
+                                      mlstm::fetch_tc_walk_error,   mlstm::fetch_tc_fwalk_error,
+                                      mlstm::fetch_tc_bwd_xl_error};
   unsigned int flag[kFlagFamilies] = {};
   for (int i = 0; i < kFlagFamilies; ++i) {
     st = cuda_status(fetch[i](&flag[i]), "device error flag");

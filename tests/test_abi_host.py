@@ -259,6 +259,20 @@ def test_launch_plans_put_every_bf16_chunk_size_on_tensor_cores(lib, variant, d)
     assert all(n.endswith("_simt") for n in names if n not in ("gate_prep", "bwd_token_prep", "gate_grad"))
 
 
+@pytest.mark.parametrize("variant", [B.SIG, B.EXP], ids=["sig", "exp"])
+def test_launch_plans_large_chunk_backward(lib, variant):
+    """bf16, d_qk = d_hv = 128, chunk >= 256: the backward's intra-chunk products run on the
+    large-chunk kernels after their gate table; other head dims keep the one-tile kernels."""
+    for L in (256, 512, 1024, 4096):
+        assert _plan(1, (2, 4, 5000, 128, 128, L, variant, B.BF16)) == [
+            "bwd_token_prep", "state_bwd_tc", "bwd_xl_table", "dq_xl", "dk_xl", "dv_xl", "gate_grad"]
+    for other in [(2, 4, 5000, 64, 64, 256, variant, B.BF16),
+                  (2, 4, 5000, 128, 256, 512, variant, B.BF16),
+                  (2, 4, 5000, 128, 128, 128, variant, B.BF16),
+                  (2, 4, 5000, 128, 128, 256, variant, B.FP32)]:
+        assert not any(n.endswith("_xl") and n != "output_fwd_xl" for n in _plan(1, other)), other
+
+
 def test_serial_launch_switch_needs_no_device(lib):
     """mlstm_set_serial_launches only sets a per-thread flag: no CUDA call, always MLSTM_OK."""
     assert lib.mlstm_set_serial_launches(1) == 0
