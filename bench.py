@@ -38,7 +38,8 @@ KERNEL_SOURCES = {
     "dv_simt": "simt_bwd.cu", "output_fwd_tc": "tc_fwd.cu", "dq_tc": "tc_bwd.cu",
     "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
     "output_fwd_xl": "tc_fwd_xl.cu", "bwd_xl_table": "tc_bwd_xl.cu", "dq_xl": "tc_bwd_xl.cu",
-    "dk_xl": "tc_bwd_xl.cu", "dv_xl": "tc_bwd_xl.cu",
+    "dk_xl": "tc_bwd_xl.cu", "dv_xl": "tc_bwd_xl.cu", "state_fwd_fix": "tc_state.cu",
+    "state_bwd_fix": "tc_state.cu",
     "state_bwd_tc": "tc_state.cu", "dkv_walk_tc": "tc_bwd_walk.cu", "fwd_walk_tc": "tc_fwd_walk.cu",
 }
 
@@ -87,6 +88,9 @@ def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
         "gate_grad": (0, T * 4 * io_bytes + 2 * tok_f),
         # the large-chunk backward's gate table: five per-token arrays in, seven out
         "bwd_xl_table": (0, 12 * tok_f),
+        # completion of a segmented state walk: every state read and written once
+        "state_fwd_fix": (0, 2 * st_full + (2 * stn if exp_variant else 0)),
+        "state_bwd_fix": (0, 2 * st_full + (2 * stn if exp_variant else 0)),
         # state gradients, dk and dv in one pass: the state-gradient recurrence and the
         # dk, dv contractions; q, k, v, dh read once, dk, dv and k.dk written, the state
         # gradients never leave the chip

@@ -137,6 +137,10 @@ cudaError_t fetch_tc_bwd_xl_error(unsigned int* flag);
 bool state_tc_supported(const Problem& p);
 cudaError_t launch_state_fwd_tc(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t s);
+// few heads and many chunks: the state walks run in segments, completed by state_*_fix
+bool state_split_needed(const Problem& p);
+cudaError_t launch_state_fwd_fix(const Problem& p, const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_state_bwd_fix(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t fetch_tc_state_error(unsigned int* flag);
 bool bwd_walk_supported(const Problem& p);
 cudaError_t launch_bwd_walk(const Problem& p, const BwdArgs& a, cudaStream_t s);

@@ -197,9 +197,10 @@ int fwd_plan(const Problem& p, FwdStep* st, bool want_h = true) {
     st[n++] = {"fwd_walk_tc", mlstm::launch_fwd_walk};
     return n;
   }
-  if (mlstm::state_tc_supported(p))
+  if (mlstm::state_tc_supported(p)) {
     st[n++] = {"state_fwd_tc", mlstm::launch_state_fwd_tc};
-  else
+    if (mlstm::state_split_needed(p)) st[n++] = {"state_fwd_fix", mlstm::launch_state_fwd_fix};
+  } else
     st[n++] = {"state_fwd_simt", mlstm::launch_state_fwd_simt};
   if (mlstm::output_fwd_xl_supported(p))
     st[n++] = {"output_fwd_xl", mlstm::launch_output_fwd_xl};
@@ -223,9 +224,10 @@ int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
     st[n++] = {"gate_grad", mlstm::launch_gate_grad, false, true};
     return n;
   }
-  if (mlstm::state_tc_supported(p))
+  if (mlstm::state_tc_supported(p)) {
     st[n++] = {"state_bwd_tc", mlstm::launch_state_bwd_tc};
-  else
+    if (mlstm::state_split_needed(p)) st[n++] = {"state_bwd_fix", mlstm::launch_state_bwd_fix};
+  } else
     st[n++] = {"state_bwd_simt", mlstm::launch_state_bwd_simt};
   if (!grads) return n;
   if (mlstm::intra_bwd_xl_supported(p)) {

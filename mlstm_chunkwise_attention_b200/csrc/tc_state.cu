@@ -14,7 +14,11 @@
 //
 // One CTA owns a 128-row (d_qk) by 64-column (d_hv) tile of the state and
 // walks the chunks in order; the fp32 running state lives in registers of the
-// four epilogue warps (one state row per thread).  Each chunk is streamed in
+// four epilogue warps (one state row per thread).  When too few CTAs would
+// walk too many chunks (few heads, long sequences), each head's chunk range is
+// split into segments walked in parallel, every segment but the first from the
+// zero state; state_fix then adds to each segment's states the true state
+// entering it, carried through the segment's decay (the recurrence is linear).  Each chunk is streamed in
 // 64-token sub-tiles through a TMA ring; two warps scale the value-side
 // operand by the per-token weight and split it into hi and lo bf16 tiles, so
 // the contraction K^T (w V) keeps fp32-level accuracy (two MMAs per step).
@@ -67,7 +71,8 @@ struct StateTcParams {
   bf16* out;      // hi plane; the lo plane follows after `plane` elements
   float* nout;    // [BH, NC, dqk] normaliser state (forward) or its gradient (backward)
   size_t plane;
-  int T, L, NC, dqk, dhv;
+  int T, L, NC, dqk, dhv, BH;
+  int seg_len, nseg;  // chunks (walk steps) per segment; segments per head (1: no split)
   float scale;
   InitState init;   // forward: the state entering chunk 0; both: its max state m0
   float *d0, *dn0;  // backward: gradient of the initial state (C, n), fp32, or null
@@ -87,13 +92,21 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   // an earlier CTA gave up: the whole block leaves together
   if (__syncthreads_or(threadIdx.x == 0 && abort_flag.raised())) return;
   // value-column tiles vary fastest so the CTAs sharing one head's key rows run together
-  const int dv0 = blockIdx.x * NV, dk0 = blockIdx.y * 128, bh = blockIdx.z;
+  const int dv0 = blockIdx.x * NV, dk0 = blockIdx.y * 128;
+  const int bh = (int)(blockIdx.z % P.BH), seg = (int)(blockIdx.z / P.BH);
   const bool with_n = EXPV && blockIdx.x == 0;
   const size_t tokh = (size_t)bh * P.T;
   const int NC = P.NC;
-  // chunks whose contribution is needed: all but the last (forward) or the first
-  // (backward), and the backward's first too when the initial state's gradient is wanted
-  const int nsteps = NC - 1 + ((BWD && P.d0 != nullptr) ? 1 : 0);
+  // this segment's walk steps [us, us + nlocal): chunks in order (forward) or in reverse
+  // (backward).  Contributions needed: every step's but the walk's last (no state leaves
+  // it), and that one too in the backward when the initial state's gradient is wanted.
+  // Slots stored: the state entering each step of the segment (the first segment's first
+  // one included, the others' first one being the previous segment's last) and, unless the
+  // segment ends the walk, the state after its last step.
+  const int us = seg * P.seg_len, nlocal = min(P.seg_len, NC - us);
+  const bool last_seg = us + nlocal == NC;
+  const int nsteps = last_seg ? nlocal - 1 + ((BWD && P.d0 != nullptr) ? 1 : 0) : nlocal;
+  const int nslots = last_seg ? nlocal : nlocal + 1;
   const float* m0 = P.init.on() ? P.init.m : nullptr;
 
   extern __shared__ uint8_t smem_raw[];
@@ -129,7 +142,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   const uint32_t tU0 = tmem;
   bool ok = true;
 
-  auto chunk_of = [&](int u) { return BWD ? NC - 1 - u : u; };
+  auto chunk_of = [&](int u) { return BWD ? NC - 1 - (us + u) : us + u; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -281,16 +294,19 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
     float S[NV];
     const float* S0 = BWD ? P.dT : P.init.C;
     const float* n0 = BWD ? P.dnT : P.init.n;
-    const bool from_init = S0 != nullptr && valid;
+    const bool from_init = S0 != nullptr && valid && seg == 0;
 #pragma unroll
     for (int j = 0; j < NV; ++j)
       S[j] = from_init ? S0[((size_t)bh * P.dqk + dk0 + i) * P.dhv + dv0 + j] : 0.f;
     float sn = (from_init && with_n) ? n0[(size_t)bh * P.dqk + dk0 + i] : 0.f;
-    for (int u = 0; u < NC; ++u) {
+    int nstored = 0;
+    for (int u = 0; u < nslots; ++u) {
       const int c = chunk_of(u);
       // store the state at this chunk boundary: rows into the swizzled staging
       // tile, then one TMA store per plane issued by thread 0 of the epilogue
-      if (u > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_STG_FREE], (u - 1) & 1, abort_flag));
+      if (u > 0 || seg == 0) {
+      if (nstored > 0)
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_STG_FREE], (nstored - 1) & 1, abort_flag));
       if (!ok) break;
       {
         uint8_t* stg_hi = smem + Cfg::OFF_STG;
@@ -316,7 +332,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(&bar[SB_STG_FULL]);
         if (i == 0) {
-          ok = tc::mbar_wait(&bar[SB_STG_FULL], u & 1, abort_flag);
+          ok = tc::mbar_wait(&bar[SB_STG_FULL], nstored & 1, abort_flag);
           if (ok) {
             const int z = bh * NC + c;
             for (int blk = 0; blk < NV / 64; ++blk) {
@@ -330,6 +346,8 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
+      }
+      ++nstored;
       }
       if (u == nsteps) break;  // the state leaving this chunk is not needed
       const int c0 = c * P.L, len = min(P.L, P.T - c0);
@@ -364,8 +382,9 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
       tc::mbar_arrive(&bar[SB_UFREE0 + ub]);
     }
     // backward with the initial state's gradient: after the first chunk's contribution
-    // the running state is the gradient of the state entering it
-    if (BWD && P.d0 != nullptr && ok && valid) {
+    // the running state is the gradient of the state entering it (this segment's share of
+    // it when the walk is split; state_fix adds the rest)
+    if (BWD && P.d0 != nullptr && last_seg && ok && valid) {
       float4* dst = reinterpret_cast<float4*>(P.d0 + ((size_t)bh * P.dqk + dk0 + i) * P.dhv + dv0);
 #pragma unroll
       for (int j = 0; j < NV; j += 4) dst[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
@@ -384,9 +403,129 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
   }
 }
 
+// Completion of a split walk: segment k > 0 started from the zero state, so each
+// of its stored states lacks the true state E entering the segment carried
+// through the segment's decay: the state after j more walk steps is
+// local_j + (beta_1 ... beta_j) E (the recurrence S <- beta S + U is linear, and
+// with the max state the stabilisers of the betas telescope, so the same factors
+// hold for the stored stabilised states).  Segments are completed in order; the
+// state entering segment k + 1 is the completed last slot of segment k, and the
+// first segment's slots are already complete.  The backward's initial-state
+// gradient, written by the last segment, is completed the same way.  One thread
+// per eight state elements (and one n element); CUDA cores, HBM-bound.
+template <bool BWD, bool EXPV>
+__global__ void __launch_bounds__(256) state_fix_kernel(
+    bf16* __restrict__ out, float* __restrict__ nout, size_t plane, const float* __restrict__ b,
+    const float* __restrict__ m, const float* __restrict__ m0, float* __restrict__ d0,
+    float* __restrict__ dn0, int T, int L, int NC, int dqk, int dhv, int seg_len, int nseg) {
+  const int bh = blockIdx.y;
+  const size_t nel = (size_t)dqk * dhv;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t e0 = (size_t)tid * 8;
+  const bool has_el = e0 < nel;
+  const bool has_n = EXPV && nout != nullptr && tid < dqk;
+  auto chunk_of = [&](int u) { return BWD ? NC - 1 - u : u; };
+  auto beta_of = [&](int c) -> float {
+    const size_t ct = (size_t)bh * T + (size_t)c * L;
+    const int len = min(L, T - c * L);
+    const float g = b[ct + len - 1];
+    if (!EXPV) return expf(g);
+    const float mc = m[ct + len - 1];
+    const float mp = chunk_mprev(m, ct, c, m0, bh);
+    return (c > 0 || m0 != nullptr) ? expf(g + mp - mc) : 0.f;
+  };
+  auto load8 = [&](int u, float (&x)[8]) {
+    const size_t o = ((size_t)bh * NC + chunk_of(u)) * nel + e0;
+    const uint4 h4 = *reinterpret_cast<const uint4*>(out + o);
+    const uint4 l4 = *reinterpret_cast<const uint4*>(out + plane + o);
+    const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w}, lw[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[e]);
+      const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162*>(&lw[e]);
+      x[2 * e] = __bfloat162float(h2.x) + __bfloat162float(l2.x);
+      x[2 * e + 1] = __bfloat162float(h2.y) + __bfloat162float(l2.y);
+    }
+  };
+  auto store8 = [&](int u, const float (&x)[8]) {
+    const size_t o = ((size_t)bh * NC + chunk_of(u)) * nel + e0;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bf16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+      hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[2 * e] - __bfloat162float(h0),
+                                                      x[2 * e + 1] - __bfloat162float(h1));
+      lw[e] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+    *reinterpret_cast<uint4*>(out + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(out + plane + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  };
+  auto nslot = [&](int u) -> float* { return nout + ((size_t)bh * NC + chunk_of(u)) * dqk + tid; };
+  // the state entering the second segment: stored by the first, which is complete
+  float E[8] = {}, En = 0.f;
+  if (has_el) load8(seg_len, E);
+  if (has_n) En = *nslot(seg_len);
+  for (int sg = 1; sg < nseg; ++sg) {
+    const int us = sg * seg_len, nlocal = min(seg_len, NC - us);
+    const bool last = us + nlocal == NC;
+    const int nslots = last ? nlocal : nlocal + 1;  // slot us is complete already
+    float D = 1.f;
+    for (int k = 1; k < nslots; ++k) {
+      D *= beta_of(chunk_of(us + k - 1));
+      if (has_el) {
+        float x[8];
+        load8(us + k, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = fmaf(D, E[e], x[e]);
+        store8(us + k, x);
+        if (k == nslots - 1 && !last) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) E[e] = x[e];
+        }
+      }
+      if (has_n) {
+        float* pn = nslot(us + k);
+        const float nv = fmaf(D, En, *pn);
+        *pn = nv;
+        if (k == nslots - 1 && !last) En = nv;
+      }
+    }
+    if (last && BWD && d0 != nullptr) {
+      // the initial state's gradient: one step more, through the first chunk
+      D *= beta_of(chunk_of(NC - 1));
+      if (has_el) {
+        float* pd = d0 + (size_t)bh * nel + e0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pd[e] = fmaf(D, E[e], pd[e]);
+      }
+      if (has_n && dn0 != nullptr) dn0[(size_t)bh * dqk + tid] = fmaf(D, En, dn0[(size_t)bh * dqk + tid]);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+
+// Segments of a split state walk: enough for the CTAs of all heads to fill the two
+// slots per SM of the 148 SMs, with at least four chunks per segment (1: no split).
+// A function of the problem alone, so the launch plan knows it without a device.
+static void state_split(const Problem& p, int& seg_len, int& nseg) {
+  const int ctas = (p.dhv / 64) * ((p.dqk + 127) / 128) * p.BH;
+  constexpr int kSlots = 2 * 148;
+  int want = kSlots / (ctas > 0 ? ctas : 1);
+  if (want > p.NC / 4) want = p.NC / 4;
+  if (want < 1) want = 1;
+  seg_len = (p.NC + want - 1) / want;
+  nseg = (p.NC + seg_len - 1) / seg_len;
+}
+
+bool state_split_needed(const Problem& p) {
+  int seg_len = 0, nseg = 0;
+  state_split(p, seg_len, nseg);
+  return nseg > 1;
+}
 
 bool state_tc_supported(const Problem& p) {
   return p.bf16() && (p.dqk == 64 || p.dqk == 128 || p.dqk == 256) && (p.dhv % 64 == 0);
@@ -411,7 +550,8 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
   P.b = b; P.li = li; P.m = m; P.inv_den = inv_den; P.da = da;
   P.out = out; P.nout = nout;
   P.plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
-  P.T = p.T; P.L = p.L; P.NC = p.NC; P.dqk = p.dqk; P.dhv = p.dhv;
+  P.T = p.T; P.L = p.L; P.NC = p.NC; P.dqk = p.dqk; P.dhv = p.dhv; P.BH = p.BH;
+  state_split(p, P.seg_len, P.nseg);
   P.scale = p.scale;
   P.init = init;
   P.d0 = d0;
@@ -422,7 +562,8 @@ static cudaError_t launch_state_tc(const Problem& p, const void* A, const void* 
   auto kern = state_tc_kernel<BWD, EXPV, NV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(p.dhv / NV), (unsigned)((p.dqk + 127) / 128), (unsigned)p.BH), block(256);
+  dim3 grid((unsigned)(p.dhv / NV), (unsigned)((p.dqk + 127) / 128), (unsigned)(p.BH * P.nseg)),
+      block(256);
   kern<<<grid, block, Cfg::SMEM, s>>>(tA, tB, tOh, tOl, P);
   return cudaGetLastError();
 }
@@ -453,6 +594,34 @@ cudaError_t launch_state_bwd_tc(const Problem& p, const BwdArgs& a, cudaStream_t
                                           a.inv_den, a.da, a.init, a.dC0, a.dn0, a.dCT, a.dnT, s);
   return launch_state_tc_nv<true, false>(p, a.q, a.dh, (bf16*)a.dC, a.dn, a.b, a.li, a.m,
                                          a.inv_den, a.da, a.init, a.dC0, a.dn0, a.dCT, a.dnT, s);
+}
+
+template <bool BWD, bool EXPV>
+static cudaError_t launch_fix(const Problem& p, bf16* out, float* nout, const float* b,
+                              const float* m, const InitState& init, float* d0, float* dn0,
+                              cudaStream_t s) {
+  int seg_len = 0, nseg = 0;
+  state_split(p, seg_len, nseg);
+  if (nseg < 2) return cudaErrorInvalidValue;  // the plan launches this only for a split walk
+  const size_t plane = (size_t)p.BH * p.NC * p.dqk * p.dhv;
+  const size_t nel = (size_t)p.dqk * p.dhv;
+  const float* m0 = (init.on() && EXPV) ? init.m : nullptr;
+  dim3 grid((unsigned)((nel / 8 + 255) / 256), (unsigned)p.BH), block(256);
+  state_fix_kernel<BWD, EXPV><<<grid, block, 0, s>>>(out, nout, plane, b, m, m0, d0, dn0, p.T, p.L,
+                                                     p.NC, p.dqk, p.dhv, seg_len, nseg);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_fwd_fix(const Problem& p, const FwdArgs& a, cudaStream_t s) {
+  if (p.exp_variant())
+    return launch_fix<false, true>(p, (bf16*)a.C, a.n, a.b, a.m, a.init, nullptr, nullptr, s);
+  return launch_fix<false, false>(p, (bf16*)a.C, nullptr, a.b, a.m, a.init, nullptr, nullptr, s);
+}
+
+cudaError_t launch_state_bwd_fix(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  if (p.exp_variant())
+    return launch_fix<true, true>(p, (bf16*)a.dC, a.dn, a.b, a.m, a.init, a.dC0, a.dn0, s);
+  return launch_fix<true, false>(p, (bf16*)a.dC, nullptr, a.b, a.m, a.init, a.dC0, nullptr, s);
 }
 
 cudaError_t fetch_tc_state_error(unsigned int* flag) {

@@ -264,13 +264,30 @@ def test_launch_plans_large_chunk_backward(lib, variant):
     """bf16, d_qk = d_hv = 128, chunk >= 256: the backward's intra-chunk products run on the
     large-chunk kernels after their gate table; other head dims keep the one-tile kernels."""
     for L in (256, 512, 1024, 4096):
-        assert _plan(1, (2, 4, 5000, 128, 128, L, variant, B.BF16)) == [
+        assert _plan(1, (8, 32, 5000, 128, 128, L, variant, B.BF16)) == [
             "bwd_token_prep", "state_bwd_tc", "bwd_xl_table", "dq_xl", "dk_xl", "dv_xl", "gate_grad"]
     for other in [(2, 4, 5000, 64, 64, 256, variant, B.BF16),
                   (2, 4, 5000, 128, 256, 512, variant, B.BF16),
                   (2, 4, 5000, 128, 128, 128, variant, B.BF16),
                   (2, 4, 5000, 128, 128, 256, variant, B.FP32)]:
         assert not any(n.endswith("_xl") and n != "output_fwd_xl" for n in _plan(1, other)), other
+
+
+@pytest.mark.parametrize("variant", [B.SIG, B.EXP], ids=["sig", "exp"])
+def test_launch_plans_split_state_walks_for_few_heads(lib, variant):
+    """Few heads with many chunks: the state kernels walk each head's chunks in segments and a
+    completion pass follows each; enough heads to fill the GPU, or fewer than eight chunks
+    (at least four per segment), keep one walk per head."""
+    long_few = (1, 8, 65536, 256, 512, 1024, variant, B.BF16)  # the long-context workload
+    fwd, bwd = _plan(0, long_few), _plan(1, long_few)
+    assert fwd[fwd.index("state_fwd_tc") + 1] == "state_fwd_fix", fwd
+    assert bwd[bwd.index("state_bwd_tc") + 1] == "state_bwd_fix", bwd
+    assert len(bwd) <= 8  # the plan's step array holds eight
+    for sizes in [(8, 32, 8192, 128, 128, 256, variant, B.BF16),   # 256 heads: one walk each
+                  (1, 2, 448, 64, 64, 64, variant, B.BF16)]:       # 7 chunks: too few to split
+        names = _plan(0, sizes) + _plan(1, sizes)
+        assert not any(n.endswith("_fix") for n in names), (sizes, names)
+    assert "state_bwd_fix" in _plan(1, (1, 2, 4096, 128, 128, 256, variant, B.BF16))
 
 
 def test_serial_launch_switch_needs_no_device(lib):

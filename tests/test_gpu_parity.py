@@ -60,6 +60,9 @@ SMALL = [
     ("exp_bf16_chunk64_t1", 1, 2, 1, 128, 128, 64, EXP, BF, -1.0, 3.0),
     ("sig_bf16_chunk64_dqk256_dhv512", 1, 1, 200, 256, 512, 64, SIG, BF, 0.0, 3.0),
     ("exp_bf16_chunk64_dqk64_dhv128_t65", 1, 2, 65, 64, 128, 64, EXP, BF, 0.0, 3.0),
+    # one head, 32 chunks: the state walks run as 8 segments of 4 chunks plus a completion
+    ("exp_bf16_chunk64_d128_split8", 1, 1, 2048, 128, 128, 64, EXP, BF, -2.0, 3.0),
+    ("sig_bf16_chunk128_d64_split4_ragged", 1, 2, 2000, 64, 64, 128, SIG, BF, 0.0, 3.0),
 ]
 
 

@@ -31,6 +31,10 @@ CASES = [
     ("bf16_chunk128", BF, 128, 128, 300),
     ("bf16_chunk256_ragged", BF, 128, 256, 700),
     ("bf16_d64_chunk512", BF, 64, 512, 600),
+    # few heads, many chunks: the state walks run in segments (4 of 4 chunks; 2 of 6 and 5),
+    # completed from the initial state, the final state's gradient and into dstate_in
+    ("bf16_chunk64_split4", BF, 64, 64, 1000),
+    ("bf16_chunk256_split2_ragged", BF, 128, 256, 2600),
 ]
 
 
