@@ -172,16 +172,51 @@ def committed_traffic(kernel, workload):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons during the timed region.
+
+    Read in-process through NVML every 5 ms by a background thread (a region of a few tens
+    of milliseconds still gets several samples); nvidia-smi polling at 200 ms when NVML
+    cannot be loaded.  Reading clocks changes nothing on the GPU."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h): the slowdowns that reject a number, and the cap
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                   ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_s=0.005):
         self.gpu_index = gpu_index
+        self.period_s = period_s
         self.proc = None
         self.out = None
+        self.thread = None
+        self.rows = []
 
     def start(self):
+        try:
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index)
+            max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+            self.stop_event = threading.Event()
+
+            def loop():
+                while True:
+                    try:
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                        bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle))
+                    except Exception:  # noqa: BLE001
+                        break
+                    self.rows.append({"sm": sm, "max": max_mhz, "bits": bits})
+                    if self.stop_event.wait(self.period_s):
+                        break
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # noqa: BLE001
+            self.thread = None
         try:
             self.out = open(os.path.join("/tmp", f"mlstm_clocks_{os.getpid()}.csv"), "w")
             self.proc = subprocess.Popen(
@@ -190,7 +225,19 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _summary(self, rows, reasons):
+        if not rows:
+            return None
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_event.set()
+            self.thread.join(timeout=5)
+            reasons = {name for r in self.rows for name, bit in self.REASON_BITS if r["bits"] & bit}
+            return self._summary(self.rows, reasons)
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -211,25 +258,22 @@ class ClockSampler:
                 except ValueError:
                     continue
         os.unlink(self.out.name)
-        if not rows:
-            return None
         reasons = set()
         for r in rows:
             for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
                               ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
                 if r[key].lower() == "active":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
-                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows)}
+        return self._summary(rows, reasons)
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle legs
 # ---------------------------------------------------------------------------
 
-def oracle_sample(spec, heads, budget_s=20.0):
-    """Time the fp64 oracle (chunkwise forward + parallel-form backward) on whole heads."""
+def oracle_sample(spec, heads, budget_s=20.0, tokens=None):
+    """Time the fp64 oracle (chunkwise forward + parallel-form backward) on whole heads, or on
+    heads of `tokens` tokens (a multiple of the chunk) when given."""
     import numpy as np
     import oracle
     from mlstm_chunkwise_attention_b200.synthetic import make_inputs
@@ -239,6 +283,9 @@ def oracle_sample(spec, heads, budget_s=20.0):
     except Exception:  # noqa: BLE001
         cores = 1
     T, dqk, dhv, L, var = spec["T"], spec["d_qk"], spec["d_hv"], spec["chunk"], spec["variant"]
+    T_all = T
+    if tokens is not None:
+        T = tokens
     done, elapsed = [], 0.0
     for (b, hh) in heads:
         x = make_inputs(1, 1, T, dqk, dhv, seed=spec["seed"] * 1000 + b * 64 + hh,
@@ -256,25 +303,37 @@ def oracle_sample(spec, heads, budget_s=20.0):
     flops = len(done) * (flops_fwd(T, dqk, dhv, L) + flops_bwd(T, dqk, dhv, L))
     return {"value": flops / elapsed / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
             "seconds": elapsed, "heads": len(done),
+            "tokens": T,
             "sample": f"{len(done)} of {spec['B'] * spec['NH']} heads of the workload "
-                      f"(T={T}, d={dqk}/{dhv}, chunk {L}): fp64 chunkwise forward + parallel-form "
-                      f"backward in numpy; throughput scaled by the algorithmic FLOPs of the heads run"}
+                      f"(T={T_all}, d={dqk}/{dhv}, chunk {L})"
+                      + (f", each on {T} of its {T_all} tokens" if T != T_all else "")
+                      + ": fp64 chunkwise forward + parallel-form backward in numpy; throughput "
+                        "scaled by the algorithmic FLOPs of the tokens run"}
 
 
 def run_reference(args, spec):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    import math
     from mlstm_chunkwise_attention_b200.synthetic import sample_heads
     heads = sample_heads(spec["B"], spec["NH"], args.warmup + args.steps, 4242)
+    T, dqk, dhv, L = spec["T"], spec["d_qk"], spec["d_hv"], spec["chunk"]
+    # Each step is one head; when --steps --warmup heads of the whole sequence would take more
+    # than about 150 s, each step runs a head on its first Ts tokens instead, Ts sized from one
+    # untimed calibration head (the parallel-form backward grows as tokens squared).
+    per_step = 150.0 / (args.warmup + args.steps)
+    Tc = min(T, 8 * L)
+    t_c = max(oracle_sample(spec, [heads[0]], budget_s=0.0, tokens=Tc)["seconds"], 1e-6)
+    Ts = T if t_c * (T / Tc) ** 2 <= per_step else int(Tc * math.sqrt(per_step / t_c)) // L * L
+    Ts = min(T, max(L, Ts))
     times = []
     info = None
     for i, hd in enumerate(heads):
-        info = oracle_sample(spec, [hd], budget_s=0.0)
+        info = oracle_sample(spec, [hd], budget_s=0.0, tokens=Ts)
         if i >= args.warmup:
             times.append(info["seconds"])
-    T, dqk, dhv, L = spec["T"], spec["d_qk"], spec["d_hv"], spec["chunk"]
-    per_head = flops_fwd(T, dqk, dhv, L) + flops_bwd(T, dqk, dhv, L)
+    per_head = flops_fwd(Ts, dqk, dhv, L) + flops_bwd(Ts, dqk, dhv, L)
     total_s = sum(times)
     value = per_head * len(times) / total_s / 1e12
     line = {
@@ -284,8 +343,9 @@ def run_reference(args, spec):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(spec, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
-                         "sample": "each step: one head of the workload, fp64 chunkwise forward + "
-                                   "parallel-form backward (numpy)"},
+                         "sample": "each step: one head of the workload"
+                                   + (f" on its first {Ts} of {T} tokens" if Ts != T else "")
+                                   + ", fp64 chunkwise forward + parallel-form backward (numpy)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -607,7 +667,7 @@ def main():
     global WORKLOAD
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
