@@ -236,6 +236,11 @@ class ClockSampler:
         if self.thread is not None:
             self.stop_event.set()
             self.thread.join(timeout=5)
+            try:  # release NVML before the per-kernel timing that follows
+                import pynvml
+                pynvml.nvmlShutdown()
+            except Exception:  # noqa: BLE001
+                pass
             reasons = {name for r in self.rows for name, bit in self.REASON_BITS if r["bits"] & bit}
             return self._summary(self.rows, reasons)
         if self.proc is None:

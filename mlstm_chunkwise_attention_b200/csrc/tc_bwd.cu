@@ -69,8 +69,11 @@ struct BwdTcCfg {
 };
 
 enum {
-  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_INTER, BB_ACC, BB_DONE, BB_STG, BB_COUNT
+  BB_FULL0 = 0, BB_EMPTY0 = 4, BB_X0 = 8, BB_Y = 10, BB_INTER, BB_ACC, BB_DONE, BB_STG,
+  BB_DRAIN,  // the MMA thread's last commit when it gives up
+  BB_COUNT
 };
+static_assert(BB_COUNT <= 16, "barrier slots");
 
 }  // namespace
 
@@ -225,6 +228,8 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
       // stay until the last copies this thread issued have landed
       if (ok && it > 0)
         ok = tc::mbar_wait(&bar[BB_FULL0 + (it - 1) % ST], ((it - 1) / ST) & 1, abort_flag);
+      // gave up: every copy still in flight lands before the CTA exits
+      if (!ok) tc::drain_ring(&bar[BB_FULL0], ST, it);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -303,6 +308,7 @@ __global__ void __launch_bounds__(192, NXBUF == 1 ? 2 : 1) intra_bwd_tc_kernel(
         if (ok && NXBUF == 1 && jj + 1 < np) ok = issue_score(jj + 1);
       }
       tc::tc_commit(&bar[BB_DONE]);
+      if (!ok) tc::drain_mma(&bar[BB_DRAIN]);  // no product still writes TMEM or reads smem
     }
   } else {
     // ------------------------------------------------------------ tile rows

@@ -55,7 +55,7 @@ struct WalkCfg {
   static constexpr int OFF_WN = OFF_W + 8 * 128 * 4;
   static constexpr int WN_BYTES = 4096;
   static constexpr int OFF_BAR = OFF_WN + 2 * WN_BYTES;
-  static constexpr int OFF_TMEM = OFF_BAR + 8 * 8;
+  static constexpr int OFF_TMEM = OFF_BAR + 9 * 8;
   static constexpr size_t SMEM = 1024 + OFF_TMEM + 16;
   static constexpr uint32_t TMEM_COLS = 512;  // dC, score / transformed tile, dv, dk
 };
@@ -69,7 +69,9 @@ enum { F_PC0 = 0, F_PC1, F_PE0, F_PE1, F_WV0, F_WV1, F_DN, F_DOT };
 // products after A, B, C; and the state update on its own barrier, which can complete
 // before the rows wait for C's products).  Each barrier's phases strictly alternate
 // with its waiter, so parity waits cannot alias.
-enum { BW_Q = 0, BW_K, BW_V, BW_H, BW_R, BW_D, BW_M, BW_S, BW_COUNT };
+// BW_DRAIN: the MMA thread's last commit when it gives up.
+enum { BW_Q = 0, BW_K, BW_V, BW_H, BW_R, BW_D, BW_M, BW_S, BW_DRAIN, BW_COUNT };
+static_assert(BW_COUNT <= 9, "barrier slots");
 
 using walk::sw_off;
 constexpr auto rows_and = walk::rows_and<256>;
@@ -217,7 +219,10 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
         }
         tc::tc_commit(&bar[BW_S]);
       }
-      if (!ok) abort_flag.raise();
+      if (!ok) {
+        abort_flag.raise();
+        tc::drain_mma(&bar[BW_DRAIN]);  // no product still writes TMEM or reads smem
+      }
     }
   } else {
     // ------------------------------------------------------------ rows
@@ -250,7 +255,9 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[b]);
     };
+    uint32_t fills[4] = {0, 0, 0, 0};  // copies the issuer started on BW_Q, BW_K, BW_V, BW_H
     auto load_tile = [&](int b, uint8_t* dst, const CUtensorMap* tm, int c) {
+      ++fills[b - BW_Q];
       tc::mbar_arrive_expect_tx(&bar[b], Cfg::TILE);
       tc::tma_load_3d(dst, tm, &bar[b], 0, c * 128, bh);
       tc::tma_load_3d(dst + 16384, tm, &bar[b], 64, c * 128, bh);
@@ -624,6 +631,9 @@ __global__ void __launch_bounds__(288, 1) bwd_walk_kernel(
         for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
       }
       if (EXPV && lead) P.dn0[(size_t)bh * 128 + row] = dn;
+    }
+    if (issuer && !ok) {  // gave up: the copies still in flight land before the CTA exits
+      for (int i = 0; i < 4; ++i) tc::drain_last(&bar[BW_Q + i], fills[i]);
     }
     if (issuer) tc::bulk_wait_all();
     if (!ok) abort_flag.raise();

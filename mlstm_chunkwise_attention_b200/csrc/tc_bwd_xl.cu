@@ -96,7 +96,8 @@ enum {
   Y_OF0 = 20,  // Acc complete (MMA commit), per Acc buffer
   Y_OE0 = 22,  // Acc read out (512 threads), per Acc buffer
   Y_XS0 = 24,  // dot-product shares exchanged (128 threads), per Acc buffer and lane quarter
-  Y_COUNT = 32
+  Y_DRAIN = 32,  // the MMA thread's last commit when it gives up
+  Y_COUNT = 33
 };
 
 struct BxItem {
@@ -295,6 +296,7 @@ __global__ void __launch_bounds__(kBxThreads, 1) intra_bwd_xl_kernel(
       tc::prefetch_tmap(&tm_glo);
     }
     int it = 0, gb = 0;
+    uint32_t na = 0;  // row-tile fills issued
     for (int k = bx_first(); k < P.total && ok; k = bx_succ(k)) {
       BxItem I;
       if (!bx_item<KIND>(k, P, I)) continue;
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(kBxThreads, 1) intra_bwd_xl_kernel(
         for (int kb = 0; kb < 2; ++kb)
           tc::tma_load_3d(sa + kb * 16384, &tm_a, af, kb * 64, I.c * P.L + I.t0, I.bh);
       }
+      ++na;
       const int nent = I.np + (I.inter ? 2 : 0);
       for (int e = 0; e < nent && ok; ++e, ++gb) {
         const int st = gb % NB;
@@ -345,6 +348,11 @@ __global__ void __launch_bounds__(kBxThreads, 1) intra_bwd_xl_kernel(
         }
       }
       ++it;
+    }
+    // gave up: the copies this warp issued land before the CTA exits
+    if (!ok && leader) {
+      tc::drain_ring(&bar[Y_AF0], NA, na);
+      tc::drain_ring(&bar[Y_BF0], NB, (uint32_t)gb);
     }
   } else if (warp == kBxEWarp) {
     // ------------------------------------------------------------ E producer
@@ -383,6 +391,7 @@ __global__ void __launch_bounds__(kBxThreads, 1) intra_bwd_xl_kernel(
         }
       }
     }
+    if (!ok && leader) tc::drain_ring(&bar[Y_EF0], NE, (uint32_t)ge);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Lane 0 alone walks the schedule, waits and issues; the shared-memory descriptors
@@ -494,6 +503,7 @@ __global__ void __launch_bounds__(kBxThreads, 1) intra_bwd_xl_kernel(
         k = kn;
         I = N;
       }
+      if (!ok) tc::drain_mma(&bar[Y_DRAIN]);  // no product still writes TMEM or reads smem
     }
   } else {
     // ------------------------------------------------------------ gate transform + epilogue

@@ -107,6 +107,23 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// Wind-down of a thread that gave up after issuing fills (TMA or bulk copies)
+// into a ring of `stages` full barriers, `issued` fills in all: the last
+// min(issued, stages) may still be landing in shared memory; wait for each,
+// bounded, so nothing lands after the CTA has exited.
+__device__ __forceinline__ void drain_ring(uint64_t* full0, uint32_t stages, uint32_t issued) {
+  const uint32_t n = issued < stages ? issued : stages;
+  for (uint32_t k = 1; k <= n; ++k) {
+    const uint32_t idx = issued - k;
+    mbar_drain(&full0[idx % stages], (idx / stages) & 1);
+  }
+}
+
+// The same for one barrier that takes one fill at a time, `issued` fills in all.
+__device__ __forceinline__ void drain_last(uint64_t* full, uint32_t issued) {
+  if (issued > 0) mbar_drain(full, (issued - 1) & 1);
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core / TMA) before signalling the thread that issues it.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -192,6 +209,14 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// Wind-down of the MMA-issuing thread: one more commit, on a barrier used for
+// nothing else, completes when every tensor-core operation it issued has
+// (their shared-memory reads and TMEM writes included); wait for it, bounded.
+__device__ __forceinline__ void drain_mma(uint64_t* drain_bar) {
+  tc_commit(drain_bar);
+  mbar_drain(drain_bar, 0);
 }
 
 // D[tmem] (+)= A[smem] * B[smem], bf16 inputs, fp32 accumulator.

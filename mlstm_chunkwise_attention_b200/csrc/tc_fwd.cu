@@ -60,7 +60,8 @@ struct OutTcCfg {
   static_assert(C_BYTES <= KC_BYTES, "the lo plane of C_prev must fit the K region");
 };
 
-enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_STG, B_COUNT };
+enum { B_Q = 0, B_K, B_V, B_C, B_S, B_P, B_PV, B_QS, B_O, B_STG, B_DRAIN, B_COUNT };
+static_assert(B_COUNT <= 16, "barrier slots");
 
 }  // namespace
 
@@ -137,10 +138,12 @@ __global__ void __launch_bounds__(192, 2) output_fwd_tc_kernel(
       tc::mbar_arrive_expect_tx(&bar[B_V], Cfg::V_BYTES);
       for (int vb = 0; vb < Cfg::VB; ++vb)
         tc::tma_load_3d(sV + vb * 16384, &tm_v, &bar[B_V], dv0 + vb * 64, c0, bh);
+      bool c_issued = false;
       if (has_prev) {
         // both planes of C_prev once P V is done: hi where V was, lo where P was
         ok = tc::mbar_wait(&bar[B_PV], 0, abort_flag);
         if (ok) {
+          c_issued = true;
           tc::mbar_arrive_expect_tx(&bar[B_C], 2 * Cfg::C_BYTES);
           for (int vb = 0; vb < Cfg::VB; ++vb) {
             tc::tma_load_3d(sV + vb * DQK * 128, &tm_chi, &bar[B_C], dv0 + vb * 64, 0, bh * NC + c);
@@ -151,6 +154,12 @@ __global__ void __launch_bounds__(192, 2) output_fwd_tc_kernel(
       // do not leave while a copy this thread issued may still be landing
       if (ok) ok = tc::mbar_wait(&bar[B_V], 0, abort_flag);
       if (ok && has_prev) ok = tc::mbar_wait(&bar[B_C], 0, abort_flag);
+      if (!ok) {  // gave up: the copies still in flight land before the CTA exits
+        tc::drain_last(&bar[B_Q], 1);
+        tc::drain_last(&bar[B_K], 1);
+        tc::drain_last(&bar[B_V], 1);
+        tc::drain_last(&bar[B_C], c_issued ? 1u : 0u);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -195,6 +204,7 @@ __global__ void __launch_bounds__(192, 2) output_fwd_tc_kernel(
         }
       }
       tc::tc_commit(&bar[B_O]);
+      if (!ok) tc::drain_mma(&bar[B_DRAIN]);  // no product still writes TMEM or reads smem
     }
   } else {
     // ------------------------------------------------------------ gate rows + epilogue

@@ -69,7 +69,9 @@ struct FwalkCfg {
 enum { F_CF0 = 0, F_CF1, F_KP0, F_KP1, F_RS0, F_RS1, F_MB };
 // mbarriers: Q tile, K/V sets, rows -> MMA (A, B), rows -> MMA (D), MMA -> rows
 // (after A, B), state update done.  Each barrier's phases alternate with its waiter.
-enum { BF_Q = 0, BF_KV0, BF_KV1, BF_R, BF_D, BF_M, BF_S, BF_COUNT };
+// BF_DRAIN: the MMA thread's last commit when it gives up.
+enum { BF_Q = 0, BF_KV0, BF_KV1, BF_R, BF_D, BF_M, BF_S, BF_DRAIN, BF_COUNT };
+static_assert(BF_COUNT <= 8, "barrier slots");
 
 }  // namespace
 
@@ -204,7 +206,10 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         }
         tc::tc_commit(&bar[BF_S]);
       }
-      if (!ok) abort_flag.raise();
+      if (!ok) {
+        abort_flag.raise();
+        tc::drain_mma(&bar[BF_DRAIN]);  // no product still writes TMEM or reads smem
+      }
     }
   } else {
     // ------------------------------------------------------------ rows
@@ -240,7 +245,9 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[b]);
     };
+    uint32_t nq_fills = 0, nkv_fills[2] = {0, 0};  // copies the issuer started, per barrier
     auto load_q = [&](int c) {
+      ++nq_fills;
       tc::mbar_arrive_expect_tx(&bar[BF_Q], TILE);
       tc::tma_load_3d(sQ, &tmQ, &bar[BF_Q], 0, c * 128, bh);
       tc::tma_load_3d(sQ + 16384, &tmQ, &bar[BF_Q], 64, c * 128, bh);
@@ -248,6 +255,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     auto load_kv = [&](int c) {
       uint8_t* st = set_of(c);
       uint64_t* b = &bar[(c & 1) ? BF_KV1 : BF_KV0];
+      ++nkv_fills[c & 1];
       tc::mbar_arrive_expect_tx(b, 2 * TILE);
       tc::tma_load_3d(st, &tmK, b, 0, c * 128, bh);
       tc::tma_load_3d(st + 16384, &tmK, b, 64, c * 128, bh);
@@ -562,6 +570,11 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     }
     // the last chunk's hand-over: every product has completed
     if (ok) ok = wait_state();
+    if (issuer && !ok) {  // gave up: the copies still in flight land before the CTA exits
+      tc::drain_last(&bar[BF_Q], nq_fills);
+      tc::drain_last(&bar[BF_KV0], nkv_fills[0]);
+      tc::drain_last(&bar[BF_KV1], nkv_fills[1]);
+    }
     if (issuer) tc::bulk_wait_all();
     if (!ok) abort_flag.raise();
   }

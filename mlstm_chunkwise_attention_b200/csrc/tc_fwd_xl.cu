@@ -87,7 +87,8 @@ enum {
   X_OF0 = 34,  // O complete (MMA commit), per O buffer
   X_OE0 = 36,  // O read out (256 threads), per O buffer
   X_XS0 = 38,  // normaliser shares exchanged (128 threads), per O buffer and lane quarter
-  X_COUNT = 46
+  X_DRAIN = 46,  // the MMA thread's last commit when it gives up
+  X_COUNT = 47
 };
 
 constexpr int kXlThreads = 608;    // K producer, MMA, 16 transform warps, V producer
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
         tc::prefetch_tmap(&tm_c);
       }
       int it = 0, g = 0;
+      uint32_t nq = 0;  // Q fills issued
       for (int k = xl_first(); k < total && ok; k = xl_succ(k)) {
         XlItem I;
         if (!xl_item(k, BH, NC, NVB, ntq, T, L, has_init, I)) continue;
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           tc::bulk_load(rp + 1024, tb + 2 * L + I.t0, 512, qf);
           if (nv) tc::bulk_load(rp + 1536, gn + ((size_t)I.bh * NC + I.c) * DQK, DQK * 4, qf);
         }
+        ++nq;
         const int nsteps = I.nkv + (I.pseudo ? 1 : 0);
         for (int s = 0; s < nsteps && ok; ++s, ++g) {
           const int kst = g % NK;
@@ -317,6 +320,11 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           }
         }
         ++it;
+      }
+      // gave up: the copies this warp issued land before the CTA exits
+      if (!ok && leader) {
+        tc::drain_ring(&bar[X_QF0], NQ, nq);
+        tc::drain_ring(&bar[X_KF0], NK, (uint32_t)g);
       }
     }
   } else if (warp == kXlVWarp) {
@@ -349,6 +357,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
           }
         }
       }
+      if (!ok && leader) tc::drain_ring(&bar[X_VF0], NV, (uint32_t)gv);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -456,6 +465,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
         k = kn;
         I = N;
       }
+      if (!ok) tc::drain_mma(&bar[X_DRAIN]);  // no product still writes TMEM or reads smem
     }
   } else {
     // ------------------------------------------------------------ gate transform + epilogue

@@ -61,8 +61,11 @@ struct StateTcCfg {
 
 enum {
   SB_FULL0 = 0, SB_SCALED0 = 3, SB_EMPTY0 = 6, SB_U0 = 9, SB_UFREE0 = 11, SB_STG_FULL = 13,
-  SB_STG_FREE = 14, SB_COUNT = 15
+  SB_STG_FREE = 14,
+  SB_DRAIN = 15,  // the MMA thread's last commit when it gives up
+  SB_COUNT = 16
 };
+static_assert(SB_COUNT <= 16, "barrier slots");
 
 }  // namespace
 
@@ -169,6 +172,8 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         const uint32_t last = it - 1;
         ok = tc::mbar_wait(&bar[SB_FULL0 + last % Cfg::STAGES], (last / Cfg::STAGES) & 1, abort_flag);
       }
+      // gave up: every copy still in flight lands before the CTA exits
+      if (!ok) tc::drain_ring(&bar[SB_FULL0], Cfg::STAGES, it);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -210,6 +215,7 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         if (!ok) break;
         tc::tc_commit(&bar[SB_U0 + ub]);
       }
+      if (!ok) tc::drain_mma(&bar[SB_DRAIN]);  // no product still writes TMEM or reads smem
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ scaling (one token row per thread)
