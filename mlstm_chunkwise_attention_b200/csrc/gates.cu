@@ -28,7 +28,8 @@ namespace mlstm {
 // factor separates as exp2(R_t + MU_j) * KP_s over a block j of 32 keys that
 // lies wholly before row t; both factors are at most 1, because the max state
 // m_t bounds every b_t - b_s + log i_s with s <= t (SIG: log i <= 0, b falls).
-// One warp handles one block of 32 keys, so MU_j is a warp max.
+// One warp handles one block of 32 keys, so MU_j is a warp max.  The CTA covers
+// chunks blockIdx.y, blockIdx.y + gridDim.y, ... of its head.
 template <bool EXPV>
 __device__ void write_xl_tables(const float* b, const float* li, const float* m, float* xt,
                                 size_t base, int T, int L, int NC, float scale,
@@ -36,8 +37,10 @@ __device__ void write_xl_tables(const float* b, const float* li, const float* m,
   constexpr float kLog2e = 1.4426950408889634f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int stride = xl_table_stride(L), bpc = L / 32;
-  for (int blk = warp; blk < NC * bpc; blk += nwarps) {
-    const int c = blk / bpc, r = (blk % bpc) * 32 + lane;
+  const int G = (int)gridDim.y, cy = (int)blockIdx.y;
+  const int nloc = (NC - cy + G - 1) / G;  // this CTA's chunks
+  for (int blk = warp; blk < nloc * bpc; blk += nwarps) {
+    const int c = cy + G * (blk / bpc), r = (blk % bpc) * 32 + lane;
     const int t = c * L + r;
     const bool valid = t < T;
     float R = -INFINITY, QF = 0.f, FL = 1.f, CC = -INFINITY;
@@ -73,7 +76,10 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const unsigned full = 0xffffffffu;
 
-  for (int c = warp; c < NC; c += nwarps) {
+  // mLSTMsig has no dependency between chunks, so a head's chunks may be spread over
+  // gridDim.y CTAs (chunks blockIdx.y, blockIdx.y + gridDim.y, ...); mLSTMexp's max-state
+  // scan needs them all in one CTA (gridDim.y == 1)
+  for (int c = (int)blockIdx.y + (int)gridDim.y * warp; c < NC; c += (int)gridDim.y * nwarps) {
     const int c0 = c * L;
     const int len = min(L, T - c0);
     const int per = (len + 31) / 32;
@@ -156,7 +162,14 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
 
 cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   const size_t smem = p.exp_variant() ? 2 * sizeof(float) * (size_t)p.NC : 0;
-  dim3 grid(p.BH), block(256);
+  // mLSTMsig with few heads: several CTAs per head, one warp per chunk, up to two CTAs per SM
+  int per_head = 1;
+  if (!p.exp_variant()) {
+    const int want = (2 * 148 + p.BH - 1) / p.BH, most = (p.NC + 7) / 8;
+    per_head = want < most ? want : most;
+    if (per_head < 1) per_head = 1;
+  }
+  dim3 grid(p.BH, per_head), block(256);
   if (p.bf16()) {
     if (p.exp_variant())
       gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale), a.init.on(), a.init.on() && p.exp_variant() ? a.init.m : nullptr);
