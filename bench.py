@@ -39,7 +39,7 @@ KERNEL_SOURCES = {
     "dk_tc": "tc_bwd.cu", "dv_tc": "tc_bwd.cu", "state_fwd_tc": "tc_state.cu",
     "output_fwd_xl": "tc_fwd_xl.cu", "bwd_xl_table": "tc_bwd_xl.cu", "dq_xl": "tc_bwd_xl.cu",
     "dk_xl": "tc_bwd_xl.cu", "dv_xl": "tc_bwd_xl.cu", "state_fwd_fix": "tc_state.cu",
-    "state_bwd_fix": "tc_state.cu",
+    "state_bwd_fix": "tc_state.cu", "gate_grad_sums": "gates.cu",
     "state_bwd_tc": "tc_state.cu", "dkv_walk_tc": "tc_bwd_walk.cu", "fwd_walk_tc": "tc_fwd_walk.cu",
 }
 
@@ -91,6 +91,8 @@ def kernel_costs(T, dqk, dhv, L, exp_variant, io_bytes):
         # completion of a segmented state walk: every state read and written once
         "state_fwd_fix": (0, 2 * st_full + (2 * stn if exp_variant else 0)),
         "state_bwd_fix": (0, 2 * st_full + (2 * stn if exp_variant else 0)),
+        # segment totals of q.dq - k.dk (few heads): pq and pk read once
+        "gate_grad_sums": (0, 2 * tok_f),
         # state gradients, dk and dv in one pass: the state-gradient recurrence and the
         # dk, dv contractions; q, k, v, dh read once, dk, dv and k.dk written, the state
         # gradients never leave the chip

@@ -264,19 +264,49 @@ cudaError_t launch_bwd_token_prep(const Problem& p, const BwdArgs& a, cudaStream
 // d log f_r = sum_{t>=r} sum_{s<r} G_ts = sum_{t>=r} (q_t . dq_t - k_t . dk_t),
 // a reverse cumulative sum over the whole sequence.  Then the chain rule to
 // the preactivations: d/dx logsigmoid(x) = sigmoid(-x); the exponential input
-// gate has log i = i~.  One CTA (32 warps) per (b, h); each warp owns one
-// contiguous segment of T.
+// gate has log i = i~.  One CTA (32 warps) per (b, h) and segment of T (one
+// segment, or with few heads gridDim.y of them, whose totals gate_grad_sums
+// wrote first); each warp owns one contiguous piece of its CTA's segment.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void grad_segment(int T, int& tb, int& te) {
+  const int G = (int)gridDim.y, Tc = (T + G - 1) / G;
+  tb = min(T, (int)blockIdx.y * Tc);
+  te = min(T, tb + Tc);
+}
+
+// The total of q.dq - k.dk over each segment of a head, for the segments after it.
+__global__ void __launch_bounds__(256) gate_grad_sums_kernel(const float* __restrict__ pq,
+                                                             const float* __restrict__ pk,
+                                                             float* __restrict__ gsum, int T) {
+  __shared__ float s_w[8];
+  const size_t base = (size_t)blockIdx.x * T;
+  int tb, te;
+  grad_segment(T, tb, te);
+  float part = 0.f;
+  for (int t = tb + (int)threadIdx.x; t < te; t += blockDim.x) part += pq[base + t] - pk[base + t];
+  part = warp_sum(part);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_w[warp] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_w[w];
+    gsum[(size_t)blockIdx.x * gridDim.y + blockIdx.y] = tot;
+  }
+}
+
 template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(1024) gate_grad_kernel(
     const TIO* __restrict__ ig, const TIO* __restrict__ fg, const float* __restrict__ pq,
     const float* __restrict__ pk, TIO* __restrict__ dig, TIO* __restrict__ dfg, int T,
-    const float* __restrict__ fdot) {
+    const float* __restrict__ fdot, const float* __restrict__ gsum) {
   __shared__ float s_tot[32];
   const size_t base = (size_t)blockIdx.x * T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int seg = (T + 31) / 32;
-  const int sb = min(warp * seg, T), se = min(sb + seg, T);
+  int tb, te;
+  grad_segment(T, tb, te);
+  const int seg = (te - tb + 31) / 32;
+  const int sb = min(tb + warp * seg, te), se = min(sb + seg, te);
   float part = 0.f;
   for (int t = sb + lane; t < se; t += 32) part += pq[base + t] - pk[base + t];
   part = warp_sum(part);
@@ -289,8 +319,12 @@ __global__ void __launch_bounds__(1024) gate_grad_kernel(
   }
   __syncthreads();
   // a loss on the final state adds <dC_T, C_T> + <dn_T, n_T> to every d log f_r: the
-  // final state is one more row after the last token, and it reads every key
-  float carry = s_tot[warp] + (fdot != nullptr ? fdot[blockIdx.x] : 0.f);
+  // final state is one more row after the last token, and it reads every key; the later
+  // segments of the head add their totals (summed from the last one down)
+  float later = 0.f;
+  for (int y = (int)gridDim.y - 1; y > (int)blockIdx.y; --y)
+    later += gsum[(size_t)blockIdx.x * gridDim.y + y];
+  float carry = s_tot[warp] + (fdot != nullptr ? fdot[blockIdx.x] : 0.f) + later;
   for (int e = se; e > sb; e -= 32) {
     const int t = e - 32 + lane;
     const bool valid = t >= sb;
@@ -308,18 +342,36 @@ __global__ void __launch_bounds__(1024) gate_grad_kernel(
   }
 }
 
+int gate_grad_segments(const Problem& p) {
+  // few heads: enough CTAs for the 148 SMs, each at least 4096 tokens, at most 64
+  int g = 148 / (p.BH > 0 ? p.BH : 1);
+  const int most = p.T / 4096;
+  if (g > most) g = most;
+  if (g > 64) g = 64;
+  return g < 1 ? 1 : g;
+}
+
+cudaError_t launch_gate_grad_sums(const Problem& p, const BwdArgs& a, cudaStream_t s) {
+  const int G = gate_grad_segments(p);
+  if (G < 2 || a.gsum == nullptr) return cudaErrorInvalidValue;  // planned only for a split
+  gate_grad_sums_kernel<<<dim3(p.BH, G), 256, 0, s>>>(a.pq, a.pk, a.gsum, p.T);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gate_grad(const Problem& p, const BwdArgs& a, cudaStream_t s) {
-  dim3 grid(p.BH), block(1024);
+  const int G = gate_grad_segments(p);
+  if (G > 1 && a.gsum == nullptr) return cudaErrorInvalidValue;
+  dim3 grid(p.BH, G), block(1024);
   if (p.bf16()) {
     if (p.exp_variant())
-      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot);
+      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot, a.gsum);
     else
-      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot);
+      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot, a.gsum);
   } else {
     if (p.exp_variant())
-      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot);
+      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot, a.gsum);
     else
-      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot);
+      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot, a.gsum);
   }
   return cudaGetLastError();
 }

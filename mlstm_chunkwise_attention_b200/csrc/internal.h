@@ -89,12 +89,16 @@ struct BwdArgs {
   const float* dnT;  // and n [BH, dqk] (mLSTMexp)
   float* fdot;       // [BH] <dC_T, C_T> + <dn_T, n_T>, added to every forget-gate gradient
   float* btab;       // per-chunk gate table of the large-chunk backward (null: not used)
+  float* gsum;       // [BH, gate_grad_segments] totals of q.dq - k.dk per segment (null: one segment)
 };
 
 // gate kernels (gates.cu)
 cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_token_prep(const Problem& p, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_gate_grad(const Problem& p, const BwdArgs& a, cudaStream_t s);
+// few heads: gate_grad runs over segments of T whose totals gate_grad_sums writes first
+int gate_grad_segments(const Problem& p);
+cudaError_t launch_gate_grad_sums(const Problem& p, const BwdArgs& a, cudaStream_t s);
 
 // CUDA-core (fp32 FMA) kernels (simt_fwd.cu, simt_bwd.cu)
 cudaError_t launch_state_fwd_simt(const Problem& p, const FwdArgs& a, cudaStream_t s);

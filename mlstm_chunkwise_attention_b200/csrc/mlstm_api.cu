@@ -109,7 +109,7 @@ mlstm::InitState init_from(const void* state, const Problem& p) {
 }
 
 struct BwdLayout {
-  size_t inv_den, da, pq, pk, dC, dn, fstate, fdot, btab, btab_bytes, total;
+  size_t inv_den, da, pq, pk, dC, dn, fstate, fdot, btab, btab_bytes, gsum, gsum_bytes, total;
 };
 
 BwdLayout bwd_layout(const Problem& p) {
@@ -130,6 +130,10 @@ BwdLayout bwd_layout(const Problem& p) {
                      ? (size_t)p.BH * p.NC * mlstm::bwd_xl_table_stride(p.L) * 4
                      : 0;
   L.btab = off;    off = align256(off + L.btab_bytes);
+  // the gate gradients' segment totals, with few heads
+  const int gseg = mlstm::gate_grad_segments(p);
+  L.gsum_bytes = gseg > 1 ? (size_t)p.BH * gseg * 4 : 0;
+  L.gsum = off;    off = align256(off + L.gsum_bytes);
   L.total = off;
   return L;
 }
@@ -154,7 +158,7 @@ typedef cudaError_t (*BwdLauncher)(const Problem&, const mlstm::BwdArgs&, cudaSt
 // caller's stream; join: the caller's stream waits for the side work before this step.
 struct FwdStep { const char* name; FwdLauncher fn; bool side = false, join = false; };
 struct BwdStep { const char* name; BwdLauncher fn; bool side = false, join = false; };
-constexpr int kMaxSteps = 8;
+constexpr int kMaxSteps = 10;
 
 // The side stream and fork / join events of the calling thread on the current device,
 // created on its first use there (a call that forks must not be the first one made during
@@ -221,7 +225,12 @@ int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
     // walker's last wave (one CTA per SM and head) leaves idle
     st[n++] = {"dkv_walk_tc", mlstm::launch_bwd_walk, true, false};
     st[n++] = {"dq_tc", mlstm::launch_dq_tc};
-    st[n++] = {"gate_grad", mlstm::launch_gate_grad, false, true};
+    if (mlstm::gate_grad_segments(p) > 1) {
+      st[n++] = {"gate_grad_sums", mlstm::launch_gate_grad_sums, false, true};
+      st[n++] = {"gate_grad", mlstm::launch_gate_grad};
+    } else {
+      st[n++] = {"gate_grad", mlstm::launch_gate_grad, false, true};
+    }
     return n;
   }
   if (mlstm::state_tc_supported(p)) {
@@ -244,6 +253,7 @@ int bwd_plan(const Problem& p, BwdStep* st, bool grads = true) {
     st[n++] = {"dk_simt", mlstm::launch_dk_simt};
     st[n++] = {"dv_simt", mlstm::launch_dv_simt};
   }
+  if (mlstm::gate_grad_segments(p) > 1) st[n++] = {"gate_grad_sums", mlstm::launch_gate_grad_sums};
   st[n++] = {"gate_grad", mlstm::launch_gate_grad};
   return n;
 }
@@ -519,6 +529,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   a.dnT = (dstate_out && p.exp_variant()) ? (const float*)((const char*)dstate_out + SL.n) : nullptr;
   a.fdot = dstate_out ? (float*)(ws + W.fdot) : nullptr;
   a.btab = W.btab_bytes ? (float*)(ws + W.btab) : nullptr;
+  a.gsum = W.gsum_bytes ? (float*)(ws + W.gsum) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
 
   st = cuda_status(cudaPeekAtLastError(), "before mlstm_bwd");

@@ -61,9 +61,12 @@ struct XlCfg {
   static constexpr int OFF_V = OFF_K + NK * K_BYTES;
   static constexpr int OFF_ROW = OFF_V + NV * V_BYTES;
   static constexpr int OFF_COL = OFF_ROW + NQ * ROWAUX;
-  static constexpr int OFF_XS = OFF_COL + NV * COLAUX;  // [2 O buffers][4 key blocks][128] floats
+  // normaliser shares [4 items][4 key blocks][128 rows] floats: an item's shares are written
+  // when its last step ends and read by its epilogue one item later; four slots keep a slot
+  // from being rewritten while any warp may still read it, however short the items
+  static constexpr int OFF_XS = OFF_COL + NV * COLAUX;
   // per transform warp: 16 rows of h (DV / 4 bf16 each), 1024-byte aligned for the swizzle
-  static constexpr int OFF_STG = (OFF_XS + 2 * 4 * 128 * 4 + 1023) & ~1023;
+  static constexpr int OFF_STG = (OFF_XS + 4 * 4 * 128 * 4 + 1023) & ~1023;
   static constexpr int STG_WARP = 8 * DV;
   static constexpr int OFF_BAR = OFF_STG + 16 * STG_WARP;
   static constexpr int OFF_TMEM = OFF_BAR + 64 * 8;
@@ -86,9 +89,9 @@ enum {
   X_PF0 = 30,  // P written (256 threads, each having seen its step's V / C_prev), per S buffer
   X_OF0 = 34,  // O complete (MMA commit), per O buffer
   X_OE0 = 36,  // O read out (256 threads), per O buffer
-  X_XS0 = 38,  // normaliser shares exchanged (128 threads), per O buffer and lane quarter
-  X_DRAIN = 46,  // the MMA thread's last commit when it gives up
-  X_COUNT = 47
+  X_XS0 = 38,  // normaliser shares written (128 threads), per item slot (it % 4) and lane quarter
+  X_DRAIN = 54,  // the MMA thread's last commit when it gives up
+  X_COUNT = 55
 };
 
 constexpr int kXlThreads = 608;    // K producer, MMA, 16 transform warps, V producer
@@ -146,7 +149,7 @@ __device__ __forceinline__ int xl_next(int k, int total, int BH, int NC, int NVB
 // its registers do not count against the gate transform it is called from.
 template <int DQK, int DV, bool EXPV>
 __device__ __noinline__ bool xl_epilogue(int it, int vb, int y0, int bh, size_t tok, bool valid,
-                                         float fl, float part, int h, int qr, int lane, uint32_t tmem,
+                                         float fl, int h, int qr, int lane, uint32_t tmem,
                                          uint8_t* smem, const CUtensorMap* tm_h,
                                          float* __restrict__ abar_out, const tc::Abort& abort_flag) {
   using Cfg = XlCfg<DQK, DV>;
@@ -158,12 +161,12 @@ __device__ __noinline__ bool xl_epilogue(int it, int vb, int y0, int bh, size_t 
   const int ob = it & 1, par = (it >> 1) & 1;
   float inv = 1.f;
   if (EXPV) {
-    // den_t = max(|a_t|, exp(-m_t)), a_t added in block order so the four threads of a row agree
-    float* x = reinterpret_cast<float*>(smem + Cfg::OFF_XS) + ob * 512;
-    x[h * 128 + row] = part;
-    uint64_t* xb = &bar[X_XS0 + 4 * ob + qr];
-    tc::mbar_arrive(xb);
-    if (!__all_sync(full, tc::mbar_wait(xb, par, abort_flag))) return false;
+    // den_t = max(|a_t|, exp(-m_t)), a_t added in block order so the four threads of a row
+    // agree; the four key blocks' shares were written when the item's last step ended
+    const int xsl = it & 3;
+    float* x = reinterpret_cast<float*>(smem + Cfg::OFF_XS) + xsl * 512;
+    uint64_t* xb = &bar[X_XS0 + 4 * xsl + qr];
+    if (!__all_sync(full, tc::mbar_wait(xb, (it >> 2) & 1, abort_flag))) return false;
     const float a = ((x[row] + x[128 + row]) + x[256 + row]) + x[384 + row];
     inv = 1.f / fmaxf(fabsf(a), fl);
     if (h == 0 && vb == 0 && valid) abar_out[tok] = a;
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       if (i == X_QE0 || i == X_QE0 + 1) cnt = kXlTransform + 1;
       if (i >= X_PF0 && i < X_PF0 + 4) cnt = kXlTransform;
       if (i >= X_OE0 && i < X_OE0 + 2) cnt = kXlTransform;
-      if (i >= X_XS0 && i < X_XS0 + 8) cnt = kXlTransform / 4;
+      if (i >= X_XS0 && i < X_XS0 + 16) cnt = kXlTransform / 4;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -482,11 +485,11 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       int it, vb, y0, bh;  // item counter; value block; token of this warp's first row; head
       size_t tok;          // token of this thread's row ([BH, T] index)
       bool valid;          // this thread's row is in the sequence
-      float fl, part;
+      float fl;
     } pe{};
     bool pend = false;
     auto epilogue = [&](const Pending& e) -> bool {
-      return xl_epilogue<DQK, DV, EXPV>(e.it, e.vb, e.y0, e.bh, e.tok, e.valid, e.fl, e.part, h, qr,
+      return xl_epilogue<DQK, DV, EXPV>(e.it, e.vb, e.y0, e.bh, e.tok, e.valid, e.fl, h, qr,
                                         lane, tmem, smem, &tm_h, abar_out, abort_flag);
     };
 
@@ -603,7 +606,13 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
         }
       }
       if (!ok) break;
-      const float2 pf = tc::f2_split(part2);
+      if (EXPV) {
+        // this block's share of the normaliser, for the item's epilogue (one item from now)
+        const float2 pf = tc::f2_split(part2);
+        const int xsl = it & 3;
+        xs[xsl * 512 + h * 128 + row] = pf.x + pf.y;
+        tc::mbar_arrive(&bar[X_XS0 + 4 * xsl + qr]);
+      }
       pe.it = it;
       pe.vb = I.vb;
       pe.y0 = I.c * L + I.t0 + 32 * qr;
@@ -611,7 +620,6 @@ __global__ void __launch_bounds__(kXlThreads, 1) output_fwd_xl_kernel(
       pe.tok = (size_t)I.bh * T + (size_t)I.c * L + I.t0 + row;
       pe.valid = I.t0 + row < I.len;
       pe.fl = FLt;
-      pe.part = pf.x + pf.y;
       pend = true;
       ++it;
     }

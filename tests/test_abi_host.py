@@ -282,7 +282,13 @@ def test_launch_plans_split_state_walks_for_few_heads(lib, variant):
     fwd, bwd = _plan(0, long_few), _plan(1, long_few)
     assert fwd[fwd.index("state_fwd_tc") + 1] == "state_fwd_fix", fwd
     assert bwd[bwd.index("state_bwd_tc") + 1] == "state_bwd_fix", bwd
-    assert len(bwd) <= 8  # the plan's step array holds eight
+    assert len(bwd) <= 10  # the plan's step array holds ten
+    # the gate gradients too run over segments of the sequence, after their totals
+    assert bwd[-2:] == ["gate_grad_sums", "gate_grad"], bwd
+    assert _plan(1, (8, 32, 8192, 128, 128, 128, variant, B.BF16))[-1] == "gate_grad"
+    assert "gate_grad_sums" not in _plan(1, (8, 32, 8192, 128, 128, 128, variant, B.BF16))
+    walk_few = _plan(1, (1, 4, 32768, 128, 128, 128, variant, B.BF16))
+    assert walk_few[-2:] == ["gate_grad_sums", "gate_grad"], walk_few
     for sizes in [(8, 32, 8192, 128, 128, 256, variant, B.BF16),   # 256 heads: one walk each
                   (1, 2, 448, 64, 64, 64, variant, B.BF16)]:       # 7 chunks: too few to split
         names = _plan(0, sizes) + _plan(1, sizes)

@@ -294,6 +294,31 @@ def _full(name, variant=None, heads_fwd=2, heads_bwd=1):
             assert err <= tol, f"{key} ({b},{hh}): {err:.3e}"
 
 
+@pytest.mark.parametrize("var", [SIG, EXP], ids=["sig", "exp"])
+def test_few_heads_long_sequence_split_walks(var):
+    """Two heads, 64 chunks of 256: the state walks run as 16 segments and a completion pass,
+    gate_prep (mLSTMsig) spreads a head's chunks over CTAs, and the gate gradients run over 4
+    segments of the sequence after their totals; both heads against the fp64 chunkwise forms."""
+    Bn, NH, T, d, L = 1, 2, 16384, 64, 256
+    cpu = inputs(Bn, NH, T, d, d, seed=91 + var, dtype=BF, ig_mean=-2.0 if var == EXP else 0.0,
+                 fg_mean=3.0)
+    dev, h, saved = gpu_fwd(cpu, L, var)
+    g = gpu_bwd(dev, h, saved, L, var)
+    for hh in range(NH):
+        x = head64(cpu, 0, hh)
+        li, lf = oracle.gate_logs(x["igate"], x["fgate"], var)
+        fwd = oracle.chunkwise_forward(x["q"], x["k"], x["v"], li, lf, var, L)
+        assert relerr(np64(h[0, hh]), fwd["h"]) <= 1e-2, f"h head {hh}"
+        cb = oracle.chunkwise_backward(x["q"], x["k"], x["v"], li, lf, var, L, x["dh"],
+                                       h_in=io_round(fwd["h"], BF))
+        di, df = oracle.preact_grads(cb["dlog_i"], cb["dlog_f"], x["igate"], x["fgate"], var)
+        ref_g = {"dq": cb["dq"], "dk": cb["dk"], "dv": cb["dv"], "digate_pre": di, "dfgate_pre": df}
+        floor = 1e-3 * max(np.max(np.abs(v)) for v in ref_g.values())
+        for key, val in ref_g.items():
+            err = relerr(np64(g[key][0, hh]), val, floor=floor)
+            assert err <= 1e-2, f"{key} head {hh}: {err:.3e}"
+
+
 def test_full_headline_exp_b8h32_t4096_fwd_bwd():
     _full("exp_b8h32_t4096_d128_c128", heads_fwd=3, heads_bwd=2)
 
