@@ -260,6 +260,9 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
         ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar[SB_FULL0 + st], ph, abort_flag));
         if (!ok) break;
         uint8_t* stg = smem + st * Cfg::STAGE_BYTES;
+        // y = w v in packed f32x2 products; hi = bf16(y) in one packed conversion per pair,
+        // lo = bf16(y - hi) likewise (a bf16 value is the upper half of its f32 bits)
+        const uint64_t wv2 = tc::f2_make(wv, wv);
 #pragma unroll
         for (int h = 0; h < NV / 64; ++h) {
 #pragma unroll
@@ -270,11 +273,11 @@ __global__ void __launch_bounds__(256, 2) state_tc_kernel(const __grid_constant_
             uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w}, hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 x2 = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
-              const float y0 = __bfloat162float(x2.x) * wv, y1 = __bfloat162float(x2.y) * wv;
-              const bf16 h0 = __float2bfloat16_rn(y0), h1 = __float2bfloat16_rn(y1);
-              hi[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-              lo[e] = tc::pack_bf16(y0 - __bfloat162float(h0), y1 - __bfloat162float(h1));
+              const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
+              const float2 y = tc::f2_split(tc::f2_mul(tc::f2_make(x0, x1), wv2));
+              hi[e] = tc::pack_bf16(y.x, y.y);
+              lo[e] = tc::pack_bf16(y.x - __uint_as_float(hi[e] << 16),
+                                    y.y - __uint_as_float(hi[e] & 0xffff0000u));
             }
             *reinterpret_cast<uint4*>(stg + Cfg::OFF_BHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4*>(stg + Cfg::OFF_BLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
