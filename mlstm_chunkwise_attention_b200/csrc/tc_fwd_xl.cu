@@ -80,15 +80,15 @@ struct XlCfg {
 
 enum {
   X_QF0 = 0,   // Q (+ row factors) full, per Q buffer
-  X_QE0 = 2,   // Q buffer free: MMA commit + 256 transform threads
+  X_QE0 = 2,   // Q buffer free: MMA commit + the 512 transform threads
   X_KF0 = 4,   // K stage full (K tile or C_prev)
   X_KE0 = 8,   // K stage free (MMA commit after the S or inter-chunk product)
   X_VF0 = 12,  // V stage full (V tile + its key tile's gate factors)
   X_VE0 = 20,  // V stage free (MMA commit after P V)
   X_SF0 = 28,  // S buffer written (MMA commit), per S buffer
-  X_PF0 = 30,  // P written (256 threads, each having seen its step's V / C_prev), per S buffer
+  X_PF0 = 30,  // P written (512 threads, each having seen its step's V / C_prev), per S buffer
   X_OF0 = 34,  // O complete (MMA commit), per O buffer
-  X_OE0 = 36,  // O read out (256 threads), per O buffer
+  X_OE0 = 36,  // O read out (512 threads), per O buffer
   X_XS0 = 38,  // normaliser shares written (128 threads), per item slot (it % 4) and lane quarter
   X_DRAIN = 54,  // the MMA thread's last commit when it gives up
   X_COUNT = 55
