@@ -65,7 +65,7 @@ __device__ void write_xl_tables(const float* b, const float* li, const float* m,
 }
 
 template <typename TIO, bool EXPV>
-__global__ void __launch_bounds__(256) gate_prep_kernel(
+__global__ void __launch_bounds__(1024) gate_prep_kernel(
     const TIO* __restrict__ ig, const TIO* __restrict__ fg, float* __restrict__ b_out,
     float* __restrict__ li_out, float* __restrict__ m_out, float* __restrict__ xt, int T, int L,
     int NC, float scale, float log2_scale, bool has_init, const float* __restrict__ m0) {
@@ -78,44 +78,94 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
 
   // mLSTMsig has no dependency between chunks, so a head's chunks may be spread over
   // gridDim.y CTAs (chunks blockIdx.y, blockIdx.y + gridDim.y, ...); mLSTMexp's max-state
-  // scan needs them all in one CTA (gridDim.y == 1)
-  for (int c = (int)blockIdx.y + (int)gridDim.y * warp; c < NC; c += (int)gridDim.y * nwarps) {
+  // scan needs them all in one CTA (gridDim.y == 1).  The CTA's chunks go to groups of
+  // wpc warps (more warps per chunk when the CTA has fewer chunks than warps); warp j of a
+  // group takes the j-th contiguous segment of its chunk, each lane a contiguous run of it.
+  // Segment totals (and, for mLSTMexp, segment maxima of log i - b) pass through shared
+  // memory, so every sum is still accumulated in fp64 and rounded once.
+  __shared__ double s_sum[32], s_max[32];
+  const int nloc = (NC - (int)blockIdx.y + (int)gridDim.y - 1) / (int)gridDim.y;  // this CTA's chunks
+  int wpc = 1;
+  while (wpc < nwarps && 2 * wpc * nloc <= nwarps) wpc *= 2;
+  const int G = nwarps / wpc, grp = warp / wpc, j = warp % wpc;
+  const int iters = (nloc + G - 1) / G;
+  for (int it = 0; it < iters; ++it) {
+    const int lc = grp + G * it;  // the CTA's local chunk index
+    const bool active = lc < nloc;
+    const int c = (int)blockIdx.y + (int)gridDim.y * (active ? lc : 0);
     const int c0 = c * L;
     const int len = min(L, T - c0);
-    const int per = (len + 31) / 32;
-    const int r0 = min(lane * per, len), r1 = min(r0 + per, len);
+    const int seglen = (len + wpc - 1) / wpc;
+    const int s0 = min(j * seglen, len), s1 = min(s0 + seglen, len);
+    const int per = (s1 - s0 + 31) / 32;
+    const int r0 = min(s0 + lane * per, s1), r1 = min(r0 + per, s1);
+    // pass 1: this lane's sum, the warp's (segment's) total; for mLSTMexp with several
+    // segments also the segment's largest log i - b, b counted from the segment's start
     double seg = 0.0;
-    for (int r = r0; r < r1; ++r) seg += (double)log_sigmoid(to_f32(fg[base + c0 + r]));
+    if (active)
+      for (int r = r0; r < r1; ++r) seg += (double)log_sigmoid(to_f32(fg[base + c0 + r]));
     const double incl = warp_incl_sum(seg);
-    double run = incl - seg;
+    const double lane_excl = incl - seg;
+    if (wpc > 1) {
+      double lmax = -INFINITY;
+      if (EXPV && active) {
+        double run = lane_excl;
+        for (int r = r0; r < r1; ++r) {
+          const size_t idx = base + c0 + r;
+          run += (double)log_sigmoid(to_f32(fg[idx]));
+          lmax = fmax(lmax, (double)to_f32(ig[idx]) - run);
+        }
+      }
+      if (EXPV) lmax = (double)warp_max((float)lmax);
+      const double wtot = __shfl_sync(full, incl, 31);
+      if (lane == 0) {
+        s_sum[warp] = wtot;
+        s_max[warp] = lmax;
+      }
+      __syncthreads();
+    }
+    // the segment's prefix within its chunk, and the largest log i - b before it
+    double prefix = 0.0, prevmax = -INFINITY;
+    for (int k = 0; k < j; ++k) {
+      prevmax = fmax(prevmax, s_max[grp * wpc + k] - prefix);
+      prefix += s_sum[grp * wpc + k];
+    }
+    // pass 2: b, log i and the running max of log i - b for this lane's run
+    double run = prefix + lane_excl;
     double umax = -INFINITY;
-    for (int r = r0; r < r1; ++r) {
-      const size_t idx = base + c0 + r;
-      run += (double)log_sigmoid(to_f32(fg[idx]));
-      const float x = to_f32(ig[idx]);
-      const float li = EXPV ? x : log_sigmoid(x);
-      b_out[idx] = (float)run;
-      li_out[idx] = li;
-      if (EXPV) {
-        umax = fmax(umax, (double)li - run);
-        m_out[idx] = (float)umax;
+    if (active) {
+      for (int r = r0; r < r1; ++r) {
+        const size_t idx = base + c0 + r;
+        run += (double)log_sigmoid(to_f32(fg[idx]));
+        const float x = to_f32(ig[idx]);
+        const float li = EXPV ? x : log_sigmoid(x);
+        b_out[idx] = (float)run;
+        li_out[idx] = li;
+        if (EXPV) {
+          umax = fmax(umax, (double)li - run);
+          m_out[idx] = (float)umax;
+        }
       }
     }
     if (EXPV) {
       const float pm = warp_incl_max((float)umax);
       float excl = __shfl_up_sync(full, pm, 1);
       if (lane == 0) excl = -INFINITY;
-      for (int r = r0; r < r1; ++r) {
-        const size_t idx = base + c0 + r;
-        m_out[idx] = fmaxf(m_out[idx], excl);
-      }
-      const double g = __shfl_sync(full, incl, 31);
-      const double tot = __shfl_sync(full, (double)pm, 31);
-      if (lane == 0) {
+      excl = fmaxf(excl, (float)prevmax);
+      if (active)
+        for (int r = r0; r < r1; ++r) {
+          const size_t idx = base + c0 + r;
+          m_out[idx] = fmaxf(m_out[idx], excl);
+        }
+      // the chunk's totals, from its last segment's warp
+      const double g = prefix + __shfl_sync(full, incl, 31);
+      const double tot = fmax(prevmax, (double)__shfl_sync(full, pm, 31));
+      if (active && j == wpc - 1 && lane == 0) {
         sg[c] = (float)g;
         su[c] = (float)(g + tot);
       }
     }
+    if (wpc > 1) __syncthreads();  // the shared partials are rewritten next iteration
   }
   if (!EXPV) {
     if (xt != nullptr) {
@@ -162,14 +212,15 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(
 
 cudaError_t launch_gate_prep(const Problem& p, const FwdArgs& a, cudaStream_t s) {
   const size_t smem = p.exp_variant() ? 2 * sizeof(float) * (size_t)p.NC : 0;
-  // mLSTMsig with few heads: several CTAs per head, one warp per chunk, up to two CTAs per SM
+  // mLSTMsig with few heads: several CTAs per head (at least a few chunks each), up to two
+  // CTAs per SM
   int per_head = 1;
   if (!p.exp_variant()) {
     const int want = (2 * 148 + p.BH - 1) / p.BH, most = (p.NC + 7) / 8;
     per_head = want < most ? want : most;
     if (per_head < 1) per_head = 1;
   }
-  dim3 grid(p.BH, per_head), block(256);
+  dim3 grid(p.BH, per_head), block(1024);
   if (p.bf16()) {
     if (p.exp_variant())
       gate_prep_kernel<bf16, true><<<grid, block, smem, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.b, a.li, a.m, a.xt, p.T, p.L, p.NC, p.scale, log2f(p.scale), a.init.on(), a.init.on() && p.exp_variant() ? a.init.m : nullptr);
