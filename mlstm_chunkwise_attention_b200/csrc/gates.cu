@@ -15,8 +15,10 @@ namespace mlstm {
 // log i_t; for EXP the max state m_t = b_t + max(m_{c-1}, max_{s<=t in c}(log i_s - b_s)),
 // where m_c (the max state at the chunk's last row) obeys the max-plus
 // recurrence m_c = max(g_c + m_{c-1}, g_c + max_{s in c}(log i_s - b_s)).
-// One CTA per (b, h); each warp owns whole chunks, each lane a contiguous
-// run of rows.  The chunk recurrence is an inclusive warp scan of the affine
+// One CTA of 32 warps per (b, h) (mLSTMsig with few heads: several, each
+// with a share of the chunks); a chunk goes to one warp, or to several warps
+// in contiguous segments when the CTA has fewer chunks than warps, each lane a
+// contiguous run of rows.  The chunk recurrence is an inclusive warp scan of the affine
 // max-plus maps x -> max(x + g_c, u_c).  The sums run in fp64 and are rounded
 // once to fp32: b reaches tens in magnitude over a long chunk, and fp32
 // partial sums would carry an error of many fp32 ulps of it into every decay
