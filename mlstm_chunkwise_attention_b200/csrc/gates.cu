@@ -327,16 +327,32 @@ __device__ __forceinline__ void grad_segment(int T, int& tb, int& te) {
   te = min(T, tb + Tc);
 }
 
+// q.dq - k.dk of one token: each is the sum of its planes in plane order (the
+// large-chunk backward stores one share per 32-column block; otherwise one plane)
+__device__ __forceinline__ float pdot_diff(const float* pq, const float* pk, size_t idx, int planes,
+                                           size_t stride, float& pkt) {
+  float q = pq[idx], k = pk[idx];
+  for (int i = 1; i < planes; ++i) {
+    q += pq[idx + (size_t)i * stride];
+    k += pk[idx + (size_t)i * stride];
+  }
+  pkt = k;
+  return q - k;
+}
+
 // The total of q.dq - k.dk over each segment of a head, for the segments after it.
 __global__ void __launch_bounds__(256) gate_grad_sums_kernel(const float* __restrict__ pq,
                                                              const float* __restrict__ pk,
-                                                             float* __restrict__ gsum, int T) {
+                                                             float* __restrict__ gsum, int T,
+                                                             int planes, size_t stride) {
   __shared__ float s_w[8];
   const size_t base = (size_t)blockIdx.x * T;
   int tb, te;
   grad_segment(T, tb, te);
   float part = 0.f;
-  for (int t = tb + (int)threadIdx.x; t < te; t += blockDim.x) part += pq[base + t] - pk[base + t];
+  float pkt;
+  for (int t = tb + (int)threadIdx.x; t < te; t += blockDim.x)
+    part += pdot_diff(pq, pk, base + t, planes, stride, pkt);
   part = warp_sum(part);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) s_w[warp] = part;
@@ -352,7 +368,7 @@ template <typename TIO, bool EXPV>
 __global__ void __launch_bounds__(1024) gate_grad_kernel(
     const TIO* __restrict__ ig, const TIO* __restrict__ fg, const float* __restrict__ pq,
     const float* __restrict__ pk, TIO* __restrict__ dig, TIO* __restrict__ dfg, int T,
-    const float* __restrict__ fdot, const float* __restrict__ gsum) {
+    const float* __restrict__ fdot, const float* __restrict__ gsum, int planes, size_t stride) {
   __shared__ float s_tot[32];
   const size_t base = (size_t)blockIdx.x * T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -361,7 +377,8 @@ __global__ void __launch_bounds__(1024) gate_grad_kernel(
   const int seg = (te - tb + 31) / 32;
   const int sb = min(tb + warp * seg, te), se = min(sb + seg, te);
   float part = 0.f;
-  for (int t = sb + lane; t < se; t += 32) part += pq[base + t] - pk[base + t];
+  float pkt;
+  for (int t = sb + lane; t < se; t += 32) part += pdot_diff(pq, pk, base + t, planes, stride, pkt);
   part = warp_sum(part);
   if (lane == 0) s_tot[warp] = part;
   __syncthreads();
@@ -381,8 +398,9 @@ __global__ void __launch_bounds__(1024) gate_grad_kernel(
   for (int e = se; e > sb; e -= 32) {
     const int t = e - 32 + lane;
     const bool valid = t >= sb;
-    const float pkt = valid ? pk[base + t] : 0.f;
-    const float x = valid ? pq[base + t] - pkt : 0.f;
+    float x = 0.f;
+    pkt = 0.f;
+    if (valid) x = pdot_diff(pq, pk, base + t, planes, stride, pkt);
     const float sfx = warp_incl_suffix_sum(x);
     const float dlf = carry + sfx;
     carry += __shfl_sync(0xffffffffu, sfx, 0);
@@ -407,7 +425,8 @@ int gate_grad_segments(const Problem& p) {
 cudaError_t launch_gate_grad_sums(const Problem& p, const BwdArgs& a, cudaStream_t s) {
   const int G = gate_grad_segments(p);
   if (G < 2 || a.gsum == nullptr) return cudaErrorInvalidValue;  // planned only for a split
-  gate_grad_sums_kernel<<<dim3(p.BH, G), 256, 0, s>>>(a.pq, a.pk, a.gsum, p.T);
+  gate_grad_sums_kernel<<<dim3(p.BH, G), 256, 0, s>>>(a.pq, a.pk, a.gsum, p.T, a.pdot_planes,
+                                                       a.pdot_stride);
   return cudaGetLastError();
 }
 
@@ -417,14 +436,14 @@ cudaError_t launch_gate_grad(const Problem& p, const BwdArgs& a, cudaStream_t s)
   dim3 grid(p.BH, G), block(1024);
   if (p.bf16()) {
     if (p.exp_variant())
-      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot, a.gsum);
+      gate_grad_kernel<bf16, true><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot, a.gsum, a.pdot_planes, a.pdot_stride);
     else
-      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot, a.gsum);
+      gate_grad_kernel<bf16, false><<<grid, block, 0, s>>>((const bf16*)a.ig, (const bf16*)a.fg, a.pq, a.pk, (bf16*)a.dig, (bf16*)a.dfg, p.T, a.fdot, a.gsum, a.pdot_planes, a.pdot_stride);
   } else {
     if (p.exp_variant())
-      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot, a.gsum);
+      gate_grad_kernel<float, true><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot, a.gsum, a.pdot_planes, a.pdot_stride);
     else
-      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot, a.gsum);
+      gate_grad_kernel<float, false><<<grid, block, 0, s>>>((const float*)a.ig, (const float*)a.fg, a.pq, a.pk, (float*)a.dig, (float*)a.dfg, p.T, a.fdot, a.gsum, a.pdot_planes, a.pdot_stride);
   }
   return cudaGetLastError();
 }

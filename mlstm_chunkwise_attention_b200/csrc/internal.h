@@ -78,8 +78,10 @@ struct BwdArgs {
   void *dq, *dk, *dv, *dig, *dfg;
   float* inv_den;  // [BH, T] 1 / den_t
   float* da;       // [BH, T] gradient of the stabilised normaliser (EXP)
-  float* pq;       // [BH, T] q_t . dq_t
-  float* pk;       // [BH, T] k_t . dk_t
+  float* pq;       // [pdot_planes, BH, T] q_t . dq_t, the sum of the planes in plane order
+  float* pk;       // [pdot_planes, BH, T] k_t . dk_t, likewise
+  int pdot_planes;    // 4 on the large-chunk backward (one share per 32 columns), else 1
+  size_t pdot_stride; // elements per plane (BH T)
   void* dC;        // [BH, NC, dqk, dhv] gradient of the state leaving each chunk (planes, see StatePlanes)
   float* dn;       // [BH, NC, dqk]
   InitState init;  // the state the forward started from (held constant)

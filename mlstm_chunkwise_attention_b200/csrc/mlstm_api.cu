@@ -118,8 +118,10 @@ BwdLayout bwd_layout(const Problem& p) {
   size_t off = 0;
   L.inv_den = off; off = align256(off + tok * 4);
   L.da = off;      off = align256(off + tok * 4);
-  L.pq = off;      off = align256(off + tok * 4);
-  L.pk = off;      off = align256(off + tok * 4);
+  // q.dq and k.dk: the large-chunk backward writes four column-block shares per token
+  const size_t planes = mlstm::intra_bwd_xl_supported(p) ? 4 : 1;
+  L.pq = off;      off = align256(off + planes * tok * 4);
+  L.pk = off;      off = align256(off + planes * tok * 4);
   L.dC = off;      off = align256(off + (size_t)p.BH * p.NC * p.dqk * p.dhv * 4);
   L.dn = off;      off = align256(off + (p.exp_variant() ? (size_t)p.BH * p.NC * p.dqk * 4 : 0));
   // the final state, rebuilt when the loss has a term on it, and its dot product with that term
@@ -520,6 +522,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* igate_pre,
   a.da = (float*)(ws + W.da);
   a.pq = (float*)(ws + W.pq);
   a.pk = (float*)(ws + W.pk);
+  a.pdot_planes = mlstm::intra_bwd_xl_supported(p) ? 4 : 1;
+  a.pdot_stride = (size_t)p.BH * p.T;
   a.dC = ws + W.dC;
   a.dn = p.exp_variant() ? (float*)(ws + W.dn) : nullptr;
   a.init = init_from(state_in, p);

@@ -70,8 +70,7 @@ struct BxCfg {
   static constexpr int OFF_E = OFF_B + NB * TILE;
   static constexpr int OFF_ROW = OFF_E + NE * TILE;
   static constexpr int OFF_COL = OFF_ROW + NA * ROWAUX;
-  static constexpr int OFF_XS = OFF_COL + NE * COLAUX;     // [2 Acc buffers][4 column blocks][128]
-  static constexpr int OFF_FW = OFF_XS + 2 * 4 * 128 * 4;  // per transform warp: 32 partner factors
+  static constexpr int OFF_FW = OFF_COL + NE * COLAUX;  // per transform warp: 32 partner factors
   // per transform warp: 16 rows of 32 bf16 output columns, 1024-byte aligned for the swizzle
   static constexpr int OFF_STG = (OFF_FW + 16 * 32 * 4 + 1023) & ~1023;
   static constexpr int STG_WARP = 1024;
@@ -95,9 +94,8 @@ enum {
   Y_IR0 = 18,  // inter-chunk product rescaled (512 threads), per Acc buffer
   Y_OF0 = 20,  // Acc complete (MMA commit), per Acc buffer
   Y_OE0 = 22,  // Acc read out (512 threads), per Acc buffer
-  Y_XS0 = 24,  // dot-product shares exchanged (128 threads), per Acc buffer and lane quarter
-  Y_DRAIN = 32,  // the MMA thread's last commit when it gives up
-  Y_COUNT = 33
+  Y_DRAIN = 24,  // the MMA thread's last commit when it gives up
+  Y_COUNT = 25
 };
 
 struct BxItem {
@@ -109,7 +107,8 @@ struct BxParams {
   const float* tab;     // per-chunk gate table (bwd_xl_table_stride(L) floats per chunk)
   const float* rowvec;  // dq: n_{c-1}, dk: dn_c [BH, NC, 128] (mLSTMexp); dv: unused
   const bf16* dot_src;  // dq: q, dk: k [BH, T, 128]
-  float* pdot;          // dq: pq, dk: pk [BH, T] (one add onto zero per token)
+  float* pdot;          // dq: pq, dk: pk [4 planes][BH, T]: the share of 32 columns h in plane h
+  size_t pdot_stride;   // elements per plane
   int T, L, NC, BH, ntq, total, tstride;
   bool init;  // the forward started from an initial state (dq: every chunk has a state)
   bool dfin;  // the final state has a gradient (dk, dv: every chunk has a state gradient)
@@ -159,8 +158,9 @@ __device__ __forceinline__ int bx_next(int k, const BxParams& P, BxItem& it) {
 // Epilogue of one item for the transform thread of row 32 qr + lane and columns
 // [32 h, 32 h + 32): the accumulator leaves TMEM (freeing it for the next items'
 // products), is scaled, dotted with the row's q (dq) or k (dk) for the gate
-// gradients (the four column blocks' shares summed in block order by the h = 0
-// thread), and stored through this warp's staging slot by 16-row TMA stores
+// gradients (this column block's share stored in plane h; the gate-gradient
+// kernels add the four planes in block order), and stored through this warp's
+// staging slot by 16-row TMA stores
 // (rows past the sequence end are clipped by the TMA unit).  Inlined: an
 // out-of-line call makes the caller save its live registers around it.
 template <int KIND>
@@ -171,7 +171,6 @@ __device__ __forceinline__ bool bx_epilogue(int it, int y0, int bh, size_t tok, 
   const unsigned full = 0xffffffffu;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + BxCfg::OFF_BAR);
   const int warp = 2 + 4 * h + ((qr + 2) & 3);  // the warp of (h, qr): lane quarter = warp % 4
-  const int row = 32 * qr + lane;
   const uint32_t lb = (uint32_t)(32 * qr) << 16;
   const int ob = it & 1, par = (it >> 1) & 1;
   // the row's 32 elements of q or k, in flight while the accumulator completes
@@ -231,13 +230,9 @@ __device__ __forceinline__ bool bx_epilogue(int it, int y0, int bh, size_t tok, 
         dot = fmaf(__bfloat162float(s2.y), __uint_as_float(o[8 * c4 + 2 * e + 1]) * fin, dot);
       }
     }
-    float* x = reinterpret_cast<float*>(smem + BxCfg::OFF_XS) + ob * 512;
-    x[h * 128 + row] = dot;
-    uint64_t* xb = &bar[Y_XS0 + 4 * ob + qr];
-    tc::mbar_arrive(xb);
-    if (!__all_sync(full, tc::mbar_wait(xb, par, abort_flag))) return false;
-    if (h == 0 && valid)
-      atomicAdd(&P.pdot[tok], ((x[row] + x[128 + row]) + x[256 + row]) + x[384 + row]);
+    // this column block's share, in its own plane; the gate-gradient kernels add the four
+    // planes in block order
+    if (valid) P.pdot[(size_t)h * P.pdot_stride + tok] = dot;
   }
   return true;
 }
@@ -268,7 +263,6 @@ __global__ void __launch_bounds__(kBxThreads, 1) intra_bwd_xl_kernel(
       if ((i >= Y_PF0 && i < Y_PF0 + 2) || (i >= Y_IR0 && i < Y_IR0 + 2) ||
           (i >= Y_OE0 && i < Y_OE0 + 2))
         cnt = kBxTransform;
-      if (i >= Y_XS0 && i < Y_XS0 + 8) cnt = kBxTransform / 4;
       tc::mbar_init(&bar[i], cnt);
     }
     tc::fence_mbar_init();
@@ -807,6 +801,8 @@ static cudaError_t launch_xl_kind(const Problem& p, const BwdArgs& a, cudaStream
   P.rowvec = KIND == BX_DQ ? a.n : a.dn;
   P.dot_src = (const bf16*)(KIND == BX_DQ ? a.q : a.k);
   P.pdot = KIND == BX_DQ ? a.pq : a.pk;
+  P.pdot_stride = a.pdot_stride;
+  if (a.pdot_planes != 4) return cudaErrorInvalidValue;
   P.T = p.T;
   P.L = p.L;
   P.NC = p.NC;
