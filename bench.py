@@ -757,21 +757,22 @@ def main():
     names = ([binding.mlstm_launch_name(0, i, *sizes) for i in range(nf)]
              + [binding.mlstm_launch_name(1, i, *sizes) for i in range(nb)])
 
-    def step(src, fwd_ev=None, bwd_ev=None):
+    def step(src, fwd_ev=None, bwd_ev=None, out=None):
+        o = out if out is not None else {"h": h, **grads}
         if fwd_ev is not None:
             binding.mlstm_set_timing_events(fwd_ev, 2 * nf)
         st = binding.mlstm_fwd(src["q"].data_ptr(), src["k"].data_ptr(), src["v"].data_ptr(),
-                               src["igate"].data_ptr(), src["fgate"].data_ptr(), h.data_ptr(),
+                               src["igate"].data_ptr(), src["fgate"].data_ptr(), o["h"].data_ptr(),
                                saved.data_ptr(), None, 0, *sizes, sh)
         if st != 0:
             raise binding.MLSTMError(st, "mlstm_fwd")
         if bwd_ev is not None:
             binding.mlstm_set_timing_events(bwd_ev, 2 * nb)
         st = binding.mlstm_bwd(src["q"].data_ptr(), src["k"].data_ptr(), src["v"].data_ptr(),
-                               src["igate"].data_ptr(), src["fgate"].data_ptr(), h.data_ptr(),
-                               src["dh"].data_ptr(), saved.data_ptr(), grads["dq"].data_ptr(),
-                               grads["dk"].data_ptr(), grads["dv"].data_ptr(),
-                               grads["dig"].data_ptr(), grads["dfg"].data_ptr(), ws.data_ptr(),
+                               src["igate"].data_ptr(), src["fgate"].data_ptr(), o["h"].data_ptr(),
+                               src["dh"].data_ptr(), saved.data_ptr(), o["dq"].data_ptr(),
+                               o["dk"].data_ptr(), o["dv"].data_ptr(),
+                               o["dig"].data_ptr(), o["dfg"].data_ptr(), ws.data_ptr(),
                                wsb, *sizes, sh)
         binding.mlstm_set_timing_events(None, 0)
         if st != 0:
@@ -860,34 +861,72 @@ def main():
                 "algorithmic_per_launch": heads * (by if bound == "hbm" else fl),
                 "ms_per_launch": per_kernel[dom]}
 
-    # ---- end to end through the C ABI with pinned host buffers
+    # ---- end to end through the C ABI with pinned host buffers: every step copies its
+    # inputs in from pinned host memory and all of its results (h and the five gradients)
+    # back out.  Timed twice: one stream (copy in, compute, copy out, step after step), and
+    # pipelined as a user streaming batches would run it, with two device buffer sets and one
+    # copy stream per direction, so step i+1's inputs cross the host link while step i's
+    # results come back (the link is full duplex) and its compute runs in between.
     host_in = {k: v.pin_memory() for k, v in cpu.items()}
-    host_out = {"h": torch.empty(h.shape, dtype=dtype).pin_memory(),
-                **{k: torch.empty(v.shape, dtype=dtype).pin_memory() for k, v in grads.items()}}
-    xd = {k: torch.empty_like(v) for k, v in x.items()}
+    out_keys = ["h"] + list(grads)
+    xd = [{k: torch.empty_like(v) for k, v in x.items()} for _ in range(2)]
+    od = [{"h": h, **grads}, {k: torch.empty_like(v) for k, v in [("h", h), *grads.items()]}]
+    host_out = [{k: torch.empty(od[0][k].shape, dtype=dtype).pin_memory() for k in out_keys}
+                for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    d2h = sum(host_out[0][k].numel() * host_out[0][k].element_size() for k in out_keys)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_in + ev_comp + ev_out:
+        e.record(stream)
 
-    def e2e_step():
-        for k_ in xd:
-            xd[k_].copy_(host_in[k_], non_blocking=True)
-        step(xd)
-        host_out["h"].copy_(h, non_blocking=True)
-        for k_, v in grads.items():
-            host_out[k_].copy_(v, non_blocking=True)
+    def e2e_serial_step():
+        for k_ in xd[0]:
+            xd[0][k_].copy_(host_in[k_], non_blocking=True)
+        step(xd[0], out=od[0])
+        for k_ in out_keys:
+            host_out[0][k_].copy_(od[0][k_], non_blocking=True)
+
+    def e2e_pipelined_step(i):
+        b = i & 1
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])  # the compute that read this input set is done
+            for k_ in xd[b]:
+                xd[b][k_].copy_(host_in[k_], non_blocking=True)
+            ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])  # this output set has been read back
+        step(xd[b], out=od[b])
+        ev_comp[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            for k_ in out_keys:
+                host_out[b][k_].copy_(od[b][k_], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    def timed(fn, pipelined):
+        for i in range(args.warmup):
+            fn(i) if pipelined else fn()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(args.steps):
+            fn(i) if pipelined else fn()
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
 
     del x
-    for _ in range(args.warmup):
-        e2e_step()
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_serial_ms = timed(e2e_serial_step, False)
+    e2e_ms = timed(e2e_pipelined_step, True)
     e2e_tflops = step_flops * args.steps * world / (e2e_ms * 1e-3) / 1e12
 
     cpu_base = None
@@ -913,7 +952,10 @@ def main():
         "roofline": roofline,
         "cpu_baseline": cpu_base,
         "e2e": {"value": e2e_tflops, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
+                "mode": "pipelined: two device buffer sets, one copy stream per direction; "
+                        "step i+1's input copies overlap step i's result copies",
+                "serial_ms_per_step": e2e_serial_ms / args.steps},
         "gpu_launches": args.steps * (nf + nb),
         "clocks": clk,
     }
