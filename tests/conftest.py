@@ -14,6 +14,6 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
-    # GPU tests fail loudly on a GPU machine if the library is missing; without a
+    # GPU tests fail loudly on a machine with a GPU if the library is missing; without a
     # GPU they are only deselected by -m "not gpu".
     pass

@@ -1,7 +1,7 @@
 """bench.py's reference arm (the fp64 oracle on the host cores) prints one JSON line with
 the keys the bench contract requires; CPU only, a few seconds.
 
-The GPU arm's line is checked on the GPU machine by running bench.py itself; this file covers the
+The GPU arm's line is checked on a machine with a GPU by running bench.py itself; this file covers the
 arm that needs no GPU, including the rule that warm-up steps are never fewer than 3.
 """
 

@@ -111,7 +111,7 @@ def test_small_forward_backward_all_heads(case):
 # normaliser sum_s A_ts does not cancel: with random signs and a large i~ the
 # normaliser's floor exp(-m_t) is negligible and |a_t| can fall orders of magnitude
 # below sum_s |A_ts|, where h = num / a amplifies any bf16 rounding by that ratio (an
-# input-conditioning limit of bf16 operands, not of the stabiliser; see DESIGN.md).
+# input-conditioning limit of bf16 operands, not of the stabiliser).
 # name, B, NH, T, d_qk, d_hv, chunk, igate mean, igate std, spike value (every 53rd
 # token from token 11 on), forget mean
 BIG_IGATE = [
