@@ -252,6 +252,16 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
       tc::tma_load_3d(sQ, &tmQ, &bar[BF_Q], 0, c * 128, bh);
       tc::tma_load_3d(sQ + 16384, &tmQ, &bar[BF_Q], 64, c * 128, bh);
     };
+    // the next chunk's tiles into L2 while this chunk runs (their loads wait for this
+    // chunk's products and stores to free the buffers)
+    auto prefetch_next = [&](int c) {
+      tc::tma_prefetch_l2_3d(&tmQ, 0, c * 128, bh);
+      tc::tma_prefetch_l2_3d(&tmQ, 64, c * 128, bh);
+      tc::tma_prefetch_l2_3d(&tmK, 0, c * 128, bh);
+      tc::tma_prefetch_l2_3d(&tmK, 64, c * 128, bh);
+      tc::tma_prefetch_l2_3d(&tmV, 0, c * 128, bh);
+      tc::tma_prefetch_l2_3d(&tmV, 64, c * 128, bh);
+    };
     auto load_kv = [&](int c) {
       uint8_t* st = set_of(c);
       uint64_t* b = &bar[(c & 1) ? BF_KV1 : BF_KV0];
@@ -439,6 +449,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
     if (issuer) {
       load_q(0);
       load_kv(0);
+      if (NC > 1) prefetch_next(1);
     }
     float n = 0.f;  // n_c (mLSTMexp), state row j
     {
@@ -465,6 +476,7 @@ __global__ void __launch_bounds__(288, 1) fwd_walk_kernel(
         if (issuer) {
           tc::bulk_wait_read_all();
           load_q(c);
+          if (c + 1 < NC) prefetch_next(c + 1);
         }
         // the previous chunk's state update is done: C_c is in TMEM
         ok = wait_state();
