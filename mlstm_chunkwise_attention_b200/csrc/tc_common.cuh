@@ -318,20 +318,6 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
       : "memory");
 }
 
-// Orders later uses of r after an earlier tmem_wait_ld (which covered every
-// outstanding load of the thread, these registers included).
-__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
-  asm volatile(
-      ""
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
-        "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
-        "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-      :
-      : "memory");
-}
-
 // Store 32 / 16 consecutive 32-bit columns of this thread's TMEM lane, not
 // waited on (tmem_wait_st before signalling a consumer).
 __device__ __forceinline__ void tmem_st32_async(uint32_t taddr, const uint32_t (&r)[32]) {
