@@ -302,3 +302,32 @@ def test_serial_launch_switch_needs_no_device(lib):
     assert lib.mlstm_set_serial_launches(0) == 0
     assert lib.mlstm_set_serial_launches(7) == 0
     assert lib.mlstm_set_serial_launches(0) == 0
+
+
+def test_bench_accounts_for_every_planned_kernel(lib):
+    """Every kernel a launch plan can name has an algorithmic (FLOPs, bytes) entry and a source
+    file in bench.py, so the bench's per-kernel roofline never meets an unknown kernel."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    seen = set()
+    for dt in (B.BF16, B.FP32):
+        for var in (B.SIG, B.EXP):
+            for (Bn, NH, T, dqk, dhv) in [(2, 4, 1000, 128, 128), (1, 2, 300, 64, 64),
+                                         (1, 8, 65536, 256, 512), (8, 32, 4096, 128, 128),
+                                         (1, 4, 32768, 128, 128), (2, 2, 640, 256, 256)]:
+                for L in (64, 128, 256, 512, 1024):
+                    sizes = (Bn, NH, T, dqk, dhv, L, var, dt)
+                    names = _plan(0, sizes) + _plan(1, sizes)
+                    costs = bench.kernel_costs(T, dqk, dhv, L, var == B.EXP, 2 if dt == B.BF16 else 4)
+                    for n in names:
+                        assert n in costs, (sizes, n)
+                        assert n in bench.KERNEL_SOURCES, (sizes, n)
+                        assert bench.kernel_bound(n) in ("hbm", "tensor", "alu")
+                        assert os.path.exists(os.path.join(ROOT, "mlstm_chunkwise_attention_b200",
+                                                           "csrc", bench.KERNEL_SOURCES[n]))
+                    seen.update(names)
+    # the walkers, the large-chunk kernels, the segmented walks and the CUDA-core path all occur
+    for n in ("fwd_walk_tc", "dkv_walk_tc", "output_fwd_xl", "dq_xl", "state_fwd_fix",
+              "gate_grad_sums", "output_fwd_simt", "dq_simt"):
+        assert n in seen, n
