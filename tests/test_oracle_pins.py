@@ -308,7 +308,33 @@ def check_rows(M, variant):
         assert rel(gr[name], g[name][rows]) < 1e-11, name
 
 
+def check_normaliser_tie(M):
+    """Reading 4, by hand: one mLSTMexp token with |a| exactly 1 takes the constant branch.
+
+    d_qk = 4, q = k = (1, 1, 0, 0), log i = 0: C = k v^T, n = k, q' = q / 2, so
+    a = n . q' = 1 = the floor (exp(-m) with m = log i = 0 in the stabilised forms) and
+    h = C^T q' / 1 = v.  With den held at the floor, L = dh . h = (dh . v)(k . q') gives
+    dq = (dh . v) k / 2, dk = (dh . v) q / 2, dv = dh, d log i = dh . v, d log f = 0.
+    Taking the |a| branch instead would make h = v (k . q') / (k . q') and dq = dk = 0.
+    """
+    q = np.array([[1.0, 1.0, 0.0, 0.0]])
+    k = q.copy()
+    v = np.array([[0.5, -1.0, 2.0]])
+    dh = np.array([[1.0, 2.0, -0.5]])
+    li, lf = np.array([0.0]), np.array([M.logsigmoid(3.0)])
+    dhv = float(dh[0] @ v[0])  # -2.5
+    want = {"dq": dhv * k / 2, "dk": dhv * q / 2, "dv": dh, "dlog_i": np.array([dhv]),
+            "dlog_f": np.array([0.0])}
+    got = [M.parallel_backward(q, k, v, li, lf, EXP, dh), M.recurrent_backward(q, k, v, li, lf, EXP, dh),
+           M.chunkwise_backward(q, k, v, li, lf, EXP, 1, dh), M.chunkwise_backward(q, k, v, li, lf, EXP, 4, dh)]
+    for g in got:
+        np.testing.assert_allclose(g["h"], v, rtol=0, atol=1e-15)
+        for name, w in want.items():
+            np.testing.assert_allclose(g[name], w, rtol=0, atol=1e-14, err_msg=name)
+
+
 ALL_CHECKS = [
+    check_normaliser_tie,
     check_hand_cases, check_logsigmoid, check_open_gates,
     lambda M: check_closed_forget(M, SIG), lambda M: check_closed_forget(M, EXP),
     check_retention, check_single_token,
@@ -328,6 +354,10 @@ ALL_CHECKS = [
 # ---------------------------------------------------------------------------
 # the pins, on the real oracle
 # ---------------------------------------------------------------------------
+
+def test_normaliser_tie_takes_the_constant_branch():
+    check_normaliser_tie(oracle)
+
 
 @pytest.mark.parametrize("variant", [SIG, EXP])
 def test_steps_and_final_state(variant):
@@ -439,6 +469,9 @@ MUTATIONS = [
     ("dk transposed", "dk = dS.T @ qs", "dk = dS @ qs"),
     ("dlog_f summed on the wrong axis", "dlog_f = np.tril(excl).sum(axis=0)", "dlog_f = np.tril(excl).sum(axis=1)"),
     ("da sign", "da = np.where(active, -np.sum(dh * h, axis=1)", "da = np.where(active, np.sum(dh * h, axis=1)"),
+    ("normaliser tie takes the |a| branch", "active = np.abs(a) > floor", "active = np.abs(a) >= floor"),
+    ("stabilised tie takes the |a| branch", 'active = np.abs(f["abar"]) > np.exp(-m_row)',
+     'active = np.abs(f["abar"]) >= np.exp(-m_row)'),
     ("forget chain rule sign", "dfgate = np.asarray(dlog_f) * sigmoid(-np.asarray(fgate_pre", "dfgate = np.asarray(dlog_f) * sigmoid(np.asarray(fgate_pre"),
     ("bptt forget grad uses C_t", "df[t] = np.sum(dC * Cs[t]) + dn @ ns[t]", "df[t] = np.sum(dC * Cs[t + 1]) + dn @ ns[t]"),
     ("column dA misses da", "dA_col = dnum[r:] @ v[r] + da[r:]", "dA_col = dnum[r:] @ v[r]"),
